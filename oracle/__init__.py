@@ -1,0 +1,205 @@
+"""CPU oracle of the UltraSketchLLM sketch -- TEST INFRASTRUCTURE ONLY.
+
+This package wraps ``usk_oracle.c`` (plain sequential C, IEEE fp32/fp64, no
+fast-math) with ctypes and numpy.  Only ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import it; the library under
+``sub_bit_weight_usk_b200/`` never does, and the two share no code.
+
+What it computes is written out in ``usk_oracle.c`` with its sources:
+"UltraSketchLLM: Sub-1-Bit LLM Compression via Sketch and Hardware-Friendly
+Operators" (gist.science/es/paper/2506.17255), Resumen Tecnico, Metodologia §1
+(AbsMaxMin sketch) and §4 (decompression as W_hat = S . P^T), plus the frozen
+format readings listed there.
+
+Parity pins (tests/test_oracle_*.py): SplitMix64 published outputs, binary16
+conversion against numpy's, round-half-even against numpy.rint, an independent
+pure-Python brute-force bucket enumeration, closed-form special cases and
+invariants, and numpy float64 matmul for the products.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "usk_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+# status values (same meanings as the library's usk_status)
+OK = 0
+ERR_NULL = 1
+ERR_SHAPE = 2
+ERR_DTYPE = 3
+ERR_NONFINITE = 8
+ERR_IMPORTANCE = 11
+ERR_SCALE_OVERFLOW = 12
+
+F32 = 0
+BF16 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile usk_oracle.c into liboracle.so next to it (gcc, IEEE-strict)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math",
+               "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i64, u64, vp = ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p
+        lib.orc_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, u64, vp, vp, vp, vp]
+        lib.orc_build.restype = ctypes.c_int
+        lib.orc_decode.argtypes = [vp, vp, i64, i64, u64, vp]
+        lib.orc_decode.restype = ctypes.c_int
+        lib.orc_gemv_f64.argtypes = [vp, vp, i64, i64, u64, vp, ctypes.c_int, i64, vp, i64, vp]
+        lib.orc_gemv_f64.restype = ctypes.c_int
+        lib.orc_bucket_index.argtypes = [i64, u64, i64, i64]
+        lib.orc_bucket_index.restype = i64
+        lib.orc_splitmix64.argtypes = [u64, u64]
+        lib.orc_splitmix64.restype = u64
+        lib.orc_tile_hash_params.argtypes = [u64, u64, vp, vp]
+        lib.orc_tile_hash_params.restype = None
+        lib.orc_f32_to_f16.argtypes = [ctypes.c_float]
+        lib.orc_f32_to_f16.restype = ctypes.c_uint16
+        lib.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.orc_f16_to_f32.restype = ctypes.c_float
+        lib.orc_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.orc_bf16_to_f32.restype = ctypes.c_float
+        lib.orc_storage_bytes.argtypes = [i64, i64, vp, vp]
+        lib.orc_storage_bytes.restype = None
+        lib.orc_f32_to_f16_array.argtypes = [vp, vp, i64]
+        lib.orc_f32_to_f16_array.restype = None
+        lib.orc_f16_to_f32_array.argtypes = [vp, vp, i64]
+        lib.orc_f16_to_f32_array.restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _weights(W):
+    """(array, dtype code): float32 arrays are fp32, uint16 arrays are bf16 bits."""
+    W = np.ascontiguousarray(W)
+    if W.dtype == np.float32:
+        return W, F32
+    if W.dtype == np.uint16:
+        return W, BF16
+    raise TypeError("weights must be float32 or uint16 (bf16 bit patterns)")
+
+
+def build_sketch(W, importance=None, seed=0, want_winners=False):
+    """Sketch of W [M, K].  Returns dict(status, codes, scales[, winner, value])."""
+    W, dt = _weights(W)
+    M, K = W.shape
+    imp = None if importance is None else np.ascontiguousarray(importance, dtype=np.float32)
+    nb = M * K // 16 if (M % 64 == 0 and K % 256 == 0 and M >= 0 and K >= 0) else 0
+    codes = np.zeros(max(nb, 1), dtype=np.int8)
+    scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
+    winner = np.full(max(nb, 1), -2, dtype=np.int64) if want_winners else None
+    value = np.zeros(max(nb, 1), dtype=np.float32) if want_winners else None
+    st = _load().orc_build(_ptr(W), dt, M, K, K, _ptr(imp), seed, _ptr(codes), _ptr(scales),
+                           _ptr(winner), _ptr(value))
+    out = {"status": st, "codes": codes[:nb], "scales": scales[: M // 64]}
+    if want_winners:
+        out["winner"] = winner[:nb]
+        out["value"] = value[:nb]
+    return out
+
+
+def decode(codes, scales, M, K, seed=0):
+    """W_hat [M, K] float32 rebuilt from the sketch."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    out = np.zeros((M, K), dtype=np.float32)
+    st = _load().orc_decode(_ptr(codes), _ptr(scales), M, K, seed, _ptr(out))
+    if st:
+        raise ValueError("orc_decode status %d" % st)
+    return out
+
+
+def gemv_f64(codes, scales, M, K, x, seed=0, rows=None):
+    """y [batch, M] (or [batch, len(rows)]) = W_hat x^T in float64.
+
+    x is [batch, K] float32 (fp32) or uint16 (bf16 bit patterns)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    xdt = F32 if x.dtype == np.float32 else BF16 if x.dtype == np.uint16 else None
+    if xdt is None:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    batch = x.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nr = M if r is None else len(r)
+    y = np.zeros((batch, nr), dtype=np.float64)
+    st = _load().orc_gemv_f64(_ptr(codes), _ptr(scales), M, K, seed, _ptr(x), xdt, batch,
+                              _ptr(r), 0 if r is None else len(r), _ptr(y))
+    if st:
+        raise ValueError("orc_gemv_f64 status %d" % st)
+    return y
+
+
+def bucket_index(K, seed, i, j):
+    """Global code index of weight (i, j)."""
+    return int(_load().orc_bucket_index(K, seed, i, j))
+
+
+def splitmix64(seed, n):
+    """Output n (1-based) of SplitMix64 seeded with `seed`."""
+    return int(_load().orc_splitmix64(seed & (2**64 - 1), n))
+
+
+def tile_hash_params(seed, tile_id):
+    a = ctypes.c_uint32()
+    c = ctypes.c_uint32()
+    _load().orc_tile_hash_params(seed, tile_id, ctypes.byref(a), ctypes.byref(c))
+    return a.value, c.value
+
+
+def f32_to_f16(x):
+    return int(_load().orc_f32_to_f16(float(np.float32(x))))
+
+
+def f16_to_f32(h):
+    return float(_load().orc_f16_to_f32(int(h)))
+
+
+def f32_to_f16_array(x):
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.zeros(x.shape, dtype=np.uint16)
+    _load().orc_f32_to_f16_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def f16_to_f32_array(h):
+    h = np.ascontiguousarray(h, dtype=np.uint16)
+    out = np.zeros(h.shape, dtype=np.float32)
+    _load().orc_f16_to_f32_array(_ptr(h), _ptr(out), h.size)
+    return out
+
+
+def bf16_to_f32(h):
+    return float(_load().orc_bf16_to_f32(int(h)))
+
+
+def storage_bytes(M, K):
+    c = ctypes.c_int64()
+    s = ctypes.c_int64()
+    _load().orc_storage_bytes(M, K, ctypes.byref(c), ctypes.byref(s))
+    return c.value, s.value

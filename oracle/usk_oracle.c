@@ -1,0 +1,333 @@
+/*
+ * usk_oracle.c -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, sequential CPU restatement of the UltraSketchLLM sketch
+ * (build, decode, reference products).  Only the test suite, the smoke check
+ * and the CPU-baseline leg of the benchmark may load this file's library; the
+ * product path never does.  It shares no code, header, table or constant
+ * generator with the CUDA library: every constant below is written out here
+ * from its published definition.
+ *
+ * Sources (page title + section):
+ *  - "UltraSketchLLM: Sub-1-Bit LLM Compression via Sketch and Hardware-Friendly
+ *    Operators" (gist.science/es/paper/2506.17255), Resumen Tecnico:
+ *      Metodologia §1 "Diseno de Sketch AbsMaxMin"  -- one value kept per hashed
+ *        bucket, chosen by magnitude;
+ *      Metodologia §4 "Mapeo de Operadores de Matriz" -- decompression is
+ *        W_hat = S . P^T, i.e. every weight reads back its bucket;
+ *      Resultados Experimentales "Eficiencia de Compresion" -- 0.5 bit/weight.
+ *    The lay part of the same page, §2 "La Solucion: El Sketch": a hash drops
+ *    weights into buckets and a bucket keeps only its largest member.
+ *  - The pages give no hash family, tie-break, block geometry or rounding.  The
+ *    readings used here (winner = max of |w|*importance, ties to the smallest
+ *    row-major index, 64-row scale blocks, 64x256 hash tiles, octet-structured
+ *    multiply-shift hash keyed by SplitMix64) are the frozen format of this
+ *    library; each one is written where it is used.
+ *  - SplitMix64: Steele, Lea, Flood, "Fast splittable pseudorandom number
+ *    generators" (OOPSLA 2014); constants as in Vigna's public-domain
+ *    splitmix64.c.
+ *  - Multiply-shift hashing: Dietzfelbinger et al., "A reliable randomized
+ *    algorithm for the closest-pair problem" (J. Algorithms 1997).
+ *  - Range reduction by a 32x32->64 multiply: Lemire, "A fast alternative to
+ *    the modulo reduction" (2016).
+ *  - IEEE 754-2008 binary16 / binary32, round to nearest, ties to even.
+ *
+ * Build: gcc -std=c99 -O2 -ffp-contract=off -fPIC -shared (no fast-math), so
+ * every float operation below is one correctly rounded IEEE operation.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* Status values returned by the oracle (same meanings as the library's). */
+#define ORC_OK 0
+#define ORC_ERR_NULL 1
+#define ORC_ERR_SHAPE 2
+#define ORC_ERR_DTYPE 3
+#define ORC_ERR_NONFINITE 8
+#define ORC_ERR_IMPORTANCE 11
+#define ORC_ERR_SCALE_OVERFLOW 12
+
+/* Format geometry. */
+#define ROWS_PER_BLOCK 64   /* scale block and hash-tile height            */
+#define TILE_COLS 256       /* hash-tile width; K % 256 == 0, so all tiles are full */
+#define WEIGHTS_PER_BUCKET 16
+#define OCTET 8             /* columns that share one hash evaluation      */
+#define CLASSES 32          /* bucket classes per slot                     */
+
+/* ---------------------------------------------------------------- numbers */
+
+static float f32_from_bits(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+static uint32_t bits_from_f32(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+
+/* bf16 is the top half of a binary32. */
+float orc_bf16_to_f32(uint16_t h) { return f32_from_bits((uint32_t)h << 16); }
+
+/* binary16 -> binary32, from the IEEE 754 encoding. */
+float orc_f16_to_f32(uint16_t h) {
+  int sign = (h >> 15) & 1, e = (h >> 10) & 31, man = h & 1023;
+  double v;
+  if (e == 31) return man ? f32_from_bits(0x7fc00000u) : (sign ? -INFINITY : INFINITY);
+  if (e == 0) v = ldexp((double)man, -24);              /* subnormal: man * 2^-24 */
+  else v = ldexp((double)(1024 + man), e - 25);         /* (1.man) * 2^(e-15)     */
+  return (float)(sign ? -v : v);
+}
+
+/* binary32 -> binary16, round to nearest, ties to even, from the definition:
+ * find the binary16 quantum for |f|, round |f| / quantum to an integer (ties
+ * to even), and encode.  Every double step below is exact. */
+uint16_t orc_f32_to_f16(float f) {
+  uint32_t u = bits_from_f32(f);
+  uint16_t sign = (uint16_t)((u >> 16) & 0x8000u);
+  if (isnan(f)) return (uint16_t)(sign | 0x7e00u);
+  double a = fabs((double)f);
+  if (isinf(f) || a >= 65520.0) return (uint16_t)(sign | 0x7c00u); /* 65520 = 65504 + half ulp */
+  if (a == 0.0) return sign;
+  int ex;
+  frexp(a, &ex);                              /* a = fr * 2^ex, fr in [0.5, 1) */
+  int e = ex - 1;                             /* a in [2^e, 2^(e+1))           */
+  double q = (e < -14) ? ldexp(1.0, -24) : ldexp(1.0, e - 10);
+  double n = nearbyint(a / q);                /* ties to even (default mode)   */
+  double r = n * q;
+  if (r == 0.0) return sign;
+  if (r < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)n); /* subnormal */
+  frexp(r, &ex);
+  e = ex - 1;
+  if (e > 15) return (uint16_t)(sign | 0x7c00u);
+  uint16_t man = (uint16_t)((r / ldexp(1.0, e) - 1.0) * 1024.0);
+  return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | man);
+}
+
+/* ------------------------------------------------------------- hashing */
+
+/* SplitMix64: output n (n = 1, 2, ...) of the generator seeded with `seed` is
+ * mix(seed + n * gamma). */
+uint64_t orc_splitmix64(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + n * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+/* Tiles per 64-row block of a K-column matrix. */
+static int64_t tiles_per_row(int64_t K) { return K / TILE_COLS; }
+
+/* Hash key of tile `tile_id`: A (odd multiplier) and C (offset) of the affine
+ * multiply-shift hash are the low and high halves of SplitMix64 output
+ * tile_id + 1. */
+void orc_tile_hash_params(uint64_t seed, uint64_t tile_id, uint32_t* A, uint32_t* C) {
+  uint64_t z = orc_splitmix64(seed, tile_id + 1);
+  *A = (uint32_t)z | 1u;
+  *C = (uint32_t)(z >> 32);
+}
+
+/* Global code index of weight (i, j) in an M x K matrix.
+ * Row block rb = i / 64 (row r inside it), tile tc = j / 256 (column c inside
+ * it).  The 8 columns of octet o = c / 8 (o in 0..31) share one hash value:
+ *   m     = r * 32 + o                           (octet's index in the tile)
+ *   h     = A * m + C  (mod 2^32)                (multiply-shift, keyed per tile)
+ *   slot  = floor(h * 4 / 2^32)                  (4 slots per class)
+ *   class = (o + r) mod 32
+ *   sub   = c mod 8
+ *   b     = (slot * 32 + class) * 8 + sub        (bucket inside the tile, 0..1023)
+ * A tile holds 64*256 weights and 1024 buckets (16 weights per bucket); its
+ * codes are stored from rb * (4K) + 1024 * tc.  Every (class, sub) pair owns
+ * exactly one octet column per row, i.e. 64 members spread over 4 slots. */
+int64_t orc_bucket_index(int64_t K, uint64_t seed, int64_t i, int64_t j) {
+  int64_t rb = i / ROWS_PER_BLOCK, r = i % ROWS_PER_BLOCK;
+  int64_t tc = j / TILE_COLS, c = j % TILE_COLS;
+  int64_t T = tiles_per_row(K);
+  int64_t o = c / OCTET, sub = c % OCTET;
+  uint32_t A, C;
+  orc_tile_hash_params(seed, (uint64_t)(rb * T + tc), &A, &C);
+  uint32_t m = (uint32_t)(r * (TILE_COLS / OCTET) + o);
+  uint32_t h = A * m + C;
+  int64_t slot = (int64_t)(((uint64_t)h * 4u) >> 32);
+  int64_t cls = (o + r) % CLASSES;
+  int64_t b = (slot * CLASSES + cls) * OCTET + sub;
+  return rb * (4 * K) + 1024 * tc + b;
+}
+
+/* ------------------------------------------------------------- shapes */
+
+static int check_shape(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return ORC_ERR_SHAPE;
+  if (M % ROWS_PER_BLOCK != 0 || K % 256 != 0) return ORC_ERR_SHAPE;
+  if (K > (1LL << 20) || M > (1LL << 22)) return ORC_ERR_SHAPE;
+  return ORC_OK;
+}
+
+static float load_elem(const void* p, int dtype, int64_t idx) {
+  if (dtype == 0) return ((const float*)p)[idx];
+  return orc_bf16_to_f32(((const uint16_t*)p)[idx]);
+}
+
+/* -------------------------------------------------------------- build */
+
+/* Build the sketch of W [M, K] (row stride ldw elements; dtype 0 = fp32,
+ * 1 = bf16 bit patterns) with per-column importance imp [K] (NULL = all ones).
+ *
+ * Per bucket the kept member is the one with the largest selection key
+ * k = fp32(|w|) * imp_j (one IEEE fp32 multiply); equal keys go to the member
+ * with the smallest row-major index.  The bucket keeps that member's signed
+ * value v (0 for a bucket with no member).  Per 64-row block the scale is
+ * s16 = binary16(max |v| / 127) and each code is
+ * clamp(round_half_even(v / float(s16)), -127, 127), or 0 when s16 == 0.
+ *
+ * Outputs: codes [M*K/16] int8, scales [M/64] binary16 bits.  Optional:
+ * winner [M*K/16] (row-major flat index i*K + j of each bucket's kept member,
+ * -1 if empty) and value [M*K/16] (the kept fp32 value).
+ *
+ * The scan below visits the weights of each tile in row-major order and keeps
+ * a running best per bucket, which is the sequential hash-and-update the pages
+ * describe; the maximum does not depend on the order. */
+int orc_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw,
+              const float* imp, uint64_t seed, int8_t* codes, uint16_t* scales,
+              int64_t* winner, float* value) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
+  if (M == 0) return ORC_OK;
+  if (!codes || !scales) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) scales[rb] = 0;
+    return ORC_OK;
+  }
+  if (!W || ldw < K) return ORC_ERR_NULL;
+  if (imp) {
+    for (int64_t j = 0; j < K; ++j) {
+      uint32_t u = bits_from_f32(imp[j]);
+      if ((u >> 31) || !isfinite(imp[j])) return ORC_ERR_IMPORTANCE;
+    }
+  }
+  int64_t nb = M * K / WEIGHTS_PER_BUCKET;
+  int64_t per_block = 4 * K;             /* buckets per 64-row block */
+  float* bestkey = (float*)malloc(sizeof(float) * (size_t)per_block);
+  int64_t* bestidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)per_block);
+  float* val = (float*)malloc(sizeof(float) * (size_t)per_block);
+  if (!bestkey || !bestidx || !val) { free(bestkey); free(bestidx); free(val); return ORC_ERR_NULL; }
+  int status = ORC_OK;
+  for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
+    for (int64_t b = 0; b < per_block; ++b) { bestkey[b] = -1.0f; bestidx[b] = -1; }
+    /* selection: a running best per bucket */
+    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
+      int64_t i = rb * ROWS_PER_BLOCK + r;
+      for (int64_t j = 0; j < K; ++j) {
+        float w = load_elem(W, dtype, i * ldw + j);
+        if (!isfinite(w)) status = ORC_ERR_NONFINITE;
+        float k = fabsf(w) * (imp ? imp[j] : 1.0f);
+        int64_t b = orc_bucket_index(K, seed, i, j) - rb * per_block;
+        int64_t flat = i * K + j;
+        /* strictly larger key wins; an equal key never displaces the earlier
+         * (smaller-index) member because the scan is in row-major order */
+        if (k > bestkey[b] || bestidx[b] < 0) { bestkey[b] = k; bestidx[b] = flat; }
+      }
+    }
+    /* kept values and the block maximum */
+    float mx = 0.0f;
+    for (int64_t b = 0; b < per_block; ++b) {
+      float v = 0.0f;
+      if (bestidx[b] >= 0) {
+        int64_t i = bestidx[b] / K, j = bestidx[b] % K;
+        v = load_elem(W, dtype, i * ldw + j);
+      }
+      val[b] = v;
+      if (fabsf(v) > mx) mx = fabsf(v);
+    }
+    /* scale */
+    uint16_t s16 = orc_f32_to_f16(mx / 127.0f);
+    if ((s16 & 0x7c00u) == 0x7c00u) status = status ? status : ORC_ERR_SCALE_OVERFLOW;
+    scales[rb] = s16;
+    float s = orc_f16_to_f32(s16);
+    /* quantization */
+    for (int64_t b = 0; b < per_block; ++b) {
+      int8_t code = 0;
+      if (s != 0.0f) {
+        float q = nearbyintf(val[b] / s);
+        if (q > 127.0f) q = 127.0f;
+        if (q < -127.0f) q = -127.0f;
+        code = (int8_t)q;           /* NaN never reaches here for finite input */
+        if (isnan(q)) code = 0;
+      }
+      int64_t g = rb * per_block + b;
+      codes[g] = code;
+      if (winner) winner[g] = bestidx[b];
+      if (value) value[g] = val[b];
+    }
+  }
+  (void)nb;
+  free(bestkey); free(bestidx); free(val);
+  return status;
+}
+
+/* ------------------------------------------------------------- decode */
+
+/* W_hat [M, K] fp32: every weight reads its bucket's code and its block scale,
+ * w_hat = float(code) * float(s16) (exact in fp32). */
+int orc_decode(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K,
+               uint64_t seed, float* What) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (M == 0 || K == 0) return ORC_OK;
+  if (!codes || !scales || !What) return ORC_ERR_NULL;
+  for (int64_t i = 0; i < M; ++i) {
+    float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+    for (int64_t j = 0; j < K; ++j)
+      What[i * K + j] = (float)codes[orc_bucket_index(K, seed, i, j)] * s;
+  }
+  return ORC_OK;
+}
+
+/* Reference product y[t][i] = sum_j w_hat[i][j] * x[t][j] in float64, for the
+ * rows listed in rows[0..nrows) (rows == NULL: all M rows, nrows ignored).
+ * x [batch, K] has dtype 0 = fp32, 1 = bf16 bits.  y is [batch, nrows] (or
+ * [batch, M]).  The decoded weight is rebuilt from its bucket for every term,
+ * exactly as W_hat = S . P^T reads it back. */
+int orc_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K,
+                 uint64_t seed, const void* x, int xdtype, int64_t batch,
+                 const int64_t* rows, int64_t nrows, double* y) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (xdtype != 0 && xdtype != 1) return ORC_ERR_DTYPE;
+  if (batch < 0) return ORC_ERR_SHAPE;
+  int64_t nr = rows ? nrows : M;
+  if (nr == 0 || batch == 0) return ORC_OK;
+  if (!y) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t q = 0; q < batch * nr; ++q) y[q] = 0.0;
+    return ORC_OK;
+  }
+  if (!codes || !scales || !x) return ORC_ERR_NULL;
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!wrow) return ORC_ERR_NULL;
+  for (int64_t q = 0; q < nr; ++q) {
+    int64_t i = rows ? rows[q] : q;
+    if (i < 0 || i >= M) { free(wrow); return ORC_ERR_SHAPE; }
+    float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+    for (int64_t j = 0; j < K; ++j)
+      wrow[j] = (double)((float)codes[orc_bucket_index(K, seed, i, j)] * s);
+    for (int64_t t = 0; t < batch; ++t) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j) acc += wrow[j] * (double)load_elem(x, xdtype, t * K + j);
+      y[t * nr + q] = acc;
+    }
+  }
+  free(wrow);
+  return ORC_OK;
+}
+
+/* Storage of a sketch in bytes: codes (1 byte per 16 weights) and scales
+ * (2 bytes per 64-row block). */
+void orc_storage_bytes(int64_t M, int64_t K, int64_t* code_bytes, int64_t* scale_bytes) {
+  *code_bytes = M * K / WEIGHTS_PER_BUCKET;
+  *scale_bytes = 2 * (M / ROWS_PER_BLOCK);
+}
+
+/* Element-wise conversions over arrays (for exhaustive pins). */
+void orc_f32_to_f16_array(const float* in, uint16_t* out, int64_t n) {
+  for (int64_t q = 0; q < n; ++q) out[q] = orc_f32_to_f16(in[q]);
+}
+void orc_f16_to_f32_array(const uint16_t* in, float* out, int64_t n) {
+  for (int64_t q = 0; q < n; ++q) out[q] = orc_f16_to_f32(in[q]);
+}

@@ -1,0 +1,84 @@
+"""Independent pure-Python restatement of the sketch, for tiny matrices.
+
+It pins the C oracle from a second, separately written reading of the format:
+Python integers for the hash, explicit member lists per bucket sorted by
+(key descending, row-major index ascending) instead of a running maximum, and
+numpy's own float16 conversion and rint for the scale and the codes.  It shares
+no code with the oracle or with the CUDA library.
+
+Format (64x256 hash tiles, 64-row scale blocks; "UltraSketchLLM" explainer,
+Metodologia §1 AbsMaxMin sketch, with the library's frozen readings):
+  tile key z = SplitMix64(seed) output number tile_id + 1, tile_id = rb*(K/256)+tc
+  A = low32(z) | 1, C = high32(z)
+  octet o = c // 8, m = 32*r + o, h = (A*m + C) mod 2^32, slot = (4*h) >> 32
+  class = (o + r) % 32, bucket = (slot*32 + class)*8 + c % 8
+"""
+from __future__ import annotations
+
+import numpy as np
+
+MASK64 = (1 << 64) - 1
+
+
+def splitmix64_output(seed: int, n: int) -> int:
+    z = (seed + n * 0x9E3779B97F4A7C15) & MASK64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & MASK64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & MASK64
+    return z ^ (z >> 31)
+
+
+def bucket_of(K: int, seed: int, i: int, j: int) -> int:
+    rb, r = divmod(i, 64)
+    tc, c = divmod(j, 256)
+    tile_id = rb * (K // 256) + tc
+    z = splitmix64_output(seed, tile_id + 1)
+    A = (z & 0xFFFFFFFF) | 1
+    C = z >> 32
+    o = c // 8
+    m = 32 * r + o
+    h = (A * m + C) & 0xFFFFFFFF
+    slot = (4 * h) >> 32
+    cls = (o + r) % 32
+    b = (slot * 32 + cls) * 8 + (c % 8)
+    return rb * 4 * K + 1024 * tc + b
+
+
+def to_f32(W: np.ndarray) -> np.ndarray:
+    if W.dtype == np.float32:
+        return W
+    return (W.astype(np.uint32) << 16).view(np.float32)
+
+
+def build(W: np.ndarray, importance=None, seed: int = 0):
+    """Returns (codes int8, scales uint16, winner int64 flat index or -1)."""
+    Wf = to_f32(np.ascontiguousarray(W))
+    M, K = Wf.shape
+    imp = np.ones(K, np.float32) if importance is None else np.asarray(importance, np.float32)
+    nb = M * K // 16
+    members = [[] for _ in range(nb)]
+    for i in range(M):
+        for j in range(K):
+            members[bucket_of(K, seed, i, j)].append(i * K + j)
+    winner = np.full(nb, -1, dtype=np.int64)
+    value = np.zeros(nb, dtype=np.float32)
+    flat = Wf.reshape(-1)
+    for b, mem in enumerate(members):
+        if not mem:
+            continue
+        keyed = [(-float(np.float32(abs(flat[q])) * imp[q % K]), q) for q in mem]
+        keyed.sort()
+        winner[b] = keyed[0][1]
+        value[b] = flat[winner[b]]
+    codes = np.zeros(nb, dtype=np.int8)
+    scales = np.zeros(M // 64, dtype=np.uint16)
+    per = 4 * K
+    for rb in range(M // 64):
+        v = value[rb * per:(rb + 1) * per]
+        mx = np.float32(np.max(np.abs(v))) if per else np.float32(0)
+        s16 = np.float16(np.float32(mx) / np.float32(127.0))
+        scales[rb] = s16.view(np.uint16)
+        s = np.float32(s16)
+        if s != 0:
+            q = np.rint(v / s)
+            codes[rb * per:(rb + 1) * per] = np.clip(q, -127, 127).astype(np.int8)
+    return codes, scales, winner
