@@ -1,0 +1,172 @@
+/*
+ * usk.h -- C ABI of libusk: UltraSketchLLM sketch weights on NVIDIA B200 (sm_100a).
+ *
+ * The library compresses a weight matrix W [M, K] into a hashed sketch at
+ * 0.5 bit per weight (one int8 code per 16 weights plus one binary16 scale per
+ * 64-row block) and multiplies the sketch with activations without ever
+ * materialising the decompressed matrix.
+ *
+ * Source of the method: "UltraSketchLLM: Sub-1-Bit LLM Compression via Sketch
+ * and Hardware-Friendly Operators" (explainer pages gist.science/es|nl/paper/
+ * 2506.17255), Resumen Tecnico:
+ *   - Metodologia §1 "Diseno de Sketch AbsMaxMin": weights are hashed into a
+ *     smaller shared bucket state and a bucket keeps a single value chosen by
+ *     magnitude (the lay section §2 "El Sketch": it keeps its largest member);
+ *   - Metodologia §2 "Asignacion consciente de la importancia": importance
+ *     decides what is preserved (here: it weights the selection key);
+ *   - Metodologia §4 "Mapeo de Operadores de Matriz": compression is one fused
+ *     select-and-update kernel; decompression is W_hat = S . P^T, i.e. each
+ *     weight reads its bucket back;
+ *   - Resultados Experimentales "Eficiencia de Compresion": 0.5 bit/weight.
+ *
+ * FORMAT (version 1).  The pages fix none of the following; this is the
+ * library's frozen reading.
+ *   Geometry: M % 64 == 0, K % 256 == 0.  Row block rb = rows [64 rb, 64 rb+64)
+ *   carries one binary16 scale.  Hash tile (rb, tc) = that row block x columns
+ *   [256 tc, 256 tc + 256); it owns 1024 buckets.
+ *   Hash of weight (i, j): r = i % 64, c = j % 256, octet o = c / 8,
+ *     z = SplitMix64 output number tile_id + 1 of `seed`, tile_id = rb*(K/256)+tc,
+ *     A = low32(z) | 1, C = high32(z), h = A*(32 r + o) + C  (mod 2^32),
+ *     slot = h >> 30, class = (o + r) mod 32,
+ *     bucket b = (slot*32 + class)*8 + c % 8   in [0, 1024).
+ *   Code storage: codes[rb*4K + 1024*tc + b] (int8), scales[rb] (binary16).
+ *   Selection: key = fp32(|w|) * importance[j] (one fp32 multiply, RN); each
+ *   bucket keeps the signed value v of its member with the largest key, ties to
+ *   the smallest row-major index; an empty bucket keeps 0.
+ *   Scale: s16 = binary16_rn(max_b |v_b| / 127) over the row block.
+ *   Code: clamp(rint_half_even(v / float(s16)), -127, 127); 0 when s16 == 0.
+ *   Decode: w_hat = float(code) * float(s16) (exact in fp32).
+ *
+ * CONVENTIONS
+ *   - All array pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no memory and keeps no state beyond cached kernel attributes.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and reentrant.
+ *   - Argument errors are returned synchronously and nothing is launched.
+ *     A failed launch returns USK_ERR_CUDA.
+ *   - Conditions found on the device (non-finite weights, bad importance, scale
+ *     overflow, a wait that gave up) are OR-ed as USK_FLAG_* bits into
+ *     *d_status when d_status is not NULL; the caller reads it after a sync.
+ *     The library never clears it.
+ */
+#ifndef USK_H_
+#define USK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define USK_API __attribute__((visibility("default")))
+#else
+#define USK_API
+#endif
+
+#define USK_FORMAT_VERSION 1
+#define USK_ROWS_PER_BLOCK 64
+#define USK_TILE_COLS 256
+#define USK_WEIGHTS_PER_BUCKET 16
+#define USK_MAX_M (1 << 21)   /* rows */
+#define USK_MAX_K (1 << 16)   /* columns */
+#define USK_GEMV_MAX_BATCH 15
+#define USK_GEMM_MIN_BATCH 16
+#define USK_GEMM_MAX_BATCH 256
+
+typedef enum {
+  USK_OK = 0,
+  USK_ERR_NULL = 1,            /* a required pointer is NULL                     */
+  USK_ERR_SHAPE = 2,           /* M % 64, K % 256, negative or above the limits   */
+  USK_ERR_DTYPE = 3,           /* unknown usk_dtype                              */
+  USK_ERR_BATCH = 4,           /* batch outside the call's range                 */
+  USK_ERR_WORKSPACE = 5,       /* workspace missing or too small                 */
+  USK_ERR_PARAMS = 6,          /* params NULL or wrong format version            */
+  USK_ERR_CUDA = 7,            /* a CUDA runtime call or a launch failed         */
+  USK_ERR_NONFINITE = 8,       /* (flag decoding) non-finite weight              */
+  USK_ERR_TIMEOUT = 9,         /* (flag decoding) a bounded device wait gave up  */
+  USK_ERR_ALIGN = 10,          /* pointer or stride misaligned (16-byte rule)    */
+  USK_ERR_IMPORTANCE = 11,     /* (flag decoding) importance < 0, -0 or non-finite */
+  USK_ERR_SCALE_OVERFLOW = 12  /* (flag decoding) max|v|/127 above binary16 range */
+} usk_status;
+
+/* Bits OR-ed into *d_status by the device. */
+#define USK_FLAG_NONFINITE_W (1u << 0)
+#define USK_FLAG_BAD_IMPORTANCE (1u << 1)
+#define USK_FLAG_SCALE_OVERFLOW (1u << 2)
+#define USK_FLAG_TIMEOUT (1u << 3)
+
+typedef enum { USK_F32 = 0, USK_BF16 = 1 } usk_dtype;
+
+/* Build parameters: version must be USK_FORMAT_VERSION; flags must be 0. */
+typedef struct {
+  uint32_t version;
+  uint32_t flags;
+  uint64_t seed;
+} usk_params;
+
+/* A built sketch (device pointers, caller-owned). */
+typedef struct {
+  int64_t M, K;
+  uint64_t seed;
+  const int8_t* codes;     /* [M*K/16], 16-byte aligned */
+  const uint16_t* scales;  /* [M/64] binary16 bits      */
+} usk_sketch;
+
+/* Storage of a sketch: code_bytes = M*K/16, scale_bytes = 2*M/64.
+ * Errors: USK_ERR_SHAPE, USK_ERR_NULL (an output pointer). */
+USK_API usk_status usk_sizes(int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes);
+
+/* Build the sketch of W (Metodologia §1 and §4: fused select-and-update).
+ *   W          [M, K] row-major, row stride ldw elements (ldw >= K); fp32 or
+ *              bf16 per wdtype.  W and every row start must be 16-byte aligned
+ *              (ldw % 4 == 0 for fp32, % 8 == 0 for bf16).
+ *   importance [K] fp32 per input column, or NULL for all ones.  Values must
+ *              be finite with the sign bit clear (else USK_FLAG_BAD_IMPORTANCE).
+ *   params     version + seed of the hash.
+ *   codes      [M*K/16] int8 output, 16-byte aligned.   scales [M/64] output.
+ *   d_status   optional device word for USK_FLAG_* bits.
+ * M == 0 is a no-op; K == 0 writes zero scales.  Codes and scales are
+ * bit-identical for any launch geometry. */
+USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t K, int64_t ldw,
+                     const float* importance, const usk_params* params, int8_t* codes,
+                     uint16_t* scales, uint32_t* d_status, void* stream);
+
+/* y = W_hat x for batch 1..15 (Metodologia §4: W_hat = S . P^T applied on the
+ * fly: every weight is rehashed and its bucket gathered; W_hat is never stored).
+ *   x  [batch, K] row-major, fp32 or bf16 per xdtype, 16-byte aligned.
+ *   y  [batch, M] fp32 output (y[t*M + i] = sum_j w_hat[i][j] x[t][j]).
+ * Products of bf16 x are exact and accumulate in fp32; fp32 x is split into
+ * two bf16 terms (|error| <= 2^-16 |x| per element).  batch == 0 or M == 0 is
+ * a no-op; K == 0 writes y = 0.  Results do not depend on the launch. */
+USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
+                    float* y, uint32_t* d_status, void* stream);
+
+/* y = W_hat x for batch 16..256 (multiple of 16) on the tcgen05 tensor cores:
+ * decoded bf16 tiles of W_hat are written to shared memory and multiplied with
+ * bf16 x tiles, fp32 accumulation in tensor memory.
+ *   x_bf16 [batch, K] bf16, 16-byte aligned.  y [batch, M] fp32.
+ *   ws / ws_bytes: unused by this version (may be NULL / 0).
+ * M == 0 is a no-op; K == 0 writes y = 0. */
+USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y,
+                    void* ws, size_t ws_bytes, uint32_t* d_status, void* stream);
+
+/* Test hook: override the launch geometry (0 = default).  build_cluster is the
+ * number of thread blocks per row block in usk_build (1..8); gemv_tiles_per_block
+ * the number of hash tiles per thread block in usk_gemv.  Results are
+ * bit-identical for every geometry; only the split of the work changes.
+ * Process-wide; not thread-safe with concurrent calls. */
+USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block);
+
+/* Static description of a status value. */
+USK_API const char* usk_status_str(usk_status status);
+
+/* Format version compiled into the library. */
+USK_API uint32_t usk_format_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* USK_H_ */

@@ -1,0 +1,28 @@
+"""UltraSketchLLM sketch weights on NVIDIA B200 (sm_100a).
+
+Thin Python face of libusk.so (C ABI in include/usk.h): ``usk_build`` compresses
+a weight matrix into a 0.5 bit/weight hashed sketch; ``usk_gemv`` (batch 1-15)
+and ``usk_gemm`` (batch 16-256) multiply the sketch with activations, rebuilding
+every weight on the fly.  PyTorch supplies device memory and streams only.
+"""
+from ._native import (  # noqa: F401
+    FLAG_BAD_IMPORTANCE,
+    FLAG_NONFINITE_W,
+    FLAG_SCALE_OVERFLOW,
+    FLAG_TIMEOUT,
+    FORMAT_VERSION,
+    GEMM_MAX_BATCH,
+    GEMM_MIN_BATCH,
+    GEMV_MAX_BATCH,
+    LIB_PATH,
+    Sketch,
+    UskError,
+    load_library,
+    usk_build,
+    usk_debug_set_geometry,
+    usk_format_version,
+    usk_gemm,
+    usk_gemv,
+    usk_sizes,
+    usk_status_str,
+)

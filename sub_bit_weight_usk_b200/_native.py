@@ -1,0 +1,206 @@
+"""ctypes binding of libusk.so (include/usk.h): argument marshalling only.
+
+Every step of the sketch build and of the sketch-decode products runs in the
+library's CUDA kernels; this module only turns torch tensors into device
+pointers, picks the current CUDA stream and raises on a non-OK status.  There
+is no CPU fallback: if the library or a GPU is missing, calls fail loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libusk.so")
+
+USK_OK = 0
+USK_F32 = 0
+USK_BF16 = 1
+FORMAT_VERSION = 1
+GEMV_MAX_BATCH = 15
+GEMM_MIN_BATCH = 16
+GEMM_MAX_BATCH = 256
+
+FLAG_NONFINITE_W = 1 << 0
+FLAG_BAD_IMPORTANCE = 1 << 1
+FLAG_SCALE_OVERFLOW = 1 << 2
+FLAG_TIMEOUT = 1 << 3
+
+STATUS_NAMES = {
+    0: "USK_OK", 1: "USK_ERR_NULL", 2: "USK_ERR_SHAPE", 3: "USK_ERR_DTYPE", 4: "USK_ERR_BATCH",
+    5: "USK_ERR_WORKSPACE", 6: "USK_ERR_PARAMS", 7: "USK_ERR_CUDA", 8: "USK_ERR_NONFINITE",
+    9: "USK_ERR_TIMEOUT", 10: "USK_ERR_ALIGN", 11: "USK_ERR_IMPORTANCE", 12: "USK_ERR_SCALE_OVERFLOW",
+}
+
+
+class UskError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (what, STATUS_NAMES.get(status, status), usk_status_str(status)))
+
+
+class UskParams(ctypes.Structure):
+    _fields_ = [("version", ctypes.c_uint32), ("flags", ctypes.c_uint32), ("seed", ctypes.c_uint64)]
+
+
+class UskSketchC(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int64), ("seed", ctypes.c_uint64),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+_lib = None
+
+EXPORTED = ["usk_sizes", "usk_build", "usk_gemv", "usk_gemm", "usk_status_str", "usk_format_version",
+            "usk_debug_set_geometry"]
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libusk.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise OSError("libusk.so not found at %s: build it with __graft_entry__.build() "
+                      "or python -m sub_bit_weight_usk_b200._build" % path)
+    lib = ctypes.CDLL(path)
+    vp, i64, u32p = ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint32)
+    lib.usk_sizes.argtypes = [i64, i64, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
+    lib.usk_sizes.restype = ctypes.c_int
+    lib.usk_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, ctypes.POINTER(UskParams), vp, vp, vp, vp]
+    lib.usk_build.restype = ctypes.c_int
+    lib.usk_gemv.argtypes = [ctypes.POINTER(UskSketchC), vp, ctypes.c_int, i64, vp, vp, vp]
+    lib.usk_gemv.restype = ctypes.c_int
+    lib.usk_gemm.argtypes = [ctypes.POINTER(UskSketchC), vp, i64, vp, vp, ctypes.c_size_t, vp, vp]
+    lib.usk_gemm.restype = ctypes.c_int
+    lib.usk_status_str.argtypes = [ctypes.c_int]
+    lib.usk_status_str.restype = ctypes.c_char_p
+    lib.usk_format_version.argtypes = []
+    lib.usk_format_version.restype = ctypes.c_uint32
+    lib.usk_debug_set_geometry.argtypes = [ctypes.c_int, ctypes.c_int]
+    lib.usk_debug_set_geometry.restype = None
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(st: int, what: str):
+    if st != USK_OK:
+        raise UskError(st, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return USK_BF16
+    if t.dtype == torch.float32:
+        return USK_F32
+    raise TypeError("expected a bfloat16 or float32 tensor, got %s" % t.dtype)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libusk works on CUDA tensors only (no CPU fallback)")
+
+
+def usk_status_str(status: int) -> str:
+    return load_library().usk_status_str(int(status)).decode()
+
+
+def usk_format_version() -> int:
+    return int(load_library().usk_format_version())
+
+
+def usk_sizes(M: int, K: int):
+    c = ctypes.c_size_t()
+    s = ctypes.c_size_t()
+    _check(load_library().usk_sizes(M, K, ctypes.byref(c), ctypes.byref(s)), "usk_sizes")
+    return c.value, s.value
+
+
+@dataclass
+class Sketch:
+    """A built sketch: int8 codes [M*K/16] and binary16 scales [M/64] on the GPU."""
+    M: int
+    K: int
+    seed: int
+    codes: torch.Tensor
+    scales: torch.Tensor  # int16 storage of binary16 bit patterns
+
+    def as_c(self) -> UskSketchC:
+        return UskSketchC(self.M, self.K, self.seed & (2**64 - 1), self.codes.data_ptr() if self.codes.numel() else None,
+                          self.scales.data_ptr() if self.scales.numel() else None)
+
+
+def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int = 0,
+              codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+              status: torch.Tensor | None = None, stream=None) -> Sketch:
+    """Sketch of W [M, K] (bf16 or fp32, CUDA).  Outputs are allocated with torch
+    when not given.  `status` is an optional int32 CUDA tensor of 1 element into
+    which device-detected USK_FLAG_* bits are OR-ed."""
+    _need_cuda(W, importance, codes, scales, status)
+    if W.dim() != 2 or W.stride(1) != 1:
+        raise ValueError("W must be a 2-D row-major tensor")
+    M, K = W.shape
+    nb = M * K // 16
+    if codes is None:
+        codes = torch.empty(max(nb, 1), dtype=torch.int8, device=W.device)[:nb]
+    if scales is None:
+        scales = torch.empty(max(M // 64, 1), dtype=torch.int16, device=W.device)[: M // 64]
+    if importance is not None and (importance.dtype != torch.float32 or not importance.is_contiguous()):
+        raise TypeError("importance must be a contiguous float32 tensor")
+    p = UskParams(FORMAT_VERSION, 0, seed & (2**64 - 1))
+    st = load_library().usk_build(_ptr(W), _dtype_code(W), M, K, W.stride(0), _ptr(importance), ctypes.byref(p),
+                                  _ptr(codes) if nb else None, _ptr(scales) if M // 64 else None,
+                                  _ptr(status), _stream(stream))
+    _check(st, "usk_build")
+    return Sketch(M, K, seed, codes, scales)
+
+
+def usk_gemv(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
+             status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [batch, M] fp32 = W_hat x^T for x [batch, K] (bf16 or fp32), batch 1..15."""
+    _need_cuda(x, y, status)
+    if x.dim() == 1:
+        x = x[None, :]
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, sketch.M), dtype=torch.float32, device=x.device)
+    sk = sketch.as_c()
+    st = load_library().usk_gemv(ctypes.byref(sk), _ptr(x), _dtype_code(x), batch, _ptr(y), _ptr(status),
+                                 _stream(stream))
+    _check(st, "usk_gemv")
+    return y
+
+
+def usk_gemm(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
+             status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [batch, M] fp32 = W_hat x^T for bf16 x [batch, K], batch 16..256 (multiple of 16)."""
+    _need_cuda(x, y, status)
+    if x.dtype != torch.bfloat16 or not x.is_contiguous() or x.dim() != 2:
+        raise TypeError("x must be a contiguous 2-D bfloat16 tensor")
+    batch = x.shape[0]
+    if y is None:
+        y = torch.empty((batch, sketch.M), dtype=torch.float32, device=x.device)
+    sk = sketch.as_c()
+    st = load_library().usk_gemm(ctypes.byref(sk), _ptr(x), batch, _ptr(y), None, 0, _ptr(status),
+                                 _stream(stream))
+    _check(st, "usk_gemm")
+    return y
+
+
+def usk_debug_set_geometry(build_cluster: int = 0, gemv_tiles_per_block: int = 0) -> None:
+    load_library().usk_debug_set_geometry(int(build_cluster), int(gemv_tiles_per_block))

@@ -1,0 +1,155 @@
+// usk_api.cu -- the C ABI of libusk (declared in include/usk.h): argument
+// validation, then one kernel launch per call.  No allocation, no global state
+// beyond CUDA's cached kernel attributes.
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "usk.h"
+
+namespace usk {
+cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
+                         uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
+                         cudaStream_t stream, int cluster_override);
+cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                        const void* x, bool xf32, int batch, float* y, cudaStream_t stream, int tpc_override);
+cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream);
+}  // namespace usk
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+usk_status check_shape(int64_t M, int64_t K) {
+  if (M < 0 || K < 0) return USK_ERR_SHAPE;
+  if (M % USK_ROWS_PER_BLOCK != 0 || K % USK_TILE_COLS != 0) return USK_ERR_SHAPE;
+  if (M > USK_MAX_M || K > USK_MAX_K) return USK_ERR_SHAPE;
+  return USK_OK;
+}
+
+usk_status check_sketch(const usk_sketch* s) {
+  if (!s) return USK_ERR_NULL;
+  usk_status st = check_shape(s->M, s->K);
+  if (st != USK_OK) return st;
+  if (s->M > 0 && s->K > 0) {
+    if (!s->codes || !s->scales) return USK_ERR_NULL;
+    if (!aligned16(s->codes)) return USK_ERR_ALIGN;
+    if ((reinterpret_cast<uintptr_t>(s->scales) & 1u) != 0) return USK_ERR_ALIGN;
+  }
+  return USK_OK;
+}
+
+usk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? USK_OK : USK_ERR_CUDA; }
+
+// Optional launch-geometry overrides (used by the determinism tests to show the
+// result does not depend on the geometry).  0 = library default.
+int g_build_cluster = 0;
+int g_gemv_tiles_per_block = 0;
+
+}  // namespace
+
+extern "C" {
+
+USK_API uint32_t usk_format_version(void) { return USK_FORMAT_VERSION; }
+
+USK_API const char* usk_status_str(usk_status status) {
+  switch (status) {
+    case USK_OK: return "ok";
+    case USK_ERR_NULL: return "a required pointer is NULL";
+    case USK_ERR_SHAPE: return "shape: M must be a multiple of 64, K a multiple of 256, within the limits";
+    case USK_ERR_DTYPE: return "unknown dtype";
+    case USK_ERR_BATCH: return "batch outside the range of this call";
+    case USK_ERR_WORKSPACE: return "workspace missing or too small";
+    case USK_ERR_PARAMS: return "params NULL, wrong format version or non-zero flags";
+    case USK_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case USK_ERR_NONFINITE: return "non-finite weight";
+    case USK_ERR_TIMEOUT: return "a bounded device wait gave up";
+    case USK_ERR_ALIGN: return "pointer or row stride not 16-byte aligned";
+    case USK_ERR_IMPORTANCE: return "importance must be finite with the sign bit clear";
+    case USK_ERR_SCALE_OVERFLOW: return "block maximum / 127 exceeds the binary16 range";
+  }
+  return "unknown status";
+}
+
+USK_API usk_status usk_sizes(int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes) {
+  usk_status st = check_shape(M, K);
+  if (st != USK_OK) return st;
+  if (!code_bytes || !scale_bytes) return USK_ERR_NULL;
+  *code_bytes = static_cast<size_t>(M) * static_cast<size_t>(K) / USK_WEIGHTS_PER_BUCKET;
+  *scale_bytes = 2 * static_cast<size_t>(M / USK_ROWS_PER_BLOCK);
+  return USK_OK;
+}
+
+USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t K, int64_t ldw,
+                     const float* importance, const usk_params* params, int8_t* codes,
+                     uint16_t* scales, uint32_t* d_status, void* stream) {
+  usk_status st = check_shape(M, K);
+  if (st != USK_OK) return st;
+  if (wdtype != USK_F32 && wdtype != USK_BF16) return USK_ERR_DTYPE;
+  if (!params) return USK_ERR_PARAMS;
+  if (params->version != USK_FORMAT_VERSION || params->flags != 0) return USK_ERR_PARAMS;
+  if (M == 0) return USK_OK;
+  if (!scales) return USK_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(scales) & 1u) != 0) return USK_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (K == 0) return from_cuda(cudaMemsetAsync(scales, 0, 2 * static_cast<size_t>(M / 64), s));
+  if (!W || !codes) return USK_ERR_NULL;
+  if (ldw < K) return USK_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(codes)) return USK_ERR_ALIGN;
+  if (ldw % (wdtype == USK_BF16 ? 8 : 4) != 0) return USK_ERR_ALIGN;
+  if (importance && !aligned16(importance)) return USK_ERR_ALIGN;
+  cudaError_t e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes,
+                                    scales, d_status, s, g_build_cluster);
+  if (e != cudaSuccess) return USK_ERR_CUDA;
+  return from_cuda(cudaGetLastError());
+}
+
+USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch, float* y,
+                    uint32_t* d_status, void* stream) {
+  (void)d_status;
+  usk_status st = check_sketch(sketch);
+  if (st != USK_OK) return st;
+  if (xdtype != USK_F32 && xdtype != USK_BF16) return USK_ERR_DTYPE;
+  if (batch < 0 || batch > USK_GEMV_MAX_BATCH) return USK_ERR_BATCH;
+  if (batch == 0 || sketch->M == 0) return USK_OK;
+  if (!y) return USK_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (sketch->K == 0)
+    return from_cuda(cudaMemsetAsync(y, 0, sizeof(float) * static_cast<size_t>(batch * sketch->M), s));
+  if (!x) return USK_ERR_NULL;
+  if (!aligned16(x)) return USK_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(y) & 3u) != 0) return USK_ERR_ALIGN;
+  cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
+                                   xdtype == USK_F32, static_cast<int>(batch), y, s, g_gemv_tiles_per_block);
+  if (e != cudaSuccess) return USK_ERR_CUDA;
+  return from_cuda(cudaGetLastError());
+}
+
+USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y, void* ws,
+                    size_t ws_bytes, uint32_t* d_status, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  usk_status st = check_sketch(sketch);
+  if (st != USK_OK) return st;
+  if (batch < USK_GEMM_MIN_BATCH || batch > USK_GEMM_MAX_BATCH || batch % 16 != 0) return USK_ERR_BATCH;
+  if (sketch->M == 0) return USK_OK;
+  if (!y) return USK_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (sketch->K == 0)
+    return from_cuda(cudaMemsetAsync(y, 0, sizeof(float) * static_cast<size_t>(batch * sketch->M), s));
+  if (!x_bf16) return USK_ERR_NULL;
+  if (!aligned16(x_bf16) || !aligned16(y)) return USK_ERR_ALIGN;
+  cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
+                                   static_cast<int>(batch), y, d_status, s);
+  if (e != cudaSuccess) return USK_ERR_CUDA;
+  return from_cuda(cudaGetLastError());
+}
+
+// Test hooks: launch-geometry overrides (0 restores the defaults).  They change
+// how work is split between thread blocks, never the result.
+USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block) {
+  g_build_cluster = build_cluster;
+  g_gemv_tiles_per_block = gemv_tiles_per_block;
+}
+
+}  // extern "C"

@@ -1,0 +1,127 @@
+// usk_common.cuh -- device helpers shared by the libusk kernels (sm_100a).
+//
+// Format constants and the hash of the sketch format (version 1, declared in
+// include/usk.h).  The hash key of a tile is a SplitMix64 output (Steele, Lea
+// and Flood, OOPSLA 2014), written here from its published definition.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "usk.h"
+
+#include <type_traits>
+#include <utility>
+
+namespace usk {
+
+// Compile-time loop: f(std::integral_constant<int, I>{}) for I = 0 .. N-1.
+template <typename F, int... I>
+__device__ __forceinline__ void static_for_impl(F&& f, std::integer_sequence<int, I...>) {
+  (f(std::integral_constant<int, I>{}), ...);
+}
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  static_for_impl(f, std::make_integer_sequence<int, N>{});
+}
+
+constexpr int kRowsPerBlock = 64;                                 // scale block and tile height
+constexpr int kTileCols = 256;                                    // hash tile width
+constexpr int kBucketsPerTile = kRowsPerBlock * kTileCols / 16;   // 1024
+constexpr int kOctetsPerRow = kTileCols / 8;                      // 32
+
+// SplitMix64 output number n of the generator seeded with `seed`.
+__host__ __device__ __forceinline__ uint64_t splitmix64(uint64_t seed, uint64_t n) {
+  uint64_t z = seed + n * 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+// Multiply-shift hash key (A odd, C) of tile `tile_id`.
+__host__ __device__ __forceinline__ uint2 tile_key(uint64_t seed, uint64_t tile_id) {
+  uint64_t z = splitmix64(seed, tile_id + 1);
+  return make_uint2(static_cast<uint32_t>(z) | 1u, static_cast<uint32_t>(z >> 32));
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void sts16(uint32_t addr, uint16_t v) {
+  asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
+// [addr + OFF] forms: the constant offset is folded into the instruction.
+template <int OFF>
+__device__ __forceinline__ uint32_t lds32_off(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(addr), "n"(OFF));
+  return v;
+}
+
+template <int OFF>
+__device__ __forceinline__ void atoms_max_u32_off(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.max.u32 [%0+%2], %1;" ::"r"(addr), "r"(v), "n"(OFF) : "memory");
+}
+
+template <int OFF>
+__device__ __forceinline__ void atoms_min_u32_off(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.min.u32 [%0+%2], %1;" ::"r"(addr), "r"(v), "n"(OFF) : "memory");
+}
+
+__device__ __forceinline__ void atoms_max_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.max.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void atoms_min_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.min.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint4 ldg_nc128(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// bf16 pair (low half = element 0) -> two fp32 values, exact.
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+__device__ __forceinline__ void report(uint32_t* d_status, uint32_t flags) {
+  if (flags && d_status) atomicOr(d_status, flags);
+}
+
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate (legacy warp-level MMA).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+}  // namespace usk

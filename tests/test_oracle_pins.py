@@ -327,3 +327,13 @@ def test_gemv_f64_matches_numpy_matmul(xdtype):
     rows = np.array([0, 63, 64, 191])
     ys = oracle.gemv_f64(o["codes"], o["scales"], M, K, x, 12, rows=rows)
     assert np.allclose(ys, ref[:, rows], rtol=1e-12, atol=1e-12)
+
+
+def test_build_rows_slice_equals_full_build():
+    W = gen.weights_normal(256, 512, 31, 0.02, "bf16")
+    full = oracle.build_sketch(W, None, 31)
+    per = 64 * 512 // 16
+    for rb0 in (1, 2):
+        part = oracle.build_sketch(W[64 * rb0:64 * rb0 + 128], None, 31, row_block0=rb0)
+        assert np.array_equal(part["codes"], full["codes"][rb0 * per:(rb0 + 2) * per])
+        assert np.array_equal(part["scales"], full["scales"][rb0:rb0 + 2])
