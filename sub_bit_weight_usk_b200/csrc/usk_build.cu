@@ -8,20 +8,23 @@
 //
 // Design (B200, sm_100a):
 //  * One thread block per (row block, group of hash tiles); the blocks of one
-//    row block form a thread-block cluster so that the row-block scale is an
+//    row block form a thread-block cluster, so the row-block scale is an
 //    exchange of per-block maxima through distributed shared memory: no
-//    workspace and one launch.
-//  * A tile (64 x 256 weights, 1024 buckets) is read once from HBM with 16-byte
-//    coalesced loads and kept in registers (64 weights per thread) while three
-//    passes resolve the winners with 32-bit shared-memory atomics, which run
-//    about four times faster than 64-bit ones on this part:
-//      pass 1  atomicMax of the key bits per bucket (order-preserving: keys are
-//              non-negative fp32, whose bit patterns sort like the values);
-//      pass 2  members whose key equals the bucket maximum atomicMin their
-//              tile-local row-major index;
-//      pass 3  the member holding that index writes its signed value.
-//  * Bucket key arrays are laid out [slot][sub][class] so that the 32 lanes of
-//    a warp (one row, 32 octets, 32 distinct classes) hit 32 distinct banks.
+//    workspace, one launch.
+//  * Weight tiles (64 x 256) stream from HBM into shared memory with 1-D bulk
+//    copies (the tensor memory accelerator) completing on mbarriers, double
+//    buffered, so the copy of tile i+1 overlaps the selection of tile i.
+//  * Selection uses order-preserving 32-bit keys and shared-memory atomics
+//    (64-bit shared atomics run about four times slower on this part):
+//      - bf16 weights, unit importance: ONE pass.  The packed word
+//        (|w| bits << 16) | (16384 - l) << 1 | sign  orders by |w|, then by
+//        the smaller tile-local row-major index l, and carries the sign, so
+//        one atomicMax per weight leaves the winner itself in the bucket.
+//      - with importance (or fp32 weights): pass 1 atomicMax of the fp32 key
+//        bits; pass 2 the members equal to the maximum atomicMin the packed
+//        (l, value) word, which keeps the smallest index and its value.
+//  * Bucket arrays are laid out [slot][sub][class]: the 32 lanes of a warp
+//    (one row, 32 octets, 32 distinct classes) hit 32 distinct banks.
 #include <cooperative_groups.h>
 
 #include "usk_common.cuh"
@@ -29,6 +32,8 @@
 namespace cg = cooperative_groups;
 
 namespace usk {
+
+constexpr int kBuildThreads = 256;
 
 struct BuildArgs {
   const void* W;
@@ -39,236 +44,249 @@ struct BuildArgs {
   int8_t* codes;
   uint16_t* scales;
   uint32_t* status;
-  int T;  // tiles per row block = K / 256
-  int C;  // thread blocks per row block (cluster size)
+  int T;     // tiles per row block = K / 256
+  int C;     // thread blocks per row block (cluster size)
+  int tpc;   // max tiles per block
+  int nbuf;  // weight-tile buffers (1 or 2)
 };
 
-constexpr int kBuildThreads = 512;
-constexpr int kUnits = kRowsPerBlock * kTileCols / 8 / kBuildThreads;  // octets per thread per tile (4)
-constexpr int kRowStep = kBuildThreads / 32;                            // rows between a thread's octets (16)
-
-// The 64 weights (8 octets) one thread owns in a tile, kept in registers.
-template <bool BF16>
-struct TileRegs;
-
-template <>
-struct TileRegs<true> {
-  uint32_t u[kUnits][4];
-  __device__ __forceinline__ void load(int q, const void* p) {
-    uint4 v = ldg_nc128(p);
-    u[q][0] = v.x; u[q][1] = v.y; u[q][2] = v.z; u[q][3] = v.w;
-  }
-  __device__ __forceinline__ float get(int q, int s) const {
-    return (s & 1) ? bf16hi(u[q][s >> 1]) : bf16lo(u[q][s >> 1]);
-  }
-  // value stored per bucket: the raw bf16 bits (exact)
-  __device__ __forceinline__ uint16_t stored(int q, int s) const {
-    return static_cast<uint16_t>((s & 1) ? (u[q][s >> 1] >> 16) : (u[q][s >> 1] & 0xFFFFu));
-  }
-  // Opaque to the compiler: keys are recomputed in each pass instead of being
-  // kept live across the barriers (64 extra registers otherwise).
-  __device__ __forceinline__ void fence() {
-#pragma unroll
-    for (int q = 0; q < kUnits; ++q)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) asm volatile("" : "+r"(u[q][i]));
-  }
+// Shared-memory layout (byte offsets from a 128-byte aligned base).
+struct BuildLayout {
+  uint32_t wbuf, keys, win, vals, bars, misc, total;
 };
 
-template <>
-struct TileRegs<false> {
-  float f[kUnits][8];
-  __device__ __forceinline__ void load(int q, const void* p) {
-    uint4 a = ldg_nc128(p);
-    uint4 b = ldg_nc128(static_cast<const char*>(p) + 16);
-    f[q][0] = __uint_as_float(a.x); f[q][1] = __uint_as_float(a.y);
-    f[q][2] = __uint_as_float(a.z); f[q][3] = __uint_as_float(a.w);
-    f[q][4] = __uint_as_float(b.x); f[q][5] = __uint_as_float(b.y);
-    f[q][6] = __uint_as_float(b.z); f[q][7] = __uint_as_float(b.w);
-  }
-  __device__ __forceinline__ float get(int q, int s) const { return f[q][s]; }
-  __device__ __forceinline__ uint32_t stored(int q, int s) const { return __float_as_uint(f[q][s]); }
-  __device__ __forceinline__ void fence() {
-#pragma unroll
-    for (int q = 0; q < kUnits; ++q)
-#pragma unroll
-      for (int i = 0; i < 8; ++i) asm volatile("" : "+f"(f[q][i]));
-  }
-};
-
-template <bool BF16>
-using ValT = typename std::conditional<BF16, uint16_t, uint32_t>::type;
-
-template <bool BF16>
-__device__ __forceinline__ float stored_to_f32(ValT<BF16> v);
-template <>
-__device__ __forceinline__ float stored_to_f32<true>(uint16_t v) { return __uint_as_float(static_cast<uint32_t>(v) << 16); }
-template <>
-__device__ __forceinline__ float stored_to_f32<false>(uint32_t v) { return __uint_as_float(v); }
-
-// Shared memory: keys[1024] u32 | widx[1024] u32 | misc[4] u32 | vals[tpc][1024]
-__host__ __device__ constexpr size_t build_smem_bytes(int tiles_per_block, bool bf16) {
-  return (2 * 1024 + 4) * 4 + static_cast<size_t>(tiles_per_block) * 1024 * (bf16 ? 2 : 4);
+__host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int tpc, int nbuf) {
+  const bool single = bf16 && !has_imp;
+  const uint32_t tile = kRowsPerBlock * kTileCols * (bf16 ? 2u : 4u);
+  BuildLayout L;
+  L.wbuf = 0;
+  L.keys = L.wbuf + nbuf * tile;
+  L.win = L.keys + (single ? 0u : 2u * 4096u);
+  L.vals = L.win + ((single || bf16) ? 2u * 4096u : 2u * 8192u);
+  L.bars = (L.vals + static_cast<uint32_t>(tpc) * 1024u * (bf16 ? 2u : 4u) + 7u) & ~7u;
+  L.misc = L.bars + 64u;
+  L.total = L.misc + 64u;
+  return L;
 }
 
 template <bool BF16, bool HAS_IMP>
-__global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs a) {
-  extern __shared__ __align__(16) uint32_t sm[];
-  uint32_t* keys = sm;
-  uint32_t* widx = sm + 1024;
-  uint32_t* misc = sm + 2048;  // [0] block max |v| bits, [1] non-finite screen
-  ValT<BF16>* vals_all = reinterpret_cast<ValT<BF16>*>(sm + 2048 + 4);
+__global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a) {
+  constexpr bool kSingle = BF16 && !HAS_IMP;
+  constexpr uint32_t kRowBytes = kTileCols * (BF16 ? 2 : 4);
+  constexpr uint32_t kTileBytes = kRowsPerBlock * kRowBytes;
+  constexpr uint32_t kWinBytes = (kSingle || BF16) ? 4096u : 8192u;  // one tile's winner words
+  extern __shared__ __align__(128) uint8_t smraw[];
+  const BuildLayout L = build_layout(BF16, HAS_IMP, a.tpc, a.nbuf);
+  const uint32_t s0 = smem_u32(smraw);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smraw + L.misc);
 
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
   const int rb = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nt = (a.T - crank + a.C - 1) / a.C;  // this block's tiles: crank, crank + C, ...
+
+  // ---- init: barriers, winner words of both slots, keys of both slots
+  if (tid == 0) {
+    for (int b = 0; b < a.nbuf; ++b) mbar_init(s0 + L.bars + 8 * b, 1);
+    mbar_fence_init();
+    misc[0] = 0u;
+  }
+  {
+    uint32_t* win32 = reinterpret_cast<uint32_t*>(smraw + L.win);
+    const uint32_t init = kSingle ? 0u : 0xFFFFFFFFu;
+    for (uint32_t q = tid; q < 2u * kWinBytes / 4u; q += kBuildThreads) win32[q] = init;
+    if (!kSingle) {
+      uint32_t* k32 = reinterpret_cast<uint32_t*>(smraw + L.keys);
+      for (int q = tid; q < 2048; q += kBuildThreads) k32[q] = 0u;
+    }
+  }
+  __syncthreads();
+
+  auto issue = [&](int i) {  // bulk-copy tile i of this block into buffer i % nbuf
+    const int tc = crank + a.C * i;
+    const int buf = i % a.nbuf;
+    const uint32_t bar = s0 + L.bars + 8 * buf;
+    const uint32_t dst = s0 + L.wbuf + buf * kTileBytes;
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    const char* src = static_cast<const char*>(a.W) +
+                      (static_cast<int64_t>(rb) * kRowsPerBlock * a.ldw + static_cast<int64_t>(tc) * kTileCols) *
+                          (BF16 ? 2 : 4);
+    const int64_t stride = a.ldw * (BF16 ? 2 : 4);
+    for (int r = 0; r < kRowsPerBlock; ++r) bulk_g2s(dst + r * kRowBytes, src + r * stride, kRowBytes, bar);
+  };
+  if (tid == 0)
+    for (int i = 0; i < a.nbuf && i < nt; ++i) issue(i);
+
   uint32_t flags = 0;
-  uint32_t vmax = 0;  // running max of |v| bits over this thread's winners
+  uint32_t vmax = 0;  // max |v| bits over the winners this thread converts
+  using ValT = typename std::conditional<BF16, uint16_t, uint32_t>::type;
+  ValT* vals_all = reinterpret_cast<ValT*>(smraw + L.vals);
 
-  int nt = 0;
-  for (int tc = crank; tc < a.T; tc += a.C, ++nt) {
-    ValT<BF16>* vals = vals_all + nt * 1024;
-    for (int q = tid; q < 1024; q += kBuildThreads) {
-      keys[q] = 0u;
-      widx[q] = 0xFFFFFFFFu;
-      vals[q] = 0;
-    }
-    if (tid == 0) misc[1] = 0u;
-
-    // Issue the tile's loads before the barrier so that their latency overlaps it.
-    const int64_t col0 = static_cast<int64_t>(tc) * kTileCols + lane * 8;
-    TileRegs<BF16> w;
-#pragma unroll
-    for (int q = 0; q < kUnits; ++q) {
-      const int64_t row = static_cast<int64_t>(rb) * kRowsPerBlock + warp + kRowStep * q;
-      const char* p = static_cast<const char*>(a.W) + (row * a.ldw + col0) * (BF16 ? 2 : 4);
-      w.load(q, p);
-    }
+  for (int i = 0; i < nt; ++i) {
+    const int tc = crank + a.C * i;
+    const int buf = i % a.nbuf;
+    const uint2 hk = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + tc);
     float imp[8];
     if (HAS_IMP) {
-      const uint4 i0 = ldg_nc128(a.imp + col0);
-      const uint4 i1 = ldg_nc128(a.imp + col0 + 4);
+      const int64_t col0 = static_cast<int64_t>(tc) * kTileCols + lane * 8;
+      const uint4 i0 = ldg_nc128(a.imp + col0), i1 = ldg_nc128(a.imp + col0 + 4);
       const uint32_t ib[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        // importance must be finite with the sign bit clear
         if ((ib[s] >> 31) || (ib[s] & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_BAD_IMPORTANCE;
         imp[s] = __uint_as_float(ib[s]);
       }
     }
-    const uint2 hk = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + tc);
-    uint32_t kb[kUnits];  // shared byte offset of (slot, sub 0, class) for each owned octet
-#pragma unroll
-    for (int q = 0; q < kUnits; ++q) {
-      const uint32_t r = warp + kRowStep * q;
+    if (!mbar_wait(s0 + L.bars + 8 * buf, (i / a.nbuf) & 1)) flags |= USK_FLAG_TIMEOUT;
+
+    const uint32_t wt = s0 + L.wbuf + buf * kTileBytes;
+    const uint32_t win_s = s0 + L.win + (i & 1) * kWinBytes;
+    const uint32_t keys_s = s0 + L.keys + (i & 1) * 4096u;
+
+    // pass 1 (and the only pass for bf16 with unit importance)
+#pragma unroll 2
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t r = warp + 8 * q;
       const uint32_t h = hk.x * (32u * r + lane) + hk.y;
-      kb[q] = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
-    }
-    const uint32_t keys_s = smem_u32(keys), widx_s = smem_u32(widx);
-    __syncthreads();
-
-    // pass 1: per-bucket maximum of the key bits
-#pragma unroll
-    for (int q = 0; q < kUnits; ++q) {
-      const uint32_t base = keys_s + kb[q];
-      static_for<8>([&](auto S) {
-        constexpr int s = decltype(S)::value;
-        const float f = w.get(q, s);
-        const float k = HAS_IMP ? fabsf(f) * imp[s] : fabsf(f);
-        atoms_max_u32_off<128 * s>(base, __float_as_uint(k));
-      });
-    }
-    __syncthreads();
-
-    // Non-finite screen: a NaN or Inf weight forces a key >= +Inf bits in its
-    // bucket (an fp32 overflow of |w| * importance can too; the exact check
-    // below separates the two).
-    {
-      const uint2 v = reinterpret_cast<const uint2*>(keys)[tid];
-      if (max(v.x, v.y) >= 0x7F800000u) misc[1] = 1u;
-    }
-
-    // pass 2: members that reach the maximum compete on their index
-    w.fence();
-    uint32_t cand = 0u;
-#pragma unroll
-    for (int q = 0; q < kUnits; ++q) {
-      const uint32_t kbase = keys_s + kb[q], wbase = widx_s + kb[q];
-      const uint32_t l0 = static_cast<uint32_t>((warp + kRowStep * q) * kTileCols + lane * 8);
-      static_for<8>([&](auto S) {
-        constexpr int s = decltype(S)::value;
-        const float f = w.get(q, s);
-        const float k = HAS_IMP ? fabsf(f) * imp[s] : fabsf(f);
-        if (__float_as_uint(k) == lds32_off<128 * s>(kbase)) {
-          atoms_min_u32_off<128 * s>(wbase, l0 + s);
-          cand |= 1u << (q * 8 + s);
-        }
-      });
-    }
-    __syncthreads();
-    if (misc[1]) {
-#pragma unroll
-      for (int q = 0; q < kUnits; ++q)
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          if ((__float_as_uint(w.get(q, s)) & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
-    }
-
-    // pass 3: the winning member writes its signed value
-    w.fence();
-    if (cand) {
-#pragma unroll
-      for (int q = 0; q < kUnits; ++q) {
-        const uint32_t wbase = widx_s + kb[q];
-        const uint32_t l0 = static_cast<uint32_t>((warp + kRowStep * q) * kTileCols + lane * 8);
+      const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+      const uint32_t l0 = r * kTileCols + lane * 8;
+      if (BF16) {
+        const uint4 v = lds128(wt + r * kRowBytes + lane * 16);
+        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
         static_for<8>([&](auto S) {
           constexpr int s = decltype(S)::value;
-          if ((cand >> (q * 8 + s)) & 1u) {
-            if (lds32_off<128 * s>(wbase) == l0 + s) {
-              vals[(kb[q] >> 2) + 32 * s] = w.stored(q, s);
-              vmax = max(vmax, __float_as_uint(fabsf(w.get(q, s))));
+          const uint32_t b16 = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
+          if (kSingle) {
+            const uint32_t p = ((b16 & 0x7FFFu) << 16) | ((16384u - (l0 + s)) << 1) | (b16 >> 15);
+            atoms_max_u32_off<128 * s>(win_s + off, p);
+          } else {
+            const float k = fabsf(__uint_as_float(b16 << 16)) * imp[s];
+            atoms_max_u32_off<128 * s>(keys_s + off, __float_as_uint(k));
+          }
+        });
+      } else {
+        const uint4 v0 = lds128(wt + r * kRowBytes + lane * 32), v1 = lds128(wt + r * kRowBytes + lane * 32 + 16);
+        const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        static_for<8>([&](auto S) {
+          constexpr int s = decltype(S)::value;
+          const float f = __uint_as_float(wv[s]);
+          const float k = HAS_IMP ? fabsf(f) * imp[s] : fabsf(f);
+          atoms_max_u32_off<128 * s>(keys_s + off, __float_as_uint(k));
+        });
+      }
+    }
+
+    if (!kSingle) {
+      __syncthreads();
+      // pass 2: members that reach the maximum keep the smallest index and its value
+#pragma unroll 2
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t r = warp + 8 * q;
+        const uint32_t h = hk.x * (32u * r + lane) + hk.y;
+        const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+        const uint32_t l0 = r * kTileCols + lane * 8;
+        uint32_t wv[8];
+        if (BF16) {
+          const uint4 v = lds128(wt + r * kRowBytes + lane * 16);
+          wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
+          wv[4] = wv[5] = wv[6] = wv[7] = 0u;
+        } else {
+          const uint4 v0 = lds128(wt + r * kRowBytes + lane * 32), v1 = lds128(wt + r * kRowBytes + lane * 32 + 16);
+          wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w; wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
+        }
+        static_for<8>([&](auto S) {
+          constexpr int s = decltype(S)::value;
+          uint32_t bits;
+          if (BF16) bits = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
+          else bits = wv[s];
+          const float f = BF16 ? __uint_as_float(bits << 16) : __uint_as_float(bits);
+          const float k = HAS_IMP ? fabsf(f) * imp[s] : fabsf(f);
+          if (__float_as_uint(k) == lds32_off<128 * s>(keys_s + off)) {
+            // every non-finite weight is a candidate, or loses to one (a NaN key)
+            if ((__float_as_uint(f) & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
+            if (BF16) {
+              atoms_min_u32_off<128 * s>(win_s + off, ((l0 + s) << 16) | bits);
+            } else {
+              atoms_min_u64_off<256 * s>(win_s + 2 * off, (static_cast<uint64_t>(l0 + s) << 32) | bits);
             }
           }
         });
       }
     }
-    __syncthreads();
+    __syncthreads();  // tile i resolved; its weight buffer is free
+    if (tid == 0 && i + a.nbuf < nt) issue(i + a.nbuf);
+
+    // compact this tile's winners into its value array and reset the slot
+    // (reused by tile i + 2, after the barrier of tile i + 1)
+    {
+      ValT* vals = vals_all + i * 1024;
+      uint32_t* win32 = reinterpret_cast<uint32_t*>(smraw + L.win + (i & 1) * kWinBytes);
+      uint64_t* win64 = reinterpret_cast<uint64_t*>(smraw + L.win + (i & 1) * kWinBytes);
+      uint32_t* k32 = reinterpret_cast<uint32_t*>(smraw + L.keys + (i & 1) * 4096u);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kidx = tid * 4 + e;
+        uint32_t vb, mag;
+        if (kSingle) {
+          const uint32_t p = win32[kidx];
+          vb = ((p >> 16) & 0x7FFFu) | ((p & 1u) << 15);
+          mag = (vb & 0x7FFFu) << 16;
+          win32[kidx] = 0u;
+        } else if (BF16) {
+          const uint32_t p = win32[kidx];
+          vb = (p == 0xFFFFFFFFu) ? 0u : (p & 0xFFFFu);
+          mag = (vb & 0x7FFFu) << 16;
+          win32[kidx] = 0xFFFFFFFFu;
+          k32[kidx] = 0u;
+        } else {
+          const uint64_t p = win64[kidx];
+          vb = (p == ~0ull) ? 0u : static_cast<uint32_t>(p);
+          mag = vb & 0x7FFFFFFFu;
+          win64[kidx] = ~0ull;
+          k32[kidx] = 0u;
+        }
+        if (kSingle && (mag & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
+        vals[kidx] = static_cast<ValT>(vb);
+        vmax = max(vmax, mag);
+      }
+    }
   }
 
-  // block maximum of |v|, then the row-block maximum across the cluster
+  // ---- row-block maximum across the cluster, scale, quantization
   vmax = __reduce_max_sync(0xFFFFFFFFu, vmax);
-  if (tid == 0) misc[0] = 0u;
-  __syncthreads();
   if (lane == 0) atomicMax(&misc[0], vmax);
-  cluster.sync();
-  uint32_t mbits = 0u;
-  for (int c = 0; c < a.C; ++c) mbits = max(mbits, *cluster.map_shared_rank(&misc[0], c));
-
-  const float m = __uint_as_float(mbits);
-  const __half s16 = __float2half_rn(m / 127.0f);
-  const float s = __half2float(s16);
+  cluster.sync();  // also orders every block's value arrays before the reads below
+  if (warp == 0) {
+    uint32_t m = 0;
+    if (lane < a.C) m = *cluster.map_shared_rank(&misc[0], lane);
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (lane == 0) misc[1] = m;
+  }
+  __syncthreads();
+  const float mx = __uint_as_float(misc[1]);
+  const __half s16 = __float2half_rn(mx / 127.0f);
+  const float sc = __half2float(s16);
   if (crank == 0 && tid == 0) {
     a.scales[rb] = __half_as_ushort(s16);
-    if (isinf(s)) flags |= USK_FLAG_SCALE_OVERFLOW;
+    if (isinf(sc)) flags |= USK_FLAG_SCALE_OVERFLOW;
   }
-
-  // quantize this block's tiles; each thread writes 4 consecutive codes
-  nt = 0;
-  for (int tc = crank; tc < a.T; tc += a.C, ++nt) {
-    const ValT<BF16>* vals = vals_all + nt * 1024;
-    const uint32_t b0 = 2u * tid;
+  for (int i = 0; i < nt; ++i) {
+    const int tc = crank + a.C * i;
+    const ValT* vals = vals_all + i * 1024;
+    const uint32_t b0 = 4u * tid;  // 4 consecutive buckets: same slot and class, subs b0 % 8 .. + 3
     const uint32_t base = (b0 >> 8) * 256u + (b0 & 7u) * 32u + ((b0 >> 3) & 31u);
     uint32_t packed = 0u;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float v = stored_to_f32<BF16>(vals[base + 32u * e]);
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t vb = vals[base + 32u * e];
+      const float v = BF16 ? __uint_as_float(vb << 16) : __uint_as_float(vb);
       int code = 0;
-      if (s != 0.0f) code = static_cast<int>(fminf(fmaxf(rintf(v / s), -127.0f), 127.0f));
+      if (sc != 0.0f) code = static_cast<int>(fminf(fmaxf(rintf(v / sc), -127.0f), 127.0f));
       packed |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * e);
     }
     int8_t* dst = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(tc) + b0;
-    *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+    *reinterpret_cast<uint32_t*>(dst) = packed;
   }
   report(a.status, flags);
   cluster.sync();  // keep this block's shared memory alive until every peer has read it
@@ -276,23 +294,52 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
 
 // ---------------------------------------------------------------- launch
 
-static int build_cluster_size(int T) { return T < 8 ? T : 8; }
+struct BuildPlan {
+  int C, tpc, nbuf;
+  uint32_t smem;
+};
+
+static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override) {
+  auto mk = [&](int C, int nbuf) {
+    BuildPlan p;
+    p.C = C < T ? C : T;
+    p.tpc = (T + p.C - 1) / p.C;
+    p.nbuf = nbuf;
+    p.smem = build_layout(bf16, has_imp, p.tpc, nbuf).total + 128;  // + alignment slack
+    return p;
+  };
+  if (cluster_override > 0) {
+    BuildPlan p = mk(cluster_override, 2);
+    if (p.smem > 220u * 1024u) p = mk(cluster_override, 1);
+    return p;
+  }
+  BuildPlan p = mk(8, 2);
+  if (p.smem > 112u * 1024u && T > 8) p = mk(16, 2);  // keep two blocks per SM
+  if (p.smem > 220u * 1024u) p = mk(p.C, 1);
+  return p;
+}
 
 template <bool BF16, bool HAS_IMP>
-static cudaError_t launch_build_t(const BuildArgs& a, int64_t RB, cudaStream_t stream) {
-  const int tpc = (a.T + a.C - 1) / a.C;
-  const size_t smem = build_smem_bytes(tpc, BF16);
+static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, int cluster_override) {
+  const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override);
+  a.C = p.C;
+  a.tpc = p.tpc;
+  a.nbuf = p.nbuf;
   auto kern = build_kernel<BF16, HAS_IMP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(p.smem));
   if (e != cudaSuccess) return e;
+  if (p.C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.gridDim = dim3(p.C, static_cast<unsigned>(RB), 1);
   cfg.blockDim = dim3(kBuildThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = p.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = a.C;
+  attr[0].val.clusterDim.x = p.C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
@@ -307,10 +354,13 @@ cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t
   a.W = W; a.ldw = ldw; a.K = K; a.imp = imp; a.seed = seed;
   a.codes = codes; a.scales = scales; a.status = status;
   a.T = static_cast<int>(K / kTileCols);
-  a.C = cluster_override > 0 ? (cluster_override < a.T ? cluster_override : a.T) : build_cluster_size(a.T);
+  a.C = a.tpc = a.nbuf = 0;
   const int64_t RB = M / kRowsPerBlock;
-  if (bf16) return imp ? launch_build_t<true, true>(a, RB, stream) : launch_build_t<true, false>(a, RB, stream);
-  return imp ? launch_build_t<false, true>(a, RB, stream) : launch_build_t<false, false>(a, RB, stream);
+  if (bf16)
+    return imp ? launch_build_t<true, true>(a, RB, stream, cluster_override)
+               : launch_build_t<true, false>(a, RB, stream, cluster_override);
+  return imp ? launch_build_t<false, true>(a, RB, stream, cluster_override)
+             : launch_build_t<false, false>(a, RB, stream, cluster_override);
 }
 
 }  // namespace usk

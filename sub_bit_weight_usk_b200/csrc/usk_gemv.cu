@@ -46,23 +46,38 @@ struct GemvArgs {
 
 constexpr int kGemvThreads = 256;
 
-// smem: key table [tpc] uint2 (padded to 16 B) | codes bf16 [tpc][1024];
-// the partial sums later alias the code area.
-__host__ __device__ constexpr size_t gemv_stage_bytes(int tpc) {
-  return static_cast<size_t>((tpc * 8 + 15) / 16 * 16) + static_cast<size_t>(tpc) * 2048;
-}
-__host__ __device__ constexpr size_t gemv_part_bytes(int nb) {
-  return static_cast<size_t>(8) * (nb * 8) * 64 * 4;  // [warp][n][row] fp32
-}
-__host__ __device__ constexpr size_t gemv_smem_bytes(int tpc, int nb, int batch) {
-  return (gemv_stage_bytes(tpc) > gemv_part_bytes(nb) ? gemv_stage_bytes(tpc) : gemv_part_bytes(nb)) +
-         static_cast<size_t>(batch) * 64 * 4;
+// Shared memory (bytes):
+//   key table  [tpc] uint2, padded to 16
+//   codes      [tpc][1024] bf16 (2 KiB per tile)
+//   x slice    [nvalid rows][tpc * 512 + 16] bf16 (rows padded by 16 B: conflict-free)
+//   block sums [batch][64] fp32
+// The per-warp partials [8][NB * 8][64] fp32 alias the first three areas after
+// the main loop.
+struct GemvLayout {
+  uint32_t keys, codes, xs, xrow, stage_end, parts, cta, total;
+};
+
+__host__ __device__ inline GemvLayout gemv_layout(int tpc, int nb, int batch, bool xf32) {
+  GemvLayout L;
+  const uint32_t nvalid = static_cast<uint32_t>(xf32 ? 2 * batch : batch);
+  L.keys = 0;
+  L.codes = (static_cast<uint32_t>(tpc) * 8u + 15u) / 16u * 16u;
+  L.xs = L.codes + static_cast<uint32_t>(tpc) * 2048u;
+  L.xrow = static_cast<uint32_t>(tpc) * 512u + 16u;
+  L.stage_end = L.xs + nvalid * L.xrow;
+  L.parts = 0;
+  const uint32_t parts_end = 8u * static_cast<uint32_t>(nb) * 8u * 64u * 4u;
+  L.cta = ((L.stage_end > parts_end ? L.stage_end : parts_end) + 15u) / 16u * 16u;
+  L.total = L.cta + static_cast<uint32_t>(batch) * 64u * 4u;
+  return L;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2_from_i8(int lo, int hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(static_cast<float>(lo), static_cast<float>(hi));
   return *reinterpret_cast<uint32_t*>(&v);
 }
+
+__device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
 template <int NB, bool XF32>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
@@ -73,32 +88,70 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);  // >= 1 by construction of C
-  uint2* keytab = reinterpret_cast<uint2*>(sm);
-  const size_t code_off = static_cast<size_t>((a.tpc * 8 + 15) / 16 * 16);
-  uint8_t* scodes = sm + code_off;
-  float* part = reinterpret_cast<float*>(sm);  // aliases the stage area after the main loop
-  float* cta_part = reinterpret_cast<float*>(
-      sm + (gemv_stage_bytes(a.tpc) > gemv_part_bytes(NB) ? gemv_stage_bytes(a.tpc) : gemv_part_bytes(NB)));
+  const int nvalid = XF32 ? 2 * a.batch : a.batch;
+  const GemvLayout L = gemv_layout(a.tpc, NB, a.batch, XF32);
+  uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
+  const uint32_t sm_s = smem_u32(sm);
 
-  // ---- stage: hash keys and codes (int8 -> bf16) of this block's tiles
+  // ---- stage: hash keys, codes (int8 -> bf16) and the x slice, all loads in flight at once
   if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
   {
-    const int8_t* src = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
-    const int n16 = nt * 64;  // 16-code chunks
-    for (int q = tid; q < n16; q += kGemvThreads) {
-      const uint4 v = ldg_nc128(src + 16 * q);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-      uint32_t o[8];
+    const int8_t* csrc = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
+    const int ncode = nt * 64;                                   // 16-byte code chunks
+    const int xchunks_row = XF32 ? nt * 64 : nt * 32;            // 16-byte x chunks per batch row
+    const int nx = a.batch * xchunks_row;
+    const int total = ncode + nx;
+    constexpr int kR = 8;  // loads in flight per thread per round
+    for (int base = 0; base < total; base += kR * kGemvThreads) {
+      uint4 v[kR];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c0 = static_cast<int8_t>(w[e] & 0xFF), c1 = static_cast<int8_t>((w[e] >> 8) & 0xFF);
-        const int c2 = static_cast<int8_t>((w[e] >> 16) & 0xFF), c3 = static_cast<int8_t>(w[e] >> 24);
-        o[2 * e] = pack_bf16x2_from_i8(c0, c1);
-        o[2 * e + 1] = pack_bf16x2_from_i8(c2, c3);
+      for (int u = 0; u < kR; ++u) {
+        const int q = base + u * kGemvThreads + tid;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (q < ncode) {
+          v[u] = ldg_nc128(csrc + 16 * q);
+        } else if (q < total) {
+          const int qx = q - ncode, n = qx / xchunks_row, c = qx % xchunks_row;
+          const char* xrow = static_cast<const char*>(a.x) + (static_cast<int64_t>(n) * a.K +
+                                                                static_cast<int64_t>(t0) * kTileCols) * (XF32 ? 4 : 2);
+          v[u] = ldg_nc128(xrow + 16 * c);
+        }
       }
-      uint4* dst = reinterpret_cast<uint4*>(scodes + 32 * q);
-      dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-      dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+#pragma unroll
+      for (int u = 0; u < kR; ++u) {
+        const int q = base + u * kGemvThreads + tid;
+        if (q < ncode) {
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+          uint32_t o[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o[2 * e] = pack_bf16x2_from_i8(static_cast<int8_t>(w[e] & 0xFF), static_cast<int8_t>((w[e] >> 8) & 0xFF));
+            o[2 * e + 1] = pack_bf16x2_from_i8(static_cast<int8_t>((w[e] >> 16) & 0xFF), static_cast<int8_t>(w[e] >> 24));
+          }
+          const uint32_t dst = sm_s + L.codes + 32u * q;
+          sts128(dst, make_uint4(o[0], o[1], o[2], o[3]));
+          sts128(dst + 16, make_uint4(o[4], o[5], o[6], o[7]));
+        } else if (q < total) {
+          const int qx = q - ncode, n = qx / xchunks_row, c = qx % xchunks_row;
+          if (!XF32) {
+            sts128(sm_s + L.xs + n * L.xrow + 16u * c, v[u]);
+          } else {
+            // 4 floats -> hi row n and lo row n + batch (x = hi + lo + O(2^-16 |x|))
+            const float f0 = __uint_as_float(v[u].x), f1 = __uint_as_float(v[u].y);
+            const float f2 = __uint_as_float(v[u].z), f3 = __uint_as_float(v[u].w);
+            const __nv_bfloat162 h01 = __floats2bfloat162_rn(f0, f1), h23 = __floats2bfloat162_rn(f2, f3);
+            const float2 g01 = __bfloat1622float2(h01), g23 = __bfloat1622float2(h23);
+            const __nv_bfloat162 l01 = __floats2bfloat162_rn(f0 - g01.x, f1 - g01.y);
+            const __nv_bfloat162 l23 = __floats2bfloat162_rn(f2 - g23.x, f3 - g23.y);
+            const uint32_t hi_dst = sm_s + L.xs + n * L.xrow + 8u * c;
+            const uint32_t lo_dst = sm_s + L.xs + (n + a.batch) * L.xrow + 8u * c;
+            asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(hi_dst), "r"(bf16x2_bits(h01)), "r"(bf16x2_bits(h23))
+                         : "memory");
+            asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(lo_dst), "r"(bf16x2_bits(l01)), "r"(bf16x2_bits(l23))
+                         : "memory");
+          }
+        }
+      }
     }
   }
   __syncthreads();
@@ -110,7 +163,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   uint32_t cls16[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) cls16[k] = ((c0 + 8u * k) & 31u) * 16u;
-  const uint32_t codes_s = smem_u32(scodes);
+  const uint32_t codes_s = sm_s + L.codes;
 
   float d[4][NB][4];
 #pragma unroll
@@ -122,44 +175,17 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
 
   for (int tt = 0; tt < nt; ++tt) {
     const uint2 hk = keytab[tt];
-    const int64_t col = static_cast<int64_t>(t0 + tt) * kTileCols + 8 * o;
     // B fragments (x) of this tile for the lane's octet: n = 8 nb + g
     uint32_t bq[NB][4];
 #pragma unroll
     for (int nb = 0; nb < NB; ++nb) {
       const int n = nb * 8 + g;
-      if (!XF32) {
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (n < a.batch) v = ldg_nc128(static_cast<const uint16_t*>(a.x) + n * a.K + col);
-        bq[nb][0] = v.x; bq[nb][1] = v.y; bq[nb][2] = v.z; bq[nb][3] = v.w;
-      } else {
-        // rows n < batch carry hi = bf16(x); rows batch <= n < 2 batch carry lo = bf16(x - hi)
-        bq[nb][0] = bq[nb][1] = bq[nb][2] = bq[nb][3] = 0u;
-        if (n < 2 * a.batch) {
-          const int src_row = n < a.batch ? n : n - a.batch;
-          const float* xp = static_cast<const float*>(a.x) + src_row * a.K + col;
-          const uint4 u0 = ldg_nc128(xp), u1 = ldg_nc128(xp + 4);
-          const float xf[8] = {__uint_as_float(u0.x), __uint_as_float(u0.y), __uint_as_float(u0.z),
-                               __uint_as_float(u0.w), __uint_as_float(u1.x), __uint_as_float(u1.y),
-                               __uint_as_float(u1.z), __uint_as_float(u1.w)};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            __nv_bfloat162 hi = __floats2bfloat162_rn(xf[2 * e], xf[2 * e + 1]);
-            uint32_t r;
-            if (n < a.batch) {
-              r = *reinterpret_cast<uint32_t*>(&hi);
-            } else {
-              const float2 hf = __bfloat1622float2(hi);
-              __nv_bfloat162 lo = __floats2bfloat162_rn(xf[2 * e] - hf.x, xf[2 * e + 1] - hf.y);
-              r = *reinterpret_cast<uint32_t*>(&lo);
-            }
-            bq[nb][e] = r;
-          }
-        }
-      }
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (n < nvalid) v = lds128(sm_s + L.xs + n * L.xrow + (tt * 32 + o) * 16);
+      bq[nb][0] = v.x; bq[nb][1] = v.y; bq[nb][2] = v.z; bq[nb][3] = v.w;
     }
     const uint32_t tile_s = codes_s + tt * 2048u;
-    uint32_t h = hk.x * (32u * g + o) + hk.y;
+    const uint32_t h = hk.x * (32u * g + o) + hk.y;
     const uint32_t d512 = hk.x * 512u, d256 = hk.x * 256u;
 #pragma unroll
     for (int mb = 0; mb < 4; ++mb) {
@@ -174,10 +200,11 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
       }
     }
   }
-  __syncthreads();  // stage area is reused for the partials below
+  __syncthreads();  // the stage area is reused for the partials below
 
-  // ---- per-warp partials -> block partial (fixed order over warps)
-  const int nvalid = XF32 ? 2 * a.batch : a.batch;
+  // ---- per-warp partials -> block sums (fixed order over warps)
+  float* part = reinterpret_cast<float*>(sm + L.parts);
+  float* cta_part = reinterpret_cast<float*>(sm + L.cta);
 #pragma unroll
   for (int mb = 0; mb < 4; ++mb) {
 #pragma unroll
@@ -203,20 +230,20 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
     }
     cta_part[q] = acc;
   }
-  (void)nvalid;
   cluster.sync();
 
-  // ---- cluster reduction (fixed order over blocks) and the row-block scale
-  if (crank == 0) {
+  // ---- cluster reduction (fixed order over blocks) and the row-block scale;
+  // block c finishes outputs c, c + C, ...
+  {
     const float s = __half2float(__ushort_as_half(a.scales[rb]));
-    for (int q = tid; q < a.batch * 64; q += kGemvThreads) {
+    for (int q = crank * kGemvThreads + tid; q < a.batch * 64; q += a.C * kGemvThreads) {
       float acc = 0.0f;
       for (int c = 0; c < a.C; ++c) acc += *cluster.map_shared_rank(&cta_part[q], c);
       const int n = q >> 6, r = q & 63;
       a.y[static_cast<int64_t>(n) * a.M + static_cast<int64_t>(rb) * 64 + r] = acc * s;
     }
   }
-  cluster.sync();  // keep shared memory alive until block 0 has read it
+  cluster.sync();  // keep shared memory alive until every peer has read it
 }
 
 // ---------------------------------------------------------------- launch
@@ -238,7 +265,7 @@ static GemvGeometry gemv_geometry(int64_t K, int tpc_override) {
 
 template <int NB, bool XF32>
 static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_smem_bytes(a.tpc, NB, a.batch);
+  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32).total;
   auto kern = gemv_kernel<NB, XF32>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;

@@ -1,0 +1,99 @@
+"""usk_gemm (tcgen05 tensor cores) on the GPU against the float64 oracle product.
+
+Tolerance: max|y - y_ref| <= 1e-3 * max|y_ref| (bf16 x, exact bf16 products,
+fp32 accumulation in tensor memory)."""
+import numpy as np
+import pytest
+import torch
+
+import gen
+import oracle
+import sub_bit_weight_usk_b200 as usk
+from tests.gpu_util import codes_np, rel_err, scales_np, status_tensor, to_dev
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+
+def _sketch(W, seed):
+    sk = usk.usk_build(to_dev(W), None, seed)
+    torch.cuda.synchronize()
+    return sk, {"codes": codes_np(sk), "scales": scales_np(sk)}
+
+
+def _check(sk, o, x, rows=None):
+    st = status_tensor()
+    y = usk.usk_gemm(sk, to_dev(x), status=st).cpu().numpy()
+    assert int(st.item()) == 0
+    ref = oracle.gemv_f64(o["codes"], o["scales"], sk.M, sk.K, x, sk.seed, rows=rows)
+    if rows is not None:
+        y = y[:, rows]
+    e = rel_err(y, ref)
+    assert e <= TOL, "relative error %.3e" % e
+
+
+@pytest.mark.parametrize("M,K", [(128, 256), (192, 1024), (128, 4352), (320, 2048)])
+@pytest.mark.parametrize("batch", [16, 32, 48, 64, 128, 256])
+def test_gemm_matches_oracle(M, K, batch):
+    W = gen.weights_student_t(M, K, 11, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _sketch(W, 5)
+    x = gen.activations(batch, K, 12, "bf16")
+    _check(sk, o, x)
+
+
+def test_gemm_equals_oracle_built_sketch():
+    W = gen.weights_normal(256, 1024, 13, 0.02, "bf16")
+    o = oracle.build_sketch(W, None, 6)
+    sk, _ = _sketch(W, 6)
+    assert np.array_equal(codes_np(sk), o["codes"])
+    _check(sk, o, gen.activations(16, 1024, 14, "bf16"))
+
+
+@pytest.mark.parametrize("batch", [16, 64])
+def test_gemm_layer_workload_full(batch):
+    cfg = gen.layer(batch)
+    sk = usk.usk_build(to_dev(cfg["W"]), to_dev(cfg["importance"]), cfg["seed"])
+    torch.cuda.synchronize()
+    _check(sk, {"codes": codes_np(sk), "scales": scales_np(sk)}, cfg["x"])
+
+
+@pytest.mark.parametrize("name", ["up", "down"])
+def test_gemm_mlp70b_sampled_rows(name):
+    cfg = gen.mlp70b(name, 64)
+    sk, o = _sketch(cfg["W"], cfg["seed"])
+    M = sk.M
+    rows = np.array([0, 1, 127, 128, M // 2, M - 65, M - 1])
+    _check(sk, o, cfg["x"], rows=rows)
+
+
+def test_gemm_matches_gemv_on_same_sketch():
+    W = gen.weights_normal(256, 2048, 15, 0.02, "bf16")
+    sk, _ = _sketch(W, 7)
+    x = to_dev(gen.activations(16, 2048, 16, "bf16"))
+    yg = usk.usk_gemm(sk, x)
+    yv = torch.cat([usk.usk_gemv(sk, x[i:i + 8]) for i in range(0, 16, 8)])
+    d = (yg - yv).abs().max().item() / yv.abs().max().item()
+    assert d <= 1e-5
+
+
+def test_gemm_repeatable_bitwise():
+    W = gen.weights_normal(512, 4096, 17, 0.02, "bf16")
+    sk, _ = _sketch(W, 8)
+    x = to_dev(gen.activations(32, 4096, 18, "bf16"))
+    a = usk.usk_gemm(sk, x)
+    for _ in range(3):
+        assert torch.equal(a, usk.usk_gemm(sk, x))
+
+
+def test_gemm_zero_sketch_and_errors():
+    sk, _ = _sketch(np.zeros((128, 512), np.float32), 3)
+    y = usk.usk_gemm(sk, to_dev(gen.activations(16, 512, 1, "bf16")))
+    assert torch.count_nonzero(y).item() == 0
+    x = to_dev(gen.activations(24, 512, 1, "bf16"))
+    with pytest.raises(usk.UskError) as e:
+        usk.usk_gemm(sk, x)  # not a multiple of 16
+    assert e.value.status == 4
+    with pytest.raises(usk.UskError) as e:
+        usk.usk_gemm(sk, x[:8])  # below 16: usk_gemv's range
+    assert e.value.status == 4
