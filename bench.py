@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the UltraSketchLLM sketch hot path on B200.
+
+One step = one pass of the whole hot path over one 4096x4096 bf16 layer:
+usk_build (key, hash, scatter-select, winner, scale, quantize), usk_gemv at
+batch 1 (rehash + gather decode, product) and usk_gemm at batch 16 (decode into
+tcgen05 tiles).  The headline value is usk_gemv GB/s (algorithmic bytes of one
+call / its average launch duration); usk_build Gweights/s rides along.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl usk|reference]
+
+For N > 1 run under torchrun (one rank per GPU): every rank sketches and
+multiplies its own layer (weak scaling, no data-path collective); the timing is
+the max over ranks.  `--impl reference` times the plain CPU oracle on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import gen  # noqa: E402
+
+M = K = 4096
+GEMV_BATCH = 1
+GEMM_BATCH = 16
+N_WCOPIES = 8      # 8 x 32 MiB of weights per build cycle  (> L2)
+N_SKETCHES = 256   # 256 x 1 MiB of codes per decode cycle  (> L2)
+GRAPH_STEPS = 256  # steps per captured CUDA graph
+
+METRIC = "usk_gemv GB/s & % roofline (4096x4096, batch 1); usk_build Gweights/s"
+WORKLOAD = ("one 4096x4096 bf16 layer, Student-t(4) x 0.02 with 0.1% outliers x20, importance = mean |x| "
+            "over 128 N(0,1) rows; usk_build + usk_gemv batch 1 + usk_gemm batch 16")
+
+# algorithmic bytes / flops per call
+N_W = M * K
+GEMV_BYTES = N_W // 16 + 2 * (M // 64) + 2 * K * GEMV_BATCH + 4 * M * GEMV_BATCH  # 1,073,280
+GEMM_BYTES = N_W // 16 + 2 * (M // 64) + 2 * K * GEMM_BATCH + 4 * M * GEMM_BATCH
+BUILD_BYTES = 2 * N_W + N_W // 16 + 4 * K + 2 * (M // 64)
+GEMM_FLOPS = 2 * N_W * GEMM_BATCH
+
+SMS = 148
+SMEM_BYTES_PER_CLK = 128  # shared-memory load bandwidth per SM per clock
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def rooflines(peaks, t_build_s, t_gemv_s, t_gemm_s, traffic):
+    """Roofline of each kernel from its algorithmic work and the measured peaks.
+
+    usk_build is HBM-bound (2 B of bf16 weight in, 1/16 B of code out per weight).
+    usk_gemv / usk_gemm decode every weight by a shared-memory gather of its
+    bucket code: at least 1 byte per weight through the 128 B/clk/SM shared
+    memory pipe, which binds before HBM (codes are 1/16 B per weight); gemm also
+    checks the dense bf16 tensor time."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    clk = peaks.get("sm_max_mhz", 1965.0) * 1e6
+    smem = SMS * SMEM_BYTES_PER_CLK * clk
+    src = peaks["source"]
+
+    def line(bound, achieved, peak, unit, tr):
+        return {"bound": bound, "achieved": round(achieved, 3), "peak": round(peak, 3), "unit": unit,
+                "frac": round(achieved / peak, 4), "traffic": tr, "peak_source": src}
+
+    out = {}
+    # build: HBM
+    out["usk_build"] = line("hbm", BUILD_BYTES / t_build_s / 1e9, hbm / 1e9, "GB/s", traffic.get("usk_build"))
+    # gemv: gather-bound; expressed in algorithmic GB/s against the bytes/time at the binding bound
+    t_bound = max(GEMV_BYTES / hbm, N_W / smem)
+    out["usk_gemv"] = line("alu", GEMV_BYTES / t_gemv_s / 1e9, GEMV_BYTES / t_bound / 1e9, "GB/s",
+                           traffic.get("usk_gemv"))
+    out["usk_gemv"]["binding"] = "shared-memory gather (1 B/weight at 128 B/clk/SM)"
+    t_bound = max(GEMM_BYTES / hbm, N_W / smem, GEMM_FLOPS / (peaks["bf16_tflops"] * 1e12))
+    out["usk_gemm"] = line("alu", GEMM_BYTES / t_gemm_s / 1e9, GEMM_BYTES / t_bound / 1e9, "GB/s",
+                           traffic.get("usk_gemm"))
+    out["usk_gemm"]["tensor_tflops"] = round(GEMM_FLOPS / t_gemm_s / 1e12, 3)
+    return out
+
+
+def source_sha(name):
+    p = os.path.join(ROOT, "sub_bit_weight_usk_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_traffic():
+    """DRAM bytes per launch from the committed ncu summary, only while the
+    kernel source still matches the one the counters were taken on."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    out = {}
+    if not os.path.exists(p):
+        return out
+    with open(p) as f:
+        d = json.load(f)
+    for kern, rec in d.items():
+        try:
+            if rec.get("source_sha") == source_sha(rec["source"]):
+                out[kern] = rec["dram_bytes_per_launch"]
+        except (KeyError, OSError):
+            pass
+    return out
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def aggregate(world, per_rank_gemv_s, per_rank_build_s, per_rank_step_s):
+    """Whole-job numbers from per-rank timings (each list has one entry per rank):
+    every rank did the same work, the time is the slowest rank's."""
+    t_gemv = max(per_rank_gemv_s)
+    t_build = max(per_rank_build_s)
+    t_step = max(per_rank_step_s)
+    return {
+        "gemv_gbs": world * GEMV_BYTES / t_gemv / 1e9,
+        "build_gweights_s": world * N_W / t_build / 1e9,
+        "ms_per_step": t_step * 1e3,
+    }
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def cpu_oracle_times(budget_s=20.0):
+    """The oracle as it stands, single-threaded on this host: GEMV over the whole
+    layer (repeated while within the budget) and the build of the whole layer."""
+    import oracle
+    cfg = gen.layer(1)
+    o = oracle.build_sketch(cfg["W"], cfg["importance"], cfg["seed"])
+    t0 = time.perf_counter()
+    oracle.build_sketch(cfg["W"], cfg["importance"], cfg["seed"])
+    t_build = time.perf_counter() - t0
+    reps, t_gemv = 0, 0.0
+    while reps == 0 or (t_gemv < budget_s * 0.5 and reps < 20):
+        t0 = time.perf_counter()
+        oracle.gemv_f64(o["codes"], o["scales"], M, K, cfg["x"], cfg["seed"])
+        t_gemv += time.perf_counter() - t0
+        reps += 1
+    return {"gemv_s": t_gemv / reps, "build_s": t_build, "reps": reps}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    cfg = gen.layer(1)
+    o = oracle.build_sketch(cfg["W"], cfg["importance"], cfg["seed"])
+    # calibrate: time one 64-row block, size each step to fit the run in about a minute
+    t0 = time.perf_counter()
+    oracle.gemv_f64(o["codes"], o["scales"], M, K, cfg["x"], cfg["seed"], rows=np.arange(64))
+    t_row = (time.perf_counter() - t0) / 64
+    total = args.steps + args.warmup
+    rows_per_step = int(max(1, min(M, (60.0 / max(total, 1)) / max(t_row, 1e-9))))
+    g = np.random.default_rng(7)
+    for _ in range(args.warmup):
+        oracle.gemv_f64(o["codes"], o["scales"], M, K, cfg["x"], cfg["seed"],
+                        rows=g.integers(0, M, rows_per_step))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gemv_f64(o["codes"], o["scales"], M, K, cfg["x"], cfg["seed"],
+                        rows=g.integers(0, M, rows_per_step))
+    t = (time.perf_counter() - t0) / max(args.steps, 1)
+    # scale the sampled rows to one full-layer call
+    t_full = t * M / rows_per_step
+    value = GEMV_BYTES / t_full / 1e9
+    sample = "%d random rows of the 4096x4096 layer per step (of %d), scaled to a full call" % (rows_per_step, M)
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(t * 1e3, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "batch": GEMV_BATCH},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_usk(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import sub_bit_weight_usk_b200 as usk
+
+    dev = torch.device("cuda", local)
+    cfg = gen.layer(GEMM_BATCH)
+    W = torch.from_numpy(cfg["W"].view(np.int16)).to(dev).view(torch.bfloat16)
+    imp = torch.from_numpy(cfg["importance"]).to(dev)
+    x16 = torch.from_numpy(cfg["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+    x1 = x16[:GEMV_BATCH].contiguous()
+    seed = cfg["seed"]
+    Ws = [W.clone() for _ in range(N_WCOPIES)]
+    sk0 = usk.usk_build(W, imp, seed)
+    sks = [usk.Sketch(M, K, seed, sk0.codes.clone(), sk0.scales.clone()) for _ in range(N_SKETCHES)]
+    y1 = torch.empty((GEMV_BATCH, M), device=dev)
+    y16 = torch.empty((GEMM_BATCH, M), device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+
+    def step(i, ev=None):
+        if ev is not None:
+            ev[0].record()
+        b = sks[i % N_SKETCHES]
+        usk.usk_build(Ws[i % N_WCOPIES], imp, seed, codes=b.codes, scales=b.scales, status=status)
+        if ev is not None:
+            ev[1].record()
+        usk.usk_gemv(sks[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1)
+        if ev is not None:
+            ev[2].record()
+        usk.usk_gemm(sks[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
+        if ev is not None:
+            ev[3].record()
+
+    # warm-up (untimed, eager)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise SystemExit("device status flags %#x during warm-up" % int(status.item()))
+
+    # timed region: exactly K steps, captured as CUDA graphs of GRAPH_STEPS steps (+ a remainder graph)
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+
+    def capture(nsteps, offset):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(nsteps)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for j in range(nsteps):
+                step(offset + j, evs[j])
+        return g, evs
+
+    full, rem = divmod(args.steps, GRAPH_STEPS)
+    g_main, ev_main = capture(min(GRAPH_STEPS, args.steps), args.warmup) if args.steps > 0 else (None, None)
+    g_rem, ev_rem = capture(rem, args.warmup) if (rem and full) else (None, None)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record()
+    if full == 0:
+        g_main.replay()
+    else:
+        for _ in range(full):
+            g_main.replay()
+        if g_rem is not None:
+            g_rem.replay()
+    e_end.record()
+    e_end.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    sampler.stop()
+    t_total = e_start.elapsed_time(e_end) * 1e-3
+    n_main = min(GRAPH_STEPS, args.steps)
+    t_build = sum(ev_main[j][0].elapsed_time(ev_main[j][1]) for j in range(n_main)) * 1e-3 / n_main
+    t_gemv = sum(ev_main[j][1].elapsed_time(ev_main[j][2]) for j in range(n_main)) * 1e-3 / n_main
+    t_gemm = sum(ev_main[j][2].elapsed_time(ev_main[j][3]) for j in range(n_main)) * 1e-3 / n_main
+    t_step = t_total / max(args.steps, 1)
+    if int(status.item()) != 0:
+        raise SystemExit("device status flags %#x in the timed region" % int(status.item()))
+
+    # end to end through the public API with host buffers: x in from pinned host memory, y back out
+    xh = x1.cpu().pin_memory()
+    yh = torch.empty((GEMV_BATCH, M), dtype=torch.float32).pin_memory()
+    n_e2e = max(50, min(2000, args.steps))
+    for i in range(5):
+        usk.usk_gemv(sks[i], xh.to(dev, non_blocking=True), y=y1)
+        yh.copy_(y1, non_blocking=True)
+        torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for i in range(n_e2e):
+        xd = xh.to(dev, non_blocking=True)
+        usk.usk_gemv(sks[i % N_SKETCHES], xd, y=y1)
+        yh.copy_(y1, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+    t_e2e = (time.perf_counter() - t0) / n_e2e
+
+    # max over ranks
+    vals = torch.tensor([t_gemv, t_build, t_gemm, t_step, t_total, t_e2e], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    t_gemv, t_build, t_gemm, t_step, t_total, t_e2e = [float(v) for v in vals.tolist()]
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        c = cpu_oracle_times()
+        cpu = {"value": round(GEMV_BYTES / c["gemv_s"] / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": "whole 4096x4096 layer, batch 1, float64 oracle GEMV (%d pass(es)); oracle build of the "
+                         "layer %.2f s = %.4f Gweights/s" % (c["reps"], c["build_s"], N_W / c["build_s"] / 1e9)}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    peaks = load_peaks()
+    agg = aggregate(world, [t_gemv], [t_build], [t_step])
+    rl = rooflines(peaks, t_build, t_gemv, t_gemm, load_traffic())
+    clocks = sampler.summary()
+    line = {
+        "metric": METRIC,
+        "value": round(agg["gemv_gbs"], 3),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t_step * 1e3, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "gemv_batch": GEMV_BATCH, "gemm_batch": GEMM_BATCH,
+                   "l2": "inputs larger than L2: builds cycle over %d weight copies (%d MiB), decodes over %d "
+                         "sketch copies (%d MiB)" % (N_WCOPIES, N_WCOPIES * 32, N_SKETCHES, N_SKETCHES),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "usk_build_gweights_per_s": round(agg["build_gweights_s"], 3),
+        "kernel_us": {"usk_build": round(t_build * 1e6, 3), "usk_gemv": round(t_gemv * 1e6, 3),
+                      "usk_gemm": round(t_gemm * 1e6, 3)},
+        "roofline": rl["usk_gemv"],
+        "rooflines": rl,
+        "clocks": clocks,
+        "e2e": {"value": round(world * GEMV_BYTES / t_e2e / 1e9, 4), "unit": "GB/s",
+                "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 4),
+                "call": "usk_gemv via the Python binding, x from pinned host memory, y read back, per step"},
+        "gpu_launches": 3 * args.steps,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="usk", choices=["usk", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_usk(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
