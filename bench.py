@@ -178,6 +178,18 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of a list of floats over all ranks (identity for one
+    process).  The only collective of the benchmark; NCCL on the GPUs, gloo in
+    the CPU tests."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 def aggregate(world, per_rank_gemv_s, per_rank_build_s, per_rank_step_s):
     """Whole-job numbers from per-rank timings (each list has one entry per rank):
     every rank did the same work, the time is the slowest rank's."""
@@ -282,42 +294,47 @@ def run_usk(args):
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     torch.cuda.synchronize()
 
-    def step(i, ev=None):
-        if ev is not None:
-            ev[0].record()
+    def build(i):
         b = sks[i % N_SKETCHES]
         usk.usk_build(Ws[i % N_WCOPIES], imp, seed, codes=b.codes, scales=b.scales, status=status)
-        if ev is not None:
-            ev[1].record()
-        usk.usk_gemv(sks[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1)
-        if ev is not None:
-            ev[2].record()
-        usk.usk_gemm(sks[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
-        if ev is not None:
-            ev[3].record()
 
-    # warm-up (untimed, eager)
+    def gemv(i):
+        usk.usk_gemv(sks[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1)
+
+    def gemm(i):
+        usk.usk_gemm(sks[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
+
+    kernels = (build, gemv, gemm)
+
+    # warm-up (untimed, eager): W full steps
     for i in range(args.warmup):
-        step(i)
+        for k in kernels:
+            k(i)
     torch.cuda.synchronize()
     if int(status.item()) != 0:
         raise SystemExit("device status flags %#x during warm-up" % int(status.item()))
 
-    # timed region: exactly K steps, captured as CUDA graphs of GRAPH_STEPS steps (+ a remainder graph)
+    # Timed region: exactly K steps.  The K steps run phase by phase (K builds,
+    # then K GEMVs, then K GEMMs; the same work as K build+gemv+gemm passes) so
+    # that each kernel's average launch duration is the CUDA-event time of its
+    # phase / K, with no timing nodes between kernels.  Each phase replays a CUDA
+    # graph of GRAPH_STEPS launches (+ one graph for the remainder).
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
 
-    def capture(nsteps, offset):
-        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)] for _ in range(nsteps)]
+    def capture(fn, n, offset):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
-            for j in range(nsteps):
-                step(offset + j, evs[j])
-        return g, evs
+            for j in range(n):
+                fn(offset + j)
+        return g
 
     full, rem = divmod(args.steps, GRAPH_STEPS)
-    g_main, ev_main = capture(min(GRAPH_STEPS, args.steps), args.warmup) if args.steps > 0 else (None, None)
-    g_rem, ev_rem = capture(rem, args.warmup) if (rem and full) else (None, None)
+    graphs = []
+    for fn in kernels:
+        main = capture(fn, GRAPH_STEPS, args.warmup) if full else None
+        tail = capture(fn, rem, args.warmup) if rem else None
+        graphs.append((main, tail))
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
@@ -326,28 +343,25 @@ def run_usk(args):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e_start = torch.cuda.Event(enable_timing=True)
-    e_end = torch.cuda.Event(enable_timing=True)
-    e_start.record()
-    if full == 0:
-        g_main.replay()
-    else:
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(kernels) + 1)]
+    ev[0].record()
+    for k, (main, tail) in enumerate(graphs):
         for _ in range(full):
-            g_main.replay()
-        if g_rem is not None:
-            g_rem.replay()
-    e_end.record()
-    e_end.synchronize()
+            main.replay()
+        if tail is not None:
+            tail.replay()
+        ev[k + 1].record()
+    ev[-1].synchronize()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     sampler.stop()
-    t_total = e_start.elapsed_time(e_end) * 1e-3
-    n_main = min(GRAPH_STEPS, args.steps)
-    t_build = sum(ev_main[j][0].elapsed_time(ev_main[j][1]) for j in range(n_main)) * 1e-3 / n_main
-    t_gemv = sum(ev_main[j][1].elapsed_time(ev_main[j][2]) for j in range(n_main)) * 1e-3 / n_main
-    t_gemm = sum(ev_main[j][2].elapsed_time(ev_main[j][3]) for j in range(n_main)) * 1e-3 / n_main
-    t_step = t_total / max(args.steps, 1)
+    n = max(args.steps, 1)
+    t_build = ev[0].elapsed_time(ev[1]) * 1e-3 / n
+    t_gemv = ev[1].elapsed_time(ev[2]) * 1e-3 / n
+    t_gemm = ev[2].elapsed_time(ev[3]) * 1e-3 / n
+    t_total = ev[0].elapsed_time(ev[3]) * 1e-3
+    t_step = t_total / n
     if int(status.item()) != 0:
         raise SystemExit("device status flags %#x in the timed region" % int(status.item()))
 
@@ -368,10 +382,8 @@ def run_usk(args):
     t_e2e = (time.perf_counter() - t0) / n_e2e
 
     # max over ranks
-    vals = torch.tensor([t_gemv, t_build, t_gemm, t_step, t_total, t_e2e], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    t_gemv, t_build, t_gemm, t_step, t_total, t_e2e = [float(v) for v in vals.tolist()]
+    t_gemv, t_build, t_gemm, t_step, t_total, t_e2e = max_over_ranks(
+        [t_gemv, t_build, t_gemm, t_step, t_total, t_e2e], device=dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -402,6 +414,8 @@ def run_usk(args):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "M": M, "K": K, "gemv_batch": GEMV_BATCH, "gemm_batch": GEMM_BATCH,
+                   "timing": "K steps run phase by phase (K builds, K GEMVs, K GEMMs) as CUDA graphs; "
+                             "kernel time = phase event time / K",
                    "l2": "inputs larger than L2: builds cycle over %d weight copies (%d MiB), decodes over %d "
                          "sketch copies (%d MiB)" % (N_WCOPIES, N_WCOPIES * 32, N_SKETCHES, N_SKETCHES),
                    "parallelism": "replicas" if world > 1 else "single"},

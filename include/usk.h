@@ -137,11 +137,24 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
  * fly: every weight is rehashed and its bucket gathered; W_hat is never stored).
  *   x  [batch, K] row-major, fp32 or bf16 per xdtype, 16-byte aligned.
  *   y  [batch, M] fp32 output (y[t*M + i] = sum_j w_hat[i][j] x[t][j]).
- * Products of bf16 x are exact and accumulate in fp32; fp32 x is split into
- * two bf16 terms (|error| <= 2^-16 |x| per element).  batch == 0 or M == 0 is
- * a no-op; K == 0 writes y = 0.  Results do not depend on the launch. */
+ * bf16 x at batch <= 4: integer tensor path, exact sum of code * x (x split
+ * into byte digit planes per block; elements outside 2^22 of the block's
+ * largest are added by an exact correction), one rounding to fp32 at the end.
+ * Other batches: bf16 tensor path, exact products, fp32 accumulation; fp32 x
+ * is split into two bf16 terms (|error| <= 2^-16 |x| per element).
+ * batch == 0 or M == 0 is a no-op; K == 0 writes y = 0.  Deterministic for a
+ * given shape (the summation order is fixed). */
 USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
                     float* y, uint32_t* d_status, void* stream);
+
+/* usk_gemv with launch flags.  USK_GEMV_PDL: launch as a programmatic
+ * dependent of the previous kernel in the stream; the kernel prefetches the
+ * sketch codes before waiting for that kernel, so the caller guarantees that
+ * no kernel still running in the stream writes this sketch (x and y may be
+ * produced / consumed by neighbouring kernels).  Other bits: USK_ERR_PARAMS. */
+#define USK_GEMV_PDL 1u
+USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
+                               float* y, uint32_t flags, uint32_t* d_status, void* stream);
 
 /* y = W_hat x for batch 16..256 (multiple of 16) on the tcgen05 tensor cores:
  * decoded bf16 tiles of W_hat are written to shared memory and multiplied with
@@ -158,6 +171,18 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
  * bit-identical for every geometry; only the split of the work changes.
  * Process-wide; not thread-safe with concurrent calls. */
 USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block);
+
+/* Test hook: choose the usk_gemv path (0 = automatic, 1 = bf16 tensor path,
+ * 2 = integer path where eligible).  Both give results within the products'
+ * tolerance; process-wide. */
+USK_API void usk_debug_set_gemv_path(int path);
+
+/* Test hook for the failure path (host-made; no device fault): kernel = 1 makes
+ * usk_build, 2 usk_gemm, 3 usk_gemv (integer path) skip one bulk copy or one
+ * MMA commit in thread block (0, 0), so that block's bounded wait gives up
+ * after about 1 s and sets USK_FLAG_TIMEOUT; the kernel still completes and the
+ * context stays usable.  0 switches it off.  Process-wide. */
+USK_API void usk_debug_inject_timeout(int kernel);
 
 /* Static description of a status value. */
 USK_API const char* usk_status_str(usk_status status);

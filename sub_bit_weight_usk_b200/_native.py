@@ -53,8 +53,9 @@ class UskSketchC(ctypes.Structure):
 
 _lib = None
 
-EXPORTED = ["usk_sizes", "usk_build", "usk_gemv", "usk_gemm", "usk_status_str", "usk_format_version",
-            "usk_debug_set_geometry"]
+EXPORTED = ["usk_sizes", "usk_build", "usk_gemv", "usk_gemv_ex", "usk_gemm", "usk_status_str",
+            "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_inject_timeout"]
+GEMV_PDL = 1
 
 
 def load_library(path: str = LIB_PATH):
@@ -73,6 +74,8 @@ def load_library(path: str = LIB_PATH):
     lib.usk_build.restype = ctypes.c_int
     lib.usk_gemv.argtypes = [ctypes.POINTER(UskSketchC), vp, ctypes.c_int, i64, vp, vp, vp]
     lib.usk_gemv.restype = ctypes.c_int
+    lib.usk_gemv_ex.argtypes = [ctypes.POINTER(UskSketchC), vp, ctypes.c_int, i64, vp, ctypes.c_uint32, vp, vp]
+    lib.usk_gemv_ex.restype = ctypes.c_int
     lib.usk_gemm.argtypes = [ctypes.POINTER(UskSketchC), vp, i64, vp, vp, ctypes.c_size_t, vp, vp]
     lib.usk_gemm.restype = ctypes.c_int
     lib.usk_status_str.argtypes = [ctypes.c_int]
@@ -81,6 +84,10 @@ def load_library(path: str = LIB_PATH):
     lib.usk_format_version.restype = ctypes.c_uint32
     lib.usk_debug_set_geometry.argtypes = [ctypes.c_int, ctypes.c_int]
     lib.usk_debug_set_geometry.restype = None
+    lib.usk_debug_set_gemv_path.argtypes = [ctypes.c_int]
+    lib.usk_debug_set_gemv_path.restype = None
+    lib.usk_debug_inject_timeout.argtypes = [ctypes.c_int]
+    lib.usk_debug_inject_timeout.restype = None
     _lib = lib
     return lib
 
@@ -169,8 +176,12 @@ def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int
 
 
 def usk_gemv(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
-             status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y [batch, M] fp32 = W_hat x^T for x [batch, K] (bf16 or fp32), batch 1..15."""
+             status: torch.Tensor | None = None, stream=None, pdl: bool = False) -> torch.Tensor:
+    """y [batch, M] fp32 = W_hat x^T for x [batch, K] (bf16 or fp32), batch 1..15.
+
+    pdl=True launches as a programmatic dependent of the previous kernel in the
+    stream (usk_gemv_ex with USK_GEMV_PDL): the sketch codes are prefetched
+    before that kernel finishes, so no kernel still running may write them."""
     _need_cuda(x, y, status)
     if x.dim() == 1:
         x = x[None, :]
@@ -180,8 +191,8 @@ def usk_gemv(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
     if y is None:
         y = torch.empty((batch, sketch.M), dtype=torch.float32, device=x.device)
     sk = sketch.as_c()
-    st = load_library().usk_gemv(ctypes.byref(sk), _ptr(x), _dtype_code(x), batch, _ptr(y), _ptr(status),
-                                 _stream(stream))
+    st = load_library().usk_gemv_ex(ctypes.byref(sk), _ptr(x), _dtype_code(x), batch, _ptr(y),
+                                    GEMV_PDL if pdl else 0, _ptr(status), _stream(stream))
     _check(st, "usk_gemv")
     return y
 
@@ -204,3 +215,14 @@ def usk_gemm(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
 
 def usk_debug_set_geometry(build_cluster: int = 0, gemv_tiles_per_block: int = 0) -> None:
     load_library().usk_debug_set_geometry(int(build_cluster), int(gemv_tiles_per_block))
+
+
+def usk_debug_set_gemv_path(path: int = 0) -> None:
+    """0 automatic, 1 bf16 tensor path, 2 integer path (where eligible)."""
+    load_library().usk_debug_set_gemv_path(int(path))
+
+
+def usk_debug_inject_timeout(kernel: int = 0) -> None:
+    """Test hook: 1 build, 2 gemm, 3 gemv (integer path) skip one copy/commit in
+    block (0, 0) so its bounded wait gives up (USK_FLAG_TIMEOUT); 0 = off."""
+    load_library().usk_debug_inject_timeout(int(kernel))

@@ -9,11 +9,12 @@
 namespace usk {
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override);
+                         cudaStream_t stream, int cluster_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
-                        const void* x, bool xf32, int batch, float* y, cudaStream_t stream, int tpc_override);
+                        const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
+                        cudaStream_t stream, int tpc_override, int inject);
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
-                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream);
+                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject);
 }  // namespace usk
 
 namespace {
@@ -45,6 +46,8 @@ usk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? USK_OK : USK_ERR
 // result does not depend on the geometry).  0 = library default.
 int g_build_cluster = 0;
 int g_gemv_tiles_per_block = 0;
+int g_gemv_path = 0;
+int g_inject = 0;  // 1 build, 2 gemm, 3 gemv (integer path): skip one copy/commit in block (0, 0)
 
 }  // namespace
 
@@ -99,18 +102,18 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (ldw % (wdtype == USK_BF16 ? 8 : 4) != 0) return USK_ERR_ALIGN;
   if (importance && !aligned16(importance)) return USK_ERR_ALIGN;
   cudaError_t e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes,
-                                    scales, d_status, s, g_build_cluster);
+                                    scales, d_status, s, g_build_cluster, g_inject == 1);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
 
-USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch, float* y,
-                    uint32_t* d_status, void* stream) {
-  (void)d_status;
+USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch, float* y,
+                               uint32_t flags, uint32_t* d_status, void* stream) {
   usk_status st = check_sketch(sketch);
   if (st != USK_OK) return st;
   if (xdtype != USK_F32 && xdtype != USK_BF16) return USK_ERR_DTYPE;
   if (batch < 0 || batch > USK_GEMV_MAX_BATCH) return USK_ERR_BATCH;
+  if ((flags & ~static_cast<uint32_t>(USK_GEMV_PDL)) != 0) return USK_ERR_PARAMS;
   if (batch == 0 || sketch->M == 0) return USK_OK;
   if (!y) return USK_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -120,9 +123,15 @@ USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype x
   if (!aligned16(x)) return USK_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(y) & 3u) != 0) return USK_ERR_ALIGN;
   cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
-                                   xdtype == USK_F32, static_cast<int>(batch), y, s, g_gemv_tiles_per_block);
+                                   xdtype == USK_F32, static_cast<int>(batch), y, d_status,
+                                   (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_inject == 3);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
+}
+
+USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch, float* y,
+                            uint32_t* d_status, void* stream) {
+  return usk_gemv_ex(sketch, x, xdtype, batch, y, 0u, d_status, stream);
 }
 
 USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y, void* ws,
@@ -140,7 +149,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   if (!x_bf16) return USK_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(y)) return USK_ERR_ALIGN;
   cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
-                                   static_cast<int>(batch), y, d_status, s);
+                                   static_cast<int>(batch), y, d_status, s, g_inject == 2);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -151,5 +160,9 @@ USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block)
   g_build_cluster = build_cluster;
   g_gemv_tiles_per_block = gemv_tiles_per_block;
 }
+
+USK_API void usk_debug_set_gemv_path(int path) { g_gemv_path = path; }
+
+USK_API void usk_debug_inject_timeout(int kernel) { g_inject = kernel; }
 
 }  // extern "C"

@@ -11,9 +11,10 @@
 //    row block form a thread-block cluster, so the row-block scale is an
 //    exchange of per-block maxima through distributed shared memory: no
 //    workspace, one launch.
-//  * Weight tiles (64 x 256) stream from HBM into shared memory with 1-D bulk
-//    copies (the tensor memory accelerator) completing on mbarriers, double
-//    buffered, so the copy of tile i+1 overlaps the selection of tile i.
+//  * Weight tiles (64 x 256) stream from HBM into shared memory with one 2-D
+//    tensor copy each (the tensor memory accelerator, tensor map over W),
+//    completing on mbarriers, double buffered, so the copy of tile i+1
+//    overlaps the selection of tile i.
 //  * Selection uses order-preserving 32-bit keys and shared-memory atomics
 //    (64-bit shared atomics run about four times slower on this part):
 //      - bf16 weights, unit importance: ONE pass.  The packed word
@@ -48,6 +49,7 @@ struct BuildArgs {
   int C;     // thread blocks per row block (cluster size)
   int tpc;   // max tiles per block
   int nbuf;  // weight-tile buffers (1 or 2)
+  int inject;  // test hook: block (0, 0) skips the copy of its first tile
 };
 
 // Shared-memory layout (byte offsets from a 128-byte aligned base).
@@ -70,14 +72,15 @@ __host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int
 }
 
 template <bool BF16, bool HAS_IMP>
-__global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a) {
+__global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
   constexpr bool kSingle = BF16 && !HAS_IMP;
   constexpr uint32_t kRowBytes = kTileCols * (BF16 ? 2 : 4);
   constexpr uint32_t kTileBytes = kRowsPerBlock * kRowBytes;
   constexpr uint32_t kWinBytes = (kSingle || BF16) ? 4096u : 8192u;  // one tile's winner words
-  extern __shared__ __align__(128) uint8_t smraw[];
+  extern __shared__ __align__(128) uint8_t smraw_unaligned[];
   const BuildLayout L = build_layout(BF16, HAS_IMP, a.tpc, a.nbuf);
-  const uint32_t s0 = smem_u32(smraw);
+  const uint32_t s0 = (smem_u32(smraw_unaligned) + 1023u) & ~1023u;  // tensor copies want 128 B; use 1 KiB
+  uint8_t* smraw = smraw_unaligned + (s0 - smem_u32(smraw_unaligned));
   uint32_t* misc = reinterpret_cast<uint32_t*>(smraw + L.misc);
 
   cg::cluster_group cluster = cg::this_cluster();
@@ -103,20 +106,16 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a)
   }
   __syncthreads();
 
-  auto issue = [&](int i) {  // bulk-copy tile i of this block into buffer i % nbuf
+  auto issue = [&](int i) {  // one tensor copy of tile i of this block into buffer i % nbuf
     const int tc = crank + a.C * i;
     const int buf = i % a.nbuf;
     const uint32_t bar = s0 + L.bars + 8 * buf;
-    const uint32_t dst = s0 + L.wbuf + buf * kTileBytes;
     mbar_arrive_expect_tx(bar, kTileBytes);
-    const char* src = static_cast<const char*>(a.W) +
-                      (static_cast<int64_t>(rb) * kRowsPerBlock * a.ldw + static_cast<int64_t>(tc) * kTileCols) *
-                          (BF16 ? 2 : 4);
-    const int64_t stride = a.ldw * (BF16 ? 2 : 4);
-    for (int r = 0; r < kRowsPerBlock; ++r) bulk_g2s(dst + r * kRowBytes, src + r * stride, kRowBytes, bar);
+    tma_load_2d(s0 + L.wbuf + buf * kTileBytes, &wmap, tc * kTileCols, rb * kRowsPerBlock, bar);
   };
   if (tid == 0)
-    for (int i = 0; i < a.nbuf && i < nt; ++i) issue(i);
+    for (int i = 0; i < a.nbuf && i < nt; ++i)
+      if (!(a.inject && i == 0 && crank == 0 && rb == 0)) issue(i);
 
   uint32_t flags = 0;
   uint32_t vmax = 0;  // max |v| bits over the winners this thread converts
@@ -305,7 +304,7 @@ static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override
     p.C = C < T ? C : T;
     p.tpc = (T + p.C - 1) / p.C;
     p.nbuf = nbuf;
-    p.smem = build_layout(bf16, has_imp, p.tpc, nbuf).total + 128;  // + alignment slack
+    p.smem = build_layout(bf16, has_imp, p.tpc, nbuf).total + 1024;  // + alignment slack
     return p;
   };
   if (cluster_override > 0) {
@@ -322,6 +321,19 @@ static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override
 template <bool BF16, bool HAS_IMP>
 static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, int cluster_override) {
   const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override);
+  // tensor map over W [M, K] (row stride ldw), one 64 x 256 box per tile
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  CUtensorMap wmap;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(RB * kRowsPerBlock)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(a.ldw) * (BF16 ? 2u : 4u)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileCols), static_cast<cuuint32_t>(kRowsPerBlock)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (encode(&wmap, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+             const_cast<void*>(a.W), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   a.C = p.C;
   a.tpc = p.tpc;
   a.nbuf = p.nbuf;
@@ -344,13 +356,14 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  return cudaLaunchKernelEx(&cfg, kern, a, wmap);
 }
 
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override) {
+                         cudaStream_t stream, int cluster_override, int inject) {
   BuildArgs a;
+  a.inject = inject;
   a.W = W; a.ldw = ldw; a.K = K; a.imp = imp; a.seed = seed;
   a.codes = codes; a.scales = scales; a.status = status;
   a.T = static_cast<int>(K / kTileCols);

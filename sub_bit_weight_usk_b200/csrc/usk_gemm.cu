@@ -49,6 +49,7 @@ struct GemmArgs {
   int N;       // batch (multiple of 16, <= 256)
   int splits;  // blocks along K per row tile (cluster size)
   uint32_t tmem_cols;
+  int inject;  // test hook: block (0, 0) skips the commit of its first chunk
 };
 
 __host__ __device__ constexpr size_t gemm_stage_a_bytes() { return kBM * kBK * 2; }  // 16 KiB
@@ -155,6 +156,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
   uint8_t* misc_g = base_g + (bar_s - base_s) + 64;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(misc_g);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(misc_g + 4);
+  volatile int* last_commit = reinterpret_cast<volatile int*>(misc_g + 8);  // last chunk whose MMAs were committed
 
   // K range of this block (whole tiles)
   const int t_begin = static_cast<int>((static_cast<int64_t>(a.T) * ks) / a.splits);
@@ -164,6 +166,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(bar_s + 8 * s, 1);
     *abort_flag = 0u;
+    *last_commit = -1;
     mbar_fence_init();
   }
   __syncwarp();
@@ -265,17 +268,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
         mma_bf16(tmem_d, sw128_desc(a_stage + 32 * kk), sw128_desc(bst + 32 * kk), idesc,
                  (c > 0 || kk > 0) ? 1u : 0u);
       }
-      mma_commit(bar_s + 8 * (c % kStages));
+      const bool skip = a.inject && c == 0 && ks == 0 && mt == 0;
+      if (!skip) {
+        mma_commit(bar_s + 8 * (c % kStages));
+        *last_commit = c;
+      }
     }
   }
   cp_async_wait<0>();
   __syncthreads();
   aborted = aborted || (*abort_flag != 0u);
 
-  // wait for the last chunk's MMAs
-  if (nk > 0 && !aborted) {
-    const int last = nk - 1;
-    if (!mbar_wait(bar_s + 8 * (last % kStages), (last / kStages) & 1)) aborted = true;
+  // Wait for the MMAs: all of them, or after a wait that gave up, the last
+  // committed chunk (a commit tracks every earlier MMA of the issuing thread),
+  // again bounded, so that no MMA is in flight when tensor memory is freed.
+  {
+    const int last = aborted ? *last_commit : nk - 1;
+    if (last >= 0 && !mbar_wait(bar_s + 8 * (last % kStages), (last / kStages) & 1)) aborted = true;
   }
   tc_fence_after();
   if (aborted) report(a.status, USK_FLAG_TIMEOUT);
@@ -348,8 +357,9 @@ static uint32_t tmem_columns(int N) {
 }
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
-                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream) {
+                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject) {
   GemmArgs a;
+  a.inject = inject;
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status;
   a.T = static_cast<int>(K / kTileCols);

@@ -284,9 +284,19 @@ static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t RB, cudaStream_t str
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+cudaError_t launch_gemv_i8(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                           const uint16_t* x, int batch, float* y, uint32_t* status, int T, int C, int tpc, bool pdl,
+                           cudaStream_t stream, int inject);
+
+// path: 0 = automatic, 1 = bf16 tensor path, 2 = integer path (bf16 x, batch <= 4 only)
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
-                        const void* x, bool xf32, int batch, float* y, cudaStream_t stream, int tpc_override) {
+                        const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
+                        cudaStream_t stream, int tpc_override, int inject) {
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
+  const bool i8_ok = !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
+  if (i8_ok && path != 1)
+    return launch_gemv_i8(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, geo.T,
+                          geo.C, geo.tpc, pdl, stream, inject);
   GemvArgs a;
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed;

@@ -1,0 +1,359 @@
+// usk_gemv_i8.cu -- y = W_hat x for bf16 x at batch 1..4 on the integer tensor
+// path: int8 codes straight from shared memory, x as four signed-byte digit
+// planes.
+//
+// "UltraSketchLLM" explainer, Metodologia §4 (decompression W_hat = S . P^T,
+// fused into the product here).  The codes are integers in [-127, 127]; the
+// product sum_j code_j x_j is formed exactly in integer arithmetic:
+//  * per thread block, each batch row of its x slice is written as
+//    v_j * 2^(E - 156) with E the largest (biased) exponent in the slice and v_j
+//    an integer of at most 30 bits (exact for every bf16 element within 2^22
+//    of the largest; any other element, and any Inf/NaN, is left out of the
+//    planes and added back by an exact scalar correction);
+//  * v_j is split into balanced base-256 digits d_p in [-128, 127]
+//    ((v + 0x80808080) ^ 0x80808080 gives their bytes), plane p = digit p;
+//  * mma.sync m16n8k32 s8 x s8 -> s32 multiplies the gathered codes (A
+//    fragment: one 8-byte load per row and octet, conflict-free because
+//    class = (octet + row) mod 32) with the digit planes (B fragment: one
+//    8-byte load), accumulating each plane in int32 (no overflow: |sum| <
+//    K_block * 127 * 128);
+//  * the four plane sums are recombined in float64 (exact) and scaled, the
+//    blocks of a row block add their float64 partials through distributed
+//    shared memory in rank order, and y = float(sum * scale).
+// Shared-memory traffic is one byte per weight (the bucket code), half of the
+// bf16 path's.
+#include <cooperative_groups.h>
+
+#include "usk_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace usk {
+
+struct GemvI8Args {
+  const int8_t* codes;
+  const uint16_t* scales;
+  const uint16_t* x;  // bf16 [batch, K]
+  float* y;
+  int64_t M, K;
+  uint64_t seed;
+  uint32_t* status;
+  int T, C, tpc, batch;
+  int pdl;     // launched as a programmatic dependent: wait before reading x
+  int inject;  // test hook: block (0, 0) skips its code copy
+};
+
+constexpr int kI8Threads = 256;
+constexpr int kI8MaxChunks = 1024;  // batch * tiles per block * 32 must not exceed this
+
+struct GemvI8Layout {
+  uint32_t codes, keys, xs, pitch, mask, emax, bar, part, cta, total;
+};
+
+__host__ __device__ inline GemvI8Layout gemv_i8_layout(int tpc, int batch) {
+  GemvI8Layout L;
+  L.codes = 0;                                                 // int8 [tpc][1024]
+  L.keys = static_cast<uint32_t>(tpc) * 1024u;                 // uint2 [tpc]
+  L.xs = (L.keys + static_cast<uint32_t>(tpc) * 8u + 15u) & ~15u;
+  L.pitch = static_cast<uint32_t>(tpc) * 256u + 8u;            // int8 plane row (+8: conflict-free)
+  L.mask = (L.xs + 4u * batch * L.pitch + 15u) & ~15u;         // u32 [batch][tpc * 8] residual bits
+  L.emax = L.mask + static_cast<uint32_t>(batch) * tpc * 32u;  // u32 [4] max exponent, [4] any-residual
+  L.bar = (L.emax + 32u + 7u) & ~7u;                           // mbarrier
+  L.part = (L.bar + 8u + 15u) & ~15u;                          // f64 [8 warps][64][batch]
+  L.cta = L.part + 8u * 64u * batch * 8u;                      // f64 [batch][64]
+  L.total = L.cta + static_cast<uint32_t>(batch) * 64u * 8u;
+  return L;
+}
+
+__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                           uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// bf16 bits -> (effective biased exponent, significand as an integer), subnormals with exponent 1
+__device__ __forceinline__ void bf16_parts(uint32_t b, int& e_eff, int& mant) {
+  const int e = static_cast<int>((b >> 7) & 0xFFu);
+  const int m = static_cast<int>(b & 0x7Fu);
+  e_eff = e == 0 ? 1 : e;
+  mant = e == 0 ? m : (128 + m);
+}
+
+template <int B>
+__global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a) {
+  constexpr int NB = (4 * B + 7) / 8;  // n tiles of 8 planes
+  constexpr int kXR = kI8MaxChunks / kI8Threads;  // x chunks (8 elements) per thread
+  extern __shared__ __align__(16) uint8_t sm[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int rb = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = crank * a.tpc;
+  const int nt = min(a.tpc, a.T - t0);
+  const GemvI8Layout L = gemv_i8_layout(a.tpc, B);
+  const uint32_t s0 = smem_u32(sm);
+  uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
+  uint32_t* mask = reinterpret_cast<uint32_t*>(sm + L.mask);
+  uint32_t* emax = reinterpret_cast<uint32_t*>(sm + L.emax);  // [0..3] exponent, [4] any residual
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // ---- stage: codes by one bulk copy (weights: independent of earlier kernels)
+  if (tid == 0) {
+    mbar_init(s0 + L.bar, 1);
+    mbar_fence_init();
+  }
+  if (tid < 8) emax[tid] = 0u;
+  for (int q = tid; q < B * a.tpc * 8; q += kI8Threads) mask[q] = 0u;
+  __syncthreads();
+  if (tid == 0 && !(a.inject && crank == 0 && rb == 0)) {
+    mbar_arrive_expect_tx(s0 + L.bar, static_cast<uint32_t>(nt) * 1024u);
+    bulk_g2s(s0 + L.codes, a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0),
+             static_cast<uint32_t>(nt) * 1024u, s0 + L.bar);
+  }
+  if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
+  if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // ---- stage x: pass 1, largest exponent per batch row
+  const int cpr = nt * 32;  // 8-element chunks per batch row
+  const int nchunks = B * cpr;
+  uint4 xv[kXR];
+#pragma unroll
+  for (int u = 0; u < kXR; ++u) {
+    const int c = tid + u * kI8Threads;
+    xv[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (c < nchunks) {
+      const int bi = c / cpr, cc = c % cpr;
+      xv[u] = ldg_nc128(a.x + static_cast<int64_t>(bi) * a.K + static_cast<int64_t>(t0) * kTileCols + 8 * cc);
+    }
+  }
+  {
+    int em[B];
+#pragma unroll
+    for (int bi = 0; bi < B; ++bi) em[bi] = 0;
+#pragma unroll
+    for (int u = 0; u < kXR; ++u) {
+      const int c = tid + u * kI8Threads;
+      if (c < nchunks) {
+        const int bi = c / cpr;
+        const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+        int m = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t b = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+          int ee, mm;
+          bf16_parts(b, ee, mm);
+          if (mm != 0 && ((b >> 7) & 0xFFu) != 0xFFu) m = max(m, ee);
+        }
+#pragma unroll
+        for (int q = 0; q < B; ++q)
+          if (q == bi) em[q] = max(em[q], m);
+      }
+    }
+#pragma unroll
+    for (int bi = 0; bi < B; ++bi) {
+      const int m = __reduce_max_sync(0xFFFFFFFFu, em[bi]);
+      if (lane == 0 && m > 0) atomicMax(&emax[bi], static_cast<uint32_t>(m));
+    }
+  }
+  __syncthreads();
+
+  // ---- stage x: pass 2, digit planes and the residual bits
+#pragma unroll
+  for (int u = 0; u < kXR; ++u) {
+    const int c = tid + u * kI8Threads;
+    if (c < nchunks) {
+      const int bi = c / cpr, cc = c % cpr;
+      const int E = static_cast<int>(emax[bi]);
+      const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+      uint32_t dw[8];
+      uint32_t rbits = 0u;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t b = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+        int ee, mm;
+        bf16_parts(b, ee, mm);
+        const int sh = ee - E + 22;
+        int v = 0;
+        if (mm != 0) {
+          if (((b >> 7) & 0xFFu) == 0xFFu || sh < 0) rbits |= 1u << e;  // handled by the exact correction
+          else v = mm << sh;
+        }
+        if (b & 0x8000u) v = -v;
+        dw[e] = (static_cast<uint32_t>(v) + 0x80808080u) ^ 0x80808080u;  // balanced base-256 digits
+      }
+      // 4x4 byte transposes: plane p gets byte p of every column's digit word
+      uint32_t pl[4][2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t t_0 = __byte_perm(dw[4 * h], dw[4 * h + 1], 0x5140);
+        const uint32_t t_1 = __byte_perm(dw[4 * h], dw[4 * h + 1], 0x7362);
+        const uint32_t t_2 = __byte_perm(dw[4 * h + 2], dw[4 * h + 3], 0x5140);
+        const uint32_t t_3 = __byte_perm(dw[4 * h + 2], dw[4 * h + 3], 0x7362);
+        pl[0][h] = __byte_perm(t_0, t_2, 0x5410);
+        pl[1][h] = __byte_perm(t_0, t_2, 0x7632);
+        pl[2][h] = __byte_perm(t_1, t_3, 0x5410);
+        pl[3][h] = __byte_perm(t_1, t_3, 0x7632);
+      }
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const uint32_t dst = s0 + L.xs + (4 * bi + p) * L.pitch + 8 * cc;
+        asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(dst), "r"(pl[p][0]), "r"(pl[p][1]) : "memory");
+      }
+      if (rbits) {
+        atomicOr(&mask[bi * a.tpc * 8 + (cc >> 2)], rbits << (8 * (cc & 3)));
+        emax[4] = 1u;
+      }
+    }
+  }
+  uint32_t flags = 0;
+  if (!mbar_wait(s0 + L.bar, 0)) flags |= USK_FLAG_TIMEOUT;
+  __syncthreads();
+
+  // ---- main loop: warp = column phase, lane (g, t) gathers octet o of rows g, g + 8
+  const int g = lane >> 2, t = lane & 3;
+  const int o = (warp & 3) + 16 * (warp >> 2) + 4 * t;
+  const uint32_t c0 = static_cast<uint32_t>(o + g) & 31u;
+  uint32_t cls8[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) cls8[k] = ((c0 + 8u * k) & 31u) * 8u;
+  int d[4][NB][4];
+#pragma unroll
+  for (int mb = 0; mb < 4; ++mb)
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[mb][nb][e] = 0;
+
+  for (int tt = 0; tt < nt; ++tt) {
+    const uint2 hk = keytab[tt];
+    uint2 bq[NB];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      const int n = nb * 8 + g;
+      bq[nb] = make_uint2(0u, 0u);
+      if (n < 4 * B) bq[nb] = lds64(s0 + L.xs + n * L.pitch + tt * 256 + 8 * o);
+    }
+    const uint32_t tile_s = s0 + L.codes + tt * 1024u;
+    const uint32_t h = hk.x * (32u * g + o) + hk.y;
+    const uint32_t d512 = hk.x * 512u, d256 = hk.x * 256u;
+#pragma unroll
+    for (int mb = 0; mb < 4; ++mb) {
+      const uint32_t h0 = h + mb * d512;
+      const uint32_t h1 = h0 + d256;
+      const uint2 q0 = lds64(tile_s + (h0 >> 30) * 256u + cls8[(2 * mb) & 3]);
+      const uint2 q1 = lds64(tile_s + (h1 >> 30) * 256u + cls8[(2 * mb + 1) & 3]);
+#pragma unroll
+      for (int nb = 0; nb < NB; ++nb) imma_16832(d[mb][nb], q0.x, q1.x, q0.y, q1.y, bq[nb].x, bq[nb].y);
+    }
+  }
+
+  // ---- recombine the planes (exact in float64): lanes with even t hold planes 0,1
+  // of batch row nb*2 + t/2, the next lane planes 2,3
+  double* part = reinterpret_cast<double*>(sm + L.part);
+#pragma unroll
+  for (int mb = 0; mb < 4; ++mb) {
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) {
+      int hi[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hi[e] = __shfl_down_sync(0xFFFFFFFFu, d[mb][nb][e], 1);
+      const int bi = nb * 2 + (t >> 1);
+      if ((t & 1) == 0 && bi < B) {
+        const double v0 = static_cast<double>(d[mb][nb][0]) + 256.0 * d[mb][nb][1] + 65536.0 * hi[0] + 16777216.0 * hi[1];
+        const double v1 = static_cast<double>(d[mb][nb][2]) + 256.0 * d[mb][nb][3] + 65536.0 * hi[2] + 16777216.0 * hi[3];
+        part[(warp * 64 + 16 * mb + g) * B + bi] = v0;
+        part[(warp * 64 + 16 * mb + g + 8) * B + bi] = v1;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- block partials: warps in order, scale, exact correction for residual columns
+  double* cta = reinterpret_cast<double*>(sm + L.cta);
+  const bool any_resid = emax[4] != 0u;
+  for (int q = tid; q < B * 64; q += kI8Threads) {
+    const int bi = q >> 6, r = q & 63;
+    double acc = 0.0;
+    for (int w = 0; w < 8; ++w) acc += part[(w * 64 + r) * B + bi];
+    acc = ldexp(acc, static_cast<int>(emax[bi]) - 156);
+    if (any_resid) {
+      double corr = 0.0;
+      for (int wd = 0; wd < nt * 8; ++wd) {
+        uint32_t bits = mask[bi * a.tpc * 8 + wd];
+        while (bits) {
+          const int j = __ffs(bits) - 1;
+          bits &= bits - 1;
+          const int col = wd * 32 + j;  // column inside this block's slice
+          const int tt = col >> 8, c = col & 255, oc = c >> 3;
+          const uint2 hk = keytab[tt];
+          const uint32_t hh = hk.x * (32u * r + oc) + hk.y;
+          const uint32_t b = ((hh >> 30) * 32u + ((oc + r) & 31u)) * 8u + (c & 7);
+          const int code = static_cast<int8_t>(sm[L.codes + tt * 1024 + b]);
+          const uint16_t xb = a.x[static_cast<int64_t>(bi) * a.K + static_cast<int64_t>(t0) * kTileCols + col];
+          corr += static_cast<double>(code) * static_cast<double>(__uint_as_float(static_cast<uint32_t>(xb) << 16));
+        }
+      }
+      acc += corr;
+    }
+    cta[bi * 64 + r] = acc;
+  }
+  report(a.status, flags);
+  cluster.sync();
+
+  // ---- cluster reduction in rank order, row-block scale, fp32 output
+  {
+    const double s = static_cast<double>(__half2float(__ushort_as_half(a.scales[rb])));
+    for (int q = crank * kI8Threads + tid; q < B * 64; q += a.C * kI8Threads) {
+      double acc = 0.0;
+      for (int c = 0; c < a.C; ++c) acc += *cluster.map_shared_rank(&cta[q], c);
+      const int bi = q >> 6, r = q & 63;
+      a.y[static_cast<int64_t>(bi) * a.M + static_cast<int64_t>(rb) * 64 + r] = static_cast<float>(acc * s);
+    }
+  }
+  cluster.sync();  // keep shared memory alive until every peer has read it
+}
+
+template <int B>
+static cudaError_t launch_i8_t(GemvI8Args a, int64_t RB, cudaStream_t stream) {
+  const size_t smem = gemv_i8_layout(a.tpc, B).total;
+  auto kern = gemv_i8_kernel<B>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.blockDim = dim3(kI8Threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// T, C, tpc: the same block geometry as the bf16 path; batch * tpc * 32 <= kI8MaxChunks.
+cudaError_t launch_gemv_i8(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                           const uint16_t* x, int batch, float* y, uint32_t* status, int T, int C, int tpc, bool pdl,
+                           cudaStream_t stream, int inject) {
+  GemvI8Args a;
+  a.inject = inject;
+  a.codes = codes; a.scales = scales; a.x = x; a.y = y;
+  a.M = M; a.K = K; a.seed = seed; a.status = status;
+  a.T = T; a.C = C; a.tpc = tpc; a.batch = batch; a.pdl = pdl ? 1 : 0;
+  const int64_t RB = M / kRowsPerBlock;
+  switch (batch) {
+    case 1: return launch_i8_t<1>(a, RB, stream);
+    case 2: return launch_i8_t<2>(a, RB, stream);
+    case 3: return launch_i8_t<3>(a, RB, stream);
+    default: return launch_i8_t<4>(a, RB, stream);
+  }
+}
+
+}  // namespace usk

@@ -1,0 +1,88 @@
+"""The C ABI without a GPU: the library loads, exports every symbol that
+include/usk.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sub_bit_weight_usk_b200 as usk
+from sub_bit_weight_usk_b200 import _build, _native
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return _native.load_library()
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            with open(os.path.join(ROOT, "include", f)) as fh:
+                names |= set(re.findall(r"USK_API\s+[\w\s\*]+?\b(usk_\w+)\s*\(", fh.read()))
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert {"usk_build", "usk_gemv", "usk_gemm", "usk_sizes"} <= names
+    raw = ctypes.CDLL(_native.LIB_PATH)
+    for n in sorted(names):
+        assert hasattr(raw, n), n
+    assert names == set(_native.EXPORTED)
+
+
+def test_sizes_and_strings(lib):
+    assert usk.usk_format_version() == 1
+    assert usk.usk_sizes(4096, 4096) == (4096 * 4096 // 16, 2 * 64)
+    assert usk.usk_sizes(0, 0) == (0, 0)
+    with pytest.raises(usk.UskError):
+        usk.usk_sizes(63, 256)
+    with pytest.raises(usk.UskError):
+        usk.usk_sizes(64, 300)
+    with pytest.raises(usk.UskError):
+        usk.usk_sizes(64, 1 << 17)
+    for st in range(13):
+        assert lib.usk_status_str(st)
+    assert lib.usk_status_str(99) == b"unknown status"
+
+
+def test_argument_errors_return_before_any_launch(lib):
+    p = _native.UskParams(1, 0, 0)
+    fake = ctypes.c_void_p(16 * 1024)  # never dereferenced: validation fails first
+    # shape
+    assert lib.usk_build(fake, 1, 63, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 2
+    assert lib.usk_build(fake, 1, 64, 200, 200, None, ctypes.byref(p), fake, fake, None, None) == 2
+    # dtype, params, null
+    assert lib.usk_build(fake, 7, 64, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 3
+    assert lib.usk_build(fake, 1, 64, 256, 256, None, None, fake, fake, None, None) == 6
+    bad = _native.UskParams(2, 0, 0)
+    assert lib.usk_build(fake, 1, 64, 256, 256, None, ctypes.byref(bad), fake, fake, None, None) == 6
+    assert lib.usk_build(None, 1, 64, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 1
+    # alignment (W at an odd address, ldw not a multiple of 8 for bf16)
+    odd = ctypes.c_void_p(16 * 1024 + 2)
+    assert lib.usk_build(odd, 1, 64, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 10
+    assert lib.usk_build(fake, 1, 64, 256, 260, None, ctypes.byref(p), fake, fake, None, None) == 10
+    # M == 0 is a no-op
+    assert lib.usk_build(None, 1, 0, 256, 256, None, ctypes.byref(p), None, None, None, None) == 0
+    sk = _native.UskSketchC(64, 256, 0, 16 * 1024, 16 * 1024)
+    assert lib.usk_gemv(None, fake, 1, 1, fake, None, None) == 1
+    assert lib.usk_gemv(ctypes.byref(sk), fake, 1, 16, fake, None, None) == 4
+    assert lib.usk_gemv(ctypes.byref(sk), fake, 5, 1, fake, None, None) == 3
+    assert lib.usk_gemv_ex(ctypes.byref(sk), fake, 1, 1, fake, 8, None, None) == 6
+    assert lib.usk_gemv(ctypes.byref(sk), fake, 1, 0, fake, None, None) == 0
+    assert lib.usk_gemm(ctypes.byref(sk), fake, 8, fake, None, 0, None, None) == 4
+    assert lib.usk_gemm(ctypes.byref(sk), fake, 24, fake, None, 0, None, None) == 4
+    assert lib.usk_gemm(ctypes.byref(sk), fake, 512, fake, None, 0, None, None) == 4
+    unaligned = _native.UskSketchC(64, 256, 0, 16 * 1024 + 1, 16 * 1024)
+    assert lib.usk_gemv(ctypes.byref(unaligned), fake, 1, 1, fake, None, None) == 10
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        usk.usk_build(torch.zeros((64, 256), dtype=torch.bfloat16))

@@ -1,0 +1,71 @@
+"""Host logic of bench.py on the CPU: whole-job aggregation and the
+max-over-ranks timing reduction with two gloo ranks."""
+import json
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def test_aggregate_weak_scaling():
+    a = bench.aggregate(1, [2e-6], [10e-6], [20e-6])
+    assert a["gemv_gbs"] == pytest.approx(bench.GEMV_BYTES / 2e-6 / 1e9)
+    assert a["build_gweights_s"] == pytest.approx(bench.N_W / 10e-6 / 1e9)
+    b = bench.aggregate(2, [2e-6, 3e-6], [10e-6, 8e-6], [20e-6, 21e-6])
+    assert b["gemv_gbs"] == pytest.approx(2 * bench.GEMV_BYTES / 3e-6 / 1e9)  # slowest rank
+    assert b["ms_per_step"] == pytest.approx(21e-3)
+
+
+def test_algorithmic_bytes():
+    assert bench.GEMV_BYTES == 1073280
+    assert bench.BUILD_BYTES == 2 * 4096 * 4096 + 4096 * 4096 // 16 + 4 * 4096 + 128
+
+
+def test_rooflines_shape():
+    peaks = {"hbm_gbs": 6540.2, "bf16_tflops": 1645.9, "sm_max_mhz": 1965.0, "source": "measured"}
+    r = bench.rooflines(peaks, 5.3e-6, 0.451e-6, 1e-6, {})
+    assert r["usk_build"]["bound"] == "hbm" and 0.9 < r["usk_build"]["frac"] < 1.1
+    assert r["usk_gemv"]["bound"] == "alu" and 0.95 < r["usk_gemv"]["frac"] < 1.05
+    for v in r.values():
+        json.dumps(v)
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        vals = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 5.0])
+        out[rank] = vals
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert out[0] == [2.0, 10.0, 5.0] and out[1] == [2.0, 10.0, 5.0]
+
+
+def test_single_process_identity():
+    assert bench.max_over_ranks([3.0, 4.0]) == [3.0, 4.0]

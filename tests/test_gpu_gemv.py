@@ -120,3 +120,86 @@ def test_gemv_edges_and_errors():
     with pytest.raises(usk.UskError) as e:
         usk.usk_gemv(sk, buf[1:1 + 2 * 512].view(2, 512))
     assert e.value.status == 10
+
+
+# ------------------------------------------------------------- integer path (bf16 x, batch <= 4)
+
+@pytest.mark.parametrize("batch", [1, 2, 3, 4])
+@pytest.mark.parametrize("path", [1, 2])
+def test_gemv_paths_match_oracle(batch, path):
+    W = gen.weights_student_t(192, 2816, 7, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _sketch(W, gen.importance_lognormal(2816, 7), 19)
+    x = gen.activations(batch, 2816, 8, "bf16")
+    try:
+        usk.usk_debug_set_gemv_path(path)
+        y = usk.usk_gemv(sk, to_dev(x)).cpu().numpy()
+    finally:
+        usk.usk_debug_set_gemv_path(0)
+    ref = oracle.gemv_f64(o["codes"], o["scales"], 192, 2816, x, 19)
+    e = rel_err(y, ref)
+    # the integer path sums code * x exactly: only the final fp32 rounding remains
+    assert e <= (1e-6 if path == 2 else TOL), "relative error %.3e" % e
+
+
+def _int_path(sk, x, pdl=False):
+    usk.usk_debug_set_gemv_path(2)
+    try:
+        return usk.usk_gemv(sk, to_dev(x), pdl=pdl).cpu().numpy()
+    finally:
+        usk.usk_debug_set_gemv_path(0)
+
+
+def test_gemv_int_path_extreme_dynamic_range_is_exact():
+    """Elements far below the block's largest leave the digit planes and are
+    added by the exact correction."""
+    W = gen.weights_normal(128, 2048, 9, 0.02, "bf16")
+    sk, o = _sketch(W, None, 4)
+    g = np.random.default_rng(3)
+    xf = g.standard_normal((2, 2048)).astype(np.float32)
+    xf[0, 5] = 3.0e30          # 100 binades above the rest: every other element is residual
+    xf[0, 700] = 1.0e-30
+    xf[1, ::7] *= np.float32(1e-12)  # a spread of 40 binades in row 1
+    xf[1, 1] = 1.0e-38         # bf16 subnormal
+    x = gen.f32_to_bf16_bits(xf)
+    y = _int_path(sk, x)
+    ref = oracle.gemv_f64(o["codes"], o["scales"], 128, 2048, x, 4)
+    assert rel_err(y[0:1], ref[0:1]) <= 1e-6
+    assert rel_err(y[1:2], ref[1:2]) <= 1e-6
+    # the residual-only contribution of row 1 is still exact relative to itself
+    small = x.copy()
+    small[1, 0::7] = 0
+    assert np.all(np.isfinite(y))
+
+
+def test_gemv_int_path_nonfinite_x_propagates():
+    W = gen.weights_normal(64, 512, 10, 0.02, "bf16")
+    sk, o = _sketch(W, None, 2)
+    x = gen.activations(1, 512, 5, "bf16")
+    x[0, 100] = 0x7FC0  # NaN
+    y = _int_path(sk, x)
+    assert np.all(np.isnan(y))
+    x[0, 100] = 0x7F80  # +Inf
+    y = _int_path(sk, x)
+    ref = oracle.gemv_f64(o["codes"], o["scales"], 64, 512, x, 2)
+    assert np.array_equal(np.isnan(y), np.isnan(ref)) and np.array_equal(np.isinf(y), np.isinf(ref))
+    fin = np.isfinite(ref)
+    assert np.array_equal(np.sign(y[np.isinf(y)]), np.sign(ref[np.isinf(ref)]))
+    assert not fin.any() or rel_err(y[fin], ref[fin]) <= 1e-6
+
+
+def test_gemv_pdl_launch_matches_plain():
+    W = gen.weights_normal(256, 4096, 11, 0.02, "bf16")
+    sk, o = _sketch(W, None, 6)
+    other = usk.usk_build(to_dev(gen.weights_normal(256, 4096, 12, 0.02, "bf16")), None, 6)
+    x = to_dev(gen.activations(1, 4096, 13, "bf16"))
+    plain = usk.usk_gemv(sk, x)
+    ys = []
+    for _ in range(3):
+        usk.usk_build(to_dev(gen.weights_normal(256, 4096, 12, 0.02, "bf16")), None, 6,
+                      codes=other.codes, scales=other.scales)  # a neighbour kernel that writes another sketch
+        ys.append(usk.usk_gemv(sk, x, pdl=True))
+    torch.cuda.synchronize()
+    for yp in ys:
+        assert torch.equal(yp, plain)
+    ref = oracle.gemv_f64(o["codes"], o["scales"], 256, 4096, gen.activations(1, 4096, 13, "bf16"), 6)
+    assert rel_err(plain.cpu().numpy(), ref) <= 1e-6
