@@ -435,6 +435,32 @@ def run_usk(args):
     return 0
 
 
+def run_profile_case(args):
+    """A few launches of one kernel on the bench workload, for ncu captures
+    (e.g. ncu --set full --clock-control none -k regex:gemv -s 3 -c 1
+    python bench.py --profile-case gemv).  Prints nothing but a status line."""
+    import torch
+    import sub_bit_weight_usk_b200 as usk
+    dev = torch.device("cuda", 0)
+    cfg = gen.layer(GEMM_BATCH)
+    W = torch.from_numpy(cfg["W"].view(np.int16)).to(dev).view(torch.bfloat16)
+    imp = torch.from_numpy(cfg["importance"]).to(dev)
+    x16 = torch.from_numpy(cfg["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+    x1 = x16[:GEMV_BATCH].contiguous()
+    sk = usk.usk_build(W, imp, cfg["seed"])
+    torch.cuda.synchronize()
+    for _ in range(3 + 3):  # 3 warm-up launches, then 3 to capture
+        if args.profile_case == "build":
+            usk.usk_build(W, imp, cfg["seed"], codes=sk.codes, scales=sk.scales)
+        elif args.profile_case == "gemv":
+            usk.usk_gemv(sk, x1)
+        else:
+            usk.usk_gemm(sk, x16)
+    torch.cuda.synchronize()
+    print("profile case %s done" % args.profile_case)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -442,7 +468,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="usk", choices=["usk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", choices=["build", "gemv", "gemm"], default=None,
+                    help="run 6 launches of one kernel on the bench workload (for ncu) and exit")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        return run_profile_case(args)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

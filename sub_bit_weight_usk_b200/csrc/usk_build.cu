@@ -89,6 +89,11 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nt = (a.T - crank + a.C - 1) / a.C;  // this block's tiles: crank, crank + C, ...
 
+  // first half of a split cluster barrier; its wait, before the first remote
+  // access, guarantees that every block of the cluster has started
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  if (tid == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
+
   // ---- init: barriers, winner words of both slots, keys of both slots
   if (tid == 0) {
     for (int b = 0; b < a.nbuf; ++b) mbar_init(s0 + L.bars + 8 * b, 1);
@@ -178,7 +183,16 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a,
 
     if (!kSingle) {
       __syncthreads();
-      // pass 2: members that reach the maximum keep the smallest index and its value
+      // Non-finite screen: a NaN or Inf weight forces a key >= +Inf bits in
+      // its bucket; an fp32 overflow of |w| * importance can too, so the exact
+      // per-weight check runs only when the screen fires (rare).
+      bool screen;
+      {
+        const uint4 mx = lds128(keys_s + 16u * tid);
+        screen = __syncthreads_or(max(max(mx.x, mx.y), max(mx.z, mx.w)) >= 0x7F800000u) != 0;
+      }
+      // pass 2: members whose key equals the bucket maximum keep the smallest
+      // index and its value (predicated reductions, no divergent branches)
 #pragma unroll 2
       for (int q = 0; q < 8; ++q) {
         const uint32_t r = warp + 8 * q;
@@ -194,22 +208,21 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a,
           const uint4 v0 = lds128(wt + r * kRowBytes + lane * 32), v1 = lds128(wt + r * kRowBytes + lane * 32 + 16);
           wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w; wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
         }
+        uint32_t kmax[8];
+        static_for<8>([&](auto S) {
+          constexpr int s = decltype(S)::value;
+          kmax[s] = lds32_off<128 * s>(keys_s + off);
+        });
         static_for<8>([&](auto S) {
           constexpr int s = decltype(S)::value;
           uint32_t bits;
           if (BF16) bits = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
           else bits = wv[s];
           const float f = BF16 ? __uint_as_float(bits << 16) : __uint_as_float(bits);
-          const float k = HAS_IMP ? fabsf(f) * imp[s] : fabsf(f);
-          if (__float_as_uint(k) == lds32_off<128 * s>(keys_s + off)) {
-            // every non-finite weight is a candidate, or loses to one (a NaN key)
-            if ((__float_as_uint(f) & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
-            if (BF16) {
-              atoms_min_u32_off<128 * s>(win_s + off, ((l0 + s) << 16) | bits);
-            } else {
-              atoms_min_u64_off<256 * s>(win_s + 2 * off, (static_cast<uint64_t>(l0 + s) << 32) | bits);
-            }
-          }
+          const uint32_t k = __float_as_uint(HAS_IMP ? fabsf(f) * imp[s] : fabsf(f));
+          if (BF16) atoms_min_u32_off_if_eq<128 * s>(win_s + off, ((l0 + s) << 16) | bits, k, kmax[s]);
+          else atoms_min_u64_off_if_eq<256 * s>(win_s + 2 * off, (static_cast<uint64_t>(l0 + s) << 32) | bits, k, kmax[s]);
+          if (screen && (__float_as_uint(f) & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
         });
       }
     }
@@ -252,18 +265,16 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a,
     }
   }
 
-  // ---- row-block maximum across the cluster, scale, quantization
+  // ---- row-block maximum: every block pushes its maximum into every peer's
+  // word (remote atomicMax), then one cluster barrier; afterwards each block
+  // reads only its own shared memory, so no block waits for its peers to exit.
   vmax = __reduce_max_sync(0xFFFFFFFFu, vmax);
   if (lane == 0) atomicMax(&misc[0], vmax);
-  cluster.sync();  // also orders every block's value arrays before the reads below
-  if (warp == 0) {
-    uint32_t m = 0;
-    if (lane < a.C) m = *cluster.map_shared_rank(&misc[0], lane);
-    m = __reduce_max_sync(0xFFFFFFFFu, m);
-    if (lane == 0) misc[1] = m;
-  }
   __syncthreads();
-  const float mx = __uint_as_float(misc[1]);
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every block has started
+  if (warp == 0 && lane < a.C && lane != crank) atomicMax(cluster.map_shared_rank(&misc[0], lane), misc[0]);
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  const float mx = __uint_as_float(misc[0]);
   const __half s16 = __float2half_rn(mx / 127.0f);
   const float sc = __half2float(s16);
   if (crank == 0 && tid == 0) {
@@ -288,7 +299,6 @@ __global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a,
     *reinterpret_cast<uint32_t*>(dst) = packed;
   }
   report(a.status, flags);
-  cluster.sync();  // keep this block's shared memory alive until every peer has read it
 }
 
 // ---------------------------------------------------------------- launch

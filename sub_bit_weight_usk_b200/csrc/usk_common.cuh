@@ -208,6 +208,23 @@ __device__ __forceinline__ uint4 lds128_off(uint32_t addr) {
   return v;
 }
 
+// Predicated forms: the reduction happens only when key == ref (no branch).
+template <int OFF>
+__device__ __forceinline__ void atoms_min_u32_off_if_eq(uint32_t addr, uint32_t v, uint32_t key, uint32_t ref) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.eq.u32 p, %2, %3;\n @p red.shared.min.u32 [%0+%4], %1;\n}" ::"r"(addr), "r"(v),
+      "r"(key), "r"(ref), "n"(OFF)
+      : "memory");
+}
+
+template <int OFF>
+__device__ __forceinline__ void atoms_min_u64_off_if_eq(uint32_t addr, uint64_t v, uint32_t key, uint32_t ref) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.eq.u32 p, %2, %3;\n @p red.shared.min.u64 [%0+%4], %1;\n}" ::"r"(addr), "l"(v),
+      "r"(key), "r"(ref), "n"(OFF)
+      : "memory");
+}
+
 template <int OFF>
 __device__ __forceinline__ void atoms_min_u64_off(uint32_t addr, uint64_t v) {
   asm volatile("red.shared.min.u64 [%0+%2], %1;" ::"r"(addr), "l"(v), "n"(OFF) : "memory");

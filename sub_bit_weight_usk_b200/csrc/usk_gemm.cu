@@ -49,14 +49,14 @@ struct GemmArgs {
   int N;       // batch (multiple of 16, <= 256)
   int splits;  // blocks along K per row tile (cluster size)
   uint32_t tmem_cols;
-  int inject;  // test hook: block (0, 0) skips the commit of its first chunk
+  int inject;  // test hook: block (0, 0) skips the commit of its last chunk
 };
 
 __host__ __device__ constexpr size_t gemm_stage_a_bytes() { return kBM * kBK * 2; }  // 16 KiB
 __host__ __device__ constexpr size_t gemm_stage_b_bytes(int N) { return static_cast<size_t>(N) * kBK * 2; }
 __host__ __device__ constexpr size_t gemm_smem_bytes(int N) {
   // 1 KiB alignment slack | A stages | B stages | 2 code buffers (2 row blocks x 1024 bf16) | barriers
-  return 1024 + kStages * (gemm_stage_a_bytes() + gemm_stage_b_bytes(N)) + 2 * 4096 + 128;
+  return 1024 + kStages * (gemm_stage_a_bytes() + gemm_stage_b_bytes(N)) + 2 * 4096 + 192;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -152,11 +152,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
   const uint32_t b_s = a_s + kStages * static_cast<uint32_t>(gemm_stage_a_bytes());
   const uint32_t bstage = static_cast<uint32_t>(gemm_stage_b_bytes(a.N));
   const uint32_t c_s = b_s + kStages * bstage;  // code buffers: [2][2 row blocks][2048 B]
-  const uint32_t bar_s = c_s + 2 * 4096;        // kStages mbarriers (8 B each)
+  const uint32_t bar_s = c_s + 2 * 4096;        // kStages stage mbarriers + 1 drain mbarrier (8 B each)
+  const uint32_t drain_s = bar_s + 8 * kStages;
   uint8_t* misc_g = base_g + (bar_s - base_s) + 64;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(misc_g);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(misc_g + 4);
-  volatile int* last_commit = reinterpret_cast<volatile int*>(misc_g + 8);  // last chunk whose MMAs were committed
 
   // K range of this block (whole tiles)
   const int t_begin = static_cast<int>((static_cast<int64_t>(a.T) * ks) / a.splits);
@@ -165,8 +165,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) mbar_init(bar_s + 8 * s, 1);
+    mbar_init(drain_s, 1);
     *abort_flag = 0u;
-    *last_commit = -1;
     mbar_fence_init();
   }
   __syncwarp();
@@ -268,26 +268,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
         mma_bf16(tmem_d, sw128_desc(a_stage + 32 * kk), sw128_desc(bst + 32 * kk), idesc,
                  (c > 0 || kk > 0) ? 1u : 0u);
       }
-      const bool skip = a.inject && c == 0 && ks == 0 && mt == 0;
-      if (!skip) {
-        mma_commit(bar_s + 8 * (c % kStages));
-        *last_commit = c;
-      }
+      const bool skip = a.inject && c == nk - 1 && ks == 0 && mt == 0;
+      if (!skip) mma_commit(bar_s + 8 * (c % kStages));
     }
   }
   cp_async_wait<0>();
   __syncthreads();
   aborted = aborted || (*abort_flag != 0u);
 
-  // Wait for the MMAs: all of them, or after a wait that gave up, the last
-  // committed chunk (a commit tracks every earlier MMA of the issuing thread),
-  // again bounded, so that no MMA is in flight when tensor memory is freed.
-  {
-    const int last = aborted ? *last_commit : nk - 1;
-    if (last >= 0 && !mbar_wait(bar_s + 8 * (last % kStages), (last / kStages) & 1)) aborted = true;
+  // Wait for the last chunk's MMAs (bounded).  If any wait gave up, thread 0
+  // commits once more to a dedicated barrier -- a commit tracks every earlier
+  // MMA of the issuing thread -- and the block waits for it (bounded again),
+  // so that no MMA is in flight when tensor memory is freed.
+  if (!aborted && nk > 0) {
+    const int last = nk - 1;
+    if (!mbar_wait(bar_s + 8 * (last % kStages), (last / kStages) & 1)) aborted = true;
+  }
+  aborted = __syncthreads_or(aborted ? 1 : 0) != 0;
+  if (aborted) {
+    if (tid == 0) mma_commit(drain_s);
+    mbar_wait(drain_s, 0);
+    report(a.status, USK_FLAG_TIMEOUT);
   }
   tc_fence_after();
-  if (aborted) report(a.status, USK_FLAG_TIMEOUT);
 
   // ---- epilogue: TMEM -> registers (this warp's 32 lanes = rows 32 warp .. +31)
   const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[rb])) : 0.0f;

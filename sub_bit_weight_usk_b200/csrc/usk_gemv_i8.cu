@@ -44,10 +44,11 @@ struct GemvI8Args {
 };
 
 constexpr int kI8Threads = 256;
-constexpr int kI8MaxChunks = 1024;  // batch * tiles per block * 32 must not exceed this
+constexpr int kI8MaxChunks = 2048;  // 4-element x chunks per block: batch * tiles per block * 64 <= this
+constexpr int kI8MaxCluster = 8;
 
 struct GemvI8Layout {
-  uint32_t codes, keys, xs, pitch, mask, emax, bar, part, cta, total;
+  uint32_t codes, keys, xs, pitch, mask, emax, bar, acc, push, total;
 };
 
 __host__ __device__ inline GemvI8Layout gemv_i8_layout(int tpc, int batch) {
@@ -59,9 +60,9 @@ __host__ __device__ inline GemvI8Layout gemv_i8_layout(int tpc, int batch) {
   L.mask = (L.xs + 4u * batch * L.pitch + 15u) & ~15u;         // u32 [batch][tpc * 8] residual bits
   L.emax = L.mask + static_cast<uint32_t>(batch) * tpc * 32u;  // u32 [4] max exponent, [4] any-residual
   L.bar = (L.emax + 32u + 7u) & ~7u;                           // mbarrier
-  L.part = (L.bar + 8u + 15u) & ~15u;                          // f64 [8 warps][64][batch]
-  L.cta = L.part + 8u * 64u * batch * 8u;                      // f64 [batch][64]
-  L.total = L.cta + static_cast<uint32_t>(batch) * 64u * 8u;
+  L.acc = (L.bar + 8u + 15u) & ~15u;                           // s64 [8 warps][64][batch] plane-combined sums
+  L.push = L.acc + 8u * 64u * batch * 8u;                      // f64 [cluster][batch][64] (used in rank 0)
+  L.total = L.push + kI8MaxCluster * 64u * batch * 8u;
   return L;
 }
 
@@ -71,6 +72,12 @@ __device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1
       "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint2 ldg_nc64(const void* p) {
+  uint2 v;
+  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
 }
 
 // bf16 bits -> (effective biased exponent, significand as an integer), subnormals with exponent 1
@@ -84,7 +91,7 @@ __device__ __forceinline__ void bf16_parts(uint32_t b, int& e_eff, int& mant) {
 template <int B>
 __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a) {
   constexpr int NB = (4 * B + 7) / 8;  // n tiles of 8 planes
-  constexpr int kXR = kI8MaxChunks / kI8Threads;  // x chunks (8 elements) per thread
+  constexpr int kXR = kI8MaxChunks / kI8Threads;  // x chunks (4 elements) per thread
   extern __shared__ __align__(16) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -97,37 +104,42 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   uint32_t* mask = reinterpret_cast<uint32_t*>(sm + L.mask);
   uint32_t* emax = reinterpret_cast<uint32_t*>(sm + L.emax);  // [0..3] exponent, [4] any residual
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  long long* acc = reinterpret_cast<long long*>(sm + L.acc);
+  // first half of a split cluster barrier: its wait (before the first remote
+  // access) then guarantees that every block of the cluster has started
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-  // ---- stage: codes by one bulk copy (weights: independent of earlier kernels)
+  // ---- codes: one bulk copy (weights are not written by the kernels this one may overlap)
   if (tid == 0) {
     mbar_init(s0 + L.bar, 1);
     mbar_fence_init();
+    if (!(a.inject && crank == 0 && rb == 0)) {
+      mbar_arrive_expect_tx(s0 + L.bar, static_cast<uint32_t>(nt) * 1024u);
+      bulk_g2s(s0 + L.codes, a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0),
+               static_cast<uint32_t>(nt) * 1024u, s0 + L.bar);
+    }
   }
-  if (tid < 8) emax[tid] = 0u;
-  for (int q = tid; q < B * a.tpc * 8; q += kI8Threads) mask[q] = 0u;
-  __syncthreads();
-  if (tid == 0 && !(a.inject && crank == 0 && rb == 0)) {
-    mbar_arrive_expect_tx(s0 + L.bar, static_cast<uint32_t>(nt) * 1024u);
-    bulk_g2s(s0 + L.codes, a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0),
-             static_cast<uint32_t>(nt) * 1024u, s0 + L.bar);
-  }
-  if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
   if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  // ---- stage x: pass 1, largest exponent per batch row
-  const int cpr = nt * 32;  // 8-element chunks per batch row
+  // ---- x: 4-element chunks, all loads in flight before anything else
+  const int cpr = nt * 64;  // chunks per batch row
   const int nchunks = B * cpr;
-  uint4 xv[kXR];
+  uint2 xv[kXR];
 #pragma unroll
   for (int u = 0; u < kXR; ++u) {
     const int c = tid + u * kI8Threads;
-    xv[u] = make_uint4(0u, 0u, 0u, 0u);
+    xv[u] = make_uint2(0u, 0u);
     if (c < nchunks) {
       const int bi = c / cpr, cc = c % cpr;
-      xv[u] = ldg_nc128(a.x + static_cast<int64_t>(bi) * a.K + static_cast<int64_t>(t0) * kTileCols + 8 * cc);
+      xv[u] = ldg_nc64(a.x + static_cast<int64_t>(bi) * a.K + static_cast<int64_t>(t0) * kTileCols + 4 * cc);
     }
   }
+  if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
+  if (tid < 8) emax[tid] = 0u;
+  for (int q = tid; q < B * a.tpc * 8; q += kI8Threads) mask[q] = 0u;
+  __syncthreads();
+
+  // ---- x pass 1: largest finite exponent per batch row
   {
     int em[B];
 #pragma unroll
@@ -137,14 +149,13 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
       const int c = tid + u * kI8Threads;
       if (c < nchunks) {
         const int bi = c / cpr;
-        const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+        const uint32_t w[2] = {xv[u].x, xv[u].y};
         int m = 0;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           const uint32_t b = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-          int ee, mm;
-          bf16_parts(b, ee, mm);
-          if (mm != 0 && ((b >> 7) & 0xFFu) != 0xFFu) m = max(m, ee);
+          const int ex = static_cast<int>((b >> 7) & 0xFFu);
+          if ((b & 0x7FFFu) != 0u && ex != 0xFF) m = max(m, ex == 0 ? 1 : ex);
         }
 #pragma unroll
         for (int q = 0; q < B; ++q)
@@ -159,18 +170,18 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
   }
   __syncthreads();
 
-  // ---- stage x: pass 2, digit planes and the residual bits
+  // ---- x pass 2: digit planes (one 4-byte word per plane per chunk) and residual bits
 #pragma unroll
   for (int u = 0; u < kXR; ++u) {
     const int c = tid + u * kI8Threads;
     if (c < nchunks) {
       const int bi = c / cpr, cc = c % cpr;
       const int E = static_cast<int>(emax[bi]);
-      const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-      uint32_t dw[8];
+      const uint32_t w[2] = {xv[u].x, xv[u].y};
+      uint32_t dw[4];
       uint32_t rbits = 0u;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
+      for (int e = 0; e < 4; ++e) {
         const uint32_t b = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
         int ee, mm;
         bf16_parts(b, ee, mm);
@@ -183,26 +194,17 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
         if (b & 0x8000u) v = -v;
         dw[e] = (static_cast<uint32_t>(v) + 0x80808080u) ^ 0x80808080u;  // balanced base-256 digits
       }
-      // 4x4 byte transposes: plane p gets byte p of every column's digit word
-      uint32_t pl[4][2];
+      // 4x4 byte transpose: plane p gets byte p of the four columns' digit words
+      const uint32_t t_0 = __byte_perm(dw[0], dw[1], 0x5140);
+      const uint32_t t_1 = __byte_perm(dw[0], dw[1], 0x7362);
+      const uint32_t t_2 = __byte_perm(dw[2], dw[3], 0x5140);
+      const uint32_t t_3 = __byte_perm(dw[2], dw[3], 0x7362);
+      const uint32_t pl[4] = {__byte_perm(t_0, t_2, 0x5410), __byte_perm(t_0, t_2, 0x7632),
+                              __byte_perm(t_1, t_3, 0x5410), __byte_perm(t_1, t_3, 0x7632)};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t t_0 = __byte_perm(dw[4 * h], dw[4 * h + 1], 0x5140);
-        const uint32_t t_1 = __byte_perm(dw[4 * h], dw[4 * h + 1], 0x7362);
-        const uint32_t t_2 = __byte_perm(dw[4 * h + 2], dw[4 * h + 3], 0x5140);
-        const uint32_t t_3 = __byte_perm(dw[4 * h + 2], dw[4 * h + 3], 0x7362);
-        pl[0][h] = __byte_perm(t_0, t_2, 0x5410);
-        pl[1][h] = __byte_perm(t_0, t_2, 0x7632);
-        pl[2][h] = __byte_perm(t_1, t_3, 0x5410);
-        pl[3][h] = __byte_perm(t_1, t_3, 0x7632);
-      }
-#pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        const uint32_t dst = s0 + L.xs + (4 * bi + p) * L.pitch + 8 * cc;
-        asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(dst), "r"(pl[p][0]), "r"(pl[p][1]) : "memory");
-      }
+      for (int p = 0; p < 4; ++p) sts32(s0 + L.xs + (4 * bi + p) * L.pitch + 4 * cc, pl[p]);
       if (rbits) {
-        atomicOr(&mask[bi * a.tpc * 8 + (cc >> 2)], rbits << (8 * (cc & 3)));
+        atomicOr(&mask[bi * a.tpc * 8 + (cc >> 3)], rbits << (4 * (cc & 7)));
         emax[4] = 1u;
       }
     }
@@ -249,9 +251,12 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
     }
   }
 
-  // ---- recombine the planes (exact in float64): lanes with even t hold planes 0,1
-  // of batch row nb*2 + t/2, the next lane planes 2,3
-  double* part = reinterpret_cast<double*>(sm + L.part);
+  // dependents may start launching now: their code prefetch overlaps this epilogue
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // ---- recombine the planes in 64-bit integers (exact); each warp stores its
+  // sums, then the block adds the 8 warps (integer addition: exact).
+  // Lanes with even t hold planes 0, 1 of batch row nb*2 + t/2, the next lane 2, 3.
 #pragma unroll
   for (int mb = 0; mb < 4; ++mb) {
 #pragma unroll
@@ -261,58 +266,75 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
       for (int e = 0; e < 4; ++e) hi[e] = __shfl_down_sync(0xFFFFFFFFu, d[mb][nb][e], 1);
       const int bi = nb * 2 + (t >> 1);
       if ((t & 1) == 0 && bi < B) {
-        const double v0 = static_cast<double>(d[mb][nb][0]) + 256.0 * d[mb][nb][1] + 65536.0 * hi[0] + 16777216.0 * hi[1];
-        const double v1 = static_cast<double>(d[mb][nb][2]) + 256.0 * d[mb][nb][3] + 65536.0 * hi[2] + 16777216.0 * hi[3];
-        part[(warp * 64 + 16 * mb + g) * B + bi] = v0;
-        part[(warp * 64 + 16 * mb + g + 8) * B + bi] = v1;
+        const long long v0 = static_cast<long long>(d[mb][nb][0]) + 256ll * d[mb][nb][1] + 65536ll * hi[0] +
+                             16777216ll * hi[1];
+        const long long v1 = static_cast<long long>(d[mb][nb][2]) + 256ll * d[mb][nb][3] + 65536ll * hi[2] +
+                             16777216ll * hi[3];
+        acc[(warp * 64 + 16 * mb + g) * B + bi] = v0;
+        acc[(warp * 64 + 16 * mb + g + 8) * B + bi] = v1;
       }
     }
   }
   __syncthreads();
 
-  // ---- block partials: warps in order, scale, exact correction for residual columns
-  double* cta = reinterpret_cast<double*>(sm + L.cta);
+  // ---- block partial: scale and the exact correction for residual columns
   const bool any_resid = emax[4] != 0u;
-  for (int q = tid; q < B * 64; q += kI8Threads) {
-    const int bi = q >> 6, r = q & 63;
-    double acc = 0.0;
-    for (int w = 0; w < 8; ++w) acc += part[(w * 64 + r) * B + bi];
-    acc = ldexp(acc, static_cast<int>(emax[bi]) - 156);
-    if (any_resid) {
-      double corr = 0.0;
-      for (int wd = 0; wd < nt * 8; ++wd) {
-        uint32_t bits = mask[bi * a.tpc * 8 + wd];
-        while (bits) {
-          const int j = __ffs(bits) - 1;
-          bits &= bits - 1;
-          const int col = wd * 32 + j;  // column inside this block's slice
-          const int tt = col >> 8, c = col & 255, oc = c >> 3;
-          const uint2 hk = keytab[tt];
-          const uint32_t hh = hk.x * (32u * r + oc) + hk.y;
-          const uint32_t b = ((hh >> 30) * 32u + ((oc + r) & 31u)) * 8u + (c & 7);
-          const int code = static_cast<int8_t>(sm[L.codes + tt * 1024 + b]);
-          const uint16_t xb = a.x[static_cast<int64_t>(bi) * a.K + static_cast<int64_t>(t0) * kTileCols + col];
-          corr += static_cast<double>(code) * static_cast<double>(__uint_as_float(static_cast<uint32_t>(xb) << 16));
+  double part[(B * 64 + kI8Threads - 1) / kI8Threads];
+#pragma unroll
+  for (int k = 0; k < (B * 64 + kI8Threads - 1) / kI8Threads; ++k) {
+    const int q = tid + k * kI8Threads;
+    part[k] = 0.0;
+    if (q < B * 64) {
+      const int bi = q >> 6, r = q & 63;
+      long long tot = 0;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) tot += acc[(w * 64 + r) * B + bi];
+      double v = ldexp(static_cast<double>(tot), static_cast<int>(emax[bi]) - 156);
+      if (any_resid) {
+        double corr = 0.0;
+        for (int wd = 0; wd < nt * 8; ++wd) {
+          uint32_t bits = mask[bi * a.tpc * 8 + wd];
+          while (bits) {
+            const int j = __ffs(bits) - 1;
+            bits &= bits - 1;
+            const int col = wd * 32 + j;  // column inside this block's slice
+            const int tt = col >> 8, c = col & 255, oc = c >> 3;
+            const uint2 hk = keytab[tt];
+            const uint32_t hh = hk.x * (32u * r + oc) + hk.y;
+            const uint32_t bkt = ((hh >> 30) * 32u + ((oc + r) & 31u)) * 8u + (c & 7);
+            const int code = static_cast<int8_t>(sm[L.codes + tt * 1024 + bkt]);
+            const uint16_t xb = a.x[static_cast<int64_t>(bi) * a.K + static_cast<int64_t>(t0) * kTileCols + col];
+            corr += static_cast<double>(code) * static_cast<double>(__uint_as_float(static_cast<uint32_t>(xb) << 16));
+          }
         }
+        v += corr;
       }
-      acc += corr;
+      part[k] = v;
     }
-    cta[bi * 64 + r] = acc;
   }
   report(a.status, flags);
-  cluster.sync();
 
-  // ---- cluster reduction in rank order, row-block scale, fp32 output
+  // ---- push the partial into block 0 of the cluster; block 0 adds them in rank order
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every block has started
   {
-    const double s = static_cast<double>(__half2float(__ushort_as_half(a.scales[rb])));
-    for (int q = crank * kI8Threads + tid; q < B * 64; q += a.C * kI8Threads) {
-      double acc = 0.0;
-      for (int c = 0; c < a.C; ++c) acc += *cluster.map_shared_rank(&cta[q], c);
-      const int bi = q >> 6, r = q & 63;
-      a.y[static_cast<int64_t>(bi) * a.M + static_cast<int64_t>(rb) * 64 + r] = static_cast<float>(acc * s);
+    double* push0 = cluster.map_shared_rank(reinterpret_cast<double*>(sm + L.push), 0);
+#pragma unroll
+    for (int k = 0; k < (B * 64 + kI8Threads - 1) / kI8Threads; ++k) {
+      const int q = tid + k * kI8Threads;
+      if (q < B * 64) push0[crank * B * 64 + q] = part[k];
     }
   }
-  cluster.sync();  // keep shared memory alive until every peer has read it
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (crank == 0) {
+    const double* push = reinterpret_cast<const double*>(sm + L.push);
+    const double s = static_cast<double>(__half2float(__ushort_as_half(a.scales[rb])));
+    for (int q = tid; q < B * 64; q += kI8Threads) {
+      double tot = 0.0;
+      for (int c = 0; c < a.C; ++c) tot += push[c * B * 64 + q];
+      const int bi = q >> 6, r = q & 63;
+      a.y[static_cast<int64_t>(bi) * a.M + static_cast<int64_t>(rb) * 64 + r] = static_cast<float>(tot * s);
+    }
+  }
 }
 
 template <int B>

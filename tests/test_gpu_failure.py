@@ -40,7 +40,7 @@ def test_build_wait_timeout_reported_then_recovers():
 
 
 def test_gemm_wait_timeout_reported_then_recovers():
-    W = gen.weights_normal(128, 256, 2, 0.02, "bf16")  # one block, four K chunks
+    W = gen.weights_normal(128, 256, 2, 0.02, "bf16")  # one block, four K chunks; the last commit is skipped
     sk = usk.usk_build(to_dev(W), None, 1)
     x = gen.activations(16, 256, 3, "bf16")
     flags = _inject(2, lambda st: usk.usk_gemm(sk, to_dev(x), status=st))
