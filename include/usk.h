@@ -157,8 +157,9 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
                                float* y, uint32_t flags, uint32_t* d_status, void* stream);
 
 /* y = W_hat x for batch 16..256 (multiple of 16) on the tcgen05 tensor cores:
- * decoded bf16 tiles of W_hat are written to shared memory and multiplied with
- * bf16 x tiles, fp32 accumulation in tensor memory.
+ * decoded bf16 tiles of W_hat are written to tensor memory and multiplied with
+ * bf16 x tiles (copied into shared memory by the tensor memory accelerator),
+ * fp32 accumulation in tensor memory.
  *   x_bf16 [batch, K] bf16, 16-byte aligned.  y [batch, M] fp32.
  *   ws / ws_bytes: unused by this version (may be NULL / 0).
  * M == 0 is a no-op; K == 0 writes y = 0. */
@@ -173,13 +174,19 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
 USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block);
 
 /* Test hook: choose the usk_gemv path (0 = automatic, 1 = bf16 tensor path,
- * 2 = integer path where eligible).  Both give results within the products'
- * tolerance; process-wide. */
+ * 2 = integer path with thread-block clusters where eligible, 3 = integer
+ * row-slab path where eligible: bf16 x and batch * K <= 16384).  Every path
+ * gives results within the products' tolerance; process-wide. */
 USK_API void usk_debug_set_gemv_path(int path);
 
+/* Test hook: rows per thread block of the row-slab path (16, 32 or 64; any
+ * other value restores the automatic choice).  The result does not depend on
+ * it; process-wide. */
+USK_API void usk_debug_set_gemv_rows(int rows);
+
 /* Test hook for the failure path (host-made; no device fault): kernel = 1 makes
- * usk_build, 2 usk_gemm, 3 usk_gemv (integer path) skip one bulk copy or one
- * MMA commit in thread block (0, 0), so that block's bounded wait gives up
+ * usk_build, 2 usk_gemm, 3 usk_gemv (integer path) skip one bulk or tensor
+ * copy in thread block (0, 0), so that block's bounded wait gives up
  * after about 1 s and sets USK_FLAG_TIMEOUT; the kernel still completes and the
  * context stays usable.  0 switches it off.  Process-wide. */
 USK_API void usk_debug_inject_timeout(int kernel);

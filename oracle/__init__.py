@@ -62,6 +62,8 @@ def _load():
         i64, u64, vp = ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p
         lib.orc_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, u64, vp, vp, vp, vp]
         lib.orc_build.restype = ctypes.c_int
+        lib.orc_build_rows.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, u64, i64, vp, vp, vp, vp]
+        lib.orc_build_rows.restype = ctypes.c_int
         lib.orc_decode.argtypes = [vp, vp, i64, i64, u64, vp]
         lib.orc_decode.restype = ctypes.c_int
         lib.orc_gemv_f64.argtypes = [vp, vp, i64, i64, u64, vp, ctypes.c_int, i64, vp, i64, vp]
@@ -102,8 +104,11 @@ def _weights(W):
     raise TypeError("weights must be float32 or uint16 (bf16 bit patterns)")
 
 
-def build_sketch(W, importance=None, seed=0, want_winners=False):
-    """Sketch of W [M, K].  Returns dict(status, codes, scales[, winner, value])."""
+def build_sketch(W, importance=None, seed=0, want_winners=False, row_block0=0):
+    """Sketch of W [M, K].  Returns dict(status, codes, scales[, winner, value]).
+
+    row_block0 > 0: W holds the rows starting at row block row_block0 of a
+    larger matrix with the same K (the hash uses the true row blocks)."""
     W, dt = _weights(W)
     M, K = W.shape
     imp = None if importance is None else np.ascontiguousarray(importance, dtype=np.float32)
@@ -112,8 +117,8 @@ def build_sketch(W, importance=None, seed=0, want_winners=False):
     scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
     winner = np.full(max(nb, 1), -2, dtype=np.int64) if want_winners else None
     value = np.zeros(max(nb, 1), dtype=np.float32) if want_winners else None
-    st = _load().orc_build(_ptr(W), dt, M, K, K, _ptr(imp), seed, _ptr(codes), _ptr(scales),
-                           _ptr(winner), _ptr(value))
+    st = _load().orc_build_rows(_ptr(W), dt, M, K, K, _ptr(imp), seed, row_block0, _ptr(codes),
+                                _ptr(scales), _ptr(winner), _ptr(value))
     out = {"status": st, "codes": codes[:nb], "scales": scales[: M // 64]}
     if want_winners:
         out["winner"] = winner[:nb]

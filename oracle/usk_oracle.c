@@ -182,11 +182,26 @@ static float load_elem(const void* p, int dtype, int64_t idx) {
  * The scan below visits the weights of each tile in row-major order and keeps
  * a running best per bucket, which is the sequential hash-and-update the pages
  * describe; the maximum does not depend on the order. */
+int orc_build_rows(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw,
+                   const float* imp, uint64_t seed, int64_t rb0, int8_t* codes,
+                   uint16_t* scales, int64_t* winner, float* value);
+
 int orc_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw,
               const float* imp, uint64_t seed, int8_t* codes, uint16_t* scales,
               int64_t* winner, float* value) {
+  return orc_build_rows(W, dtype, M, K, ldw, imp, seed, 0, codes, scales, winner, value);
+}
+
+/* Same as orc_build for the M rows starting at row block rb0 of a larger
+ * matrix: W holds rows [64*rb0, 64*rb0 + M), the hash uses their true row
+ * blocks, codes/scales/winner/value are those rows' slices (winner indices are
+ * relative to W). */
+int orc_build_rows(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw,
+                   const float* imp, uint64_t seed, int64_t rb0, int8_t* codes,
+                   uint16_t* scales, int64_t* winner, float* value) {
   int st = check_shape(M, K);
   if (st) return st;
+  if (rb0 < 0) return ORC_ERR_SHAPE;
   if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
   if (M == 0) return ORC_OK;
   if (!codes || !scales) return ORC_ERR_NULL;
@@ -217,7 +232,7 @@ int orc_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw,
         float w = load_elem(W, dtype, i * ldw + j);
         if (!isfinite(w)) status = ORC_ERR_NONFINITE;
         float k = fabsf(w) * (imp ? imp[j] : 1.0f);
-        int64_t b = orc_bucket_index(K, seed, i, j) - rb * per_block;
+        int64_t b = orc_bucket_index(K, seed, i + rb0 * ROWS_PER_BLOCK, j) - (rb + rb0) * per_block;
         int64_t flat = i * K + j;
         /* strictly larger key wins; an equal key never displaces the earlier
          * (smaller-index) member because the scan is in row-major order */

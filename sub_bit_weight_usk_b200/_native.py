@@ -54,7 +54,8 @@ class UskSketchC(ctypes.Structure):
 _lib = None
 
 EXPORTED = ["usk_sizes", "usk_build", "usk_gemv", "usk_gemv_ex", "usk_gemm", "usk_status_str",
-            "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_inject_timeout"]
+            "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_set_gemv_rows",
+            "usk_debug_inject_timeout"]
 GEMV_PDL = 1
 
 
@@ -86,6 +87,8 @@ def load_library(path: str = LIB_PATH):
     lib.usk_debug_set_geometry.restype = None
     lib.usk_debug_set_gemv_path.argtypes = [ctypes.c_int]
     lib.usk_debug_set_gemv_path.restype = None
+    lib.usk_debug_set_gemv_rows.argtypes = [ctypes.c_int]
+    lib.usk_debug_set_gemv_rows.restype = None
     lib.usk_debug_inject_timeout.argtypes = [ctypes.c_int]
     lib.usk_debug_inject_timeout.restype = None
     _lib = lib
@@ -218,8 +221,14 @@ def usk_debug_set_geometry(build_cluster: int = 0, gemv_tiles_per_block: int = 0
 
 
 def usk_debug_set_gemv_path(path: int = 0) -> None:
-    """0 automatic, 1 bf16 tensor path, 2 integer path (where eligible)."""
+    """0 automatic, 1 bf16 tensor path, 2 integer path with clusters, 3 integer
+    row-slab path (2 and 3 where eligible)."""
     load_library().usk_debug_set_gemv_path(int(path))
+
+
+def usk_debug_set_gemv_rows(rows: int = 0) -> None:
+    """Rows per block of the row-slab path (16, 32, 64; other values = automatic)."""
+    load_library().usk_debug_set_gemv_rows(int(rows))
 
 
 def usk_debug_inject_timeout(kernel: int = 0) -> None:

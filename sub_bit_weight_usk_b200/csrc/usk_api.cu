@@ -12,9 +12,10 @@ cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t
                          cudaStream_t stream, int cluster_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int inject);
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject);
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject);
+bool gemm_supported(int64_t K, int batch);
 }  // namespace usk
 
 namespace {
@@ -47,6 +48,7 @@ usk_status from_cuda(cudaError_t e) { return e == cudaSuccess ? USK_OK : USK_ERR
 int g_build_cluster = 0;
 int g_gemv_tiles_per_block = 0;
 int g_gemv_path = 0;
+int g_gemv_rows = 0;
 int g_inject = 0;  // 1 build, 2 gemm, 3 gemv (integer path): skip one copy/commit in block (0, 0)
 
 }  // namespace
@@ -124,7 +126,8 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
   if ((reinterpret_cast<uintptr_t>(y) & 3u) != 0) return USK_ERR_ALIGN;
   cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
                                    xdtype == USK_F32, static_cast<int>(batch), y, d_status,
-                                   (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_inject == 3);
+                                   (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows,
+                                   g_inject == 3);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -141,6 +144,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   usk_status st = check_sketch(sketch);
   if (st != USK_OK) return st;
   if (batch < USK_GEMM_MIN_BATCH || batch > USK_GEMM_MAX_BATCH || batch % 16 != 0) return USK_ERR_BATCH;
+  if (!usk::gemm_supported(sketch->K, static_cast<int>(batch))) return USK_ERR_SHAPE;
   if (sketch->M == 0) return USK_OK;
   if (!y) return USK_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -162,6 +166,8 @@ USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block)
 }
 
 USK_API void usk_debug_set_gemv_path(int path) { g_gemv_path = path; }
+
+USK_API void usk_debug_set_gemv_rows(int rows) { g_gemv_rows = rows; }
 
 USK_API void usk_debug_inject_timeout(int kernel) { g_inject = kernel; }
 

@@ -72,7 +72,7 @@ __host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int
 }
 
 template <bool BF16, bool HAS_IMP>
-__global__ void __launch_bounds__(kBuildThreads) build_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
+__global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
   constexpr bool kSingle = BF16 && !HAS_IMP;
   constexpr uint32_t kRowBytes = kTileCols * (BF16 ? 2 : 4);
   constexpr uint32_t kTileBytes = kRowsPerBlock * kRowBytes;
@@ -322,8 +322,11 @@ static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override
     if (p.smem > 220u * 1024u) p = mk(cluster_override, 1);
     return p;
   }
-  BuildPlan p = mk(8, 2);
-  if (p.smem > 112u * 1024u && T > 8) p = mk(16, 2);  // keep two blocks per SM
+  // 4 blocks per row block measured fastest at 4096 x 4096 and 28672 x 8192;
+  // larger clusters only to keep two blocks per SM when K is long
+  BuildPlan p = mk(4, 2);
+  if (p.smem > 112u * 1024u && T > 4) p = mk(8, 2);
+  if (p.smem > 112u * 1024u && T > 8) p = mk(16, 2);
   if (p.smem > 220u * 1024u) p = mk(p.C, 1);
   return p;
 }

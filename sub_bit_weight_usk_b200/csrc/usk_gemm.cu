@@ -5,25 +5,32 @@
 // product W_hat = S . P^T; here W_hat is decoded tile by tile straight into the
 // tensor-core operand layout and never reaches global memory.
 //
-// Design (B200, sm_100a):
+// Design (B200, sm_100a), warp-specialised pipeline:
 //  * A thread block owns 128 output rows (two 64-row scale blocks) and a range
-//    of the K dimension; blocks that split K for the same rows form a cluster
-//    and add their fp32 partials through distributed shared memory in rank
-//    order (deterministic, no workspace).
-//  * K advances in chunks of 64 columns.  Per chunk, each of the 128 threads
-//    decodes the 8 octets of its row: rehash (one multiply-add per octet),
-//    gather the 8 bf16 bucket codes with one 16-byte shared load from the
-//    staged tile codes (conflict-free because class = (octet + row) mod 32),
-//    and store them as one 16-byte chunk of the 128-byte-swizzled K-major
-//    operand tile.  x is copied into the B operand tile with cp.async.
-//  * One thread issues four tcgen05.mma (M=128, N=batch, K=16, bf16 x bf16 ->
-//    fp32) per chunk and commits them to the chunk's stage barrier; a ring of
-//    4 stages lets decoding run ahead of the tensor core.  Codes are exact in
-//    bf16 and so are the products; the row-block scale is applied in the
-//    epilogue after tcgen05.ld.
-//  * Every mbarrier wait is bounded (about 1 s of globaltimer); a wait that
-//    gives up sets USK_FLAG_TIMEOUT, the block skips the remaining work, frees
-//    its tensor memory and returns.
+//    of whole hash tiles along K; blocks that split K for the same rows form a
+//    cluster and add their fp32 partials through distributed shared memory in
+//    rank order (deterministic, no workspace).
+//  * At start the block's int8 codes (2 row blocks x its tiles) arrive in
+//    shared memory with two bulk copies.  Once per tile the decoders widen that
+//    tile's 2 x 1024 codes to bf16 (exact) in a double buffer, so a code is
+//    converted once instead of once per use (16 uses); a bounded per-tile
+//    mbarrier among the decoders orders the buffer reuse.
+//  * 8 decoder warps: per 64-column chunk each thread rebuilds 4 octets of one
+//    row -- one multiply-add of the hash per octet, one 16-byte conflict-free
+//    gather of the 8 bf16 codes (class = (octet + row) mod 32) -- and writes
+//    the 32 weights straight into tensor memory (tcgen05.st, its row is its
+//    TMEM lane): the A operand never touches shared memory, which leaves the
+//    shared-memory bandwidth to the code gathers and the B (x) operand.
+//  * 1 copy warp: per chunk, as soon as the stage is free, one tensor copy of
+//    the x tile (B operand, 128-byte swizzle) onto the stage's "full" barrier.
+//  * 1 MMA warp: per chunk, once the stage is full, four tcgen05.mma (M=128,
+//    N=batch, K=16, A from tensor memory, B from shared memory, bf16 -> fp32)
+//    and a commit to the stage's "empty" mbarrier.  A ring of stages lets
+//    decode, copy and MMA overlap.
+//  * Epilogue: tcgen05.ld of the accumulator, x row-block scale, y.
+//  * Every mbarrier wait is bounded (about 1 s); a wait that gives up sets
+//    USK_FLAG_TIMEOUT, the pipeline stops, one final commit drains the tensor
+//    core before tensor memory is freed, and the kernel returns.
 #include <cooperative_groups.h>
 
 #include "usk_common.cuh"
@@ -32,15 +39,19 @@ namespace cg = cooperative_groups;
 
 namespace usk {
 
-constexpr int kGemmThreads = 128;
+constexpr int kDecWarps = 8;
+constexpr int kMmaWarp = kDecWarps;       // lane 0 issues the MMAs; the warp owns TMEM
+constexpr int kCopyWarp = kDecWarps + 1;  // lane 0 copies the x tiles ahead of the MMAs
+constexpr int kGemmThreads = (kDecWarps + 2) * 32;
+constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kStages = 4;
+constexpr int kMaxTiles = 32;  // hash tiles per block (codes staged up front)
 
 struct GemmArgs {
   const int8_t* codes;
   const uint16_t* scales;
-  const uint16_t* x;
   float* y;
   int64_t M, K;
   uint64_t seed;
@@ -49,26 +60,42 @@ struct GemmArgs {
   int N;       // batch (multiple of 16, <= 256)
   int splits;  // blocks along K per row tile (cluster size)
   uint32_t tmem_cols;
-  int inject;  // test hook: block (0, 0) skips the commit of its last chunk
+  uint32_t a_col;  // first tensor-memory column of the A stages
+  int inject;  // test hook: block (0, 0) skips the x copy of its first chunk
 };
 
-__host__ __device__ constexpr size_t gemm_stage_a_bytes() { return kBM * kBK * 2; }  // 16 KiB
-__host__ __device__ constexpr size_t gemm_stage_b_bytes(int N) { return static_cast<size_t>(N) * kBK * 2; }
-__host__ __device__ constexpr size_t gemm_smem_bytes(int N) {
-  // 1 KiB alignment slack | A stages | B stages | 2 code buffers (2 row blocks x 1024 bf16) | barriers
-  return 1024 + kStages * (gemm_stage_a_bytes() + gemm_stage_b_bytes(N)) + 2 * 4096 + 192;
+struct GemmLayout {
+  uint32_t b, cbf, codes, keys, bars, misc, total;
+};
+
+__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta) {
+  GemmLayout L;
+  L.b = 0;                                                             // [stages][N x 64] bf16, SW128
+  L.cbf = L.b + kStages * static_cast<uint32_t>(N) * kBK * 2;          // bf16 [2 buffers][2][1024]
+  L.codes = L.cbf + 2u * 2u * 1024u * 2u;                              // int8 [2][tcta][1024]
+  L.keys = L.codes + 2u * tcta * 1024u;                                // uint2 [2][tcta]
+  L.bars = (L.keys + 2u * tcta * 8u + 7u) & ~7u;                       // full[S], empty[S], codes, done, tile
+  L.misc = L.bars + (2 * kStages + 3) * 8;                             // tmem holder, abort
+  L.total = L.misc + 16;
+  return L;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// Tensor-memory columns: the fp32 accumulator [0, N), then kStages A stages of
+// 32 columns (128 rows x 64 bf16) from column a_col(N).
+__host__ __device__ inline uint32_t gemm_a_col(int N) { return (static_cast<uint32_t>(N) + 31u) & ~31u; }
+__host__ __device__ inline uint32_t gemm_tmem_cols(int N) {
+  const uint32_t need = gemm_a_col(N) + kStages * 32u;
+  uint32_t c = 32;
+  while (c < need) c <<= 1;
+  return c;
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint32_t addr) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(addr) : "memory");
+}
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (start address and offsets in 16-byte units).
@@ -87,237 +114,255 @@ __device__ __forceinline__ uint32_t idesc_bf16_f32(int N) {
          (static_cast<uint32_t>(kBM >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  const uint32_t no_mask = 0u;  // no output lane disabled
+// D (tmem) += A (tmem) * B (smem descriptor); accumulate = 0 overwrites D.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(no_mask)
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void mma_commit(uint32_t mbar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ uint32_t bf16x2_from_i8(int lo, int hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(static_cast<float>(lo), static_cast<float>(hi));
-  return *reinterpret_cast<uint32_t*>(&v);
+// two int8 codes (bytes 0 and 1 of w) -> one bf16 pair, exact (|code| <= 127)
+__device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w) {
+  const float f0 = static_cast<float>(static_cast<int8_t>(w & 0xFFu));
+  const float f1 = static_cast<float>(static_cast<int8_t>((w >> 8) & 0xFFu));
+  __nv_bfloat162 p = __floats2bfloat162_rn(f0, f1);
+  return *reinterpret_cast<uint32_t*>(&p);
 }
 
-// Load 16 codes (one 16-byte chunk) of tile tc for the block's row block
-// rb_local, or zeros for a row block past the end of the matrix.
-__device__ __forceinline__ uint4 load_code_chunk(const GemmArgs& a, int64_t rb, int tc, int chunk) {
-  if (rb >= a.M / kRowsPerBlock) return make_uint4(0u, 0u, 0u, 0u);
-  return ldg_nc128(a.codes + rb * 4 * a.K + 1024 * static_cast<int64_t>(tc) + 16 * chunk);
-}
-
-__device__ __forceinline__ void store_code_chunk(uint32_t dst, uint4 v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t o[8];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    o[2 * e] = bf16x2_from_i8(static_cast<int8_t>(w[e] & 0xFF), static_cast<int8_t>((w[e] >> 8) & 0xFF));
-    o[2 * e + 1] = bf16x2_from_i8(static_cast<int8_t>((w[e] >> 16) & 0xFF), static_cast<int8_t>(w[e] >> 24));
-  }
-  sts128(dst, make_uint4(o[0], o[1], o[2], o[3]));
-  sts128(dst + 16, make_uint4(o[4], o[5], o[6], o[7]));
-}
-
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a) {
+__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ks = static_cast<int>(cluster.block_rank());
   const int mt = blockIdx.y;
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   const uint32_t raw_s = smem_u32(sm_raw);
-  const uint32_t base_s = (raw_s + 1023u) & ~1023u;
-  uint8_t* base_g = sm_raw + (base_s - raw_s);
-  const uint32_t a_s = base_s;
-  const uint32_t b_s = a_s + kStages * static_cast<uint32_t>(gemm_stage_a_bytes());
-  const uint32_t bstage = static_cast<uint32_t>(gemm_stage_b_bytes(a.N));
-  const uint32_t c_s = b_s + kStages * bstage;  // code buffers: [2][2 row blocks][2048 B]
-  const uint32_t bar_s = c_s + 2 * 4096;        // kStages stage mbarriers + 1 drain mbarrier (8 B each)
-  const uint32_t drain_s = bar_s + 8 * kStages;
-  uint8_t* misc_g = base_g + (bar_s - base_s) + 64;
-  volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(misc_g);
-  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(misc_g + 4);
+  const uint32_t s0 = (raw_s + 1023u) & ~1023u;
+  uint8_t* sm = sm_raw + (s0 - raw_s);
 
-  // K range of this block (whole tiles)
   const int t_begin = static_cast<int>((static_cast<int64_t>(a.T) * ks) / a.splits);
   const int t_end = static_cast<int>((static_cast<int64_t>(a.T) * (ks + 1)) / a.splits);
-  const int nk = (t_end - t_begin) * (kTileCols / kBK);  // chunks
+  const int tcta = t_end - t_begin;
+  const int nk = tcta * (kTileCols / kBK);  // 64-column chunks
+  const GemmLayout L = gemm_layout(a.N, tcta);
+  const uint32_t bstage = static_cast<uint32_t>(a.N) * kBK * 2;
+  const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * kStages, codes_bar = empty_s + 8 * kStages;
+  const uint32_t done_bar = codes_bar + 8, tile_bar = done_bar + 8;
+  volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(sm + L.misc);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
+  uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
+  const int64_t RB = a.M / kRowsPerBlock;
+  const int rb0 = 2 * mt;
+  const bool second_rb = rb0 + 1 < RB;
 
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(bar_s + 8 * s, 1);
-    mbar_init(drain_s, 1);
-    *abort_flag = 0u;
-    mbar_fence_init();
-  }
-  __syncwarp();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(full_s + 8 * s, kDecThreads + 1);
+        mbar_init(empty_s + 8 * s, 1);
+      }
+      mbar_init(codes_bar, 1);
+      mbar_init(done_bar, 1);
+      mbar_init(tile_bar, kDecThreads);
+      *abort_flag = 0u;
+      mbar_fence_init();
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+      // the block's codes: two contiguous runs (one per row block)
+      const uint32_t bytes = static_cast<uint32_t>(tcta) * 1024u;
+      mbar_arrive_expect_tx(codes_bar, bytes * (second_rb ? 2u : 1u));
+      bulk_g2s(s0 + L.codes, a.codes + static_cast<int64_t>(rb0) * 4 * a.K + 1024 * static_cast<int64_t>(t_begin),
+               bytes, codes_bar);
+      if (second_rb)
+        bulk_g2s(s0 + L.codes + bytes,
+                 a.codes + static_cast<int64_t>(rb0 + 1) * 4 * a.K + 1024 * static_cast<int64_t>(t_begin), bytes,
+                 codes_bar);
+    }
+    __syncwarp();
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(const_cast<uint32_t*>(tmem_holder))),
                  "r"(a.tmem_cols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-
-  // this thread's decode row
-  const int m = tid;
-  const int64_t row = static_cast<int64_t>(mt) * kBM + m;
-  const bool row_ok = row < a.M;
-  const int rbl = m >> 6;                                   // row block inside the 128-row tile
-  const int64_t rb = static_cast<int64_t>(mt) * 2 + rbl;    // global row block
-  const uint32_t r = static_cast<uint32_t>(m & 63);
-
-  // stage the first tile's codes; prefetch the next one into registers
-  const int crbl = tid >> 6, cchunk = tid & 63;  // staging role: row block, 16-code chunk
-  const int64_t crb = static_cast<int64_t>(mt) * 2 + crbl;
-  uint4 pre = make_uint4(0u, 0u, 0u, 0u);
-  if (nk > 0) {
-    store_code_chunk(c_s + crbl * 2048 + 32 * cchunk, load_code_chunk(a, crb, t_begin, cchunk));
-    if (t_begin + 1 < t_end) pre = load_code_chunk(a, crb, t_begin + 1, cchunk);
+  } else if (tid < 2 * tcta) {
+    const int rbl = tid / tcta, tl = tid % tcta;
+    keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb0 + rbl) * a.T + t_begin + tl);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = *tmem_holder;
-  const uint32_t idesc = idesc_bf16_f32(a.N);
   bool aborted = false;
 
-  // B (x) copies of chunk c into stage c % kStages
-  auto issue_x = [&](int c) {
-    const uint32_t dst_stage = b_s + (c % kStages) * bstage;
-    const int64_t k0 = static_cast<int64_t>(t_begin) * kTileCols + static_cast<int64_t>(c) * kBK;
-    for (int p = tid; p < a.N * 8; p += kGemmThreads) {
-      const int n = p >> 3, c8 = p & 7;
-      const uint32_t dst = dst_stage + (n >> 3) * 1024 + (n & 7) * 128 + ((c8 ^ (n & 7)) << 4);
-      cp_async16(dst, a.x + static_cast<int64_t>(n) * a.K + k0 + 8 * c8);
-    }
-    cp_async_commit();
-  };
-
-  if (nk > 0) issue_x(0);
-  uint2 hk = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t_begin);
-
-  for (int c = 0; c < nk; ++c) {
-    const int tl = c >> 2;  // tile index inside this block's range
-    const int tc = t_begin + tl;
-    if ((c & 3) == 0 && c > 0) hk = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + tc);
-
-    // the stage of chunk c + 1 must have been consumed by the MMAs of chunk c + 1 - kStages
-    if (c + 1 < nk) {
-      const int prev = c + 1 - kStages;
-      if (prev >= 0 && !aborted) {
-        if (!mbar_wait(bar_s + 8 * (prev % kStages), (prev / kStages) & 1)) aborted = true;
+  if (warp < kDecWarps) {
+    // ---------------- decoders
+    const int m = tid & 127;             // row in the 128-row tile
+    const int half = tid >> 7;           // octets 4*half .. 4*half + 3 of each chunk
+    const int rbl = m >> 6;
+    const uint32_t r = static_cast<uint32_t>(m & 63);
+    const bool row_ok = static_cast<int64_t>(mt) * kBM + m < a.M;
+    // this thread's tensor-memory lane (= its row) and its 16 columns of an A stage
+    const uint32_t a_taddr = tmem_d + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + a.a_col + half * 16u;
+    // widen tile tl's codes (both row blocks) into bf16 buffer tl % 2: 8 per thread
+    auto widen = [&](int tl) {
+      const int wrb = tid >> 7, part = tid & 127;
+      const uint2 w = lds64(s0 + L.codes + static_cast<uint32_t>(wrb * tcta + tl) * 1024u + part * 8u);
+      const uint4 v = make_uint4(i8x2_to_bf16x2(w.x), i8x2_to_bf16x2(w.x >> 16), i8x2_to_bf16x2(w.y),
+                                 i8x2_to_bf16x2(w.y >> 16));
+      sts128(s0 + L.cbf + (tl & 1) * 4096u + wrb * 2048u + part * 16u, v);
+    };
+    // loop exits are warp-uniform: tcgen05.st is a whole-warp instruction
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(codes_bar, 0))) aborted = true;
+    if (!aborted && nk > 0) widen(0);
+    for (int c = 0; c < nk && !aborted; ++c) {
+      const int s = c % kStages;
+      const int tl = c >> 2;
+      if ((c & 3) == 0) {
+        // every decoder has finished tile tl - 1 and widened tile tl; buffer
+        // (tl + 1) % 2 is free for tile tl + 1
+        mbar_arrive(tile_bar);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(tile_bar, tl & 1))) {
+          aborted = true;
+          break;
+        }
+        if (tl + 1 < tcta) widen(tl + 1);
       }
-      issue_x(c + 1);
-    } else {
-      cp_async_commit();  // keep the group count uniform
-    }
-
-    // decode the 8 octets of row m in this chunk into stage c % kStages
-    const uint32_t a_stage = a_s + (c % kStages) * static_cast<uint32_t>(gemm_stage_a_bytes());
-    const uint32_t cbuf = c_s + (tl & 1) * 4096 + rbl * 2048;
-    const uint32_t arow = a_stage + (m >> 3) * 1024 + (m & 7) * 128;
-    const uint32_t ob = static_cast<uint32_t>((c & 3) * 8);
-    uint32_t h = hk.x * (32u * r + ob) + hk.y;
+      if (c >= kStages) {
+        // the MMAs that read this A stage have completed
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_s + 8 * s, ((c / kStages) - 1) & 1))) {
+          aborted = true;
+          break;
+        }
+        tc_fence_after();
+      }
+      const uint2 hk = keytab[rbl * tcta + tl];
+      const uint32_t ob = static_cast<uint32_t>((c & 3) * 8 + half * 4);
+      uint32_t h = hk.x * (32u * r + ob) + hk.y;
+      const uint32_t tile_codes = s0 + L.cbf + (tl & 1) * 4096u + rbl * 2048u;
+      uint32_t v[16];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (row_ok) {
-        const uint32_t cls = (ob + j + r) & 31u;
-        v = lds128(cbuf + ((h >> 30) * 32u + cls) * 16u);
+      for (int j = 0; j < 4; ++j) {
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (row_ok) {
+          const uint32_t cls = (ob + j + r) & 31u;
+          q = lds128(tile_codes + ((h >> 30) * 32u + cls) * 16u);
+        }
+        v[4 * j + 0] = q.x;
+        v[4 * j + 1] = q.y;
+        v[4 * j + 2] = q.z;
+        v[4 * j + 3] = q.w;
+        h += hk.x;
       }
-      sts128(arow + ((static_cast<uint32_t>(j) ^ static_cast<uint32_t>(m & 7)) << 4), v);
-      h += hk.x;
+      tmem_st16(a_taddr + s * 32u, v);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(full_s + 8 * s);
     }
-
-    // last chunk of a tile: stage the next tile's codes into the other buffer
-    if ((c & 3) == 3 && tl + 1 < t_end - t_begin) {
-      store_code_chunk(c_s + ((tl + 1) & 1) * 4096 + crbl * 2048 + 32 * cchunk, pre);
-      if (tc + 2 < t_end) pre = load_code_chunk(a, crb, tc + 2, cchunk);
+  } else if (warp == kCopyWarp && lane == 0) {
+    // ---------------- x tiles, up to kStages chunks ahead of the MMAs
+    for (int c = 0; c < nk && !aborted; ++c) {
+      const int s = c % kStages;
+      if (c >= kStages && !mbar_wait(empty_s + 8 * s, ((c / kStages) - 1) & 1)) {
+        aborted = true;
+        break;
+      }
+      if (a.inject && c == 0 && ks == 0 && mt == 0) continue;
+      mbar_arrive_expect_tx(full_s + 8 * s, bstage);
+      tma_load_2d(s0 + L.b + s * bstage, &xmap, t_begin * kTileCols + c * kBK, 0, full_s + 8 * s);
     }
-
-    cp_async_wait<1>();  // this chunk's x copies have landed
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-    if (aborted) *abort_flag = 1u;
-    if (tid == 0 && !*abort_flag) {
+  } else if (warp == kMmaWarp && lane == 0) {
+    // ---------------- MMAs
+    const uint32_t idesc = idesc_bf16_f32(a.N);
+    for (int c = 0; c < nk && !aborted; ++c) {
+      const int s = c % kStages;
+      if (!mbar_wait(full_s + 8 * s, (c / kStages) & 1)) {
+        aborted = true;
+        break;
+      }
       tc_fence_after();
-      const uint32_t bst = b_s + (c % kStages) * bstage;
+      const uint32_t a_tm = tmem_d + a.a_col + s * 32u;
+      const uint32_t bst = s0 + L.b + s * bstage;
 #pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk) {
-        mma_bf16(tmem_d, sw128_desc(a_stage + 32 * kk), sw128_desc(bst + 32 * kk), idesc,
-                 (c > 0 || kk > 0) ? 1u : 0u);
-      }
-      const bool skip = a.inject && c == nk - 1 && ks == 0 && mt == 0;
-      if (!skip) mma_commit(bar_s + 8 * (c % kStages));
+      for (int kk = 0; kk < kBK / 16; ++kk)
+        mma_bf16_ts(tmem_d, a_tm + 8u * kk, sw128_desc(bst + 32 * kk), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+      mma_commit(empty_s + 8 * s);
     }
+    // one more commit: tracks every MMA issued above (also after a failed wait)
+    mma_commit(done_bar);
   }
-  cp_async_wait<0>();
+  if (aborted) *abort_flag = 1u;
+  // every thread waits for the tensor core to drain (bounded)
+  if (!mbar_wait(done_bar, 0)) *abort_flag = 1u;
+  tc_fence_before();
   __syncthreads();
-  aborted = aborted || (*abort_flag != 0u);
-
-  // Wait for the last chunk's MMAs (bounded).  If any wait gave up, thread 0
-  // commits once more to a dedicated barrier -- a commit tracks every earlier
-  // MMA of the issuing thread -- and the block waits for it (bounded again),
-  // so that no MMA is in flight when tensor memory is freed.
-  if (!aborted && nk > 0) {
-    const int last = nk - 1;
-    if (!mbar_wait(bar_s + 8 * (last % kStages), (last / kStages) & 1)) aborted = true;
-  }
-  aborted = __syncthreads_or(aborted ? 1 : 0) != 0;
-  if (aborted) {
-    if (tid == 0) mma_commit(drain_s);
-    mbar_wait(drain_s, 0);
-    report(a.status, USK_FLAG_TIMEOUT);
-  }
   tc_fence_after();
+  const bool failed = *abort_flag != 0u;
+  if (failed && tid == 0) report(a.status, USK_FLAG_TIMEOUT);
 
-  // ---- epilogue: TMEM -> registers (this warp's 32 lanes = rows 32 warp .. +31)
-  const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[rb])) : 0.0f;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  if (a.splits == 1) {
-    for (int n0 = 0; n0 < a.N; n0 += 16) {
-      float v[16];
-      tmem_ld16(tmem_d + lane_base + n0, v);
-      if (row_ok && nk > 0 && !aborted) {
+  // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31,
+  // warps 0-3 the first half of the columns, warps 4-7 the second
+  if (warp < kDecWarps) {
+    const int sub = warp & 3;
+    const int m = sub * 32 + lane;
+    const int64_t row = static_cast<int64_t>(mt) * kBM + m;
+    const bool row_ok = row < a.M;
+    const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[row / kRowsPerBlock])) : 0.0f;
+    const int half_n = a.N / 2;
+    const int n_lo = (warp < 4) ? 0 : half_n, n_hi = (warp < 4) ? half_n : a.N;
+    const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
+    if (a.splits == 1) {
+      for (int n0 = n_lo; n0 < n_hi; n0 += 8) {
+        float v[8];
+        tmem_ld8(tmem_d + lane_base + n0, v);
+        if (row_ok) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a.y[static_cast<int64_t>(n0 + i) * a.M + row] = v[i] * scale;
-      } else if (row_ok) {
+          for (int i = 0; i < 8; ++i)
+            a.y[static_cast<int64_t>(n0 + i) * a.M + row] = (nk > 0 && !failed) ? v[i] * scale : 0.0f;
+        }
+      }
+    } else {
+      float* part = reinterpret_cast<float*>(sm + L.b);  // [N][128]: the x stage ring is free now
+      for (int n0 = n_lo; n0 < n_hi; n0 += 8) {
+        float v[8];
+        tmem_ld8(tmem_d + lane_base + n0, v);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) a.y[static_cast<int64_t>(n0 + i) * a.M + row] = 0.0f;
+        for (int i = 0; i < 8; ++i) part[(n0 + i) * kBM + m] = (nk > 0 && !failed) ? v[i] : 0.0f;
       }
     }
-  } else {
-    // partials to this block's shared memory as [n][128] (the stage area is free now)
-    float* part = reinterpret_cast<float*>(base_g);
-    for (int n0 = 0; n0 < a.N; n0 += 16) {
-      float v[16];
-      tmem_ld16(tmem_d + lane_base + n0, v);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) part[(n0 + i) * kBM + m] = (nk > 0 && !aborted) ? v[i] : 0.0f;
-    }
+  }
+  if (a.splits > 1) {
     cluster.sync();
-    // rank ks reduces a slice of the outputs, adding the blocks in rank order
+    // rank ks finishes a slice of the outputs, adding the blocks in rank order
+    float* part = reinterpret_cast<float*>(sm + L.b);
     const int total = a.N * kBM;
     const int per = (total + a.splits - 1) / a.splits;
     const int q0 = ks * per, q1 = min(total, q0 + per);
@@ -336,7 +381,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(a.tmem_cols)
                  : "memory");
@@ -345,35 +390,90 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a)
 
 // ---------------------------------------------------------------- launch
 
-static int gemm_splits(int64_t m_tiles, int T) {
-  int s = static_cast<int>(296 / (m_tiles > 0 ? m_tiles : 1));
-  if (s < 1) s = 1;
-  if (s > 8) s = 8;
-  if (s > T) s = T;
-  return s;
+constexpr uint32_t kSmemLimit = 227u * 1024u;
+
+// Largest number of tiles whose codes fit next to the stage ring for batch N.
+static int gemm_max_tiles(int N) {
+  int t = kMaxTiles;
+  while (t > 1 && gemm_layout(N, t).total + 1024u > kSmemLimit) --t;
+  return t;
 }
 
-static uint32_t tmem_columns(int N) {
-  uint32_t c = 32;
-  while (c < static_cast<uint32_t>(N)) c <<= 1;
-  return c;
+// Dynamic shared memory of a launch: the layout, padded so that no more blocks
+// share an SM than its 512 tensor-memory columns can hold (a block waiting in
+// tcgen05.alloc for a co-resident block of its own cluster would never proceed).
+static uint32_t gemm_smem_bytes(int N, int tpb) {
+  uint32_t smem = gemm_layout(N, tpb).total + 1024u;  // + alignment slack
+  const uint32_t max_blocks = 512u / gemm_tmem_cols(N);
+  const uint32_t floor_bytes = 233472u / (max_blocks + 1u) + 1u - 1024u;  // 228 KiB per SM, 1 KiB reserved per block
+  return smem > floor_bytes ? smem : floor_bytes;
+}
+
+// Blocks along K per 128-row tile: minimise (waves of blocks) x (tiles per
+// block + 1), the +1 standing for a block's fixed cost (prologue, pipeline
+// fill, epilogue and the cluster reduction), subject to the shared-memory
+// bound on tiles per block and clusters of at most 16.
+static int gemm_splits(int64_t m_tiles, int T, int N, int sms) {
+  const int max_tiles = gemm_max_tiles(N);
+  int best = -1;
+  int64_t best_cost = -1;
+  for (int s = 1; s <= 16 && s <= T; ++s) {
+    const int tpb = (T + s - 1) / s;
+    if (tpb > max_tiles) continue;
+    int occ = static_cast<int>(233472u / (gemm_smem_bytes(N, tpb) + 1024u));
+    if (occ < 1) occ = 1;
+    const int64_t slots = static_cast<int64_t>(sms) * occ;
+    const int64_t waves = (m_tiles * s + slots - 1) / slots;
+    const int64_t cost = waves * (tpb + 1);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+// Whether K fits: at most 16 blocks along K, each staging the codes of up to
+// gemm_max_tiles(batch) tiles (32 for every batch: K <= 131072).
+bool gemm_supported(int64_t K, int batch) {
+  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch));
 }
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject) {
   GemmArgs a;
-  a.inject = inject;
-  a.codes = codes; a.scales = scales; a.x = x; a.y = y;
-  a.M = M; a.K = K; a.seed = seed; a.status = status;
+  a.codes = codes; a.scales = scales; a.y = y;
+  a.M = M; a.K = K; a.seed = seed; a.status = status; a.inject = inject;
   a.T = static_cast<int>(K / kTileCols);
   a.N = batch;
   const int64_t m_tiles = (M + kBM - 1) / kBM;
-  a.splits = gemm_splits(m_tiles, a.T);
-  a.tmem_cols = tmem_columns(batch);
-  const size_t smem = gemm_smem_bytes(batch);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  a.splits = gemm_splits(m_tiles, a.T, batch, sms);
+  if (a.splits < 1) return cudaErrorInvalidValue;  // K beyond 16 blocks x the tiles one block can stage
+  a.tmem_cols = gemm_tmem_cols(batch);
+  a.a_col = gemm_a_col(batch);
+  const int tcta_max = (a.T + a.splits - 1) / a.splits;
+  const size_t smem = gemm_smem_bytes(batch, tcta_max);
+  // tensor map over x [batch, K] bf16: one 64-column x batch box per chunk, 128-byte swizzle
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  CUtensorMap xmap;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(batch)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2u};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(batch)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (encode(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(x), gdim, gstride, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
+  if (a.splits > 8) {
+    e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.splits, static_cast<unsigned>(m_tiles), 1);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
@@ -386,7 +486,7 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel, a);
+  return cudaLaunchKernelEx(&cfg, gemm_kernel, a, xmap);
 }
 
 }  // namespace usk

@@ -288,10 +288,24 @@ cudaError_t launch_gemv_i8(const int8_t* codes, const uint16_t* scales, int64_t 
                            const uint16_t* x, int batch, float* y, uint32_t* status, int T, int C, int tpc, bool pdl,
                            cudaStream_t stream, int inject);
 
-// path: 0 = automatic, 1 = bf16 tensor path, 2 = integer path (bf16 x, batch <= 4 only)
+bool slab_supported(int64_t K, int batch);
+cudaError_t launch_gemv_slab(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                             const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl,
+                             cudaStream_t stream, int rows_override, int inject);
+
+// path: 0 = automatic, 1 = bf16 tensor path, 2 = integer path with clusters,
+// 3 = integer row-slab path (bf16 x, batch * K <= 16384)
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int inject) {
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject) {
+  // the row-slab kernel pays its x preparation once per block: it wins once
+  // there are more than two row blocks per SM (measured at 28672 x 8192)
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const bool slab = path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms);
+  if (!xf32 && slab && slab_supported(K, batch))
+    return launch_gemv_slab(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl,
+                            stream, rows_override, inject);
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
   const bool i8_ok = !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
   if (i8_ok && path != 1)

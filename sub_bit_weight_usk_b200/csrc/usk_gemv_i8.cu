@@ -66,28 +66,6 @@ __host__ __device__ inline GemvI8Layout gemv_i8_layout(int tpc, int batch) {
   return L;
 }
 
-__device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                           uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint2 ldg_nc64(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-  return v;
-}
-
-// bf16 bits -> (effective biased exponent, significand as an integer), subnormals with exponent 1
-__device__ __forceinline__ void bf16_parts(uint32_t b, int& e_eff, int& mant) {
-  const int e = static_cast<int>((b >> 7) & 0xFFu);
-  const int m = static_cast<int>(b & 0x7Fu);
-  e_eff = e == 0 ? 1 : e;
-  mant = e == 0 ? m : (128 + m);
-}
-
 template <int B>
 __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a) {
   constexpr int NB = (4 * B + 7) / 8;  // n tiles of 8 planes

@@ -1,8 +1,7 @@
 """Failure path of the bounded device waits, injected from the host.
 
-A test hook makes thread block (0, 0) skip one bulk copy (usk_build, usk_gemv)
-or one MMA commit (usk_gemm); its bounded mbarrier wait gives up after about
-one second, sets USK_FLAG_TIMEOUT in the status word and the kernel completes.
+A test hook makes thread block (0, 0) skip one bulk or tensor copy (usk_build,
+usk_gemv, usk_gemm); its bounded mbarrier wait gives up after about one second, sets USK_FLAG_TIMEOUT in the status word and the kernel completes.
 No trap, no assert, no fault: the context stays usable, which the follow-up
 call checks against the oracle."""
 import numpy as np
@@ -40,7 +39,7 @@ def test_build_wait_timeout_reported_then_recovers():
 
 
 def test_gemm_wait_timeout_reported_then_recovers():
-    W = gen.weights_normal(128, 256, 2, 0.02, "bf16")  # one block, four K chunks; the last commit is skipped
+    W = gen.weights_normal(128, 256, 2, 0.02, "bf16")  # one block; the x copy of its first chunk is skipped
     sk = usk.usk_build(to_dev(W), None, 1)
     x = gen.activations(16, 256, 3, "bf16")
     flags = _inject(2, lambda st: usk.usk_gemm(sk, to_dev(x), status=st))
@@ -52,14 +51,19 @@ def test_gemm_wait_timeout_reported_then_recovers():
     assert rel_err(y, oracle.gemv_f64(o["codes"], o["scales"], 128, 256, x, 1)) <= 1e-3
 
 
-def test_gemv_wait_timeout_reported_then_recovers():
+@pytest.mark.parametrize("path", [2, 3])
+def test_gemv_wait_timeout_reported_then_recovers(path):
     W = gen.weights_normal(64, 256, 4, 0.02, "bf16")
     sk = usk.usk_build(to_dev(W), None, 2)
     x = gen.activations(1, 256, 5, "bf16")
-    flags = _inject(3, lambda st: usk.usk_gemv(sk, to_dev(x), status=st))
-    assert flags & usk.FLAG_TIMEOUT
-    st = status_tensor()
-    y = usk.usk_gemv(sk, to_dev(x), status=st).cpu().numpy()
+    usk.usk_debug_set_gemv_path(path)
+    try:
+        flags = _inject(3, lambda st: usk.usk_gemv(sk, to_dev(x), status=st))
+        assert flags & usk.FLAG_TIMEOUT
+        st = status_tensor()
+        y = usk.usk_gemv(sk, to_dev(x), status=st).cpu().numpy()
+    finally:
+        usk.usk_debug_set_gemv_path(0)
     assert int(st.item()) == 0
     o = oracle.build_sketch(W, None, 2)
     assert rel_err(y, oracle.gemv_f64(o["codes"], o["scales"], 64, 256, x, 2)) <= 1e-6

@@ -125,7 +125,7 @@ def test_gemv_edges_and_errors():
 # ------------------------------------------------------------- integer path (bf16 x, batch <= 4)
 
 @pytest.mark.parametrize("batch", [1, 2, 3, 4])
-@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("path", [1, 2, 3])
 def test_gemv_paths_match_oracle(batch, path):
     W = gen.weights_student_t(192, 2816, 7, 4.0, 0.02, 0.001, 20.0, "bf16")
     sk, o = _sketch(W, gen.importance_lognormal(2816, 7), 19)
@@ -137,19 +137,65 @@ def test_gemv_paths_match_oracle(batch, path):
         usk.usk_debug_set_gemv_path(0)
     ref = oracle.gemv_f64(o["codes"], o["scales"], 192, 2816, x, 19)
     e = rel_err(y, ref)
-    # the integer path sums code * x exactly: only the final fp32 rounding remains
-    assert e <= (1e-6 if path == 2 else TOL), "relative error %.3e" % e
+    # the integer paths sum code * x exactly: only the final fp32 rounding remains
+    assert e <= (1e-6 if path in (2, 3) else TOL), "relative error %.3e" % e
 
 
-def _int_path(sk, x, pdl=False):
-    usk.usk_debug_set_gemv_path(2)
+def _int_path(sk, x, pdl=False, path=2):
+    usk.usk_debug_set_gemv_path(path)
     try:
         return usk.usk_gemv(sk, to_dev(x), pdl=pdl).cpu().numpy()
     finally:
         usk.usk_debug_set_gemv_path(0)
 
 
-def test_gemv_int_path_extreme_dynamic_range_is_exact():
+# ------------------------------------------------------------- row-slab path (batch * K <= 16384)
+
+@pytest.mark.parametrize("rows", [16, 32, 64])
+@pytest.mark.parametrize("M,K,batch", [(64, 256, 1), (192, 2816, 3), (128, 4352, 2), (320, 1024, 4)])
+def test_gemv_slab_rows_match_oracle(rows, M, K, batch):
+    """Every slab height, ragged tile counts (11 and 17 tiles: partial copy
+    groups), row blocks that are not a multiple of the slab count."""
+    W = gen.weights_student_t(M, K, 21, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _sketch(W, gen.importance_lognormal(K, 21), 23)
+    x = gen.activations(batch, K, 24, "bf16")
+    usk.usk_debug_set_gemv_rows(rows)
+    try:
+        y = _int_path(sk, x, path=3)
+    finally:
+        usk.usk_debug_set_gemv_rows(0)
+    assert rel_err(y, oracle.gemv_f64(o["codes"], o["scales"], M, K, x, 23)) <= 1e-6
+
+
+@pytest.mark.parametrize("K,batch", [(16384, 1), (8192, 2), (4096, 4)])
+def test_gemv_slab_largest_x(K, batch):
+    """batch * K at the slab path's limit (x of the whole row in registers)."""
+    W = gen.weights_normal(128, K, 25, 0.02, "bf16")
+    sk, o = _sketch(W, None, 26)
+    x = gen.activations(batch, K, 27, "bf16")
+    y = _int_path(sk, x, path=3)
+    assert rel_err(y, oracle.gemv_f64(o["codes"], o["scales"], 128, K, x, 26)) <= 1e-6
+
+
+def test_gemv_slab_rows_do_not_change_result():
+    W = gen.weights_normal(256, 4096, 28, 0.02, "bf16")
+    sk, _ = _sketch(W, None, 29)
+    x = to_dev(gen.activations(2, 4096, 30, "bf16"))
+    ys = []
+    usk.usk_debug_set_gemv_path(3)
+    try:
+        for rows in (16, 32, 64):
+            usk.usk_debug_set_gemv_rows(rows)
+            ys.append(usk.usk_gemv(sk, x))
+    finally:
+        usk.usk_debug_set_gemv_rows(0)
+        usk.usk_debug_set_gemv_path(0)
+    # each output is one exact integer sum rounded once: identical bits
+    assert torch.equal(ys[0], ys[1]) and torch.equal(ys[0], ys[2])
+
+
+@pytest.mark.parametrize("path", [2, 3])
+def test_gemv_int_path_extreme_dynamic_range_is_exact(path):
     """Elements far below the block's largest leave the digit planes and are
     added by the exact correction."""
     W = gen.weights_normal(128, 2048, 9, 0.02, "bf16")
@@ -161,7 +207,7 @@ def test_gemv_int_path_extreme_dynamic_range_is_exact():
     xf[1, ::7] *= np.float32(1e-12)  # a spread of 40 binades in row 1
     xf[1, 1] = 1.0e-38         # bf16 subnormal
     x = gen.f32_to_bf16_bits(xf)
-    y = _int_path(sk, x)
+    y = _int_path(sk, x, path=path)
     ref = oracle.gemv_f64(o["codes"], o["scales"], 128, 2048, x, 4)
     assert rel_err(y[0:1], ref[0:1]) <= 1e-6
     assert rel_err(y[1:2], ref[1:2]) <= 1e-6
@@ -171,15 +217,16 @@ def test_gemv_int_path_extreme_dynamic_range_is_exact():
     assert np.all(np.isfinite(y))
 
 
-def test_gemv_int_path_nonfinite_x_propagates():
+@pytest.mark.parametrize("path", [2, 3])
+def test_gemv_int_path_nonfinite_x_propagates(path):
     W = gen.weights_normal(64, 512, 10, 0.02, "bf16")
     sk, o = _sketch(W, None, 2)
     x = gen.activations(1, 512, 5, "bf16")
     x[0, 100] = 0x7FC0  # NaN
-    y = _int_path(sk, x)
+    y = _int_path(sk, x, path=path)
     assert np.all(np.isnan(y))
     x[0, 100] = 0x7F80  # +Inf
-    y = _int_path(sk, x)
+    y = _int_path(sk, x, path=path)
     ref = oracle.gemv_f64(o["codes"], o["scales"], 64, 512, x, 2)
     assert np.array_equal(np.isnan(y), np.isnan(ref)) and np.array_equal(np.isinf(y), np.isinf(ref))
     fin = np.isfinite(ref)
