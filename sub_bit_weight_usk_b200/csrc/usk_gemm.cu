@@ -15,10 +15,10 @@
 //    tile's 2 x 1024 codes to bf16 (exact) in a double buffer, so a code is
 //    converted once instead of once per use (16 uses); a bounded per-tile
 //    mbarrier among the decoders orders the buffer reuse.
-//  * 8 decoder warps: per 64-column chunk each thread rebuilds 4 octets of one
+//  * 16 decoder warps: per 64-column chunk each thread rebuilds 2 octets of one
 //    row -- one multiply-add of the hash per octet, one 16-byte conflict-free
 //    gather of the 8 bf16 codes (class = (octet + row) mod 32) -- and writes
-//    the 32 weights straight into tensor memory (tcgen05.st, its row is its
+//    the 16 weights straight into tensor memory (tcgen05.st, its row is its
 //    TMEM lane): the A operand never touches shared memory, which leaves the
 //    shared-memory bandwidth to the code gathers and the B (x) operand.
 //  * 1 copy warp: per chunk, as soon as the stage is free, one tensor copy of
@@ -39,14 +39,16 @@ namespace cg = cooperative_groups;
 
 namespace usk {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 16;
+constexpr int kDecGroups = kDecWarps / 4;        // thread groups of 128 (one per row) splitting each chunk
+constexpr int kOctPerThread = 8 / kDecGroups;    // octets of a 64-column chunk per decoder thread
 constexpr int kMmaWarp = kDecWarps;       // lane 0 issues the MMAs; the warp owns TMEM
 constexpr int kCopyWarp = kDecWarps + 1;  // lane 0 copies the x tiles ahead of the MMAs
 constexpr int kGemmThreads = (kDecWarps + 2) * 32;
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 16;  // pipeline stages (A in tensor memory, B in shared memory)
 constexpr int kMaxTiles = 32;  // hash tiles per block (codes staged up front)
 
 struct GemmArgs {
@@ -61,6 +63,7 @@ struct GemmArgs {
   int splits;  // blocks along K per row tile (cluster size)
   uint32_t tmem_cols;
   uint32_t a_col;  // first tensor-memory column of the A stages
+  int S;           // pipeline stages
   int inject;  // test hook: block (0, 0) skips the x copy of its first chunk
 };
 
@@ -68,27 +71,24 @@ struct GemmLayout {
   uint32_t b, cbf, codes, keys, bars, misc, total;
 };
 
-__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta) {
+__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S) {
   GemmLayout L;
-  L.b = 0;                                                             // [stages][N x 64] bf16, SW128
-  L.cbf = L.b + kStages * static_cast<uint32_t>(N) * kBK * 2;          // bf16 [2 buffers][2][1024]
+  L.b = 0;  // [S][N x 64] bf16, SW128; after the main loop the K-split partials [N][128] fp32
+  const uint32_t ring = static_cast<uint32_t>(S) * N * kBK * 2, parts = static_cast<uint32_t>(N) * kBM * 4;
+  L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [2 buffers][2][1024]
   L.codes = L.cbf + 2u * 2u * 1024u * 2u;                              // int8 [2][tcta][1024]
   L.keys = L.codes + 2u * tcta * 1024u;                                // uint2 [2][tcta]
   L.bars = (L.keys + 2u * tcta * 8u + 7u) & ~7u;                       // full[S], empty[S], codes, done, tile
-  L.misc = L.bars + (2 * kStages + 3) * 8;                             // tmem holder, abort
+  L.misc = L.bars + (2 * S + 3) * 8;                                   // tmem holder, abort
   L.total = L.misc + 16;
   return L;
 }
 
-// Tensor-memory columns: the fp32 accumulator [0, N), then kStages A stages of
-// 32 columns (128 rows x 64 bf16) from column a_col(N).
+// Tensor memory: the fp32 accumulator [0, N), then the A stages, 32 columns
+// (128 rows x 64 bf16) each, from column a_col(N).  A block takes 256 columns
+// (two blocks per SM) when 2 or more stages fit next to the accumulator, else
+// all 512 (one block per SM).
 __host__ __device__ inline uint32_t gemm_a_col(int N) { return (static_cast<uint32_t>(N) + 31u) & ~31u; }
-__host__ __device__ inline uint32_t gemm_tmem_cols(int N) {
-  const uint32_t need = gemm_a_col(N) + kStages * 32u;
-  uint32_t c = 32;
-  while (c < need) c <<= 1;
-  return c;
-}
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -124,14 +124,19 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// 16 consecutive 32-bit columns of this thread's tensor-memory lane.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+// 8 or 16 consecutive 32-bit columns of this thread's tensor-memory lane.
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
           taddr),
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
+}
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -174,9 +179,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
   const int t_end = static_cast<int>((static_cast<int64_t>(a.T) * (ks + 1)) / a.splits);
   const int tcta = t_end - t_begin;
   const int nk = tcta * (kTileCols / kBK);  // 64-column chunks
-  const GemmLayout L = gemm_layout(a.N, tcta);
+  const int S = a.S;
+  const GemmLayout L = gemm_layout(a.N, tcta, S);
   const uint32_t bstage = static_cast<uint32_t>(a.N) * kBK * 2;
-  const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * kStages, codes_bar = empty_s + 8 * kStages;
+  const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * S, codes_bar = empty_s + 8 * S;
   const uint32_t done_bar = codes_bar + 8, tile_bar = done_bar + 8;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(sm + L.misc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
@@ -187,7 +193,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
 
   if (warp == kMmaWarp) {
     if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < S; ++s) {
         mbar_init(full_s + 8 * s, kDecThreads + 1);
         mbar_init(empty_s + 8 * s, 1);
       }
@@ -226,25 +232,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
   if (warp < kDecWarps) {
     // ---------------- decoders
     const int m = tid & 127;             // row in the 128-row tile
-    const int half = tid >> 7;           // octets 4*half .. 4*half + 3 of each chunk
+    const int grp = tid >> 7;            // octets kOctPerThread*grp .. + kOctPerThread - 1 of each chunk
     const int rbl = m >> 6;
     const uint32_t r = static_cast<uint32_t>(m & 63);
     const bool row_ok = static_cast<int64_t>(mt) * kBM + m < a.M;
-    // this thread's tensor-memory lane (= its row) and its 16 columns of an A stage
-    const uint32_t a_taddr = tmem_d + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + a.a_col + half * 16u;
-    // widen tile tl's codes (both row blocks) into bf16 buffer tl % 2: 8 per thread
+    // this thread's tensor-memory lane (= its row) and its columns of an A stage
+    const uint32_t a_taddr =
+        tmem_d + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + a.a_col + grp * (4u * kOctPerThread);
+    // widen tile tl's codes (both row blocks) into bf16 buffer tl % 2
     auto widen = [&](int tl) {
-      const int wrb = tid >> 7, part = tid & 127;
-      const uint2 w = lds64(s0 + L.codes + static_cast<uint32_t>(wrb * tcta + tl) * 1024u + part * 8u);
-      const uint4 v = make_uint4(i8x2_to_bf16x2(w.x), i8x2_to_bf16x2(w.x >> 16), i8x2_to_bf16x2(w.y),
-                                 i8x2_to_bf16x2(w.y >> 16));
-      sts128(s0 + L.cbf + (tl & 1) * 4096u + wrb * 2048u + part * 16u, v);
+      constexpr int per = 2048 / kDecThreads;  // codes per thread
+      const int wrb = (tid * per) >> 10, part = (tid * per) & 1023;
+      const uint32_t src = s0 + L.codes + static_cast<uint32_t>(wrb * tcta + tl) * 1024u + part;
+      const uint32_t dst = s0 + L.cbf + (tl & 1) * 4096u + wrb * 2048u + part * 2u;
+      if (per == 8) {
+        const uint2 w = lds64(src);
+        sts128(dst, make_uint4(i8x2_to_bf16x2(w.x), i8x2_to_bf16x2(w.x >> 16), i8x2_to_bf16x2(w.y),
+                               i8x2_to_bf16x2(w.y >> 16)));
+      } else {
+        const uint32_t w = lds32(src);
+        sts64(dst, make_uint2(i8x2_to_bf16x2(w), i8x2_to_bf16x2(w >> 16)));
+      }
     };
     // loop exits are warp-uniform: tcgen05.st is a whole-warp instruction
     if (!__all_sync(0xFFFFFFFFu, mbar_wait(codes_bar, 0))) aborted = true;
     if (!aborted && nk > 0) widen(0);
-    for (int c = 0; c < nk && !aborted; ++c) {
-      const int s = c % kStages;
+    int s = 0;
+    uint32_t ph = 0;  // phase parity of stage s's current use
+    for (int c = 0; c < nk && !aborted; ++c, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
       const int tl = c >> 2;
       if ((c & 3) == 0) {
         // every decoder has finished tile tl - 1 and widened tile tl; buffer
@@ -256,21 +271,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
         }
         if (tl + 1 < tcta) widen(tl + 1);
       }
-      if (c >= kStages) {
+      if (c >= S) {
         // the MMAs that read this A stage have completed
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_s + 8 * s, ((c / kStages) - 1) & 1))) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_s + 8 * s, ph ^ 1u))) {
           aborted = true;
           break;
         }
         tc_fence_after();
       }
       const uint2 hk = keytab[rbl * tcta + tl];
-      const uint32_t ob = static_cast<uint32_t>((c & 3) * 8 + half * 4);
+      const uint32_t ob = static_cast<uint32_t>((c & 3) * 8 + grp * kOctPerThread);
       uint32_t h = hk.x * (32u * r + ob) + hk.y;
       const uint32_t tile_codes = s0 + L.cbf + (tl & 1) * 4096u + rbl * 2048u;
-      uint32_t v[16];
+      uint32_t v[4 * kOctPerThread];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < kOctPerThread; ++j) {
         uint4 q = make_uint4(0u, 0u, 0u, 0u);
         if (row_ok) {
           const uint32_t cls = (ob + j + r) & 31u;
@@ -282,42 +297,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
         v[4 * j + 3] = q.w;
         h += hk.x;
       }
-      tmem_st16(a_taddr + s * 32u, v);
+      tmem_st(a_taddr + s * 32u, v);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(full_s + 8 * s);
     }
-  } else if (warp == kCopyWarp && lane == 0) {
-    // ---------------- x tiles, up to kStages chunks ahead of the MMAs
-    for (int c = 0; c < nk && !aborted; ++c) {
-      const int s = c % kStages;
-      if (c >= kStages && !mbar_wait(empty_s + 8 * s, ((c / kStages) - 1) & 1)) {
+  } else if (warp == kCopyWarp) {
+    // ---------------- x tiles, up to S chunks ahead of the MMAs.  The whole
+    // warp runs the loop (a lane spinning elsewhere would steal the warp from
+    // the issuing lane); lane 0 issues.
+    int s = 0;
+    uint32_t ph = 0;
+    for (int c = 0; c < nk && !aborted; ++c, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
+      if (c >= S && !__all_sync(0xFFFFFFFFu, mbar_wait(empty_s + 8 * s, ph ^ 1u))) {
         aborted = true;
         break;
       }
-      if (a.inject && c == 0 && ks == 0 && mt == 0) continue;
-      mbar_arrive_expect_tx(full_s + 8 * s, bstage);
-      tma_load_2d(s0 + L.b + s * bstage, &xmap, t_begin * kTileCols + c * kBK, 0, full_s + 8 * s);
+      if (lane == 0 && !(a.inject && c == 0 && ks == 0 && mt == 0)) {
+        mbar_arrive_expect_tx(full_s + 8 * s, bstage);
+        tma_load_2d(s0 + L.b + s * bstage, &xmap, t_begin * kTileCols + c * kBK, 0, full_s + 8 * s);
+      }
+      __syncwarp();
     }
-  } else if (warp == kMmaWarp && lane == 0) {
-    // ---------------- MMAs
+  } else if (warp == kMmaWarp) {
+    // ---------------- MMAs (whole warp in the loop, lane 0 issues)
     const uint32_t idesc = idesc_bf16_f32(a.N);
-    for (int c = 0; c < nk && !aborted; ++c) {
-      const int s = c % kStages;
-      if (!mbar_wait(full_s + 8 * s, (c / kStages) & 1)) {
+    int s = 0;
+    uint32_t ph = 0;
+    for (int c = 0; c < nk && !aborted; ++c, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(full_s + 8 * s, ph))) {
         aborted = true;
         break;
       }
       tc_fence_after();
-      const uint32_t a_tm = tmem_d + a.a_col + s * 32u;
-      const uint32_t bst = s0 + L.b + s * bstage;
+      if (lane == 0) {
+        const uint32_t a_tm = tmem_d + a.a_col + s * 32u;
+        const uint32_t bst = s0 + L.b + s * bstage;
 #pragma unroll
-      for (int kk = 0; kk < kBK / 16; ++kk)
-        mma_bf16_ts(tmem_d, a_tm + 8u * kk, sw128_desc(bst + 32 * kk), idesc, (c > 0 || kk > 0) ? 1u : 0u);
-      mma_commit(empty_s + 8 * s);
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          mma_bf16_ts(tmem_d, a_tm + 8u * kk, sw128_desc(bst + 32 * kk), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(empty_s + 8 * s);
+      }
+      __syncwarp();
     }
     // one more commit: tracks every MMA issued above (also after a failed wait)
-    mma_commit(done_bar);
+    if (lane == 0) mma_commit(done_bar);
+    __syncwarp();
   }
   if (aborted) *abort_flag = 1u;
   // every thread waits for the tensor core to drain (bounded)
@@ -328,32 +353,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
   const bool failed = *abort_flag != 0u;
   if (failed && tid == 0) report(a.status, USK_FLAG_TIMEOUT);
 
-  // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31,
-  // warps 0-3 the first half of the columns, warps 4-7 the second
+  // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31; the
+  // kDecGroups groups of four warps take the 8-column groups round robin
   if (warp < kDecWarps) {
-    const int sub = warp & 3;
+    const int sub = warp & 3, grp = warp >> 2;
     const int m = sub * 32 + lane;
     const int64_t row = static_cast<int64_t>(mt) * kBM + m;
     const bool row_ok = row < a.M;
     const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[row / kRowsPerBlock])) : 0.0f;
-    const int half_n = a.N / 2;
-    const int n_lo = (warp < 4) ? 0 : half_n, n_hi = (warp < 4) ? half_n : a.N;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
-    if (a.splits == 1) {
-      for (int n0 = n_lo; n0 < n_hi; n0 += 8) {
-        float v[8];
-        tmem_ld8(tmem_d + lane_base + n0, v);
+    float* part = reinterpret_cast<float*>(sm + L.b);  // [N][128]: the x stage ring is free now
+    for (int n0 = 8 * grp; n0 < a.N; n0 += 8 * kDecGroups) {
+      float v[8];
+      tmem_ld8(tmem_d + lane_base + n0, v);
+      if (a.splits == 1) {
         if (row_ok) {
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             a.y[static_cast<int64_t>(n0 + i) * a.M + row] = (nk > 0 && !failed) ? v[i] * scale : 0.0f;
         }
-      }
-    } else {
-      float* part = reinterpret_cast<float*>(sm + L.b);  // [N][128]: the x stage ring is free now
-      for (int n0 = n_lo; n0 < n_hi; n0 += 8) {
-        float v[8];
-        tmem_ld8(tmem_d + lane_base + n0, v);
+      } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i) part[(n0 + i) * kBM + m] = (nk > 0 && !failed) ? v[i] : 0.0f;
       }
@@ -392,18 +411,33 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
 
 constexpr uint32_t kSmemLimit = 227u * 1024u;
 
-// Largest number of tiles whose codes fit next to the stage ring for batch N.
+__host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N) + 2u * 32u <= 256u ? 256u : 512u; }
+
+// Pipeline stages for batch N and tpb tiles per block: as many as tensor
+// memory and shared memory (the B stages next to the staged codes; half of the
+// SM's when two blocks share it) hold, at most kMaxStages; 0 if fewer than 2.
+static int gemm_stages(int N, int tpb) {
+  const uint32_t cols = gemm_tmem_cols(N);
+  const uint32_t smem_cap = cols == 256u ? 233472u / 2u - 1024u : kSmemLimit;
+  int S = static_cast<int>((cols - gemm_a_col(N)) / 32u);
+  if (S > kMaxStages) S = kMaxStages;
+  while (S >= 2 && gemm_layout(N, tpb, S).total + 1024u > smem_cap) --S;
+  return S >= 2 ? S : 0;
+}
+
+// Largest number of tiles per block (codes staged up front) that still leaves
+// a two-stage pipeline for batch N.
 static int gemm_max_tiles(int N) {
   int t = kMaxTiles;
-  while (t > 1 && gemm_layout(N, t).total + 1024u > kSmemLimit) --t;
+  while (t > 1 && gemm_stages(N, t) == 0) --t;
   return t;
 }
 
 // Dynamic shared memory of a launch: the layout, padded so that no more blocks
-// share an SM than its 512 tensor-memory columns can hold (a block waiting in
+// share an SM than its 512 tensor-memory columns hold (a block waiting in
 // tcgen05.alloc for a co-resident block of its own cluster would never proceed).
-static uint32_t gemm_smem_bytes(int N, int tpb) {
-  uint32_t smem = gemm_layout(N, tpb).total + 1024u;  // + alignment slack
+static uint32_t gemm_smem_bytes(int N, int tpb, int S) {
+  const uint32_t smem = gemm_layout(N, tpb, S).total + 1024u;  // + alignment slack
   const uint32_t max_blocks = 512u / gemm_tmem_cols(N);
   const uint32_t floor_bytes = 233472u / (max_blocks + 1u) + 1u - 1024u;  // 228 KiB per SM, 1 KiB reserved per block
   return smem > floor_bytes ? smem : floor_bytes;
@@ -411,18 +445,16 @@ static uint32_t gemm_smem_bytes(int N, int tpb) {
 
 // Blocks along K per 128-row tile: minimise (waves of blocks) x (tiles per
 // block + 1), the +1 standing for a block's fixed cost (prologue, pipeline
-// fill, epilogue and the cluster reduction), subject to the shared-memory
-// bound on tiles per block and clusters of at most 16.
+// fill, epilogue and the cluster reduction), within the shared-memory bound on
+// tiles per block and clusters of at most 16.
 static int gemm_splits(int64_t m_tiles, int T, int N, int sms) {
   const int max_tiles = gemm_max_tiles(N);
+  const int64_t slots = static_cast<int64_t>(sms) * (512 / static_cast<int>(gemm_tmem_cols(N)));
   int best = -1;
   int64_t best_cost = -1;
   for (int s = 1; s <= 16 && s <= T; ++s) {
     const int tpb = (T + s - 1) / s;
     if (tpb > max_tiles) continue;
-    int occ = static_cast<int>(233472u / (gemm_smem_bytes(N, tpb) + 1024u));
-    if (occ < 1) occ = 1;
-    const int64_t slots = static_cast<int64_t>(sms) * occ;
     const int64_t waves = (m_tiles * s + slots - 1) / slots;
     const int64_t cost = waves * (tpb + 1);
     if (best_cost < 0 || cost < best_cost) {
@@ -454,7 +486,9 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.tmem_cols = gemm_tmem_cols(batch);
   a.a_col = gemm_a_col(batch);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
-  const size_t smem = gemm_smem_bytes(batch, tcta_max);
+  a.S = gemm_stages(batch, tcta_max);
+  if (a.S < 2) return cudaErrorInvalidValue;
+  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S);
   // tensor map over x [batch, K] bf16: one 64-column x batch box per chunk, 128-byte swizzle
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
