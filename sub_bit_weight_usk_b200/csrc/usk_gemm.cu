@@ -23,10 +23,14 @@
 //    shared-memory bandwidth to the code gathers and the B (x) operand.
 //  * 1 copy warp: per chunk, as soon as the stage is free, one tensor copy of
 //    the x tile (B operand, 128-byte swizzle) onto the stage's "full" barrier.
-//  * 1 MMA warp: per chunk, once the stage is full, four tcgen05.mma (M=128,
-//    N=batch, K=16, A from tensor memory, B from shared memory, bf16 -> fp32)
-//    and a commit to the stage's "empty" mbarrier.  A ring of stages lets
-//    decode, copy and MMA overlap.
+//  * I = 1, 2 or 4 MMA warps: warp i takes the chunks c = i (mod I); once the
+//    stage is full, four tcgen05.mma (M=128, N=batch, K=16, A from tensor
+//    memory, B from shared memory, bf16 -> fp32) into its own accumulator and
+//    a commit to the stage's "empty" mbarrier.  A tcgen05.mma keeps its issuing
+//    warp busy for about 180 cycles whatever N is (measured on B200), so at
+//    small batches one issuer leaves the tensor core mostly idle; I x N <= 256
+//    issuers fill it.  The epilogue adds the I accumulators in a fixed order.
+//    A ring of stages lets decode, copy and MMA overlap.
 //  * Epilogue: tcgen05.ld of the accumulator, x row-block scale, y.
 //  * Every mbarrier wait is bounded (about 1 s); a wait that gives up sets
 //    USK_FLAG_TIMEOUT, the pipeline stops, one final commit drains the tensor
@@ -40,11 +44,13 @@ namespace cg = cooperative_groups;
 namespace usk {
 
 constexpr int kDecWarps = 16;
-constexpr int kDecGroups = kDecWarps / 4;        // thread groups of 128 (one per row) splitting each chunk
-constexpr int kOctPerThread = 8 / kDecGroups;    // octets of a 64-column chunk per decoder thread
-constexpr int kMmaWarp = kDecWarps;       // lane 0 issues the MMAs; the warp owns TMEM
-constexpr int kCopyWarp = kDecWarps + 1;  // lane 0 copies the x tiles ahead of the MMAs
-constexpr int kGemmThreads = (kDecWarps + 2) * 32;
+constexpr int kDecGroups = kDecWarps / 4;  // groups of 128 threads (one per row); group g decodes chunk g of every tile
+constexpr int kWidenWarp = kDecWarps;      // widens each tile's codes to bf16, up to kTileRing tiles ahead
+constexpr int kCopyWarp = kDecWarps + 1;   // lane 0 copies the x tiles ahead of the MMAs
+constexpr int kMmaWarp0 = kDecWarps + 2;   // first MMA warp; it also owns the TMEM allocation
+constexpr int kMaxIssuers = 4;             // MMA warps: a tcgen05.mma holds its issuing warp ~180 cycles
+constexpr int kGemmThreads = (kDecWarps + 2 + kMaxIssuers) * 32;
+constexpr int kTileRing = 4;               // bf16 tile-code buffers
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
@@ -64,6 +70,7 @@ struct GemmArgs {
   uint32_t tmem_cols;
   uint32_t a_col;  // first tensor-memory column of the A stages
   int S;           // pipeline stages
+  int I;           // MMA issuer warps, each with its own accumulator (columns [i N, (i + 1) N))
   int inject;  // test hook: block (0, 0) skips the x copy of its first chunk
 };
 
@@ -75,20 +82,21 @@ __host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S) {
   GemmLayout L;
   L.b = 0;  // [S][N x 64] bf16, SW128; after the main loop the K-split partials [N][128] fp32
   const uint32_t ring = static_cast<uint32_t>(S) * N * kBK * 2, parts = static_cast<uint32_t>(N) * kBM * 4;
-  L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [2 buffers][2][1024]
-  L.codes = L.cbf + 2u * 2u * 1024u * 2u;                              // int8 [2][tcta][1024]
+  L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [kTileRing][2][1024]
+  L.codes = L.cbf + kTileRing * 2u * 1024u * 2u;                       // int8 [2][tcta][1024]
   L.keys = L.codes + 2u * tcta * 1024u;                                // uint2 [2][tcta]
-  L.bars = (L.keys + 2u * tcta * 8u + 7u) & ~7u;                       // full[S], empty[S], codes, done, tile
-  L.misc = L.bars + (2 * S + 3) * 8;                                   // tmem holder, abort
+  L.bars = (L.keys + 2u * tcta * 8u + 7u) & ~7u;  // full[S], empty[S], codes, done, ready[ring], free[ring]
+  L.misc = L.bars + (2 * S + 2 + 2 * kTileRing) * 8;                   // tmem holder, abort
   L.total = L.misc + 16;
   return L;
 }
 
-// Tensor memory: the fp32 accumulator [0, N), then the A stages, 32 columns
-// (128 rows x 64 bf16) each, from column a_col(N).  A block takes 256 columns
-// (two blocks per SM) when 2 or more stages fit next to the accumulator, else
-// all 512 (one block per SM).
-__host__ __device__ inline uint32_t gemm_a_col(int N) { return (static_cast<uint32_t>(N) + 31u) & ~31u; }
+// Tensor memory: the issuers' fp32 accumulators [0, I N), then the A stages,
+// 32 columns (128 rows x 64 bf16) each, from column a_col(N).
+__host__ __device__ inline int gemm_issuers(int N) { return N <= 64 ? 4 : (N <= 128 ? 2 : 1); }
+__host__ __device__ inline uint32_t gemm_a_col(int N) {
+  return (static_cast<uint32_t>(gemm_issuers(N) * N) + 31u) & ~31u;
+}
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -124,7 +132,7 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// 8 or 16 consecutive 32-bit columns of this thread's tensor-memory lane.
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -132,11 +140,6 @@ __device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[16])
       "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
       "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
-}
-__device__ __forceinline__ void tmem_st(uint32_t taddr, const uint32_t (&v)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(v[0]),
-               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
@@ -164,7 +167,7 @@ __device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w) {
   return *reinterpret_cast<uint32_t*>(&p);
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
+__global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ks = static_cast<int>(cluster.block_rank());
@@ -183,7 +186,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
   const GemmLayout L = gemm_layout(a.N, tcta, S);
   const uint32_t bstage = static_cast<uint32_t>(a.N) * kBK * 2;
   const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * S, codes_bar = empty_s + 8 * S;
-  const uint32_t done_bar = codes_bar + 8, tile_bar = done_bar + 8;
+  const uint32_t done_bar = codes_bar + 8, ready_s = done_bar + 8, free_s = ready_s + 8 * kTileRing;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(sm + L.misc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
@@ -191,15 +194,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
   const int rb0 = 2 * mt;
   const bool second_rb = rb0 + 1 < RB;
 
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     if (lane == 0) {
       for (int s = 0; s < S; ++s) {
-        mbar_init(full_s + 8 * s, kDecThreads + 1);
+        mbar_init(full_s + 8 * s, 128 + 1);  // one decoder group + the x copy
         mbar_init(empty_s + 8 * s, 1);
       }
       mbar_init(codes_bar, 1);
-      mbar_init(done_bar, 1);
-      mbar_init(tile_bar, kDecThreads);
+      mbar_init(done_bar, a.I);
+      for (int q = 0; q < kTileRing; ++q) {
+        mbar_init(ready_s + 8 * q, 32);           // the widen warp
+        mbar_init(free_s + 8 * q, kDecThreads);   // every decoder
+      }
       *abort_flag = 0u;
       mbar_fence_init();
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
@@ -230,77 +236,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
   bool aborted = false;
 
   if (warp < kDecWarps) {
-    // ---------------- decoders
-    const int m = tid & 127;             // row in the 128-row tile
-    const int grp = tid >> 7;            // octets kOctPerThread*grp .. + kOctPerThread - 1 of each chunk
+    // ---------------- decoders: group g = warp / 4 rebuilds chunk g (octets
+    // 8g .. 8g + 7) of every tile, thread = row; the four groups work on
+    // different chunks concurrently
+    const int m = tid & 127;  // row in the 128-row tile
+    const int g = tid >> 7;
     const int rbl = m >> 6;
     const uint32_t r = static_cast<uint32_t>(m & 63);
     const bool row_ok = static_cast<int64_t>(mt) * kBM + m < a.M;
-    // this thread's tensor-memory lane (= its row) and its columns of an A stage
-    const uint32_t a_taddr =
-        tmem_d + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + a.a_col + grp * (4u * kOctPerThread);
-    // widen tile tl's codes (both row blocks) into bf16 buffer tl % 2
-    auto widen = [&](int tl) {
-      constexpr int per = 2048 / kDecThreads;  // codes per thread
-      const int wrb = (tid * per) >> 10, part = (tid * per) & 1023;
-      const uint32_t src = s0 + L.codes + static_cast<uint32_t>(wrb * tcta + tl) * 1024u + part;
-      const uint32_t dst = s0 + L.cbf + (tl & 1) * 4096u + wrb * 2048u + part * 2u;
-      if (per == 8) {
-        const uint2 w = lds64(src);
-        sts128(dst, make_uint4(i8x2_to_bf16x2(w.x), i8x2_to_bf16x2(w.x >> 16), i8x2_to_bf16x2(w.y),
-                               i8x2_to_bf16x2(w.y >> 16)));
-      } else {
-        const uint32_t w = lds32(src);
-        sts64(dst, make_uint2(i8x2_to_bf16x2(w), i8x2_to_bf16x2(w >> 16)));
-      }
-    };
+    // this thread's tensor-memory lane (= its row) in the A stages
+    const uint32_t a_taddr = tmem_d + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + a.a_col;
     // loop exits are warp-uniform: tcgen05.st is a whole-warp instruction
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(codes_bar, 0))) aborted = true;
-    if (!aborted && nk > 0) widen(0);
-    int s = 0;
-    uint32_t ph = 0;  // phase parity of stage s's current use
-    for (int c = 0; c < nk && !aborted; ++c, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
-      const int tl = c >> 2;
-      if ((c & 3) == 0) {
-        // every decoder has finished tile tl - 1 and widened tile tl; buffer
-        // (tl + 1) % 2 is free for tile tl + 1
-        mbar_arrive(tile_bar);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(tile_bar, tl & 1))) {
-          aborted = true;
-          break;
-        }
-        if (tl + 1 < tcta) widen(tl + 1);
+    for (int t = 0; t < tcta && !aborted; ++t) {
+      const int c = 4 * t + g;
+      const int q = t % kTileRing;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(ready_s + 8 * q, static_cast<uint32_t>(t / kTileRing) & 1u))) {
+        aborted = true;
+        break;
       }
+      const int s = c % S;
       if (c >= S) {
         // the MMAs that read this A stage have completed
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_s + 8 * s, ph ^ 1u))) {
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_s + 8 * s, static_cast<uint32_t>(c / S - 1) & 1u))) {
           aborted = true;
           break;
         }
         tc_fence_after();
       }
-      const uint2 hk = keytab[rbl * tcta + tl];
-      const uint32_t ob = static_cast<uint32_t>((c & 3) * 8 + grp * kOctPerThread);
+      const uint2 hk = keytab[rbl * tcta + t];
+      const uint32_t ob = static_cast<uint32_t>(8 * g);
       uint32_t h = hk.x * (32u * r + ob) + hk.y;
-      const uint32_t tile_codes = s0 + L.cbf + (tl & 1) * 4096u + rbl * 2048u;
-      uint32_t v[4 * kOctPerThread];
+      const uint32_t tile_codes = s0 + L.cbf + q * 4096u + rbl * 2048u;
 #pragma unroll
-      for (int j = 0; j < kOctPerThread; ++j) {
-        uint4 q = make_uint4(0u, 0u, 0u, 0u);
-        if (row_ok) {
-          const uint32_t cls = (ob + j + r) & 31u;
-          q = lds128(tile_codes + ((h >> 30) * 32u + cls) * 16u);
+      for (int hh = 0; hh < 2; ++hh) {  // octets 4hh .. 4hh + 3 -> columns 16hh .. 16hh + 15 of the stage
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint4 w = make_uint4(0u, 0u, 0u, 0u);
+          if (row_ok) {
+            const uint32_t cls = (ob + 4u * hh + j + r) & 31u;
+            w = lds128(tile_codes + ((h >> 30) * 32u + cls) * 16u);
+          }
+          v[4 * j + 0] = w.x;
+          v[4 * j + 1] = w.y;
+          v[4 * j + 2] = w.z;
+          v[4 * j + 3] = w.w;
+          h += hk.x;
         }
-        v[4 * j + 0] = q.x;
-        v[4 * j + 1] = q.y;
-        v[4 * j + 2] = q.z;
-        v[4 * j + 3] = q.w;
-        h += hk.x;
+        tmem_st(a_taddr + s * 32u + 16u * hh, v);
       }
-      tmem_st(a_taddr + s * 32u, v);
+      mbar_arrive(free_s + 8 * q);  // this thread is done with the tile's codes
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(full_s + 8 * s);
+    }
+  } else if (warp == kWidenWarp) {
+    // ---------------- tile codes int8 -> bf16 (exact), kTileRing tiles ahead
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(codes_bar, 0))) aborted = true;
+    for (int t = 0; t < tcta && !aborted; ++t) {
+      const int q = t % kTileRing;
+      if (t >= kTileRing &&
+          !__all_sync(0xFFFFFFFFu, mbar_wait(free_s + 8 * q, static_cast<uint32_t>(t / kTileRing - 1) & 1u))) {
+        aborted = true;
+        break;
+      }
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {  // 2 x 1024 codes, 4 per lane per step
+        const uint32_t idx = static_cast<uint32_t>(lane) * 4u + static_cast<uint32_t>(i) * 128u;
+        const uint32_t wrb = idx >> 10, b = idx & 1023u;
+        const uint32_t w = lds32(s0 + L.codes + (wrb * tcta + t) * 1024u + b);
+        sts64(s0 + L.cbf + q * 4096u + wrb * 2048u + 2u * b, make_uint2(i8x2_to_bf16x2(w), i8x2_to_bf16x2(w >> 16)));
+      }
+      mbar_arrive(ready_s + 8 * q);
     }
   } else if (warp == kCopyWarp) {
     // ---------------- x tiles, up to S chunks ahead of the MMAs.  The whole
@@ -319,13 +326,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
       }
       __syncwarp();
     }
-  } else if (warp == kMmaWarp) {
-    // ---------------- MMAs (whole warp in the loop, lane 0 issues)
+  } else if (warp >= kMmaWarp0 && warp < kMmaWarp0 + a.I) {
+    // ---------------- MMAs: warp i takes chunks i, i + I, ... into accumulator i
+    // (whole warp in the loop, lane 0 issues)
+    const int i = warp - kMmaWarp0;
     const uint32_t idesc = idesc_bf16_f32(a.N);
-    int s = 0;
-    uint32_t ph = 0;
-    for (int c = 0; c < nk && !aborted; ++c, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(full_s + 8 * s, ph))) {
+    const uint32_t d_tm = tmem_d + static_cast<uint32_t>(i * a.N);
+    for (int c = i; c < nk && !aborted; c += a.I) {
+      const int s = c % S;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(full_s + 8 * s, static_cast<uint32_t>(c / S) & 1u))) {
         aborted = true;
         break;
       }
@@ -335,18 +344,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
         const uint32_t bst = s0 + L.b + s * bstage;
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
-          mma_bf16_ts(tmem_d, a_tm + 8u * kk, sw128_desc(bst + 32 * kk), idesc, (c > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(d_tm, a_tm + 8u * kk, sw128_desc(bst + 32 * kk), idesc, (c > i || kk > 0) ? 1u : 0u);
         mma_commit(empty_s + 8 * s);
       }
       __syncwarp();
     }
-    // one more commit: tracks every MMA issued above (also after a failed wait)
+    // one more commit per issuer: tracks every MMA it issued (also after a failed wait)
     if (lane == 0) mma_commit(done_bar);
     __syncwarp();
   }
   if (aborted) *abort_flag = 1u;
-  // every thread waits for the tensor core to drain (bounded)
-  if (!mbar_wait(done_bar, 0)) *abort_flag = 1u;
+  // one thread waits (bounded) for the tensor core to drain; the others wait in
+  // the block barrier, which does not poll shared memory
+  if (warp == kMmaWarp0 && lane == 0 && !mbar_wait(done_bar, 0)) *abort_flag = 1u;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -366,6 +376,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
     for (int n0 = 8 * grp; n0 < a.N; n0 += 8 * kDecGroups) {
       float v[8];
       tmem_ld8(tmem_d + lane_base + n0, v);
+      for (int i = 1; i < a.I; ++i) {  // the issuers' accumulators, in order
+        float u[8];
+        tmem_ld8(tmem_d + lane_base + static_cast<uint32_t>(i * a.N) + n0, u);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] += u[e];
+      }
       if (a.splits == 1) {
         if (row_ok) {
 #pragma unroll
@@ -400,7 +416,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kMmaWarp0) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_d), "r"(a.tmem_cols)
                  : "memory");
@@ -411,7 +427,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const GemmArgs a,
 
 constexpr uint32_t kSmemLimit = 227u * 1024u;
 
-__host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N) + 2u * 32u <= 256u ? 256u : 512u; }
+// 256 columns (two blocks per SM) when four stages fit next to the accumulators, else 512
+__host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N) + 4u * 32u <= 256u ? 256u : 512u; }
 
 // Pipeline stages for batch N and tpb tiles per block: as many as tensor
 // memory and shared memory (the B stages next to the staged codes; half of the
@@ -444,9 +461,10 @@ static uint32_t gemm_smem_bytes(int N, int tpb, int S) {
 }
 
 // Blocks along K per 128-row tile: minimise (waves of blocks) x (tiles per
-// block + 1), the +1 standing for a block's fixed cost (prologue, pipeline
-// fill, epilogue and the cluster reduction), within the shared-memory bound on
-// tiles per block and clusters of at most 16.
+// block + 4), the 4 standing for a block's fixed cost in tiles (prologue,
+// pipeline fill, epilogue and the cluster reduction: 4 to 5 us measured against
+// about 1.3 us per tile at batch 16), within the shared-memory bound on tiles
+// per block and clusters of at most 16.
 static int gemm_splits(int64_t m_tiles, int T, int N, int sms) {
   const int max_tiles = gemm_max_tiles(N);
   const int64_t slots = static_cast<int64_t>(sms) * (512 / static_cast<int>(gemm_tmem_cols(N)));
@@ -456,7 +474,7 @@ static int gemm_splits(int64_t m_tiles, int T, int N, int sms) {
     const int tpb = (T + s - 1) / s;
     if (tpb > max_tiles) continue;
     const int64_t waves = (m_tiles * s + slots - 1) / slots;
-    const int64_t cost = waves * (tpb + 1);
+    const int64_t cost = waves * (tpb + 4);
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = s;
@@ -485,6 +503,7 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   if (a.splits < 1) return cudaErrorInvalidValue;  // K beyond 16 blocks x the tiles one block can stage
   a.tmem_cols = gemm_tmem_cols(batch);
   a.a_col = gemm_a_col(batch);
+  a.I = gemm_issuers(batch);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
   a.S = gemm_stages(batch, tcta_max);
   if (a.S < 2) return cudaErrorInvalidValue;
