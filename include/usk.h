@@ -185,10 +185,11 @@ USK_API void usk_debug_set_gemv_path(int path);
 USK_API void usk_debug_set_gemv_rows(int rows);
 
 /* Test hook for the failure path (host-made; no device fault): kernel = 1 makes
- * usk_build, 2 usk_gemm, 3 usk_gemv (integer path) skip one bulk or tensor
- * copy in thread block (0, 0), so that block's bounded wait gives up
- * after about 1 s and sets USK_FLAG_TIMEOUT; the kernel still completes and the
- * context stays usable.  0 switches it off.  Process-wide. */
+ * usk_build, 2 usk_gemm, 3 usk_gemv skip one bulk or tensor copy in thread
+ * block (0, 0) (for the usk_gemv path without copies: the partial sums of
+ * block 1 of row block 0), so a bounded wait gives up after about 1 s and sets
+ * USK_FLAG_TIMEOUT; the kernel still completes and the context stays usable.
+ * 0 switches it off.  Process-wide. */
 USK_API void usk_debug_inject_timeout(int kernel);
 
 /* Static description of a status value. */

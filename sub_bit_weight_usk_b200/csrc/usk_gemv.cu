@@ -293,8 +293,14 @@ cudaError_t launch_gemv_slab(const int8_t* codes, const uint16_t* scales, int64_
                              const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl,
                              cudaStream_t stream, int rows_override, int inject);
 
-// path: 0 = automatic, 1 = bf16 tensor path, 2 = integer path with clusters,
-// 3 = integer row-slab path (bf16 x, batch * K <= 16384)
+bool gemv_bf_supported(int64_t K, int batch, int tpc_override);
+cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                           const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
+                           int tpc_override, int inject);
+
+// path: 0 = automatic, 1 = bf16 tensor path (staged x), 2 = integer path with
+// clusters, 3 = integer row-slab path (bf16 x, batch * K <= 16384), 4 = bf16
+// path with x fragments from global memory (bf16 x, batch <= 8)
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
                         cudaStream_t stream, int tpc_override, int rows_override, int inject) {
@@ -302,6 +308,9 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   // there are more than two row blocks per SM (measured at 28672 x 8192)
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (!xf32 && (path == 0 || path == 4) && gemv_bf_supported(K, batch, tpc_override))
+    return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
+                          tpc_override, inject);
   const bool slab = path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms);
   if (!xf32 && slab && slab_supported(K, batch))
     return launch_gemv_slab(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl,

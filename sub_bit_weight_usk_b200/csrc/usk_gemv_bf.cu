@@ -1,0 +1,315 @@
+// usk_gemv_bf.cu -- y = W_hat x for bf16 x at batch 1..8 with the fewest
+// serial steps: x goes straight from global memory into the tensor-core B
+// fragment, and the blocks of a row block meet only through one-way
+// asynchronous stores into the first block's shared memory.
+//
+// "UltraSketchLLM" explainer, Metodologia §4: decompression is the product
+// W_hat = S . P^T with a one-hot P; every weight (i, j) reads the code of the
+// bucket its index hashes to, rehashed in registers once per octet of 8 columns.
+//
+// Design (B200, sm_100a):
+//  * One thread block per (64-row block, tpc hash tiles); the C blocks of a row
+//    block form a cluster.  The first instructions issue every global load the
+//    block needs: lane (g, t) of warp w loads, for every tile, the 8 bf16 x
+//    values of octet o = (w & 1) + 8 (w >> 1) + 2t of batch row g -- already
+//    the B fragment of two mma.sync m16n8k16 (the reduction index is permuted
+//    the same way for A and B, which the sum does not see) -- and 16 codes per
+//    thread per 16 tiles' worth of codes.  No x staging, no x preparation, no
+//    barrier set-up or bulk-copy issue ahead of the loads (measured: those
+//    cost about 1000 cycles before the first byte moved).
+//  * The codes are widened to bf16 in registers on arrival (exact: |code| <=
+//    127), stored once, and gathered per (row, octet) with one 16-byte shared
+//    load; because class = (o + row) mod 32 and the lanes of a quarter warp
+//    cover rows g, g+1 and octets o0 + 2t, the 8 lanes hit 8 distinct 16-byte
+//    bank groups.  Two accumulator sets (even and odd tiles) double the
+//    independent MMA chains.
+//  * fp32 accumulation of exact bf16 products; the 8 warps' sums are added in
+//    a fixed order, then every block but the first writes its 64 x batch
+//    partials into the first block's shared memory with st.async, which counts
+//    the bytes on the first block's mbarrier; the first block waits only for
+//    those bytes, adds the partials in rank order (deterministic) and scales.
+#include <cooperative_groups.h>
+
+#include "usk_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace usk {
+
+struct GemvBfArgs {
+  const int8_t* codes;
+  const uint16_t* scales;
+  const uint16_t* x;  // bf16 [batch, K]
+  float* y;
+  int64_t M, K;
+  uint64_t seed;
+  uint32_t* status;
+  int T, C, tpc;
+  int pdl;     // launched as a programmatic dependent: wait before reading x
+  int inject;  // test hook: block 1 of row block 0 skips its partial-sum stores
+};
+
+constexpr int kBfThreads = 256;
+constexpr int kBfMaxTiles = 8;  // tiles per block (x fragments live in registers)
+
+struct GemvBfLayout {
+  uint32_t cbf, keys, red, push, bars, total;
+};
+
+__host__ __device__ inline GemvBfLayout gemv_bf_layout(int tpc, int batch, int C) {
+  GemvBfLayout L;
+  L.cbf = 0;                                                       // bf16 [tpc][1024]
+  L.keys = L.cbf + static_cast<uint32_t>(tpc) * 2048u;             // uint2 [tpc]
+  L.red = (L.keys + static_cast<uint32_t>(tpc) * 8u + 15u) & ~15u;  // fp32 [8 warps][batch][64]
+  L.push = L.red + 8u * batch * 64u * 4u;                          // fp32 [C][batch][64] (used in rank 0)
+  L.bars = (L.push + static_cast<uint32_t>(C) * batch * 64u * 4u + 7u) & ~7u;  // push
+  L.total = L.bars + 8u;
+  return L;
+}
+
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// remote 4-byte store into a peer block's shared memory, completing `4` bytes
+// of the transaction count of the peer's mbarrier
+__device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+
+// bytes 0 and 1 of w (int8 codes) -> one bf16 pair, exact (|code| <= 127)
+__device__ __forceinline__ uint32_t pack_i8x2_bf16(uint32_t w) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(static_cast<float>(static_cast<int8_t>(w & 0xFFu)),
+                                           static_cast<float>(static_cast<int8_t>((w >> 8) & 0xFFu)));
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+template <int B>
+__global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int rb = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t0 = crank * a.tpc;
+  const int nt = min(a.tpc, a.T - t0);
+  const GemvBfLayout L = gemv_bf_layout(a.tpc, B, a.C);
+  const uint32_t s0 = smem_u32(sm);
+  const uint32_t push_bar = s0 + L.bars;
+  uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
+  float* red = reinterpret_cast<float*>(sm + L.red);
+  float* push = reinterpret_cast<float*>(sm + L.push);
+  constexpr uint32_t kPartBytes = static_cast<uint32_t>(B) * 64u * 4u;
+  constexpr int kCodeLoads = kBfMaxTiles * 1024 / 16 / kBfThreads;  // 16-byte code loads per thread (at most)
+
+  if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+  // ---- every global load first: x B fragments and the codes
+  const int g = lane >> 2, t = lane & 3;
+  const int o = (warp & 1) + 8 * (warp >> 1) + 2 * t;  // this lane's octet in every tile
+  uint4 xv[kBfMaxTiles];
+#pragma unroll
+  for (int tt = 0; tt < kBfMaxTiles; ++tt) {
+    xv[tt] = make_uint4(0u, 0u, 0u, 0u);
+    if (tt < nt && g < B)
+      xv[tt] = ldg_nc128(a.x + static_cast<int64_t>(g) * a.K + static_cast<int64_t>(t0 + tt) * kTileCols + 8 * o);
+  }
+  const int8_t* codes_blk = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
+  uint4 cv[kCodeLoads];
+#pragma unroll
+  for (int u = 0; u < kCodeLoads; ++u) {
+    const int q = tid + u * kBfThreads;  // 16-code chunk
+    cv[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (q < nt * 64) cv[u] = ldg_nc128(codes_blk + 16 * q);
+  }
+  if (tid == 0 && a.C > 1) {
+    mbar_init(push_bar, 1);
+    mbar_fence_init();
+    if (crank == 0) mbar_arrive_expect_tx(push_bar, static_cast<uint32_t>(a.C - 1) * kPartBytes);
+  }
+  // first half of a split cluster barrier; its wait, before the first remote
+  // store, guarantees that the first block's push barrier is initialised and
+  // armed (the init is published by its cluster-scope fence).  Relaxed: a
+  // release arrive would first wait for this thread's loads in flight.
+  if (a.C > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
+
+  // ---- codes: widen to bf16 once
+#pragma unroll
+  for (int u = 0; u < kCodeLoads; ++u) {
+    const int q = tid + u * kBfThreads;
+    if (q < nt * 64) {
+      const uint32_t ws[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
+      uint32_t o8[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        o8[2 * e] = pack_i8x2_bf16(ws[e]);
+        o8[2 * e + 1] = pack_i8x2_bf16(ws[e] >> 16);
+      }
+      sts128(s0 + L.cbf + 32u * q, make_uint4(o8[0], o8[1], o8[2], o8[3]));
+      sts128(s0 + L.cbf + 32u * q + 16u, make_uint4(o8[4], o8[5], o8[6], o8[7]));
+    }
+  }
+  __syncthreads();
+  // blocks other than the first: the first block's push barrier is ready (this
+  // wait overlaps nothing on their own path but is far from their tail)
+  if (a.C > 1 && crank != 0) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+
+  // ---- main loop: per tile and 16-row group, two MMAs (columns 0-3, 4-7 of
+  // the octet); even and odd tiles accumulate into separate sets
+  float d[2][4][4];
+#pragma unroll
+  for (int st = 0; st < 2; ++st)
+#pragma unroll
+    for (int mb = 0; mb < 4; ++mb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) d[st][mb][e] = 0.0f;
+#pragma unroll
+  for (int tt = 0; tt < kBfMaxTiles; ++tt) {
+    if (tt < nt) {
+      const uint2 hk = keytab[tt];
+      const uint32_t tile_s = s0 + L.cbf + tt * 2048u;
+      const uint32_t h = hk.x * (32u * g + o) + hk.y;
+#pragma unroll
+      for (int mb = 0; mb < 4; ++mb) {
+        const uint32_t h0 = h + static_cast<uint32_t>(mb) * 512u * hk.x;  // row 16 mb + g
+        const uint32_t h1 = h0 + 256u * hk.x;                              // row 16 mb + g + 8
+        const uint32_t c0 = (static_cast<uint32_t>(o + g) + 16u * mb) & 31u;
+        const uint4 q0 = lds128(tile_s + ((h0 >> 30) * 32u + c0) * 16u);
+        const uint4 q1 = lds128(tile_s + ((h1 >> 30) * 32u + ((c0 + 8u) & 31u)) * 16u);
+        mma_bf16_16816(d[tt & 1][mb], q0.x, q1.x, q0.y, q1.y, xv[tt].x, xv[tt].y);
+        mma_bf16_16816(d[tt & 1][mb], q0.z, q1.z, q0.w, q1.w, xv[tt].z, xv[tt].w);
+      }
+    }
+  }
+  // dependents may start launching now: their code prefetch overlaps this epilogue
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  // ---- block sums: lane (g, t) holds rows 16 mb + g (+8) of batch rows 2t, 2t + 1
+#pragma unroll
+  for (int mb = 0; mb < 4; ++mb) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int bi = 2 * t + (e & 1);
+      const int r = 16 * mb + g + 8 * (e >> 1);
+      if (bi < B) red[(warp * B + bi) * 64 + r] = d[0][mb][e] + d[1][mb][e];
+    }
+  }
+  __syncthreads();
+  // (batch row, row) pairs q = bi * 64 + r, kQ per thread
+  constexpr int kQ = (B * 64 + kBfThreads - 1) / kBfThreads;
+  float part[kQ];
+#pragma unroll
+  for (int k = 0; k < kQ; ++k) {
+    const int q = tid + k * kBfThreads;
+    part[k] = 0.0f;
+    if (q < B * 64) {
+#pragma unroll
+      for (int w = 0; w < 8; ++w) part[k] += red[w * B * 64 + q];
+    }
+  }
+  const float s = __half2float(__ushort_as_half(a.scales[rb]));
+  float* yrb = a.y + static_cast<int64_t>(rb) * 64;
+  if (a.C == 1) {
+#pragma unroll
+    for (int k = 0; k < kQ; ++k) {
+      const int q = tid + k * kBfThreads;
+      if (q < B * 64) yrb[static_cast<int64_t>(q / 64) * a.M + q % 64] = part[k] * s;
+    }
+    return;
+  }
+  if (crank != 0) {
+    if (a.inject && crank == 1 && rb == 0) return;  // test hook: the first block's wait gives up
+    const uint32_t bar0 = mapa_shared(push_bar, 0);
+#pragma unroll
+    for (int k = 0; k < kQ; ++k) {
+      const int q = tid + k * kBfThreads;
+      if (q < B * 64)
+        st_async_f32(mapa_shared(s0 + L.push + (static_cast<uint32_t>(crank) * B * 64u + q) * 4u, 0), part[k], bar0);
+    }
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < kQ; ++k) {
+    const int q = tid + k * kBfThreads;
+    if (q < B * 64) push[q] = part[k];
+  }
+  if (!mbar_wait(push_bar, 0)) report(a.status, USK_FLAG_TIMEOUT);  // bounded (about 1 s)
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kQ; ++k) {
+    const int q = tid + k * kBfThreads;
+    if (q < B * 64) {
+      float tot = 0.0f;
+      for (int c = 0; c < a.C; ++c) tot += push[c * B * 64 + q];
+      yrb[static_cast<int64_t>(q / 64) * a.M + q % 64] = tot * s;
+    }
+  }
+}
+
+template <int B>
+static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
+  const size_t smem = gemv_bf_layout(a.tpc, B, a.C).total;
+  auto kern = gemv_bf_kernel<B>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  if (a.C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.blockDim = dim3(kBfThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// Tiles per block: tpc_override if given, else the fewest tiles per block
+// (most blocks) that keeps the cluster within 16 blocks, at least 4.
+bool gemv_bf_supported(int64_t K, int batch, int tpc_override) {
+  const int T = static_cast<int>(K / kTileCols);
+  int tpc = tpc_override > 0 ? tpc_override : 4;
+  while ((T + tpc - 1) / tpc > 16) ++tpc;
+  return batch >= 1 && batch <= 8 && T >= 1 && tpc <= kBfMaxTiles;
+}
+
+cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                           const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
+                           int tpc_override, int inject) {
+  GemvBfArgs a;
+  a.codes = codes; a.scales = scales; a.x = x; a.y = y;
+  a.M = M; a.K = K; a.seed = seed; a.status = status;
+  a.T = static_cast<int>(K / kTileCols);
+  a.tpc = tpc_override > 0 ? tpc_override : 4;
+  if (a.tpc > a.T) a.tpc = a.T;
+  while ((a.T + a.tpc - 1) / a.tpc > 16) ++a.tpc;
+  a.C = (a.T + a.tpc - 1) / a.tpc;
+  a.pdl = pdl ? 1 : 0;
+  a.inject = inject;
+  const int64_t RB = M / kRowsPerBlock;
+  switch (batch) {
+    case 1: return launch_bf_t<1>(a, RB, stream);
+    case 2: return launch_bf_t<2>(a, RB, stream);
+    case 3: return launch_bf_t<3>(a, RB, stream);
+    case 4: return launch_bf_t<4>(a, RB, stream);
+    case 5: return launch_bf_t<5>(a, RB, stream);
+    case 6: return launch_bf_t<6>(a, RB, stream);
+    case 7: return launch_bf_t<7>(a, RB, stream);
+    default: return launch_bf_t<8>(a, RB, stream);
+  }
+}
+
+}  // namespace usk

@@ -125,7 +125,7 @@ def test_gemv_edges_and_errors():
 # ------------------------------------------------------------- integer path (bf16 x, batch <= 4)
 
 @pytest.mark.parametrize("batch", [1, 2, 3, 4])
-@pytest.mark.parametrize("path", [1, 2, 3])
+@pytest.mark.parametrize("path", [1, 2, 3, 4])
 def test_gemv_paths_match_oracle(batch, path):
     W = gen.weights_student_t(192, 2816, 7, 4.0, 0.02, 0.001, 20.0, "bf16")
     sk, o = _sketch(W, gen.importance_lognormal(2816, 7), 19)
@@ -147,6 +147,33 @@ def _int_path(sk, x, pdl=False, path=2):
         return usk.usk_gemv(sk, to_dev(x), pdl=pdl).cpu().numpy()
     finally:
         usk.usk_debug_set_gemv_path(0)
+
+
+# ------------------------------------------------------------- bf16 path with x fragments from global memory
+
+@pytest.mark.parametrize("tpc", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("M,K,batch", [(64, 256, 1), (192, 2816, 5), (128, 4352, 8), (320, 11008, 2)])
+def test_gemv_direct_x_path_geometries(tpc, M, K, batch):
+    """Tiles per block 1..8 (clusters of 1 to 16 blocks, ragged last block),
+    every batch width of the path."""
+    W = gen.weights_student_t(M, K, 31, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _sketch(W, None, 32)
+    x = gen.activations(batch, K, 33, "bf16")
+    usk.usk_debug_set_geometry(0, tpc)
+    try:
+        y = _int_path(sk, x, path=4)
+    finally:
+        usk.usk_debug_set_geometry(0, 0)
+    assert rel_err(y, oracle.gemv_f64(o["codes"], o["scales"], M, K, x, 32)) <= TOL
+
+
+def test_gemv_direct_x_path_nonfinite_x_propagates():
+    W = gen.weights_normal(64, 512, 10, 0.02, "bf16")
+    sk, o = _sketch(W, None, 2)
+    x = gen.activations(1, 512, 5, "bf16")
+    x[0, 100] = 0x7FC0  # NaN
+    y = _int_path(sk, x, path=4)
+    assert np.all(np.isnan(y))
 
 
 # ------------------------------------------------------------- row-slab path (batch * K <= 16384)
