@@ -299,7 +299,9 @@ def run_usk(args):
         usk.usk_build(Ws[i % N_WCOPIES], imp, seed, codes=b.codes, scales=b.scales, status=status)
 
     def gemv(i):
-        usk.usk_gemv(sks[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1)
+        # consecutive decode calls: each launches as a programmatic dependent of
+        # the previous one (its set-up overlaps the previous call's tail)
+        usk.usk_gemv(sks[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1, pdl=True)
 
     def gemm(i):
         usk.usk_gemm(sks[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
@@ -416,6 +418,7 @@ def run_usk(args):
         "config": {"workload": WORKLOAD, "M": M, "K": K, "gemv_batch": GEMV_BATCH, "gemm_batch": GEMM_BATCH,
                    "timing": "K steps run phase by phase (K builds, K GEMVs, K GEMMs) as CUDA graphs; "
                              "kernel time = phase event time / K",
+                   "gemv_launch": "programmatic dependent launch (USK_GEMV_PDL) between consecutive GEMV calls",
                    "l2": "inputs larger than L2: builds cycle over %d weight copies (%d MiB), decodes over %d "
                          "sketch copies (%d MiB)" % (N_WCOPIES, N_WCOPIES * 32, N_SKETCHES, N_SKETCHES),
                    "parallelism": "replicas" if world > 1 else "single"},
