@@ -94,11 +94,32 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   if (tid == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
 
-  // ---- init: barriers, winner words of both slots, keys of both slots
+  // importance of this lane's 8 columns, one tile ahead (the loads of tile 0
+  // go out before the weight copies fill the memory queues)
+  uint4 ipre0 = make_uint4(0u, 0u, 0u, 0u), ipre1 = ipre0;
+  auto load_imp = [&](int i) {
+    if (HAS_IMP && i < nt) {
+      const int64_t col0 = static_cast<int64_t>(crank + a.C * i) * kTileCols + lane * 8;
+      ipre0 = ldg_nc128(a.imp + col0);
+      ipre1 = ldg_nc128(a.imp + col0 + 4);
+    }
+  };
+  load_imp(0);
+  auto issue = [&](int i) {  // one tensor copy of tile i of this block into buffer i % nbuf
+    const int tc = crank + a.C * i;
+    const int buf = i % a.nbuf;
+    const uint32_t bar = s0 + L.bars + 8 * buf;
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    tma_load_2d(s0 + L.wbuf + buf * kTileBytes, &wmap, tc * kTileCols, rb * kRowsPerBlock, bar);
+  };
+  // ---- init: the first tile copies go out first, then the winner and key
+  // words of both slots are cleared while the weights stream in
   if (tid == 0) {
     for (int b = 0; b < a.nbuf; ++b) mbar_init(s0 + L.bars + 8 * b, 1);
     mbar_fence_init();
     misc[0] = 0u;
+    for (int i = 0; i < a.nbuf && i < nt; ++i)
+      if (!(a.inject && i == 0 && crank == 0 && rb == 0)) issue(i);
   }
   {
     uint32_t* win32 = reinterpret_cast<uint32_t*>(smraw + L.win);
@@ -111,17 +132,6 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   }
   __syncthreads();
 
-  auto issue = [&](int i) {  // one tensor copy of tile i of this block into buffer i % nbuf
-    const int tc = crank + a.C * i;
-    const int buf = i % a.nbuf;
-    const uint32_t bar = s0 + L.bars + 8 * buf;
-    mbar_arrive_expect_tx(bar, kTileBytes);
-    tma_load_2d(s0 + L.wbuf + buf * kTileBytes, &wmap, tc * kTileCols, rb * kRowsPerBlock, bar);
-  };
-  if (tid == 0)
-    for (int i = 0; i < a.nbuf && i < nt; ++i)
-      if (!(a.inject && i == 0 && crank == 0 && rb == 0)) issue(i);
-
   uint32_t flags = 0;
   uint32_t vmax = 0;  // max |v| bits over the winners this thread converts
   using ValT = typename std::conditional<BF16, uint16_t, uint32_t>::type;
@@ -133,14 +143,13 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
     const uint2 hk = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + tc);
     float imp[8];
     if (HAS_IMP) {
-      const int64_t col0 = static_cast<int64_t>(tc) * kTileCols + lane * 8;
-      const uint4 i0 = ldg_nc128(a.imp + col0), i1 = ldg_nc128(a.imp + col0 + 4);
-      const uint32_t ib[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+      const uint32_t ib[8] = {ipre0.x, ipre0.y, ipre0.z, ipre0.w, ipre1.x, ipre1.y, ipre1.z, ipre1.w};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
         if ((ib[s] >> 31) || (ib[s] & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_BAD_IMPORTANCE;
         imp[s] = __uint_as_float(ib[s]);
       }
+      load_imp(i + 1);
     }
     if (!mbar_wait(s0 + L.bars + 8 * buf, (i / a.nbuf) & 1)) flags |= USK_FLAG_TIMEOUT;
 
@@ -148,66 +157,38 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
     const uint32_t win_s = s0 + L.win + (i & 1) * kWinBytes;
     const uint32_t keys_s = s0 + L.keys + (i & 1) * 4096u;
 
-    // pass 1 (and the only pass for bf16 with unit importance)
-#pragma unroll 2
-    for (int q = 0; q < 8; ++q) {
-      const uint32_t r = warp + 8 * q;
-      const uint32_t h = hk.x * (32u * r + lane) + hk.y;
-      const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
-      const uint32_t l0 = r * kTileCols + lane * 8;
-      if (BF16) {
-        const uint4 v = lds128(wt + r * kRowBytes + lane * 16);
-        const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    if (BF16 && HAS_IMP) {
+      // pass 1: key maxima; the tile's weight words stay in registers for pass 2,
+      // and a per-word test flags Inf/NaN weights exactly (exponent field all
+      // ones <=> (bits & 0x7F80) + 0x80 reaches 0x8000, per half word)
+      uint4 wq[8];
+      uint32_t nf = 0u;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t r = warp + 8 * q;
+        const uint32_t h = hk.x * (32u * r + lane) + hk.y;
+        const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+        wq[q] = lds128(wt + r * kRowBytes + lane * 16);
+        const uint32_t wv[4] = {wq[q].x, wq[q].y, wq[q].z, wq[q].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) nf |= (wv[e] & 0x7F807F80u) + 0x00800080u;
         static_for<8>([&](auto S) {
           constexpr int s = decltype(S)::value;
-          const uint32_t b16 = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
-          if (kSingle) {
-            const uint32_t p = ((b16 & 0x7FFFu) << 16) | ((16384u - (l0 + s)) << 1) | (b16 >> 15);
-            atoms_max_u32_off<128 * s>(win_s + off, p);
-          } else {
-            const float k = fabsf(__uint_as_float(b16 << 16)) * imp[s];
-            atoms_max_u32_off<128 * s>(keys_s + off, __float_as_uint(k));
-          }
-        });
-      } else {
-        const uint4 v0 = lds128(wt + r * kRowBytes + lane * 32), v1 = lds128(wt + r * kRowBytes + lane * 32 + 16);
-        const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-        static_for<8>([&](auto S) {
-          constexpr int s = decltype(S)::value;
-          const float f = __uint_as_float(wv[s]);
-          const float k = HAS_IMP ? fabsf(f) * imp[s] : fabsf(f);
-          atoms_max_u32_off<128 * s>(keys_s + off, __float_as_uint(k));
+          const float f = (s & 1) ? __uint_as_float(wv[s >> 1] & 0xFFFF0000u) : __uint_as_float(wv[s >> 1] << 16);
+          atoms_max_u32_off<128 * s>(keys_s + off, __float_as_uint(fabsf(f) * imp[s]));
         });
       }
-    }
-
-    if (!kSingle) {
+      if (nf & 0x80008000u) flags |= USK_FLAG_NONFINITE_W;
       __syncthreads();
-      // Non-finite screen: a NaN or Inf weight forces a key >= +Inf bits in
-      // its bucket; an fp32 overflow of |w| * importance can too, so the exact
-      // per-weight check runs only when the screen fires (rare).
-      bool screen;
-      {
-        const uint4 mx = lds128(keys_s + 16u * tid);
-        screen = __syncthreads_or(max(max(mx.x, mx.y), max(mx.z, mx.w)) >= 0x7F800000u) != 0;
-      }
       // pass 2: members whose key equals the bucket maximum keep the smallest
       // index and its value (predicated reductions, no divergent branches)
-#pragma unroll 2
+#pragma unroll
       for (int q = 0; q < 8; ++q) {
         const uint32_t r = warp + 8 * q;
         const uint32_t h = hk.x * (32u * r + lane) + hk.y;
         const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
         const uint32_t l0 = r * kTileCols + lane * 8;
-        uint32_t wv[8];
-        if (BF16) {
-          const uint4 v = lds128(wt + r * kRowBytes + lane * 16);
-          wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
-          wv[4] = wv[5] = wv[6] = wv[7] = 0u;
-        } else {
-          const uint4 v0 = lds128(wt + r * kRowBytes + lane * 32), v1 = lds128(wt + r * kRowBytes + lane * 32 + 16);
-          wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w; wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
-        }
+        const uint32_t wv[4] = {wq[q].x, wq[q].y, wq[q].z, wq[q].w};
         uint32_t kmax[8];
         static_for<8>([&](auto S) {
           constexpr int s = decltype(S)::value;
@@ -215,15 +196,89 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
         });
         static_for<8>([&](auto S) {
           constexpr int s = decltype(S)::value;
-          uint32_t bits;
-          if (BF16) bits = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
-          else bits = wv[s];
-          const float f = BF16 ? __uint_as_float(bits << 16) : __uint_as_float(bits);
-          const uint32_t k = __float_as_uint(HAS_IMP ? fabsf(f) * imp[s] : fabsf(f));
-          if (BF16) atoms_min_u32_off_if_eq<128 * s>(win_s + off, ((l0 + s) << 16) | bits, k, kmax[s]);
-          else atoms_min_u64_off_if_eq<256 * s>(win_s + 2 * off, (static_cast<uint64_t>(l0 + s) << 32) | bits, k, kmax[s]);
-          if (screen && (__float_as_uint(f) & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
+          const uint32_t bits = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
+          const uint32_t k = __float_as_uint(fabsf(__uint_as_float(bits << 16)) * imp[s]);
+          atoms_min_u32_off_if_eq<128 * s>(win_s + off, ((l0 + s) << 16) | bits, k, kmax[s]);
         });
+      }
+    } else {
+      // pass 1 (and the only pass for bf16 with unit importance)
+  #pragma unroll 2
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t r = warp + 8 * q;
+        const uint32_t h = hk.x * (32u * r + lane) + hk.y;
+        const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+        const uint32_t l0 = r * kTileCols + lane * 8;
+        if (BF16) {
+          const uint4 v = lds128(wt + r * kRowBytes + lane * 16);
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          static_for<8>([&](auto S) {
+            constexpr int s = decltype(S)::value;
+            const uint32_t b16 = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
+            if (kSingle) {
+              const uint32_t p = ((b16 & 0x7FFFu) << 16) | ((16384u - (l0 + s)) << 1) | (b16 >> 15);
+              atoms_max_u32_off<128 * s>(win_s + off, p);
+            } else {
+              const float k = fabsf(__uint_as_float(b16 << 16)) * imp[s];
+              atoms_max_u32_off<128 * s>(keys_s + off, __float_as_uint(k));
+            }
+          });
+        } else {
+          const uint4 v0 = lds128(wt + r * kRowBytes + lane * 32), v1 = lds128(wt + r * kRowBytes + lane * 32 + 16);
+          const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          static_for<8>([&](auto S) {
+            constexpr int s = decltype(S)::value;
+            const float f = __uint_as_float(wv[s]);
+            const float k = HAS_IMP ? fabsf(f) * imp[s] : fabsf(f);
+            atoms_max_u32_off<128 * s>(keys_s + off, __float_as_uint(k));
+          });
+        }
+      }
+
+      if (!kSingle) {
+        __syncthreads();
+        // Non-finite screen: a NaN or Inf weight forces a key >= +Inf bits in
+        // its bucket; an fp32 overflow of |w| * importance can too, so the exact
+        // per-weight check runs only when the screen fires (rare).
+        bool screen;
+        {
+          const uint4 mx = lds128(keys_s + 16u * tid);
+          screen = __syncthreads_or(max(max(mx.x, mx.y), max(mx.z, mx.w)) >= 0x7F800000u) != 0;
+        }
+        // pass 2: members whose key equals the bucket maximum keep the smallest
+        // index and its value (predicated reductions, no divergent branches)
+  #pragma unroll 2
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t r = warp + 8 * q;
+          const uint32_t h = hk.x * (32u * r + lane) + hk.y;
+          const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+          const uint32_t l0 = r * kTileCols + lane * 8;
+          uint32_t wv[8];
+          if (BF16) {
+            const uint4 v = lds128(wt + r * kRowBytes + lane * 16);
+            wv[0] = v.x; wv[1] = v.y; wv[2] = v.z; wv[3] = v.w;
+            wv[4] = wv[5] = wv[6] = wv[7] = 0u;
+          } else {
+            const uint4 v0 = lds128(wt + r * kRowBytes + lane * 32), v1 = lds128(wt + r * kRowBytes + lane * 32 + 16);
+            wv[0] = v0.x; wv[1] = v0.y; wv[2] = v0.z; wv[3] = v0.w; wv[4] = v1.x; wv[5] = v1.y; wv[6] = v1.z; wv[7] = v1.w;
+          }
+          uint32_t kmax[8];
+          static_for<8>([&](auto S) {
+            constexpr int s = decltype(S)::value;
+            kmax[s] = lds32_off<128 * s>(keys_s + off);
+          });
+          static_for<8>([&](auto S) {
+            constexpr int s = decltype(S)::value;
+            uint32_t bits;
+            if (BF16) bits = (s & 1) ? (wv[s >> 1] >> 16) : (wv[s >> 1] & 0xFFFFu);
+            else bits = wv[s];
+            const float f = BF16 ? __uint_as_float(bits << 16) : __uint_as_float(bits);
+            const uint32_t k = __float_as_uint(HAS_IMP ? fabsf(f) * imp[s] : fabsf(f));
+            if (BF16) atoms_min_u32_off_if_eq<128 * s>(win_s + off, ((l0 + s) << 16) | bits, k, kmax[s]);
+            else atoms_min_u64_off_if_eq<256 * s>(win_s + 2 * off, (static_cast<uint64_t>(l0 + s) << 32) | bits, k, kmax[s]);
+            if (screen && (__float_as_uint(f) & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
+          });
+        }
       }
     }
     __syncthreads();  // tile i resolved; its weight buffer is free
@@ -238,7 +293,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
       uint32_t* k32 = reinterpret_cast<uint32_t*>(smraw + L.keys + (i & 1) * 4096u);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int kidx = tid * 4 + e;
+        const int kidx = tid + kBuildThreads * e;  // consecutive lanes, consecutive words: no bank conflicts
         uint32_t vb, mag;
         if (kSingle) {
           const uint32_t p = win32[kidx];

@@ -74,6 +74,26 @@ def test_build_special_cases():
     assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
 
 
+@pytest.mark.parametrize("scale_exp", [-6, -14, 3])
+def test_build_half_way_quotients_round_to_even(scale_exp):
+    """Winners at exact half-integer multiples of the scale: the quantizer must
+    round those ties to even, as rint of the IEEE quotient does.  Scales 2^-6,
+    2^-14 (the smallest normal binary16) and 2^3."""
+    g = np.random.default_rng(77 + scale_exp)
+    s = 2.0 ** scale_exp
+    M, K = 128, 1024
+    n = g.integers(0, 127, size=(M, K))
+    w = ((2 * n + 1) / 2.0) * s * np.where(g.random((M, K)) < 0.5, -1.0, 1.0)
+    w[::64, 0] = 127.0 * s  # each row block's maximum: s16 = s exactly
+    W = gen.f32_to_bf16_bits(w.astype(np.float32))
+    assert np.array_equal(gen.bf16_bits_to_f32(W), w.astype(np.float32))  # every value exact in bf16
+    o = oracle.build_sketch(W, None, 5, want_winners=True)
+    assert np.all(o["scales"] == np.float16(s).view(np.uint16))
+    ties = np.abs(o["value"]) / np.float32(s)
+    assert np.count_nonzero(ties != np.round(ties)) > 1000  # plenty of half-way quotients
+    _compare(W, None, 5)
+
+
 def test_build_row_stride():
     W = gen.weights_normal(128, 768, 7, 0.02, "bf16")
     big = np.zeros((128, 1024), np.uint16)
