@@ -304,17 +304,21 @@ cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t 
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
                         cudaStream_t stream, int tpc_override, int rows_override, int inject) {
-  // the row-slab kernel pays its x preparation once per block: it wins once
-  // there are more than two row blocks per SM (measured at 28672 x 8192)
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (!xf32 && (path == 0 || path == 4) && gemv_bf_supported(K, batch, tpc_override))
-    return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
-                          tpc_override, inject);
+  // automatic choice (measured on B200, graphs of back-to-back calls):
+  //  * tall matrices (more than two row blocks per SM): integer row slabs;
+  //  * batch >= 2, or batch 1 up to 4096 x 4096: bf16 with direct x fragments;
+  //  * batch 1 with longer K or taller M: the integer cluster kernel (half the
+  //    shared-memory gather bytes; its x preparation is amortised over more tiles)
   const bool slab = path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms);
   if (!xf32 && slab && slab_supported(K, batch))
     return launch_gemv_slab(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl,
                             stream, rows_override, inject);
+  const bool direct = path == 4 || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
+  if (!xf32 && direct && gemv_bf_supported(K, batch, tpc_override))
+    return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
+                          tpc_override, inject);
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
   const bool i8_ok = !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
   if (i8_ok && path != 1)

@@ -17,11 +17,16 @@
 //    class = (octet + row) mod 32) with the digit planes (B fragment: one
 //    8-byte load), accumulating each plane in int32 (no overflow: |sum| <
 //    K_block * 127 * 128);
-//  * the four plane sums are recombined in float64 (exact) and scaled, the
-//    blocks of a row block add their float64 partials through distributed
-//    shared memory in rank order, and y = float(sum * scale).
-// Shared-memory traffic is one byte per weight (the bucket code), half of the
-// bf16 path's.
+//  * the four plane sums are recombined in 64-bit integers and the 8 warps
+//    added (exact), scaled to float64, and the blocks of a row block send
+//    their float64 partials into the first block's shared memory with
+//    st.async (counted on its mbarrier); the first block adds them in rank
+//    order and writes y = float(sum * scale).
+// Shared-memory traffic of the gathers is one byte per weight (the bucket
+// code), half of the bf16 path's.  Start-up follows the measured costs: every
+// global load is issued first (codes with plain 16-byte loads, no bulk copy or
+// barrier set-up ahead of them), no integer division in the x indexing, and a
+// relaxed cluster arrive (a release arrive waits for the loads in flight).
 #include <cooperative_groups.h>
 
 #include "usk_common.cuh"
@@ -40,36 +45,57 @@ struct GemvI8Args {
   uint32_t* status;
   int T, C, tpc, batch;
   int pdl;     // launched as a programmatic dependent: wait before reading x
-  int inject;  // test hook: block (0, 0) skips its code copy
+  int inject;  // test hook: block 1 of row block 0 skips its partial sums
 };
 
 constexpr int kI8Threads = 256;
-constexpr int kI8MaxChunks = 2048;  // 4-element x chunks per block: batch * tiles per block * 64 <= this
-constexpr int kI8MaxCluster = 8;
+constexpr int kI8MaxTiles = 32;                                     // tiles per block
+constexpr int kI8CodeLoads = kI8MaxTiles * 1024 / 16 / kI8Threads;  // 16-byte code loads per thread
+constexpr int kI8MaxChunks = 2048;                                  // 4-element x chunks: batch * tpc * 64
+constexpr int kI8XR = kI8MaxChunks / kI8Threads;                    // x chunks per thread
 
 struct GemvI8Layout {
-  uint32_t codes, keys, xs, pitch, mask, emax, bar, acc, push, total;
+  uint32_t codes, keys, xs, pitch, mask, emax, acc, push, bar, total;
 };
 
-__host__ __device__ inline GemvI8Layout gemv_i8_layout(int tpc, int batch) {
+__host__ __device__ inline GemvI8Layout gemv_i8_layout(int tpc, int batch, int C) {
   GemvI8Layout L;
   L.codes = 0;                                                 // int8 [tpc][1024]
   L.keys = static_cast<uint32_t>(tpc) * 1024u;                 // uint2 [tpc]
   L.xs = (L.keys + static_cast<uint32_t>(tpc) * 8u + 15u) & ~15u;
   L.pitch = static_cast<uint32_t>(tpc) * 256u + 8u;            // int8 plane row (+8: conflict-free)
   L.mask = (L.xs + 4u * batch * L.pitch + 15u) & ~15u;         // u32 [batch][tpc * 8] residual bits
-  L.emax = L.mask + static_cast<uint32_t>(batch) * tpc * 32u;  // u32 [4] max exponent, [4] any-residual
-  L.bar = (L.emax + 32u + 7u) & ~7u;                           // mbarrier
-  L.acc = (L.bar + 8u + 15u) & ~15u;                           // s64 [8 warps][64][batch] plane-combined sums
-  L.push = L.acc + 8u * 64u * batch * 8u;                      // f64 [cluster][batch][64] (used in rank 0)
-  L.total = L.push + kI8MaxCluster * 64u * batch * 8u;
+  L.emax = L.mask + static_cast<uint32_t>(batch) * tpc * 32u;  // u32 [8]: exponents, any-residual
+  L.acc = (L.emax + 32u + 15u) & ~15u;                         // s64 [8 warps][64][batch]
+  L.push = L.acc + 8u * 64u * batch * 8u;                      // f64 [C][batch][64] (used in rank 0)
+  L.bar = L.push + static_cast<uint32_t>(C) * 64u * batch * 8u;  // mbarrier
+  L.total = L.bar + 8u;
   return L;
+}
+
+__device__ __forceinline__ uint32_t mapa_shared_u32(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// remote 8-byte store into a peer block's shared memory, completing 8 bytes of
+// the transaction count of the peer's mbarrier
+__device__ __forceinline__ void st_async_f64(uint32_t remote_addr, double v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b64 [%0], %1, [%2];" ::"r"(remote_addr),
+               "l"(__double_as_longlong(v)), "r"(remote_bar)
+               : "memory");
+}
+
+// batch row of x chunk c when a row has cpr chunks (batch <= 4, no division)
+__device__ __forceinline__ int chunk_row(int c, int cpr) {
+  return c >= cpr ? (c >= 2 * cpr ? (c >= 3 * cpr ? 3 : 2) : 1) : 0;
 }
 
 template <int B>
 __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a) {
   constexpr int NB = (4 * B + 7) / 8;  // n tiles of 8 planes
-  constexpr int kXR = kI8MaxChunks / kI8Threads;  // x chunks (4 elements) per thread
+  constexpr int kQ = (B * 64 + kI8Threads - 1) / kI8Threads;
   extern __shared__ __align__(16) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -77,45 +103,55 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);
-  const GemvI8Layout L = gemv_i8_layout(a.tpc, B);
+  const GemvI8Layout L = gemv_i8_layout(a.tpc, B, a.C);
   const uint32_t s0 = smem_u32(sm);
+  const uint32_t push_bar = s0 + L.bar;
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   uint32_t* mask = reinterpret_cast<uint32_t*>(sm + L.mask);
   uint32_t* emax = reinterpret_cast<uint32_t*>(sm + L.emax);  // [0..3] exponent, [4] any residual
   long long* acc = reinterpret_cast<long long*>(sm + L.acc);
-  // first half of a split cluster barrier: its wait (before the first remote
-  // access) then guarantees that every block of the cluster has started
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  constexpr uint32_t kPartBytes = static_cast<uint32_t>(B) * 64u * 8u;
 
-  // ---- codes: one bulk copy (weights are not written by the kernels this one may overlap)
-  if (tid == 0) {
-    mbar_init(s0 + L.bar, 1);
-    mbar_fence_init();
-    if (!(a.inject && crank == 0 && rb == 0)) {
-      mbar_arrive_expect_tx(s0 + L.bar, static_cast<uint32_t>(nt) * 1024u);
-      bulk_g2s(s0 + L.codes, a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0),
-               static_cast<uint32_t>(nt) * 1024u, s0 + L.bar);
-    }
+  // ---- every global load first.  The codes are never written by a neighbour
+  // in a programmatic-dependent chain (the caller's contract), so they go
+  // before the dependency wait; x after it.
+  const int8_t* codes_blk = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
+  uint4 cv[kI8CodeLoads];
+#pragma unroll
+  for (int u = 0; u < kI8CodeLoads; ++u) {
+    const int q = tid + u * kI8Threads;  // 16-code chunk
+    cv[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (q < nt * 64) cv[u] = ldg_nc128(codes_blk + 16 * q);
   }
   if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
-
-  // ---- x: 4-element chunks, all loads in flight before anything else
-  const int cpr = nt * 64;  // chunks per batch row
-  const int nchunks = B * cpr;
-  uint2 xv[kXR];
+  const int cpr = nt * 64;  // 4-element chunks per batch row
+  uint2 xv[kI8XR];
 #pragma unroll
-  for (int u = 0; u < kXR; ++u) {
+  for (int u = 0; u < kI8XR; ++u) {
     const int c = tid + u * kI8Threads;
     xv[u] = make_uint2(0u, 0u);
-    if (c < nchunks) {
-      const int bi = c / cpr, cc = c % cpr;
+    if (c < B * cpr) {
+      const int bi = chunk_row(c, cpr), cc = c - bi * cpr;
       xv[u] = ldg_nc64(a.x + static_cast<int64_t>(bi) * a.K + static_cast<int64_t>(t0) * kTileCols + 4 * cc);
     }
   }
+  if (tid == 0 && a.C > 1) {
+    mbar_init(push_bar, 1);
+    mbar_fence_init();
+    if (crank == 0) mbar_arrive_expect_tx(push_bar, static_cast<uint32_t>(a.C - 1) * kPartBytes);
+  }
+  // first half of a split cluster barrier; its wait, before the first remote
+  // store, guarantees that the first block's push barrier is set up (relaxed:
+  // a release arrive would wait for this thread's loads in flight)
+  if (a.C > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
   if (tid < 8) emax[tid] = 0u;
   for (int q = tid; q < B * a.tpc * 8; q += kI8Threads) mask[q] = 0u;
-  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < kI8CodeLoads; ++u) {
+    const int q = tid + u * kI8Threads;
+    if (q < nt * 64) sts128(s0 + L.codes + 16u * q, cv[u]);
+  }
 
   // ---- x pass 1: largest finite exponent per batch row
   {
@@ -123,10 +159,10 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
 #pragma unroll
     for (int bi = 0; bi < B; ++bi) em[bi] = 0;
 #pragma unroll
-    for (int u = 0; u < kXR; ++u) {
+    for (int u = 0; u < kI8XR; ++u) {
       const int c = tid + u * kI8Threads;
-      if (c < nchunks) {
-        const int bi = c / cpr;
+      if (c < B * cpr) {
+        const int bi = chunk_row(c, cpr);
         const uint32_t w[2] = {xv[u].x, xv[u].y};
         int m = 0;
 #pragma unroll
@@ -150,10 +186,10 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
 
   // ---- x pass 2: digit planes (one 4-byte word per plane per chunk) and residual bits
 #pragma unroll
-  for (int u = 0; u < kXR; ++u) {
+  for (int u = 0; u < kI8XR; ++u) {
     const int c = tid + u * kI8Threads;
-    if (c < nchunks) {
-      const int bi = c / cpr, cc = c % cpr;
+    if (c < B * cpr) {
+      const int bi = chunk_row(c, cpr), cc = c - bi * cpr;
       const int E = static_cast<int>(emax[bi]);
       const uint32_t w[2] = {xv[u].x, xv[u].y};
       uint32_t dw[4];
@@ -187,9 +223,9 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
       }
     }
   }
-  uint32_t flags = 0;
-  if (!mbar_wait(s0 + L.bar, 0)) flags |= USK_FLAG_TIMEOUT;
   __syncthreads();
+  // blocks other than the first: the first block's push barrier is set up
+  if (a.C > 1 && crank != 0) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 
   // ---- main loop: warp = column phase, lane (g, t) gathers octet o of rows g, g + 8
   const int g = lane >> 2, t = lane & 3;
@@ -257,10 +293,10 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
 
   // ---- block partial: scale and the exact correction for residual columns
   const bool any_resid = emax[4] != 0u;
-  double part[(B * 64 + kI8Threads - 1) / kI8Threads];
+  double part[kQ];
 #pragma unroll
-  for (int k = 0; k < (B * 64 + kI8Threads - 1) / kI8Threads; ++k) {
-    const int q = tid + k * kI8Threads;
+  for (int k = 0; k < kQ; ++k) {
+    const int q = tid + k * kI8Threads;  // q = bi * 64 + r
     part[k] = 0.0;
     if (q < B * 64) {
       const int bi = q >> 6, r = q & 63;
@@ -290,34 +326,52 @@ __global__ void __launch_bounds__(kI8Threads) gemv_i8_kernel(const GemvI8Args a)
       part[k] = v;
     }
   }
-  report(a.status, flags);
 
-  // ---- push the partial into block 0 of the cluster; block 0 adds them in rank order
-  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every block has started
-  {
-    double* push0 = cluster.map_shared_rank(reinterpret_cast<double*>(sm + L.push), 0);
+  // ---- partials of the row block: into the first block, added in rank order
+  const double s = static_cast<double>(__half2float(__ushort_as_half(a.scales[rb])));
+  float* yrb = a.y + static_cast<int64_t>(rb) * 64;
+  if (a.C == 1) {
 #pragma unroll
-    for (int k = 0; k < (B * 64 + kI8Threads - 1) / kI8Threads; ++k) {
+    for (int k = 0; k < kQ; ++k) {
       const int q = tid + k * kI8Threads;
-      if (q < B * 64) push0[crank * B * 64 + q] = part[k];
+      if (q < B * 64) yrb[static_cast<int64_t>(q >> 6) * a.M + (q & 63)] = static_cast<float>(part[k] * s);
     }
+    return;
   }
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-  if (crank == 0) {
-    const double* push = reinterpret_cast<const double*>(sm + L.push);
-    const double s = static_cast<double>(__half2float(__ushort_as_half(a.scales[rb])));
-    for (int q = tid; q < B * 64; q += kI8Threads) {
+  double* push = reinterpret_cast<double*>(sm + L.push);
+  if (crank != 0) {
+    if (a.inject && crank == 1 && rb == 0) return;  // test hook: the first block's wait gives up
+    const uint32_t bar0 = mapa_shared_u32(push_bar, 0);
+#pragma unroll
+    for (int k = 0; k < kQ; ++k) {
+      const int q = tid + k * kI8Threads;
+      if (q < B * 64)
+        st_async_f64(mapa_shared_u32(s0 + L.push + (static_cast<uint32_t>(crank) * B * 64u + q) * 8u, 0), part[k],
+                     bar0);
+    }
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < kQ; ++k) {
+    const int q = tid + k * kI8Threads;
+    if (q < B * 64) push[q] = part[k];
+  }
+  if (!mbar_wait(push_bar, 0)) report(a.status, USK_FLAG_TIMEOUT);  // bounded (about 1 s)
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kQ; ++k) {
+    const int q = tid + k * kI8Threads;
+    if (q < B * 64) {
       double tot = 0.0;
       for (int c = 0; c < a.C; ++c) tot += push[c * B * 64 + q];
-      const int bi = q >> 6, r = q & 63;
-      a.y[static_cast<int64_t>(bi) * a.M + static_cast<int64_t>(rb) * 64 + r] = static_cast<float>(tot * s);
+      yrb[static_cast<int64_t>(q >> 6) * a.M + (q & 63)] = static_cast<float>(tot * s);
     }
   }
 }
 
 template <int B>
 static cudaError_t launch_i8_t(GemvI8Args a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_i8_layout(a.tpc, B).total;
+  const size_t smem = gemv_i8_layout(a.tpc, B, a.C).total;
   auto kern = gemv_i8_kernel<B>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -338,7 +392,8 @@ static cudaError_t launch_i8_t(GemvI8Args a, int64_t RB, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-// T, C, tpc: the same block geometry as the bf16 path; batch * tpc * 32 <= kI8MaxChunks.
+// T, C, tpc: the same block geometry as the staged-x bf16 path (C <= 8);
+// batch * tpc * 64 <= kI8MaxChunks.
 cudaError_t launch_gemv_i8(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, int T, int C, int tpc, bool pdl,
                            cudaStream_t stream, int inject) {

@@ -53,9 +53,9 @@ def test_gemm_wait_timeout_reported_then_recovers():
 
 @pytest.mark.parametrize("path", [2, 3, 4])
 def test_gemv_wait_timeout_reported_then_recovers(path):
-    """Paths 2 and 3 skip a code copy; path 4 (no copies) has block 1 of row
+    """Path 3 skips a code copy; paths 2 and 4 (no copies) have block 1 of row
     block 0 skip its partial sums, so the first block's wait gives up."""
-    K = 2048 if path == 4 else 256
+    K = 2048 if path in (2, 4) else 256
     W = gen.weights_normal(64, K, 4, 0.02, "bf16")
     sk = usk.usk_build(to_dev(W), None, 2)
     x = gen.activations(1, K, 5, "bf16")
