@@ -253,6 +253,21 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Bytes 0, 1 (sel 0x4140) or 2, 3 (sel 0x4342) of w, int8 codes, -> one bf16
+// pair, exact, in four integer/FMA-pipe instructions (no conversion unit): the
+// permute puts each byte b under a 0x43 high byte; with bit 7 cleared that is
+// the bf16 value 128 + (b & 127), with only bit 7 kept it is 128 or 256; their
+// difference is b as a two's-complement integer, exactly representable.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t i8pair_to_bf16x2(uint32_t w) {
+  const uint32_t p = __byte_perm(w, 0x43434343u, SEL);
+  const uint32_t mag = p & 0xFF7FFF7Fu;                 // 128 + (b & 127)
+  const uint32_t off = (p & 0x00800080u) | 0x43004300u;  // 128, or 256 when b < 0
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(mag), "r"(off));
+  return r;
+}
+
 // ---- integer tensor path helpers (mma.sync m16n8k32 s8)
 
 __device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -11,10 +11,11 @@
 //    cluster and add their fp32 partials through distributed shared memory in
 //    rank order (deterministic, no workspace).
 //  * At start the block's int8 codes (2 row blocks x its tiles) arrive in
-//    shared memory with two bulk copies.  Once per tile the decoders widen that
-//    tile's 2 x 1024 codes to bf16 (exact) in a double buffer, so a code is
-//    converted once instead of once per use (16 uses); a bounded per-tile
-//    mbarrier among the decoders orders the buffer reuse.
+//    shared memory with two bulk copies; a widen warp converts each tile's
+//    2 x 1024 codes to bf16 once (instead of once per use: 16 uses) with an
+//    exact integer/FMA-pipe bit trick (the conversion unit of one sub-partition
+//    was measured as the bottleneck), into a ring of tile buffers guarded by
+//    ready/free mbarriers.
 //  * 16 decoder warps: per 64-column chunk each thread rebuilds 2 octets of one
 //    row -- one multiply-add of the hash per octet, one 16-byte conflict-free
 //    gather of the 8 bf16 codes (class = (octet + row) mod 32) -- and writes
@@ -159,14 +160,6 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// two int8 codes (bytes 0 and 1 of w) -> one bf16 pair, exact (|code| <= 127)
-__device__ __forceinline__ uint32_t i8x2_to_bf16x2(uint32_t w) {
-  const float f0 = static_cast<float>(static_cast<int8_t>(w & 0xFFu));
-  const float f1 = static_cast<float>(static_cast<int8_t>((w >> 8) & 0xFFu));
-  __nv_bfloat162 p = __floats2bfloat162_rn(f0, f1);
-  return *reinterpret_cast<uint32_t*>(&p);
-}
-
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
   extern __shared__ __align__(16) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -300,12 +293,21 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
         aborted = true;
         break;
       }
-#pragma unroll 4
-      for (int i = 0; i < 16; ++i) {  // 2 x 1024 codes, 4 per lane per step
-        const uint32_t idx = static_cast<uint32_t>(lane) * 4u + static_cast<uint32_t>(i) * 128u;
-        const uint32_t wrb = idx >> 10, b = idx & 1023u;
-        const uint32_t w = lds32(s0 + L.codes + (wrb * tcta + t) * 1024u + b);
-        sts64(s0 + L.cbf + q * 4096u + wrb * 2048u + 2u * b, make_uint2(i8x2_to_bf16x2(w), i8x2_to_bf16x2(w >> 16)));
+      // 2 x 1024 codes, 16 per lane per step; all four loads in flight first
+      uint4 w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t idx = static_cast<uint32_t>(lane) * 16u + static_cast<uint32_t>(i) * 512u;
+        w[i] = lds128(s0 + L.codes + ((idx >> 10) * tcta + t) * 1024u + (idx & 1023u));
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t idx = static_cast<uint32_t>(lane) * 16u + static_cast<uint32_t>(i) * 512u;
+        const uint32_t dst = s0 + L.cbf + q * 4096u + (idx >> 10) * 2048u + 2u * (idx & 1023u);
+        sts128(dst, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].x), i8pair_to_bf16x2<0x4342>(w[i].x),
+                               i8pair_to_bf16x2<0x4140>(w[i].y), i8pair_to_bf16x2<0x4342>(w[i].y)));
+        sts128(dst + 16u, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].z), i8pair_to_bf16x2<0x4342>(w[i].z),
+                                     i8pair_to_bf16x2<0x4140>(w[i].w), i8pair_to_bf16x2<0x4342>(w[i].w)));
       }
       mbar_arrive(ready_s + 8 * q);
     }
@@ -402,8 +404,13 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
     const int per = (total + a.splits - 1) / a.splits;
     const int q0 = ks * per, q1 = min(total, q0 + per);
     for (int q = q0 + tid; q < q1; q += kGemmThreads) {
+      // all remote loads in flight at once, then the sum in rank order
+      float v[16];
+#pragma unroll
+      for (int s = 0; s < 16; ++s) v[s] = s < a.splits ? *cluster.map_shared_rank(&part[q], s) : 0.0f;
       float acc = 0.0f;
-      for (int s = 0; s < a.splits; ++s) acc += *cluster.map_shared_rank(&part[q], s);
+#pragma unroll
+      for (int s = 0; s < 16; ++s) acc += v[s];
       const int n = q / kBM, mm = q % kBM;
       const int64_t orow = static_cast<int64_t>(mt) * kBM + mm;
       if (orow < a.M) {
@@ -432,18 +439,25 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N)
 
 // Pipeline stages for batch N and tpb tiles per block: as many as tensor
 // memory and shared memory (the B stages next to the staged codes; half of the
-// SM's when two blocks share it) hold, at most kMaxStages; 0 if fewer than 2.
+// SM's when two blocks share it) hold, at most kMaxStages; 0 if fewer than 4.
+//
+// S is a multiple of 4: stage s = c mod S is then always filled by decoder
+// group s mod 4 and consumed by MMA warp s mod I (I divides 4), so every
+// mbarrier has one in-order waiter per role.  Otherwise consecutive uses of a
+// stage belong to different warps, and a warp running ahead can take a
+// completed phase of use n - 2 for use n (a phase wait only tells parity).
 static int gemm_stages(int N, int tpb) {
   const uint32_t cols = gemm_tmem_cols(N);
   const uint32_t smem_cap = cols == 256u ? 233472u / 2u - 1024u : kSmemLimit;
   int S = static_cast<int>((cols - gemm_a_col(N)) / 32u);
   if (S > kMaxStages) S = kMaxStages;
-  while (S >= 2 && gemm_layout(N, tpb, S).total + 1024u > smem_cap) --S;
-  return S >= 2 ? S : 0;
+  S &= ~3;
+  while (S >= 4 && gemm_layout(N, tpb, S).total + 1024u > smem_cap) S -= 4;
+  return S >= 4 ? S : 0;
 }
 
 // Largest number of tiles per block (codes staged up front) that still leaves
-// a two-stage pipeline for batch N.
+// a four-stage pipeline for batch N.
 static int gemm_max_tiles(int N) {
   int t = kMaxTiles;
   while (t > 1 && gemm_stages(N, t) == 0) --t;
@@ -474,7 +488,9 @@ static int gemm_splits(int64_t m_tiles, int T, int N, int sms) {
     const int tpb = (T + s - 1) / s;
     if (tpb > max_tiles) continue;
     const int64_t waves = (m_tiles * s + slots - 1) / slots;
-    const int64_t cost = waves * (tpb + 4);
+    // clusters above 4 blocks launch with a visible spread (up to 3 us measured
+    // for 8 blocks of 704 threads): charge them 2 tiles more
+    const int64_t cost = waves * (tpb + 4 + (s > 4 ? 2 : 0));
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = s;
@@ -506,7 +522,7 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.I = gemm_issuers(batch);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
   a.S = gemm_stages(batch, tcta_max);
-  if (a.S < 2) return cudaErrorInvalidValue;
+  if (a.S < 4 || a.S % 4 != 0) return cudaErrorInvalidValue;
   const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S);
   // tensor map over x [batch, K] bf16: one 64-column x batch box per chunk, 128-byte swizzle
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();

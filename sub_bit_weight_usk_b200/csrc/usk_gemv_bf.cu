@@ -81,13 +81,6 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
                : "memory");
 }
 
-// bytes 0 and 1 of w (int8 codes) -> one bf16 pair, exact (|code| <= 127)
-__device__ __forceinline__ uint32_t pack_i8x2_bf16(uint32_t w) {
-  __nv_bfloat162 p = __floats2bfloat162_rn(static_cast<float>(static_cast<int8_t>(w & 0xFFu)),
-                                           static_cast<float>(static_cast<int8_t>((w >> 8) & 0xFFu)));
-  return *reinterpret_cast<uint32_t*>(&p);
-}
-
 template <int B>
 __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a) {
   extern __shared__ __align__(128) uint8_t sm[];
@@ -146,8 +139,8 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
       uint32_t o8[8];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        o8[2 * e] = pack_i8x2_bf16(ws[e]);
-        o8[2 * e + 1] = pack_i8x2_bf16(ws[e] >> 16);
+        o8[2 * e] = i8pair_to_bf16x2<0x4140>(ws[e]);
+        o8[2 * e + 1] = i8pair_to_bf16x2<0x4342>(ws[e]);
       }
       sts128(s0 + L.cbf + 32u * q, make_uint4(o8[0], o8[1], o8[2], o8[3]));
       sts128(s0 + L.cbf + 32u * q + 16u, make_uint4(o8[4], o8[5], o8[6], o8[7]));
