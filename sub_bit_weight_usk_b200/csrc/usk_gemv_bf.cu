@@ -99,8 +99,18 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   constexpr uint32_t kPartBytes = static_cast<uint32_t>(B) * 64u * 4u;
   constexpr int kCodeLoads = kBfMaxTiles * 1024 / 16 / kBfThreads;  // 16-byte code loads per thread (at most)
 
+  // ---- every global load first.  The codes are never written by a neighbour
+  // in a programmatic-dependent chain (the caller's contract), so they go
+  // before the dependency wait and overlap the previous kernel's tail; x after.
+  const int8_t* codes_blk = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
+  uint4 cv[kCodeLoads];
+#pragma unroll
+  for (int u = 0; u < kCodeLoads; ++u) {
+    const int q = tid + u * kBfThreads;  // 16-code chunk
+    cv[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (q < nt * 64) cv[u] = ldg_nc128(codes_blk + 16 * q);
+  }
   if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
-  // ---- every global load first: x B fragments and the codes
   const int g = lane >> 2, t = lane & 3;
   const int o = (warp & 1) + 8 * (warp >> 1) + 2 * t;  // this lane's octet in every tile
   uint4 xv[kBfMaxTiles];
@@ -109,14 +119,6 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
     xv[tt] = make_uint4(0u, 0u, 0u, 0u);
     if (tt < nt && g < B)
       xv[tt] = ldg_nc128(a.x + static_cast<int64_t>(g) * a.K + static_cast<int64_t>(t0 + tt) * kTileCols + 8 * o);
-  }
-  const int8_t* codes_blk = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
-  uint4 cv[kCodeLoads];
-#pragma unroll
-  for (int u = 0; u < kCodeLoads; ++u) {
-    const int q = tid + u * kBfThreads;  // 16-code chunk
-    cv[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (q < nt * 64) cv[u] = ldg_nc128(codes_blk + 16 * q);
   }
   if (tid == 0 && a.C > 1) {
     mbar_init(push_bar, 1);
