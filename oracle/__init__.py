@@ -9,7 +9,9 @@ What it computes is written out in ``usk_oracle.c`` with its sources:
 "UltraSketchLLM: Sub-1-Bit LLM Compression via Sketch and Hardware-Friendly
 Operators" (gist.science/es/paper/2506.17255), Resumen Tecnico, Metodologia §1
 (AbsMaxMin sketch) and §4 (decompression as W_hat = S . P^T), plus the frozen
-format readings listed there.
+format readings listed there: format 1 (one hash row, largest key kept) and
+format 2 (the multi-row AbsMaxMin sketch: smallest magnitude kept per bucket,
+largest magnitude over the hash rows on decode; the ``*_amm`` functions).
 
 Parity pins (tests/test_oracle_*.py): SplitMix64 published outputs, binary16
 conversion against numpy's, round-half-even against numpy.rint, an independent
@@ -82,6 +84,16 @@ def _load():
         lib.orc_bf16_to_f32.restype = ctypes.c_float
         lib.orc_storage_bytes.argtypes = [i64, i64, vp, vp]
         lib.orc_storage_bytes.restype = None
+        lib.orc_amm_bucket_index.argtypes = [i64, u64, ctypes.c_int, ctypes.c_int, i64, i64]
+        lib.orc_amm_bucket_index.restype = i64
+        lib.orc_amm_build_rows.argtypes = [vp, ctypes.c_int, i64, i64, i64, u64, ctypes.c_int, i64, vp, vp,
+                                           vp, vp]
+        lib.orc_amm_build_rows.restype = ctypes.c_int
+        lib.orc_amm_decode.argtypes = [vp, vp, i64, i64, u64, ctypes.c_int, vp]
+        lib.orc_amm_decode.restype = ctypes.c_int
+        lib.orc_amm_gemv_f64.argtypes = [vp, vp, i64, i64, u64, ctypes.c_int, vp, ctypes.c_int, i64, vp, i64,
+                                         vp]
+        lib.orc_amm_gemv_f64.restype = ctypes.c_int
         lib.orc_f32_to_f16_array.argtypes = [vp, vp, i64]
         lib.orc_f32_to_f16_array.restype = None
         lib.orc_f16_to_f32_array.argtypes = [vp, vp, i64]
@@ -124,6 +136,62 @@ def build_sketch(W, importance=None, seed=0, want_winners=False, row_block0=0):
         out["winner"] = winner[:nb]
         out["value"] = value[:nb]
     return out
+
+
+def build_sketch_amm(W, seed=0, depth=2, want_winners=False, row_block0=0):
+    """Depth-`depth` AbsMaxMin sketch of W [M, K] (format 2: min-|w| store,
+    max-magnitude decode over the hash rows).  Returns dict as build_sketch."""
+    W, dt = _weights(W)
+    M, K = W.shape
+    nb = M * K // 16 if (M % 64 == 0 and K % 256 == 0 and M >= 0 and K >= 0) else 0
+    codes = np.zeros(max(nb, 1), dtype=np.int8)
+    scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
+    winner = np.full(max(nb, 1), -2, dtype=np.int64) if want_winners else None
+    value = np.zeros(max(nb, 1), dtype=np.float32) if want_winners else None
+    st = _load().orc_amm_build_rows(_ptr(W), dt, M, K, K, seed, depth, row_block0, _ptr(codes),
+                                    _ptr(scales), _ptr(winner), _ptr(value))
+    out = {"status": st, "codes": codes[:nb], "scales": scales[: M // 64]}
+    if want_winners:
+        out["winner"] = winner[:nb]
+        out["value"] = value[:nb]
+    return out
+
+
+def decode_amm(codes, scales, M, K, seed=0, depth=2):
+    """W_hat [M, K] float32 of a format-2 sketch."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    out = np.zeros((M, K), dtype=np.float32)
+    st = _load().orc_amm_decode(_ptr(codes), _ptr(scales), M, K, seed, depth, _ptr(out))
+    if st:
+        raise ValueError("orc_amm_decode status %d" % st)
+    return out
+
+
+def gemv_amm_f64(codes, scales, M, K, x, seed=0, depth=2, rows=None):
+    """y = W_hat x^T in float64 for a format-2 sketch (arguments as gemv_f64)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    xdt = F32 if x.dtype == np.float32 else BF16 if x.dtype == np.uint16 else None
+    if xdt is None:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    batch = x.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nr = M if r is None else len(r)
+    y = np.zeros((batch, nr), dtype=np.float64)
+    st = _load().orc_amm_gemv_f64(_ptr(codes), _ptr(scales), M, K, seed, depth, _ptr(x), xdt, batch,
+                                  _ptr(r), 0 if r is None else len(r), _ptr(y))
+    if st:
+        raise ValueError("orc_amm_gemv_f64 status %d" % st)
+    return y
+
+
+def amm_bucket_index(K, seed, depth, rho, i, j):
+    """Global code index of weight (i, j) in hash row rho of a format-2 sketch."""
+    return int(_load().orc_amm_bucket_index(K, seed, depth, rho, i, j))
 
 
 def decode(codes, scales, M, K, seed=0):

@@ -346,3 +346,187 @@ void orc_f32_to_f16_array(const float* in, uint16_t* out, int64_t n) {
 void orc_f16_to_f32_array(const uint16_t* in, float* out, int64_t n) {
   for (int64_t q = 0; q < n; ++q) out[q] = orc_f16_to_f32(in[q]);
 }
+
+/* ================================================================ format 2
+ *
+ * The multi-row AbsMaxMin sketch ("UltraSketchLLM" explainer, Resumen Tecnico,
+ * Metodologia §1 "Diseno de Sketch AbsMaxMin"): a bucket stores the member
+ * with the SMALLEST absolute value, decompression takes the MAX over several
+ * independently hashed sketch rows, and the rebuilt weight is the original one
+ * or one of smaller magnitude.  Readings (the pages give no more detail):
+ *  - depth D in {1, 2, 4} hash rows share the tile's 1024 buckets, so the
+ *    storage stays one int8 code per 16 weights (Resultados, 0.5 bit/weight):
+ *    row rho owns buckets [rho*1024/D, (rho+1)*1024/D) of the tile;
+ *  - row rho of tile tile_id is keyed by SplitMix64 output tile_id*D + rho + 1,
+ *    slot = floor(4h / 2^32) as in format 1, class = (o + r) mod (32/D),
+ *    bucket = rho*1024/D + (slot*(32/D) + class)*8 + c mod 8.  With D = 1 this
+ *    is exactly the format-1 hash;
+ *  - the kept member has the smallest |w|, ties to the smallest row-major
+ *    index; an empty bucket keeps 0.  No importance weighting (a weighted key
+ *    would break the magnitude bound);
+ *  - scale as format 1: s16 = binary16(max over the block's buckets of |v| / 127);
+ *  - code = sign(v) * min(127, floor(|v| / s)) (toward zero), so that
+ *    |code * s| <= |v| and the bound survives quantisation;
+ *  - decode: the code of largest magnitude among the weight's D buckets (ties
+ *    to the lowest row), times s. */
+
+static int amm_depth_ok(int depth) { return depth == 1 || depth == 2 || depth == 4; }
+
+/* Global code index of weight (i, j) in hash row rho of a depth-D sketch. */
+int64_t orc_amm_bucket_index(int64_t K, uint64_t seed, int depth, int rho, int64_t i, int64_t j) {
+  int64_t rb = i / ROWS_PER_BLOCK, r = i % ROWS_PER_BLOCK;
+  int64_t tc = j / TILE_COLS, c = j % TILE_COLS;
+  int64_t T = tiles_per_row(K);
+  int64_t o = c / OCTET, sub = c % OCTET;
+  int64_t nclass = CLASSES / depth, per_row = 1024 / depth;
+  uint32_t A, C;
+  orc_tile_hash_params(seed, (uint64_t)((rb * T + tc) * depth + rho), &A, &C);
+  uint32_t m = (uint32_t)(r * (TILE_COLS / OCTET) + o);
+  uint32_t h = A * m + C;
+  int64_t slot = (int64_t)(((uint64_t)h * 4u) >> 32);
+  int64_t cls = (o + r) % nclass;
+  int64_t b = rho * per_row + (slot * nclass + cls) * OCTET + sub;
+  return rb * (4 * K) + 1024 * tc + b;
+}
+
+/* Largest n in [0, 127] with n * s <= a (a >= 0, s > 0); every product and
+ * comparison below is exact in double (an 8-bit integer times a binary16). */
+static int floor_code(double a, double s) {
+  double n = floor(a / s);
+  if (n > 127.0) n = 127.0;
+  while (n < 127.0 && (n + 1.0) * s <= a) n += 1.0;
+  while (n > 0.0 && n * s > a) n -= 1.0;
+  return (int)n;
+}
+
+/* Build a depth-D AbsMaxMin sketch of W [M, K] (rows starting at row block rb0
+ * of a larger matrix, as orc_build_rows).  Outputs as orc_build_rows: codes,
+ * scales, optional winner (flat index into W, -1 if empty) and value. */
+int orc_amm_build_rows(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw,
+                       uint64_t seed, int depth, int64_t rb0, int8_t* codes,
+                       uint16_t* scales, int64_t* winner, float* value) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (rb0 < 0) return ORC_ERR_SHAPE;
+  if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
+  if (!amm_depth_ok(depth)) return ORC_ERR_SHAPE;
+  if (M == 0) return ORC_OK;
+  if (!codes || !scales) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) scales[rb] = 0;
+    return ORC_OK;
+  }
+  if (!W || ldw < K) return ORC_ERR_NULL;
+  int64_t per_block = 4 * K;
+  float* bestmag = (float*)malloc(sizeof(float) * (size_t)per_block);
+  int64_t* bestidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)per_block);
+  float* val = (float*)malloc(sizeof(float) * (size_t)per_block);
+  if (!bestmag || !bestidx || !val) { free(bestmag); free(bestidx); free(val); return ORC_ERR_NULL; }
+  int status = ORC_OK;
+  for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
+    for (int64_t b = 0; b < per_block; ++b) { bestmag[b] = 0.0f; bestidx[b] = -1; }
+    /* every weight updates its bucket in each hash row: keep the smallest |w|;
+     * the row-major scan keeps the earlier member on equal magnitudes */
+    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
+      int64_t i = rb * ROWS_PER_BLOCK + r;
+      for (int64_t j = 0; j < K; ++j) {
+        float w = load_elem(W, dtype, i * ldw + j);
+        if (!isfinite(w)) status = ORC_ERR_NONFINITE;
+        float mag = fabsf(w);
+        for (int rho = 0; rho < depth; ++rho) {
+          int64_t b = orc_amm_bucket_index(K, seed, depth, rho, i + rb0 * ROWS_PER_BLOCK, j) -
+                      (rb + rb0) * per_block;
+          if (bestidx[b] < 0 || mag < bestmag[b]) { bestmag[b] = mag; bestidx[b] = i * K + j; }
+        }
+      }
+    }
+    float mx = 0.0f;
+    for (int64_t b = 0; b < per_block; ++b) {
+      float v = 0.0f;
+      if (bestidx[b] >= 0) {
+        int64_t i = bestidx[b] / K, j = bestidx[b] % K;
+        v = load_elem(W, dtype, i * ldw + j);
+      }
+      val[b] = v;
+      if (fabsf(v) > mx) mx = fabsf(v);
+    }
+    uint16_t s16 = orc_f32_to_f16(mx / 127.0f);
+    if ((s16 & 0x7c00u) == 0x7c00u) status = status ? status : ORC_ERR_SCALE_OVERFLOW;
+    scales[rb] = s16;
+    double s = (double)orc_f16_to_f32(s16);
+    for (int64_t b = 0; b < per_block; ++b) {
+      int code = 0;
+      if (s != 0.0 && isfinite(s) && isfinite(val[b])) {
+        code = floor_code(fabs((double)val[b]), s);
+        if (val[b] < 0.0f) code = -code;
+      }
+      int64_t g = rb * per_block + b;
+      codes[g] = (int8_t)code;
+      if (winner) winner[g] = bestidx[b];
+      if (value) value[g] = val[b];
+    }
+  }
+  free(bestmag); free(bestidx); free(val);
+  return status;
+}
+
+/* Code of weight (i, j): the largest-magnitude code over the D rows (ties to
+ * the lowest row). */
+static int amm_code(const int8_t* codes, int64_t K, uint64_t seed, int depth, int64_t i, int64_t j) {
+  int best = codes[orc_amm_bucket_index(K, seed, depth, 0, i, j)];
+  for (int rho = 1; rho < depth; ++rho) {
+    int c = codes[orc_amm_bucket_index(K, seed, depth, rho, i, j)];
+    if (abs(c) > abs(best)) best = c;
+  }
+  return best;
+}
+
+/* W_hat [M, K] of a depth-D sketch: w_hat = float(code) * float(s16). */
+int orc_amm_decode(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K,
+                   uint64_t seed, int depth, float* What) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (!amm_depth_ok(depth)) return ORC_ERR_SHAPE;
+  if (M == 0 || K == 0) return ORC_OK;
+  if (!codes || !scales || !What) return ORC_ERR_NULL;
+  for (int64_t i = 0; i < M; ++i) {
+    float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+    for (int64_t j = 0; j < K; ++j) What[i * K + j] = (float)amm_code(codes, K, seed, depth, i, j) * s;
+  }
+  return ORC_OK;
+}
+
+/* Reference product of a depth-D sketch in float64 (arguments as orc_gemv_f64). */
+int orc_amm_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K,
+                     uint64_t seed, int depth, const void* x, int xdtype, int64_t batch,
+                     const int64_t* rows, int64_t nrows, double* y) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (!amm_depth_ok(depth)) return ORC_ERR_SHAPE;
+  if (xdtype != 0 && xdtype != 1) return ORC_ERR_DTYPE;
+  if (batch < 0) return ORC_ERR_SHAPE;
+  int64_t nr = rows ? nrows : M;
+  if (nr == 0 || batch == 0) return ORC_OK;
+  if (!y) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t q = 0; q < batch * nr; ++q) y[q] = 0.0;
+    return ORC_OK;
+  }
+  if (!codes || !scales || !x) return ORC_ERR_NULL;
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!wrow) return ORC_ERR_NULL;
+  for (int64_t q = 0; q < nr; ++q) {
+    int64_t i = rows ? rows[q] : q;
+    if (i < 0 || i >= M) { free(wrow); return ORC_ERR_SHAPE; }
+    float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+    for (int64_t j = 0; j < K; ++j)
+      wrow[j] = (double)((float)amm_code(codes, K, seed, depth, i, j) * s);
+    for (int64_t t = 0; t < batch; ++t) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j) acc += wrow[j] * (double)load_elem(x, xdtype, t * K + j);
+      y[t * nr + q] = acc;
+    }
+  }
+  free(wrow);
+  return ORC_OK;
+}

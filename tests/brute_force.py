@@ -82,3 +82,76 @@ def build(W: np.ndarray, importance=None, seed: int = 0):
             q = np.rint(v / s)
             codes[rb * per:(rb + 1) * per] = np.clip(q, -127, 127).astype(np.int8)
     return codes, scales, winner
+
+
+# ---- format 2: the multi-row AbsMaxMin sketch (Metodologia §1: a bucket keeps
+# its member of smallest magnitude; decompression takes the largest magnitude
+# over the hash rows).  depth D rows share the tile's 1024 buckets; row rho is
+# keyed by SplitMix64 output tile_id*D + rho + 1; class = (o + r) % (32 // D).
+
+def bucket_of_amm(K: int, seed: int, depth: int, rho: int, i: int, j: int) -> int:
+    rb, r = divmod(i, 64)
+    tc, c = divmod(j, 256)
+    tile_id = rb * (K // 256) + tc
+    z = splitmix64_output(seed, tile_id * depth + rho + 1)
+    A = (z & 0xFFFFFFFF) | 1
+    C = z >> 32
+    o = c // 8
+    h = (A * (32 * r + o) + C) & 0xFFFFFFFF
+    slot = (4 * h) >> 32
+    ncls = 32 // depth
+    b = rho * (1024 // depth) + (slot * ncls + (o + r) % ncls) * 8 + (c % 8)
+    return rb * 4 * K + 1024 * tc + b
+
+
+def build_amm(W: np.ndarray, seed: int = 0, depth: int = 2):
+    """Returns (codes, scales, winner).  Members listed per bucket and sorted by
+    (|w|, row-major index); codes by exact rational arithmetic (Fraction):
+    sign(v) * min(127, floor(|v| / s))."""
+    from fractions import Fraction
+    Wf = to_f32(np.ascontiguousarray(W))
+    M, K = Wf.shape
+    nb = M * K // 16
+    members = [[] for _ in range(nb)]
+    for i in range(M):
+        for j in range(K):
+            for rho in range(depth):
+                members[bucket_of_amm(K, seed, depth, rho, i, j)].append(i * K + j)
+    flat = Wf.reshape(-1)
+    winner = np.full(nb, -1, dtype=np.int64)
+    value = np.zeros(nb, dtype=np.float32)
+    for b, mem in enumerate(members):
+        if mem:
+            winner[b] = min(mem, key=lambda q: (abs(float(flat[q])), q))
+            value[b] = flat[winner[b]]
+    codes = np.zeros(nb, dtype=np.int8)
+    scales = np.zeros(M // 64, dtype=np.uint16)
+    per = 4 * K
+    for rb in range(M // 64):
+        v = value[rb * per:(rb + 1) * per]
+        mx = np.float32(np.max(np.abs(v)))
+        s16 = np.float16(mx / np.float32(127.0))
+        scales[rb] = s16.view(np.uint16)
+        s = Fraction(float(s16))
+        if s != 0:
+            for q in range(per):
+                a = Fraction(float(abs(v[q])))
+                n = min(127, int(a / s))  # floor of a non-negative rational
+                codes[rb * per + q] = -n if v[q] < 0 else n
+    return codes, scales, winner
+
+
+def decode_amm(codes, scales, M: int, K: int, seed: int = 0, depth: int = 2) -> np.ndarray:
+    """W_hat: per weight the code of largest magnitude over the rows, ties to
+    the lowest row, times the block scale."""
+    out = np.zeros((M, K), dtype=np.float64)
+    for i in range(M):
+        s = float(np.uint16(scales[i // 64]).view(np.float16))
+        for j in range(K):
+            cs = [int(codes[bucket_of_amm(K, seed, depth, rho, i, j)]) for rho in range(depth)]
+            best = cs[0]
+            for c in cs[1:]:
+                if abs(c) > abs(best):
+                    best = c
+            out[i, j] = best * s
+    return out
