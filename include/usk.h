@@ -37,6 +37,22 @@
  *   Code: clamp(rint_half_even(v / float(s16)), -127, 127); 0 when s16 == 0.
  *   Decode: w_hat = float(code) * float(s16) (exact in fp32).
  *
+ * FORMAT 2 (multi-row AbsMaxMin; Metodologia §1: the sketch state keeps the
+ * member of SMALLEST absolute value per bucket, several independently hashed
+ * sketch rows are kept, decompression takes the MAX, so every rebuilt weight
+ * is the original or one of smaller magnitude).  Same geometry, scales and
+ * storage size as format 1 (0.5 bit/weight); depth D in {1, 2, 4}:
+ *   Hash row rho in [0, D) of tile tile_id: z = SplitMix64 output number
+ *     tile_id*D + rho + 1, A, C, h and slot as above, class = (o + r) mod (32/D),
+ *     b = rho*(1024/D) + (slot*(32/D) + class)*8 + c % 8   (D = 1: the format-1 hash).
+ *   Selection: every weight updates its bucket in each hash row; a bucket keeps
+ *   the signed value of its member with the smallest |w|, ties to the smallest
+ *   row-major index; an empty bucket keeps 0.  No importance weighting.
+ *   Code: sign(v) * min(127, floor(|v| / float(s16))) (toward zero, so
+ *   |code * s16| <= |v|); 0 when s16 == 0.
+ *   Decode: w_hat = float(c) * float(s16), c = the code of largest magnitude
+ *   among the weight's D buckets, ties to the lowest row.  |w_hat| <= |w|.
+ *
  * CONVENTIONS
  *   - All array pointers are DEVICE pointers owned by the caller; the library
  *     allocates no memory and keeps no state beyond cached kernel attributes.
@@ -65,7 +81,9 @@ extern "C" {
 #define USK_API
 #endif
 
-#define USK_FORMAT_VERSION 1
+#define USK_FORMAT_MAXKEY 1     /* format 1: one hash row, largest key kept   */
+#define USK_FORMAT_ABSMAXMIN 2  /* format 2: multi-row AbsMaxMin              */
+#define USK_FORMAT_VERSION 2    /* highest format this library builds and reads */
 #define USK_ROWS_PER_BLOCK 64
 #define USK_TILE_COLS 256
 #define USK_WEIGHTS_PER_BUCKET 16
@@ -82,7 +100,7 @@ typedef enum {
   USK_ERR_DTYPE = 3,           /* unknown usk_dtype                              */
   USK_ERR_BATCH = 4,           /* batch outside the call's range                 */
   USK_ERR_WORKSPACE = 5,       /* workspace missing or too small                 */
-  USK_ERR_PARAMS = 6,          /* params NULL or wrong format version            */
+  USK_ERR_PARAMS = 6,          /* params NULL, unknown format, bad depth or flags */
   USK_ERR_CUDA = 7,            /* a CUDA runtime call or a launch failed         */
   USK_ERR_NONFINITE = 8,       /* (flag decoding) non-finite weight              */
   USK_ERR_TIMEOUT = 9,         /* (flag decoding) a bounded device wait gave up  */
@@ -99,19 +117,26 @@ typedef enum {
 
 typedef enum { USK_F32 = 0, USK_BF16 = 1 } usk_dtype;
 
-/* Build parameters: version must be USK_FORMAT_VERSION; flags must be 0. */
+/* Build parameters.  version: USK_FORMAT_MAXKEY or USK_FORMAT_ABSMAXMIN;
+ * flags and reserved must be 0; depth = hash rows: 0 or 1 for format 1, 1, 2
+ * or 4 for format 2.  Anything else: USK_ERR_PARAMS. */
 typedef struct {
   uint32_t version;
   uint32_t flags;
   uint64_t seed;
+  uint32_t depth;
+  uint32_t reserved;
 } usk_params;
 
-/* A built sketch (device pointers, caller-owned). */
+/* A built sketch (device pointers, caller-owned).  version / depth as built
+ * (version 0 is read as format 1; depth 0 as 1). */
 typedef struct {
   int64_t M, K;
   uint64_t seed;
   const int8_t* codes;     /* [M*K/16], 16-byte aligned */
   const uint16_t* scales;  /* [M/64] binary16 bits      */
+  uint32_t version;
+  uint32_t depth;
 } usk_sketch;
 
 /* Storage of a sketch: code_bytes = M*K/16, scale_bytes = 2*M/64.
@@ -124,7 +149,8 @@ USK_API usk_status usk_sizes(int64_t M, int64_t K, size_t* code_bytes, size_t* s
  *              (ldw % 4 == 0 for fp32, % 8 == 0 for bf16).
  *   importance [K] fp32 per input column, or NULL for all ones.  Values must
  *              be finite with the sign bit clear (else USK_FLAG_BAD_IMPORTANCE).
- *   params     version + seed of the hash.
+ *              Format 2 takes no importance: non-NULL is USK_ERR_PARAMS.
+ *   params     format, depth and seed of the hash.
  *   codes      [M*K/16] int8 output, 16-byte aligned.   scales [M/64] output.
  *   d_status   optional device word for USK_FLAG_* bits.
  * M == 0 is a no-op; K == 0 writes zero scales.  Codes and scales are
@@ -137,10 +163,12 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
  * fly: every weight is rehashed and its bucket gathered; W_hat is never stored).
  *   x  [batch, K] row-major, fp32 or bf16 per xdtype, 16-byte aligned.
  *   y  [batch, M] fp32 output (y[t*M + i] = sum_j w_hat[i][j] x[t][j]).
- * bf16 x at batch <= 4: integer tensor path, exact sum of code * x (x split
+ * Single-row sketches (format 1, or format 2 at depth 1), bf16 x at batch <= 4:
+ * integer tensor path, exact sum of code * x (x split
  * into byte digit planes per block; elements outside 2^22 of the block's
  * largest are added by an exact correction), one rounding to fp32 at the end.
- * Other batches: bf16 tensor path, exact products, fp32 accumulation; fp32 x
+ * Other batches and multi-row sketches: bf16 tensor path (each hash row
+ * gathered, the code of largest magnitude kept), exact products, fp32 accumulation; fp32 x
  * is split into two bf16 terms (|error| <= 2^-16 |x| per element).
  * batch == 0 or M == 0 is a no-op; K == 0 writes y = 0.  Deterministic for a
  * given shape (the summation order is fixed). */
@@ -175,8 +203,10 @@ USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block)
 
 /* Test hook: choose the usk_gemv path (0 = automatic, 1 = bf16 tensor path,
  * 2 = integer path with thread-block clusters where eligible, 3 = integer
- * row-slab path where eligible: bf16 x and batch * K <= 16384).  Every path
- * gives results within the products' tolerance; process-wide. */
+ * row-slab path where eligible: bf16 x and batch * K <= 16384; single-row
+ * sketches only), 4 = bf16 path with x fragments from global memory (bf16 x,
+ * batch <= 8).  Every path gives results within the products' tolerance;
+ * process-wide. */
 USK_API void usk_debug_set_gemv_path(int path);
 
 /* Test hook: rows per thread block of the row-slab path (16, 32 or 64; any

@@ -1,7 +1,8 @@
 """UltraSketchLLM sketch weights on NVIDIA B200 (sm_100a).
 
 Thin Python face of libusk.so (C ABI in include/usk.h): ``usk_build`` compresses
-a weight matrix into a 0.5 bit/weight hashed sketch; ``usk_gemv`` (batch 1-15)
+a weight matrix into a 0.5 bit/weight hashed sketch (format 1: one hash row,
+largest key kept; format 2: the multi-row AbsMaxMin sketch); ``usk_gemv`` (batch 1-15)
 and ``usk_gemm`` (batch 16-256) multiply the sketch with activations, rebuilding
 every weight on the fly.  PyTorch supplies device memory and streams only.
 """
@@ -10,6 +11,8 @@ from ._native import (  # noqa: F401
     FLAG_NONFINITE_W,
     FLAG_SCALE_OVERFLOW,
     FLAG_TIMEOUT,
+    FORMAT_ABSMAXMIN,
+    FORMAT_MAXKEY,
     FORMAT_VERSION,
     GEMM_MAX_BATCH,
     GEMM_MIN_BATCH,

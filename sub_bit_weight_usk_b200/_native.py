@@ -19,7 +19,9 @@ LIB_PATH = os.path.join(_PKG, "libusk.so")
 USK_OK = 0
 USK_F32 = 0
 USK_BF16 = 1
-FORMAT_VERSION = 1
+FORMAT_MAXKEY = 1      # format 1: one hash row, the largest key kept per bucket
+FORMAT_ABSMAXMIN = 2   # format 2: multi-row AbsMaxMin (smallest |w| kept, largest over rows decoded)
+FORMAT_VERSION = 2     # highest format the library builds and reads
 GEMV_MAX_BATCH = 15
 GEMM_MIN_BATCH = 16
 GEMM_MAX_BATCH = 256
@@ -43,12 +45,14 @@ class UskError(RuntimeError):
 
 
 class UskParams(ctypes.Structure):
-    _fields_ = [("version", ctypes.c_uint32), ("flags", ctypes.c_uint32), ("seed", ctypes.c_uint64)]
+    _fields_ = [("version", ctypes.c_uint32), ("flags", ctypes.c_uint32), ("seed", ctypes.c_uint64),
+                ("depth", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
 
 
 class UskSketchC(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int64), ("seed", ctypes.c_uint64),
-                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("version", ctypes.c_uint32), ("depth", ctypes.c_uint32)]
 
 
 _lib = None
@@ -141,24 +145,30 @@ def usk_sizes(M: int, K: int):
 
 @dataclass
 class Sketch:
-    """A built sketch: int8 codes [M*K/16] and binary16 scales [M/64] on the GPU."""
+    """A built sketch: int8 codes [M*K/16] and binary16 scales [M/64] on the GPU,
+    with its format (1 or 2) and number of hash rows."""
     M: int
     K: int
     seed: int
     codes: torch.Tensor
     scales: torch.Tensor  # int16 storage of binary16 bit patterns
+    version: int = FORMAT_MAXKEY
+    depth: int = 1
 
     def as_c(self) -> UskSketchC:
         return UskSketchC(self.M, self.K, self.seed & (2**64 - 1), self.codes.data_ptr() if self.codes.numel() else None,
-                          self.scales.data_ptr() if self.scales.numel() else None)
+                          self.scales.data_ptr() if self.scales.numel() else None, self.version, self.depth)
 
 
 def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int = 0,
               codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
-              status: torch.Tensor | None = None, stream=None) -> Sketch:
+              status: torch.Tensor | None = None, stream=None, version: int = FORMAT_MAXKEY,
+              depth: int = 1) -> Sketch:
     """Sketch of W [M, K] (bf16 or fp32, CUDA).  Outputs are allocated with torch
     when not given.  `status` is an optional int32 CUDA tensor of 1 element into
-    which device-detected USK_FLAG_* bits are OR-ed."""
+    which device-detected USK_FLAG_* bits are OR-ed.  version=FORMAT_ABSMAXMIN
+    builds the multi-row AbsMaxMin sketch with `depth` (1, 2 or 4) hash rows
+    (no importance)."""
     _need_cuda(W, importance, codes, scales, status)
     if W.dim() != 2 or W.stride(1) != 1:
         raise ValueError("W must be a 2-D row-major tensor")
@@ -170,12 +180,12 @@ def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int
         scales = torch.empty(max(M // 64, 1), dtype=torch.int16, device=W.device)[: M // 64]
     if importance is not None and (importance.dtype != torch.float32 or not importance.is_contiguous()):
         raise TypeError("importance must be a contiguous float32 tensor")
-    p = UskParams(FORMAT_VERSION, 0, seed & (2**64 - 1))
+    p = UskParams(version, 0, seed & (2**64 - 1), depth, 0)
     st = load_library().usk_build(_ptr(W), _dtype_code(W), M, K, W.stride(0), _ptr(importance), ctypes.byref(p),
                                   _ptr(codes) if nb else None, _ptr(scales) if M // 64 else None,
                                   _ptr(status), _stream(stream))
     _check(st, "usk_build")
-    return Sketch(M, K, seed, codes, scales)
+    return Sketch(M, K, seed, codes, scales, version, depth)
 
 
 def usk_gemv(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,

@@ -10,12 +10,16 @@ namespace usk {
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
                          cudaStream_t stream, int cluster_override, int inject);
+cudaError_t launch_build_amm(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed, int depth,
+                             int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
+                             int cluster_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject);
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth);
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
-                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject);
-bool gemm_supported(int64_t K, int batch);
+                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
+                        int depth);
+bool gemm_supported(int64_t K, int batch, int depth);
 }  // namespace usk
 
 namespace {
@@ -29,8 +33,16 @@ usk_status check_shape(int64_t M, int64_t K) {
   return USK_OK;
 }
 
+// Hash rows of a sketch or a build request; 0 if the (format, depth) pair is not valid.
+int format_depth(uint32_t version, uint32_t depth) {
+  if (version == 0 || version == USK_FORMAT_MAXKEY) return depth <= 1 ? 1 : 0;
+  if (version == USK_FORMAT_ABSMAXMIN) return (depth == 1 || depth == 2 || depth == 4) ? static_cast<int>(depth) : 0;
+  return 0;
+}
+
 usk_status check_sketch(const usk_sketch* s) {
   if (!s) return USK_ERR_NULL;
+  if (format_depth(s->version, s->depth) == 0) return USK_ERR_PARAMS;
   usk_status st = check_shape(s->M, s->K);
   if (st != USK_OK) return st;
   if (s->M > 0 && s->K > 0) {
@@ -65,7 +77,7 @@ USK_API const char* usk_status_str(usk_status status) {
     case USK_ERR_DTYPE: return "unknown dtype";
     case USK_ERR_BATCH: return "batch outside the range of this call";
     case USK_ERR_WORKSPACE: return "workspace missing or too small";
-    case USK_ERR_PARAMS: return "params NULL, wrong format version or non-zero flags";
+    case USK_ERR_PARAMS: return "params NULL, unknown format, bad depth, non-zero flags or importance with format 2";
     case USK_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     case USK_ERR_NONFINITE: return "non-finite weight";
     case USK_ERR_TIMEOUT: return "a bounded device wait gave up";
@@ -92,7 +104,12 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (st != USK_OK) return st;
   if (wdtype != USK_F32 && wdtype != USK_BF16) return USK_ERR_DTYPE;
   if (!params) return USK_ERR_PARAMS;
-  if (params->version != USK_FORMAT_VERSION || params->flags != 0) return USK_ERR_PARAMS;
+  if (params->flags != 0 || params->reserved != 0) return USK_ERR_PARAMS;
+  if (params->version != USK_FORMAT_MAXKEY && params->version != USK_FORMAT_ABSMAXMIN) return USK_ERR_PARAMS;
+  const int depth = format_depth(params->version, params->depth);
+  if (depth == 0) return USK_ERR_PARAMS;
+  const bool amm = params->version == USK_FORMAT_ABSMAXMIN;
+  if (amm && importance) return USK_ERR_PARAMS;
   if (M == 0) return USK_OK;
   if (!scales) return USK_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(scales) & 1u) != 0) return USK_ERR_ALIGN;
@@ -103,8 +120,10 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (!aligned16(W) || !aligned16(codes)) return USK_ERR_ALIGN;
   if (ldw % (wdtype == USK_BF16 ? 8 : 4) != 0) return USK_ERR_ALIGN;
   if (importance && !aligned16(importance)) return USK_ERR_ALIGN;
-  cudaError_t e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes,
-                                    scales, d_status, s, g_build_cluster, g_inject == 1);
+  cudaError_t e = amm ? usk::launch_build_amm(W, wdtype == USK_BF16, M, K, ldw, params->seed, depth, codes, scales,
+                                               d_status, s, g_build_cluster, g_inject == 1)
+                      : usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes,
+                                          scales, d_status, s, g_build_cluster, g_inject == 1);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -127,7 +146,7 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
   cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
                                    xdtype == USK_F32, static_cast<int>(batch), y, d_status,
                                    (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows,
-                                   g_inject == 3);
+                                   g_inject == 3, format_depth(sketch->version, sketch->depth));
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -144,7 +163,8 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   usk_status st = check_sketch(sketch);
   if (st != USK_OK) return st;
   if (batch < USK_GEMM_MIN_BATCH || batch > USK_GEMM_MAX_BATCH || batch % 16 != 0) return USK_ERR_BATCH;
-  if (!usk::gemm_supported(sketch->K, static_cast<int>(batch))) return USK_ERR_SHAPE;
+  const int depth = format_depth(sketch->version, sketch->depth);
+  if (!usk::gemm_supported(sketch->K, static_cast<int>(batch), depth)) return USK_ERR_SHAPE;
   if (sketch->M == 0) return USK_OK;
   if (!y) return USK_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -153,7 +173,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   if (!x_bf16) return USK_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(y)) return USK_ERR_ALIGN;
   cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
-                                   static_cast<int>(batch), y, d_status, s, g_inject == 2);
+                                   static_cast<int>(batch), y, d_status, s, g_inject == 2, depth);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }

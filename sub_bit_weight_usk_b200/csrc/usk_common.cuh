@@ -268,6 +268,27 @@ __device__ __forceinline__ uint32_t i8pair_to_bf16x2(uint32_t w) {
   return r;
 }
 
+// Format 2 (multi-row AbsMaxMin) decode: per 16-bit half, the bf16 code of
+// larger magnitude of a and b (integer codes, |code| <= 127); ties keep a, the
+// lower hash row.  (a | 0x8000) - |b| per half never borrows across halves and
+// keeps bit 15 exactly when |a| >= |b| (bf16 magnitude bits order like values).
+__device__ __forceinline__ uint32_t absmax_sel_bf16x2(uint32_t a, uint32_t b) {
+  const uint32_t d = (a | 0x80008000u) - (b & 0x7FFF7FFFu);
+  const uint32_t m = ((d >> 15) & 0x00010001u) * 0xFFFFu;
+  return (a & m) | (b & ~m);
+}
+
+__device__ __forceinline__ uint4 absmax_sel(uint4 a, uint4 b) {
+  return make_uint4(absmax_sel_bf16x2(a.x, b.x), absmax_sel_bf16x2(a.y, b.y), absmax_sel_bf16x2(a.z, b.z),
+                    absmax_sel_bf16x2(a.w, b.w));
+}
+
+// Key of hash row rho of tile `tile_id` in a depth-D sketch (format 2): the
+// SplitMix64 output tile_id * D + rho + 1; D = 1 gives the format-1 key.
+__host__ __device__ __forceinline__ uint2 row_key(uint64_t seed, uint64_t tile_id, int depth, int rho) {
+  return tile_key(seed, tile_id * static_cast<uint64_t>(depth) + static_cast<uint64_t>(rho));
+}
+
 // ---- integer tensor path helpers (mma.sync m16n8k32 s8)
 
 __device__ __forceinline__ void imma_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -22,6 +22,10 @@
 //    the 16 weights straight into tensor memory (tcgen05.st, its row is its
 //    TMEM lane): the A operand never touches shared memory, which leaves the
 //    shared-memory bandwidth to the code gathers and the B (x) operand.
+//    For a multi-row AbsMaxMin sketch (format 2, depth D) the thread gathers
+//    the octet from each of the D hash rows (segments of 2048/D bytes of the
+//    widened tile, class = (octet + row) mod 32/D) and keeps, per weight, the
+//    code of largest magnitude (integer select on the bf16 pairs).
 //  * 1 copy warp: per chunk, as soon as the stage is free, one tensor copy of
 //    the x tile (B operand, 128-byte swizzle) onto the stage's "full" barrier.
 //  * I = 1, 2 or 4 MMA warps: warp i takes the chunks c = i (mod I); once the
@@ -79,14 +83,14 @@ struct GemmLayout {
   uint32_t b, cbf, codes, keys, bars, misc, total;
 };
 
-__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S) {
+__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int depth) {
   GemmLayout L;
   L.b = 0;  // [S][N x 64] bf16, SW128; after the main loop the K-split partials [N][128] fp32
   const uint32_t ring = static_cast<uint32_t>(S) * N * kBK * 2, parts = static_cast<uint32_t>(N) * kBM * 4;
   L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [kTileRing][2][1024]
   L.codes = L.cbf + kTileRing * 2u * 1024u * 2u;                       // int8 [2][tcta][1024]
-  L.keys = L.codes + 2u * tcta * 1024u;                                // uint2 [2][tcta]
-  L.bars = (L.keys + 2u * tcta * 8u + 7u) & ~7u;  // full[S], empty[S], codes, done, ready[ring], free[ring]
+  L.keys = L.codes + 2u * tcta * 1024u;                                // uint2 [2][tcta][depth]
+  L.bars = (L.keys + 2u * tcta * depth * 8u + 7u) & ~7u;  // full[S], empty[S], codes, done, ready[ring], free[ring]
   L.misc = L.bars + (2 * S + 2 + 2 * kTileRing) * 8;                   // tmem holder, abort
   L.total = L.misc + 16;
   return L;
@@ -160,7 +164,12 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// D = hash rows of the sketch (1: format 1 or format 2 at depth 1; 2, 4: the
+// multi-row AbsMaxMin sketch: the decoders gather every row and keep the code
+// of largest magnitude)
+template <int D>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
+  constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
   extern __shared__ __align__(16) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ks = static_cast<int>(cluster.block_rank());
@@ -176,7 +185,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   const int tcta = t_end - t_begin;
   const int nk = tcta * (kTileCols / kBK);  // 64-column chunks
   const int S = a.S;
-  const GemmLayout L = gemm_layout(a.N, tcta, S);
+  const GemmLayout L = gemm_layout(a.N, tcta, S, D);
   const uint32_t bstage = static_cast<uint32_t>(a.N) * kBK * 2;
   const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * S, codes_bar = empty_s + 8 * S;
   const uint32_t done_bar = codes_bar + 8, ready_s = done_bar + 8, free_s = ready_s + 8 * kTileRing;
@@ -218,9 +227,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
                  "r"(a.tmem_cols)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  } else if (tid < 2 * tcta) {
-    const int rbl = tid / tcta, tl = tid % tcta;
-    keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb0 + rbl) * a.T + t_begin + tl);
+  } else if (tid < 2 * tcta * D) {
+    const int rbl = tid / (tcta * D), tl = (tid / D) % tcta;
+    keytab[tid] = row_key(a.seed, static_cast<uint64_t>(rb0 + rbl) * a.T + t_begin + tl, D, tid % D);
   }
   tc_fence_before();
   __syncthreads();
@@ -256,9 +265,14 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
         }
         tc_fence_after();
       }
-      const uint2 hk = keytab[rbl * tcta + t];
       const uint32_t ob = static_cast<uint32_t>(8 * g);
-      uint32_t h = hk.x * (32u * r + ob) + hk.y;
+      uint2 hk[D];
+      uint32_t h[D];
+#pragma unroll
+      for (int rho = 0; rho < D; ++rho) {
+        hk[rho] = keytab[(rbl * tcta + t) * D + rho];
+        h[rho] = hk[rho].x * (32u * r + ob) + hk[rho].y;
+      }
       const uint32_t tile_codes = s0 + L.cbf + q * 4096u + rbl * 2048u;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {  // octets 4hh .. 4hh + 3 -> columns 16hh .. 16hh + 15 of the stage
@@ -267,14 +281,20 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
         for (int j = 0; j < 4; ++j) {
           uint4 w = make_uint4(0u, 0u, 0u, 0u);
           if (row_ok) {
-            const uint32_t cls = (ob + 4u * hh + j + r) & 31u;
-            w = lds128(tile_codes + ((h >> 30) * 32u + cls) * 16u);
+            const uint32_t cls = (ob + 4u * hh + j + r) & (kNc - 1u);
+#pragma unroll
+            for (int rho = 0; rho < D; ++rho) {
+              const uint4 u = lds128(tile_codes + static_cast<uint32_t>(rho) * (2048u / D) +
+                                     ((h[rho] >> 30) * kNc + cls) * 16u);
+              w = rho == 0 ? u : absmax_sel(w, u);
+            }
           }
           v[4 * j + 0] = w.x;
           v[4 * j + 1] = w.y;
           v[4 * j + 2] = w.z;
           v[4 * j + 3] = w.w;
-          h += hk.x;
+#pragma unroll
+          for (int rho = 0; rho < D; ++rho) h[rho] += hk[rho].x;
         }
         tmem_st(a_taddr + s * 32u + 16u * hh, v);
       }
@@ -446,29 +466,29 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N)
 // mbarrier has one in-order waiter per role.  Otherwise consecutive uses of a
 // stage belong to different warps, and a warp running ahead can take a
 // completed phase of use n - 2 for use n (a phase wait only tells parity).
-static int gemm_stages(int N, int tpb) {
+static int gemm_stages(int N, int tpb, int depth) {
   const uint32_t cols = gemm_tmem_cols(N);
   const uint32_t smem_cap = cols == 256u ? 233472u / 2u - 1024u : kSmemLimit;
   int S = static_cast<int>((cols - gemm_a_col(N)) / 32u);
   if (S > kMaxStages) S = kMaxStages;
   S &= ~3;
-  while (S >= 4 && gemm_layout(N, tpb, S).total + 1024u > smem_cap) S -= 4;
+  while (S >= 4 && gemm_layout(N, tpb, S, depth).total + 1024u > smem_cap) S -= 4;
   return S >= 4 ? S : 0;
 }
 
 // Largest number of tiles per block (codes staged up front) that still leaves
 // a four-stage pipeline for batch N.
-static int gemm_max_tiles(int N) {
+static int gemm_max_tiles(int N, int depth) {
   int t = kMaxTiles;
-  while (t > 1 && gemm_stages(N, t) == 0) --t;
+  while (t > 1 && gemm_stages(N, t, depth) == 0) --t;
   return t;
 }
 
 // Dynamic shared memory of a launch: the layout, padded so that no more blocks
 // share an SM than its 512 tensor-memory columns hold (a block waiting in
 // tcgen05.alloc for a co-resident block of its own cluster would never proceed).
-static uint32_t gemm_smem_bytes(int N, int tpb, int S) {
-  const uint32_t smem = gemm_layout(N, tpb, S).total + 1024u;  // + alignment slack
+static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth) {
+  const uint32_t smem = gemm_layout(N, tpb, S, depth).total + 1024u;  // + alignment slack
   const uint32_t max_blocks = 512u / gemm_tmem_cols(N);
   const uint32_t floor_bytes = 233472u / (max_blocks + 1u) + 1u - 1024u;  // 228 KiB per SM, 1 KiB reserved per block
   return smem > floor_bytes ? smem : floor_bytes;
@@ -479,8 +499,8 @@ static uint32_t gemm_smem_bytes(int N, int tpb, int S) {
 // pipeline fill, epilogue and the cluster reduction: 4 to 5 us measured against
 // about 1.3 us per tile at batch 16), within the shared-memory bound on tiles
 // per block and clusters of at most 16.
-static int gemm_splits(int64_t m_tiles, int T, int N, int sms) {
-  const int max_tiles = gemm_max_tiles(N);
+static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth) {
+  const int max_tiles = gemm_max_tiles(N, depth);
   const int64_t slots = static_cast<int64_t>(sms) * (512 / static_cast<int>(gemm_tmem_cols(N)));
   int best = -1;
   int64_t best_cost = -1;
@@ -501,12 +521,14 @@ static int gemm_splits(int64_t m_tiles, int T, int N, int sms) {
 
 // Whether K fits: at most 16 blocks along K, each staging the codes of up to
 // gemm_max_tiles(batch) tiles (32 for every batch: K <= 131072).
-bool gemm_supported(int64_t K, int batch) {
-  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch));
+bool gemm_supported(int64_t K, int batch, int depth) {
+  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch, depth));
 }
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
-                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject) {
+                        const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
+                        int depth) {
+  if (depth != 1 && depth != 2 && depth != 4) return cudaErrorInvalidValue;
   GemmArgs a;
   a.codes = codes; a.scales = scales; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status; a.inject = inject;
@@ -515,15 +537,15 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   const int64_t m_tiles = (M + kBM - 1) / kBM;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  a.splits = gemm_splits(m_tiles, a.T, batch, sms);
+  a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth);
   if (a.splits < 1) return cudaErrorInvalidValue;  // K beyond 16 blocks x the tiles one block can stage
   a.tmem_cols = gemm_tmem_cols(batch);
   a.a_col = gemm_a_col(batch);
   a.I = gemm_issuers(batch);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
-  a.S = gemm_stages(batch, tcta_max);
+  a.S = gemm_stages(batch, tcta_max, depth);
   if (a.S < 4 || a.S % 4 != 0) return cudaErrorInvalidValue;
-  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S);
+  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth);
   // tensor map over x [batch, K] bf16: one 64-column x batch box per chunk, 128-byte swizzle
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -536,11 +558,11 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  auto kern = depth == 4 ? gemm_kernel<4> : (depth == 2 ? gemm_kernel<2> : gemm_kernel<1>);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.splits > 8) {
-    e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
@@ -555,7 +577,7 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemm_kernel, a, xmap);
+  return cudaLaunchKernelEx(&cfg, kern, a, xmap);
 }
 
 }  // namespace usk

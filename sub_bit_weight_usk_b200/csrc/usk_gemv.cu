@@ -47,7 +47,7 @@ struct GemvArgs {
 constexpr int kGemvThreads = 256;
 
 // Shared memory (bytes):
-//   key table  [tpc] uint2, padded to 16
+//   key table  [tpc][depth] uint2, padded to 16
 //   codes      [tpc][1024] bf16 (2 KiB per tile)
 //   x slice    [nvalid rows][tpc * 512 + 16] bf16 (rows padded by 16 B: conflict-free)
 //   block sums [batch][64] fp32
@@ -57,11 +57,11 @@ struct GemvLayout {
   uint32_t keys, codes, xs, xrow, stage_end, parts, cta, total;
 };
 
-__host__ __device__ inline GemvLayout gemv_layout(int tpc, int nb, int batch, bool xf32) {
+__host__ __device__ inline GemvLayout gemv_layout(int tpc, int nb, int batch, bool xf32, int depth) {
   GemvLayout L;
   const uint32_t nvalid = static_cast<uint32_t>(xf32 ? 2 * batch : batch);
   L.keys = 0;
-  L.codes = (static_cast<uint32_t>(tpc) * 8u + 15u) / 16u * 16u;
+  L.codes = (static_cast<uint32_t>(tpc * depth) * 8u + 15u) / 16u * 16u;
   L.xs = L.codes + static_cast<uint32_t>(tpc) * 2048u;
   L.xrow = static_cast<uint32_t>(tpc) * 512u + 16u;
   L.stage_end = L.xs + nvalid * L.xrow;
@@ -79,8 +79,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2_from_i8(int lo, int hi) {
 
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t*>(&v); }
 
-template <int NB, bool XF32>
+// D = hash rows (1: format 1 or format 2 at depth 1; 2, 4: the multi-row
+// AbsMaxMin sketch, each row gathered from its own 2048/D-byte segment of the
+// tile and reduced to the code of largest magnitude)
+template <int NB, bool XF32, int D>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
+  constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
   extern __shared__ __align__(16) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -89,12 +93,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);  // >= 1 by construction of C
   const int nvalid = XF32 ? 2 * a.batch : a.batch;
-  const GemvLayout L = gemv_layout(a.tpc, NB, a.batch, XF32);
+  const GemvLayout L = gemv_layout(a.tpc, NB, a.batch, XF32, D);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   const uint32_t sm_s = smem_u32(sm);
 
   // ---- stage: hash keys, codes (int8 -> bf16) and the x slice, all loads in flight at once
-  if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
+  if (tid < nt * D) keytab[tid] = row_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid / D, D, tid % D);
   {
     const int8_t* csrc = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
     const int ncode = nt * 64;                                   // 16-byte code chunks
@@ -159,10 +163,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   // ---- main loop
   const int g = lane >> 2, t = lane & 3;
   const int o = 8 * (warp >> 1) + (warp & 1) + 2 * t;  // this lane's octet in every tile
-  const uint32_t c0 = static_cast<uint32_t>(o + g) & 31u;
+  const uint32_t c0 = static_cast<uint32_t>(o + g) & (kNc - 1u);
   uint32_t cls16[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) cls16[k] = ((c0 + 8u * k) & 31u) * 16u;
+  for (int k = 0; k < 4; ++k) cls16[k] = ((c0 + 8u * k) & (kNc - 1u)) * 16u;
   const uint32_t codes_s = sm_s + L.codes;
 
   float d[4][NB][4];
@@ -174,7 +178,6 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
       for (int e = 0; e < 4; ++e) d[mb][nb][e] = 0.0f;
 
   for (int tt = 0; tt < nt; ++tt) {
-    const uint2 hk = keytab[tt];
     // B fragments (x) of this tile for the lane's octet: n = 8 nb + g
     uint32_t bq[NB][4];
 #pragma unroll
@@ -185,14 +188,26 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
       bq[nb][0] = v.x; bq[nb][1] = v.y; bq[nb][2] = v.z; bq[nb][3] = v.w;
     }
     const uint32_t tile_s = codes_s + tt * 2048u;
-    const uint32_t h = hk.x * (32u * g + o) + hk.y;
-    const uint32_t d512 = hk.x * 512u, d256 = hk.x * 256u;
+    uint2 hk[D];
+    uint32_t h[D];
+#pragma unroll
+    for (int rho = 0; rho < D; ++rho) {
+      hk[rho] = keytab[tt * D + rho];
+      h[rho] = hk[rho].x * (32u * g + o) + hk[rho].y;
+    }
 #pragma unroll
     for (int mb = 0; mb < 4; ++mb) {
-      const uint32_t h0 = h + mb * d512;
-      const uint32_t h1 = h0 + d256;
-      const uint4 q0 = lds128(tile_s + (h0 >> 30) * 512u + cls16[(2 * mb) & 3]);
-      const uint4 q1 = lds128(tile_s + (h1 >> 30) * 512u + cls16[(2 * mb + 1) & 3]);
+      uint4 q0 = make_uint4(0u, 0u, 0u, 0u), q1 = q0;
+#pragma unroll
+      for (int rho = 0; rho < D; ++rho) {
+        const uint32_t h0 = h[rho] + mb * (hk[rho].x * 512u);
+        const uint32_t h1 = h0 + hk[rho].x * 256u;
+        const uint32_t seg = tile_s + static_cast<uint32_t>(rho) * (2048u / D);
+        const uint4 u0 = lds128(seg + (h0 >> 30) * (kNc * 16u) + cls16[(2 * mb) & 3]);
+        const uint4 u1 = lds128(seg + (h1 >> 30) * (kNc * 16u) + cls16[(2 * mb + 1) & 3]);
+        q0 = rho == 0 ? u0 : absmax_sel(q0, u0);
+        q1 = rho == 0 ? u1 : absmax_sel(q1, u1);
+      }
 #pragma unroll
       for (int nb = 0; nb < NB; ++nb) {
         mma_bf16_16816(d[mb][nb], q0.x, q1.x, q0.y, q1.y, bq[nb][0], bq[nb][1]);
@@ -263,10 +278,10 @@ static GemvGeometry gemv_geometry(int64_t K, int tpc_override) {
   return g;
 }
 
-template <int NB, bool XF32>
+template <int NB, bool XF32, int D>
 static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32).total;
-  auto kern = gemv_kernel<NB, XF32>;
+  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32, D).total;
+  auto kern = gemv_kernel<NB, XF32, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -296,14 +311,31 @@ cudaError_t launch_gemv_slab(const int8_t* codes, const uint16_t* scales, int64_
 bool gemv_bf_supported(int64_t K, int batch, int tpc_override);
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject);
+                           int tpc_override, int inject, int depth);
+
+template <int D>
+static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaStream_t stream) {
+  const int rows = xf32 ? 2 * a.batch : a.batch;
+  const int nb = (rows + 7) / 8;
+  if (!xf32) {
+    if (nb == 1) return launch_gemv_t<1, false, D>(a, RB, stream);
+    return launch_gemv_t<2, false, D>(a, RB, stream);
+  }
+  switch (nb) {
+    case 1: return launch_gemv_t<1, true, D>(a, RB, stream);
+    case 2: return launch_gemv_t<2, true, D>(a, RB, stream);
+    case 3: return launch_gemv_t<3, true, D>(a, RB, stream);
+    default: return launch_gemv_t<4, true, D>(a, RB, stream);
+  }
+}
 
 // path: 0 = automatic, 1 = bf16 tensor path (staged x), 2 = integer path with
 // clusters, 3 = integer row-slab path (bf16 x, batch * K <= 16384), 4 = bf16
-// path with x fragments from global memory (bf16 x, batch <= 8)
+// path with x fragments from global memory (bf16 x, batch <= 8).  depth = hash
+// rows of the sketch: the integer paths read single-row sketches only.
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject) {
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // automatic choice (measured on B200, graphs of back-to-back calls):
@@ -311,16 +343,18 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   //  * batch >= 2, or batch 1 up to 4096 x 4096: bf16 with direct x fragments;
   //  * batch 1 with longer K or taller M: the integer cluster kernel (half the
   //    shared-memory gather bytes; its x preparation is amortised over more tiles)
-  const bool slab = path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms);
+  const bool slab = depth == 1 && (path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms));
   if (!xf32 && slab && slab_supported(K, batch))
     return launch_gemv_slab(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl,
                             stream, rows_override, inject);
-  const bool direct = path == 4 || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
+  // multi-row sketches: the direct path unless the staged one is asked for
+  const bool direct =
+      path == 4 || (depth > 1 && path != 1) || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
   if (!xf32 && direct && gemv_bf_supported(K, batch, tpc_override))
     return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
-                          tpc_override, inject);
+                          tpc_override, inject, depth);
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
-  const bool i8_ok = !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
+  const bool i8_ok = depth == 1 && !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
   if (i8_ok && path != 1)
     return launch_gemv_i8(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, geo.T,
                           geo.C, geo.tpc, pdl, stream, inject);
@@ -329,18 +363,9 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.M = M; a.K = K; a.seed = seed;
   a.T = geo.T; a.C = geo.C; a.tpc = geo.tpc; a.batch = batch;
   const int64_t RB = M / kRowsPerBlock;
-  const int rows = xf32 ? 2 * batch : batch;
-  const int nb = (rows + 7) / 8;
-  if (!xf32) {
-    if (nb == 1) return launch_gemv_t<1, false>(a, RB, stream);
-    return launch_gemv_t<2, false>(a, RB, stream);
-  }
-  switch (nb) {
-    case 1: return launch_gemv_t<1, true>(a, RB, stream);
-    case 2: return launch_gemv_t<2, true>(a, RB, stream);
-    case 3: return launch_gemv_t<3, true>(a, RB, stream);
-    default: return launch_gemv_t<4, true>(a, RB, stream);
-  }
+  if (depth == 2) return launch_staged<2>(a, xf32, RB, stream);
+  if (depth == 4) return launch_staged<4>(a, xf32, RB, stream);
+  return launch_staged<1>(a, xf32, RB, stream);
 }
 
 }  // namespace usk

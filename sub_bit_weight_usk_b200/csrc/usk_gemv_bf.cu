@@ -23,6 +23,11 @@
 //    cover rows g, g+1 and octets o0 + 2t, the 8 lanes hit 8 distinct 16-byte
 //    bank groups.  Two accumulator sets (even and odd tiles) double the
 //    independent MMA chains.
+//  * Multi-row AbsMaxMin sketches (format 2, depth D): each hash row is
+//    gathered the same way from its own 2048/D-byte segment of the widened
+//    tile (class = (o + row) mod 32/D keeps a quarter warp on 8 distinct bank
+//    groups), and the D words reduce to the code of largest magnitude with four
+//    integer instructions per bf16 pair before the MMA.
 //  * fp32 accumulation of exact bf16 products; the 8 warps' sums are added in
 //    a fixed order, then every block but the first writes its 64 x batch
 //    partials into the first block's shared memory with st.async, which counts
@@ -56,11 +61,11 @@ struct GemvBfLayout {
   uint32_t cbf, keys, red, push, bars, total;
 };
 
-__host__ __device__ inline GemvBfLayout gemv_bf_layout(int tpc, int batch, int C) {
+__host__ __device__ inline GemvBfLayout gemv_bf_layout(int tpc, int batch, int C, int depth) {
   GemvBfLayout L;
   L.cbf = 0;                                                       // bf16 [tpc][1024]
-  L.keys = L.cbf + static_cast<uint32_t>(tpc) * 2048u;             // uint2 [tpc]
-  L.red = (L.keys + static_cast<uint32_t>(tpc) * 8u + 15u) & ~15u;  // fp32 [8 warps][batch][64]
+  L.keys = L.cbf + static_cast<uint32_t>(tpc) * 2048u;             // uint2 [tpc][depth]
+  L.red = (L.keys + static_cast<uint32_t>(tpc * depth) * 8u + 15u) & ~15u;  // fp32 [8 warps][batch][64]
   L.push = L.red + 8u * batch * 64u * 4u;                          // fp32 [C][batch][64] (used in rank 0)
   L.bars = (L.push + static_cast<uint32_t>(C) * batch * 64u * 4u + 7u) & ~7u;  // push
   L.total = L.bars + 8u;
@@ -81,8 +86,12 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
                : "memory");
 }
 
-template <int B>
+// D = hash rows of the sketch (1: format 1, or format 2 at depth 1; 2, 4: the
+// multi-row AbsMaxMin sketch, whose rows are gathered and reduced to the code
+// of largest magnitude before the MMA)
+template <int B, int D>
 __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a) {
+  constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
   extern __shared__ __align__(128) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -90,7 +99,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);
-  const GemvBfLayout L = gemv_bf_layout(a.tpc, B, a.C);
+  const GemvBfLayout L = gemv_bf_layout(a.tpc, B, a.C, D);
   const uint32_t s0 = smem_u32(sm);
   const uint32_t push_bar = s0 + L.bars;
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
@@ -130,7 +139,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   // armed (the init is published by its cluster-scope fence).  Relaxed: a
   // release arrive would first wait for this thread's loads in flight.
   if (a.C > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-  if (tid < nt) keytab[tid] = tile_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid);
+  if (tid < nt * D) keytab[tid] = row_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid / D, D, tid % D);
 
   // ---- codes: widen to bf16 once
 #pragma unroll
@@ -165,16 +174,29 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
 #pragma unroll
   for (int tt = 0; tt < kBfMaxTiles; ++tt) {
     if (tt < nt) {
-      const uint2 hk = keytab[tt];
       const uint32_t tile_s = s0 + L.cbf + tt * 2048u;
-      const uint32_t h = hk.x * (32u * g + o) + hk.y;
+      uint2 hk[D];
+      uint32_t h[D];
+#pragma unroll
+      for (int rho = 0; rho < D; ++rho) {
+        hk[rho] = keytab[tt * D + rho];
+        h[rho] = hk[rho].x * (32u * g + o) + hk[rho].y;
+      }
 #pragma unroll
       for (int mb = 0; mb < 4; ++mb) {
-        const uint32_t h0 = h + static_cast<uint32_t>(mb) * 512u * hk.x;  // row 16 mb + g
-        const uint32_t h1 = h0 + 256u * hk.x;                              // row 16 mb + g + 8
-        const uint32_t c0 = (static_cast<uint32_t>(o + g) + 16u * mb) & 31u;
-        const uint4 q0 = lds128(tile_s + ((h0 >> 30) * 32u + c0) * 16u);
-        const uint4 q1 = lds128(tile_s + ((h1 >> 30) * 32u + ((c0 + 8u) & 31u)) * 16u);
+        const uint32_t c0 = (static_cast<uint32_t>(o + g) + 16u * mb) & (kNc - 1u);  // row 16 mb + g
+        const uint32_t c1 = (c0 + 8u) & (kNc - 1u);                                  // row 16 mb + g + 8
+        uint4 q0 = make_uint4(0u, 0u, 0u, 0u), q1 = q0;
+#pragma unroll
+        for (int rho = 0; rho < D; ++rho) {
+          const uint32_t h0 = h[rho] + static_cast<uint32_t>(mb) * 512u * hk[rho].x;
+          const uint32_t h1 = h0 + 256u * hk[rho].x;
+          const uint32_t seg = tile_s + static_cast<uint32_t>(rho) * (2048u / D);
+          const uint4 u0 = lds128(seg + ((h0 >> 30) * kNc + c0) * 16u);
+          const uint4 u1 = lds128(seg + ((h1 >> 30) * kNc + c1) * 16u);
+          q0 = rho == 0 ? u0 : absmax_sel(q0, u0);
+          q1 = rho == 0 ? u1 : absmax_sel(q1, u1);
+        }
         mma_bf16_16816(d[tt & 1][mb], q0.x, q1.x, q0.y, q1.y, xv[tt].x, xv[tt].y);
         mma_bf16_16816(d[tt & 1][mb], q0.z, q1.z, q0.w, q1.w, xv[tt].z, xv[tt].w);
       }
@@ -245,10 +267,10 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   }
 }
 
-template <int B>
+template <int B, int D>
 static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_bf_layout(a.tpc, B, a.C).total;
-  auto kern = gemv_bf_kernel<B>;
+  const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D).total;
+  auto kern = gemv_bf_kernel<B, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -272,6 +294,20 @@ static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+template <int D>
+static cudaError_t launch_bf_batch(const GemvBfArgs& a, int batch, int64_t RB, cudaStream_t stream) {
+  switch (batch) {
+    case 1: return launch_bf_t<1, D>(a, RB, stream);
+    case 2: return launch_bf_t<2, D>(a, RB, stream);
+    case 3: return launch_bf_t<3, D>(a, RB, stream);
+    case 4: return launch_bf_t<4, D>(a, RB, stream);
+    case 5: return launch_bf_t<5, D>(a, RB, stream);
+    case 6: return launch_bf_t<6, D>(a, RB, stream);
+    case 7: return launch_bf_t<7, D>(a, RB, stream);
+    default: return launch_bf_t<8, D>(a, RB, stream);
+  }
+}
+
 // Tiles per block: tpc_override if given, else the fewest tiles per block
 // (most blocks) that keeps the cluster within 16 blocks, at least 4.
 bool gemv_bf_supported(int64_t K, int batch, int tpc_override) {
@@ -283,7 +319,7 @@ bool gemv_bf_supported(int64_t K, int batch, int tpc_override) {
 
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject) {
+                           int tpc_override, int inject, int depth) {
   GemvBfArgs a;
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status;
@@ -295,16 +331,9 @@ cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t 
   a.pdl = pdl ? 1 : 0;
   a.inject = inject;
   const int64_t RB = M / kRowsPerBlock;
-  switch (batch) {
-    case 1: return launch_bf_t<1>(a, RB, stream);
-    case 2: return launch_bf_t<2>(a, RB, stream);
-    case 3: return launch_bf_t<3>(a, RB, stream);
-    case 4: return launch_bf_t<4>(a, RB, stream);
-    case 5: return launch_bf_t<5>(a, RB, stream);
-    case 6: return launch_bf_t<6>(a, RB, stream);
-    case 7: return launch_bf_t<7>(a, RB, stream);
-    default: return launch_bf_t<8>(a, RB, stream);
-  }
+  if (depth == 2) return launch_bf_batch<2>(a, batch, RB, stream);
+  if (depth == 4) return launch_bf_batch<4>(a, batch, RB, stream);
+  return launch_bf_batch<1>(a, batch, RB, stream);
 }
 
 }  // namespace usk

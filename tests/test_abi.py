@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_sizes_and_strings(lib):
-    assert usk.usk_format_version() == 1
+    assert usk.usk_format_version() == 2
     assert usk.usk_sizes(4096, 4096) == (4096 * 4096 // 16, 2 * 64)
     assert usk.usk_sizes(0, 0) == (0, 0)
     with pytest.raises(usk.UskError):
@@ -60,8 +60,12 @@ def test_argument_errors_return_before_any_launch(lib):
     # dtype, params, null
     assert lib.usk_build(fake, 7, 64, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 3
     assert lib.usk_build(fake, 1, 64, 256, 256, None, None, fake, fake, None, None) == 6
-    bad = _native.UskParams(2, 0, 0)
-    assert lib.usk_build(fake, 1, 64, 256, 256, None, ctypes.byref(bad), fake, fake, None, None) == 6
+    # unknown format, bad depth for the format, reserved bits, importance with format 2
+    for bad in (_native.UskParams(3, 0, 0, 1, 0), _native.UskParams(2, 0, 0, 0, 0), _native.UskParams(2, 0, 0, 3, 0),
+                _native.UskParams(1, 0, 0, 2, 0), _native.UskParams(2, 0, 0, 2, 1), _native.UskParams(1, 1, 0, 1, 0)):
+        assert lib.usk_build(fake, 1, 64, 256, 256, None, ctypes.byref(bad), fake, fake, None, None) == 6
+    amm = _native.UskParams(2, 0, 0, 2, 0)
+    assert lib.usk_build(fake, 1, 64, 256, 256, fake, ctypes.byref(amm), fake, fake, None, None) == 6
     assert lib.usk_build(None, 1, 64, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 1
     # alignment (W at an odd address, ldw not a multiple of 8 for bf16)
     odd = ctypes.c_void_p(16 * 1024 + 2)
@@ -78,6 +82,10 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.usk_gemm(ctypes.byref(sk), fake, 8, fake, None, 0, None, None) == 4
     assert lib.usk_gemm(ctypes.byref(sk), fake, 24, fake, None, 0, None, None) == 4
     assert lib.usk_gemm(ctypes.byref(sk), fake, 512, fake, None, 0, None, None) == 4
+    for version, depth in ((2, 3), (2, 0), (1, 2), (5, 1)):
+        bad_sk = _native.UskSketchC(64, 256, 0, 16 * 1024, 16 * 1024, version, depth)
+        assert lib.usk_gemv(ctypes.byref(bad_sk), fake, 1, 1, fake, None, None) == 6
+        assert lib.usk_gemm(ctypes.byref(bad_sk), fake, 16, fake, None, 0, None, None) == 6
     unaligned = _native.UskSketchC(64, 256, 0, 16 * 1024 + 1, 16 * 1024)
     assert lib.usk_gemv(ctypes.byref(unaligned), fake, 1, 1, fake, None, None) == 10
 
