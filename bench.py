@@ -5,7 +5,9 @@ One step = one pass of the whole hot path over one 4096x4096 bf16 layer:
 usk_build (key, hash, scatter-select, winner, scale, quantize), usk_gemv at
 batch 1 (rehash + gather decode, product) and usk_gemm at batch 16 (decode into
 tcgen05 tiles).  The headline value is usk_gemv GB/s (algorithmic bytes of one
-call / its average launch duration); usk_build Gweights/s rides along.
+call / its average launch duration); usk_build Gweights/s rides along.  A second
+timed region runs the same three calls K times on the multi-row AbsMaxMin sketch
+(format 2, depth 2) of the same layer and reports them under "absmaxmin".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl usk|reference]
 
@@ -40,6 +42,7 @@ GEMM_BATCH = 16
 N_WCOPIES = 8      # 8 x 32 MiB of weights per build cycle  (> L2)
 N_SKETCHES = 256   # 256 x 1 MiB of codes per decode cycle  (> L2)
 GRAPH_STEPS = 256  # steps per captured CUDA graph
+AMM_DEPTH = 2      # hash rows of the format-2 (multi-row AbsMaxMin) measurement
 
 METRIC = "usk_gemv GB/s & % roofline (4096x4096, batch 1); usk_build Gweights/s"
 WORKLOAD = ("one 4096x4096 bf16 layer, Student-t(4) x 0.02 with 0.1% outliers x20, importance = mean |x| "
@@ -69,14 +72,15 @@ def load_peaks():
     return d
 
 
-def rooflines(peaks, t_build_s, t_gemv_s, t_gemm_s, traffic):
+def rooflines(peaks, t_build_s, t_gemv_s, t_gemm_s, traffic, depth=1, build_bytes=None):
     """Roofline of each kernel from its algorithmic work and the measured peaks.
 
     usk_build is HBM-bound (2 B of bf16 weight in, 1/16 B of code out per weight).
     usk_gemv / usk_gemm decode every weight by a shared-memory gather of its
     bucket code: at least 1 byte per weight through the 128 B/clk/SM shared
     memory pipe, which binds before HBM (codes are 1/16 B per weight); gemm also
-    checks the dense bf16 tensor time."""
+    checks the dense bf16 tensor time.  A depth-D sketch gathers D codes per
+    weight."""
     hbm = peaks["hbm_gbs"] * 1e9
     clk = peaks.get("sm_max_mhz", 1965.0) * 1e6
     smem = SMS * SMEM_BYTES_PER_CLK * clk
@@ -88,13 +92,14 @@ def rooflines(peaks, t_build_s, t_gemv_s, t_gemm_s, traffic):
 
     out = {}
     # build: HBM
-    out["usk_build"] = line("hbm", BUILD_BYTES / t_build_s / 1e9, hbm / 1e9, "GB/s", traffic.get("usk_build"))
+    bb = BUILD_BYTES if build_bytes is None else build_bytes
+    out["usk_build"] = line("hbm", bb / t_build_s / 1e9, hbm / 1e9, "GB/s", traffic.get("usk_build"))
     # gemv: gather-bound; expressed in algorithmic GB/s against the bytes/time at the binding bound
-    t_bound = max(GEMV_BYTES / hbm, N_W / smem)
+    t_bound = max(GEMV_BYTES / hbm, depth * N_W / smem)
     out["usk_gemv"] = line("alu", GEMV_BYTES / t_gemv_s / 1e9, GEMV_BYTES / t_bound / 1e9, "GB/s",
                            traffic.get("usk_gemv"))
-    out["usk_gemv"]["binding"] = "shared-memory gather (1 B/weight at 128 B/clk/SM)"
-    t_bound = max(GEMM_BYTES / hbm, N_W / smem, GEMM_FLOPS / (peaks["bf16_tflops"] * 1e12))
+    out["usk_gemv"]["binding"] = "shared-memory gather (%d B/weight at 128 B/clk/SM)" % depth
+    t_bound = max(GEMM_BYTES / hbm, depth * N_W / smem, GEMM_FLOPS / (peaks["bf16_tflops"] * 1e12))
     out["usk_gemm"] = line("alu", GEMM_BYTES / t_gemm_s / 1e9, GEMM_BYTES / t_bound / 1e9, "GB/s",
                            traffic.get("usk_gemm"))
     out["usk_gemm"]["tensor_tflops"] = round(GEMM_FLOPS / t_gemm_s / 1e12, 3)
@@ -306,21 +311,22 @@ def run_usk(args):
     def gemm(i):
         usk.usk_gemm(sks[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
 
-    kernels = (build, gemv, gemm)
+    # the same three calls on the multi-row AbsMaxMin sketch (format 2) of the layer
+    amm = usk.FORMAT_ABSMAXMIN
+    sk2 = usk.usk_build(W, None, seed, version=amm, depth=AMM_DEPTH)
+    sks2 = [usk.Sketch(M, K, seed, sk2.codes.clone(), sk2.scales.clone(), amm, AMM_DEPTH) for _ in range(N_SKETCHES)]
 
-    # warm-up (untimed, eager): W full steps
-    for i in range(args.warmup):
-        for k in kernels:
-            k(i)
-    torch.cuda.synchronize()
-    if int(status.item()) != 0:
-        raise SystemExit("device status flags %#x during warm-up" % int(status.item()))
+    def build2(i):
+        b = sks2[i % N_SKETCHES]
+        usk.usk_build(Ws[i % N_WCOPIES], None, seed, codes=b.codes, scales=b.scales, status=status, version=amm,
+                      depth=AMM_DEPTH)
 
-    # Timed region: exactly K steps.  The K steps run phase by phase (K builds,
-    # then K GEMVs, then K GEMMs; the same work as K build+gemv+gemm passes) so
-    # that each kernel's average launch duration is the CUDA-event time of its
-    # phase / K, with no timing nodes between kernels.  Each phase replays a CUDA
-    # graph of GRAPH_STEPS launches (+ one graph for the remainder).
+    def gemv2(i):
+        usk.usk_gemv(sks2[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1, pdl=True)
+
+    def gemm2(i):
+        usk.usk_gemm(sks2[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
+
     s = torch.cuda.Stream(device=dev)
     s.wait_stream(torch.cuda.current_stream())
 
@@ -332,40 +338,59 @@ def run_usk(args):
         return g
 
     full, rem = divmod(args.steps, GRAPH_STEPS)
-    graphs = []
-    for fn in kernels:
-        main = capture(fn, GRAPH_STEPS, args.warmup) if full else None
-        tail = capture(fn, rem, args.warmup) if rem else None
-        graphs.append((main, tail))
-    torch.cuda.synchronize()
 
+    def prepare(kernels):
+        # warm-up (untimed, eager): W full steps, then one graph per phase
+        for i in range(args.warmup):
+            for k in kernels:
+                k(i)
+        torch.cuda.synchronize()
+        if int(status.item()) != 0:
+            raise SystemExit("device status flags %#x during warm-up" % int(status.item()))
+        graphs = []
+        for fn in kernels:
+            main = capture(fn, GRAPH_STEPS, args.warmup) if full else None
+            tail = capture(fn, rem, args.warmup) if rem else None
+            graphs.append((main, tail))
+        torch.cuda.synchronize()
+        return graphs
+
+    def timed(graphs):
+        # Timed region: exactly K steps.  The K steps run phase by phase (K
+        # builds, then K GEMVs, then K GEMMs; the same work as K build+gemv+gemm
+        # passes) so that each kernel's average launch duration is the CUDA-event
+        # time of its phase / K, with no timing nodes between kernels.  Each phase
+        # replays a CUDA graph of GRAPH_STEPS launches (+ one for the remainder).
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
+        ev[0].record()
+        for k, (main, tail) in enumerate(graphs):
+            for _ in range(full):
+                main.replay()
+            if tail is not None:
+                tail.replay()
+            ev[k + 1].record()
+        ev[-1].synchronize()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        if int(status.item()) != 0:
+            raise SystemExit("device status flags %#x in the timed region" % int(status.item()))
+        n = max(args.steps, 1)
+        return [ev[k].elapsed_time(ev[k + 1]) * 1e-3 / n for k in range(len(graphs))] + \
+            [ev[0].elapsed_time(ev[-1]) * 1e-3]
+
+    graphs1 = prepare((build, gemv, gemm))
+    graphs2 = prepare((build2, gemv2, gemm2))
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(kernels) + 1)]
-    ev[0].record()
-    for k, (main, tail) in enumerate(graphs):
-        for _ in range(full):
-            main.replay()
-        if tail is not None:
-            tail.replay()
-        ev[k + 1].record()
-    ev[-1].synchronize()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    t_build, t_gemv, t_gemm, t_total = timed(graphs1)
+    t_build2, t_gemv2, t_gemm2, _ = timed(graphs2)
     sampler.stop()
-    n = max(args.steps, 1)
-    t_build = ev[0].elapsed_time(ev[1]) * 1e-3 / n
-    t_gemv = ev[1].elapsed_time(ev[2]) * 1e-3 / n
-    t_gemm = ev[2].elapsed_time(ev[3]) * 1e-3 / n
-    t_total = ev[0].elapsed_time(ev[3]) * 1e-3
-    t_step = t_total / n
-    if int(status.item()) != 0:
-        raise SystemExit("device status flags %#x in the timed region" % int(status.item()))
+    t_step = t_total / max(args.steps, 1)
 
     # end to end through the public API with host buffers: x in from pinned host memory, y back out
     xh = x1.cpu().pin_memory()
@@ -384,8 +409,8 @@ def run_usk(args):
     t_e2e = (time.perf_counter() - t0) / n_e2e
 
     # max over ranks
-    t_gemv, t_build, t_gemm, t_step, t_total, t_e2e = max_over_ranks(
-        [t_gemv, t_build, t_gemm, t_step, t_total, t_e2e], device=dev)
+    t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2 = max_over_ranks(
+        [t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2], device=dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -400,7 +425,10 @@ def run_usk(args):
         return 0
     peaks = load_peaks()
     agg = aggregate(world, [t_gemv], [t_build], [t_step])
-    rl = rooflines(peaks, t_build, t_gemv, t_gemm, load_traffic())
+    tr = load_traffic()
+    rl = rooflines(peaks, t_build, t_gemv, t_gemm, tr)
+    tr2 = {k[len("amm_"):]: v for k, v in tr.items() if k.startswith("amm_")}
+    rl2 = rooflines(peaks, t_build2, t_gemv2, t_gemm2, tr2, depth=AMM_DEPTH, build_bytes=BUILD_BYTES - 4 * K)
     clocks = sampler.summary()
     line = {
         "metric": METRIC,
@@ -433,6 +461,18 @@ def run_usk(args):
                 "call": "usk_gemv via the Python binding, x from pinned host memory, y read back, per step"},
         "gpu_launches": 3 * args.steps,
         "cpu_baseline": cpu,
+        "absmaxmin": {
+            "format": "multi-row AbsMaxMin sketch (format 2): smallest |w| kept per bucket, largest magnitude "
+                      "over %d hash rows decoded; same layer, no importance" % AMM_DEPTH,
+            "depth": AMM_DEPTH,
+            "timing": "a second timed region: K builds, K GEMVs (batch 1), K GEMMs (batch 16) as CUDA graphs",
+            "usk_gemv_gbs": round(world * GEMV_BYTES / t_gemv2 / 1e9, 3),
+            "usk_build_gweights_per_s": round(world * N_W / t_build2 / 1e9, 3),
+            "kernel_us": {"usk_build": round(t_build2 * 1e6, 3), "usk_gemv": round(t_gemv2 * 1e6, 3),
+                          "usk_gemm": round(t_gemm2 * 1e6, 3)},
+            "rooflines": rl2,
+            "gpu_launches": 3 * args.steps,
+        },
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -450,12 +490,15 @@ def run_profile_case(args):
     imp = torch.from_numpy(cfg["importance"]).to(dev)
     x16 = torch.from_numpy(cfg["x"].view(np.int16)).to(dev).view(torch.bfloat16)
     x1 = x16[:GEMV_BATCH].contiguous()
-    sk = usk.usk_build(W, imp, cfg["seed"])
+    case = args.profile_case
+    fmt = {} if not case.endswith("_amm") else {"version": usk.FORMAT_ABSMAXMIN, "depth": AMM_DEPTH}
+    imp_c = imp if not fmt else None
+    sk = usk.usk_build(W, imp_c, cfg["seed"], **fmt)
     torch.cuda.synchronize()
     for _ in range(3 + 3):  # 3 warm-up launches, then 3 to capture
-        if args.profile_case == "build":
-            usk.usk_build(W, imp, cfg["seed"], codes=sk.codes, scales=sk.scales)
-        elif args.profile_case == "gemv":
+        if case.startswith("build"):
+            usk.usk_build(W, imp_c, cfg["seed"], codes=sk.codes, scales=sk.scales, **fmt)
+        elif case.startswith("gemv"):
             usk.usk_gemv(sk, x1)
         else:
             usk.usk_gemm(sk, x16)
@@ -471,7 +514,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="usk", choices=["usk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["build", "gemv", "gemm"], default=None,
+    ap.add_argument("--profile-case", choices=["build", "gemv", "gemm", "build_amm", "gemv_amm", "gemm_amm"],
+                    default=None,
                     help="run 6 launches of one kernel on the bench workload (for ncu) and exit")
     args = ap.parse_args(argv)
     if args.profile_case:

@@ -30,3 +30,12 @@ def rel_err(y: np.ndarray, ref: np.ndarray) -> float:
     den = float(np.max(np.abs(ref)))
     num = float(np.max(np.abs(y.astype(np.float64) - ref)))
     return num / den if den > 0 else num
+
+
+def sketch_from_oracle(o, M: int, K: int, seed: int, version: int = 1, depth: int = 1):
+    """A device sketch holding the ORACLE's codes and scales (uploaded), so that a
+    product test's expected value never depends on the CUDA build."""
+    import sub_bit_weight_usk_b200 as usk
+    codes = torch.from_numpy(np.ascontiguousarray(o["codes"]).copy()).cuda()
+    scales = torch.from_numpy(np.ascontiguousarray(o["scales"]).view(np.int16).copy()).cuda()
+    return usk.Sketch(M, K, seed, codes, scales, version, depth)

@@ -114,19 +114,6 @@ def test_amm_build_layer_workload_full(depth):
     _compare_build(cfg["W"], cfg["seed"], depth)
 
 
-def test_amm_build_mlp70b_sampled_row_blocks():
-    cfg = gen.mlp70b("up", 16)
-    W = cfg["W"]
-    sk = _gpu_build(W, cfg["seed"], 2)
-    c, s = codes_np(sk), scales_np(sk)
-    per = 4 * W.shape[1]
-    RB = W.shape[0] // 64
-    for rb in (0, 1, RB // 2, RB - 1):
-        o = oracle.build_sketch_amm(W[64 * rb:64 * rb + 64], cfg["seed"], 2, row_block0=rb)
-        assert np.array_equal(s[rb:rb + 1], o["scales"]), "scale of row block %d" % rb
-        assert np.array_equal(c[rb * per:(rb + 1) * per], o["codes"]), "codes of row block %d" % rb
-
-
 def test_amm_build_flags_and_argument_errors():
     W = gen.weights_normal(64, 256, 1, 0.02, "f32")
     Wn = W.copy()
@@ -217,10 +204,15 @@ def test_amm_layer_workload_products(depth):
     _check_product(sk, o, cfg["x"], gemm=True)
 
 
-def test_amm_mlp70b_products_sampled_rows():
+def test_amm_mlp70b_build_and_products():
+    """28672 x 8192 at depth 2: the whole build bit-exact; GEMV at 1 and GEMM at
+    16 and 64 on sampled rows of the oracle's sketch."""
     cfg = gen.mlp70b("up", 64)
     W = cfg["W"]
+    gsk = _gpu_build(W, cfg["seed"], 2)
     sk, o = _oracle_sketch(W, cfg["seed"], 2)
+    assert np.array_equal(scales_np(gsk), o["scales"]) and np.array_equal(codes_np(gsk), o["codes"])
+    del gsk
     M = W.shape[0]
     rows = np.array([0, 1, 127, 128, M // 2, M - 65, M - 1])
     _check_product(sk, o, cfg["x"][:1], rows=rows)

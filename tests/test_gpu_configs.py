@@ -1,10 +1,10 @@
 """The five workload configurations end to end on the GPU against the oracle.
 
-Builds are compared bit-exact (whole matrices where the oracle finishes in
-seconds, sampled row blocks otherwise: a row block's sketch depends only on its
-own rows); products within max|y - y_ref| <= 1e-3 max|y_ref| on every output or
-on sampled rows.  The kernels run in the launch configurations the library picks
-for these shapes."""
+Builds are compared bit-exact (whole matrices, up to 28672 x 8192; sampled row
+blocks for the 32-layer stack: a row block's sketch depends only on its own
+rows); products run on the ORACLE's sketch, uploaded, within
+max|y - y_ref| <= 1e-3 max|y_ref| on every output or on sampled rows.  The
+kernels run in the launch configurations the library picks for these shapes."""
 import numpy as np
 import pytest
 import torch
@@ -12,11 +12,22 @@ import torch
 import gen
 import oracle
 import sub_bit_weight_usk_b200 as usk
-from tests.gpu_util import codes_np, rel_err, scales_np, to_dev
+from tests.gpu_util import codes_np, rel_err, scales_np, sketch_from_oracle, to_dev
 
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-3
+
+
+def _build_checked(W, imp, seed):
+    """GPU build compared bit-exact with the oracle's; returns the oracle's
+    sketch uploaded (for the products) and the oracle's arrays."""
+    sk = usk.usk_build(to_dev(W), None if imp is None else to_dev(imp), seed)
+    torch.cuda.synchronize()
+    o = oracle.build_sketch(W, imp, seed)
+    assert np.array_equal(scales_np(sk), o["scales"]), "scales differ"
+    assert np.array_equal(codes_np(sk), o["codes"]), "codes differ"
+    return sketch_from_oracle(o, W.shape[0], W.shape[1], seed), o
 
 
 def _build(W, imp, seed):
@@ -33,10 +44,10 @@ def _check_rows_built(W, seed, c, s, row_blocks):
         assert np.array_equal(c[rb * per:(rb + 1) * per], o["codes"]), "codes of row block %d" % rb
 
 
-def _check_product(sk, c, s, x, rows=None, gemm=False):
+def _check_product(sk, o, x, rows=None, gemm=False):
     xd = to_dev(x)
     y = (usk.usk_gemm(sk, xd) if gemm else usk.usk_gemv(sk, xd)).cpu().numpy()
-    ref = oracle.gemv_f64(c, s, sk.M, sk.K, x, sk.seed, rows=rows)
+    ref = oracle.gemv_f64(o["codes"], o["scales"], sk.M, sk.K, x, sk.seed, rows=rows)
     if rows is not None:
         y = y[:, rows]
     e = rel_err(y, ref)
@@ -46,21 +57,17 @@ def _check_product(sk, c, s, x, rows=None, gemm=False):
 def test_config_small_fp32():
     """256x1024 fp32 weights, lognormal importance, GEMV at batch 1 (fp32 and bf16 x)."""
     cfg = gen.small("f32")
-    sk, c, s = _build(cfg["W"], cfg["importance"], cfg["seed"])
-    o = oracle.build_sketch(cfg["W"], cfg["importance"], cfg["seed"])
-    assert np.array_equal(c, o["codes"]) and np.array_equal(s, o["scales"])
-    _check_product(sk, c, s, cfg["x"])
-    _check_product(sk, c, s, gen.small("bf16")["x"])
+    sk, o = _build_checked(cfg["W"], cfg["importance"], cfg["seed"])
+    _check_product(sk, o, cfg["x"])
+    _check_product(sk, o, gen.small("bf16")["x"])
 
 
 def test_config_layer_4096():
     """One 4096x4096 layer with outliers and calibration importance; GEMV at 1 and 4."""
     cfg = gen.layer(4)
-    sk, c, s = _build(cfg["W"], cfg["importance"], cfg["seed"])
-    o = oracle.build_sketch(cfg["W"], cfg["importance"], cfg["seed"])
-    assert np.array_equal(c, o["codes"]) and np.array_equal(s, o["scales"])
-    _check_product(sk, c, s, cfg["x"][:1])
-    _check_product(sk, c, s, cfg["x"])
+    sk, o = _build_checked(cfg["W"], cfg["importance"], cfg["seed"])
+    _check_product(sk, o, cfg["x"][:1])
+    _check_product(sk, o, cfg["x"])
 
 
 @pytest.mark.parametrize("name", gen.LLAMA7B_ORDER)
@@ -69,30 +76,26 @@ def test_config_llama7b_layer_set(name):
     and 4, GEMM at batch 16 (sampled rows for the products)."""
     cfg = gen.llama7b_layer(name, 16)
     W = cfg["W"]
-    sk, c, s = _build(W, None, cfg["seed"])
-    o = oracle.build_sketch(W, None, cfg["seed"])
-    assert np.array_equal(c, o["codes"]) and np.array_equal(s, o["scales"])
+    sk, o = _build_checked(W, None, cfg["seed"])
     M = W.shape[0]
     rows = np.array([0, 63, 64, M // 2 + 5, M - 1])
-    _check_product(sk, c, s, cfg["x"][:1], rows=rows)
-    _check_product(sk, c, s, cfg["x"][:4], rows=rows)
-    _check_product(sk, c, s, cfg["x"], rows=rows, gemm=True)
+    _check_product(sk, o, cfg["x"][:1], rows=rows)
+    _check_product(sk, o, cfg["x"][:4], rows=rows)
+    _check_product(sk, o, cfg["x"], rows=rows, gemm=True)
 
 
 @pytest.mark.parametrize("name", ["up", "down"])
 def test_config_mlp70b(name):
-    """28672x8192 and 8192x28672: sampled row blocks of the build, GEMM at 16
-    and 32 and GEMV at 1 on sampled rows."""
+    """28672x8192 and 8192x28672: the whole build bit-exact, GEMM at 16 and 32
+    and GEMV at 1 on sampled rows."""
     cfg = gen.mlp70b(name, 32)
     W = cfg["W"]
-    sk, c, s = _build(W, None, cfg["seed"])
-    RB = W.shape[0] // 64
-    _check_rows_built(W, cfg["seed"], c, s, (0, 1, RB // 2, RB - 1))
+    sk, o = _build_checked(W, None, cfg["seed"])
     M = W.shape[0]
     rows = np.array([0, 1, 127, 128, M // 2, M - 65, M - 1])
-    _check_product(sk, c, s, cfg["x"][:16], rows=rows, gemm=True)
-    _check_product(sk, c, s, cfg["x"], rows=rows, gemm=True)
-    _check_product(sk, c, s, cfg["x"][:1], rows=rows)
+    _check_product(sk, o, cfg["x"][:16], rows=rows, gemm=True)
+    _check_product(sk, o, cfg["x"], rows=rows, gemm=True)
+    _check_product(sk, o, cfg["x"][:1], rows=rows)
 
 
 @pytest.mark.parametrize("layer,linear", [(0, "q"), (0, "down"), (17, "gate"), (31, "o"), (31, "up")])
@@ -105,5 +108,6 @@ def test_config_stack7b_sampled(layer, linear):
     sk, c, s = _build(W, None, seed)
     RB = M // 64
     _check_rows_built(W, seed, c, s, (0, RB // 3, RB - 1))
+    o = oracle.build_sketch(W, None, seed)
     x = gen.activations(1, K, seed, "bf16")
-    _check_product(sk, c, s, x, rows=np.array([0, 64 * (RB // 3) + 7, M - 1]))
+    _check_product(sketch_from_oracle(o, M, K, seed), o, x, rows=np.array([0, 64 * (RB // 3) + 7, M - 1]))

@@ -9,17 +9,18 @@ import torch
 import gen
 import oracle
 import sub_bit_weight_usk_b200 as usk
-from tests.gpu_util import codes_np, rel_err, scales_np, status_tensor, to_dev
+from tests.gpu_util import codes_np, rel_err, scales_np, sketch_from_oracle, status_tensor, to_dev
 
 pytestmark = pytest.mark.gpu
 
 TOL = 1e-3
 
 
-def _sketch(W, seed):
-    sk = usk.usk_build(to_dev(W), None, seed)
-    torch.cuda.synchronize()
-    return sk, {"codes": codes_np(sk), "scales": scales_np(sk)}
+def _sketch(W, seed, imp=None):
+    """The oracle's sketch of W, uploaded (the build kernel is pinned elsewhere)."""
+    o = oracle.build_sketch(W, imp, seed)
+    assert o["status"] == oracle.OK
+    return sketch_from_oracle(o, W.shape[0], W.shape[1], seed), o
 
 
 def _check(sk, o, x, rows=None):
@@ -42,20 +43,21 @@ def test_gemm_matches_oracle(M, K, batch):
     _check(sk, o, x)
 
 
-def test_gemm_equals_oracle_built_sketch():
+def test_gemm_on_gpu_built_sketch():
+    """The whole product path: GPU build (checked bit-exact) then GPU GEMM."""
     W = gen.weights_normal(256, 1024, 13, 0.02, "bf16")
     o = oracle.build_sketch(W, None, 6)
-    sk, _ = _sketch(W, 6)
-    assert np.array_equal(codes_np(sk), o["codes"])
+    sk = usk.usk_build(to_dev(W), None, 6)
+    torch.cuda.synchronize()
+    assert np.array_equal(codes_np(sk), o["codes"]) and np.array_equal(scales_np(sk), o["scales"])
     _check(sk, o, gen.activations(16, 1024, 14, "bf16"))
 
 
 @pytest.mark.parametrize("batch", [16, 64])
 def test_gemm_layer_workload_full(batch):
     cfg = gen.layer(batch)
-    sk = usk.usk_build(to_dev(cfg["W"]), to_dev(cfg["importance"]), cfg["seed"])
-    torch.cuda.synchronize()
-    _check(sk, {"codes": codes_np(sk), "scales": scales_np(sk)}, cfg["x"])
+    sk, o = _sketch(cfg["W"], cfg["seed"], cfg["importance"])
+    _check(sk, o, cfg["x"])
 
 
 @pytest.mark.parametrize("name", ["up", "down"])
