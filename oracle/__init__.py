@@ -11,7 +11,8 @@ Operators" (gist.science/es/paper/2506.17255), Resumen Tecnico, Metodologia §1
 (AbsMaxMin sketch) and §4 (decompression as W_hat = S . P^T), plus the frozen
 format readings listed there: format 1 (one hash row, largest key kept) and
 format 2 (the multi-row AbsMaxMin sketch: smallest magnitude kept per bucket,
-largest magnitude over the hash rows on decode; the ``*_amm`` functions).
+largest magnitude over the hash rows on decode; the ``*_amm`` functions) and
+format 3 (the column-shared projection W_hat = S . P^T; the ``*_cs`` functions).
 
 Parity pins (tests/test_oracle_*.py): SplitMix64 published outputs, binary16
 conversion against numpy's, round-half-even against numpy.rint, an independent
@@ -94,6 +95,16 @@ def _load():
         lib.orc_amm_gemv_f64.argtypes = [vp, vp, i64, i64, u64, ctypes.c_int, vp, ctypes.c_int, i64, vp, i64,
                                          vp]
         lib.orc_amm_gemv_f64.restype = ctypes.c_int
+        lib.orc_cs_sigma.argtypes = [u64, i64, ctypes.c_int]
+        lib.orc_cs_sigma.restype = ctypes.c_int
+        lib.orc_cs_bucket.argtypes = [i64, u64, i64]
+        lib.orc_cs_bucket.restype = i64
+        lib.orc_cs_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, u64, vp, vp, vp, vp]
+        lib.orc_cs_build.restype = ctypes.c_int
+        lib.orc_cs_decode.argtypes = [vp, vp, i64, i64, u64, vp]
+        lib.orc_cs_decode.restype = ctypes.c_int
+        lib.orc_cs_gemv_f64.argtypes = [vp, vp, i64, i64, u64, vp, ctypes.c_int, i64, vp, i64, vp]
+        lib.orc_cs_gemv_f64.restype = ctypes.c_int
         lib.orc_f32_to_f16_array.argtypes = [vp, vp, i64]
         lib.orc_f32_to_f16_array.restype = None
         lib.orc_f16_to_f32_array.argtypes = [vp, vp, i64]
@@ -192,6 +203,67 @@ def gemv_amm_f64(codes, scales, M, K, x, seed=0, depth=2, rows=None):
 def amm_bucket_index(K, seed, depth, rho, i, j):
     """Global code index of weight (i, j) in hash row rho of a format-2 sketch."""
     return int(_load().orc_amm_bucket_index(K, seed, depth, rho, i, j))
+
+
+def build_sketch_cs(W, seed=0, want_winners=False):
+    """Column-shared projection sketch of W [M, K] (format 3: W_hat = S . P^T with
+    a one-hot P shared by all rows; S keeps the smallest |w| per row and
+    bucket).  Returns dict as build_sketch; codes are row-major [M, K/16]."""
+    W, dt = _weights(W)
+    M, K = W.shape
+    nb = M * K // 16 if (M % 64 == 0 and K % 256 == 0 and M >= 0 and K >= 0) else 0
+    codes = np.zeros(max(nb, 1), dtype=np.int8)
+    scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
+    winner = np.full(max(nb, 1), -2, dtype=np.int64) if want_winners else None
+    value = np.zeros(max(nb, 1), dtype=np.float32) if want_winners else None
+    st = _load().orc_cs_build(_ptr(W), dt, M, K, K, seed, _ptr(codes), _ptr(scales), _ptr(winner), _ptr(value))
+    out = {"status": st, "codes": codes[:nb], "scales": scales[: M // 64]}
+    if want_winners:
+        out["winner"] = winner[:nb]
+        out["value"] = value[:nb]
+    return out
+
+
+def decode_cs(codes, scales, M, K, seed=0):
+    """W_hat [M, K] float32 of a format-3 sketch."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    out = np.zeros((M, K), dtype=np.float32)
+    st = _load().orc_cs_decode(_ptr(codes), _ptr(scales), M, K, seed, _ptr(out))
+    if st:
+        raise ValueError("orc_cs_decode status %d" % st)
+    return out
+
+
+def gemv_cs_f64(codes, scales, M, K, x, seed=0, rows=None):
+    """y = W_hat x^T in float64 for a format-3 sketch (arguments as gemv_f64)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    xdt = F32 if x.dtype == np.float32 else BF16 if x.dtype == np.uint16 else None
+    if xdt is None:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    batch = x.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nr = M if r is None else len(r)
+    y = np.zeros((batch, nr), dtype=np.float64)
+    st = _load().orc_cs_gemv_f64(_ptr(codes), _ptr(scales), M, K, seed, _ptr(x), xdt, batch,
+                                 _ptr(r), 0 if r is None else len(r), _ptr(y))
+    if st:
+        raise ValueError("orc_cs_gemv_f64 status %d" % st)
+    return y
+
+
+def cs_sigma(seed, tc, u):
+    """sigma_tc(u): position u of tile column tc's column list (format 3)."""
+    return int(_load().orc_cs_sigma(seed & (2**64 - 1), tc, u))
+
+
+def cs_bucket(K, seed, j):
+    """Global bucket of column j in a format-3 sketch."""
+    return int(_load().orc_cs_bucket(K, seed, j))
 
 
 def decode(codes, scales, M, K, seed=0):

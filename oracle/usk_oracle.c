@@ -530,3 +530,155 @@ int orc_amm_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int
   free(wrow);
   return ORC_OK;
 }
+
+/* ================================================================ format 3
+ *
+ * The column-shared projection ("UltraSketchLLM" explainer, Resumen Tecnico,
+ * Metodologia §4 "Mapeo de Operadores de Matriz Amigables con el Hardware"):
+ * compression is a modified matrix product of W with a projection matrix P
+ * whose reduction is a MIN over absolute values, and decompression is the plain
+ * product W_hat = S . P^T.  Readings (the pages give no more detail):
+ *  - P is one-hot per input column and shared by every row: within each
+ *    256-column tile tc, a seeded bijection sigma_tc of [0, 256) lists the
+ *    columns, and bucket b' in [0, 16) of the tile holds the 16 columns
+ *    sigma_tc(16 b' + k), k = 0..15 (every bucket exactly 16 members);
+ *    global bucket b = 16 tc + b', K/16 buckets per row;
+ *  - sigma_tc: z = SplitMix64 output tc + 1 of the seed, A = (z & 255) | 1,
+ *    B = (z >> 8) & 255, C = ((z >> 16) & 255) | 1; for u in [0, 256):
+ *    v1 = (A u + B) mod 256, v2 = v1 xor (v1 >> 4), v3 = (C v2) mod 256,
+ *    sigma(u) = v3 xor (v3 >> 3) -- each step is a bijection of 8-bit values;
+ *  - S[i][b] = the signed value of row i's member of bucket b with the smallest
+ *    |w| (the MIN reduction), ties to the smallest column; no importance;
+ *  - scale and codes as format 2 (binary16 of max|v|/127 per 64-row block,
+ *    codes toward zero); storage row-major: codes[i * K/16 + b];
+ *  - decode: w_hat[i][j] = code[i][bucket of column j] * s. */
+
+/* sigma_tc(u) of tile column tc. */
+int orc_cs_sigma(uint64_t seed, int64_t tc, int u) {
+  uint64_t z = orc_splitmix64(seed, (uint64_t)tc + 1);
+  unsigned A = (unsigned)(z & 255u) | 1u, B = (unsigned)((z >> 8) & 255u), C = (unsigned)((z >> 16) & 255u) | 1u;
+  unsigned v1 = (A * (unsigned)u + B) & 255u;
+  unsigned v2 = v1 ^ (v1 >> 4);
+  unsigned v3 = (C * v2) & 255u;
+  return (int)(v3 ^ (v3 >> 3));
+}
+
+/* Bucket (global, in [0, K/16)) of column j: the position of j's in-tile
+ * column in sigma's list, divided by 16 (found by searching the list). */
+int64_t orc_cs_bucket(int64_t K, uint64_t seed, int64_t j) {
+  int64_t tc = j / TILE_COLS, c = j % TILE_COLS;
+  (void)K;
+  for (int u = 0; u < TILE_COLS; ++u)
+    if (orc_cs_sigma(seed, tc, u) == c) return tc * (TILE_COLS / WEIGHTS_PER_BUCKET) + u / WEIGHTS_PER_BUCKET;
+  return -1; /* not reached: sigma is a bijection */
+}
+
+int orc_cs_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw, uint64_t seed,
+                 int8_t* codes, uint16_t* scales, int64_t* winner, float* value) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
+  if (M == 0) return ORC_OK;
+  if (!codes || !scales) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) scales[rb] = 0;
+    return ORC_OK;
+  }
+  if (!W || ldw < K) return ORC_ERR_NULL;
+  int64_t nb = K / WEIGHTS_PER_BUCKET;  /* buckets per row */
+  int64_t* bucket_of = (int64_t*)malloc(sizeof(int64_t) * (size_t)K);
+  float* val = (float*)malloc(sizeof(float) * (size_t)(ROWS_PER_BLOCK * nb));
+  int64_t* idx = (int64_t*)malloc(sizeof(int64_t) * (size_t)(ROWS_PER_BLOCK * nb));
+  if (!bucket_of || !val || !idx) { free(bucket_of); free(val); free(idx); return ORC_ERR_NULL; }
+  for (int64_t j = 0; j < K; ++j) bucket_of[j] = orc_cs_bucket(K, seed, j);
+  int status = ORC_OK;
+  for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
+    float mx = 0.0f;
+    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
+      int64_t i = rb * ROWS_PER_BLOCK + r;
+      float* vr = val + r * nb;
+      int64_t* ir = idx + r * nb;
+      for (int64_t b = 0; b < nb; ++b) ir[b] = -1;
+      /* scan the row in column order: the first member of smallest |w| stays */
+      for (int64_t j = 0; j < K; ++j) {
+        float w = load_elem(W, dtype, i * ldw + j);
+        if (!isfinite(w)) status = ORC_ERR_NONFINITE;
+        int64_t b = bucket_of[j];
+        if (ir[b] < 0 || fabsf(w) < fabsf(vr[b])) { vr[b] = w; ir[b] = j; }
+      }
+      for (int64_t b = 0; b < nb; ++b)
+        if (fabsf(vr[b]) > mx) mx = fabsf(vr[b]);
+    }
+    uint16_t s16 = orc_f32_to_f16(mx / 127.0f);
+    if ((s16 & 0x7c00u) == 0x7c00u) status = status ? status : ORC_ERR_SCALE_OVERFLOW;
+    scales[rb] = s16;
+    double s = (double)orc_f16_to_f32(s16);
+    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
+      int64_t i = rb * ROWS_PER_BLOCK + r;
+      for (int64_t b = 0; b < nb; ++b) {
+        float v = val[r * nb + b];
+        int code = 0;
+        if (s != 0.0 && isfinite(s) && isfinite(v)) {
+          code = floor_code(fabs((double)v), s);
+          if (v < 0.0f) code = -code;
+        }
+        codes[i * nb + b] = (int8_t)code;
+        if (winner) winner[i * nb + b] = i * K + idx[r * nb + b];
+        if (value) value[i * nb + b] = v;
+      }
+    }
+  }
+  free(bucket_of); free(val); free(idx);
+  return status;
+}
+
+/* W_hat [M, K] of a format-3 sketch. */
+int orc_cs_decode(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                  float* What) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (M == 0 || K == 0) return ORC_OK;
+  if (!codes || !scales || !What) return ORC_ERR_NULL;
+  int64_t nb = K / WEIGHTS_PER_BUCKET;
+  for (int64_t j = 0; j < K; ++j) {
+    int64_t b = orc_cs_bucket(K, seed, j);
+    for (int64_t i = 0; i < M; ++i)
+      What[i * K + j] = (float)codes[i * nb + b] * orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+  }
+  return ORC_OK;
+}
+
+/* Reference product of a format-3 sketch in float64, from the definition
+ * y[t][i] = sum_j w_hat[i][j] x[t][j] (arguments as orc_gemv_f64). */
+int orc_cs_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                    const void* x, int xdtype, int64_t batch, const int64_t* rows, int64_t nrows, double* y) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (xdtype != 0 && xdtype != 1) return ORC_ERR_DTYPE;
+  if (batch < 0) return ORC_ERR_SHAPE;
+  int64_t nr = rows ? nrows : M;
+  if (nr == 0 || batch == 0) return ORC_OK;
+  if (!y) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t q = 0; q < batch * nr; ++q) y[q] = 0.0;
+    return ORC_OK;
+  }
+  if (!codes || !scales || !x) return ORC_ERR_NULL;
+  int64_t nb = K / WEIGHTS_PER_BUCKET;
+  int64_t* bucket_of = (int64_t*)malloc(sizeof(int64_t) * (size_t)K);
+  if (!bucket_of) return ORC_ERR_NULL;
+  for (int64_t j = 0; j < K; ++j) bucket_of[j] = orc_cs_bucket(K, seed, j);
+  for (int64_t q = 0; q < nr; ++q) {
+    int64_t i = rows ? rows[q] : q;
+    if (i < 0 || i >= M) { free(bucket_of); return ORC_ERR_SHAPE; }
+    float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+    for (int64_t t = 0; t < batch; ++t) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j)
+        acc += (double)((float)codes[i * nb + bucket_of[j]] * s) * (double)load_elem(x, xdtype, t * K + j);
+      y[t * nr + q] = acc;
+    }
+  }
+  free(bucket_of);
+  return ORC_OK;
+}

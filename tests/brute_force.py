@@ -155,3 +155,49 @@ def decode_amm(codes, scales, M: int, K: int, seed: int = 0, depth: int = 2) -> 
                     best = c
             out[i, j] = best * s
     return out
+
+
+# ---- format 3: the column-shared projection (Metodologia §4: W_hat = S . P^T,
+# compression a MIN reduction over |w|).  Bucket b' of tile tc holds the columns
+# sigma_tc(16 b' + k); S keeps per row and bucket the member of smallest |w|.
+
+def sigma_cs(seed: int, tc: int, u: int) -> int:
+    z = splitmix64_output(seed, tc + 1)
+    A, B, C = (z & 255) | 1, (z >> 8) & 255, ((z >> 16) & 255) | 1
+    v1 = (A * u + B) % 256
+    v2 = v1 ^ (v1 >> 4)
+    v3 = (C * v2) % 256
+    return v3 ^ (v3 >> 3)
+
+
+def build_cs(W: np.ndarray, seed: int = 0):
+    """Returns (codes row-major [M*K/16], scales, winner flat index)."""
+    from fractions import Fraction
+    Wf = to_f32(np.ascontiguousarray(W))
+    M, K = Wf.shape
+    nb = K // 16
+    groups = []  # global bucket -> its 16 columns
+    for tc in range(K // 256):
+        for bp in range(16):
+            groups.append([256 * tc + sigma_cs(seed, tc, 16 * bp + k) for k in range(16)])
+    winner = np.zeros(M * nb, dtype=np.int64)
+    value = np.zeros(M * nb, dtype=np.float32)
+    for i in range(M):
+        for b, cols in enumerate(groups):
+            j = min(cols, key=lambda c: (abs(float(Wf[i, c])), c))
+            winner[i * nb + b] = i * K + j
+            value[i * nb + b] = Wf[i, j]
+    codes = np.zeros(M * nb, dtype=np.int8)
+    scales = np.zeros(M // 64, dtype=np.uint16)
+    for rb in range(M // 64):
+        sl = slice(rb * 64 * nb, (rb + 1) * 64 * nb)
+        v = value[sl]
+        s16 = np.float16(np.float32(np.max(np.abs(v))) / np.float32(127.0))
+        scales[rb] = s16.view(np.uint16)
+        s = Fraction(float(s16))
+        if s != 0:
+            out = codes[sl]
+            for q in range(len(v)):
+                n = min(127, int(Fraction(float(abs(v[q]))) / s))
+                out[q] = -n if v[q] < 0 else n
+    return codes, scales, winner
