@@ -53,6 +53,23 @@
  *   Decode: w_hat = float(c) * float(s16), c = the code of largest magnitude
  *   among the weight's D buckets, ties to the lowest row.  |w_hat| <= |w|.
  *
+ * FORMAT 3 (column-shared projection; Metodologia §4: compression is a matrix
+ * product with a projection P whose reduction is a MIN over |w|, decompression
+ * the plain product W_hat = S . P^T).  P is one-hot per input column and shared
+ * by all rows; same geometry, scales and storage size (0.5 bit/weight):
+ *   Column list of tile tc: z = SplitMix64 output number tc + 1 of `seed`,
+ *     A = (z & 255) | 1, B = (z >> 8) & 255, C = ((z >> 16) & 255) | 1,
+ *     sigma(u) = v3 ^ (v3 >> 3), v3 = (C * v2) mod 256, v2 = v1 ^ (v1 >> 4),
+ *     v1 = (A u + B) mod 256, for u in [0, 256) (a bijection).
+ *   Bucket b' in [0, 16) of the tile holds columns 256 tc + sigma(16 b' + k),
+ *   k = 0..15; global bucket b = 16 tc + b'.
+ *   Selection: per row and bucket the member with the smallest |w|, ties to the
+ *   smallest column; no importance.  Scale and codes as format 2.
+ *   Code storage: row-major, codes[i * K/16 + b].
+ *   Decode: w_hat[i][j] = float(codes[i][bucket of j]) * float(s16); the product
+ *   is computed as y = S (P^T x): bucket sums of x, then a dense code product.
+ *   usk_gemm does not take format 3 (USK_ERR_PARAMS); usk_gemv covers batch 1..15.
+ *
  * CONVENTIONS
  *   - All array pointers are DEVICE pointers owned by the caller; the library
  *     allocates no memory and keeps no state beyond cached kernel attributes.
@@ -83,7 +100,8 @@ extern "C" {
 
 #define USK_FORMAT_MAXKEY 1     /* format 1: one hash row, largest key kept   */
 #define USK_FORMAT_ABSMAXMIN 2  /* format 2: multi-row AbsMaxMin              */
-#define USK_FORMAT_VERSION 2    /* highest format this library builds and reads */
+#define USK_FORMAT_COLSHARED 3  /* format 3: column-shared projection, W_hat = S . P^T */
+#define USK_FORMAT_VERSION 3    /* highest format this library builds and reads */
 #define USK_ROWS_PER_BLOCK 64
 #define USK_TILE_COLS 256
 #define USK_WEIGHTS_PER_BUCKET 16
@@ -117,9 +135,9 @@ typedef enum {
 
 typedef enum { USK_F32 = 0, USK_BF16 = 1 } usk_dtype;
 
-/* Build parameters.  version: USK_FORMAT_MAXKEY or USK_FORMAT_ABSMAXMIN;
- * flags and reserved must be 0; depth = hash rows: 0 or 1 for format 1, 1, 2
- * or 4 for format 2.  Anything else: USK_ERR_PARAMS. */
+/* Build parameters.  version: USK_FORMAT_MAXKEY, USK_FORMAT_ABSMAXMIN or
+ * USK_FORMAT_COLSHARED; flags and reserved must be 0; depth = hash rows: 0 or 1
+ * for formats 1 and 3, 1, 2 or 4 for format 2.  Anything else: USK_ERR_PARAMS. */
 typedef struct {
   uint32_t version;
   uint32_t flags;
@@ -149,7 +167,7 @@ USK_API usk_status usk_sizes(int64_t M, int64_t K, size_t* code_bytes, size_t* s
  *              (ldw % 4 == 0 for fp32, % 8 == 0 for bf16).
  *   importance [K] fp32 per input column, or NULL for all ones.  Values must
  *              be finite with the sign bit clear (else USK_FLAG_BAD_IMPORTANCE).
- *              Format 2 takes no importance: non-NULL is USK_ERR_PARAMS.
+ *              Formats 2 and 3 take no importance: non-NULL is USK_ERR_PARAMS.
  *   params     format, depth and seed of the hash.
  *   codes      [M*K/16] int8 output, 16-byte aligned.   scales [M/64] output.
  *   d_status   optional device word for USK_FLAG_* bits.

@@ -2,7 +2,8 @@
 
 Thin Python face of libusk.so (C ABI in include/usk.h): ``usk_build`` compresses
 a weight matrix into a 0.5 bit/weight hashed sketch (format 1: one hash row,
-largest key kept; format 2: the multi-row AbsMaxMin sketch); ``usk_gemv`` (batch 1-15)
+largest key kept; format 2: the multi-row AbsMaxMin sketch; format 3: the
+column-shared projection W_hat = S . P^T, multiplied as S (P^T x)); ``usk_gemv`` (batch 1-15)
 and ``usk_gemm`` (batch 16-256) multiply the sketch with activations, rebuilding
 every weight on the fly.  PyTorch supplies device memory and streams only.
 """
@@ -12,6 +13,7 @@ from ._native import (  # noqa: F401
     FLAG_SCALE_OVERFLOW,
     FLAG_TIMEOUT,
     FORMAT_ABSMAXMIN,
+    FORMAT_COLSHARED,
     FORMAT_MAXKEY,
     FORMAT_VERSION,
     GEMM_MAX_BATCH,

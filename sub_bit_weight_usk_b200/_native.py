@@ -21,7 +21,8 @@ USK_F32 = 0
 USK_BF16 = 1
 FORMAT_MAXKEY = 1      # format 1: one hash row, the largest key kept per bucket
 FORMAT_ABSMAXMIN = 2   # format 2: multi-row AbsMaxMin (smallest |w| kept, largest over rows decoded)
-FORMAT_VERSION = 2     # highest format the library builds and reads
+FORMAT_COLSHARED = 3   # format 3: column-shared projection, W_hat = S . P^T, product as S (P^T x)
+FORMAT_VERSION = 3     # highest format the library builds and reads
 GEMV_MAX_BATCH = 15
 GEMM_MIN_BATCH = 16
 GEMM_MAX_BATCH = 256
@@ -167,8 +168,9 @@ def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int
     """Sketch of W [M, K] (bf16 or fp32, CUDA).  Outputs are allocated with torch
     when not given.  `status` is an optional int32 CUDA tensor of 1 element into
     which device-detected USK_FLAG_* bits are OR-ed.  version=FORMAT_ABSMAXMIN
-    builds the multi-row AbsMaxMin sketch with `depth` (1, 2 or 4) hash rows
-    (no importance)."""
+    builds the multi-row AbsMaxMin sketch with `depth` (1, 2 or 4) hash rows,
+    version=FORMAT_COLSHARED the column-shared projection sketch (no importance
+    for either)."""
     _need_cuda(W, importance, codes, scales, status)
     if W.dim() != 2 or W.stride(1) != 1:
         raise ValueError("W must be a 2-D row-major tensor")

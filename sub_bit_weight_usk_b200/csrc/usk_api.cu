@@ -13,6 +13,12 @@ cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t
 cudaError_t launch_build_amm(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed, int depth,
                              int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
                              int cluster_override, int inject);
+cudaError_t launch_build_cs(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed,
+                            int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
+                            int cluster_override, int inject);
+cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                           const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl,
+                           cudaStream_t stream, int tpb_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
                         cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth);
@@ -37,6 +43,7 @@ usk_status check_shape(int64_t M, int64_t K) {
 int format_depth(uint32_t version, uint32_t depth) {
   if (version == 0 || version == USK_FORMAT_MAXKEY) return depth <= 1 ? 1 : 0;
   if (version == USK_FORMAT_ABSMAXMIN) return (depth == 1 || depth == 2 || depth == 4) ? static_cast<int>(depth) : 0;
+  if (version == USK_FORMAT_COLSHARED) return depth <= 1 ? 1 : 0;
   return 0;
 }
 
@@ -77,7 +84,9 @@ USK_API const char* usk_status_str(usk_status status) {
     case USK_ERR_DTYPE: return "unknown dtype";
     case USK_ERR_BATCH: return "batch outside the range of this call";
     case USK_ERR_WORKSPACE: return "workspace missing or too small";
-    case USK_ERR_PARAMS: return "params NULL, unknown format, bad depth, non-zero flags or importance with format 2";
+    case USK_ERR_PARAMS:
+      return "params NULL, unknown format, bad depth, non-zero flags, importance with format 2 or 3, or usk_gemm "
+             "on a format-3 sketch";
     case USK_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     case USK_ERR_NONFINITE: return "non-finite weight";
     case USK_ERR_TIMEOUT: return "a bounded device wait gave up";
@@ -105,11 +114,13 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (wdtype != USK_F32 && wdtype != USK_BF16) return USK_ERR_DTYPE;
   if (!params) return USK_ERR_PARAMS;
   if (params->flags != 0 || params->reserved != 0) return USK_ERR_PARAMS;
-  if (params->version != USK_FORMAT_MAXKEY && params->version != USK_FORMAT_ABSMAXMIN) return USK_ERR_PARAMS;
+  if (params->version != USK_FORMAT_MAXKEY && params->version != USK_FORMAT_ABSMAXMIN &&
+      params->version != USK_FORMAT_COLSHARED)
+    return USK_ERR_PARAMS;
   const int depth = format_depth(params->version, params->depth);
   if (depth == 0) return USK_ERR_PARAMS;
-  const bool amm = params->version == USK_FORMAT_ABSMAXMIN;
-  if (amm && importance) return USK_ERR_PARAMS;
+  const bool amm = params->version == USK_FORMAT_ABSMAXMIN, cs = params->version == USK_FORMAT_COLSHARED;
+  if ((amm || cs) && importance) return USK_ERR_PARAMS;
   if (M == 0) return USK_OK;
   if (!scales) return USK_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(scales) & 1u) != 0) return USK_ERR_ALIGN;
@@ -120,10 +131,16 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (!aligned16(W) || !aligned16(codes)) return USK_ERR_ALIGN;
   if (ldw % (wdtype == USK_BF16 ? 8 : 4) != 0) return USK_ERR_ALIGN;
   if (importance && !aligned16(importance)) return USK_ERR_ALIGN;
-  cudaError_t e = amm ? usk::launch_build_amm(W, wdtype == USK_BF16, M, K, ldw, params->seed, depth, codes, scales,
-                                               d_status, s, g_build_cluster, g_inject == 1)
-                      : usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes,
-                                          scales, d_status, s, g_build_cluster, g_inject == 1);
+  cudaError_t e;
+  if (cs)
+    e = usk::launch_build_cs(W, wdtype == USK_BF16, M, K, ldw, params->seed, codes, scales, d_status, s,
+                             g_build_cluster, g_inject == 1);
+  else if (amm)
+    e = usk::launch_build_amm(W, wdtype == USK_BF16, M, K, ldw, params->seed, depth, codes, scales, d_status, s,
+                              g_build_cluster, g_inject == 1);
+  else
+    e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes, scales, d_status, s,
+                          g_build_cluster, g_inject == 1);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -143,6 +160,13 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
   if (!x) return USK_ERR_NULL;
   if (!aligned16(x)) return USK_ERR_ALIGN;
   if ((reinterpret_cast<uintptr_t>(y) & 3u) != 0) return USK_ERR_ALIGN;
+  if (sketch->version == USK_FORMAT_COLSHARED) {
+    cudaError_t e = usk::launch_gemv_cs(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
+                                        xdtype == USK_F32, static_cast<int>(batch), y, d_status,
+                                        (flags & USK_GEMV_PDL) != 0, s, g_gemv_tiles_per_block, g_inject == 3);
+    if (e != cudaSuccess) return USK_ERR_CUDA;
+    return from_cuda(cudaGetLastError());
+  }
   cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
                                    xdtype == USK_F32, static_cast<int>(batch), y, d_status,
                                    (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows,
@@ -162,6 +186,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   (void)ws_bytes;
   usk_status st = check_sketch(sketch);
   if (st != USK_OK) return st;
+  if (sketch->version == USK_FORMAT_COLSHARED) return USK_ERR_PARAMS;  // format 3: usk_gemv only
   if (batch < USK_GEMM_MIN_BATCH || batch > USK_GEMM_MAX_BATCH || batch % 16 != 0) return USK_ERR_BATCH;
   const int depth = format_depth(sketch->version, sketch->depth);
   if (!usk::gemm_supported(sketch->K, static_cast<int>(batch), depth)) return USK_ERR_SHAPE;

@@ -1,0 +1,542 @@
+// usk_cs.cu -- the column-shared projection sketch (format 3): build and
+// y = W_hat x for batch 1..15 as y = S (P^T x).
+//
+// "UltraSketchLLM" explainer, Resumen Tecnico, Metodologia §4 "Mapeo de
+// Operadores de Matriz Amigables con el Hardware": compression is a matrix
+// product with a projection matrix P whose reduction is a MIN over absolute
+// values, decompression the plain product W_hat = S . P^T, which turns the
+// irregular hash-and-gather access into coalesced, matrix-shaped traffic.
+//
+// Format 3 (include/usk.h): P is one-hot per input column and shared by all
+// rows.  Inside 256-column tile tc a seeded bijection sigma_tc of [0, 256) lists
+// the columns; bucket b' of the tile holds sigma_tc(16 b' + k), k = 0..15.  S
+// keeps per row and bucket the member of smallest |w| (ties: smallest column);
+// codes toward zero; row-major codes [M][K/16], one binary16 scale per 64 rows.
+//
+// Design (B200, sm_100a):
+//  * build: the format-1 skeleton (64 x 256 weight tiles by 2-D tensor copies
+//    into a double-buffered ring, a cluster per row block, the scale exchange
+//    through distributed shared memory).  The selection needs no atomics: a
+//    thread owns (row, bucket) pairs, reads the bucket's 16 members through the
+//    tile's sigma table and keeps the minimum of packed (|w|, column, sign) keys
+//    in registers.  Lanes of the second row of a warp walk the members from the
+//    middle so the two rows read different columns (fewer bank conflicts).
+//  * product: P^T x is a bucket sum of x -- K/16 values per batch row -- so the
+//    dense part S z streams one int8 code per 16 weights from HBM with coalesced
+//    16-byte loads, no gathers.  One thread block per (64-row block, 4 tiles);
+//    the blocks of a row block form a cluster.  Each block first issues its code
+//    loads, then builds z for its 64 buckets from x (four threads per bucket, 4
+//    members each, added in a fixed order), then every thread dots 16 codes per
+//    tile with z; the four lanes of a row combine by shuffles and the blocks'
+//    partials meet in the first block (st.async onto a transaction-counted
+//    mbarrier, added in rank order: deterministic).
+#include <cooperative_groups.h>
+
+#include "usk_common.cuh"
+
+namespace cg = cooperative_groups;
+
+namespace usk {
+
+// sigma_tc(u): seeded bijection of [0, 256) (every step is invertible on 8 bits).
+__device__ __forceinline__ uint32_t cs_sigma(uint3 key, uint32_t u) {
+  const uint32_t v1 = (key.x * u + key.y) & 255u;
+  const uint32_t v2 = v1 ^ (v1 >> 4);
+  const uint32_t v3 = (key.z * v2) & 255u;
+  return v3 ^ (v3 >> 3);
+}
+
+__host__ __device__ __forceinline__ uint3 cs_key(uint64_t seed, uint64_t tc) {
+  const uint64_t z = splitmix64(seed, tc + 1);
+  return make_uint3(static_cast<uint32_t>(z & 255u) | 1u, static_cast<uint32_t>((z >> 8) & 255u),
+                    static_cast<uint32_t>((z >> 16) & 255u) | 1u);
+}
+
+// ============================================================ build
+
+constexpr int kCsThreads = 256;
+
+struct BuildCsArgs {
+  const void* W;
+  int64_t ldw;
+  int64_t K;
+  uint64_t seed;
+  int8_t* codes;
+  uint16_t* scales;
+  uint32_t* status;
+  int T, C, tpc, nbuf;
+  int inject;  // test hook: block (0, 0) skips the copy of its first tile
+};
+
+struct BuildCsLayout {
+  uint32_t wbuf, sig, vals, bars, misc, total;
+};
+
+__host__ __device__ inline BuildCsLayout build_cs_layout(bool bf16, int tpc, int nbuf) {
+  const uint32_t tile = kRowsPerBlock * kTileCols * (bf16 ? 2u : 4u);
+  BuildCsLayout L;
+  L.wbuf = 0;
+  L.sig = L.wbuf + nbuf * tile;                                      // u8 [tpc][256]
+  L.vals = L.sig + static_cast<uint32_t>(tpc) * 256u;               // [tpc][64][16] kept values
+  L.bars = (L.vals + static_cast<uint32_t>(tpc) * 1024u * (bf16 ? 2u : 4u) + 7u) & ~7u;
+  L.misc = L.bars + 64u;
+  L.total = L.misc + 64u;
+  return L;
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kCsThreads, 2)
+    build_cs_kernel(const BuildCsArgs a, const __grid_constant__ CUtensorMap wmap) {
+  constexpr uint32_t kRowBytes = kTileCols * (BF16 ? 2 : 4);
+  constexpr uint32_t kTileBytes = kRowsPerBlock * kRowBytes;
+  extern __shared__ __align__(128) uint8_t smraw_unaligned[];
+  const BuildCsLayout L = build_cs_layout(BF16, a.tpc, a.nbuf);
+  const uint32_t s0 = (smem_u32(smraw_unaligned) + 1023u) & ~1023u;
+  uint8_t* smraw = smraw_unaligned + (s0 - smem_u32(smraw_unaligned));
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smraw + L.misc);
+  uint8_t* sig_all = smraw + L.sig;
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int rb = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nt = (a.T - crank + a.C - 1) / a.C;  // this block's tiles: crank, crank + C, ...
+
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  if (tid == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
+  auto issue = [&](int i) {
+    const int tc = crank + a.C * i;
+    const int buf = i % a.nbuf;
+    const uint32_t bar = s0 + L.bars + 8 * buf;
+    mbar_arrive_expect_tx(bar, kTileBytes);
+    tma_load_2d(s0 + L.wbuf + buf * kTileBytes, &wmap, tc * kTileCols, rb * kRowsPerBlock, bar);
+  };
+  if (tid == 0) {
+    for (int b = 0; b < a.nbuf; ++b) mbar_init(s0 + L.bars + 8 * b, 1);
+    mbar_fence_init();
+    misc[0] = 0u;
+    for (int i = 0; i < a.nbuf && i < nt; ++i)
+      if (!(a.inject && i == 0 && crank == 0 && rb == 0)) issue(i);
+  }
+  // the column lists of this block's tiles, while the first weights stream in
+  for (int q = tid; q < nt * 256; q += kCsThreads) {
+    const int i = q >> 8;
+    sig_all[q] = static_cast<uint8_t>(cs_sigma(cs_key(a.seed, static_cast<uint64_t>(crank + a.C * i)), q & 255));
+  }
+  __syncthreads();
+
+  uint32_t flags = 0;
+  uint32_t vmax = 0;
+  using ValT = typename std::conditional<BF16, uint16_t, uint32_t>::type;
+  ValT* vals_all = reinterpret_cast<ValT*>(smraw + L.vals);
+  // pair p = tid + 256 e: row r = p / 16, bucket b' = p % 16; a warp covers 2 rows
+  const int bq = tid & 15;
+  const int kofs = (lane >> 4) * 8;  // second row of the warp starts half-way round
+
+  for (int i = 0; i < nt; ++i) {
+    const int buf = i % a.nbuf;
+    if (!mbar_wait(s0 + L.bars + 8 * buf, (i / a.nbuf) & 1)) flags |= USK_FLAG_TIMEOUT;
+    const uint8_t* wt = smraw + L.wbuf + buf * kTileBytes;
+    const uint8_t* sig = sig_all + i * 256 + 16 * bq;
+    ValT* vals = vals_all + i * 1024;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = (tid >> 4) + 16 * e;
+      if (BF16) {
+        const uint16_t* wrow = reinterpret_cast<const uint16_t*>(wt + r * kRowBytes);
+        uint32_t best = 0xFFFFFFFFu, nf = 0u;
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          const uint32_t c = sig[(kk + kofs) & 15];
+          const uint32_t b16 = wrow[c];
+          nf |= (b16 & 0x7F80u) + 0x80u;  // exponent all ones -> bit 15
+          best = min(best, ((b16 & 0x7FFFu) << 16) | (c << 1) | (b16 >> 15));
+        }
+        if (nf & 0x8000u) flags |= USK_FLAG_NONFINITE_W;
+        const uint32_t vb = ((best >> 16) & 0x7FFFu) | ((best & 1u) << 15);
+        vals[r * 16 + bq] = static_cast<ValT>(vb);
+        vmax = max(vmax, (vb & 0x7FFFu) << 16);
+      } else {
+        const uint32_t* wrow = reinterpret_cast<const uint32_t*>(wt + r * kRowBytes);
+        uint64_t best = ~0ull;
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          const uint32_t c = sig[(kk + kofs) & 15];
+          const uint32_t wb = wrow[c];
+          if ((wb & 0x7F800000u) == 0x7F800000u) flags |= USK_FLAG_NONFINITE_W;
+          best = min(best, (static_cast<uint64_t>(wb & 0x7FFFFFFFu) << 32) | (c << 1) | (wb >> 31));
+        }
+        const uint32_t vb = static_cast<uint32_t>(best >> 32) | (static_cast<uint32_t>(best & 1u) << 31);
+        vals[r * 16 + bq] = static_cast<ValT>(vb);
+        vmax = max(vmax, vb & 0x7FFFFFFFu);
+      }
+    }
+    __syncthreads();  // tile i resolved; its weight buffer is free
+    if (tid == 0 && i + a.nbuf < nt) issue(i + a.nbuf);
+  }
+
+  // ---- row-block maximum through distributed shared memory (as format 1)
+  vmax = __reduce_max_sync(0xFFFFFFFFu, vmax);
+  if (lane == 0) atomicMax(&misc[0], vmax);
+  __syncthreads();
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (warp == 0 && lane < a.C && lane != crank) atomicMax(cluster.map_shared_rank(&misc[0], lane), misc[0]);
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  const float mx = __uint_as_float(misc[0]);
+  const __half s16 = __float2half_rn(mx / 127.0f);
+  const float sc = __half2float(s16);
+  if (crank == 0 && tid == 0) {
+    a.scales[rb] = __half_as_ushort(s16);
+    if (isinf(sc)) flags |= USK_FLAG_SCALE_OVERFLOW;
+  }
+  // codes toward zero (as format 2); one 16-byte store per (row, tile):
+  // codes[(64 rb + r) * K/16 + 16 tc + b']
+  const int64_t nbk = a.K / 16;
+  for (int q = tid; q < nt * 64; q += kCsThreads) {
+    const int i = q >> 6, r = q & 63;
+    const int tc = crank + a.C * i;
+    const ValT* v16 = vals_all + i * 1024 + r * 16;
+    uint32_t w4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const uint32_t vb = v16[e];
+      const float v = BF16 ? __uint_as_float(vb << 16) : __uint_as_float(vb);
+      int code = 0;
+      if (sc != 0.0f) {
+        const float m = fabsf(v);
+        float t = fminf(truncf(m / sc), 127.0f);
+        if (t * sc > m) t -= 1.0f;
+        code = static_cast<int>(t);
+        if (v < 0.0f) code = -code;
+      }
+      w4[e >> 2] |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * (e & 3));
+    }
+    int8_t* dst = a.codes + (static_cast<int64_t>(rb) * 64 + r) * nbk + 16 * static_cast<int64_t>(tc);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+  report(a.status, flags);
+}
+
+template <bool BF16>
+static cudaError_t launch_build_cs_t(BuildCsArgs a, int64_t RB, cudaStream_t stream, int cluster_override) {
+  auto mk = [&](int C, int nbuf) {
+    a.C = C < a.T ? C : a.T;
+    a.tpc = (a.T + a.C - 1) / a.C;
+    a.nbuf = nbuf;
+    return build_cs_layout(BF16, a.tpc, nbuf).total + 1024u;  // + alignment slack
+  };
+  uint32_t smem;
+  if (cluster_override > 0) {
+    smem = mk(cluster_override, 2);
+    if (smem > 220u * 1024u) smem = mk(cluster_override, 1);
+  } else {
+    smem = mk(4, 2);
+    if (smem > 112u * 1024u && a.T > 4) smem = mk(8, 2);
+    if (smem > 112u * 1024u && a.T > 8) smem = mk(16, 2);
+    if (smem > 220u * 1024u) smem = mk(a.C, 1);
+  }
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  CUtensorMap wmap;
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(RB * kRowsPerBlock)};
+  const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(a.ldw) * (BF16 ? 2u : 4u)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileCols), static_cast<cuuint32_t>(kRowsPerBlock)};
+  const cuuint32_t estride[2] = {1, 1};
+  if (encode(&wmap, BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+             const_cast<void*>(a.W), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  auto kern = build_cs_kernel<BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  if (a.C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.blockDim = dim3(kCsThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, wmap);
+}
+
+cudaError_t launch_build_cs(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed,
+                            int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
+                            int cluster_override, int inject) {
+  BuildCsArgs a;
+  a.W = W; a.ldw = ldw; a.K = K; a.seed = seed;
+  a.codes = codes; a.scales = scales; a.status = status;
+  a.T = static_cast<int>(K / kTileCols);
+  a.C = a.tpc = a.nbuf = 0;
+  a.inject = inject;
+  const int64_t RB = M / kRowsPerBlock;
+  return bf16 ? launch_build_cs_t<true>(a, RB, stream, cluster_override)
+              : launch_build_cs_t<false>(a, RB, stream, cluster_override);
+}
+
+// ============================================================ product
+
+struct GemvCsArgs {
+  const int8_t* codes;
+  const uint16_t* scales;
+  const void* x;
+  float* y;
+  int64_t M, K;
+  uint64_t seed;
+  uint32_t* status;
+  int T, C, tpb;  // tiles per row block, blocks per row block, tiles per block
+  int pdl;
+  int inject;  // test hook: block 1 of row block 0 skips its partial sums
+};
+
+constexpr int kCsMaxTiles = 16;  // tiles per block
+constexpr int kCsMaxBatch = 15;
+
+struct GemvCsLayout {
+  uint32_t z, red, push, bars, total;
+};
+
+__host__ __device__ inline GemvCsLayout gemv_cs_layout(int tpb, int batch, int C) {
+  GemvCsLayout L;
+  L.z = 0;                                                                  // fp32 [batch][16 tpb]
+  L.red = L.z + static_cast<uint32_t>(batch * 16 * tpb) * 4u;              // (unused slot, keeps 16-B alignment)
+  L.push = (L.red + 15u) & ~15u;                                            // fp32 [C][batch][64] (rank 0)
+  L.bars = (L.push + static_cast<uint32_t>(C * batch * 64) * 4u + 7u) & ~7u;
+  L.total = L.bars + 8u;
+  return L;
+}
+
+__device__ __forceinline__ uint32_t cs_mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cs_st_async_f32(uint32_t remote_addr, float v, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(remote_addr),
+               "r"(__float_as_uint(v)), "r"(remote_bar)
+               : "memory");
+}
+
+template <int B, bool XF32>
+__global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = static_cast<int>(cluster.block_rank());
+  const int rb = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int t0 = crank * a.tpb;
+  const int nt = min(a.tpb, a.T - t0);
+  const GemvCsLayout L = gemv_cs_layout(a.tpb, B, a.C);
+  const uint32_t s0 = smem_u32(sm);
+  const uint32_t push_bar = s0 + L.bars;
+  float* zs = reinterpret_cast<float*>(sm + L.z);
+  float* push = reinterpret_cast<float*>(sm + L.push);
+  const int nbk = 16 * a.tpb;  // bucket slots per block (z row stride)
+  constexpr uint32_t kPartBytes = static_cast<uint32_t>(B) * 64u * 4u;
+
+  // ---- code loads first (never written by a programmatic-dependent neighbour):
+  // thread (row r, quarter q) takes tiles q, q + 4, ... of its row
+  const int r = tid >> 2, q4 = tid & 3;
+  const int8_t* crow = a.codes + (static_cast<int64_t>(rb) * 64 + r) * (a.K / 16) + 16 * static_cast<int64_t>(t0);
+  uint4 cv[kCsMaxTiles / 4];
+#pragma unroll
+  for (int u = 0; u < kCsMaxTiles / 4; ++u) {
+    const int tl = q4 + 4 * u;
+    cv[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (tl < nt) cv[u] = ldg_nc128(crow + 16 * tl);
+  }
+  if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0 && a.C > 1) {
+    mbar_init(push_bar, 1);
+    mbar_fence_init();
+    if (crank == 0) mbar_arrive_expect_tx(push_bar, static_cast<uint32_t>(a.C - 1) * kPartBytes);
+  }
+  if (a.C > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+
+  // ---- z = P^T x for this block's buckets: four threads per bucket, members
+  // 4 m4 .. 4 m4 + 3 each, added in member order, then the quarters in order
+  for (int bb = tid >> 2; bb < nt * 16; bb += kCsThreads / 4) {
+    const int m4 = tid & 3;
+    const int tl = bb >> 4, bp = bb & 15;
+    const uint3 key = cs_key(a.seed, static_cast<uint64_t>(t0 + tl));
+    const int64_t col0 = static_cast<int64_t>(t0 + tl) * kTileCols;
+    uint32_t c[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) c[k] = cs_sigma(key, static_cast<uint32_t>(16 * bp + 4 * m4 + k));
+    float xv[B][4];
+#pragma unroll
+    for (int t = 0; t < B; ++t)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int64_t idx = static_cast<int64_t>(t) * a.K + col0 + c[k];
+        if (XF32) xv[t][k] = __ldg(static_cast<const float*>(a.x) + idx);
+        else xv[t][k] = __uint_as_float(static_cast<uint32_t>(__ldg(static_cast<const unsigned short*>(a.x) + idx)) << 16);
+      }
+#pragma unroll
+    for (int t = 0; t < B; ++t) {
+      float s = ((xv[t][0] + xv[t][1]) + xv[t][2]) + xv[t][3];
+      const float s1 = __shfl_xor_sync(0xFFFFFFFFu, s, 1);
+      const float pair = (m4 & 1) ? (s1 + s) : (s + s1);     // (q0 + q1), (q2 + q3)
+      const float p2 = __shfl_xor_sync(0xFFFFFFFFu, pair, 2);
+      const float tot = (m4 & 2) ? (p2 + pair) : (pair + p2);  // (q0 + q1) + (q2 + q3)
+      if (m4 == 0) zs[t * nbk + bb] = tot;
+    }
+  }
+  __syncthreads();
+  if (a.C > 1 && crank != 0) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+
+  // ---- S z: 16 codes per tile per thread against the tile's 16 z values
+  float acc[B];
+#pragma unroll
+  for (int t = 0; t < B; ++t) acc[t] = 0.0f;
+#pragma unroll
+  for (int u = 0; u < kCsMaxTiles / 4; ++u) {
+    const int tl = q4 + 4 * u;
+    if (tl < nt) {
+      const uint32_t ws[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
+      float cf[16];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = i8pair_to_bf16x2<0x4140>(ws[e]), hi = i8pair_to_bf16x2<0x4342>(ws[e]);
+        cf[4 * e + 0] = bf16lo(lo);
+        cf[4 * e + 1] = bf16hi(lo);
+        cf[4 * e + 2] = bf16lo(hi);
+        cf[4 * e + 3] = bf16hi(hi);
+      }
+#pragma unroll
+      for (int t = 0; t < B; ++t) {
+        const float4* zt = reinterpret_cast<const float4*>(zs + t * nbk + 16 * tl);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 z4 = zt[e];
+          acc[t] = fmaf(cf[4 * e + 0], z4.x, acc[t]);
+          acc[t] = fmaf(cf[4 * e + 1], z4.y, acc[t]);
+          acc[t] = fmaf(cf[4 * e + 2], z4.z, acc[t]);
+          acc[t] = fmaf(cf[4 * e + 3], z4.w, acc[t]);
+        }
+      }
+    }
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // the four lanes of a row, in quarter order
+#pragma unroll
+  for (int t = 0; t < B; ++t) {
+    const float o1 = __shfl_xor_sync(0xFFFFFFFFu, acc[t], 1);
+    const float pr = (q4 & 1) ? (o1 + acc[t]) : (acc[t] + o1);
+    const float o2 = __shfl_xor_sync(0xFFFFFFFFu, pr, 2);
+    acc[t] = (q4 & 2) ? (o2 + pr) : (pr + o2);
+  }
+  const float s = __half2float(__ushort_as_half(a.scales[rb]));
+  float* yrb = a.y + static_cast<int64_t>(rb) * 64;
+  if (a.C == 1) {
+    if (q4 == 0) {
+#pragma unroll
+      for (int t = 0; t < B; ++t) yrb[static_cast<int64_t>(t) * a.M + r] = acc[t] * s;
+    }
+    return;
+  }
+  if (crank != 0) {
+    if (a.inject && crank == 1 && rb == 0) return;  // test hook: the first block's wait gives up
+    if (q4 == 0) {
+      const uint32_t bar0 = cs_mapa(push_bar, 0);
+#pragma unroll
+      for (int t = 0; t < B; ++t)
+        cs_st_async_f32(cs_mapa(s0 + L.push + (static_cast<uint32_t>(crank * B + t) * 64u + r) * 4u, 0), acc[t],
+                        bar0);
+    }
+    return;
+  }
+  if (q4 == 0) {
+#pragma unroll
+    for (int t = 0; t < B; ++t) push[t * 64 + r] = acc[t];
+  }
+  if (!mbar_wait(push_bar, 0)) report(a.status, USK_FLAG_TIMEOUT);  // bounded (about 1 s)
+  __syncthreads();
+  for (int qq = tid; qq < B * 64; qq += kCsThreads) {
+    float tot = 0.0f;
+    for (int c = 0; c < a.C; ++c) tot += push[c * B * 64 + qq];
+    yrb[static_cast<int64_t>(qq / 64) * a.M + qq % 64] = tot * s;
+  }
+  (void)lane;
+}
+
+template <int B, bool XF32>
+static cudaError_t launch_gemv_cs_t(GemvCsArgs a, int64_t RB, cudaStream_t stream) {
+  const size_t smem = gemv_cs_layout(a.tpb, B, a.C).total;
+  auto kern = gemv_cs_kernel<B, XF32>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  if (a.C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.blockDim = dim3(kCsThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <bool XF32>
+static cudaError_t launch_gemv_cs_b(const GemvCsArgs& a, int batch, int64_t RB, cudaStream_t stream) {
+  switch (batch) {
+    case 1: return launch_gemv_cs_t<1, XF32>(a, RB, stream);
+    case 2: return launch_gemv_cs_t<2, XF32>(a, RB, stream);
+    case 3: return launch_gemv_cs_t<3, XF32>(a, RB, stream);
+    case 4: return launch_gemv_cs_t<4, XF32>(a, RB, stream);
+    case 5: return launch_gemv_cs_t<5, XF32>(a, RB, stream);
+    case 6: return launch_gemv_cs_t<6, XF32>(a, RB, stream);
+    case 7: return launch_gemv_cs_t<7, XF32>(a, RB, stream);
+    case 8: return launch_gemv_cs_t<8, XF32>(a, RB, stream);
+    case 9: return launch_gemv_cs_t<9, XF32>(a, RB, stream);
+    case 10: return launch_gemv_cs_t<10, XF32>(a, RB, stream);
+    case 11: return launch_gemv_cs_t<11, XF32>(a, RB, stream);
+    case 12: return launch_gemv_cs_t<12, XF32>(a, RB, stream);
+    case 13: return launch_gemv_cs_t<13, XF32>(a, RB, stream);
+    case 14: return launch_gemv_cs_t<14, XF32>(a, RB, stream);
+    default: return launch_gemv_cs_t<15, XF32>(a, RB, stream);
+  }
+}
+
+// Tiles per block: tpb_override if given, else 4; raised until the cluster has
+// at most 16 blocks.
+cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                           const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl,
+                           cudaStream_t stream, int tpb_override, int inject) {
+  GemvCsArgs a;
+  a.codes = codes; a.scales = scales; a.x = x; a.y = y;
+  a.M = M; a.K = K; a.seed = seed; a.status = status;
+  a.T = static_cast<int>(K / kTileCols);
+  a.tpb = tpb_override > 0 ? tpb_override : 4;
+  if (a.tpb > kCsMaxTiles) a.tpb = kCsMaxTiles;
+  if (a.tpb > a.T) a.tpb = a.T;
+  while ((a.T + a.tpb - 1) / a.tpb > 16 && a.tpb < kCsMaxTiles) ++a.tpb;
+  a.C = (a.T + a.tpb - 1) / a.tpb;
+  if (a.C > 16 || batch < 1 || batch > kCsMaxBatch) return cudaErrorInvalidValue;
+  a.pdl = pdl ? 1 : 0;
+  a.inject = inject;
+  const int64_t RB = M / kRowsPerBlock;
+  return xf32 ? launch_gemv_cs_b<true>(a, batch, RB, stream) : launch_gemv_cs_b<false>(a, batch, RB, stream);
+}
+
+}  // namespace usk
