@@ -7,7 +7,11 @@ batch 1 (rehash + gather decode, product) and usk_gemm at batch 16 (decode into
 tcgen05 tiles).  The headline value is usk_gemv GB/s (algorithmic bytes of one
 call / its average launch duration); usk_build Gweights/s rides along.  A second
 timed region runs the same three calls K times on the multi-row AbsMaxMin sketch
-(format 2, depth 2) of the same layer and reports them under "absmaxmin".
+(format 2, depth 2) of the same layer and reports them under "absmaxmin"; a
+third runs K builds and K batch-1 GEMVs of the column-shared projection sketch
+(format 3, y = S (P^T x)) and a fourth the "matrix vs hash" A/B: K batch-1 GEMVs
+of a 28672x8192 layer in format 1 (per-weight rehash and gather) and in format 3
+(bucket sums of x, then dense codes), reported under "colshared".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl usk|reference]
 
@@ -43,6 +47,8 @@ N_WCOPIES = 8      # 8 x 32 MiB of weights per build cycle  (> L2)
 N_SKETCHES = 256   # 256 x 1 MiB of codes per decode cycle  (> L2)
 GRAPH_STEPS = 256  # steps per captured CUDA graph
 AMM_DEPTH = 2      # hash rows of the format-2 (multi-row AbsMaxMin) measurement
+AB_M, AB_K = 28672, 8192  # the matrix-vs-hash A/B shape (70B MLP up-projection)
+AB_COPIES = 10            # 10 x 14 MiB of codes per format (> L2)
 
 METRIC = "usk_gemv GB/s & % roofline (4096x4096, batch 1); usk_build Gweights/s"
 WORKLOAD = ("one 4096x4096 bf16 layer, Student-t(4) x 0.02 with 0.1% outliers x20, importance = mean |x| "
@@ -104,6 +110,22 @@ def rooflines(peaks, t_build_s, t_gemv_s, t_gemm_s, traffic, depth=1, build_byte
                            traffic.get("usk_gemm"))
     out["usk_gemm"]["tensor_tflops"] = round(GEMM_FLOPS / t_gemm_s / 1e12, 3)
     return out
+
+
+def colshared_rooflines(peaks, t_build_s, t_gemv_s, t_gemv_ab_s, traffic):
+    """Format 3: the build reads W once (HBM); the product streams 1/16 B of
+    code per weight with no gathers, so its bound is HBM too."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    src = peaks["source"]
+
+    def line(achieved, tr):
+        return {"bound": "hbm", "achieved": round(achieved, 3), "peak": round(hbm / 1e9, 3), "unit": "GB/s",
+                "frac": round(achieved / (hbm / 1e9), 4), "traffic": tr, "peak_source": src}
+
+    ab_bytes = AB_M * AB_K // 16 + 2 * (AB_M // 64) + 2 * AB_K + 4 * AB_M
+    return {"usk_build": line((BUILD_BYTES - 4 * K) / t_build_s / 1e9, traffic.get("cs_usk_build")),
+            "usk_gemv": line(GEMV_BYTES / t_gemv_s / 1e9, traffic.get("cs_usk_gemv")),
+            "usk_gemv_%dx%d" % (AB_M, AB_K): line(ab_bytes / t_gemv_ab_s / 1e9, traffic.get("cs_usk_gemv_ab"))}
 
 
 def source_sha(name):
@@ -382,13 +404,46 @@ def run_usk(args):
         return [ev[k].elapsed_time(ev[k + 1]) * 1e-3 / n for k in range(len(graphs))] + \
             [ev[0].elapsed_time(ev[-1]) * 1e-3]
 
+    # format 3 (column-shared projection) on the same layer: build and GEMV
+    cs = usk.FORMAT_COLSHARED
+    sk3 = usk.usk_build(W, None, seed, version=cs)
+    sks3 = [usk.Sketch(M, K, seed, sk3.codes.clone(), sk3.scales.clone(), cs, 1) for _ in range(N_SKETCHES)]
+
+    def build3(i):
+        b = sks3[i % N_SKETCHES]
+        usk.usk_build(Ws[i % N_WCOPIES], None, seed, codes=b.codes, scales=b.scales, status=status, version=cs)
+
+    def gemv3(i):
+        usk.usk_gemv(sks3[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1, pdl=True)
+
+    # the matrix-vs-hash A/B at 28672 x 8192, batch 1 (device-drawn N(0, 0.02^2)
+    # weights: the values do not change the decode work)
+    Wab = gen.device_weights_normal(AB_M, AB_K, 3, 0.02, dev)
+    skh = usk.usk_build(Wab, None, 3)
+    skm = usk.usk_build(Wab, None, 3, version=cs)
+    del Wab
+    abh = [usk.Sketch(AB_M, AB_K, 3, skh.codes.clone(), skh.scales.clone()) for _ in range(AB_COPIES)]
+    abm = [usk.Sketch(AB_M, AB_K, 3, skm.codes.clone(), skm.scales.clone(), cs, 1) for _ in range(AB_COPIES)]
+    xab = torch.from_numpy(gen.activations(1, AB_K, 3, "bf16").view(np.int16)).to(dev).view(torch.bfloat16)
+    yab = torch.empty((1, AB_M), device=dev)
+
+    def gemv_hash(i):
+        usk.usk_gemv(abh[i % AB_COPIES], xab, y=yab, pdl=True)
+
+    def gemv_matrix(i):
+        usk.usk_gemv(abm[i % AB_COPIES], xab, y=yab, pdl=True)
+
     graphs1 = prepare((build, gemv, gemm))
     graphs2 = prepare((build2, gemv2, gemm2))
+    graphs3 = prepare((build3, gemv3))
+    graphs4 = prepare((gemv_hash, gemv_matrix))
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
     t_build, t_gemv, t_gemm, t_total = timed(graphs1)
     t_build2, t_gemv2, t_gemm2, _ = timed(graphs2)
+    t_build3, t_gemv3, _ = timed(graphs3)
+    t_hash, t_matrix, _ = timed(graphs4)
     sampler.stop()
     t_step = t_total / max(args.steps, 1)
 
@@ -409,8 +464,9 @@ def run_usk(args):
     t_e2e = (time.perf_counter() - t0) / n_e2e
 
     # max over ranks
-    t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2 = max_over_ranks(
-        [t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2], device=dev)
+    (t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2, t_build3, t_gemv3, t_hash,
+     t_matrix) = max_over_ranks([t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2,
+                                 t_build3, t_gemv3, t_hash, t_matrix], device=dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -473,6 +529,24 @@ def run_usk(args):
             "rooflines": rl2,
             "gpu_launches": 3 * args.steps,
         },
+        "colshared": {
+            "format": "column-shared projection sketch (format 3): W_hat = S . P^T with one seeded one-hot P "
+                      "shared by all rows; product y = S (P^T x); same layer, no importance",
+            "timing": "third timed region: K builds and K GEMVs (batch 1) as CUDA graphs; fourth: K batch-1 "
+                      "GEMVs of a %dx%d layer in format 1 and in format 3, %d sketch copies each (> L2)"
+                      % (AB_M, AB_K, AB_COPIES),
+            "usk_gemv_gbs": round(world * GEMV_BYTES / t_gemv3 / 1e9, 3),
+            "usk_build_gweights_per_s": round(world * N_W / t_build3 / 1e9, 3),
+            "kernel_us": {"usk_build": round(t_build3 * 1e6, 3), "usk_gemv": round(t_gemv3 * 1e6, 3)},
+            "rooflines": colshared_rooflines(peaks, t_build3, t_gemv3, t_matrix, tr),
+            "matrix_vs_hash": {
+                "shape": "%dx%d" % (AB_M, AB_K), "batch": 1, "data": "device-drawn bf16 N(0, 0.02^2) weights",
+                "hash_gemv_us": round(t_hash * 1e6, 3), "matrix_gemv_us": round(t_matrix * 1e6, 3),
+                "speedup": round(t_hash / t_matrix, 2),
+                "layer_4096_speedup": round(t_gemv / t_gemv3, 2),
+            },
+            "gpu_launches": 4 * args.steps,
+        },
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -491,8 +565,15 @@ def run_profile_case(args):
     x16 = torch.from_numpy(cfg["x"].view(np.int16)).to(dev).view(torch.bfloat16)
     x1 = x16[:GEMV_BATCH].contiguous()
     case = args.profile_case
-    fmt = {} if not case.endswith("_amm") else {"version": usk.FORMAT_ABSMAXMIN, "depth": AMM_DEPTH}
-    imp_c = imp if not fmt else None
+    fmt = {}
+    if case.endswith("_amm"):
+        fmt = {"version": usk.FORMAT_ABSMAXMIN, "depth": AMM_DEPTH}
+    elif "_cs" in case:
+        fmt = {"version": usk.FORMAT_COLSHARED}
+    if case.endswith("_ab"):  # the 28672 x 8192 A/B shape, device-drawn weights
+        W = gen.device_weights_normal(AB_M, AB_K, 3, 0.02, dev)
+        x1 = torch.from_numpy(gen.activations(1, AB_K, 3, "bf16").view(np.int16)).to(dev).view(torch.bfloat16)
+    imp_c = imp if not fmt and not case.endswith("_ab") else None
     sk = usk.usk_build(W, imp_c, cfg["seed"], **fmt)
     torch.cuda.synchronize()
     for _ in range(3 + 3):  # 3 warm-up launches, then 3 to capture
@@ -514,7 +595,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="usk", choices=["usk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile-case", choices=["build", "gemv", "gemm", "build_amm", "gemv_amm", "gemm_amm"],
+    ap.add_argument("--profile-case", choices=["build", "gemv", "gemm", "build_amm", "gemv_amm", "gemm_amm",
+                                               "build_cs", "gemv_cs", "gemv_ab", "gemv_cs_ab"],
                     default=None,
                     help="run 6 launches of one kernel on the bench workload (for ncu) and exit")
     args = ap.parse_args(argv)

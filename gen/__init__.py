@@ -1,9 +1,10 @@
 """Seeded synthetic inputs shared by the tests, the smoke check and the bench.
 
 This module holds none of the sketch's arithmetic: it only draws weights,
-importance vectors and activations with numpy's PCG64 generator (or torch's
-generator for the device-side bulk fill of the largest workloads) and rounds
-float32 draws to bfloat16 bit patterns.  Both the CPU oracle and the CUDA path
+importance vectors and activations with numpy's PCG64 generator and rounds
+float32 draws to bfloat16 bit patterns (``device_weights_normal`` draws with
+torch's seeded CUDA generator instead: a fast fill of the largest matrices for
+timing runs only, where the values do not change the work).  Both the CPU oracle and the CUDA path
 consume the arrays it returns, so neither side generates its own inputs.
 
 bf16 arrays are returned as numpy uint16 bit patterns (numpy has no bfloat16).
@@ -137,6 +138,15 @@ def mlp70b(name: str, batch: int = 16):
     M, K = MLP70B_SHAPES[name]
     return {"seed": seed, "W": weights_student_t(M, K, seed, 4.0, 0.02, 0.0, 20.0, "bf16"),
             "importance": None, "x": activations(batch, K, seed, "bf16")}
+
+
+def device_weights_normal(M: int, K: int, seed: int, std: float = 0.02, device="cuda"):
+    """bf16 N(0, std^2) [M, K] drawn on the device by torch's seeded generator
+    (timing inputs only; not reproducible against the numpy streams)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return (torch.randn((M, K), generator=g, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
 
 
 def stack7b_seed(layer_idx: int, linear: str) -> int:

@@ -227,9 +227,9 @@ USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block)
  * process-wide. */
 USK_API void usk_debug_set_gemv_path(int path);
 
-/* Test hook: rows per thread block of the row-slab path (16, 32 or 64; any
- * other value restores the automatic choice).  The result does not depend on
- * it; process-wide. */
+/* Test hook: rows per thread block of the row-slab path (16, 32 or 64) and of
+ * the format-3 product (64 or 256); any other value restores the automatic
+ * choice.  Results stay within the products' tolerance; process-wide. */
 USK_API void usk_debug_set_gemv_rows(int rows);
 
 /* Test hook for the failure path (host-made; no device fault): kernel = 1 makes

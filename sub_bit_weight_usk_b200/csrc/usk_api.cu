@@ -18,7 +18,7 @@ cudaError_t launch_build_cs(const void* W, bool bf16, int64_t M, int64_t K, int6
                             int cluster_override, int inject);
 cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl,
-                           cudaStream_t stream, int tpb_override, int inject);
+                           cudaStream_t stream, int tpb_override, int rows_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
                         cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth);
@@ -163,7 +163,8 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
   if (sketch->version == USK_FORMAT_COLSHARED) {
     cudaError_t e = usk::launch_gemv_cs(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
                                         xdtype == USK_F32, static_cast<int>(batch), y, d_status,
-                                        (flags & USK_GEMV_PDL) != 0, s, g_gemv_tiles_per_block, g_inject == 3);
+                                        (flags & USK_GEMV_PDL) != 0, s, g_gemv_tiles_per_block, g_gemv_rows,
+                                        g_inject == 3);
     if (e != cudaSuccess) return USK_ERR_CUDA;
     return from_cuda(cudaGetLastError());
   }

@@ -23,13 +23,16 @@
 //    middle so the two rows read different columns (fewer bank conflicts).
 //  * product: P^T x is a bucket sum of x -- K/16 values per batch row -- so the
 //    dense part S z streams one int8 code per 16 weights from HBM with coalesced
-//    16-byte loads, no gathers.  One thread block per (64-row block, 4 tiles);
-//    the blocks of a row block form a cluster.  Each block first issues its code
-//    loads, then builds z for its 64 buckets from x (four threads per bucket, 4
-//    members each, added in a fixed order), then every thread dots 16 codes per
-//    tile with z; the four lanes of a row combine by shuffles and the blocks'
-//    partials meet in the first block (st.async onto a transaction-counted
-//    mbarrier, added in rank order: deterministic).
+//    16-byte loads, no gathers.  One thread block per (R rows, tpb tiles), R =
+//    64 or 256; the blocks along K form a cluster.  Each block first issues
+//    its code loads, then builds z for its 16 tpb buckets from x (16/tpb threads
+//    per bucket, added in a fixed order), then every thread dots its row's codes
+//    with z (broadcast shared-memory reads); the lanes of a row combine by
+//    shuffles and the blocks' partials meet in the first block (st.async onto a
+//    transaction-counted mbarrier, added in rank order: deterministic).  Tall
+//    matrices take 256-row blocks, which amortise the bucket sums over more
+//    rows (at 64 rows the kernel was measured instruction-bound, 78 % issue, on
+//    28672 x 8192); smaller ones keep 64-row blocks with fewer registers.
 #include <cooperative_groups.h>
 
 #include "usk_common.cuh"
@@ -293,24 +296,24 @@ struct GemvCsArgs {
   int64_t M, K;
   uint64_t seed;
   uint32_t* status;
-  int T, C, tpb;  // tiles per row block, blocks per row block, tiles per block
+  int T, C, tpb;  // tiles per row, blocks along K (cluster size), tiles per block (power of two)
+  int R;          // rows per block: 64 or 256
   int pdl;
-  int inject;  // test hook: block 1 of row block 0 skips its partial sums
+  int inject;  // test hook: block 1 of the first row group skips its partial sums
 };
 
 constexpr int kCsMaxTiles = 16;  // tiles per block
 constexpr int kCsMaxBatch = 15;
 
 struct GemvCsLayout {
-  uint32_t z, red, push, bars, total;
+  uint32_t z, push, bars, total;
 };
 
-__host__ __device__ inline GemvCsLayout gemv_cs_layout(int tpb, int batch, int C) {
+__host__ __device__ inline GemvCsLayout gemv_cs_layout(int tpb, int batch, int C, int R) {
   GemvCsLayout L;
   L.z = 0;                                                                  // fp32 [batch][16 tpb]
-  L.red = L.z + static_cast<uint32_t>(batch * 16 * tpb) * 4u;              // (unused slot, keeps 16-B alignment)
-  L.push = (L.red + 15u) & ~15u;                                            // fp32 [C][batch][64] (rank 0)
-  L.bars = (L.push + static_cast<uint32_t>(C * batch * 64) * 4u + 7u) & ~7u;
+  L.push = L.z + static_cast<uint32_t>(batch * 16 * tpb) * 4u;             // fp32 [C][batch][R] (rank 0)
+  L.bars = (L.push + static_cast<uint32_t>(C * batch * R) * 4u + 7u) & ~7u;
   L.total = L.bars + 8u;
   return L;
 }
@@ -327,39 +330,46 @@ __device__ __forceinline__ void cs_st_async_f32(uint32_t remote_addr, float v, u
                : "memory");
 }
 
-template <int B, bool XF32>
+// TPR threads per row (4: 64-row blocks, up to 16 tiles; 1: 256-row blocks, up
+// to 8 tiles): thread (row r, part q) takes tiles q, q + TPR, ... of its row
+// (16 codes each; the TPR lanes of a row read adjacent 16-byte pieces).  The
+// bucket sums use four threads per bucket, four members each, all loads of a
+// thread in flight at once.
+template <int B, bool XF32, int TPR>
 __global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a) {
+  constexpr int R = kCsThreads / TPR, tpr = TPR;
+  constexpr int kCsChunks = TPR == 4 ? 4 : 8;  // 16-code pieces per thread
   extern __shared__ __align__(128) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
-  const int rb = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x;
   const int t0 = crank * a.tpb;
   const int nt = min(a.tpb, a.T - t0);
-  const GemvCsLayout L = gemv_cs_layout(a.tpb, B, a.C);
+  const GemvCsLayout L = gemv_cs_layout(a.tpb, B, a.C, R);
   const uint32_t s0 = smem_u32(sm);
   const uint32_t push_bar = s0 + L.bars;
   float* zs = reinterpret_cast<float*>(sm + L.z);
   float* push = reinterpret_cast<float*>(sm + L.push);
-  const int nbk = 16 * a.tpb;  // bucket slots per block (z row stride)
-  constexpr uint32_t kPartBytes = static_cast<uint32_t>(B) * 64u * 4u;
+  const int nbk = 16 * a.tpb;  // z row stride
+  const uint32_t part_bytes = static_cast<uint32_t>(B * R) * 4u;
 
-  // ---- code loads first (never written by a programmatic-dependent neighbour):
-  // thread (row r, quarter q) takes tiles q, q + 4, ... of its row
-  const int r = tid >> 2, q4 = tid & 3;
-  const int8_t* crow = a.codes + (static_cast<int64_t>(rb) * 64 + r) * (a.K / 16) + 16 * static_cast<int64_t>(t0);
-  uint4 cv[kCsMaxTiles / 4];
+  // ---- code loads first (never written by a programmatic-dependent neighbour)
+  const int r = tid / tpr, q = tid % tpr;
+  const int64_t row = static_cast<int64_t>(blockIdx.y) * R + r;
+  const bool row_ok = row < a.M;
+  const int8_t* crow = a.codes + row * (a.K / 16) + 16 * static_cast<int64_t>(t0);
+  uint4 cv[kCsChunks];
 #pragma unroll
-  for (int u = 0; u < kCsMaxTiles / 4; ++u) {
-    const int tl = q4 + 4 * u;
+  for (int u = 0; u < kCsChunks; ++u) {
+    const int tl = q + tpr * u;
     cv[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (tl < nt) cv[u] = ldg_nc128(crow + 16 * tl);
+    if (row_ok && tl < nt) cv[u] = ldg_nc128(crow + 16 * tl);
   }
   if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0 && a.C > 1) {
     mbar_init(push_bar, 1);
     mbar_fence_init();
-    if (crank == 0) mbar_arrive_expect_tx(push_bar, static_cast<uint32_t>(a.C - 1) * kPartBytes);
+    if (crank == 0) mbar_arrive_expect_tx(push_bar, static_cast<uint32_t>(a.C - 1) * part_bytes);
   }
   if (a.C > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
@@ -384,9 +394,9 @@ __global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a)
       }
 #pragma unroll
     for (int t = 0; t < B; ++t) {
-      float s = ((xv[t][0] + xv[t][1]) + xv[t][2]) + xv[t][3];
-      const float s1 = __shfl_xor_sync(0xFFFFFFFFu, s, 1);
-      const float pair = (m4 & 1) ? (s1 + s) : (s + s1);     // (q0 + q1), (q2 + q3)
+      const float sq = ((xv[t][0] + xv[t][1]) + xv[t][2]) + xv[t][3];
+      const float s1 = __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
+      const float pair = (m4 & 1) ? (s1 + sq) : (sq + s1);     // (q0 + q1), (q2 + q3)
       const float p2 = __shfl_xor_sync(0xFFFFFFFFu, pair, 2);
       const float tot = (m4 & 2) ? (p2 + pair) : (pair + p2);  // (q0 + q1) + (q2 + q3)
       if (m4 == 0) zs[t * nbk + bb] = tot;
@@ -395,13 +405,13 @@ __global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a)
   __syncthreads();
   if (a.C > 1 && crank != 0) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 
-  // ---- S z: 16 codes per tile per thread against the tile's 16 z values
+  // ---- S z: 16 codes per tile against the tile's 16 bucket sums
   float acc[B];
 #pragma unroll
   for (int t = 0; t < B; ++t) acc[t] = 0.0f;
 #pragma unroll
-  for (int u = 0; u < kCsMaxTiles / 4; ++u) {
-    const int tl = q4 + 4 * u;
+  for (int u = 0; u < kCsChunks; ++u) {
+    const int tl = q + tpr * u;
     if (tl < nt) {
       const uint32_t ws[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
       float cf[16];
@@ -428,52 +438,56 @@ __global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a)
     }
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // the four lanes of a row, in quarter order
+  // the tpr lanes of a row, in part order
+  for (int w = 1; w < tpr; w <<= 1) {
 #pragma unroll
-  for (int t = 0; t < B; ++t) {
-    const float o1 = __shfl_xor_sync(0xFFFFFFFFu, acc[t], 1);
-    const float pr = (q4 & 1) ? (o1 + acc[t]) : (acc[t] + o1);
-    const float o2 = __shfl_xor_sync(0xFFFFFFFFu, pr, 2);
-    acc[t] = (q4 & 2) ? (o2 + pr) : (pr + o2);
+    for (int t = 0; t < B; ++t) {
+      const float o = __shfl_xor_sync(0xFFFFFFFFu, acc[t], w);
+      acc[t] = (q & w) ? (o + acc[t]) : (acc[t] + o);
+    }
   }
-  const float s = __half2float(__ushort_as_half(a.scales[rb]));
-  float* yrb = a.y + static_cast<int64_t>(rb) * 64;
+  const float s = row_ok ? __half2float(__ushort_as_half(a.scales[row / kRowsPerBlock])) : 0.0f;
+  // one scale per block when the block is one row block
+  const float sblk = R == kRowsPerBlock ? __half2float(__ushort_as_half(a.scales[blockIdx.y])) : 0.0f;
   if (a.C == 1) {
-    if (q4 == 0) {
+    if (q == 0 && row_ok) {
 #pragma unroll
-      for (int t = 0; t < B; ++t) yrb[static_cast<int64_t>(t) * a.M + r] = acc[t] * s;
+      for (int t = 0; t < B; ++t) a.y[static_cast<int64_t>(t) * a.M + row] = acc[t] * s;
     }
     return;
   }
   if (crank != 0) {
-    if (a.inject && crank == 1 && rb == 0) return;  // test hook: the first block's wait gives up
-    if (q4 == 0) {
+    if (a.inject && crank == 1 && blockIdx.y == 0) return;  // test hook: the first block's wait gives up
+    if (q == 0) {
       const uint32_t bar0 = cs_mapa(push_bar, 0);
 #pragma unroll
       for (int t = 0; t < B; ++t)
-        cs_st_async_f32(cs_mapa(s0 + L.push + (static_cast<uint32_t>(crank * B + t) * 64u + r) * 4u, 0), acc[t],
+        cs_st_async_f32(cs_mapa(s0 + L.push + (static_cast<uint32_t>((crank * B + t) * R + r)) * 4u, 0), acc[t],
                         bar0);
     }
     return;
   }
-  if (q4 == 0) {
+  if (q == 0) {
 #pragma unroll
-    for (int t = 0; t < B; ++t) push[t * 64 + r] = acc[t];
+    for (int t = 0; t < B; ++t) push[t * R + r] = acc[t];
   }
   if (!mbar_wait(push_bar, 0)) report(a.status, USK_FLAG_TIMEOUT);  // bounded (about 1 s)
   __syncthreads();
-  for (int qq = tid; qq < B * 64; qq += kCsThreads) {
-    float tot = 0.0f;
-    for (int c = 0; c < a.C; ++c) tot += push[c * B * 64 + qq];
-    yrb[static_cast<int64_t>(qq / 64) * a.M + qq % 64] = tot * s;
+  for (int qq = tid; qq < B * R; qq += kCsThreads) {
+    const int64_t orow = static_cast<int64_t>(blockIdx.y) * R + qq % R;
+    if (orow < a.M) {
+      float tot = 0.0f;
+      for (int c = 0; c < a.C; ++c) tot += push[c * B * R + qq];
+      const float so = R == kRowsPerBlock ? sblk : __half2float(__ushort_as_half(a.scales[orow / kRowsPerBlock]));
+      a.y[static_cast<int64_t>(qq / R) * a.M + orow] = tot * so;
+    }
   }
-  (void)lane;
 }
 
 template <int B, bool XF32>
-static cudaError_t launch_gemv_cs_t(GemvCsArgs a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_cs_layout(a.tpb, B, a.C).total;
-  auto kern = gemv_cs_kernel<B, XF32>;
+static cudaError_t launch_gemv_cs_t(GemvCsArgs a, cudaStream_t stream) {
+  const size_t smem = gemv_cs_layout(a.tpb, B, a.C, a.R).total;
+  auto kern = a.R == 64 ? gemv_cs_kernel<B, XF32, 4> : gemv_cs_kernel<B, XF32, 1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -481,7 +495,7 @@ static cudaError_t launch_gemv_cs_t(GemvCsArgs a, int64_t RB, cudaStream_t strea
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.gridDim = dim3(a.C, static_cast<unsigned>((a.M + a.R - 1) / a.R), 1);
   cfg.blockDim = dim3(kCsThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -498,45 +512,73 @@ static cudaError_t launch_gemv_cs_t(GemvCsArgs a, int64_t RB, cudaStream_t strea
 }
 
 template <bool XF32>
-static cudaError_t launch_gemv_cs_b(const GemvCsArgs& a, int batch, int64_t RB, cudaStream_t stream) {
+static cudaError_t launch_gemv_cs_b(const GemvCsArgs& a, int batch, cudaStream_t stream) {
   switch (batch) {
-    case 1: return launch_gemv_cs_t<1, XF32>(a, RB, stream);
-    case 2: return launch_gemv_cs_t<2, XF32>(a, RB, stream);
-    case 3: return launch_gemv_cs_t<3, XF32>(a, RB, stream);
-    case 4: return launch_gemv_cs_t<4, XF32>(a, RB, stream);
-    case 5: return launch_gemv_cs_t<5, XF32>(a, RB, stream);
-    case 6: return launch_gemv_cs_t<6, XF32>(a, RB, stream);
-    case 7: return launch_gemv_cs_t<7, XF32>(a, RB, stream);
-    case 8: return launch_gemv_cs_t<8, XF32>(a, RB, stream);
-    case 9: return launch_gemv_cs_t<9, XF32>(a, RB, stream);
-    case 10: return launch_gemv_cs_t<10, XF32>(a, RB, stream);
-    case 11: return launch_gemv_cs_t<11, XF32>(a, RB, stream);
-    case 12: return launch_gemv_cs_t<12, XF32>(a, RB, stream);
-    case 13: return launch_gemv_cs_t<13, XF32>(a, RB, stream);
-    case 14: return launch_gemv_cs_t<14, XF32>(a, RB, stream);
-    default: return launch_gemv_cs_t<15, XF32>(a, RB, stream);
+    case 1: return launch_gemv_cs_t<1, XF32>(a, stream);
+    case 2: return launch_gemv_cs_t<2, XF32>(a, stream);
+    case 3: return launch_gemv_cs_t<3, XF32>(a, stream);
+    case 4: return launch_gemv_cs_t<4, XF32>(a, stream);
+    case 5: return launch_gemv_cs_t<5, XF32>(a, stream);
+    case 6: return launch_gemv_cs_t<6, XF32>(a, stream);
+    case 7: return launch_gemv_cs_t<7, XF32>(a, stream);
+    case 8: return launch_gemv_cs_t<8, XF32>(a, stream);
+    case 9: return launch_gemv_cs_t<9, XF32>(a, stream);
+    case 10: return launch_gemv_cs_t<10, XF32>(a, stream);
+    case 11: return launch_gemv_cs_t<11, XF32>(a, stream);
+    case 12: return launch_gemv_cs_t<12, XF32>(a, stream);
+    case 13: return launch_gemv_cs_t<13, XF32>(a, stream);
+    case 14: return launch_gemv_cs_t<14, XF32>(a, stream);
+    default: return launch_gemv_cs_t<15, XF32>(a, stream);
   }
 }
 
-// Tiles per block: tpb_override if given, else 4; raised until the cluster has
-// at most 16 blocks.
+// Blocks along K for rows-per-block R (64 or 256) and tiles per block tpb: tpb
+// is at most 16 (R = 64) or 8 (R = 256); it doubles, then R drops to 64, until
+// the cluster has at most 16 blocks.
+static void cs_geometry(GemvCsArgs& a, int R, int tpb) {
+  a.R = R;
+  a.tpb = tpb;
+  for (;;) {
+    const int cap = a.R == 64 ? 16 : 8;
+    if (a.tpb > cap) a.tpb = cap;
+    if ((a.T + a.tpb - 1) / a.tpb <= 16) break;
+    if (a.tpb < cap) a.tpb *= 2;
+    else if (a.R > 64) a.R = 64;
+    else break;
+  }
+  a.C = (a.T + a.tpb - 1) / a.tpb;
+}
+
+// Geometry: tpb_override (rounded down to a power of two) and rows_override (64
+// or 256) if given; else 256-row blocks of 8 tiles for tall matrices (at least
+// two row blocks of 64 per SM: the bucket sums of x are amortised over more
+// rows and the grid stays within one wave), 256-row blocks of 4 tiles from
+// batch 4 (the bucket sums grow with the batch), 64-row blocks of 4 tiles
+// otherwise (fewer registers, more blocks in flight) -- measured on B200.
 cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl,
-                           cudaStream_t stream, int tpb_override, int inject) {
+                           cudaStream_t stream, int tpb_override, int rows_override, int inject) {
   GemvCsArgs a;
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status;
   a.T = static_cast<int>(K / kTileCols);
-  a.tpb = tpb_override > 0 ? tpb_override : 4;
-  if (a.tpb > kCsMaxTiles) a.tpb = kCsMaxTiles;
-  if (a.tpb > a.T) a.tpb = a.T;
-  while ((a.T + a.tpb - 1) / a.tpb > 16 && a.tpb < kCsMaxTiles) ++a.tpb;
-  a.C = (a.T + a.tpb - 1) / a.tpb;
-  if (a.C > 16 || batch < 1 || batch > kCsMaxBatch) return cudaErrorInvalidValue;
   a.pdl = pdl ? 1 : 0;
   a.inject = inject;
-  const int64_t RB = M / kRowsPerBlock;
-  return xf32 ? launch_gemv_cs_b<true>(a, batch, RB, stream) : launch_gemv_cs_b<false>(a, batch, RB, stream);
+  if (batch < 1 || batch > kCsMaxBatch) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int tpb_given = 0;
+  if (tpb_override > 0) {
+    tpb_given = 1;
+    while (tpb_given * 2 <= tpb_override && tpb_given < kCsMaxTiles) tpb_given *= 2;
+  }
+  const bool tall = M / kRowsPerBlock >= 2 * sms;
+  const int R = (rows_override == 64 || rows_override == 256) ? rows_override : ((tall || batch >= 4) ? 256 : 64);
+  cs_geometry(a, R, tpb_given ? tpb_given : ((R == 256 && tall) ? 8 : 4));
+  // the first block's receive area: 64-row blocks when it would not fit
+  if (gemv_cs_layout(a.tpb, batch, a.C, a.R).total > 200u * 1024u) cs_geometry(a, 64, a.tpb);
+  if (a.C > 16) return cudaErrorInvalidValue;
+  return xf32 ? launch_gemv_cs_b<true>(a, batch, stream) : launch_gemv_cs_b<false>(a, batch, stream);
 }
 
 }  // namespace usk

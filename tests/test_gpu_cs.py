@@ -127,16 +127,34 @@ def test_cs_gemv_matches_oracle(M, K, xdtype, batch):
     _check_product(sk, o, gen.activations(batch, K, 32, xdtype))
 
 
-@pytest.mark.parametrize("tpb", [1, 2, 3, 5, 8, 16])
-def test_cs_gemv_geometries(tpb):
-    W = gen.weights_student_t(128, 4352, 33, 4.0, 0.02, 0.001, 20.0, "bf16")
+@pytest.mark.parametrize("tpb", [1, 2, 3, 4, 8, 16])
+@pytest.mark.parametrize("rows", [64, 256])
+def test_cs_gemv_geometries(tpb, rows):
+    """Tiles per block (rounded down to a power of two, capped at 8 for
+    256-row blocks) and rows per block; M = 320 is not a multiple of 256
+    (partial last row group)."""
+    W = gen.weights_student_t(320, 4352, 33, 4.0, 0.02, 0.001, 20.0, "bf16")
     sk, o = _oracle_sketch(W, 14)
     usk.usk_debug_set_geometry(0, tpb)
+    usk.usk_debug_set_gemv_rows(rows)
     try:
-        for batch in (1, 7):
+        for batch in (1, 7, 15):
             _check_product(sk, o, gen.activations(batch, 4352, 34, "bf16"))
     finally:
         usk.usk_debug_set_geometry(0, 0)
+        usk.usk_debug_set_gemv_rows(0)
+
+
+@pytest.mark.parametrize("M,K", [(320, 2816), (256, 11008), (8192, 4096), (64, 65536)])
+def test_cs_gemv_more_shapes(M, K):
+    """Ragged tile counts (11, 43), a tall matrix (automatic 256-row blocks) and
+    the largest K (16 tiles per block)."""
+    W = gen.weights_student_t(M, K, 37, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _oracle_sketch(W, 16)
+    rows = None if M <= 320 else np.array([0, 1, 31, 32, 255, 256, M // 2 + 3, M - 1])
+    for batch in (1, 2, 3, 9, 15):
+        _check_product(sk, o, gen.activations(batch, K, 38, "bf16"), rows=rows)
+    _check_product(sk, o, gen.activations(2, K, 39, "f32"), rows=rows)
 
 
 def test_cs_gemv_repeatable_and_pdl():
@@ -195,6 +213,9 @@ def test_cs_flags_and_argument_errors():
 
 
 def test_cs_wait_timeouts_reported_then_recover():
+    """Build: block (0, 0) skips a weight-tile copy; product: block 1 of the
+    first row group skips its partial sums.  Each bounded wait gives up and
+    sets the flag."""
     W = gen.weights_normal(64, 2048, 2, 0.02, "bf16")  # two blocks per row block in the product
     x = gen.activations(1, 2048, 3, "bf16")
     for kind in (1, 3):
