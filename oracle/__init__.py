@@ -12,7 +12,8 @@ Operators" (gist.science/es/paper/2506.17255), Resumen Tecnico, Metodologia §1
 format readings listed there: format 1 (one hash row, largest key kept) and
 format 2 (the multi-row AbsMaxMin sketch: smallest magnitude kept per bucket,
 largest magnitude over the hash rows on decode; the ``*_amm`` functions) and
-format 3 (the column-shared projection W_hat = S . P^T; the ``*_cs`` functions).
+format 3 (the column-shared projection W_hat = S . P^T; the ``*_cs`` functions)
+and format 4 (format 1 with 4-bit codes and 8 weights per bucket; ``*_q4``).
 
 Parity pins (tests/test_oracle_*.py): SplitMix64 published outputs, binary16
 conversion against numpy's, round-half-even against numpy.rint, an independent
@@ -105,6 +106,14 @@ def _load():
         lib.orc_cs_decode.restype = ctypes.c_int
         lib.orc_cs_gemv_f64.argtypes = [vp, vp, i64, i64, u64, vp, ctypes.c_int, i64, vp, i64, vp]
         lib.orc_cs_gemv_f64.restype = ctypes.c_int
+        lib.orc_q4_bucket.argtypes = [i64, u64, i64, i64]
+        lib.orc_q4_bucket.restype = i64
+        lib.orc_q4_build_rows.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, u64, i64, vp, vp, vp, vp]
+        lib.orc_q4_build_rows.restype = ctypes.c_int
+        lib.orc_q4_decode.argtypes = [vp, vp, i64, i64, u64, vp]
+        lib.orc_q4_decode.restype = ctypes.c_int
+        lib.orc_q4_gemv_f64.argtypes = [vp, vp, i64, i64, u64, vp, ctypes.c_int, i64, vp, i64, vp]
+        lib.orc_q4_gemv_f64.restype = ctypes.c_int
         lib.orc_f32_to_f16_array.argtypes = [vp, vp, i64]
         lib.orc_f32_to_f16_array.restype = None
         lib.orc_f16_to_f32_array.argtypes = [vp, vp, i64]
@@ -264,6 +273,66 @@ def cs_sigma(seed, tc, u):
 def cs_bucket(K, seed, j):
     """Global bucket of column j in a format-3 sketch."""
     return int(_load().orc_cs_bucket(K, seed, j))
+
+
+def build_sketch_q4(W, importance=None, seed=0, want_winners=False, row_block0=0):
+    """Format-4 sketch of W [M, K]: the format-1 rule with 8 weights per bucket
+    and 4-bit codes (two per byte).  Returns dict as build_sketch; winner and
+    value have M*K/8 entries (buckets)."""
+    W, dt = _weights(W)
+    M, K = W.shape
+    ok = M % 64 == 0 and K % 256 == 0 and M >= 0 and K >= 0
+    nbytes = M * K // 16 if ok else 0
+    nb = M * K // 8 if ok else 0
+    imp = None if importance is None else np.ascontiguousarray(importance, dtype=np.float32)
+    codes = np.zeros(max(nbytes, 1), dtype=np.int8)
+    scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
+    winner = np.full(max(nb, 1), -2, dtype=np.int64) if want_winners else None
+    value = np.zeros(max(nb, 1), dtype=np.float32) if want_winners else None
+    st = _load().orc_q4_build_rows(_ptr(W), dt, M, K, K, _ptr(imp), seed, row_block0, _ptr(codes),
+                                   _ptr(scales), _ptr(winner), _ptr(value))
+    out = {"status": st, "codes": codes[:nbytes], "scales": scales[: M // 64]}
+    if want_winners:
+        out["winner"] = winner[:nb]
+        out["value"] = value[:nb]
+    return out
+
+
+def decode_q4(codes, scales, M, K, seed=0):
+    """W_hat [M, K] float32 of a format-4 sketch."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    out = np.zeros((M, K), dtype=np.float32)
+    st = _load().orc_q4_decode(_ptr(codes), _ptr(scales), M, K, seed, _ptr(out))
+    if st:
+        raise ValueError("orc_q4_decode status %d" % st)
+    return out
+
+
+def gemv_q4_f64(codes, scales, M, K, x, seed=0, rows=None):
+    """y = W_hat x^T in float64 for a format-4 sketch (arguments as gemv_f64)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    xdt = F32 if x.dtype == np.float32 else BF16 if x.dtype == np.uint16 else None
+    if xdt is None:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    batch = x.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nr = M if r is None else len(r)
+    y = np.zeros((batch, nr), dtype=np.float64)
+    st = _load().orc_q4_gemv_f64(_ptr(codes), _ptr(scales), M, K, seed, _ptr(x), xdt, batch,
+                                 _ptr(r), 0 if r is None else len(r), _ptr(y))
+    if st:
+        raise ValueError("orc_q4_gemv_f64 status %d" % st)
+    return y
+
+
+def q4_bucket(K, seed, i, j):
+    """Bucket of weight (i, j) within its 64-row block (format 4): 2048 tc + b."""
+    return int(_load().orc_q4_bucket(K, seed, i, j))
 
 
 def decode(codes, scales, M, K, seed=0):

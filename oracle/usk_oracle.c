@@ -682,3 +682,153 @@ int orc_cs_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int6
   free(bucket_of);
   return ORC_OK;
 }
+
+/* ================================================================ format 4
+ *
+ * The format-1 sketch with 4-bit codes ("UltraSketchLLM" explainer, Resultados
+ * Experimentales: 0.5 bit/weight with 4-bit quantisation): a bucket holds 8
+ * weights instead of 16, so a 64 x 256 tile owns 2048 buckets and a code is a
+ * signed 4-bit integer; storage stays M*K/16 bytes.  Readings:
+ *  - hash as format 1 with 8 slots: slot = floor(8h / 2^32), class = (o + r) mod
+ *    32, bucket b = (slot*32 + class)*8 + c mod 8 in [0, 2048);
+ *  - selection as format 1 (largest fp32(|w|) * importance, ties to the
+ *    smallest row-major index, empty bucket 0);
+ *  - scale s16 = binary16(max |v| / 7); code = clamp(round_half_even(v / s), -7, 7);
+ *  - storage: bucket b of tile (rb, tc) is nibble b mod 2 (0 = low) of byte
+ *    rb*4K + 1024*tc + b/2; a nibble is two's complement. */
+
+/* Bucket of weight (i, j) within its 64-row block: 2048 tc + b, in [0, 8K). */
+int64_t orc_q4_bucket(int64_t K, uint64_t seed, int64_t i, int64_t j) {
+  int64_t rb = i / ROWS_PER_BLOCK, r = i % ROWS_PER_BLOCK;
+  int64_t tc = j / TILE_COLS, c = j % TILE_COLS;
+  int64_t o = c / OCTET, sub = c % OCTET;
+  uint32_t A, C;
+  orc_tile_hash_params(seed, (uint64_t)(rb * tiles_per_row(K) + tc), &A, &C);
+  uint32_t h = A * (uint32_t)(r * (TILE_COLS / OCTET) + o) + C;
+  int64_t slot = (int64_t)(((uint64_t)h * 8u) >> 32);
+  int64_t cls = (o + r) % CLASSES;
+  return 2048 * tc + (slot * CLASSES + cls) * OCTET + sub;
+}
+
+/* Signed value of the 4-bit code of block bucket q (row block rb). */
+static int q4_code(const int8_t* codes, int64_t K, int64_t rb, int64_t q) {
+  uint8_t byte = (uint8_t)codes[rb * 4 * K + q / 2];
+  int nib = (q % 2) ? (byte >> 4) : (byte & 15);
+  return nib >= 8 ? nib - 16 : nib;
+}
+
+int orc_q4_build_rows(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw, const float* imp,
+                      uint64_t seed, int64_t rb0, int8_t* codes, uint16_t* scales, int64_t* winner,
+                      float* value) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (rb0 < 0) return ORC_ERR_SHAPE;
+  if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
+  if (M == 0) return ORC_OK;
+  if (!codes || !scales) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) scales[rb] = 0;
+    return ORC_OK;
+  }
+  if (!W || ldw < K) return ORC_ERR_NULL;
+  if (imp) {
+    for (int64_t j = 0; j < K; ++j) {
+      uint32_t u = bits_from_f32(imp[j]);
+      if ((u >> 31) || !isfinite(imp[j])) return ORC_ERR_IMPORTANCE;
+    }
+  }
+  int64_t per_block = 8 * K;  /* buckets per 64-row block */
+  float* bestkey = (float*)malloc(sizeof(float) * (size_t)per_block);
+  int64_t* bestidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)per_block);
+  float* val = (float*)malloc(sizeof(float) * (size_t)per_block);
+  if (!bestkey || !bestidx || !val) { free(bestkey); free(bestidx); free(val); return ORC_ERR_NULL; }
+  int status = ORC_OK;
+  for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
+    for (int64_t b = 0; b < per_block; ++b) { bestkey[b] = -1.0f; bestidx[b] = -1; }
+    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
+      int64_t i = rb * ROWS_PER_BLOCK + r;
+      for (int64_t j = 0; j < K; ++j) {
+        float w = load_elem(W, dtype, i * ldw + j);
+        if (!isfinite(w)) status = ORC_ERR_NONFINITE;
+        float k = fabsf(w) * (imp ? imp[j] : 1.0f);
+        int64_t b = orc_q4_bucket(K, seed, i + rb0 * ROWS_PER_BLOCK, j);
+        if (k > bestkey[b] || bestidx[b] < 0) { bestkey[b] = k; bestidx[b] = i * K + j; }
+      }
+    }
+    float mx = 0.0f;
+    for (int64_t b = 0; b < per_block; ++b) {
+      float v = 0.0f;
+      if (bestidx[b] >= 0) v = load_elem(W, dtype, (bestidx[b] / K) * ldw + bestidx[b] % K);
+      val[b] = v;
+      if (fabsf(v) > mx) mx = fabsf(v);
+    }
+    uint16_t s16 = orc_f32_to_f16(mx / 7.0f);
+    if ((s16 & 0x7c00u) == 0x7c00u) status = status ? status : ORC_ERR_SCALE_OVERFLOW;
+    scales[rb] = s16;
+    float s = orc_f16_to_f32(s16);
+    for (int64_t q = 0; q < 4 * K; ++q) codes[rb * 4 * K + q] = 0;
+    for (int64_t b = 0; b < per_block; ++b) {
+      int code = 0;
+      if (s != 0.0f) {
+        float qv = nearbyintf(val[b] / s);
+        if (qv > 7.0f) qv = 7.0f;
+        if (qv < -7.0f) qv = -7.0f;
+        code = isnan(qv) ? 0 : (int)qv;
+      }
+      uint8_t* byte = (uint8_t*)&codes[rb * 4 * K + b / 2];
+      *byte = (uint8_t)(*byte | (((unsigned)code & 15u) << (4 * (b % 2))));
+      if (winner) winner[rb * per_block + b] = bestidx[b];
+      if (value) value[rb * per_block + b] = val[b];
+    }
+  }
+  free(bestkey); free(bestidx); free(val);
+  return status;
+}
+
+int orc_q4_decode(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                  float* What) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (M == 0 || K == 0) return ORC_OK;
+  if (!codes || !scales || !What) return ORC_ERR_NULL;
+  for (int64_t i = 0; i < M; ++i) {
+    int64_t rb = i / ROWS_PER_BLOCK;
+    float s = orc_f16_to_f32(scales[rb]);
+    for (int64_t j = 0; j < K; ++j)
+      What[i * K + j] = (float)q4_code(codes, K, rb, orc_q4_bucket(K, seed, i, j)) * s;
+  }
+  return ORC_OK;
+}
+
+int orc_q4_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                    const void* x, int xdtype, int64_t batch, const int64_t* rows, int64_t nrows, double* y) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (xdtype != 0 && xdtype != 1) return ORC_ERR_DTYPE;
+  if (batch < 0) return ORC_ERR_SHAPE;
+  int64_t nr = rows ? nrows : M;
+  if (nr == 0 || batch == 0) return ORC_OK;
+  if (!y) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t q = 0; q < batch * nr; ++q) y[q] = 0.0;
+    return ORC_OK;
+  }
+  if (!codes || !scales || !x) return ORC_ERR_NULL;
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!wrow) return ORC_ERR_NULL;
+  for (int64_t q = 0; q < nr; ++q) {
+    int64_t i = rows ? rows[q] : q;
+    if (i < 0 || i >= M) { free(wrow); return ORC_ERR_SHAPE; }
+    int64_t rb = i / ROWS_PER_BLOCK;
+    float s = orc_f16_to_f32(scales[rb]);
+    for (int64_t j = 0; j < K; ++j)
+      wrow[j] = (double)((float)q4_code(codes, K, rb, orc_q4_bucket(K, seed, i, j)) * s);
+    for (int64_t t = 0; t < batch; ++t) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j) acc += wrow[j] * (double)load_elem(x, xdtype, t * K + j);
+      y[t * nr + q] = acc;
+    }
+  }
+  free(wrow);
+  return ORC_OK;
+}

@@ -201,3 +201,53 @@ def build_cs(W: np.ndarray, seed: int = 0):
                 n = min(127, int(Fraction(float(abs(v[q]))) / s))
                 out[q] = -n if v[q] < 0 else n
     return codes, scales, winner
+
+
+# ---- format 4: the format-1 rule with 8 weights per bucket and 4-bit codes
+# (Resultados: 0.5 bit/weight with 4-bit quantisation).  8 slots per class.
+
+def bucket_of_q4(K: int, seed: int, i: int, j: int) -> int:
+    """Global bucket index rb * 8K + 2048 tc + b."""
+    rb, r = divmod(i, 64)
+    tc, c = divmod(j, 256)
+    z = splitmix64_output(seed, rb * (K // 256) + tc + 1)
+    A = (z & 0xFFFFFFFF) | 1
+    C = z >> 32
+    o = c // 8
+    h = (A * (32 * r + o) + C) & 0xFFFFFFFF
+    slot = (8 * h) >> 32
+    b = (slot * 32 + (o + r) % 32) * 8 + (c % 8)
+    return rb * 8 * K + 2048 * tc + b
+
+
+def build_q4(W: np.ndarray, importance=None, seed: int = 0):
+    """Returns (packed codes [M*K/16] int8, scales, winner per bucket)."""
+    Wf = to_f32(np.ascontiguousarray(W))
+    M, K = Wf.shape
+    imp = np.ones(K, np.float32) if importance is None else np.asarray(importance, np.float32)
+    nb = M * K // 8
+    members = [[] for _ in range(nb)]
+    for i in range(M):
+        for j in range(K):
+            members[bucket_of_q4(K, seed, i, j)].append(i * K + j)
+    flat = Wf.reshape(-1)
+    winner = np.full(nb, -1, dtype=np.int64)
+    value = np.zeros(nb, dtype=np.float32)
+    for b, mem in enumerate(members):
+        if mem:
+            keyed = sorted((-float(np.float32(abs(flat[q])) * imp[q % K]), q) for q in mem)
+            winner[b] = keyed[0][1]
+            value[b] = flat[winner[b]]
+    nib = np.zeros(nb, dtype=np.int64)
+    scales = np.zeros(M // 64, dtype=np.uint16)
+    per = 8 * K
+    for rb in range(M // 64):
+        v = value[rb * per:(rb + 1) * per]
+        s16 = np.float16(np.float32(np.max(np.abs(v))) / np.float32(7.0))
+        scales[rb] = s16.view(np.uint16)
+        s = np.float32(s16)
+        if s != 0:
+            nib[rb * per:(rb + 1) * per] = np.clip(np.rint(v / s), -7, 7).astype(np.int64)
+    u = (nib & 15).astype(np.uint8)
+    packed = (u[0::2] | (u[1::2] << 4)).astype(np.uint8).view(np.int8)
+    return packed, scales, winner
