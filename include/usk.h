@@ -70,6 +70,14 @@
  *   is computed as y = S (P^T x): bucket sums of x, then a dense code product.
  *   usk_gemm does not take format 3 (USK_ERR_PARAMS); usk_gemv covers batch 1..15.
  *
+ * FORMAT 4 (format 1 with 4-bit codes; Resultados: 0.5 bit/weight with 4-bit
+ * quantisation): 8 weights per bucket, 2048 buckets per tile, same storage size.
+ *   Hash as format 1 with 8 slots: slot = h >> 29, b = (slot*32 + class)*8 + c % 8.
+ *   Selection as format 1 (importance allowed).  Scale s16 = binary16_rn(max|v| / 7);
+ *   code = clamp(rint_half_even(v / float(s16)), -7, 7), two's complement nibble.
+ *   Storage: bucket b of tile (rb, tc) is nibble b % 2 (0 = low) of byte
+ *   codes[rb*4K + 1024*tc + b/2].
+ *
  * CONVENTIONS
  *   - All array pointers are DEVICE pointers owned by the caller; the library
  *     allocates no memory and keeps no state beyond cached kernel attributes.
@@ -101,7 +109,8 @@ extern "C" {
 #define USK_FORMAT_MAXKEY 1     /* format 1: one hash row, largest key kept   */
 #define USK_FORMAT_ABSMAXMIN 2  /* format 2: multi-row AbsMaxMin              */
 #define USK_FORMAT_COLSHARED 3  /* format 3: column-shared projection, W_hat = S . P^T */
-#define USK_FORMAT_VERSION 3    /* highest format this library builds and reads */
+#define USK_FORMAT_Q4 4         /* format 4: format 1 with 4-bit codes, 8 weights per bucket */
+#define USK_FORMAT_VERSION 4    /* highest format this library builds and reads */
 #define USK_ROWS_PER_BLOCK 64
 #define USK_TILE_COLS 256
 #define USK_WEIGHTS_PER_BUCKET 16
@@ -135,9 +144,10 @@ typedef enum {
 
 typedef enum { USK_F32 = 0, USK_BF16 = 1 } usk_dtype;
 
-/* Build parameters.  version: USK_FORMAT_MAXKEY, USK_FORMAT_ABSMAXMIN or
- * USK_FORMAT_COLSHARED; flags and reserved must be 0; depth = hash rows: 0 or 1
- * for formats 1 and 3, 1, 2 or 4 for format 2.  Anything else: USK_ERR_PARAMS. */
+/* Build parameters.  version: USK_FORMAT_MAXKEY, USK_FORMAT_ABSMAXMIN,
+ * USK_FORMAT_COLSHARED or USK_FORMAT_Q4; flags and reserved must be 0; depth =
+ * hash rows: 0 or 1 for formats 1, 3 and 4, 1, 2 or 4 for format 2.  Anything
+ * else: USK_ERR_PARAMS. */
 typedef struct {
   uint32_t version;
   uint32_t flags;
@@ -181,11 +191,11 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
  * fly: every weight is rehashed and its bucket gathered; W_hat is never stored).
  *   x  [batch, K] row-major, fp32 or bf16 per xdtype, 16-byte aligned.
  *   y  [batch, M] fp32 output (y[t*M + i] = sum_j w_hat[i][j] x[t][j]).
- * Single-row sketches (format 1, or format 2 at depth 1), bf16 x at batch <= 4:
+ * Single-row 8-bit sketches (format 1, or format 2 at depth 1), bf16 x at batch <= 4:
  * integer tensor path, exact sum of code * x (x split
  * into byte digit planes per block; elements outside 2^22 of the block's
  * largest are added by an exact correction), one rounding to fp32 at the end.
- * Other batches and multi-row sketches: bf16 tensor path (each hash row
+ * Other batches, multi-row and 4-bit sketches: bf16 tensor path (each hash row
  * gathered, the code of largest magnitude kept), exact products, fp32 accumulation; fp32 x
  * is split into two bf16 terms (|error| <= 2^-16 |x| per element).
  * batch == 0 or M == 0 is a no-op; K == 0 writes y = 0.  Deterministic for a

@@ -3,7 +3,8 @@
 Thin Python face of libusk.so (C ABI in include/usk.h): ``usk_build`` compresses
 a weight matrix into a 0.5 bit/weight hashed sketch (format 1: one hash row,
 largest key kept; format 2: the multi-row AbsMaxMin sketch; format 3: the
-column-shared projection W_hat = S . P^T, multiplied as S (P^T x)); ``usk_gemv`` (batch 1-15)
+column-shared projection W_hat = S . P^T, multiplied as S (P^T x); format 4:
+format 1 with 4-bit codes and 8 weights per bucket); ``usk_gemv`` (batch 1-15)
 and ``usk_gemm`` (batch 16-256) multiply the sketch with activations, rebuilding
 every weight on the fly.  PyTorch supplies device memory and streams only.
 """
@@ -15,6 +16,7 @@ from ._native import (  # noqa: F401
     FORMAT_ABSMAXMIN,
     FORMAT_COLSHARED,
     FORMAT_MAXKEY,
+    FORMAT_Q4,
     FORMAT_VERSION,
     GEMM_MAX_BATCH,
     GEMM_MIN_BATCH,

@@ -22,7 +22,8 @@ USK_BF16 = 1
 FORMAT_MAXKEY = 1      # format 1: one hash row, the largest key kept per bucket
 FORMAT_ABSMAXMIN = 2   # format 2: multi-row AbsMaxMin (smallest |w| kept, largest over rows decoded)
 FORMAT_COLSHARED = 3   # format 3: column-shared projection, W_hat = S . P^T, product as S (P^T x)
-FORMAT_VERSION = 3     # highest format the library builds and reads
+FORMAT_Q4 = 4          # format 4: format 1 with 4-bit codes, 8 weights per bucket
+FORMAT_VERSION = 4     # highest format the library builds and reads
 GEMV_MAX_BATCH = 15
 GEMM_MIN_BATCH = 16
 GEMM_MAX_BATCH = 256
@@ -170,7 +171,7 @@ def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int
     which device-detected USK_FLAG_* bits are OR-ed.  version=FORMAT_ABSMAXMIN
     builds the multi-row AbsMaxMin sketch with `depth` (1, 2 or 4) hash rows,
     version=FORMAT_COLSHARED the column-shared projection sketch (no importance
-    for either)."""
+    for either), version=FORMAT_Q4 the format-1 sketch with 4-bit codes."""
     _need_cuda(W, importance, codes, scales, status)
     if W.dim() != 2 or W.stride(1) != 1:
         raise ValueError("W must be a 2-D row-major tensor")

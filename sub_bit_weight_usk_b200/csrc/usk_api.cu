@@ -9,7 +9,7 @@
 namespace usk {
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override, int inject);
+                         cudaStream_t stream, int cluster_override, int inject, bool q4);
 cudaError_t launch_build_amm(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed, int depth,
                              int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
                              int cluster_override, int inject);
@@ -21,11 +21,11 @@ cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t 
                            cudaStream_t stream, int tpb_override, int rows_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth);
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, bool q4);
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth);
-bool gemm_supported(int64_t K, int batch, int depth);
+                        int depth, bool q4);
+bool gemm_supported(int64_t K, int batch, int depth, bool q4);
 }  // namespace usk
 
 namespace {
@@ -43,7 +43,7 @@ usk_status check_shape(int64_t M, int64_t K) {
 int format_depth(uint32_t version, uint32_t depth) {
   if (version == 0 || version == USK_FORMAT_MAXKEY) return depth <= 1 ? 1 : 0;
   if (version == USK_FORMAT_ABSMAXMIN) return (depth == 1 || depth == 2 || depth == 4) ? static_cast<int>(depth) : 0;
-  if (version == USK_FORMAT_COLSHARED) return depth <= 1 ? 1 : 0;
+  if (version == USK_FORMAT_COLSHARED || version == USK_FORMAT_Q4) return depth <= 1 ? 1 : 0;
   return 0;
 }
 
@@ -115,7 +115,7 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (!params) return USK_ERR_PARAMS;
   if (params->flags != 0 || params->reserved != 0) return USK_ERR_PARAMS;
   if (params->version != USK_FORMAT_MAXKEY && params->version != USK_FORMAT_ABSMAXMIN &&
-      params->version != USK_FORMAT_COLSHARED)
+      params->version != USK_FORMAT_COLSHARED && params->version != USK_FORMAT_Q4)
     return USK_ERR_PARAMS;
   const int depth = format_depth(params->version, params->depth);
   if (depth == 0) return USK_ERR_PARAMS;
@@ -140,7 +140,7 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
                               g_build_cluster, g_inject == 1);
   else
     e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes, scales, d_status, s,
-                          g_build_cluster, g_inject == 1);
+                          g_build_cluster, g_inject == 1, params->version == USK_FORMAT_Q4);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -171,7 +171,8 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
   cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
                                    xdtype == USK_F32, static_cast<int>(batch), y, d_status,
                                    (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows,
-                                   g_inject == 3, format_depth(sketch->version, sketch->depth));
+                                   g_inject == 3, format_depth(sketch->version, sketch->depth),
+                                   sketch->version == USK_FORMAT_Q4);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -190,7 +191,8 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   if (sketch->version == USK_FORMAT_COLSHARED) return USK_ERR_PARAMS;  // format 3: usk_gemv only
   if (batch < USK_GEMM_MIN_BATCH || batch > USK_GEMM_MAX_BATCH || batch % 16 != 0) return USK_ERR_BATCH;
   const int depth = format_depth(sketch->version, sketch->depth);
-  if (!usk::gemm_supported(sketch->K, static_cast<int>(batch), depth)) return USK_ERR_SHAPE;
+  const bool q4 = sketch->version == USK_FORMAT_Q4;
+  if (!usk::gemm_supported(sketch->K, static_cast<int>(batch), depth, q4)) return USK_ERR_SHAPE;
   if (sketch->M == 0) return USK_OK;
   if (!y) return USK_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -199,7 +201,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   if (!x_bf16) return USK_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(y)) return USK_ERR_ALIGN;
   cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
-                                   static_cast<int>(batch), y, d_status, s, g_inject == 2, depth);
+                                   static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, q4);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }

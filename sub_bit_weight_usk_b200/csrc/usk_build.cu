@@ -57,28 +57,34 @@ struct BuildLayout {
   uint32_t wbuf, keys, win, vals, bars, misc, total;
 };
 
-__host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int tpc, int nbuf) {
+// q4: the 4-bit-code format (8 hash slots, 2048 buckets per tile).
+__host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int tpc, int nbuf, bool q4) {
   const bool single = bf16 && !has_imp;
   const uint32_t tile = kRowsPerBlock * kTileCols * (bf16 ? 2u : 4u);
+  const uint32_t nbk = q4 ? 2048u : 1024u;  // buckets per tile
   BuildLayout L;
   L.wbuf = 0;
   L.keys = L.wbuf + nbuf * tile;
-  L.win = L.keys + (single ? 0u : 2u * 4096u);
-  L.vals = L.win + ((single || bf16) ? 2u * 4096u : 2u * 8192u);
-  L.bars = (L.vals + static_cast<uint32_t>(tpc) * 1024u * (bf16 ? 2u : 4u) + 7u) & ~7u;
+  L.win = L.keys + (single ? 0u : 2u * 4u * nbk);
+  L.vals = L.win + ((single || bf16) ? 2u * 4u * nbk : 2u * 8u * nbk);
+  L.bars = (L.vals + static_cast<uint32_t>(tpc) * nbk * (bf16 ? 2u : 4u) + 7u) & ~7u;
   L.misc = L.bars + 64u;
   L.total = L.misc + 64u;
   return L;
 }
 
-template <bool BF16, bool HAS_IMP>
+// Q4: the 4-bit-code format -- 8 hash slots (slot = h >> 29), 2048 buckets per
+// tile, scale max |v| / 7, codes clamp(rint(v / s), -7, 7) packed two per byte.
+template <bool BF16, bool HAS_IMP, bool Q4>
 __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
   constexpr bool kSingle = BF16 && !HAS_IMP;
   constexpr uint32_t kRowBytes = kTileCols * (BF16 ? 2 : 4);
   constexpr uint32_t kTileBytes = kRowsPerBlock * kRowBytes;
-  constexpr uint32_t kWinBytes = (kSingle || BF16) ? 4096u : 8192u;  // one tile's winner words
+  constexpr uint32_t kBk = Q4 ? 2048u : 1024u;   // buckets per tile
+  constexpr uint32_t kShift = Q4 ? 29u : 30u;    // slot = h >> kShift
+  constexpr uint32_t kWinBytes = (kSingle || BF16) ? 4u * kBk : 8u * kBk;  // one tile's winner words
   extern __shared__ __align__(128) uint8_t smraw_unaligned[];
-  const BuildLayout L = build_layout(BF16, HAS_IMP, a.tpc, a.nbuf);
+  const BuildLayout L = build_layout(BF16, HAS_IMP, a.tpc, a.nbuf, Q4);
   const uint32_t s0 = (smem_u32(smraw_unaligned) + 1023u) & ~1023u;  // tensor copies want 128 B; use 1 KiB
   uint8_t* smraw = smraw_unaligned + (s0 - smem_u32(smraw_unaligned));
   uint32_t* misc = reinterpret_cast<uint32_t*>(smraw + L.misc);
@@ -127,7 +133,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
     for (uint32_t q = tid; q < 2u * kWinBytes / 4u; q += kBuildThreads) win32[q] = init;
     if (!kSingle) {
       uint32_t* k32 = reinterpret_cast<uint32_t*>(smraw + L.keys);
-      for (int q = tid; q < 2048; q += kBuildThreads) k32[q] = 0u;
+      for (uint32_t q = tid; q < 2u * kBk; q += kBuildThreads) k32[q] = 0u;
     }
   }
   __syncthreads();
@@ -155,7 +161,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
 
     const uint32_t wt = s0 + L.wbuf + buf * kTileBytes;
     const uint32_t win_s = s0 + L.win + (i & 1) * kWinBytes;
-    const uint32_t keys_s = s0 + L.keys + (i & 1) * 4096u;
+    const uint32_t keys_s = s0 + L.keys + (i & 1) * (4u * kBk);
 
     if (BF16 && HAS_IMP) {
       // pass 1: key maxima; the tile's weight words stay in registers for pass 2,
@@ -167,7 +173,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
       for (int q = 0; q < 8; ++q) {
         const uint32_t r = warp + 8 * q;
         const uint32_t h = hk.x * (32u * r + lane) + hk.y;
-        const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+        const uint32_t off = ((h >> kShift) * 256u + ((lane + r) & 31u)) * 4u;
         wq[q] = lds128(wt + r * kRowBytes + lane * 16);
         const uint32_t wv[4] = {wq[q].x, wq[q].y, wq[q].z, wq[q].w};
 #pragma unroll
@@ -186,7 +192,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
       for (int q = 0; q < 8; ++q) {
         const uint32_t r = warp + 8 * q;
         const uint32_t h = hk.x * (32u * r + lane) + hk.y;
-        const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+        const uint32_t off = ((h >> kShift) * 256u + ((lane + r) & 31u)) * 4u;
         const uint32_t l0 = r * kTileCols + lane * 8;
         const uint32_t wv[4] = {wq[q].x, wq[q].y, wq[q].z, wq[q].w};
         uint32_t kmax[8];
@@ -207,7 +213,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
       for (int q = 0; q < 8; ++q) {
         const uint32_t r = warp + 8 * q;
         const uint32_t h = hk.x * (32u * r + lane) + hk.y;
-        const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+        const uint32_t off = ((h >> kShift) * 256u + ((lane + r) & 31u)) * 4u;
         const uint32_t l0 = r * kTileCols + lane * 8;
         if (BF16) {
           const uint4 v = lds128(wt + r * kRowBytes + lane * 16);
@@ -242,8 +248,13 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
         // per-weight check runs only when the screen fires (rare).
         bool screen;
         {
-          const uint4 mx = lds128(keys_s + 16u * tid);
-          screen = __syncthreads_or(max(max(mx.x, mx.y), max(mx.z, mx.w)) >= 0x7F800000u) != 0;
+          uint32_t m = 0u;
+#pragma unroll
+          for (uint32_t part = 0; part < kBk / 1024u; ++part) {  // every key word of the tile
+            const uint4 mx = lds128(keys_s + 16u * (tid + part * kBuildThreads));
+            m = max(m, max(max(mx.x, mx.y), max(mx.z, mx.w)));
+          }
+          screen = __syncthreads_or(m >= 0x7F800000u) != 0;
         }
         // pass 2: members whose key equals the bucket maximum keep the smallest
         // index and its value (predicated reductions, no divergent branches)
@@ -251,7 +262,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
         for (int q = 0; q < 8; ++q) {
           const uint32_t r = warp + 8 * q;
           const uint32_t h = hk.x * (32u * r + lane) + hk.y;
-          const uint32_t off = ((h >> 30) * 256u + ((lane + r) & 31u)) * 4u;
+          const uint32_t off = ((h >> kShift) * 256u + ((lane + r) & 31u)) * 4u;
           const uint32_t l0 = r * kTileCols + lane * 8;
           uint32_t wv[8];
           if (BF16) {
@@ -287,12 +298,12 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
     // compact this tile's winners into its value array and reset the slot
     // (reused by tile i + 2, after the barrier of tile i + 1)
     {
-      ValT* vals = vals_all + i * 1024;
+      ValT* vals = vals_all + i * kBk;
       uint32_t* win32 = reinterpret_cast<uint32_t*>(smraw + L.win + (i & 1) * kWinBytes);
       uint64_t* win64 = reinterpret_cast<uint64_t*>(smraw + L.win + (i & 1) * kWinBytes);
-      uint32_t* k32 = reinterpret_cast<uint32_t*>(smraw + L.keys + (i & 1) * 4096u);
+      uint32_t* k32 = reinterpret_cast<uint32_t*>(smraw + L.keys + (i & 1) * (4u * kBk));
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
+      for (int e = 0; e < static_cast<int>(kBk / kBuildThreads); ++e) {
         const int kidx = tid + kBuildThreads * e;  // consecutive lanes, consecutive words: no bank conflicts
         uint32_t vb, mag;
         if (kSingle) {
@@ -330,7 +341,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   if (warp == 0 && lane < a.C && lane != crank) atomicMax(cluster.map_shared_rank(&misc[0], lane), misc[0]);
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
   const float mx = __uint_as_float(misc[0]);
-  const __half s16 = __float2half_rn(mx / 127.0f);
+  const __half s16 = __float2half_rn(mx / (Q4 ? 7.0f : 127.0f));
   const float sc = __half2float(s16);
   if (crank == 0 && tid == 0) {
     a.scales[rb] = __half_as_ushort(s16);
@@ -338,19 +349,23 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   }
   for (int i = 0; i < nt; ++i) {
     const int tc = crank + a.C * i;
-    const ValT* vals = vals_all + i * 1024;
-    const uint32_t b0 = 4u * tid;  // 4 consecutive buckets: same slot and class, subs b0 % 8 .. + 3
+    const ValT* vals = vals_all + i * kBk;
+    // Q4: 8 consecutive buckets (same slot and class, subs 0..7) -> 8 nibbles;
+    // else 4 consecutive buckets (subs b0 % 8 .. + 3) -> 4 bytes
+    constexpr uint32_t kPer = Q4 ? 8u : 4u;
+    const uint32_t b0 = kPer * tid;
     const uint32_t base = (b0 >> 8) * 256u + (b0 & 7u) * 32u + ((b0 >> 3) & 31u);
     uint32_t packed = 0u;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
+    for (int e = 0; e < static_cast<int>(kPer); ++e) {
       const uint32_t vb = vals[base + 32u * e];
       const float v = BF16 ? __uint_as_float(vb << 16) : __uint_as_float(vb);
+      constexpr float kQmax = Q4 ? 7.0f : 127.0f;
       int code = 0;
-      if (sc != 0.0f) code = static_cast<int>(fminf(fmaxf(rintf(v / sc), -127.0f), 127.0f));
-      packed |= (static_cast<uint32_t>(code) & 0xFFu) << (8 * e);
+      if (sc != 0.0f) code = static_cast<int>(fminf(fmaxf(rintf(v / sc), -kQmax), kQmax));
+      packed |= Q4 ? ((static_cast<uint32_t>(code) & 0xFu) << (4 * e)) : ((static_cast<uint32_t>(code) & 0xFFu) << (8 * e));
     }
-    int8_t* dst = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(tc) + b0;
+    int8_t* dst = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(tc) + 4u * tid;
     *reinterpret_cast<uint32_t*>(dst) = packed;
   }
   report(a.status, flags);
@@ -363,13 +378,13 @@ struct BuildPlan {
   uint32_t smem;
 };
 
-static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override) {
+static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override, bool q4) {
   auto mk = [&](int C, int nbuf) {
     BuildPlan p;
     p.C = C < T ? C : T;
     p.tpc = (T + p.C - 1) / p.C;
     p.nbuf = nbuf;
-    p.smem = build_layout(bf16, has_imp, p.tpc, nbuf).total + 1024;  // + alignment slack
+    p.smem = build_layout(bf16, has_imp, p.tpc, nbuf, q4).total + 1024;  // + alignment slack
     return p;
   };
   if (cluster_override > 0) {
@@ -386,9 +401,9 @@ static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override
   return p;
 }
 
-template <bool BF16, bool HAS_IMP>
+template <bool BF16, bool HAS_IMP, bool Q4>
 static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, int cluster_override) {
-  const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override);
+  const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override, Q4);
   // tensor map over W [M, K] (row stride ldw), one 64 x 256 box per tile
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -405,7 +420,7 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, 
   a.C = p.C;
   a.tpc = p.tpc;
   a.nbuf = p.nbuf;
-  auto kern = build_kernel<BF16, HAS_IMP>;
+  auto kern = build_kernel<BF16, HAS_IMP, Q4>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(p.smem));
   if (e != cudaSuccess) return e;
   if (p.C > 8) {
@@ -429,7 +444,7 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, 
 
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override, int inject) {
+                         cudaStream_t stream, int cluster_override, int inject, bool q4) {
   BuildArgs a;
   a.inject = inject;
   a.W = W; a.ldw = ldw; a.K = K; a.imp = imp; a.seed = seed;
@@ -437,11 +452,18 @@ cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t
   a.T = static_cast<int>(K / kTileCols);
   a.C = a.tpc = a.nbuf = 0;
   const int64_t RB = M / kRowsPerBlock;
+  if (q4) {
+    if (bf16)
+      return imp ? launch_build_t<true, true, true>(a, RB, stream, cluster_override)
+                 : launch_build_t<true, false, true>(a, RB, stream, cluster_override);
+    return imp ? launch_build_t<false, true, true>(a, RB, stream, cluster_override)
+               : launch_build_t<false, false, true>(a, RB, stream, cluster_override);
+  }
   if (bf16)
-    return imp ? launch_build_t<true, true>(a, RB, stream, cluster_override)
-               : launch_build_t<true, false>(a, RB, stream, cluster_override);
-  return imp ? launch_build_t<false, true>(a, RB, stream, cluster_override)
-             : launch_build_t<false, false>(a, RB, stream, cluster_override);
+    return imp ? launch_build_t<true, true, false>(a, RB, stream, cluster_override)
+               : launch_build_t<true, false, false>(a, RB, stream, cluster_override);
+  return imp ? launch_build_t<false, true, false>(a, RB, stream, cluster_override)
+             : launch_build_t<false, false, false>(a, RB, stream, cluster_override);
 }
 
 }  // namespace usk

@@ -268,6 +268,23 @@ __device__ __forceinline__ uint32_t i8pair_to_bf16x2(uint32_t w) {
   return r;
 }
 
+// Format 4: 8 signed 4-bit codes (storage byte k holds bucket 2k in its low
+// nibble, bucket 2k + 1 in its high nibble) -> 4 bf16 pairs in bucket order,
+// exact: each nibble biased to u = n + 8 sits under a 0x43 exponent byte (the
+// bf16 value 128 + u); subtracting 136 leaves n.
+__device__ __forceinline__ void i4x8_to_bf16x8(uint32_t w, uint32_t (&o)[4]) {
+  const uint32_t lo = (w & 0x0F0F0F0Fu) ^ 0x08080808u;         // biased low nibbles, one per byte
+  const uint32_t hi = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // biased high nibbles
+  static_for<4>([&](auto Kc) {
+    constexpr uint32_t k = decltype(Kc)::value;
+    const uint32_t p = __byte_perm(lo, hi, k | (k << 4) | ((4u + k) << 8) | ((4u + k) << 12));
+    const uint32_t v = (p & 0x00FF00FFu) | 0x43004300u;
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(0x43084308u));
+    o[k] = r;
+  });
+}
+
 // Format 2 (multi-row AbsMaxMin) decode: per 16-bit half, the bf16 code of
 // larger magnitude of a and b (integer codes, |code| <= 127); ties keep a, the
 // lower hash row.  (a | 0x8000) - |b| per half never borrows across halves and

@@ -83,12 +83,13 @@ struct GemmLayout {
   uint32_t b, cbf, codes, keys, bars, misc, total;
 };
 
-__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int depth) {
+// q4: 4-bit codes (2048 buckets per tile: 4 KiB of bf16 per row block and tile)
+__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int depth, bool q4) {
   GemmLayout L;
   L.b = 0;  // [S][N x 64] bf16, SW128; after the main loop the K-split partials [N][128] fp32
   const uint32_t ring = static_cast<uint32_t>(S) * N * kBK * 2, parts = static_cast<uint32_t>(N) * kBM * 4;
-  L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [kTileRing][2][1024]
-  L.codes = L.cbf + kTileRing * 2u * 1024u * 2u;                       // int8 [2][tcta][1024]
+  L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [kTileRing][2][1024 or 2048]
+  L.codes = L.cbf + kTileRing * 2u * (q4 ? 4096u : 2048u);             // int8 [2][tcta][1024]
   L.keys = L.codes + 2u * tcta * 1024u;                                // uint2 [2][tcta][depth]
   L.bars = (L.keys + 2u * tcta * depth * 8u + 7u) & ~7u;  // full[S], empty[S], codes, done, ready[ring], free[ring]
   L.misc = L.bars + (2 * S + 2 + 2 * kTileRing) * 8;                   // tmem holder, abort
@@ -167,9 +168,13 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 // D = hash rows of the sketch (1: format 1 or format 2 at depth 1; 2, 4: the
 // multi-row AbsMaxMin sketch: the decoders gather every row and keep the code
 // of largest magnitude)
-template <int D>
+// Q4: 4-bit codes (D == 1): 8 slots, the widen warp expands 1024 bytes of
+// nibbles per row block and tile into 2048 bf16.
+template <int D, bool Q4>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
+  constexpr uint32_t kRbBf = Q4 ? 4096u : 2048u;  // widened bytes per row block and tile
+  constexpr uint32_t kShift = Q4 ? 29u : 30u;
   extern __shared__ __align__(16) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ks = static_cast<int>(cluster.block_rank());
@@ -185,7 +190,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   const int tcta = t_end - t_begin;
   const int nk = tcta * (kTileCols / kBK);  // 64-column chunks
   const int S = a.S;
-  const GemmLayout L = gemm_layout(a.N, tcta, S, D);
+  const GemmLayout L = gemm_layout(a.N, tcta, S, D, Q4);
   const uint32_t bstage = static_cast<uint32_t>(a.N) * kBK * 2;
   const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * S, codes_bar = empty_s + 8 * S;
   const uint32_t done_bar = codes_bar + 8, ready_s = done_bar + 8, free_s = ready_s + 8 * kTileRing;
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
         hk[rho] = keytab[(rbl * tcta + t) * D + rho];
         h[rho] = hk[rho].x * (32u * r + ob) + hk[rho].y;
       }
-      const uint32_t tile_codes = s0 + L.cbf + q * 4096u + rbl * 2048u;
+      const uint32_t tile_codes = s0 + L.cbf + q * (2u * kRbBf) + rbl * kRbBf;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {  // octets 4hh .. 4hh + 3 -> columns 16hh .. 16hh + 15 of the stage
         uint32_t v[16];
@@ -285,7 +290,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
 #pragma unroll
             for (int rho = 0; rho < D; ++rho) {
               const uint4 u = lds128(tile_codes + static_cast<uint32_t>(rho) * (2048u / D) +
-                                     ((h[rho] >> 30) * kNc + cls) * 16u);
+                                     ((h[rho] >> kShift) * kNc + cls) * 16u);
               w = rho == 0 ? u : absmax_sel(w, u);
             }
           }
@@ -323,11 +328,22 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t idx = static_cast<uint32_t>(lane) * 16u + static_cast<uint32_t>(i) * 512u;
-        const uint32_t dst = s0 + L.cbf + q * 4096u + (idx >> 10) * 2048u + 2u * (idx & 1023u);
-        sts128(dst, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].x), i8pair_to_bf16x2<0x4342>(w[i].x),
-                               i8pair_to_bf16x2<0x4140>(w[i].y), i8pair_to_bf16x2<0x4342>(w[i].y)));
-        sts128(dst + 16u, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].z), i8pair_to_bf16x2<0x4342>(w[i].z),
-                                     i8pair_to_bf16x2<0x4140>(w[i].w), i8pair_to_bf16x2<0x4342>(w[i].w)));
+        if constexpr (Q4) {
+          const uint32_t dst = s0 + L.cbf + q * (2u * kRbBf) + (idx >> 10) * kRbBf + 4u * (idx & 1023u);
+          const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t o4[4];
+            i4x8_to_bf16x8(ws[e], o4);
+            sts128(dst + 16u * e, make_uint4(o4[0], o4[1], o4[2], o4[3]));
+          }
+        } else {
+          const uint32_t dst = s0 + L.cbf + q * 4096u + (idx >> 10) * 2048u + 2u * (idx & 1023u);
+          sts128(dst, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].x), i8pair_to_bf16x2<0x4342>(w[i].x),
+                                 i8pair_to_bf16x2<0x4140>(w[i].y), i8pair_to_bf16x2<0x4342>(w[i].y)));
+          sts128(dst + 16u, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].z), i8pair_to_bf16x2<0x4342>(w[i].z),
+                                       i8pair_to_bf16x2<0x4140>(w[i].w), i8pair_to_bf16x2<0x4342>(w[i].w)));
+        }
       }
       mbar_arrive(ready_s + 8 * q);
     }
@@ -466,29 +482,29 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N)
 // mbarrier has one in-order waiter per role.  Otherwise consecutive uses of a
 // stage belong to different warps, and a warp running ahead can take a
 // completed phase of use n - 2 for use n (a phase wait only tells parity).
-static int gemm_stages(int N, int tpb, int depth) {
+static int gemm_stages(int N, int tpb, int depth, bool q4) {
   const uint32_t cols = gemm_tmem_cols(N);
   const uint32_t smem_cap = cols == 256u ? 233472u / 2u - 1024u : kSmemLimit;
   int S = static_cast<int>((cols - gemm_a_col(N)) / 32u);
   if (S > kMaxStages) S = kMaxStages;
   S &= ~3;
-  while (S >= 4 && gemm_layout(N, tpb, S, depth).total + 1024u > smem_cap) S -= 4;
+  while (S >= 4 && gemm_layout(N, tpb, S, depth, q4).total + 1024u > smem_cap) S -= 4;
   return S >= 4 ? S : 0;
 }
 
 // Largest number of tiles per block (codes staged up front) that still leaves
 // a four-stage pipeline for batch N.
-static int gemm_max_tiles(int N, int depth) {
+static int gemm_max_tiles(int N, int depth, bool q4) {
   int t = kMaxTiles;
-  while (t > 1 && gemm_stages(N, t, depth) == 0) --t;
+  while (t > 1 && gemm_stages(N, t, depth, q4) == 0) --t;
   return t;
 }
 
 // Dynamic shared memory of a launch: the layout, padded so that no more blocks
 // share an SM than its 512 tensor-memory columns hold (a block waiting in
 // tcgen05.alloc for a co-resident block of its own cluster would never proceed).
-static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth) {
-  const uint32_t smem = gemm_layout(N, tpb, S, depth).total + 1024u;  // + alignment slack
+static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, bool q4) {
+  const uint32_t smem = gemm_layout(N, tpb, S, depth, q4).total + 1024u;  // + alignment slack
   const uint32_t max_blocks = 512u / gemm_tmem_cols(N);
   const uint32_t floor_bytes = 233472u / (max_blocks + 1u) + 1u - 1024u;  // 228 KiB per SM, 1 KiB reserved per block
   return smem > floor_bytes ? smem : floor_bytes;
@@ -499,8 +515,8 @@ static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth) {
 // pipeline fill, epilogue and the cluster reduction: 4 to 5 us measured against
 // about 1.3 us per tile at batch 16), within the shared-memory bound on tiles
 // per block and clusters of at most 16.
-static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth) {
-  const int max_tiles = gemm_max_tiles(N, depth);
+static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, bool q4) {
+  const int max_tiles = gemm_max_tiles(N, depth, q4);
   const int64_t slots = static_cast<int64_t>(sms) * (512 / static_cast<int>(gemm_tmem_cols(N)));
   int best = -1;
   int64_t best_cost = -1;
@@ -521,14 +537,14 @@ static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth) {
 
 // Whether K fits: at most 16 blocks along K, each staging the codes of up to
 // gemm_max_tiles(batch) tiles (32 for every batch: K <= 131072).
-bool gemm_supported(int64_t K, int batch, int depth) {
-  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch, depth));
+bool gemm_supported(int64_t K, int batch, int depth, bool q4) {
+  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch, depth, q4));
 }
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth) {
-  if (depth != 1 && depth != 2 && depth != 4) return cudaErrorInvalidValue;
+                        int depth, bool q4) {
+  if ((depth != 1 && depth != 2 && depth != 4) || (q4 && depth != 1)) return cudaErrorInvalidValue;
   GemmArgs a;
   a.codes = codes; a.scales = scales; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status; a.inject = inject;
@@ -537,15 +553,15 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   const int64_t m_tiles = (M + kBM - 1) / kBM;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth);
+  a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth, q4);
   if (a.splits < 1) return cudaErrorInvalidValue;  // K beyond 16 blocks x the tiles one block can stage
   a.tmem_cols = gemm_tmem_cols(batch);
   a.a_col = gemm_a_col(batch);
   a.I = gemm_issuers(batch);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
-  a.S = gemm_stages(batch, tcta_max, depth);
+  a.S = gemm_stages(batch, tcta_max, depth, q4);
   if (a.S < 4 || a.S % 4 != 0) return cudaErrorInvalidValue;
-  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth);
+  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth, q4);
   // tensor map over x [batch, K] bf16: one 64-column x batch box per chunk, 128-byte swizzle
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -558,7 +574,8 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = depth == 4 ? gemm_kernel<4> : (depth == 2 ? gemm_kernel<2> : gemm_kernel<1>);
+  auto kern = q4 ? gemm_kernel<1, true>
+                 : (depth == 4 ? gemm_kernel<4, false> : (depth == 2 ? gemm_kernel<2, false> : gemm_kernel<1, false>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.splits > 8) {

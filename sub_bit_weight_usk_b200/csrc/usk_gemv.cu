@@ -57,12 +57,12 @@ struct GemvLayout {
   uint32_t keys, codes, xs, xrow, stage_end, parts, cta, total;
 };
 
-__host__ __device__ inline GemvLayout gemv_layout(int tpc, int nb, int batch, bool xf32, int depth) {
+__host__ __device__ inline GemvLayout gemv_layout(int tpc, int nb, int batch, bool xf32, int depth, bool q4) {
   GemvLayout L;
   const uint32_t nvalid = static_cast<uint32_t>(xf32 ? 2 * batch : batch);
   L.keys = 0;
   L.codes = (static_cast<uint32_t>(tpc * depth) * 8u + 15u) / 16u * 16u;
-  L.xs = L.codes + static_cast<uint32_t>(tpc) * 2048u;
+  L.xs = L.codes + static_cast<uint32_t>(tpc) * (q4 ? 4096u : 2048u);
   L.xrow = static_cast<uint32_t>(tpc) * 512u + 16u;
   L.stage_end = L.xs + nvalid * L.xrow;
   L.parts = 0;
@@ -82,9 +82,12 @@ __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *rein
 // D = hash rows (1: format 1 or format 2 at depth 1; 2, 4: the multi-row
 // AbsMaxMin sketch, each row gathered from its own 2048/D-byte segment of the
 // tile and reduced to the code of largest magnitude)
-template <int NB, bool XF32, int D>
+// Q4: 4-bit codes (D == 1): 8 slots, 4 KiB of widened codes per tile.
+template <int NB, bool XF32, int D, bool Q4>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
+  constexpr uint32_t kTileBf = Q4 ? 4096u : 2048u;
+  constexpr uint32_t kShift = Q4 ? 29u : 30u;
   extern __shared__ __align__(16) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -93,7 +96,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);  // >= 1 by construction of C
   const int nvalid = XF32 ? 2 * a.batch : a.batch;
-  const GemvLayout L = gemv_layout(a.tpc, NB, a.batch, XF32, D);
+  const GemvLayout L = gemv_layout(a.tpc, NB, a.batch, XF32, D, Q4);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   const uint32_t sm_s = smem_u32(sm);
 
@@ -126,15 +129,24 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
         const int q = base + u * kGemvThreads + tid;
         if (q < ncode) {
           const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-          uint32_t o[8];
+          if constexpr (Q4) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            o[2 * e] = pack_bf16x2_from_i8(static_cast<int8_t>(w[e] & 0xFF), static_cast<int8_t>((w[e] >> 8) & 0xFF));
-            o[2 * e + 1] = pack_bf16x2_from_i8(static_cast<int8_t>((w[e] >> 16) & 0xFF), static_cast<int8_t>(w[e] >> 24));
+            for (int e = 0; e < 4; ++e) {
+              uint32_t o4[4];
+              i4x8_to_bf16x8(w[e], o4);
+              sts128(sm_s + L.codes + 64u * q + 16u * e, make_uint4(o4[0], o4[1], o4[2], o4[3]));
+            }
+          } else {
+            uint32_t o[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              o[2 * e] = pack_bf16x2_from_i8(static_cast<int8_t>(w[e] & 0xFF), static_cast<int8_t>((w[e] >> 8) & 0xFF));
+              o[2 * e + 1] = pack_bf16x2_from_i8(static_cast<int8_t>((w[e] >> 16) & 0xFF), static_cast<int8_t>(w[e] >> 24));
+            }
+            const uint32_t dst = sm_s + L.codes + 32u * q;
+            sts128(dst, make_uint4(o[0], o[1], o[2], o[3]));
+            sts128(dst + 16, make_uint4(o[4], o[5], o[6], o[7]));
           }
-          const uint32_t dst = sm_s + L.codes + 32u * q;
-          sts128(dst, make_uint4(o[0], o[1], o[2], o[3]));
-          sts128(dst + 16, make_uint4(o[4], o[5], o[6], o[7]));
         } else if (q < total) {
           const int qx = q - ncode, n = qx / xchunks_row, c = qx % xchunks_row;
           if (!XF32) {
@@ -187,7 +199,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
       if (n < nvalid) v = lds128(sm_s + L.xs + n * L.xrow + (tt * 32 + o) * 16);
       bq[nb][0] = v.x; bq[nb][1] = v.y; bq[nb][2] = v.z; bq[nb][3] = v.w;
     }
-    const uint32_t tile_s = codes_s + tt * 2048u;
+    const uint32_t tile_s = codes_s + tt * kTileBf;
     uint2 hk[D];
     uint32_t h[D];
 #pragma unroll
@@ -203,8 +215,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
         const uint32_t h0 = h[rho] + mb * (hk[rho].x * 512u);
         const uint32_t h1 = h0 + hk[rho].x * 256u;
         const uint32_t seg = tile_s + static_cast<uint32_t>(rho) * (2048u / D);
-        const uint4 u0 = lds128(seg + (h0 >> 30) * (kNc * 16u) + cls16[(2 * mb) & 3]);
-        const uint4 u1 = lds128(seg + (h1 >> 30) * (kNc * 16u) + cls16[(2 * mb + 1) & 3]);
+        const uint4 u0 = lds128(seg + (h0 >> kShift) * (kNc * 16u) + cls16[(2 * mb) & 3]);
+        const uint4 u1 = lds128(seg + (h1 >> kShift) * (kNc * 16u) + cls16[(2 * mb + 1) & 3]);
         q0 = rho == 0 ? u0 : absmax_sel(q0, u0);
         q1 = rho == 0 ? u1 : absmax_sel(q1, u1);
       }
@@ -278,10 +290,10 @@ static GemvGeometry gemv_geometry(int64_t K, int tpc_override) {
   return g;
 }
 
-template <int NB, bool XF32, int D>
+template <int NB, bool XF32, int D, bool Q4>
 static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32, D).total;
-  auto kern = gemv_kernel<NB, XF32, D>;
+  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32, D, Q4).total;
+  auto kern = gemv_kernel<NB, XF32, D, Q4>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -311,21 +323,21 @@ cudaError_t launch_gemv_slab(const int8_t* codes, const uint16_t* scales, int64_
 bool gemv_bf_supported(int64_t K, int batch, int tpc_override);
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth);
+                           int tpc_override, int inject, int depth, bool q4);
 
-template <int D>
+template <int D, bool Q4>
 static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaStream_t stream) {
   const int rows = xf32 ? 2 * a.batch : a.batch;
   const int nb = (rows + 7) / 8;
   if (!xf32) {
-    if (nb == 1) return launch_gemv_t<1, false, D>(a, RB, stream);
-    return launch_gemv_t<2, false, D>(a, RB, stream);
+    if (nb == 1) return launch_gemv_t<1, false, D, Q4>(a, RB, stream);
+    return launch_gemv_t<2, false, D, Q4>(a, RB, stream);
   }
   switch (nb) {
-    case 1: return launch_gemv_t<1, true, D>(a, RB, stream);
-    case 2: return launch_gemv_t<2, true, D>(a, RB, stream);
-    case 3: return launch_gemv_t<3, true, D>(a, RB, stream);
-    default: return launch_gemv_t<4, true, D>(a, RB, stream);
+    case 1: return launch_gemv_t<1, true, D, Q4>(a, RB, stream);
+    case 2: return launch_gemv_t<2, true, D, Q4>(a, RB, stream);
+    case 3: return launch_gemv_t<3, true, D, Q4>(a, RB, stream);
+    default: return launch_gemv_t<4, true, D, Q4>(a, RB, stream);
   }
 }
 
@@ -335,7 +347,7 @@ static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaS
 // rows of the sketch: the integer paths read single-row sketches only.
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth) {
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, bool q4) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // automatic choice (measured on B200, graphs of back-to-back calls):
@@ -343,18 +355,19 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   //  * batch >= 2, or batch 1 up to 4096 x 4096: bf16 with direct x fragments;
   //  * batch 1 with longer K or taller M: the integer cluster kernel (half the
   //    shared-memory gather bytes; its x preparation is amortised over more tiles)
-  const bool slab = depth == 1 && (path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms));
+  const bool single = depth == 1 && !q4;  // the integer paths read one-row 8-bit sketches
+  const bool slab = single && (path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms));
   if (!xf32 && slab && slab_supported(K, batch))
     return launch_gemv_slab(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl,
                             stream, rows_override, inject);
   // multi-row sketches: the direct path unless the staged one is asked for
   const bool direct =
-      path == 4 || (depth > 1 && path != 1) || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
+      path == 4 || (!single && path != 1) || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
   if (!xf32 && direct && gemv_bf_supported(K, batch, tpc_override))
     return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
-                          tpc_override, inject, depth);
+                          tpc_override, inject, depth, q4);
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
-  const bool i8_ok = depth == 1 && !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
+  const bool i8_ok = single && !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
   if (i8_ok && path != 1)
     return launch_gemv_i8(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, geo.T,
                           geo.C, geo.tpc, pdl, stream, inject);
@@ -363,9 +376,10 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.M = M; a.K = K; a.seed = seed;
   a.T = geo.T; a.C = geo.C; a.tpc = geo.tpc; a.batch = batch;
   const int64_t RB = M / kRowsPerBlock;
-  if (depth == 2) return launch_staged<2>(a, xf32, RB, stream);
-  if (depth == 4) return launch_staged<4>(a, xf32, RB, stream);
-  return launch_staged<1>(a, xf32, RB, stream);
+  if (q4) return launch_staged<1, true>(a, xf32, RB, stream);
+  if (depth == 2) return launch_staged<2, false>(a, xf32, RB, stream);
+  if (depth == 4) return launch_staged<4, false>(a, xf32, RB, stream);
+  return launch_staged<1, false>(a, xf32, RB, stream);
 }
 
 }  // namespace usk

@@ -28,6 +28,8 @@
 //    tile (class = (o + row) mod 32/D keeps a quarter warp on 8 distinct bank
 //    groups), and the D words reduce to the code of largest magnitude with four
 //    integer instructions per bf16 pair before the MMA.
+//  * 4-bit codes (format 4): the 16-byte loads hold 32 nibbles, widened to bf16
+//    the same way (exact), 4 KiB per tile; 8 hash slots (slot = h >> 29).
 //  * fp32 accumulation of exact bf16 products; the 8 warps' sums are added in
 //    a fixed order, then every block but the first writes its 64 x batch
 //    partials into the first block's shared memory with st.async, which counts
@@ -61,10 +63,11 @@ struct GemvBfLayout {
   uint32_t cbf, keys, red, push, bars, total;
 };
 
-__host__ __device__ inline GemvBfLayout gemv_bf_layout(int tpc, int batch, int C, int depth) {
+// q4: 4-bit codes, 2048 buckets per tile (4 KiB of bf16)
+__host__ __device__ inline GemvBfLayout gemv_bf_layout(int tpc, int batch, int C, int depth, bool q4) {
   GemvBfLayout L;
-  L.cbf = 0;                                                       // bf16 [tpc][1024]
-  L.keys = L.cbf + static_cast<uint32_t>(tpc) * 2048u;             // uint2 [tpc][depth]
+  L.cbf = 0;                                                       // bf16 [tpc][1024 or 2048]
+  L.keys = L.cbf + static_cast<uint32_t>(tpc) * (q4 ? 4096u : 2048u);  // uint2 [tpc][depth]
   L.red = (L.keys + static_cast<uint32_t>(tpc * depth) * 8u + 15u) & ~15u;  // fp32 [8 warps][batch][64]
   L.push = L.red + 8u * batch * 64u * 4u;                          // fp32 [C][batch][64] (used in rank 0)
   L.bars = (L.push + static_cast<uint32_t>(C) * batch * 64u * 4u + 7u) & ~7u;  // push
@@ -89,9 +92,13 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
 // D = hash rows of the sketch (1: format 1, or format 2 at depth 1; 2, 4: the
 // multi-row AbsMaxMin sketch, whose rows are gathered and reduced to the code
 // of largest magnitude before the MMA)
-template <int B, int D>
+// Q4: the 4-bit-code format (D == 1): 8 slots (slot = h >> 29), 2048 buckets and
+// 4 KiB of widened codes per tile; each 16-byte load holds 32 codes.
+template <int B, int D, bool Q4>
 __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a) {
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
+  constexpr uint32_t kTileBf = Q4 ? 4096u : 2048u;  // widened bytes per tile
+  constexpr uint32_t kShift = Q4 ? 29u : 30u;
   extern __shared__ __align__(128) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -99,7 +106,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);
-  const GemvBfLayout L = gemv_bf_layout(a.tpc, B, a.C, D);
+  const GemvBfLayout L = gemv_bf_layout(a.tpc, B, a.C, D, Q4);
   const uint32_t s0 = smem_u32(sm);
   const uint32_t push_bar = s0 + L.bars;
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
@@ -147,14 +154,23 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
     const int q = tid + u * kBfThreads;
     if (q < nt * 64) {
       const uint32_t ws[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
-      uint32_t o8[8];
+      if constexpr (Q4) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        o8[2 * e] = i8pair_to_bf16x2<0x4140>(ws[e]);
-        o8[2 * e + 1] = i8pair_to_bf16x2<0x4342>(ws[e]);
+        for (int e = 0; e < 4; ++e) {
+          uint32_t o4[4];
+          i4x8_to_bf16x8(ws[e], o4);
+          sts128(s0 + L.cbf + 64u * q + 16u * e, make_uint4(o4[0], o4[1], o4[2], o4[3]));
+        }
+      } else {
+        uint32_t o8[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          o8[2 * e] = i8pair_to_bf16x2<0x4140>(ws[e]);
+          o8[2 * e + 1] = i8pair_to_bf16x2<0x4342>(ws[e]);
+        }
+        sts128(s0 + L.cbf + 32u * q, make_uint4(o8[0], o8[1], o8[2], o8[3]));
+        sts128(s0 + L.cbf + 32u * q + 16u, make_uint4(o8[4], o8[5], o8[6], o8[7]));
       }
-      sts128(s0 + L.cbf + 32u * q, make_uint4(o8[0], o8[1], o8[2], o8[3]));
-      sts128(s0 + L.cbf + 32u * q + 16u, make_uint4(o8[4], o8[5], o8[6], o8[7]));
     }
   }
   __syncthreads();
@@ -174,7 +190,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
 #pragma unroll
   for (int tt = 0; tt < kBfMaxTiles; ++tt) {
     if (tt < nt) {
-      const uint32_t tile_s = s0 + L.cbf + tt * 2048u;
+      const uint32_t tile_s = s0 + L.cbf + tt * kTileBf;
       uint2 hk[D];
       uint32_t h[D];
 #pragma unroll
@@ -192,8 +208,8 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
           const uint32_t h0 = h[rho] + static_cast<uint32_t>(mb) * 512u * hk[rho].x;
           const uint32_t h1 = h0 + 256u * hk[rho].x;
           const uint32_t seg = tile_s + static_cast<uint32_t>(rho) * (2048u / D);
-          const uint4 u0 = lds128(seg + ((h0 >> 30) * kNc + c0) * 16u);
-          const uint4 u1 = lds128(seg + ((h1 >> 30) * kNc + c1) * 16u);
+          const uint4 u0 = lds128(seg + ((h0 >> kShift) * kNc + c0) * 16u);
+          const uint4 u1 = lds128(seg + ((h1 >> kShift) * kNc + c1) * 16u);
           q0 = rho == 0 ? u0 : absmax_sel(q0, u0);
           q1 = rho == 0 ? u1 : absmax_sel(q1, u1);
         }
@@ -267,10 +283,10 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   }
 }
 
-template <int B, int D>
+template <int B, int D, bool Q4>
 static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D).total;
-  auto kern = gemv_bf_kernel<B, D>;
+  const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D, Q4).total;
+  auto kern = gemv_bf_kernel<B, D, Q4>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -294,17 +310,17 @@ static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int D>
+template <int D, bool Q4>
 static cudaError_t launch_bf_batch(const GemvBfArgs& a, int batch, int64_t RB, cudaStream_t stream) {
   switch (batch) {
-    case 1: return launch_bf_t<1, D>(a, RB, stream);
-    case 2: return launch_bf_t<2, D>(a, RB, stream);
-    case 3: return launch_bf_t<3, D>(a, RB, stream);
-    case 4: return launch_bf_t<4, D>(a, RB, stream);
-    case 5: return launch_bf_t<5, D>(a, RB, stream);
-    case 6: return launch_bf_t<6, D>(a, RB, stream);
-    case 7: return launch_bf_t<7, D>(a, RB, stream);
-    default: return launch_bf_t<8, D>(a, RB, stream);
+    case 1: return launch_bf_t<1, D, Q4>(a, RB, stream);
+    case 2: return launch_bf_t<2, D, Q4>(a, RB, stream);
+    case 3: return launch_bf_t<3, D, Q4>(a, RB, stream);
+    case 4: return launch_bf_t<4, D, Q4>(a, RB, stream);
+    case 5: return launch_bf_t<5, D, Q4>(a, RB, stream);
+    case 6: return launch_bf_t<6, D, Q4>(a, RB, stream);
+    case 7: return launch_bf_t<7, D, Q4>(a, RB, stream);
+    default: return launch_bf_t<8, D, Q4>(a, RB, stream);
   }
 }
 
@@ -319,7 +335,7 @@ bool gemv_bf_supported(int64_t K, int batch, int tpc_override) {
 
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth) {
+                           int tpc_override, int inject, int depth, bool q4) {
   GemvBfArgs a;
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status;
@@ -331,9 +347,10 @@ cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t 
   a.pdl = pdl ? 1 : 0;
   a.inject = inject;
   const int64_t RB = M / kRowsPerBlock;
-  if (depth == 2) return launch_bf_batch<2>(a, batch, RB, stream);
-  if (depth == 4) return launch_bf_batch<4>(a, batch, RB, stream);
-  return launch_bf_batch<1>(a, batch, RB, stream);
+  if (q4) return launch_bf_batch<1, true>(a, batch, RB, stream);
+  if (depth == 2) return launch_bf_batch<2, false>(a, batch, RB, stream);
+  if (depth == 4) return launch_bf_batch<4, false>(a, batch, RB, stream);
+  return launch_bf_batch<1, false>(a, batch, RB, stream);
 }
 
 }  // namespace usk

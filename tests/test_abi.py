@@ -37,7 +37,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_sizes_and_strings(lib):
-    assert usk.usk_format_version() == 3
+    assert usk.usk_format_version() == 4
     assert usk.usk_sizes(4096, 4096) == (4096 * 4096 // 16, 2 * 64)
     assert usk.usk_sizes(0, 0) == (0, 0)
     with pytest.raises(usk.UskError):
@@ -61,7 +61,7 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.usk_build(fake, 7, 64, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 3
     assert lib.usk_build(fake, 1, 64, 256, 256, None, None, fake, fake, None, None) == 6
     # unknown format, bad depth for the format, reserved bits, importance with format 2
-    for bad in (_native.UskParams(4, 0, 0, 1, 0), _native.UskParams(3, 0, 0, 2, 0), _native.UskParams(2, 0, 0, 0, 0), _native.UskParams(2, 0, 0, 3, 0),
+    for bad in (_native.UskParams(5, 0, 0, 1, 0), _native.UskParams(4, 0, 0, 2, 0), _native.UskParams(3, 0, 0, 2, 0), _native.UskParams(2, 0, 0, 0, 0), _native.UskParams(2, 0, 0, 3, 0),
                 _native.UskParams(1, 0, 0, 2, 0), _native.UskParams(2, 0, 0, 2, 1), _native.UskParams(1, 1, 0, 1, 0)):
         assert lib.usk_build(fake, 1, 64, 256, 256, None, ctypes.byref(bad), fake, fake, None, None) == 6
     amm = _native.UskParams(2, 0, 0, 2, 0)

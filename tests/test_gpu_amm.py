@@ -131,7 +131,7 @@ def test_amm_build_flags_and_argument_errors():
     Wd = to_dev(W)
     imp = torch.ones(256, dtype=torch.float32, device="cuda")
     for kwargs in ({"version": AMM, "depth": 3}, {"version": AMM, "depth": 0}, {"version": 1, "depth": 2},
-                   {"version": 3, "depth": 1}):
+                   {"version": 9, "depth": 1}):
         with pytest.raises(usk.UskError) as ei:
             usk.usk_build(Wd, None, 0, **kwargs)
         assert ei.value.status == 6
