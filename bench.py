@@ -11,7 +11,8 @@ timed region runs the same three calls K times on the multi-row AbsMaxMin sketch
 third runs K builds and K batch-1 GEMVs of the column-shared projection sketch
 (format 3, y = S (P^T x)) and a fourth the "matrix vs hash" A/B: K batch-1 GEMVs
 of a 28672x8192 layer in format 1 (per-weight rehash and gather) and in format 3
-(bucket sums of x, then dense codes), reported under "colshared".
+(bucket sums of x, then dense codes), reported under "colshared"; a fifth runs
+the three calls on the 4-bit-code sketch (format 4) of the layer ("q4").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl usk|reference]
 
@@ -433,10 +434,26 @@ def run_usk(args):
     def gemv_matrix(i):
         usk.usk_gemv(abm[i % AB_COPIES], xab, y=yab, pdl=True)
 
+    # format 4 (4-bit codes, 8 weights per bucket) on the same layer, with importance
+    q4 = usk.FORMAT_Q4
+    sk4 = usk.usk_build(W, imp, seed, version=q4)
+    sks4 = [usk.Sketch(M, K, seed, sk4.codes.clone(), sk4.scales.clone(), q4, 1) for _ in range(N_SKETCHES)]
+
+    def build4(i):
+        b = sks4[i % N_SKETCHES]
+        usk.usk_build(Ws[i % N_WCOPIES], imp, seed, codes=b.codes, scales=b.scales, status=status, version=q4)
+
+    def gemv4(i):
+        usk.usk_gemv(sks4[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1, pdl=True)
+
+    def gemm4(i):
+        usk.usk_gemm(sks4[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
+
     graphs1 = prepare((build, gemv, gemm))
     graphs2 = prepare((build2, gemv2, gemm2))
     graphs3 = prepare((build3, gemv3))
     graphs4 = prepare((gemv_hash, gemv_matrix))
+    graphs5 = prepare((build4, gemv4, gemm4))
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
@@ -444,6 +461,7 @@ def run_usk(args):
     t_build2, t_gemv2, t_gemm2, _ = timed(graphs2)
     t_build3, t_gemv3, _ = timed(graphs3)
     t_hash, t_matrix, _ = timed(graphs4)
+    t_build4, t_gemv4, t_gemm4, _ = timed(graphs5)
     sampler.stop()
     t_step = t_total / max(args.steps, 1)
 
@@ -465,8 +483,9 @@ def run_usk(args):
 
     # max over ranks
     (t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2, t_build3, t_gemv3, t_hash,
-     t_matrix) = max_over_ranks([t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2,
-                                 t_build3, t_gemv3, t_hash, t_matrix], device=dev)
+     t_matrix, t_build4, t_gemv4, t_gemm4) = max_over_ranks(
+        [t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2, t_build3, t_gemv3, t_hash,
+         t_matrix, t_build4, t_gemv4, t_gemm4], device=dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -485,6 +504,8 @@ def run_usk(args):
     rl = rooflines(peaks, t_build, t_gemv, t_gemm, tr)
     tr2 = {k[len("amm_"):]: v for k, v in tr.items() if k.startswith("amm_")}
     rl2 = rooflines(peaks, t_build2, t_gemv2, t_gemm2, tr2, depth=AMM_DEPTH, build_bytes=BUILD_BYTES - 4 * K)
+    tr4 = {k[len("q4_"):]: v for k, v in tr.items() if k.startswith("q4_")}
+    rl4 = rooflines(peaks, t_build4, t_gemv4, t_gemm4, tr4)
     clocks = sampler.summary()
     line = {
         "metric": METRIC,
@@ -547,6 +568,17 @@ def run_usk(args):
             },
             "gpu_launches": 4 * args.steps,
         },
+        "q4": {
+            "format": "4-bit-code sketch (format 4): the format-1 rule with 8 weights per bucket and a signed "
+                      "4-bit code each (0.5 bit/weight); same layer and importance",
+            "timing": "fifth timed region: K builds, K GEMVs (batch 1), K GEMMs (batch 16) as CUDA graphs",
+            "usk_gemv_gbs": round(world * GEMV_BYTES / t_gemv4 / 1e9, 3),
+            "usk_build_gweights_per_s": round(world * N_W / t_build4 / 1e9, 3),
+            "kernel_us": {"usk_build": round(t_build4 * 1e6, 3), "usk_gemv": round(t_gemv4 * 1e6, 3),
+                          "usk_gemm": round(t_gemm4 * 1e6, 3)},
+            "rooflines": rl4,
+            "gpu_launches": 3 * args.steps,
+        },
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -570,10 +602,12 @@ def run_profile_case(args):
         fmt = {"version": usk.FORMAT_ABSMAXMIN, "depth": AMM_DEPTH}
     elif "_cs" in case:
         fmt = {"version": usk.FORMAT_COLSHARED}
+    elif case.endswith("_q4"):
+        fmt = {"version": usk.FORMAT_Q4}
     if case.endswith("_ab"):  # the 28672 x 8192 A/B shape, device-drawn weights
         W = gen.device_weights_normal(AB_M, AB_K, 3, 0.02, dev)
         x1 = torch.from_numpy(gen.activations(1, AB_K, 3, "bf16").view(np.int16)).to(dev).view(torch.bfloat16)
-    imp_c = imp if not fmt and not case.endswith("_ab") else None
+    imp_c = imp if (not fmt or case.endswith("_q4")) and not case.endswith("_ab") else None
     sk = usk.usk_build(W, imp_c, cfg["seed"], **fmt)
     torch.cuda.synchronize()
     for _ in range(3 + 3):  # 3 warm-up launches, then 3 to capture
@@ -596,7 +630,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="usk", choices=["usk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["build", "gemv", "gemm", "build_amm", "gemv_amm", "gemm_amm",
-                                               "build_cs", "gemv_cs", "gemv_ab", "gemv_cs_ab"],
+                                               "build_cs", "gemv_cs", "gemv_ab", "gemv_cs_ab", "build_q4", "gemv_q4",
+                                               "gemm_q4"],
                     default=None,
                     help="run 6 launches of one kernel on the bench workload (for ncu) and exit")
     args = ap.parse_args(argv)
