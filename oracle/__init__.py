@@ -114,6 +114,12 @@ def _load():
         lib.orc_q4_decode.restype = ctypes.c_int
         lib.orc_q4_gemv_f64.argtypes = [vp, vp, i64, i64, u64, vp, ctypes.c_int, i64, vp, i64, vp]
         lib.orc_q4_gemv_f64.restype = ctypes.c_int
+        lib.orc_rate_bucket.argtypes = [i64, u64, ctypes.c_int, i64, i64]
+        lib.orc_rate_bucket.restype = i64
+        lib.orc_rate_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, u64, ctypes.c_int, vp, vp]
+        lib.orc_rate_build.restype = ctypes.c_int
+        lib.orc_rate_gemv_f64.argtypes = [vp, vp, i64, i64, u64, ctypes.c_int, vp, ctypes.c_int, i64, vp, i64, vp]
+        lib.orc_rate_gemv_f64.restype = ctypes.c_int
         lib.orc_f32_to_f16_array.argtypes = [vp, vp, i64]
         lib.orc_f32_to_f16_array.restype = None
         lib.orc_f16_to_f32_array.argtypes = [vp, vp, i64]
@@ -333,6 +339,86 @@ def gemv_q4_f64(codes, scales, M, K, x, seed=0, rows=None):
 def q4_bucket(K, seed, i, j):
     """Bucket of weight (i, j) within its 64-row block (format 4): 2048 tc + b."""
     return int(_load().orc_q4_bucket(K, seed, i, j))
+
+
+def build_sketch_rate(W, importance=None, seed=0, slots=4):
+    """Format-1 sketch with `slots` (2, 4 or 8) hash slots per class: 32, 16 or 8
+    weights per bucket, 0.25, 0.5 or 1 bit/weight.  Returns dict(status, codes,
+    scales); codes [M*K*slots/64]."""
+    W, dt = _weights(W)
+    M, K = W.shape
+    ok = M % 64 == 0 and K % 256 == 0 and M >= 0 and K >= 0 and slots in (2, 4, 8)
+    nb = M * K * slots // 64 if ok else 0
+    imp = None if importance is None else np.ascontiguousarray(importance, dtype=np.float32)
+    codes = np.zeros(max(nb, 1), dtype=np.int8)
+    scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
+    st = _load().orc_rate_build(_ptr(W), dt, M, K, K, _ptr(imp), seed, slots, _ptr(codes), _ptr(scales))
+    return {"status": st, "codes": codes[:nb], "scales": scales[: M // 64]}
+
+
+def gemv_rate_f64(codes, scales, M, K, x, seed=0, slots=4, rows=None):
+    """y = W_hat x^T in float64 for a `slots`-slot format-1 sketch."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    xdt = F32 if x.dtype == np.float32 else BF16 if x.dtype == np.uint16 else None
+    if xdt is None:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    batch = x.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nr = M if r is None else len(r)
+    y = np.zeros((batch, nr), dtype=np.float64)
+    st = _load().orc_rate_gemv_f64(_ptr(codes), _ptr(scales), M, K, seed, slots, _ptr(x), xdt, batch,
+                                   _ptr(r), 0 if r is None else len(r), _ptr(y))
+    if st:
+        raise ValueError("orc_rate_gemv_f64 status %d" % st)
+    return y
+
+
+def rate_bucket(K, seed, slots, i, j):
+    """Global code index of weight (i, j) in a `slots`-slot format-1 sketch."""
+    return int(_load().orc_rate_bucket(K, seed, slots, i, j))
+
+
+# bits per weight of each slot count (8-bit codes)
+SLOT_BITS = {2: 0.25, 4: 0.5, 8: 1.0}
+
+
+def plan_slots(weights, importance, budget_bits):
+    """Importance-aware space allocation (Metodologia §2: units of higher
+    importance get more buckets), written as a plain greedy procedure:
+
+    every unit starts at 2 slots; the upgrades 2 -> 4 and 4 -> 8 of every unit
+    are visited in decreasing order of importance gained per bit -- with the
+    distortion of a unit taken as importance x weights / slots, upgrade s -> 2s
+    gains importance x weights / (2 s) for (bits(2s) - bits(s)) x weights bits,
+    i.e. a ratio of importance (2 -> 4) or importance / 4 (4 -> 8) -- ties in
+    the order go to the lower level, then to the lower index; an upgrade is
+    taken when the unit is at its starting level and the total stays within
+    budget_bits x total weights.  Returns a list of slot counts."""
+    n = len(weights)
+    w = [int(v) for v in weights]
+    imp = [float(v) for v in importance]
+    total = sum(w)
+    cap = budget_bits * total
+    slots = [2] * n
+    used = sum(0.25 * wi for wi in w)
+    cands = []
+    for i in range(n):
+        cands.append((-imp[i], 0, i))        # 2 -> 4, ratio imp
+        cands.append((-imp[i] / 4.0, 1, i))  # 4 -> 8, ratio imp / 4
+    cands.sort()
+    for _, level, i in cands:
+        frm = 2 if level == 0 else 4
+        if slots[i] != frm:
+            continue
+        cost = (SLOT_BITS[2 * frm] - SLOT_BITS[frm]) * w[i]
+        if used + cost <= cap:
+            slots[i] = 2 * frm
+            used += cost
+    return slots
 
 
 def decode(codes, scales, M, K, seed=0):

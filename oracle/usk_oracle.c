@@ -832,3 +832,119 @@ int orc_q4_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int6
   free(wrow);
   return ORC_OK;
 }
+
+/* ================================================================ rates
+ *
+ * Importance-aware space allocation ("UltraSketchLLM" explainer, Resumen
+ * Tecnico, Metodologia §2: rows or layers of higher importance E[a^2] receive
+ * larger sketch spaces, more buckets).  Reading: the space is chosen per sketch
+ * (a layer); format 1 takes S = 2, 4 or 8 hash slots per class, i.e. 512, 1024
+ * or 2048 buckets per 64 x 256 tile (32, 16 or 8 weights per bucket; 0.25, 0.5
+ * or 1 bit/weight with 8-bit codes).  S = 4 is format 1 exactly.
+ *  - slot = floor(S h / 2^32); bucket b = (slot*32 + class)*8 + c mod 8;
+ *  - storage: codes[rb*S*K + 256*S*tc + b];
+ *  - selection, scale (max|v| / 127) and codes as format 1. */
+
+int64_t orc_rate_bucket(int64_t K, uint64_t seed, int slots, int64_t i, int64_t j) {
+  int64_t rb = i / ROWS_PER_BLOCK, r = i % ROWS_PER_BLOCK;
+  int64_t tc = j / TILE_COLS, c = j % TILE_COLS;
+  int64_t o = c / OCTET, sub = c % OCTET;
+  uint32_t A, C;
+  orc_tile_hash_params(seed, (uint64_t)(rb * tiles_per_row(K) + tc), &A, &C);
+  uint32_t h = A * (uint32_t)(r * (TILE_COLS / OCTET) + o) + C;
+  int64_t slot = (int64_t)(((uint64_t)h * (uint64_t)slots) >> 32);
+  int64_t b = (slot * CLASSES + (o + r) % CLASSES) * OCTET + sub;
+  return rb * slots * K + 256 * slots * tc + b;
+}
+
+int orc_rate_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw, const float* imp,
+                   uint64_t seed, int slots, int8_t* codes, uint16_t* scales) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
+  if (slots != 2 && slots != 4 && slots != 8) return ORC_ERR_SHAPE;
+  if (M == 0) return ORC_OK;
+  if (!codes || !scales) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) scales[rb] = 0;
+    return ORC_OK;
+  }
+  if (!W || ldw < K) return ORC_ERR_NULL;
+  if (imp) {
+    for (int64_t j = 0; j < K; ++j) {
+      uint32_t u = bits_from_f32(imp[j]);
+      if ((u >> 31) || !isfinite(imp[j])) return ORC_ERR_IMPORTANCE;
+    }
+  }
+  int64_t per_block = slots * K;
+  float* bestkey = (float*)malloc(sizeof(float) * (size_t)per_block);
+  int64_t* bestidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)per_block);
+  if (!bestkey || !bestidx) { free(bestkey); free(bestidx); return ORC_ERR_NULL; }
+  int status = ORC_OK;
+  for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
+    for (int64_t b = 0; b < per_block; ++b) { bestkey[b] = -1.0f; bestidx[b] = -1; }
+    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
+      int64_t i = rb * ROWS_PER_BLOCK + r;
+      for (int64_t j = 0; j < K; ++j) {
+        float w = load_elem(W, dtype, i * ldw + j);
+        if (!isfinite(w)) status = ORC_ERR_NONFINITE;
+        float k = fabsf(w) * (imp ? imp[j] : 1.0f);
+        int64_t b = orc_rate_bucket(K, seed, slots, i, j) - rb * per_block;
+        if (k > bestkey[b] || bestidx[b] < 0) { bestkey[b] = k; bestidx[b] = i * K + j; }
+      }
+    }
+    float mx = 0.0f;
+    for (int64_t b = 0; b < per_block; ++b) {
+      float v = bestidx[b] >= 0 ? load_elem(W, dtype, (bestidx[b] / K) * ldw + bestidx[b] % K) : 0.0f;
+      bestkey[b] = v;  /* reuse as the kept value */
+      if (fabsf(v) > mx) mx = fabsf(v);
+    }
+    uint16_t s16 = orc_f32_to_f16(mx / 127.0f);
+    if ((s16 & 0x7c00u) == 0x7c00u) status = status ? status : ORC_ERR_SCALE_OVERFLOW;
+    scales[rb] = s16;
+    float s = orc_f16_to_f32(s16);
+    for (int64_t b = 0; b < per_block; ++b) {
+      int code = 0;
+      if (s != 0.0f) {
+        float q = nearbyintf(bestkey[b] / s);
+        if (q > 127.0f) q = 127.0f;
+        if (q < -127.0f) q = -127.0f;
+        code = isnan(q) ? 0 : (int)q;
+      }
+      codes[rb * per_block + b] = (int8_t)code;
+    }
+  }
+  free(bestkey); free(bestidx);
+  return status;
+}
+
+int orc_rate_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed, int slots,
+                      const void* x, int xdtype, int64_t batch, const int64_t* rows, int64_t nrows, double* y) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (slots != 2 && slots != 4 && slots != 8) return ORC_ERR_SHAPE;
+  if (xdtype != 0 && xdtype != 1) return ORC_ERR_DTYPE;
+  int64_t nr = rows ? nrows : M;
+  if (nr == 0 || batch <= 0) return ORC_OK;
+  if (!y) return ORC_ERR_NULL;
+  if (K == 0) {
+    for (int64_t q = 0; q < batch * nr; ++q) y[q] = 0.0;
+    return ORC_OK;
+  }
+  if (!codes || !scales || !x) return ORC_ERR_NULL;
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!wrow) return ORC_ERR_NULL;
+  for (int64_t q = 0; q < nr; ++q) {
+    int64_t i = rows ? rows[q] : q;
+    if (i < 0 || i >= M) { free(wrow); return ORC_ERR_SHAPE; }
+    float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+    for (int64_t j = 0; j < K; ++j) wrow[j] = (double)((float)codes[orc_rate_bucket(K, seed, slots, i, j)] * s);
+    for (int64_t t = 0; t < batch; ++t) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j) acc += wrow[j] * (double)load_elem(x, xdtype, t * K + j);
+      y[t * nr + q] = acc;
+    }
+  }
+  free(wrow);
+  return ORC_OK;
+}
