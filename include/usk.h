@@ -70,6 +70,12 @@
  *   is computed as y = S (P^T x): bucket sums of x, then a dense code product.
  *   usk_gemm does not take format 3 (USK_ERR_PARAMS); usk_gemv covers batch 1..15.
  *
+ * RATES (Metodologia §2, importance-aware space): format 1 takes slots = 2, 4
+ *   (default) or 8 hash slots per class -- slot = floor(slots * h / 2^32),
+ *   256 * slots buckets per tile (32, 16 or 8 weights per bucket; 0.25, 0.5 or
+ *   1 bit/weight), codes[(rb * K/256 + tc) * 256 * slots + b]; everything else
+ *   as format 1.  usk_plan_slots chooses slot counts per layer from importance.
+ *
  * FORMAT 4 (format 1 with 4-bit codes; Resultados: 0.5 bit/weight with 4-bit
  * quantisation): 8 weights per bucket, 2048 buckets per tile, same storage size.
  *   Hash as format 1 with 8 slots: slot = h >> 29, b = (slot*32 + class)*8 + c % 8.
@@ -145,15 +151,16 @@ typedef enum {
 typedef enum { USK_F32 = 0, USK_BF16 = 1 } usk_dtype;
 
 /* Build parameters.  version: USK_FORMAT_MAXKEY, USK_FORMAT_ABSMAXMIN,
- * USK_FORMAT_COLSHARED or USK_FORMAT_Q4; flags and reserved must be 0; depth =
- * hash rows: 0 or 1 for formats 1, 3 and 4, 1, 2 or 4 for format 2.  Anything
- * else: USK_ERR_PARAMS. */
+ * USK_FORMAT_COLSHARED or USK_FORMAT_Q4; flags must be 0; depth = hash rows: 0
+ * or 1 for formats 1, 3 and 4, 1, 2 or 4 for format 2; slots: 0, 2, 4 or 8 for
+ * format 1, 0 or 8 for format 4, 0 or 4 otherwise.  Anything else:
+ * USK_ERR_PARAMS. */
 typedef struct {
   uint32_t version;
   uint32_t flags;
   uint64_t seed;
   uint32_t depth;
-  uint32_t reserved;
+  uint32_t slots;  /* hash slots per class; 0 = the format's default (see RATES) */
 } usk_params;
 
 /* A built sketch (device pointers, caller-owned).  version / depth as built
@@ -165,11 +172,35 @@ typedef struct {
   const uint16_t* scales;  /* [M/64] binary16 bits      */
   uint32_t version;
   uint32_t depth;
+  uint32_t slots;          /* as built (0 = the format's default) */
+  uint32_t pad;
 } usk_sketch;
 
 /* Storage of a sketch: code_bytes = M*K/16, scale_bytes = 2*M/64.
  * Errors: USK_ERR_SHAPE, USK_ERR_NULL (an output pointer). */
 USK_API usk_status usk_sizes(int64_t M, int64_t K, size_t* code_bytes, size_t* scale_bytes);
+
+/* Storage of a sketch of a given format and slot count: code_bytes =
+ * M*K*slots/64 for format 1 (M*K/16 for the other formats and the defaults),
+ * scale_bytes = 2*M/64.  Errors: USK_ERR_SHAPE, USK_ERR_NULL, USK_ERR_PARAMS. */
+USK_API usk_status usk_sizes_ex(int64_t M, int64_t K, uint32_t version, uint32_t slots, size_t* code_bytes,
+                                size_t* scale_bytes);
+
+/* Importance-aware space allocation (Metodologia §2 "Asignacion de Espacio
+ * Consciente de la Importancia": units of higher importance E[a^2] receive
+ * larger sketch spaces).  For n units (e.g. the linear layers of a model) with
+ * weights[i] > 0 weights and importance[i] >= 0 (finite), writes slots[i] in
+ * {2, 4, 8} (format-1 rates of 0.25, 0.5 and 1 bit/weight) such that
+ * sum(weights[i] * slots[i] / 8) <= budget_bits * sum(weights).  Procedure:
+ * every unit starts at 2 slots; the steps 2 -> 4 and 4 -> 8 of all units are
+ * visited in decreasing importance gained per bit -- with a unit's distortion
+ * taken as importance x weights / slots this is importance for 2 -> 4 and
+ * importance / 4 for 4 -> 8 -- ties to the 2 -> 4 step, then to the lower index;
+ * a step is taken when the unit is at its starting level and the budget holds.
+ * budget_bits in [0.25, 1].  Host only (no GPU).  Errors: USK_ERR_NULL,
+ * USK_ERR_SHAPE (n < 0), USK_ERR_PARAMS (budget, weights or importance). */
+USK_API usk_status usk_plan_slots(int64_t n, const int64_t* weights, const double* importance, double budget_bits,
+                                  uint32_t* slots);
 
 /* Build the sketch of W (Metodologia §1 and §4: fused select-and-update).
  *   W          [M, K] row-major, row stride ldw elements (ldw >= K); fp32 or

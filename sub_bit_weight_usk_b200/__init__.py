@@ -33,6 +33,8 @@ from ._native import (  # noqa: F401
     usk_format_version,
     usk_gemm,
     usk_gemv,
+    usk_plan_slots,
     usk_sizes,
+    usk_sizes_ex,
     usk_status_str,
 )

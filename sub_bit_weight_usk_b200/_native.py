@@ -48,18 +48,19 @@ class UskError(RuntimeError):
 
 class UskParams(ctypes.Structure):
     _fields_ = [("version", ctypes.c_uint32), ("flags", ctypes.c_uint32), ("seed", ctypes.c_uint64),
-                ("depth", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+                ("depth", ctypes.c_uint32), ("slots", ctypes.c_uint32)]
 
 
 class UskSketchC(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int64), ("seed", ctypes.c_uint64),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
-                ("version", ctypes.c_uint32), ("depth", ctypes.c_uint32)]
+                ("version", ctypes.c_uint32), ("depth", ctypes.c_uint32), ("slots", ctypes.c_uint32),
+                ("pad", ctypes.c_uint32)]
 
 
 _lib = None
 
-EXPORTED = ["usk_sizes", "usk_build", "usk_gemv", "usk_gemv_ex", "usk_gemm", "usk_status_str",
+EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_build", "usk_gemv", "usk_gemv_ex", "usk_gemm", "usk_status_str",
             "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_set_gemv_rows",
             "usk_debug_inject_timeout"]
 GEMV_PDL = 1
@@ -77,6 +78,12 @@ def load_library(path: str = LIB_PATH):
     vp, i64, u32p = ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_uint32)
     lib.usk_sizes.argtypes = [i64, i64, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
     lib.usk_sizes.restype = ctypes.c_int
+    lib.usk_sizes_ex.argtypes = [i64, i64, ctypes.c_uint32, ctypes.c_uint32, ctypes.POINTER(ctypes.c_size_t),
+                                 ctypes.POINTER(ctypes.c_size_t)]
+    lib.usk_sizes_ex.restype = ctypes.c_int
+    lib.usk_plan_slots.argtypes = [i64, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double),
+                                   ctypes.c_double, ctypes.POINTER(ctypes.c_uint32)]
+    lib.usk_plan_slots.restype = ctypes.c_int
     lib.usk_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, ctypes.POINTER(UskParams), vp, vp, vp, vp]
     lib.usk_build.restype = ctypes.c_int
     lib.usk_gemv.argtypes = [ctypes.POINTER(UskSketchC), vp, ctypes.c_int, i64, vp, vp, vp]
@@ -138,6 +145,24 @@ def usk_format_version() -> int:
     return int(load_library().usk_format_version())
 
 
+def usk_plan_slots(weights, importance, budget_bits: float):
+    """Hash slots per unit (2, 4 or 8) from importance under a bits-per-weight
+    budget (host computation in the library; see include/usk.h)."""
+    n = len(weights)
+    w = (ctypes.c_int64 * max(n, 1))(*[int(v) for v in weights])
+    imp = (ctypes.c_double * max(n, 1))(*[float(v) for v in importance])
+    out = (ctypes.c_uint32 * max(n, 1))()
+    _check(load_library().usk_plan_slots(n, w, imp, ctypes.c_double(budget_bits), out), "usk_plan_slots")
+    return [int(out[i]) for i in range(n)]
+
+
+def usk_sizes_ex(M: int, K: int, version: int = FORMAT_MAXKEY, slots: int = 0):
+    c = ctypes.c_size_t()
+    s = ctypes.c_size_t()
+    _check(load_library().usk_sizes_ex(M, K, version, slots, ctypes.byref(c), ctypes.byref(s)), "usk_sizes_ex")
+    return c.value, s.value
+
+
 def usk_sizes(M: int, K: int):
     c = ctypes.c_size_t()
     s = ctypes.c_size_t()
@@ -156,39 +181,42 @@ class Sketch:
     scales: torch.Tensor  # int16 storage of binary16 bit patterns
     version: int = FORMAT_MAXKEY
     depth: int = 1
+    slots: int = 0  # hash slots per class as built (0 = the format's default)
 
     def as_c(self) -> UskSketchC:
         return UskSketchC(self.M, self.K, self.seed & (2**64 - 1), self.codes.data_ptr() if self.codes.numel() else None,
-                          self.scales.data_ptr() if self.scales.numel() else None, self.version, self.depth)
+                          self.scales.data_ptr() if self.scales.numel() else None, self.version, self.depth,
+                          self.slots, 0)
 
 
 def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int = 0,
               codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
               status: torch.Tensor | None = None, stream=None, version: int = FORMAT_MAXKEY,
-              depth: int = 1) -> Sketch:
+              depth: int = 1, slots: int = 0) -> Sketch:
     """Sketch of W [M, K] (bf16 or fp32, CUDA).  Outputs are allocated with torch
     when not given.  `status` is an optional int32 CUDA tensor of 1 element into
     which device-detected USK_FLAG_* bits are OR-ed.  version=FORMAT_ABSMAXMIN
     builds the multi-row AbsMaxMin sketch with `depth` (1, 2 or 4) hash rows,
     version=FORMAT_COLSHARED the column-shared projection sketch (no importance
-    for either), version=FORMAT_Q4 the format-1 sketch with 4-bit codes."""
+    for either), version=FORMAT_Q4 the format-1 sketch with 4-bit codes.  slots
+    (format 1): 2, 4 or 8 hash slots per class, 0.25, 0.5 or 1 bit/weight."""
     _need_cuda(W, importance, codes, scales, status)
     if W.dim() != 2 or W.stride(1) != 1:
         raise ValueError("W must be a 2-D row-major tensor")
     M, K = W.shape
-    nb = M * K // 16
+    nb = M * K * (slots if (version == FORMAT_MAXKEY and slots in (2, 8)) else 4) // 64
     if codes is None:
         codes = torch.empty(max(nb, 1), dtype=torch.int8, device=W.device)[:nb]
     if scales is None:
         scales = torch.empty(max(M // 64, 1), dtype=torch.int16, device=W.device)[: M // 64]
     if importance is not None and (importance.dtype != torch.float32 or not importance.is_contiguous()):
         raise TypeError("importance must be a contiguous float32 tensor")
-    p = UskParams(version, 0, seed & (2**64 - 1), depth, 0)
+    p = UskParams(version, 0, seed & (2**64 - 1), depth, slots)
     st = load_library().usk_build(_ptr(W), _dtype_code(W), M, K, W.stride(0), _ptr(importance), ctypes.byref(p),
                                   _ptr(codes) if nb else None, _ptr(scales) if M // 64 else None,
                                   _ptr(status), _stream(stream))
     _check(st, "usk_build")
-    return Sketch(M, K, seed, codes, scales, version, depth)
+    return Sketch(M, K, seed, codes, scales, version, depth, slots)
 
 
 def usk_gemv(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,

@@ -1,7 +1,10 @@
 // usk_api.cu -- the C ABI of libusk (declared in include/usk.h): argument
 // validation, then one kernel launch per call.  No allocation, no global state
 // beyond CUDA's cached kernel attributes.
+#include <algorithm>
 #include <cstdint>
+#include <vector>
+
 #include <cuda_runtime.h>
 
 #include "usk.h"
@@ -9,7 +12,7 @@
 namespace usk {
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override, int inject, bool q4);
+                         cudaStream_t stream, int cluster_override, int inject, int var);
 cudaError_t launch_build_amm(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed, int depth,
                              int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
                              int cluster_override, int inject);
@@ -21,11 +24,11 @@ cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t 
                            cudaStream_t stream, int tpb_override, int rows_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, bool q4);
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var);
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth, bool q4);
-bool gemm_supported(int64_t K, int batch, int depth, bool q4);
+                        int depth, int var);
+bool gemm_supported(int64_t K, int batch, int depth, int var);
 }  // namespace usk
 
 namespace {
@@ -47,9 +50,30 @@ int format_depth(uint32_t version, uint32_t depth) {
   return 0;
 }
 
+// Code layout of a (format, slots) pair: 0 = 4 slots 8-bit (format 1 default,
+// and formats 2 and 3), 1 = 8 slots 4-bit (format 4), 2 = 2 slots 8-bit,
+// 3 = 8 slots 8-bit (format 1 at 0.25 / 1 bit per weight); -1 if not valid.
+int layout_of(uint32_t version, uint32_t slots) {
+  if (version == 0 || version == USK_FORMAT_MAXKEY) {
+    if (slots == 0 || slots == 4) return 0;
+    if (slots == 2) return 2;
+    if (slots == 8) return 3;
+    return -1;
+  }
+  if (version == USK_FORMAT_Q4) return (slots == 0 || slots == 8) ? 1 : -1;
+  return (slots == 0 || slots == 4) ? 0 : -1;
+}
+
+// Code bytes of an M x K sketch in a layout.
+size_t layout_code_bytes(int64_t M, int64_t K, int layout) {
+  const size_t n = static_cast<size_t>(M) * static_cast<size_t>(K);
+  return layout == 2 ? n / 32 : (layout == 3 ? n / 8 : n / 16);
+}
+
 usk_status check_sketch(const usk_sketch* s) {
   if (!s) return USK_ERR_NULL;
   if (format_depth(s->version, s->depth) == 0) return USK_ERR_PARAMS;
+  if (layout_of(s->version, s->slots) < 0) return USK_ERR_PARAMS;
   usk_status st = check_shape(s->M, s->K);
   if (st != USK_OK) return st;
   if (s->M > 0 && s->K > 0) {
@@ -106,6 +130,68 @@ USK_API usk_status usk_sizes(int64_t M, int64_t K, size_t* code_bytes, size_t* s
   return USK_OK;
 }
 
+USK_API usk_status usk_sizes_ex(int64_t M, int64_t K, uint32_t version, uint32_t slots, size_t* code_bytes,
+                                size_t* scale_bytes) {
+  usk_status st = check_shape(M, K);
+  if (st != USK_OK) return st;
+  if (!code_bytes || !scale_bytes) return USK_ERR_NULL;
+  const int layout = layout_of(version, slots);
+  if (layout < 0 || (version > USK_FORMAT_VERSION)) return USK_ERR_PARAMS;
+  *code_bytes = layout_code_bytes(M, K, layout);
+  *scale_bytes = 2 * static_cast<size_t>(M / USK_ROWS_PER_BLOCK);
+  return USK_OK;
+}
+
+// Importance-aware space allocation: every unit starts at 2 slots; the upgrades
+// 2 -> 4 (gain per bit = importance) and 4 -> 8 (importance / 4) of all units are
+// visited in decreasing gain order (ties: the 2 -> 4 step first, then the lower
+// index) and taken while the unit is at the step's starting level and the total
+// stays within the budget.
+USK_API usk_status usk_plan_slots(int64_t n, const int64_t* weights, const double* importance, double budget_bits,
+                                  uint32_t* slots) {
+  if (n < 0) return USK_ERR_SHAPE;
+  if (n == 0) return USK_OK;
+  if (!weights || !importance || !slots) return USK_ERR_NULL;
+  if (!(budget_bits >= 0.25 && budget_bits <= 1.0)) return USK_ERR_PARAMS;
+  double total = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    if (weights[i] <= 0 || !(importance[i] >= 0.0) || importance[i] > 1e300) return USK_ERR_PARAMS;
+    total += static_cast<double>(weights[i]);
+  }
+  struct Step {
+    double gain;
+    int level;
+    int64_t unit;
+  };
+  std::vector<Step> steps;
+  steps.reserve(static_cast<size_t>(2 * n));
+  for (int64_t i = 0; i < n; ++i) {
+    steps.push_back({importance[i], 0, i});
+    steps.push_back({importance[i] / 4.0, 1, i});
+  }
+  std::stable_sort(steps.begin(), steps.end(), [](const Step& x, const Step& y) {
+    if (x.gain != y.gain) return x.gain > y.gain;
+    if (x.level != y.level) return x.level < y.level;
+    return x.unit < y.unit;
+  });
+  const double cap = budget_bits * total;
+  double used = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    slots[i] = 2u;
+    used += 0.25 * static_cast<double>(weights[i]);
+  }
+  for (const Step& st : steps) {
+    const uint32_t from = st.level == 0 ? 2u : 4u;
+    if (slots[st.unit] != from) continue;
+    const double cost = (st.level == 0 ? 0.25 : 0.5) * static_cast<double>(weights[st.unit]);
+    if (used + cost <= cap) {
+      slots[st.unit] = 2u * from;
+      used += cost;
+    }
+  }
+  return USK_OK;
+}
+
 USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t K, int64_t ldw,
                      const float* importance, const usk_params* params, int8_t* codes,
                      uint16_t* scales, uint32_t* d_status, void* stream) {
@@ -113,12 +199,14 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (st != USK_OK) return st;
   if (wdtype != USK_F32 && wdtype != USK_BF16) return USK_ERR_DTYPE;
   if (!params) return USK_ERR_PARAMS;
-  if (params->flags != 0 || params->reserved != 0) return USK_ERR_PARAMS;
+  if (params->flags != 0) return USK_ERR_PARAMS;
   if (params->version != USK_FORMAT_MAXKEY && params->version != USK_FORMAT_ABSMAXMIN &&
       params->version != USK_FORMAT_COLSHARED && params->version != USK_FORMAT_Q4)
     return USK_ERR_PARAMS;
   const int depth = format_depth(params->version, params->depth);
   if (depth == 0) return USK_ERR_PARAMS;
+  const int layout = layout_of(params->version, params->slots);
+  if (layout < 0) return USK_ERR_PARAMS;
   const bool amm = params->version == USK_FORMAT_ABSMAXMIN, cs = params->version == USK_FORMAT_COLSHARED;
   if ((amm || cs) && importance) return USK_ERR_PARAMS;
   if (M == 0) return USK_OK;
@@ -140,7 +228,7 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
                               g_build_cluster, g_inject == 1);
   else
     e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes, scales, d_status, s,
-                          g_build_cluster, g_inject == 1, params->version == USK_FORMAT_Q4);
+                          g_build_cluster, g_inject == 1, layout);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -172,7 +260,7 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
                                    xdtype == USK_F32, static_cast<int>(batch), y, d_status,
                                    (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows,
                                    g_inject == 3, format_depth(sketch->version, sketch->depth),
-                                   sketch->version == USK_FORMAT_Q4);
+                                   layout_of(sketch->version, sketch->slots));
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -191,8 +279,8 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   if (sketch->version == USK_FORMAT_COLSHARED) return USK_ERR_PARAMS;  // format 3: usk_gemv only
   if (batch < USK_GEMM_MIN_BATCH || batch > USK_GEMM_MAX_BATCH || batch % 16 != 0) return USK_ERR_BATCH;
   const int depth = format_depth(sketch->version, sketch->depth);
-  const bool q4 = sketch->version == USK_FORMAT_Q4;
-  if (!usk::gemm_supported(sketch->K, static_cast<int>(batch), depth, q4)) return USK_ERR_SHAPE;
+  const int layout = layout_of(sketch->version, sketch->slots);
+  if (!usk::gemm_supported(sketch->K, static_cast<int>(batch), depth, layout)) return USK_ERR_SHAPE;
   if (sketch->M == 0) return USK_OK;
   if (!y) return USK_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -201,7 +289,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   if (!x_bf16) return USK_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(y)) return USK_ERR_ALIGN;
   cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
-                                   static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, q4);
+                                   static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, layout);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }

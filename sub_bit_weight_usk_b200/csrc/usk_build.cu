@@ -57,11 +57,10 @@ struct BuildLayout {
   uint32_t wbuf, keys, win, vals, bars, misc, total;
 };
 
-// q4: the 4-bit-code format (8 hash slots, 2048 buckets per tile).
-__host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int tpc, int nbuf, bool q4) {
+// nbk: buckets per tile (256 x hash slots per class)
+__host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int tpc, int nbuf, uint32_t nbk) {
   const bool single = bf16 && !has_imp;
   const uint32_t tile = kRowsPerBlock * kTileCols * (bf16 ? 2u : 4u);
-  const uint32_t nbk = q4 ? 2048u : 1024u;  // buckets per tile
   BuildLayout L;
   L.wbuf = 0;
   L.keys = L.wbuf + nbuf * tile;
@@ -73,18 +72,21 @@ __host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int
   return L;
 }
 
-// Q4: the 4-bit-code format -- 8 hash slots (slot = h >> 29), 2048 buckets per
-// tile, scale max |v| / 7, codes clamp(rint(v / s), -7, 7) packed two per byte.
-template <bool BF16, bool HAS_IMP, bool Q4>
+// VAR: code layout (CodeFmt): 2, 4 or 8 hash slots per class (slot = h >> kShift,
+// 256 x slots buckets per tile) and 8-bit codes, or 8 slots with 4-bit codes
+// (scale max |v| / 7, codes clamp(rint(v / s), -7, 7) packed two per byte).
+template <bool BF16, bool HAS_IMP, int VAR>
 __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
+  using F = CodeFmt<VAR>;
+  constexpr bool Q4 = F::kNibble;
   constexpr bool kSingle = BF16 && !HAS_IMP;
   constexpr uint32_t kRowBytes = kTileCols * (BF16 ? 2 : 4);
   constexpr uint32_t kTileBytes = kRowsPerBlock * kRowBytes;
-  constexpr uint32_t kBk = Q4 ? 2048u : 1024u;   // buckets per tile
-  constexpr uint32_t kShift = Q4 ? 29u : 30u;    // slot = h >> kShift
+  constexpr uint32_t kBk = F::kBuckets;          // buckets per tile
+  constexpr uint32_t kShift = F::kShift;         // slot = h >> kShift
   constexpr uint32_t kWinBytes = (kSingle || BF16) ? 4u * kBk : 8u * kBk;  // one tile's winner words
   extern __shared__ __align__(128) uint8_t smraw_unaligned[];
-  const BuildLayout L = build_layout(BF16, HAS_IMP, a.tpc, a.nbuf, Q4);
+  const BuildLayout L = build_layout(BF16, HAS_IMP, a.tpc, a.nbuf, kBk);
   const uint32_t s0 = (smem_u32(smraw_unaligned) + 1023u) & ~1023u;  // tensor copies want 128 B; use 1 KiB
   uint8_t* smraw = smraw_unaligned + (s0 - smem_u32(smraw_unaligned));
   uint32_t* misc = reinterpret_cast<uint32_t*>(smraw + L.misc);
@@ -250,7 +252,8 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
         {
           uint32_t m = 0u;
 #pragma unroll
-          for (uint32_t part = 0; part < kBk / 1024u; ++part) {  // every key word of the tile
+          for (uint32_t part = 0; part < (kBk + 1023u) / 1024u; ++part) {  // every key word of the tile
+            if (tid + part * kBuildThreads >= kBk / 4u) break;
             const uint4 mx = lds128(keys_s + 16u * (tid + part * kBuildThreads));
             m = max(m, max(max(mx.x, mx.y), max(mx.z, mx.w)));
           }
@@ -303,7 +306,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
       uint64_t* win64 = reinterpret_cast<uint64_t*>(smraw + L.win + (i & 1) * kWinBytes);
       uint32_t* k32 = reinterpret_cast<uint32_t*>(smraw + L.keys + (i & 1) * (4u * kBk));
 #pragma unroll
-      for (int e = 0; e < static_cast<int>(kBk / kBuildThreads); ++e) {
+      for (int e = 0; e < static_cast<int>(kBk / kBuildThreads); ++e) {  // 2, 4 or 8 words per thread
         const int kidx = tid + kBuildThreads * e;  // consecutive lanes, consecutive words: no bank conflicts
         uint32_t vb, mag;
         if (kSingle) {
@@ -350,12 +353,12 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   for (int i = 0; i < nt; ++i) {
     const int tc = crank + a.C * i;
     const ValT* vals = vals_all + i * kBk;
-    // Q4: 8 consecutive buckets (same slot and class, subs 0..7) -> 8 nibbles;
-    // else 4 consecutive buckets (subs b0 % 8 .. + 3) -> 4 bytes
-    constexpr uint32_t kPer = Q4 ? 8u : 4u;
+    // kPer = slots consecutive buckets per thread (same slot and class, subs
+    // b0 % 8 .. + kPer - 1): 8-bit codes -> kPer bytes; 4-bit codes -> 8 nibbles
+    constexpr uint32_t kPer = F::kSlots;
     const uint32_t b0 = kPer * tid;
     const uint32_t base = (b0 >> 8) * 256u + (b0 & 7u) * 32u + ((b0 >> 3) & 31u);
-    uint32_t packed = 0u;
+    uint64_t packed = 0u;
 #pragma unroll
     for (int e = 0; e < static_cast<int>(kPer); ++e) {
       const uint32_t vb = vals[base + 32u * e];
@@ -363,10 +366,13 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
       constexpr float kQmax = Q4 ? 7.0f : 127.0f;
       int code = 0;
       if (sc != 0.0f) code = static_cast<int>(fminf(fmaxf(rintf(v / sc), -kQmax), kQmax));
-      packed |= Q4 ? ((static_cast<uint32_t>(code) & 0xFu) << (4 * e)) : ((static_cast<uint32_t>(code) & 0xFFu) << (8 * e));
+      packed |= Q4 ? (static_cast<uint64_t>(static_cast<uint32_t>(code) & 0xFu) << (4 * e))
+                   : (static_cast<uint64_t>(static_cast<uint32_t>(code) & 0xFFu) << (8 * e));
     }
-    int8_t* dst = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(tc) + 4u * tid;
-    *reinterpret_cast<uint32_t*>(dst) = packed;
+    int8_t* dst = a.codes + (static_cast<int64_t>(rb) * a.T + tc) * F::kTileBytes + (Q4 ? 4u : kPer) * tid;
+    if (Q4 || kPer == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(packed);
+    else if (kPer == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
+    else *reinterpret_cast<uint64_t*>(dst) = packed;
   }
   report(a.status, flags);
 }
@@ -378,13 +384,13 @@ struct BuildPlan {
   uint32_t smem;
 };
 
-static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override, bool q4) {
+static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override, uint32_t nbk) {
   auto mk = [&](int C, int nbuf) {
     BuildPlan p;
     p.C = C < T ? C : T;
     p.tpc = (T + p.C - 1) / p.C;
     p.nbuf = nbuf;
-    p.smem = build_layout(bf16, has_imp, p.tpc, nbuf, q4).total + 1024;  // + alignment slack
+    p.smem = build_layout(bf16, has_imp, p.tpc, nbuf, nbk).total + 1024;  // + alignment slack
     return p;
   };
   if (cluster_override > 0) {
@@ -401,9 +407,9 @@ static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override
   return p;
 }
 
-template <bool BF16, bool HAS_IMP, bool Q4>
+template <bool BF16, bool HAS_IMP, int VAR>
 static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, int cluster_override) {
-  const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override, Q4);
+  const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override, CodeFmt<VAR>::kBuckets);
   // tensor map over W [M, K] (row stride ldw), one 64 x 256 box per tile
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -420,7 +426,7 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, 
   a.C = p.C;
   a.tpc = p.tpc;
   a.nbuf = p.nbuf;
-  auto kern = build_kernel<BF16, HAS_IMP, Q4>;
+  auto kern = build_kernel<BF16, HAS_IMP, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(p.smem));
   if (e != cudaSuccess) return e;
   if (p.C > 8) {
@@ -444,7 +450,7 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, 
 
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override, int inject, bool q4) {
+                         cudaStream_t stream, int cluster_override, int inject, int var) {
   BuildArgs a;
   a.inject = inject;
   a.W = W; a.ldw = ldw; a.K = K; a.imp = imp; a.seed = seed;
@@ -452,18 +458,20 @@ cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t
   a.T = static_cast<int>(K / kTileCols);
   a.C = a.tpc = a.nbuf = 0;
   const int64_t RB = M / kRowsPerBlock;
-  if (q4) {
+  auto go = [&](auto V) {
+    constexpr int kVar = decltype(V)::value;
     if (bf16)
-      return imp ? launch_build_t<true, true, true>(a, RB, stream, cluster_override)
-                 : launch_build_t<true, false, true>(a, RB, stream, cluster_override);
-    return imp ? launch_build_t<false, true, true>(a, RB, stream, cluster_override)
-               : launch_build_t<false, false, true>(a, RB, stream, cluster_override);
+      return imp ? launch_build_t<true, true, kVar>(a, RB, stream, cluster_override)
+                 : launch_build_t<true, false, kVar>(a, RB, stream, cluster_override);
+    return imp ? launch_build_t<false, true, kVar>(a, RB, stream, cluster_override)
+               : launch_build_t<false, false, kVar>(a, RB, stream, cluster_override);
+  };
+  switch (var) {
+    case 1: return go(std::integral_constant<int, 1>{});
+    case 2: return go(std::integral_constant<int, 2>{});
+    case 3: return go(std::integral_constant<int, 3>{});
+    default: return go(std::integral_constant<int, 0>{});
   }
-  if (bf16)
-    return imp ? launch_build_t<true, true, false>(a, RB, stream, cluster_override)
-               : launch_build_t<true, false, false>(a, RB, stream, cluster_override);
-  return imp ? launch_build_t<false, true, false>(a, RB, stream, cluster_override)
-             : launch_build_t<false, false, false>(a, RB, stream, cluster_override);
 }
 
 }  // namespace usk

@@ -268,6 +268,23 @@ __device__ __forceinline__ uint32_t i8pair_to_bf16x2(uint32_t w) {
   return r;
 }
 
+// Code layouts of the single-row max-key sketch (formats 1 and 4), by variant:
+//   0: 4 slots per class, 8-bit codes (format 1, 0.5 bit/weight)
+//   1: 8 slots, 4-bit codes (format 4, 0.5 bit/weight)
+//   2: 2 slots, 8-bit codes (format 1 at 0.25 bit/weight)
+//   3: 8 slots, 8-bit codes (format 1 at 1 bit/weight)
+// slot = h >> kShift; a tile owns 256 * kSlots buckets; codes of tile (rb, tc)
+// start at byte (rb * K/256 + tc) * kTileBytes.
+template <int VAR>
+struct CodeFmt {
+  static constexpr uint32_t kSlots = VAR == 0 ? 4u : (VAR == 2 ? 2u : 8u);
+  static constexpr bool kNibble = VAR == 1;
+  static constexpr uint32_t kShift = kSlots == 2 ? 31u : (kSlots == 4 ? 30u : 29u);
+  static constexpr uint32_t kBuckets = 256u * kSlots;                        // per tile
+  static constexpr uint32_t kTileBytes = kNibble ? kBuckets / 2 : kBuckets;  // stored per tile
+  static constexpr uint32_t kTileBf = 2u * kBuckets;                         // widened to bf16
+};
+
 // Format 4: 8 signed 4-bit codes (storage byte k holds bucket 2k in its low
 // nibble, bucket 2k + 1 in its high nibble) -> 4 bf16 pairs in bucket order,
 // exact: each nibble biased to u = n + 8 sits under a 0x43 exponent byte (the

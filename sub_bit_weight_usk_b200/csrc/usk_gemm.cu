@@ -83,14 +83,15 @@ struct GemmLayout {
   uint32_t b, cbf, codes, keys, bars, misc, total;
 };
 
-// q4: 4-bit codes (2048 buckets per tile: 4 KiB of bf16 per row block and tile)
-__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int depth, bool q4) {
+// tile_bytes / tile_bf: stored and widened bytes per row block and tile
+__host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int depth, uint32_t tile_bytes,
+                                                  uint32_t tile_bf) {
   GemmLayout L;
   L.b = 0;  // [S][N x 64] bf16, SW128; after the main loop the K-split partials [N][128] fp32
   const uint32_t ring = static_cast<uint32_t>(S) * N * kBK * 2, parts = static_cast<uint32_t>(N) * kBM * 4;
   L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [kTileRing][2][1024 or 2048]
-  L.codes = L.cbf + kTileRing * 2u * (q4 ? 4096u : 2048u);             // int8 [2][tcta][1024]
-  L.keys = L.codes + 2u * tcta * 1024u;                                // uint2 [2][tcta][depth]
+  L.codes = L.cbf + kTileRing * 2u * tile_bf;                          // codes [2][tcta][tile_bytes]
+  L.keys = L.codes + 2u * tcta * tile_bytes;                           // uint2 [2][tcta][depth]
   L.bars = (L.keys + 2u * tcta * depth * 8u + 7u) & ~7u;  // full[S], empty[S], codes, done, ready[ring], free[ring]
   L.misc = L.bars + (2 * S + 2 + 2 * kTileRing) * 8;                   // tmem holder, abort
   L.total = L.misc + 16;
@@ -168,13 +169,16 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 // D = hash rows of the sketch (1: format 1 or format 2 at depth 1; 2, 4: the
 // multi-row AbsMaxMin sketch: the decoders gather every row and keep the code
 // of largest magnitude)
-// Q4: 4-bit codes (D == 1): 8 slots, the widen warp expands 1024 bytes of
-// nibbles per row block and tile into 2048 bf16.
-template <int D, bool Q4>
+// VAR: code layout (CodeFmt; D == 1 unless VAR == 0): the widen warp expands
+// each row block's stored tile (512 to 2048 bytes) into 256 x slots bf16.
+template <int D, int VAR>
 __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
+  using F = CodeFmt<VAR>;
+  constexpr bool Q4 = F::kNibble;
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
-  constexpr uint32_t kRbBf = Q4 ? 4096u : 2048u;  // widened bytes per row block and tile
-  constexpr uint32_t kShift = Q4 ? 29u : 30u;
+  constexpr uint32_t kRbBf = F::kTileBf;         // widened bytes per row block and tile
+  constexpr uint32_t kRbBytes = F::kTileBytes;   // stored bytes per row block and tile
+  constexpr uint32_t kShift = F::kShift;
   extern __shared__ __align__(16) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ks = static_cast<int>(cluster.block_rank());
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   const int tcta = t_end - t_begin;
   const int nk = tcta * (kTileCols / kBK);  // 64-column chunks
   const int S = a.S;
-  const GemmLayout L = gemm_layout(a.N, tcta, S, D, Q4);
+  const GemmLayout L = gemm_layout(a.N, tcta, S, D, kRbBytes, kRbBf);
   const uint32_t bstage = static_cast<uint32_t>(a.N) * kBK * 2;
   const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * S, codes_bar = empty_s + 8 * S;
   const uint32_t done_bar = codes_bar + 8, ready_s = done_bar + 8, free_s = ready_s + 8 * kTileRing;
@@ -217,13 +221,11 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
       mbar_fence_init();
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
       // the block's codes: two contiguous runs (one per row block)
-      const uint32_t bytes = static_cast<uint32_t>(tcta) * 1024u;
+      const uint32_t bytes = static_cast<uint32_t>(tcta) * kRbBytes;
       mbar_arrive_expect_tx(codes_bar, bytes * (second_rb ? 2u : 1u));
-      bulk_g2s(s0 + L.codes, a.codes + static_cast<int64_t>(rb0) * 4 * a.K + 1024 * static_cast<int64_t>(t_begin),
-               bytes, codes_bar);
+      bulk_g2s(s0 + L.codes, a.codes + (static_cast<int64_t>(rb0) * a.T + t_begin) * kRbBytes, bytes, codes_bar);
       if (second_rb)
-        bulk_g2s(s0 + L.codes + bytes,
-                 a.codes + static_cast<int64_t>(rb0 + 1) * 4 * a.K + 1024 * static_cast<int64_t>(t_begin), bytes,
+        bulk_g2s(s0 + L.codes + bytes, a.codes + (static_cast<int64_t>(rb0 + 1) * a.T + t_begin) * kRbBytes, bytes,
                  codes_bar);
     }
     __syncwarp();
@@ -318,18 +320,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
         aborted = true;
         break;
       }
-      // 2 x 1024 codes, 16 per lane per step; all four loads in flight first
-      uint4 w[4];
+      // 2 x kRbBytes stored bytes, 16 per lane per step; all loads in flight first
+      constexpr int kSteps = static_cast<int>(2u * kRbBytes / 512u);
+      uint4 w[kSteps];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kSteps; ++i) {
         const uint32_t idx = static_cast<uint32_t>(lane) * 16u + static_cast<uint32_t>(i) * 512u;
-        w[i] = lds128(s0 + L.codes + ((idx >> 10) * tcta + t) * 1024u + (idx & 1023u));
+        w[i] = lds128(s0 + L.codes + ((idx / kRbBytes) * tcta + t) * kRbBytes + (idx % kRbBytes));
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < kSteps; ++i) {
         const uint32_t idx = static_cast<uint32_t>(lane) * 16u + static_cast<uint32_t>(i) * 512u;
         if constexpr (Q4) {
-          const uint32_t dst = s0 + L.cbf + q * (2u * kRbBf) + (idx >> 10) * kRbBf + 4u * (idx & 1023u);
+          const uint32_t dst = s0 + L.cbf + q * (2u * kRbBf) + (idx / kRbBytes) * kRbBf + 4u * (idx % kRbBytes);
           const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -338,7 +341,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
             sts128(dst + 16u * e, make_uint4(o4[0], o4[1], o4[2], o4[3]));
           }
         } else {
-          const uint32_t dst = s0 + L.cbf + q * 4096u + (idx >> 10) * 2048u + 2u * (idx & 1023u);
+          const uint32_t dst = s0 + L.cbf + q * (2u * kRbBf) + (idx / kRbBytes) * kRbBf + 2u * (idx % kRbBytes);
           sts128(dst, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].x), i8pair_to_bf16x2<0x4342>(w[i].x),
                                  i8pair_to_bf16x2<0x4140>(w[i].y), i8pair_to_bf16x2<0x4342>(w[i].y)));
           sts128(dst + 16u, make_uint4(i8pair_to_bf16x2<0x4140>(w[i].z), i8pair_to_bf16x2<0x4342>(w[i].z),
@@ -470,6 +473,15 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
 
 constexpr uint32_t kSmemLimit = 227u * 1024u;
 
+static uint32_t var_tile_bytes(int var) {
+  return var == 1 ? CodeFmt<1>::kTileBytes : var == 2 ? CodeFmt<2>::kTileBytes : var == 3 ? CodeFmt<3>::kTileBytes
+                                                                                         : CodeFmt<0>::kTileBytes;
+}
+static uint32_t var_tile_bf(int var) {
+  return var == 1 ? CodeFmt<1>::kTileBf : var == 2 ? CodeFmt<2>::kTileBf : var == 3 ? CodeFmt<3>::kTileBf
+                                                                                   : CodeFmt<0>::kTileBf;
+}
+
 // 256 columns (two blocks per SM) when four stages fit next to the accumulators, else 512
 __host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N) + 4u * 32u <= 256u ? 256u : 512u; }
 
@@ -482,29 +494,30 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N)
 // mbarrier has one in-order waiter per role.  Otherwise consecutive uses of a
 // stage belong to different warps, and a warp running ahead can take a
 // completed phase of use n - 2 for use n (a phase wait only tells parity).
-static int gemm_stages(int N, int tpb, int depth, bool q4) {
+static int gemm_stages(int N, int tpb, int depth, int var) {
   const uint32_t cols = gemm_tmem_cols(N);
   const uint32_t smem_cap = cols == 256u ? 233472u / 2u - 1024u : kSmemLimit;
   int S = static_cast<int>((cols - gemm_a_col(N)) / 32u);
   if (S > kMaxStages) S = kMaxStages;
   S &= ~3;
-  while (S >= 4 && gemm_layout(N, tpb, S, depth, q4).total + 1024u > smem_cap) S -= 4;
+  while (S >= 4 && gemm_layout(N, tpb, S, depth, var_tile_bytes(var), var_tile_bf(var)).total + 1024u > smem_cap)
+    S -= 4;
   return S >= 4 ? S : 0;
 }
 
 // Largest number of tiles per block (codes staged up front) that still leaves
 // a four-stage pipeline for batch N.
-static int gemm_max_tiles(int N, int depth, bool q4) {
+static int gemm_max_tiles(int N, int depth, int var) {
   int t = kMaxTiles;
-  while (t > 1 && gemm_stages(N, t, depth, q4) == 0) --t;
+  while (t > 1 && gemm_stages(N, t, depth, var) == 0) --t;
   return t;
 }
 
 // Dynamic shared memory of a launch: the layout, padded so that no more blocks
 // share an SM than its 512 tensor-memory columns hold (a block waiting in
 // tcgen05.alloc for a co-resident block of its own cluster would never proceed).
-static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, bool q4) {
-  const uint32_t smem = gemm_layout(N, tpb, S, depth, q4).total + 1024u;  // + alignment slack
+static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, int var) {
+  const uint32_t smem = gemm_layout(N, tpb, S, depth, var_tile_bytes(var), var_tile_bf(var)).total + 1024u;
   const uint32_t max_blocks = 512u / gemm_tmem_cols(N);
   const uint32_t floor_bytes = 233472u / (max_blocks + 1u) + 1u - 1024u;  // 228 KiB per SM, 1 KiB reserved per block
   return smem > floor_bytes ? smem : floor_bytes;
@@ -515,8 +528,8 @@ static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, bool q4) {
 // pipeline fill, epilogue and the cluster reduction: 4 to 5 us measured against
 // about 1.3 us per tile at batch 16), within the shared-memory bound on tiles
 // per block and clusters of at most 16.
-static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, bool q4) {
-  const int max_tiles = gemm_max_tiles(N, depth, q4);
+static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, int var) {
+  const int max_tiles = gemm_max_tiles(N, depth, var);
   const int64_t slots = static_cast<int64_t>(sms) * (512 / static_cast<int>(gemm_tmem_cols(N)));
   int best = -1;
   int64_t best_cost = -1;
@@ -537,14 +550,15 @@ static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, bool q
 
 // Whether K fits: at most 16 blocks along K, each staging the codes of up to
 // gemm_max_tiles(batch) tiles (32 for every batch: K <= 131072).
-bool gemm_supported(int64_t K, int batch, int depth, bool q4) {
-  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch, depth, q4));
+bool gemm_supported(int64_t K, int batch, int depth, int var) {
+  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch, depth, var));
 }
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth, bool q4) {
-  if ((depth != 1 && depth != 2 && depth != 4) || (q4 && depth != 1)) return cudaErrorInvalidValue;
+                        int depth, int var) {
+  if ((depth != 1 && depth != 2 && depth != 4) || (var != 0 && depth != 1) || var < 0 || var > 3)
+    return cudaErrorInvalidValue;
   GemmArgs a;
   a.codes = codes; a.scales = scales; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status; a.inject = inject;
@@ -553,15 +567,15 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   const int64_t m_tiles = (M + kBM - 1) / kBM;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth, q4);
+  a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth, var);
   if (a.splits < 1) return cudaErrorInvalidValue;  // K beyond 16 blocks x the tiles one block can stage
   a.tmem_cols = gemm_tmem_cols(batch);
   a.a_col = gemm_a_col(batch);
   a.I = gemm_issuers(batch);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
-  a.S = gemm_stages(batch, tcta_max, depth, q4);
+  a.S = gemm_stages(batch, tcta_max, depth, var);
   if (a.S < 4 || a.S % 4 != 0) return cudaErrorInvalidValue;
-  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth, q4);
+  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth, var);
   // tensor map over x [batch, K] bf16: one 64-column x batch box per chunk, 128-byte swizzle
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -574,8 +588,10 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = q4 ? gemm_kernel<1, true>
-                 : (depth == 4 ? gemm_kernel<4, false> : (depth == 2 ? gemm_kernel<2, false> : gemm_kernel<1, false>));
+  auto kern = var == 1 ? gemm_kernel<1, 1>
+             : var == 2 ? gemm_kernel<1, 2>
+             : var == 3 ? gemm_kernel<1, 3>
+             : (depth == 4 ? gemm_kernel<4, 0> : (depth == 2 ? gemm_kernel<2, 0> : gemm_kernel<1, 0>));
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.splits > 8) {

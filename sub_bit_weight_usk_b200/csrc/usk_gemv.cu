@@ -57,12 +57,12 @@ struct GemvLayout {
   uint32_t keys, codes, xs, xrow, stage_end, parts, cta, total;
 };
 
-__host__ __device__ inline GemvLayout gemv_layout(int tpc, int nb, int batch, bool xf32, int depth, bool q4) {
+__host__ __device__ inline GemvLayout gemv_layout(int tpc, int nb, int batch, bool xf32, int depth, uint32_t tile_bf) {
   GemvLayout L;
   const uint32_t nvalid = static_cast<uint32_t>(xf32 ? 2 * batch : batch);
   L.keys = 0;
   L.codes = (static_cast<uint32_t>(tpc * depth) * 8u + 15u) / 16u * 16u;
-  L.xs = L.codes + static_cast<uint32_t>(tpc) * (q4 ? 4096u : 2048u);
+  L.xs = L.codes + static_cast<uint32_t>(tpc) * tile_bf;
   L.xrow = static_cast<uint32_t>(tpc) * 512u + 16u;
   L.stage_end = L.xs + nvalid * L.xrow;
   L.parts = 0;
@@ -82,12 +82,14 @@ __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *rein
 // D = hash rows (1: format 1 or format 2 at depth 1; 2, 4: the multi-row
 // AbsMaxMin sketch, each row gathered from its own 2048/D-byte segment of the
 // tile and reduced to the code of largest magnitude)
-// Q4: 4-bit codes (D == 1): 8 slots, 4 KiB of widened codes per tile.
-template <int NB, bool XF32, int D, bool Q4>
+// VAR: code layout (CodeFmt; D == 1 unless VAR == 0).
+template <int NB, bool XF32, int D, int VAR>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
+  using F = CodeFmt<VAR>;
+  constexpr bool Q4 = F::kNibble;
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
-  constexpr uint32_t kTileBf = Q4 ? 4096u : 2048u;
-  constexpr uint32_t kShift = Q4 ? 29u : 30u;
+  constexpr uint32_t kTileBf = F::kTileBf;
+  constexpr uint32_t kShift = F::kShift;
   extern __shared__ __align__(16) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -96,15 +98,15 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);  // >= 1 by construction of C
   const int nvalid = XF32 ? 2 * a.batch : a.batch;
-  const GemvLayout L = gemv_layout(a.tpc, NB, a.batch, XF32, D, Q4);
+  const GemvLayout L = gemv_layout(a.tpc, NB, a.batch, XF32, D, kTileBf);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   const uint32_t sm_s = smem_u32(sm);
 
   // ---- stage: hash keys, codes (int8 -> bf16) and the x slice, all loads in flight at once
   if (tid < nt * D) keytab[tid] = row_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid / D, D, tid % D);
   {
-    const int8_t* csrc = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
-    const int ncode = nt * 64;                                   // 16-byte code chunks
+    const int8_t* csrc = a.codes + (static_cast<int64_t>(rb) * a.T + t0) * F::kTileBytes;
+    const int ncode = nt * static_cast<int>(F::kTileBytes / 16u);  // 16-byte code chunks
     const int xchunks_row = XF32 ? nt * 64 : nt * 32;            // 16-byte x chunks per batch row
     const int nx = a.batch * xchunks_row;
     const int total = ncode + nx;
@@ -290,10 +292,10 @@ static GemvGeometry gemv_geometry(int64_t K, int tpc_override) {
   return g;
 }
 
-template <int NB, bool XF32, int D, bool Q4>
+template <int NB, bool XF32, int D, int VAR>
 static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32, D, Q4).total;
-  auto kern = gemv_kernel<NB, XF32, D, Q4>;
+  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32, D, CodeFmt<VAR>::kTileBf).total;
+  auto kern = gemv_kernel<NB, XF32, D, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -323,21 +325,21 @@ cudaError_t launch_gemv_slab(const int8_t* codes, const uint16_t* scales, int64_
 bool gemv_bf_supported(int64_t K, int batch, int tpc_override);
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth, bool q4);
+                           int tpc_override, int inject, int depth, int var);
 
-template <int D, bool Q4>
+template <int D, int VAR>
 static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaStream_t stream) {
   const int rows = xf32 ? 2 * a.batch : a.batch;
   const int nb = (rows + 7) / 8;
   if (!xf32) {
-    if (nb == 1) return launch_gemv_t<1, false, D, Q4>(a, RB, stream);
-    return launch_gemv_t<2, false, D, Q4>(a, RB, stream);
+    if (nb == 1) return launch_gemv_t<1, false, D, VAR>(a, RB, stream);
+    return launch_gemv_t<2, false, D, VAR>(a, RB, stream);
   }
   switch (nb) {
-    case 1: return launch_gemv_t<1, true, D, Q4>(a, RB, stream);
-    case 2: return launch_gemv_t<2, true, D, Q4>(a, RB, stream);
-    case 3: return launch_gemv_t<3, true, D, Q4>(a, RB, stream);
-    default: return launch_gemv_t<4, true, D, Q4>(a, RB, stream);
+    case 1: return launch_gemv_t<1, true, D, VAR>(a, RB, stream);
+    case 2: return launch_gemv_t<2, true, D, VAR>(a, RB, stream);
+    case 3: return launch_gemv_t<3, true, D, VAR>(a, RB, stream);
+    default: return launch_gemv_t<4, true, D, VAR>(a, RB, stream);
   }
 }
 
@@ -347,7 +349,7 @@ static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaS
 // rows of the sketch: the integer paths read single-row sketches only.
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, bool q4) {
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // automatic choice (measured on B200, graphs of back-to-back calls):
@@ -355,7 +357,7 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   //  * batch >= 2, or batch 1 up to 4096 x 4096: bf16 with direct x fragments;
   //  * batch 1 with longer K or taller M: the integer cluster kernel (half the
   //    shared-memory gather bytes; its x preparation is amortised over more tiles)
-  const bool single = depth == 1 && !q4;  // the integer paths read one-row 8-bit sketches
+  const bool single = depth == 1 && var == 0;  // the integer paths read format-1 layouts of 4 slots
   const bool slab = single && (path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms));
   if (!xf32 && slab && slab_supported(K, batch))
     return launch_gemv_slab(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl,
@@ -365,7 +367,7 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
       path == 4 || (!single && path != 1) || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
   if (!xf32 && direct && gemv_bf_supported(K, batch, tpc_override))
     return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
-                          tpc_override, inject, depth, q4);
+                          tpc_override, inject, depth, var);
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
   const bool i8_ok = single && !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
   if (i8_ok && path != 1)
@@ -376,10 +378,12 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.M = M; a.K = K; a.seed = seed;
   a.T = geo.T; a.C = geo.C; a.tpc = geo.tpc; a.batch = batch;
   const int64_t RB = M / kRowsPerBlock;
-  if (q4) return launch_staged<1, true>(a, xf32, RB, stream);
-  if (depth == 2) return launch_staged<2, false>(a, xf32, RB, stream);
-  if (depth == 4) return launch_staged<4, false>(a, xf32, RB, stream);
-  return launch_staged<1, false>(a, xf32, RB, stream);
+  if (var == 1) return launch_staged<1, 1>(a, xf32, RB, stream);
+  if (var == 2) return launch_staged<1, 2>(a, xf32, RB, stream);
+  if (var == 3) return launch_staged<1, 3>(a, xf32, RB, stream);
+  if (depth == 2) return launch_staged<2, 0>(a, xf32, RB, stream);
+  if (depth == 4) return launch_staged<4, 0>(a, xf32, RB, stream);
+  return launch_staged<1, 0>(a, xf32, RB, stream);
 }
 
 }  // namespace usk

@@ -63,11 +63,11 @@ struct GemvBfLayout {
   uint32_t cbf, keys, red, push, bars, total;
 };
 
-// q4: 4-bit codes, 2048 buckets per tile (4 KiB of bf16)
-__host__ __device__ inline GemvBfLayout gemv_bf_layout(int tpc, int batch, int C, int depth, bool q4) {
+// tile_bf: widened bytes per tile (2 x buckets per tile)
+__host__ __device__ inline GemvBfLayout gemv_bf_layout(int tpc, int batch, int C, int depth, uint32_t tile_bf) {
   GemvBfLayout L;
-  L.cbf = 0;                                                       // bf16 [tpc][1024 or 2048]
-  L.keys = L.cbf + static_cast<uint32_t>(tpc) * (q4 ? 4096u : 2048u);  // uint2 [tpc][depth]
+  L.cbf = 0;                                                       // bf16 [tpc][buckets per tile]
+  L.keys = L.cbf + static_cast<uint32_t>(tpc) * tile_bf;          // uint2 [tpc][depth]
   L.red = (L.keys + static_cast<uint32_t>(tpc * depth) * 8u + 15u) & ~15u;  // fp32 [8 warps][batch][64]
   L.push = L.red + 8u * batch * 64u * 4u;                          // fp32 [C][batch][64] (used in rank 0)
   L.bars = (L.push + static_cast<uint32_t>(C) * batch * 64u * 4u + 7u) & ~7u;  // push
@@ -92,13 +92,16 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
 // D = hash rows of the sketch (1: format 1, or format 2 at depth 1; 2, 4: the
 // multi-row AbsMaxMin sketch, whose rows are gathered and reduced to the code
 // of largest magnitude before the MMA)
-// Q4: the 4-bit-code format (D == 1): 8 slots (slot = h >> 29), 2048 buckets and
-// 4 KiB of widened codes per tile; each 16-byte load holds 32 codes.
-template <int B, int D, bool Q4>
+// VAR: code layout (CodeFmt; D == 1 unless VAR == 0): 2, 4 or 8 slots per
+// class, 8-bit codes, or 8 slots with 4-bit codes (32 codes per 16-byte load).
+template <int B, int D, int VAR>
 __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a) {
+  using F = CodeFmt<VAR>;
+  constexpr bool Q4 = F::kNibble;
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
-  constexpr uint32_t kTileBf = Q4 ? 4096u : 2048u;  // widened bytes per tile
-  constexpr uint32_t kShift = Q4 ? 29u : 30u;
+  constexpr uint32_t kTileBf = F::kTileBf;  // widened bytes per tile
+  constexpr uint32_t kShift = F::kShift;
+  constexpr int kChunks = static_cast<int>(F::kTileBytes / 16u);  // 16-byte code loads per tile
   extern __shared__ __align__(128) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
@@ -106,25 +109,25 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);
-  const GemvBfLayout L = gemv_bf_layout(a.tpc, B, a.C, D, Q4);
+  const GemvBfLayout L = gemv_bf_layout(a.tpc, B, a.C, D, kTileBf);
   const uint32_t s0 = smem_u32(sm);
   const uint32_t push_bar = s0 + L.bars;
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   float* red = reinterpret_cast<float*>(sm + L.red);
   float* push = reinterpret_cast<float*>(sm + L.push);
   constexpr uint32_t kPartBytes = static_cast<uint32_t>(B) * 64u * 4u;
-  constexpr int kCodeLoads = kBfMaxTiles * 1024 / 16 / kBfThreads;  // 16-byte code loads per thread (at most)
+  constexpr int kCodeLoads = kBfMaxTiles * kChunks / kBfThreads;  // 16-byte code loads per thread (at most)
 
   // ---- every global load first.  The codes are never written by a neighbour
   // in a programmatic-dependent chain (the caller's contract), so they go
   // before the dependency wait and overlap the previous kernel's tail; x after.
-  const int8_t* codes_blk = a.codes + static_cast<int64_t>(rb) * 4 * a.K + 1024 * static_cast<int64_t>(t0);
+  const int8_t* codes_blk = a.codes + (static_cast<int64_t>(rb) * a.T + t0) * F::kTileBytes;
   uint4 cv[kCodeLoads];
 #pragma unroll
   for (int u = 0; u < kCodeLoads; ++u) {
     const int q = tid + u * kBfThreads;  // 16-code chunk
     cv[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (q < nt * 64) cv[u] = ldg_nc128(codes_blk + 16 * q);
+    if (q < nt * kChunks) cv[u] = ldg_nc128(codes_blk + 16 * q);
   }
   if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int g = lane >> 2, t = lane & 3;
@@ -152,7 +155,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
 #pragma unroll
   for (int u = 0; u < kCodeLoads; ++u) {
     const int q = tid + u * kBfThreads;
-    if (q < nt * 64) {
+    if (q < nt * kChunks) {
       const uint32_t ws[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
       if constexpr (Q4) {
 #pragma unroll
@@ -283,10 +286,10 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   }
 }
 
-template <int B, int D, bool Q4>
+template <int B, int D, int VAR>
 static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
-  const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D, Q4).total;
-  auto kern = gemv_bf_kernel<B, D, Q4>;
+  const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D, CodeFmt<VAR>::kTileBf).total;
+  auto kern = gemv_bf_kernel<B, D, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -310,17 +313,17 @@ static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int D, bool Q4>
+template <int D, int VAR>
 static cudaError_t launch_bf_batch(const GemvBfArgs& a, int batch, int64_t RB, cudaStream_t stream) {
   switch (batch) {
-    case 1: return launch_bf_t<1, D, Q4>(a, RB, stream);
-    case 2: return launch_bf_t<2, D, Q4>(a, RB, stream);
-    case 3: return launch_bf_t<3, D, Q4>(a, RB, stream);
-    case 4: return launch_bf_t<4, D, Q4>(a, RB, stream);
-    case 5: return launch_bf_t<5, D, Q4>(a, RB, stream);
-    case 6: return launch_bf_t<6, D, Q4>(a, RB, stream);
-    case 7: return launch_bf_t<7, D, Q4>(a, RB, stream);
-    default: return launch_bf_t<8, D, Q4>(a, RB, stream);
+    case 1: return launch_bf_t<1, D, VAR>(a, RB, stream);
+    case 2: return launch_bf_t<2, D, VAR>(a, RB, stream);
+    case 3: return launch_bf_t<3, D, VAR>(a, RB, stream);
+    case 4: return launch_bf_t<4, D, VAR>(a, RB, stream);
+    case 5: return launch_bf_t<5, D, VAR>(a, RB, stream);
+    case 6: return launch_bf_t<6, D, VAR>(a, RB, stream);
+    case 7: return launch_bf_t<7, D, VAR>(a, RB, stream);
+    default: return launch_bf_t<8, D, VAR>(a, RB, stream);
   }
 }
 
@@ -335,7 +338,7 @@ bool gemv_bf_supported(int64_t K, int batch, int tpc_override) {
 
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth, bool q4) {
+                           int tpc_override, int inject, int depth, int var) {
   GemvBfArgs a;
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status;
@@ -347,10 +350,12 @@ cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t 
   a.pdl = pdl ? 1 : 0;
   a.inject = inject;
   const int64_t RB = M / kRowsPerBlock;
-  if (q4) return launch_bf_batch<1, true>(a, batch, RB, stream);
-  if (depth == 2) return launch_bf_batch<2, false>(a, batch, RB, stream);
-  if (depth == 4) return launch_bf_batch<4, false>(a, batch, RB, stream);
-  return launch_bf_batch<1, false>(a, batch, RB, stream);
+  if (var == 1) return launch_bf_batch<1, 1>(a, batch, RB, stream);
+  if (var == 2) return launch_bf_batch<1, 2>(a, batch, RB, stream);
+  if (var == 3) return launch_bf_batch<1, 3>(a, batch, RB, stream);
+  if (depth == 2) return launch_bf_batch<2, 0>(a, batch, RB, stream);
+  if (depth == 4) return launch_bf_batch<4, 0>(a, batch, RB, stream);
+  return launch_bf_batch<1, 0>(a, batch, RB, stream);
 }
 
 }  // namespace usk

@@ -61,8 +61,9 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.usk_build(fake, 7, 64, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 3
     assert lib.usk_build(fake, 1, 64, 256, 256, None, None, fake, fake, None, None) == 6
     # unknown format, bad depth for the format, reserved bits, importance with format 2
-    for bad in (_native.UskParams(5, 0, 0, 1, 0), _native.UskParams(4, 0, 0, 2, 0), _native.UskParams(3, 0, 0, 2, 0), _native.UskParams(2, 0, 0, 0, 0), _native.UskParams(2, 0, 0, 3, 0),
-                _native.UskParams(1, 0, 0, 2, 0), _native.UskParams(2, 0, 0, 2, 1), _native.UskParams(1, 1, 0, 1, 0)):
+    for bad in (_native.UskParams(5, 0, 0, 1, 0), _native.UskParams(4, 0, 0, 2, 0), _native.UskParams(1, 0, 0, 1, 3),
+                _native.UskParams(4, 0, 0, 1, 4), _native.UskParams(2, 0, 0, 2, 8), _native.UskParams(3, 0, 0, 2, 0), _native.UskParams(2, 0, 0, 0, 0), _native.UskParams(2, 0, 0, 3, 0),
+                _native.UskParams(1, 0, 0, 2, 0), _native.UskParams(1, 1, 0, 1, 0)):
         assert lib.usk_build(fake, 1, 64, 256, 256, None, ctypes.byref(bad), fake, fake, None, None) == 6
     amm = _native.UskParams(2, 0, 0, 2, 0)
     assert lib.usk_build(fake, 1, 64, 256, 256, fake, ctypes.byref(amm), fake, fake, None, None) == 6
@@ -94,3 +95,39 @@ def test_binding_refuses_cpu_tensors(lib):
     import torch
     with pytest.raises(ValueError):
         usk.usk_build(torch.zeros((64, 256), dtype=torch.bfloat16))
+
+
+def test_plan_slots_matches_the_oracle_procedure(lib):
+    """The library's allocation (C++) against the oracle's (Python), written
+    separately from the same definition: identical slot counts."""
+    import numpy as np
+    import oracle
+    g = np.random.default_rng(17)
+    for trial in range(200):
+        n = int(g.integers(1, 60))
+        w = [int(v) * 16384 for v in g.integers(1, 300, size=n)]
+        imp = [float(v) for v in g.lognormal(0, 2, size=n)]
+        if trial % 7 == 0:
+            imp = [float(int(v)) for v in g.integers(0, 3, size=n)]  # many ties
+        budget = float(g.uniform(0.25, 1.0))
+        assert usk.usk_plan_slots(w, imp, budget) == oracle.plan_slots(w, imp, budget)
+    assert usk.usk_plan_slots([], [], 0.5) == []
+    for bad in ((0.2,), (1.5,)):
+        with pytest.raises(usk.UskError):
+            usk.usk_plan_slots([1], [1.0], bad[0])
+    with pytest.raises(usk.UskError):
+        usk.usk_plan_slots([1], [-1.0], 0.5)
+    with pytest.raises(usk.UskError):
+        usk.usk_plan_slots([0], [1.0], 0.5)
+
+
+def test_sizes_ex(lib):
+    assert usk.usk_sizes_ex(4096, 4096) == (4096 * 4096 // 16, 128)
+    assert usk.usk_sizes_ex(4096, 4096, 1, 2) == (4096 * 4096 // 32, 128)
+    assert usk.usk_sizes_ex(4096, 4096, 1, 8) == (4096 * 4096 // 8, 128)
+    assert usk.usk_sizes_ex(4096, 4096, 4, 0) == (4096 * 4096 // 16, 128)
+    assert usk.usk_sizes_ex(4096, 4096, 2, 4) == (4096 * 4096 // 16, 128)
+    with pytest.raises(usk.UskError):
+        usk.usk_sizes_ex(4096, 4096, 2, 8)
+    with pytest.raises(usk.UskError):
+        usk.usk_sizes_ex(4096, 4096, 1, 3)
