@@ -308,7 +308,10 @@ __device__ __forceinline__ void i4x8_to_bf16x8(uint32_t w, uint32_t (&o)[4]) {
 // keeps bit 15 exactly when |a| >= |b| (bf16 magnitude bits order like values).
 __device__ __forceinline__ uint32_t absmax_sel_bf16x2(uint32_t a, uint32_t b) {
   const uint32_t d = (a | 0x80008000u) - (b & 0x7FFF7FFFu);
-  const uint32_t m = ((d >> 15) & 0x00010001u) * 0xFFFFu;
+  // mask 0xFFFF per half where bit 15 of the half is set: a byte permute whose
+  // selectors 9 and 11 replicate the sign bit of bytes 1 and 3 (PTX prmt, default mode)
+  uint32_t m;
+  asm("prmt.b32 %0, %1, 0, 0xBB99;" : "=r"(m) : "r"(d));
   return (a & m) | (b & ~m);
 }
 
