@@ -306,15 +306,19 @@ constexpr int kCsMaxTiles = 16;  // tiles per block
 constexpr int kCsMaxBatch = 15;
 
 struct GemvCsLayout {
-  uint32_t z, push, bars, total;
+  uint32_t ctile, z, push, bars, total;
 };
 
+// 256-row blocks stage their codes (256 rows x 128 bytes, 128-byte swizzle) at
+// the 1024-byte aligned start; then z, the first block's receive area and two
+// mbarriers (partial sums, code tile).
 __host__ __device__ inline GemvCsLayout gemv_cs_layout(int tpb, int batch, int C, int R) {
   GemvCsLayout L;
-  L.z = 0;                                                                  // fp32 [batch][16 tpb]
+  L.ctile = 0;
+  L.z = R == 256 ? 256u * 128u : 0u;                                        // fp32 [batch][16 tpb]
   L.push = L.z + static_cast<uint32_t>(batch * 16 * tpb) * 4u;             // fp32 [C][batch][R] (rank 0)
   L.bars = (L.push + static_cast<uint32_t>(C * batch * R) * 4u + 7u) & ~7u;
-  L.total = L.bars + 8u;
+  L.total = L.bars + 16u;
   return L;
 }
 
@@ -330,24 +334,30 @@ __device__ __forceinline__ void cs_st_async_f32(uint32_t remote_addr, float v, u
                : "memory");
 }
 
-// TPR threads per row (4: 64-row blocks, up to 16 tiles; 1: 256-row blocks, up
-// to 8 tiles): thread (row r, part q) takes tiles q, q + TPR, ... of its row
-// (16 codes each; the TPR lanes of a row read adjacent 16-byte pieces).  The
-// bucket sums use four threads per bucket, four members each, all loads of a
-// thread in flight at once.
+// TPR threads per row.  4: 64-row blocks of up to 16 tiles; thread (row r,
+// part q) loads tiles q, q + 4, ... of its row (16 codes each, the four lanes of
+// a row read adjacent 16-byte pieces).  1: 256-row blocks of 8 tiles; the block's
+// codes (256 rows x 128 bytes, rows K/16 bytes apart) arrive by one 2-D tensor
+// copy into 128-byte-swizzled shared memory -- as per-thread loads each warp
+// instruction touched 32 separate lines and issuing them took 1.4 us (traced)
+// -- and thread r reads row r's 8 pieces conflict-free.  The bucket sums use
+// four threads per bucket, four members each, all loads in flight at once.
 template <int B, bool XF32, int TPR>
-__global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a) {
+__global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a,
+                                                             const __grid_constant__ CUtensorMap cmap) {
   constexpr int R = kCsThreads / TPR, tpr = TPR;
   constexpr int kCsChunks = TPR == 4 ? 4 : 8;  // 16-code pieces per thread
-  extern __shared__ __align__(128) uint8_t sm[];
+  extern __shared__ __align__(128) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
   const int tid = threadIdx.x;
   const int t0 = crank * a.tpb;
   const int nt = min(a.tpb, a.T - t0);
   const GemvCsLayout L = gemv_cs_layout(a.tpb, B, a.C, R);
-  const uint32_t s0 = smem_u32(sm);
-  const uint32_t push_bar = s0 + L.bars;
+  const uint32_t raw_s = smem_u32(sm_raw);
+  const uint32_t s0 = (raw_s + 1023u) & ~1023u;  // the swizzled code tile wants 1024-byte alignment
+  uint8_t* sm = sm_raw + (s0 - raw_s);
+  const uint32_t push_bar = s0 + L.bars, code_bar = push_bar + 8u;
   float* zs = reinterpret_cast<float*>(sm + L.z);
   float* push = reinterpret_cast<float*>(sm + L.push);
   const int nbk = 16 * a.tpb;  // z row stride
@@ -359,11 +369,19 @@ __global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a)
   const bool row_ok = row < a.M;
   const int8_t* crow = a.codes + row * (a.K / 16) + 16 * static_cast<int64_t>(t0);
   uint4 cv[kCsChunks];
+  if constexpr (TPR == 4) {
 #pragma unroll
-  for (int u = 0; u < kCsChunks; ++u) {
-    const int tl = q + tpr * u;
-    cv[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (row_ok && tl < nt) cv[u] = ldg_nc128(crow + 16 * tl);
+    for (int u = 0; u < kCsChunks; ++u) {
+      const int tl = q + tpr * u;
+      cv[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (row_ok && tl < nt) cv[u] = ldg_nc128(crow + 16 * tl);
+    }
+  } else if (tid == 0) {
+    // rows and columns outside the matrix are filled with zeros by the copy
+    mbar_init(code_bar, 1);
+    mbar_fence_init();
+    mbar_arrive_expect_tx(code_bar, 256u * 128u);
+    tma_load_2d(s0 + L.ctile, &cmap, 16 * t0, static_cast<int>(blockIdx.y) * R, code_bar);
   }
   if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0 && a.C > 1) {
@@ -405,6 +423,12 @@ __global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a)
   __syncthreads();
   if (a.C > 1 && crank != 0) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 
+  if constexpr (TPR == 1) {
+    if (!mbar_wait(code_bar, 0)) report(a.status, USK_FLAG_TIMEOUT);  // bounded (about 1 s)
+#pragma unroll
+    for (int u = 0; u < kCsChunks; ++u)  // piece u of row r, 128-byte swizzle
+      cv[u] = lds128(s0 + L.ctile + static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>(u ^ (r & 7)) * 16u));
+  }
   // ---- S z: 16 codes per tile against the tile's 16 bucket sums
   float acc[B];
 #pragma unroll
@@ -486,8 +510,22 @@ __global__ void __launch_bounds__(kCsThreads) gemv_cs_kernel(const GemvCsArgs a)
 
 template <int B, bool XF32>
 static cudaError_t launch_gemv_cs_t(GemvCsArgs a, cudaStream_t stream) {
-  const size_t smem = gemv_cs_layout(a.tpb, B, a.C, a.R).total;
+  const size_t smem = gemv_cs_layout(a.tpb, B, a.C, a.R).total + 1024;  // + alignment slack
   auto kern = a.R == 64 ? gemv_cs_kernel<B, XF32, 4> : gemv_cs_kernel<B, XF32, 1>;
+  CUtensorMap cmap = {};
+  if (a.R == 256) {
+    // codes [M][K/16] bytes; one 128-byte x 256-row box per block, 128-byte swizzle
+    const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) return cudaErrorNotSupported;
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(a.K / 16), static_cast<cuuint64_t>(a.M)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(a.K / 16)};
+    const cuuint32_t box[2] = {128u, 256u};
+    const cuuint32_t estride[2] = {1, 1};
+    if (encode(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(a.codes), gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -508,7 +546,7 @@ static cudaError_t launch_gemv_cs_t(GemvCsArgs a, cudaStream_t stream) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, kern, a);
+  return cudaLaunchKernelEx(&cfg, kern, a, cmap);
 }
 
 template <bool XF32>
@@ -536,25 +574,25 @@ static cudaError_t launch_gemv_cs_b(const GemvCsArgs& a, int batch, cudaStream_t
 // is at most 16 (R = 64) or 8 (R = 256); it doubles, then R drops to 64, until
 // the cluster has at most 16 blocks.
 static void cs_geometry(GemvCsArgs& a, int R, int tpb) {
-  a.R = R;
-  a.tpb = tpb;
+  a.R = (R == 256 && a.T >= 8) ? 256 : 64;
+  a.tpb = a.R == 256 ? 8 : tpb;  // 256-row blocks copy 128 bytes (8 tiles) of each row
   for (;;) {
     const int cap = a.R == 64 ? 16 : 8;
     if (a.tpb > cap) a.tpb = cap;
     if ((a.T + a.tpb - 1) / a.tpb <= 16) break;
     if (a.tpb < cap) a.tpb *= 2;
-    else if (a.R > 64) a.R = 64;
+    else if (a.R > 64) a.R = 64, a.tpb = 16;
     else break;
   }
   a.C = (a.T + a.tpb - 1) / a.tpb;
 }
 
-// Geometry: tpb_override (rounded down to a power of two) and rows_override (64
-// or 256) if given; else 256-row blocks of 8 tiles for tall matrices (at least
-// two row blocks of 64 per SM: the bucket sums of x are amortised over more
-// rows and the grid stays within one wave), 256-row blocks of 4 tiles from
-// batch 4 (the bucket sums grow with the batch), 64-row blocks of 4 tiles
-// otherwise (fewer registers, more blocks in flight) -- measured on B200.
+// Geometry: tpb_override (rounded down to a power of two; 256-row blocks always
+// take 8 tiles) and rows_override (64 or 256) if given; else 256-row blocks for
+// tall matrices (at least two row blocks of 64 per SM: the bucket sums of x are
+// amortised over more rows, the codes arrive by one tensor copy per block and
+// the grid stays within one wave) and from batch 4 when there is at least one
+// row block per SM, 64-row blocks of 4 tiles otherwise -- measured on B200.
 cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl,
                            cudaStream_t stream, int tpb_override, int rows_override, int inject) {
@@ -573,8 +611,9 @@ cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t 
     while (tpb_given * 2 <= tpb_override && tpb_given < kCsMaxTiles) tpb_given *= 2;
   }
   const bool tall = M / kRowsPerBlock >= 2 * sms;
-  const int R = (rows_override == 64 || rows_override == 256) ? rows_override : ((tall || batch >= 4) ? 256 : 64);
-  cs_geometry(a, R, tpb_given ? tpb_given : ((R == 256 && tall) ? 8 : 4));
+  const bool wide = tall || (batch >= 4 && M / kRowsPerBlock >= sms);
+  const int R = (rows_override == 64 || rows_override == 256) ? rows_override : (wide ? 256 : 64);
+  cs_geometry(a, R, tpb_given ? tpb_given : 4);
   // the first block's receive area: 64-row blocks when it would not fit
   if (gemv_cs_layout(a.tpb, batch, a.C, a.R).total > 200u * 1024u) cs_geometry(a, 64, a.tpb);
   if (a.C > 16) return cudaErrorInvalidValue;
