@@ -12,7 +12,9 @@ third runs K builds and K batch-1 GEMVs of the column-shared projection sketch
 (format 3, y = S (P^T x)) and a fourth the "matrix vs hash" A/B: K batch-1 GEMVs
 of a 28672x8192 layer in format 1 (per-weight rehash and gather) and in format 3
 (bucket sums of x, then dense codes), reported under "colshared"; a fifth runs
-the three calls on the 4-bit-code sketch (format 4) of the layer ("q4").
+the three calls on the 4-bit-code sketch (format 4) of the layer ("q4"), and a
+sixth K builds and K batch-1 GEMVs of the layer at 2 and 8 hash slots per class
+(0.25 and 1 bit/weight, the rates of the importance-aware allocation, "rates").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl usk|reference]
 
@@ -449,11 +451,30 @@ def run_usk(args):
     def gemm4(i):
         usk.usk_gemm(sks4[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
 
+    # format 1 at 2 and 8 hash slots per class (0.25 and 1 bit/weight)
+    rate_sk = {}
+    for nsl in (2, 8):
+        skr = usk.usk_build(W, imp, seed, slots=nsl)
+        rate_sk[nsl] = [usk.Sketch(M, K, seed, skr.codes.clone(), skr.scales.clone(), usk.FORMAT_MAXKEY, 1, nsl)
+                        for _ in range(N_SKETCHES)]
+
+    def build_rate(nsl):
+        def f(i):
+            b = rate_sk[nsl][i % N_SKETCHES]
+            usk.usk_build(Ws[i % N_WCOPIES], imp, seed, codes=b.codes, scales=b.scales, status=status, slots=nsl)
+        return f
+
+    def gemv_rate(nsl):
+        def f(i):
+            usk.usk_gemv(rate_sk[nsl][(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1, pdl=True)
+        return f
+
     graphs1 = prepare((build, gemv, gemm))
     graphs2 = prepare((build2, gemv2, gemm2))
     graphs3 = prepare((build3, gemv3))
     graphs4 = prepare((gemv_hash, gemv_matrix))
     graphs5 = prepare((build4, gemv4, gemm4))
+    graphs6 = prepare((build_rate(2), gemv_rate(2), build_rate(8), gemv_rate(8)))
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
@@ -462,6 +483,7 @@ def run_usk(args):
     t_build3, t_gemv3, _ = timed(graphs3)
     t_hash, t_matrix, _ = timed(graphs4)
     t_build4, t_gemv4, t_gemm4, _ = timed(graphs5)
+    t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8, _ = timed(graphs6)
     sampler.stop()
     t_step = t_total / max(args.steps, 1)
 
@@ -483,9 +505,9 @@ def run_usk(args):
 
     # max over ranks
     (t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2, t_build3, t_gemv3, t_hash,
-     t_matrix, t_build4, t_gemv4, t_gemm4) = max_over_ranks(
+     t_matrix, t_build4, t_gemv4, t_gemm4, t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8) = max_over_ranks(
         [t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2, t_build3, t_gemv3, t_hash,
-         t_matrix, t_build4, t_gemv4, t_gemm4], device=dev)
+         t_matrix, t_build4, t_gemv4, t_gemm4, t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8], device=dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -578,6 +600,18 @@ def run_usk(args):
                           "usk_gemm": round(t_gemm4 * 1e6, 3)},
             "rooflines": rl4,
             "gpu_launches": 3 * args.steps,
+        },
+        "rates": {
+            "format": "format 1 at 2 and 8 hash slots per class (0.25 and 1 bit/weight), the rates the "
+                      "importance-aware allocation (usk_plan_slots) assigns; same layer and importance",
+            "timing": "sixth timed region: K builds and K GEMVs (batch 1) at each rate as CUDA graphs",
+            "slots_2": {"kernel_us": {"usk_build": round(t_build_r2 * 1e6, 3), "usk_gemv": round(t_gemv_r2 * 1e6, 3)},
+                        "usk_gemv_gbs": round(world * (GEMV_BYTES - N_W // 32) / t_gemv_r2 / 1e9, 3),
+                        "usk_build_gweights_per_s": round(world * N_W / t_build_r2 / 1e9, 3)},
+            "slots_8": {"kernel_us": {"usk_build": round(t_build_r8 * 1e6, 3), "usk_gemv": round(t_gemv_r8 * 1e6, 3)},
+                        "usk_gemv_gbs": round(world * (GEMV_BYTES + N_W // 16) / t_gemv_r8 / 1e9, 3),
+                        "usk_build_gweights_per_s": round(world * N_W / t_build_r8 / 1e9, 3)},
+            "gpu_launches": 4 * args.steps,
         },
     }
     print(json.dumps(line), flush=True)
