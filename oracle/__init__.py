@@ -120,6 +120,14 @@ def _load():
         lib.orc_rate_build.restype = ctypes.c_int
         lib.orc_rate_gemv_f64.argtypes = [vp, vp, i64, i64, u64, ctypes.c_int, vp, ctypes.c_int, i64, vp, i64, vp]
         lib.orc_rate_gemv_f64.restype = ctypes.c_int
+        lib.orc_vr_offsets.argtypes = [i64, i64, vp, vp]
+        lib.orc_vr_offsets.restype = i64
+        lib.orc_vr_bucket.argtypes = [i64, u64, vp, i64, i64]
+        lib.orc_vr_bucket.restype = i64
+        lib.orc_vr_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, u64, vp, vp, vp]
+        lib.orc_vr_build.restype = ctypes.c_int
+        lib.orc_vr_gemv_f64.argtypes = [vp, vp, i64, i64, u64, vp, vp, ctypes.c_int, i64, vp, i64, vp]
+        lib.orc_vr_gemv_f64.restype = ctypes.c_int
         lib.orc_f32_to_f16_array.argtypes = [vp, vp, i64]
         lib.orc_f32_to_f16_array.restype = None
         lib.orc_f16_to_f32_array.argtypes = [vp, vp, i64]
@@ -380,6 +388,67 @@ def gemv_rate_f64(codes, scales, M, K, x, seed=0, slots=4, rows=None):
 def rate_bucket(K, seed, slots, i, j):
     """Global code index of weight (i, j) in a `slots`-slot format-1 sketch."""
     return int(_load().orc_rate_bucket(K, seed, slots, i, j))
+
+
+def _slots_u32(slots):
+    return np.ascontiguousarray(np.asarray(slots, dtype=np.uint32))
+
+
+def vr_offsets(M, K, slots):
+    """Per-row-block rates: (offsets, total code bytes); row block rb's codes
+    start at K * (slots[0] + ... + slots[rb - 1])."""
+    sl = _slots_u32(slots)
+    off = np.zeros(max(M // 64, 1), dtype=np.int64)
+    total = int(_load().orc_vr_offsets(M, K, _ptr(sl), _ptr(off)))
+    if total < 0:
+        raise ValueError("slot counts must be 2, 4 or 8")
+    return off[: M // 64], total
+
+
+def build_sketch_vr(W, importance=None, seed=0, slots=None):
+    """Format-1 sketch whose 64-row block rb has slots[rb] (2, 4 or 8) hash
+    slots per class, codes of the blocks back to back in matrix order.
+    Returns dict(status, codes, scales)."""
+    W, dt = _weights(W)
+    M, K = W.shape
+    sl = _slots_u32(slots)
+    if sl.shape != (M // 64,):
+        raise ValueError("one slot count per 64-row block")
+    ok = M % 64 == 0 and K % 256 == 0 and all(v in (2, 4, 8) for v in sl.tolist())
+    nb = int(K * int(sl.astype(np.int64).sum())) if ok else 0
+    imp = None if importance is None else np.ascontiguousarray(importance, dtype=np.float32)
+    codes = np.zeros(max(nb, 1), dtype=np.int8)
+    scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
+    st = _load().orc_vr_build(_ptr(W), dt, M, K, K, _ptr(imp), seed, _ptr(sl), _ptr(codes), _ptr(scales))
+    return {"status": st, "codes": codes[:nb], "scales": scales[: M // 64]}
+
+
+def gemv_vr_f64(codes, scales, M, K, x, seed=0, slots=None, rows=None):
+    """y = W_hat x^T in float64 for a per-row-block-rate sketch."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    sl = _slots_u32(slots)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    xdt = F32 if x.dtype == np.float32 else BF16 if x.dtype == np.uint16 else None
+    if xdt is None:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    batch = x.shape[0]
+    r = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    nr = M if r is None else len(r)
+    y = np.zeros((batch, nr), dtype=np.float64)
+    st = _load().orc_vr_gemv_f64(_ptr(codes), _ptr(scales), M, K, seed, _ptr(sl), _ptr(x), xdt, batch,
+                                 _ptr(r), 0 if r is None else len(r), _ptr(y))
+    if st:
+        raise ValueError("orc_vr_gemv_f64 status %d" % st)
+    return y
+
+
+def vr_bucket(K, seed, slots, i, j):
+    """Global code index of weight (i, j) in a per-row-block-rate sketch."""
+    sl = _slots_u32(slots)
+    return int(_load().orc_vr_bucket(K, seed, _ptr(sl), i, j))
 
 
 # bits per weight of each slot count (8-bit codes)

@@ -857,6 +857,59 @@ int64_t orc_rate_bucket(int64_t K, uint64_t seed, int slots, int64_t i, int64_t 
   return rb * slots * K + 256 * slots * tc + b;
 }
 
+/* Selection, scale and codes of row block rb at `slots` slots per class: the
+ * block's slots*K codes go to out[0 .. slots*K), its scale to *scale16.  The
+ * caller has checked the shape, the dtype and the importance. */
+static int rate_build_block(const void* W, int dtype, int64_t K, int64_t ldw, const float* imp, uint64_t seed,
+                            int slots, int64_t rb, float* bestkey, int64_t* bestidx, int8_t* out,
+                            uint16_t* scale16) {
+  int status = ORC_OK;
+  int64_t per_block = slots * K;
+  for (int64_t b = 0; b < per_block; ++b) { bestkey[b] = -1.0f; bestidx[b] = -1; }
+  for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
+    int64_t i = rb * ROWS_PER_BLOCK + r;
+    for (int64_t j = 0; j < K; ++j) {
+      float w = load_elem(W, dtype, i * ldw + j);
+      if (!isfinite(w)) status = ORC_ERR_NONFINITE;
+      float k = fabsf(w) * (imp ? imp[j] : 1.0f);
+      int64_t b = orc_rate_bucket(K, seed, slots, i, j) - rb * per_block;
+      if (k > bestkey[b] || bestidx[b] < 0) { bestkey[b] = k; bestidx[b] = i * K + j; }
+    }
+  }
+  float mx = 0.0f;
+  for (int64_t b = 0; b < per_block; ++b) {
+    float v = bestidx[b] >= 0 ? load_elem(W, dtype, (bestidx[b] / K) * ldw + bestidx[b] % K) : 0.0f;
+    bestkey[b] = v;  /* reuse as the kept value */
+    if (fabsf(v) > mx) mx = fabsf(v);
+  }
+  uint16_t s16 = orc_f32_to_f16(mx / 127.0f);
+  if ((s16 & 0x7c00u) == 0x7c00u) status = status ? status : ORC_ERR_SCALE_OVERFLOW;
+  *scale16 = s16;
+  float s = orc_f16_to_f32(s16);
+  for (int64_t b = 0; b < per_block; ++b) {
+    int code = 0;
+    if (s != 0.0f) {
+      float q = nearbyintf(bestkey[b] / s);
+      if (q > 127.0f) q = 127.0f;
+      if (q < -127.0f) q = -127.0f;
+      code = isnan(q) ? 0 : (int)q;
+    }
+    out[b] = (int8_t)code;
+  }
+  return status;
+}
+
+/* Argument checks shared by the rate builds; ORC_OK when the build may go on. */
+static int rate_check_imp(int64_t K, const float* imp) {
+  if (imp) {
+    for (int64_t j = 0; j < K; ++j) {
+      uint32_t u = bits_from_f32(imp[j]);
+      if ((u >> 31) || !isfinite(imp[j])) return ORC_ERR_IMPORTANCE;
+    }
+  }
+  return ORC_OK;
+}
+
 int orc_rate_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw, const float* imp,
                    uint64_t seed, int slots, int8_t* codes, uint16_t* scales) {
   int st = check_shape(M, K);
@@ -870,49 +923,17 @@ int orc_rate_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw, 
     return ORC_OK;
   }
   if (!W || ldw < K) return ORC_ERR_NULL;
-  if (imp) {
-    for (int64_t j = 0; j < K; ++j) {
-      uint32_t u = bits_from_f32(imp[j]);
-      if ((u >> 31) || !isfinite(imp[j])) return ORC_ERR_IMPORTANCE;
-    }
-  }
+  st = rate_check_imp(K, imp);
+  if (st) return st;
   int64_t per_block = slots * K;
   float* bestkey = (float*)malloc(sizeof(float) * (size_t)per_block);
   int64_t* bestidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)per_block);
   if (!bestkey || !bestidx) { free(bestkey); free(bestidx); return ORC_ERR_NULL; }
   int status = ORC_OK;
   for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
-    for (int64_t b = 0; b < per_block; ++b) { bestkey[b] = -1.0f; bestidx[b] = -1; }
-    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) {
-      int64_t i = rb * ROWS_PER_BLOCK + r;
-      for (int64_t j = 0; j < K; ++j) {
-        float w = load_elem(W, dtype, i * ldw + j);
-        if (!isfinite(w)) status = ORC_ERR_NONFINITE;
-        float k = fabsf(w) * (imp ? imp[j] : 1.0f);
-        int64_t b = orc_rate_bucket(K, seed, slots, i, j) - rb * per_block;
-        if (k > bestkey[b] || bestidx[b] < 0) { bestkey[b] = k; bestidx[b] = i * K + j; }
-      }
-    }
-    float mx = 0.0f;
-    for (int64_t b = 0; b < per_block; ++b) {
-      float v = bestidx[b] >= 0 ? load_elem(W, dtype, (bestidx[b] / K) * ldw + bestidx[b] % K) : 0.0f;
-      bestkey[b] = v;  /* reuse as the kept value */
-      if (fabsf(v) > mx) mx = fabsf(v);
-    }
-    uint16_t s16 = orc_f32_to_f16(mx / 127.0f);
-    if ((s16 & 0x7c00u) == 0x7c00u) status = status ? status : ORC_ERR_SCALE_OVERFLOW;
-    scales[rb] = s16;
-    float s = orc_f16_to_f32(s16);
-    for (int64_t b = 0; b < per_block; ++b) {
-      int code = 0;
-      if (s != 0.0f) {
-        float q = nearbyintf(bestkey[b] / s);
-        if (q > 127.0f) q = 127.0f;
-        if (q < -127.0f) q = -127.0f;
-        code = isnan(q) ? 0 : (int)q;
-      }
-      codes[rb * per_block + b] = (int8_t)code;
-    }
+    int bs = rate_build_block(W, dtype, K, ldw, imp, seed, slots, rb, bestkey, bestidx, codes + rb * per_block,
+                              &scales[rb]);
+    if (bs == ORC_ERR_NONFINITE || (bs && !status)) status = bs;
   }
   free(bestkey); free(bestidx);
   return status;
@@ -939,6 +960,96 @@ int orc_rate_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, in
     if (i < 0 || i >= M) { free(wrow); return ORC_ERR_SHAPE; }
     float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
     for (int64_t j = 0; j < K; ++j) wrow[j] = (double)((float)codes[orc_rate_bucket(K, seed, slots, i, j)] * s);
+    for (int64_t t = 0; t < batch; ++t) {
+      double acc = 0.0;
+      for (int64_t j = 0; j < K; ++j) acc += wrow[j] * (double)load_elem(x, xdtype, t * K + j);
+      y[t * nr + q] = acc;
+    }
+  }
+  free(wrow);
+  return ORC_OK;
+}
+
+/* ================================================================ per-row-block rates
+ *
+ * Importance-aware space allocation at row-block granularity (Metodologia §2:
+ * rows of higher importance E[a^2] receive larger sketch spaces).  Reading:
+ * each 64-row block rb carries its own slot count S_rb in {2, 4, 8}; its codes
+ * are the S_rb-slot format-1 codes of that block (same hash tile ids rb*T + tc),
+ * stored at byte offset off_rb = K * (S_0 + ... + S_{rb-1}) -- the row blocks in
+ * matrix order, each block's slots*K codes contiguous.  Total code bytes
+ * K * sum(S_rb). */
+
+/* off[rb] for every row block; returns the total code bytes, -1 on a bad slot count. */
+int64_t orc_vr_offsets(int64_t M, int64_t K, const uint32_t* slots, int64_t* off) {
+  int64_t acc = 0;
+  for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
+    if (slots[rb] != 2 && slots[rb] != 4 && slots[rb] != 8) return -1;
+    if (off) off[rb] = acc;
+    acc += (int64_t)slots[rb] * K;
+  }
+  return acc;
+}
+
+int64_t orc_vr_bucket(int64_t K, uint64_t seed, const uint32_t* slots, int64_t i, int64_t j) {
+  int64_t rb = i / ROWS_PER_BLOCK, off = 0;
+  for (int64_t q = 0; q < rb; ++q) off += (int64_t)slots[q] * K;
+  int S = (int)slots[rb];
+  return off + (orc_rate_bucket(K, seed, S, i, j) - rb * S * K);
+}
+
+int orc_vr_build(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw, const float* imp, uint64_t seed,
+                 const uint32_t* slots, int8_t* codes, uint16_t* scales) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
+  if (M == 0) return ORC_OK;
+  if (!slots || !codes || !scales) return ORC_ERR_NULL;
+  if (orc_vr_offsets(M, K, slots, NULL) < 0) return ORC_ERR_SHAPE;
+  if (K == 0) {
+    for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) scales[rb] = 0;
+    return ORC_OK;
+  }
+  if (!W || ldw < K) return ORC_ERR_NULL;
+  st = rate_check_imp(K, imp);
+  if (st) return st;
+  float* bestkey = (float*)malloc(sizeof(float) * (size_t)(8 * K));
+  int64_t* bestidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)(8 * K));
+  if (!bestkey || !bestidx) { free(bestkey); free(bestidx); return ORC_ERR_NULL; }
+  int status = ORC_OK;
+  int64_t off = 0;
+  for (int64_t rb = 0; rb < M / ROWS_PER_BLOCK; ++rb) {
+    int S = (int)slots[rb];
+    int bs = rate_build_block(W, dtype, K, ldw, imp, seed, S, rb, bestkey, bestidx, codes + off, &scales[rb]);
+    if (bs == ORC_ERR_NONFINITE || (bs && !status)) status = bs;
+    off += (int64_t)S * K;
+  }
+  free(bestkey); free(bestidx);
+  return status;
+}
+
+int orc_vr_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
+                    const uint32_t* slots, const void* x, int xdtype, int64_t batch, const int64_t* rows,
+                    int64_t nrows, double* y) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (xdtype != 0 && xdtype != 1) return ORC_ERR_DTYPE;
+  int64_t nr = rows ? nrows : M;
+  if (nr == 0 || batch <= 0) return ORC_OK;
+  if (!y || !slots) return ORC_ERR_NULL;
+  if (orc_vr_offsets(M, K, slots, NULL) < 0) return ORC_ERR_SHAPE;
+  if (K == 0) {
+    for (int64_t q = 0; q < batch * nr; ++q) y[q] = 0.0;
+    return ORC_OK;
+  }
+  if (!codes || !scales || !x) return ORC_ERR_NULL;
+  double* wrow = (double*)malloc(sizeof(double) * (size_t)K);
+  if (!wrow) return ORC_ERR_NULL;
+  for (int64_t q = 0; q < nr; ++q) {
+    int64_t i = rows ? rows[q] : q;
+    if (i < 0 || i >= M) { free(wrow); return ORC_ERR_SHAPE; }
+    float s = orc_f16_to_f32(scales[i / ROWS_PER_BLOCK]);
+    for (int64_t j = 0; j < K; ++j) wrow[j] = (double)((float)codes[orc_vr_bucket(K, seed, slots, i, j)] * s);
     for (int64_t t = 0; t < batch; ++t) {
       double acc = 0.0;
       for (int64_t j = 0; j < K; ++j) acc += wrow[j] * (double)load_elem(x, xdtype, t * K + j);

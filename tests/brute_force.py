@@ -251,3 +251,51 @@ def build_q4(W: np.ndarray, importance=None, seed: int = 0):
     u = (nib & 15).astype(np.uint8)
     packed = (u[0::2] | (u[1::2] << 4)).astype(np.uint8).view(np.int8)
     return packed, scales, winner
+
+
+def bucket_of_vr(K: int, seed: int, slots, i: int, j: int) -> int:
+    """Per-row-block rates: row block rb has slots[rb] hash slots per class
+    (slot = (slots[rb] * h) >> 32) and its codes start after those of the
+    blocks above it (K * slots[q] bytes each)."""
+    rb, r = divmod(i, 64)
+    tc, c = divmod(j, 256)
+    S = int(slots[rb])
+    z = splitmix64_output(seed, rb * (K // 256) + tc + 1)
+    A = (z & 0xFFFFFFFF) | 1
+    C = z >> 32
+    o = c // 8
+    h = (A * (32 * r + o) + C) & 0xFFFFFFFF
+    b = (((S * h) >> 32) * 32 + (o + r) % 32) * 8 + c % 8
+    start = sum(int(s) * K for s in slots[:rb])
+    return start + 256 * S * tc + b
+
+
+def build_vr(W: np.ndarray, importance=None, seed: int = 0, slots=None):
+    """Returns (codes int8, scales uint16) of the per-row-block-rate sketch."""
+    Wf = to_f32(np.ascontiguousarray(W))
+    M, K = Wf.shape
+    imp = np.ones(K, np.float32) if importance is None else np.asarray(importance, np.float32)
+    nb = K * sum(int(s) for s in slots)
+    members = [[] for _ in range(nb)]
+    for i in range(M):
+        for j in range(K):
+            members[bucket_of_vr(K, seed, slots, i, j)].append(i * K + j)
+    flat = Wf.reshape(-1)
+    value = np.zeros(nb, np.float32)
+    for b, mem in enumerate(members):
+        if mem:
+            best = sorted((-float(np.float32(np.float32(abs(flat[m])) * imp[m % K])), m) for m in mem)[0][1]
+            value[b] = flat[best]
+    codes = np.zeros(nb, np.int8)
+    scales = np.zeros(M // 64, np.uint16)
+    start = 0
+    for rb in range(M // 64):
+        n = int(slots[rb]) * K
+        v = value[start:start + n]
+        s16 = np.float16(np.float32(np.max(np.abs(v))) / np.float32(127.0))
+        scales[rb] = s16.view(np.uint16)
+        s = np.float32(s16)
+        if s != 0:
+            codes[start:start + n] = np.clip(np.rint(v / s), -127, 127).astype(np.int8)
+        start += n
+    return codes, scales
