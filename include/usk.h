@@ -76,6 +76,14 @@
  *   1 bit/weight), codes[(rb * K/256 + tc) * 256 * slots + b]; everything else
  *   as format 1.  usk_plan_slots chooses slot counts per layer from importance.
  *
+ * PER-ROW-BLOCK RATES (Metodologia §2 at row granularity: rows of higher
+ *   importance get larger spaces): a format-1 sketch whose 64-row block rb has
+ *   its own slot count S_rb in {2, 4, 8}.  Block rb's codes are exactly those
+ *   of row block rb of the uniform S_rb sketch (same hash tiles rb*K/256 + tc),
+ *   stored from byte off_rb = K * (S_0 + ... + S_{rb-1}) on: codes[off_rb +
+ *   256*S_rb*tc + b].  Total code bytes K * sum(S_rb).  The per-block table
+ *   lives in a usk_rate_map (usk_rate_map_plan fills it from the slot counts).
+ *
  * FORMAT 4 (format 1 with 4-bit codes; Resultados: 0.5 bit/weight with 4-bit
  * quantisation): 8 weights per bucket, 2048 buckets per tile, same storage size.
  *   Hash as format 1 with 8 slots: slot = h >> 29, b = (slot*32 + class)*8 + c % 8.
@@ -147,8 +155,27 @@ typedef enum {
 #define USK_FLAG_BAD_IMPORTANCE (1u << 1)
 #define USK_FLAG_SCALE_OVERFLOW (1u << 2)
 #define USK_FLAG_TIMEOUT (1u << 3)
+#define USK_FLAG_RATE_MAP (1u << 4) /* a rate-map entry out of range: that row block was skipped */
 
 typedef enum { USK_F32 = 0, USK_BF16 = 1 } usk_dtype;
+
+/* Per-row-block rate table of a format-1 sketch (see PER-ROW-BLOCK RATES).
+ * offset and order are DEVICE arrays of M/64 entries owned by the caller:
+ *   offset[rb]  byte offset of row block rb's codes (K * slots of the blocks above);
+ *   order       the row blocks at 2 slots, then those at 4, then those at 8,
+ *               each group in increasing row-block order (the kernels take one
+ *               group per launch);
+ *   count[g]    host value: row blocks at 2 (g = 0), 4 (g = 1) and 8 (g = 2) slots;
+ *   code_bytes  host value: K * sum of the slots (the codes array's size).
+ * The library checks the counts against M on the host; on the device an order
+ * entry outside [0, M/64) or an offset whose block would end past code_bytes
+ * skips that row block (its outputs are not written) and sets USK_FLAG_RATE_MAP. */
+typedef struct {
+  const int64_t* offset;
+  const int32_t* order;
+  int64_t count[3];
+  int64_t code_bytes;
+} usk_rate_map;
 
 /* Build parameters.  version: USK_FORMAT_MAXKEY, USK_FORMAT_ABSMAXMIN,
  * USK_FORMAT_COLSHARED or USK_FORMAT_Q4; flags must be 0; depth = hash rows: 0
@@ -161,6 +188,7 @@ typedef struct {
   uint64_t seed;
   uint32_t depth;
   uint32_t slots;  /* hash slots per class; 0 = the format's default (see RATES) */
+  const usk_rate_map* rates; /* per-row-block rates (format 1, slots 0, depth <= 1); NULL = uniform */
 } usk_params;
 
 /* A built sketch (device pointers, caller-owned).  version / depth as built
@@ -174,6 +202,7 @@ typedef struct {
   uint32_t depth;
   uint32_t slots;          /* as built (0 = the format's default) */
   uint32_t pad;
+  const usk_rate_map* rates; /* as built; NULL = one rate for the whole sketch */
 } usk_sketch;
 
 /* Storage of a sketch: code_bytes = M*K/16, scale_bytes = 2*M/64.
@@ -202,6 +231,15 @@ USK_API usk_status usk_sizes_ex(int64_t M, int64_t K, uint32_t version, uint32_t
 USK_API usk_status usk_plan_slots(int64_t n, const int64_t* weights, const double* importance, double budget_bits,
                                   uint32_t* slots);
 
+/* Rate table of a per-row-block-rate sketch, on the host: from slots[M/64]
+ * (each 2, 4 or 8) writes offset[M/64] (byte offsets, matrix order),
+ * order[M/64] (row blocks grouped by slot count 2, 4, 8, increasing within a
+ * group), count[3] and *code_bytes = K * sum(slots).  All HOST arrays; the
+ * caller copies offset and order to the device for a usk_rate_map.  Host only.
+ * Errors: USK_ERR_SHAPE, USK_ERR_NULL, USK_ERR_PARAMS (a slot count). */
+USK_API usk_status usk_rate_map_plan(int64_t M, int64_t K, const uint32_t* slots, int64_t* offset, int32_t* order,
+                                     int64_t* count, int64_t* code_bytes);
+
 /* Build the sketch of W (Metodologia §1 and §4: fused select-and-update).
  *   W          [M, K] row-major, row stride ldw elements (ldw >= K); fp32 or
  *              bf16 per wdtype.  W and every row start must be 16-byte aligned
@@ -210,7 +248,10 @@ USK_API usk_status usk_plan_slots(int64_t n, const int64_t* weights, const doubl
  *              be finite with the sign bit clear (else USK_FLAG_BAD_IMPORTANCE).
  *              Formats 2 and 3 take no importance: non-NULL is USK_ERR_PARAMS.
  *   params     format, depth and seed of the hash.
- *   codes      [M*K/16] int8 output, 16-byte aligned.   scales [M/64] output.
+ *   codes      int8 output, 16-byte aligned: M*K/16 bytes (usk_sizes_ex for
+ *              other formats and slot counts; rate-map code_bytes with
+ *              params->rates).   scales [M/64] output.
+ *   params->rates  per-row-block rates: one launch per slot group present.
  *   d_status   optional device word for USK_FLAG_* bits.
  * M == 0 is a no-op; K == 0 writes zero scales.  Codes and scales are
  * bit-identical for any launch geometry. */

@@ -32,6 +32,7 @@ FLAG_NONFINITE_W = 1 << 0
 FLAG_BAD_IMPORTANCE = 1 << 1
 FLAG_SCALE_OVERFLOW = 1 << 2
 FLAG_TIMEOUT = 1 << 3
+FLAG_RATE_MAP = 1 << 4
 
 STATUS_NAMES = {
     0: "USK_OK", 1: "USK_ERR_NULL", 2: "USK_ERR_SHAPE", 3: "USK_ERR_DTYPE", 4: "USK_ERR_BATCH",
@@ -46,21 +47,26 @@ class UskError(RuntimeError):
         super().__init__("%s: %s (%s)" % (what, STATUS_NAMES.get(status, status), usk_status_str(status)))
 
 
+class UskRateMapC(ctypes.Structure):
+    _fields_ = [("offset", ctypes.c_void_p), ("order", ctypes.c_void_p), ("count", ctypes.c_int64 * 3),
+                ("code_bytes", ctypes.c_int64)]
+
+
 class UskParams(ctypes.Structure):
     _fields_ = [("version", ctypes.c_uint32), ("flags", ctypes.c_uint32), ("seed", ctypes.c_uint64),
-                ("depth", ctypes.c_uint32), ("slots", ctypes.c_uint32)]
+                ("depth", ctypes.c_uint32), ("slots", ctypes.c_uint32), ("rates", ctypes.POINTER(UskRateMapC))]
 
 
 class UskSketchC(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int64), ("seed", ctypes.c_uint64),
                 ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("version", ctypes.c_uint32), ("depth", ctypes.c_uint32), ("slots", ctypes.c_uint32),
-                ("pad", ctypes.c_uint32)]
+                ("pad", ctypes.c_uint32), ("rates", ctypes.POINTER(UskRateMapC))]
 
 
 _lib = None
 
-EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_build", "usk_gemv", "usk_gemv_ex", "usk_gemm", "usk_status_str",
+EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_rate_map_plan", "usk_build", "usk_gemv", "usk_gemv_ex", "usk_gemm", "usk_status_str",
             "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_set_gemv_rows",
             "usk_debug_inject_timeout"]
 GEMV_PDL = 1
@@ -84,6 +90,9 @@ def load_library(path: str = LIB_PATH):
     lib.usk_plan_slots.argtypes = [i64, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_double),
                                    ctypes.c_double, ctypes.POINTER(ctypes.c_uint32)]
     lib.usk_plan_slots.restype = ctypes.c_int
+    lib.usk_rate_map_plan.argtypes = [i64, i64, u32p, ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int32),
+                                      ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]
+    lib.usk_rate_map_plan.restype = ctypes.c_int
     lib.usk_build.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, ctypes.POINTER(UskParams), vp, vp, vp, vp]
     lib.usk_build.restype = ctypes.c_int
     lib.usk_gemv.argtypes = [ctypes.POINTER(UskSketchC), vp, ctypes.c_int, i64, vp, vp, vp]
@@ -170,6 +179,49 @@ def usk_sizes(M: int, K: int):
     return c.value, s.value
 
 
+def usk_rate_map_plan(M: int, K: int, slots):
+    """Host rate table of a per-row-block-rate sketch: (offset list, order list,
+    (count2, count4, count8), code_bytes) from one slot count per 64-row block."""
+    n = M // 64 if M > 0 else 0
+    sl = (ctypes.c_uint32 * max(n, 1))(*[int(v) for v in slots])
+    off = (ctypes.c_int64 * max(n, 1))()
+    order = (ctypes.c_int32 * max(n, 1))()
+    cnt = (ctypes.c_int64 * 3)()
+    total = ctypes.c_int64()
+    if len(slots) != n:
+        raise ValueError("one slot count per 64-row block")
+    _check(load_library().usk_rate_map_plan(M, K, sl, off, order, cnt, ctypes.byref(total)), "usk_rate_map_plan")
+    return [int(off[i]) for i in range(n)], [int(order[i]) for i in range(n)], tuple(int(c) for c in cnt), total.value
+
+
+@dataclass
+class RateMap:
+    """Per-row-block rates of a format-1 sketch: slot counts (2, 4 or 8) per
+    64-row block and the device tables the kernels read (byte offset of each
+    block's codes; row blocks grouped by slot count)."""
+    slots: list
+    offset: torch.Tensor  # int64 [M/64], device
+    order: torch.Tensor   # int32 [M/64], device
+    count: tuple
+    code_bytes: int
+
+    def as_c(self) -> UskRateMapC:
+        c = UskRateMapC(self.offset.data_ptr() if self.offset.numel() else None,
+                        self.order.data_ptr() if self.order.numel() else None)
+        for g in range(3):
+            c.count[g] = int(self.count[g])
+        c.code_bytes = int(self.code_bytes)
+        return c
+
+
+def usk_rate_map(M: int, K: int, slots, device="cuda") -> RateMap:
+    """RateMap for an M x K sketch: the library plans the table on the host,
+    torch copies it to the device."""
+    off, order, count, total = usk_rate_map_plan(M, K, slots)
+    return RateMap([int(v) for v in slots], torch.tensor(off, dtype=torch.int64, device=device),
+                   torch.tensor(order, dtype=torch.int32, device=device), count, total)
+
+
 @dataclass
 class Sketch:
     """A built sketch: int8 codes [M*K/16] and binary16 scales [M/64] on the GPU,
@@ -182,29 +234,38 @@ class Sketch:
     version: int = FORMAT_MAXKEY
     depth: int = 1
     slots: int = 0  # hash slots per class as built (0 = the format's default)
+    rates: RateMap | None = None  # per-row-block rates (format 1)
 
     def as_c(self) -> UskSketchC:
-        return UskSketchC(self.M, self.K, self.seed & (2**64 - 1), self.codes.data_ptr() if self.codes.numel() else None,
-                          self.scales.data_ptr() if self.scales.numel() else None, self.version, self.depth,
-                          self.slots, 0)
+        c = UskSketchC(self.M, self.K, self.seed & (2**64 - 1), self.codes.data_ptr() if self.codes.numel() else None,
+                       self.scales.data_ptr() if self.scales.numel() else None, self.version, self.depth,
+                       self.slots, 0)
+        if self.rates is not None:
+            c._rates = self.rates.as_c()  # kept alive with the struct
+            c.rates = ctypes.pointer(c._rates)
+        return c
 
 
 def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int = 0,
               codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
               status: torch.Tensor | None = None, stream=None, version: int = FORMAT_MAXKEY,
-              depth: int = 1, slots: int = 0) -> Sketch:
+              depth: int = 1, slots: int = 0, rates: RateMap | None = None) -> Sketch:
     """Sketch of W [M, K] (bf16 or fp32, CUDA).  Outputs are allocated with torch
     when not given.  `status` is an optional int32 CUDA tensor of 1 element into
     which device-detected USK_FLAG_* bits are OR-ed.  version=FORMAT_ABSMAXMIN
     builds the multi-row AbsMaxMin sketch with `depth` (1, 2 or 4) hash rows,
     version=FORMAT_COLSHARED the column-shared projection sketch (no importance
     for either), version=FORMAT_Q4 the format-1 sketch with 4-bit codes.  slots
-    (format 1): 2, 4 or 8 hash slots per class, 0.25, 0.5 or 1 bit/weight."""
+    (format 1): 2, 4 or 8 hash slots per class, 0.25, 0.5 or 1 bit/weight.
+    rates (format 1, slots 0): a RateMap giving every 64-row block its own slot
+    count (usk_rate_map)."""
     _need_cuda(W, importance, codes, scales, status)
     if W.dim() != 2 or W.stride(1) != 1:
         raise ValueError("W must be a 2-D row-major tensor")
     M, K = W.shape
     nb = M * K * (slots if (version == FORMAT_MAXKEY and slots in (2, 8)) else 4) // 64
+    if rates is not None:
+        nb = int(rates.code_bytes)
     if codes is None:
         codes = torch.empty(max(nb, 1), dtype=torch.int8, device=W.device)[:nb]
     if scales is None:
@@ -212,11 +273,14 @@ def usk_build(W: torch.Tensor, importance: torch.Tensor | None = None, seed: int
     if importance is not None and (importance.dtype != torch.float32 or not importance.is_contiguous()):
         raise TypeError("importance must be a contiguous float32 tensor")
     p = UskParams(version, 0, seed & (2**64 - 1), depth, slots)
+    if rates is not None:
+        rc = rates.as_c()
+        p.rates = ctypes.pointer(rc)
     st = load_library().usk_build(_ptr(W), _dtype_code(W), M, K, W.stride(0), _ptr(importance), ctypes.byref(p),
                                   _ptr(codes) if nb else None, _ptr(scales) if M // 64 else None,
                                   _ptr(status), _stream(stream))
     _check(st, "usk_build")
-    return Sketch(M, K, seed, codes, scales, version, depth, slots)
+    return Sketch(M, K, seed, codes, scales, version, depth, slots, rates)
 
 
 def usk_gemv(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,

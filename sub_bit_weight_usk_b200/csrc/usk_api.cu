@@ -1,6 +1,7 @@
 // usk_api.cu -- the C ABI of libusk (declared in include/usk.h): argument
-// validation, then one kernel launch per call.  No allocation, no global state
-// beyond CUDA's cached kernel attributes.
+// validation, then one kernel launch per call (one per slot group for a sketch
+// with per-row-block rates).  No allocation, no global state beyond CUDA's
+// cached kernel attributes.
 #include <algorithm>
 #include <cstdint>
 #include <vector>
@@ -8,11 +9,13 @@
 #include <cuda_runtime.h>
 
 #include "usk.h"
+#include "usk_common.cuh"
 
 namespace usk {
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override, int inject, int var);
+                         cudaStream_t stream, int cluster_override, int inject, int var, const RbMap& map,
+                         int64_t nrb);
 cudaError_t launch_build_amm(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed, int depth,
                              int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
                              int cluster_override, int inject);
@@ -24,10 +27,11 @@ cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t 
                            cudaStream_t stream, int tpb_override, int rows_override, int inject);
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var);
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var,
+                        const RbMap& map, int64_t nrb);
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth, int var);
+                        int depth, int var, const RbMap& map, int64_t nrb);
 bool gemm_supported(int64_t K, int batch, int depth, int var);
 }  // namespace usk
 
@@ -70,12 +74,48 @@ size_t layout_code_bytes(int64_t M, int64_t K, int layout) {
   return layout == 2 ? n / 32 : (layout == 3 ? n / 8 : n / 16);
 }
 
+// A rate map for an M x K format-1 sketch: counts that add up to the row
+// blocks, code_bytes = K * (2 c0 + 4 c1 + 8 c2), aligned device arrays.
+usk_status check_rate_map(const usk_rate_map* m, int64_t M, int64_t K) {
+  const int64_t RB = M / USK_ROWS_PER_BLOCK;
+  if (m->count[0] < 0 || m->count[1] < 0 || m->count[2] < 0) return USK_ERR_PARAMS;
+  if (m->count[0] + m->count[1] + m->count[2] != RB) return USK_ERR_PARAMS;
+  if (m->code_bytes != K * (2 * m->count[0] + 4 * m->count[1] + 8 * m->count[2])) return USK_ERR_PARAMS;
+  if (RB > 0 && (!m->offset || !m->order)) return USK_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(m->offset) & 7u) != 0 || (reinterpret_cast<uintptr_t>(m->order) & 3u) != 0)
+    return USK_ERR_ALIGN;
+  return USK_OK;
+}
+
+// Launch groups of a sketch: one per slot count present (rate map), else one
+// over every row block.  fn(layout, RbMap, row blocks) returns a cudaError_t.
+template <class Fn>
+cudaError_t for_each_group(const usk_rate_map* rm, int64_t M, int layout, Fn&& fn) {
+  const int64_t RB = M / USK_ROWS_PER_BLOCK;
+  if (!rm) return fn(layout, usk::RbMap{nullptr, nullptr, 0, RB}, RB);
+  static const int kLayouts[3] = {2, 0, 3};  // 2, 4 and 8 slots
+  int64_t start = 0;
+  for (int g = 0; g < 3; ++g) {
+    if (rm->count[g] > 0) {
+      cudaError_t e = fn(kLayouts[g], usk::RbMap{rm->order + start, rm->offset, rm->code_bytes, RB}, rm->count[g]);
+      if (e != cudaSuccess) return e;
+    }
+    start += rm->count[g];
+  }
+  return cudaSuccess;
+}
+
 usk_status check_sketch(const usk_sketch* s) {
   if (!s) return USK_ERR_NULL;
   if (format_depth(s->version, s->depth) == 0) return USK_ERR_PARAMS;
   if (layout_of(s->version, s->slots) < 0) return USK_ERR_PARAMS;
   usk_status st = check_shape(s->M, s->K);
   if (st != USK_OK) return st;
+  if (s->rates) {
+    if ((s->version != 0 && s->version != USK_FORMAT_MAXKEY) || s->slots != 0) return USK_ERR_PARAMS;
+    st = check_rate_map(s->rates, s->M, s->K);
+    if (st != USK_OK) return st;
+  }
   if (s->M > 0 && s->K > 0) {
     if (!s->codes || !s->scales) return USK_ERR_NULL;
     if (!aligned16(s->codes)) return USK_ERR_ALIGN;
@@ -192,6 +232,33 @@ USK_API usk_status usk_plan_slots(int64_t n, const int64_t* weights, const doubl
   return USK_OK;
 }
 
+USK_API usk_status usk_rate_map_plan(int64_t M, int64_t K, const uint32_t* slots, int64_t* offset, int32_t* order,
+                                     int64_t* count, int64_t* code_bytes) {
+  usk_status st = check_shape(M, K);
+  if (st != USK_OK) return st;
+  if (!count || !code_bytes) return USK_ERR_NULL;
+  const int64_t RB = M / USK_ROWS_PER_BLOCK;
+  if (RB > 0 && (!slots || !offset || !order)) return USK_ERR_NULL;
+  for (int64_t rb = 0; rb < RB; ++rb)
+    if (slots[rb] != 2 && slots[rb] != 4 && slots[rb] != 8) return USK_ERR_PARAMS;
+  int64_t acc = 0, n = 0;
+  count[0] = count[1] = count[2] = 0;
+  for (int64_t rb = 0; rb < RB; ++rb) {
+    offset[rb] = acc;
+    acc += K * static_cast<int64_t>(slots[rb]);
+  }
+  for (int g = 0; g < 3; ++g) {
+    const uint32_t want = 2u << g;
+    for (int64_t rb = 0; rb < RB; ++rb)
+      if (slots[rb] == want) {
+        order[n++] = static_cast<int32_t>(rb);
+        ++count[g];
+      }
+  }
+  *code_bytes = acc;
+  return USK_OK;
+}
+
 USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t K, int64_t ldw,
                      const float* importance, const usk_params* params, int8_t* codes,
                      uint16_t* scales, uint32_t* d_status, void* stream) {
@@ -209,6 +276,12 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   if (layout < 0) return USK_ERR_PARAMS;
   const bool amm = params->version == USK_FORMAT_ABSMAXMIN, cs = params->version == USK_FORMAT_COLSHARED;
   if ((amm || cs) && importance) return USK_ERR_PARAMS;
+  const usk_rate_map* rm = params->rates;
+  if (rm) {
+    if (params->version != USK_FORMAT_MAXKEY || params->slots != 0) return USK_ERR_PARAMS;
+    st = check_rate_map(rm, M, K);
+    if (st != USK_OK) return st;
+  }
   if (M == 0) return USK_OK;
   if (!scales) return USK_ERR_NULL;
   if ((reinterpret_cast<uintptr_t>(scales) & 1u) != 0) return USK_ERR_ALIGN;
@@ -227,8 +300,10 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
     e = usk::launch_build_amm(W, wdtype == USK_BF16, M, K, ldw, params->seed, depth, codes, scales, d_status, s,
                               g_build_cluster, g_inject == 1);
   else
-    e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes, scales, d_status, s,
-                          g_build_cluster, g_inject == 1, layout);
+    e = for_each_group(rm, M, layout, [&](int lay, const usk::RbMap& map, int64_t nrb) {
+      return usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes, scales, d_status,
+                               s, g_build_cluster, g_inject == 1, lay, map, nrb);
+    });
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -256,11 +331,14 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
     if (e != cudaSuccess) return USK_ERR_CUDA;
     return from_cuda(cudaGetLastError());
   }
-  cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
-                                   xdtype == USK_F32, static_cast<int>(batch), y, d_status,
-                                   (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows,
-                                   g_inject == 3, format_depth(sketch->version, sketch->depth),
-                                   layout_of(sketch->version, sketch->slots));
+  cudaError_t e = for_each_group(
+      sketch->rates, sketch->M, layout_of(sketch->version, sketch->slots),
+      [&](int lay, const usk::RbMap& map, int64_t nrb) {
+        return usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
+                                xdtype == USK_F32, static_cast<int>(batch), y, d_status, (flags & USK_GEMV_PDL) != 0,
+                                g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows, g_inject == 3,
+                                format_depth(sketch->version, sketch->depth), lay, map, nrb);
+      });
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -281,6 +359,8 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   const int depth = format_depth(sketch->version, sketch->depth);
   const int layout = layout_of(sketch->version, sketch->slots);
   if (!usk::gemm_supported(sketch->K, static_cast<int>(batch), depth, layout)) return USK_ERR_SHAPE;
+  if (sketch->rates && !usk::gemm_supported(sketch->K, static_cast<int>(batch), 1, 3))
+    return USK_ERR_SHAPE;  // the 8-slot group stages the most codes
   if (sketch->M == 0) return USK_OK;
   if (!y) return USK_ERR_NULL;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -288,8 +368,10 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
     return from_cuda(cudaMemsetAsync(y, 0, sizeof(float) * static_cast<size_t>(batch * sketch->M), s));
   if (!x_bf16) return USK_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(y)) return USK_ERR_ALIGN;
-  cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
-                                   static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, layout);
+  cudaError_t e = for_each_group(sketch->rates, sketch->M, layout, [&](int lay, const usk::RbMap& map, int64_t nrb) {
+    return usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
+                            static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, lay, map, nrb);
+  });
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }

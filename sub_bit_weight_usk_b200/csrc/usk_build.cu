@@ -50,6 +50,7 @@ struct BuildArgs {
   int tpc;   // max tiles per block
   int nbuf;  // weight-tile buffers (1 or 2)
   int inject;  // test hook: block (0, 0) skips the copy of its first tile
+  RbMap map;   // grid row -> row block and code offset
 };
 
 // Shared-memory layout (byte offsets from a 128-byte aligned base).
@@ -93,7 +94,12 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
 
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
-  const int rb = blockIdx.y;
+  int rb;
+  int64_t code_base;
+  if (!rb_resolve(a.map, blockIdx.y, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
+    if (threadIdx.x == 0 && crank == 0) report(a.status, USK_FLAG_RATE_MAP);
+    return;  // the whole cluster (same grid row) leaves before any cluster barrier
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nt = (a.T - crank + a.C - 1) / a.C;  // this block's tiles: crank, crank + C, ...
 
@@ -369,7 +375,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
       packed |= Q4 ? (static_cast<uint64_t>(static_cast<uint32_t>(code) & 0xFu) << (4 * e))
                    : (static_cast<uint64_t>(static_cast<uint32_t>(code) & 0xFFu) << (8 * e));
     }
-    int8_t* dst = a.codes + (static_cast<int64_t>(rb) * a.T + tc) * F::kTileBytes + (Q4 ? 4u : kPer) * tid;
+    int8_t* dst = a.codes + code_base + static_cast<int64_t>(tc) * F::kTileBytes + (Q4 ? 4u : kPer) * tid;
     if (Q4 || kPer == 4) *reinterpret_cast<uint32_t*>(dst) = static_cast<uint32_t>(packed);
     else if (kPer == 2) *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
     else *reinterpret_cast<uint64_t*>(dst) = packed;
@@ -408,13 +414,13 @@ static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override
 }
 
 template <bool BF16, bool HAS_IMP, int VAR>
-static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, int cluster_override) {
+static cudaError_t launch_build_t(BuildArgs a, int64_t nrb, cudaStream_t stream, int cluster_override) {
   const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override, CodeFmt<VAR>::kBuckets);
   // tensor map over W [M, K] (row stride ldw), one 64 x 256 box per tile
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   CUtensorMap wmap;
-  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(RB * kRowsPerBlock)};
+  const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(a.K), static_cast<cuuint64_t>(a.map.RB * kRowsPerBlock)};
   const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(a.ldw) * (BF16 ? 2u : 4u)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTileCols), static_cast<cuuint32_t>(kRowsPerBlock)};
   const cuuint32_t estride[2] = {1, 1};
@@ -434,7 +440,7 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, 
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.C, static_cast<unsigned>(RB), 1);
+  cfg.gridDim = dim3(p.C, static_cast<unsigned>(nrb), 1);
   cfg.blockDim = dim3(kBuildThreads, 1, 1);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = stream;
@@ -450,14 +456,17 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t RB, cudaStream_t stream, 
 
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
-                         cudaStream_t stream, int cluster_override, int inject, int var) {
+                         cudaStream_t stream, int cluster_override, int inject, int var, const RbMap& map,
+                         int64_t nrb) {
   BuildArgs a;
   a.inject = inject;
+  a.map = map;
+  a.map.RB = M / kRowsPerBlock;
   a.W = W; a.ldw = ldw; a.K = K; a.imp = imp; a.seed = seed;
   a.codes = codes; a.scales = scales; a.status = status;
   a.T = static_cast<int>(K / kTileCols);
   a.C = a.tpc = a.nbuf = 0;
-  const int64_t RB = M / kRowsPerBlock;
+  const int64_t RB = nrb;
   auto go = [&](auto V) {
     constexpr int kVar = decltype(V)::value;
     if (bf16)

@@ -350,4 +350,32 @@ __device__ __forceinline__ void bf16_parts(uint32_t b, int& e_eff, int& mant) {
   mant = e == 0 ? m : (128 + m);
 }
 
+// Row blocks of one launch.  Uniform sketches: grid row g is row block g, its
+// codes at g * T * tile bytes.  Per-row-block rates: grid row g is row block
+// order[g] of the launch's slot group, its codes at offset[rb]; an entry out of
+// range (rb outside [0, RB), or a block ending past code_bytes, or an offset not
+// 16-byte aligned) is reported and skipped by the whole cluster (every block of
+// a cluster shares the grid row, so they all skip together).
+struct RbMap {
+  const int32_t* order;   // nullptr: identity
+  const int64_t* offset;
+  int64_t code_bytes;
+  int64_t RB;
+};
+
+__device__ __forceinline__ bool rb_resolve(const RbMap& m, int64_t g, int64_t rb_bytes, int& rb, int64_t& off) {
+  if (m.order == nullptr) {
+    rb = static_cast<int>(g);
+    off = g * rb_bytes;
+    return true;
+  }
+  const int64_t r = m.order[g];
+  if (r < 0 || r >= m.RB) return false;
+  const int64_t o = m.offset[r];
+  if (o < 0 || (o & 15) != 0 || o + rb_bytes > m.code_bytes) return false;
+  rb = static_cast<int>(r);
+  off = o;
+  return true;
+}
+
 }  // namespace usk

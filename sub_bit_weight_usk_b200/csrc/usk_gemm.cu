@@ -77,6 +77,8 @@ struct GemmArgs {
   int S;           // pipeline stages
   int I;           // MMA issuer warps, each with its own accumulator (columns [i N, (i + 1) N))
   int inject;  // test hook: block (0, 0) skips the x copy of its first chunk
+  RbMap map;    // grid rows -> row blocks and code offsets
+  int64_t nrb;  // row blocks of this launch (a tile takes grid rows 2 mt and 2 mt + 1)
 };
 
 struct GemmLayout {
@@ -201,9 +203,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(sm + L.misc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
-  const int64_t RB = a.M / kRowsPerBlock;
-  const int rb0 = 2 * mt;
-  const bool second_rb = rb0 + 1 < RB;
+  // the tile's two row blocks and where their codes start
+  const bool second_rb = 2 * static_cast<int64_t>(mt) + 1 < a.nrb;
+  int rbA = 0, rbB = 0;
+  int64_t cbA = 0, cbB = 0;
+  {
+    const int64_t rb_bytes = static_cast<int64_t>(a.T) * kRbBytes;
+    bool ok = rb_resolve(a.map, 2 * static_cast<int64_t>(mt), rb_bytes, rbA, cbA);
+    if (second_rb) ok = ok && rb_resolve(a.map, 2 * static_cast<int64_t>(mt) + 1, rb_bytes, rbB, cbB);
+    if (!ok) {
+      if (tid == 0 && ks == 0) report(a.status, USK_FLAG_RATE_MAP);
+      return;  // the whole cluster (same tile) leaves before any barrier or allocation
+    }
+  }
 
   if (warp == kMmaWarp0) {
     if (lane == 0) {
@@ -223,10 +235,9 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
       // the block's codes: two contiguous runs (one per row block)
       const uint32_t bytes = static_cast<uint32_t>(tcta) * kRbBytes;
       mbar_arrive_expect_tx(codes_bar, bytes * (second_rb ? 2u : 1u));
-      bulk_g2s(s0 + L.codes, a.codes + (static_cast<int64_t>(rb0) * a.T + t_begin) * kRbBytes, bytes, codes_bar);
+      bulk_g2s(s0 + L.codes, a.codes + cbA + static_cast<int64_t>(t_begin) * kRbBytes, bytes, codes_bar);
       if (second_rb)
-        bulk_g2s(s0 + L.codes + bytes, a.codes + (static_cast<int64_t>(rb0 + 1) * a.T + t_begin) * kRbBytes, bytes,
-                 codes_bar);
+        bulk_g2s(s0 + L.codes + bytes, a.codes + cbB + static_cast<int64_t>(t_begin) * kRbBytes, bytes, codes_bar);
     }
     __syncwarp();
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -236,7 +247,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   } else if (tid < 2 * tcta * D) {
     const int rbl = tid / (tcta * D), tl = (tid / D) % tcta;
-    keytab[tid] = row_key(a.seed, static_cast<uint64_t>(rb0 + rbl) * a.T + t_begin + tl, D, tid % D);
+    keytab[tid] = row_key(a.seed, static_cast<uint64_t>(rbl ? rbB : rbA) * a.T + t_begin + tl, D, tid % D);
   }
   tc_fence_before();
   __syncthreads();
@@ -252,7 +263,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
     const int g = tid >> 7;
     const int rbl = m >> 6;
     const uint32_t r = static_cast<uint32_t>(m & 63);
-    const bool row_ok = static_cast<int64_t>(mt) * kBM + m < a.M;
+    const bool row_ok = m < kRowsPerBlock || second_rb;
     // this thread's tensor-memory lane (= its row) in the A stages
     const uint32_t a_taddr = tmem_d + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + a.a_col;
     // loop exits are warp-uniform: tcgen05.st is a whole-warp instruction
@@ -409,9 +420,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   if (warp < kDecWarps) {
     const int sub = warp & 3, grp = warp >> 2;
     const int m = sub * 32 + lane;
-    const int64_t row = static_cast<int64_t>(mt) * kBM + m;
-    const bool row_ok = row < a.M;
-    const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[row / kRowsPerBlock])) : 0.0f;
+    const int rbm = m < kRowsPerBlock ? rbA : rbB;
+    const int64_t row = static_cast<int64_t>(rbm) * kRowsPerBlock + (m & 63);
+    const bool row_ok = m < kRowsPerBlock || second_rb;
+    const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[rbm])) : 0.0f;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     float* part = reinterpret_cast<float*>(sm + L.b);  // [N][128]: the x stage ring is free now
     for (int n0 = 8 * grp; n0 < a.N; n0 += 8 * kDecGroups) {
@@ -451,9 +463,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
 #pragma unroll
       for (int s = 0; s < 16; ++s) acc += v[s];
       const int n = q / kBM, mm = q % kBM;
-      const int64_t orow = static_cast<int64_t>(mt) * kBM + mm;
-      if (orow < a.M) {
-        const float sc = __half2float(__ushort_as_half(a.scales[orow / kRowsPerBlock]));
+      if (mm < kRowsPerBlock || second_rb) {
+        const int rbm = mm < kRowsPerBlock ? rbA : rbB;
+        const int64_t orow = static_cast<int64_t>(rbm) * kRowsPerBlock + (mm & 63);
+        const float sc = __half2float(__ushort_as_half(a.scales[rbm]));
         a.y[static_cast<int64_t>(n) * a.M + orow] = acc * sc;
       }
     }
@@ -556,7 +569,7 @@ bool gemm_supported(int64_t K, int batch, int depth, int var) {
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth, int var) {
+                        int depth, int var, const RbMap& map, int64_t nrb) {
   if ((depth != 1 && depth != 2 && depth != 4) || (var != 0 && depth != 1) || var < 0 || var > 3)
     return cudaErrorInvalidValue;
   GemmArgs a;
@@ -564,7 +577,10 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.M = M; a.K = K; a.seed = seed; a.status = status; a.inject = inject;
   a.T = static_cast<int>(K / kTileCols);
   a.N = batch;
-  const int64_t m_tiles = (M + kBM - 1) / kBM;
+  a.map = map;
+  a.map.RB = M / kRowsPerBlock;
+  a.nrb = nrb;
+  const int64_t m_tiles = (nrb + 1) / 2;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth, var);

@@ -42,6 +42,8 @@ struct GemvArgs {
   int C;      // blocks per row block (cluster size)
   int tpc;    // tiles per block (the last block of a row block may have fewer)
   int batch;  // 1..15
+  uint32_t* status;
+  RbMap map;  // grid row -> row block and code offset
 };
 
 constexpr int kGemvThreads = 256;
@@ -93,7 +95,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
-  const int rb = blockIdx.y;
+  int rb;
+  int64_t code_base;
+  if (!rb_resolve(a.map, blockIdx.y, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
+    if (threadIdx.x == 0 && crank == 0) report(a.status, USK_FLAG_RATE_MAP);
+    return;  // the whole cluster (same grid row) leaves before any cluster barrier
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);  // >= 1 by construction of C
@@ -105,7 +112,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   // ---- stage: hash keys, codes (int8 -> bf16) and the x slice, all loads in flight at once
   if (tid < nt * D) keytab[tid] = row_key(a.seed, static_cast<uint64_t>(rb) * a.T + t0 + tid / D, D, tid % D);
   {
-    const int8_t* csrc = a.codes + (static_cast<int64_t>(rb) * a.T + t0) * F::kTileBytes;
+    const int8_t* csrc = a.codes + code_base + static_cast<int64_t>(t0) * F::kTileBytes;
     const int ncode = nt * static_cast<int>(F::kTileBytes / 16u);  // 16-byte code chunks
     const int xchunks_row = XF32 ? nt * 64 : nt * 32;            // 16-byte x chunks per batch row
     const int nx = a.batch * xchunks_row;
@@ -293,13 +300,13 @@ static GemvGeometry gemv_geometry(int64_t K, int tpc_override) {
 }
 
 template <int NB, bool XF32, int D, int VAR>
-static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t RB, cudaStream_t stream) {
+static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t nrb, cudaStream_t stream) {
   const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32, D, CodeFmt<VAR>::kTileBf).total;
   auto kern = gemv_kernel<NB, XF32, D, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.gridDim = dim3(a.C, static_cast<unsigned>(nrb), 1);
   cfg.blockDim = dim3(kGemvThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -325,7 +332,7 @@ cudaError_t launch_gemv_slab(const int8_t* codes, const uint16_t* scales, int64_
 bool gemv_bf_supported(int64_t K, int batch, int tpc_override);
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth, int var);
+                           int tpc_override, int inject, int depth, int var, const RbMap& map, int64_t nrb);
 
 template <int D, int VAR>
 static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaStream_t stream) {
@@ -349,7 +356,8 @@ static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaS
 // rows of the sketch: the integer paths read single-row sketches only.
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
-                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var) {
+                        cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var,
+                        const RbMap& map, int64_t nrb) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // automatic choice (measured on B200, graphs of back-to-back calls):
@@ -357,7 +365,8 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   //  * batch >= 2, or batch 1 up to 4096 x 4096: bf16 with direct x fragments;
   //  * batch 1 with longer K or taller M: the integer cluster kernel (half the
   //    shared-memory gather bytes; its x preparation is amortised over more tiles)
-  const bool single = depth == 1 && var == 0;  // the integer paths read format-1 layouts of 4 slots
+  // the integer paths read uniform format-1 layouts of 4 slots
+  const bool single = depth == 1 && var == 0 && map.order == nullptr;
   const bool slab = single && (path == 3 || (path == 0 && M / kRowsPerBlock > 2 * sms));
   if (!xf32 && slab && slab_supported(K, batch))
     return launch_gemv_slab(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl,
@@ -367,7 +376,7 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
       path == 4 || (!single && path != 1) || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
   if (!xf32 && direct && gemv_bf_supported(K, batch, tpc_override))
     return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
-                          tpc_override, inject, depth, var);
+                          tpc_override, inject, depth, var, map, nrb);
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
   const bool i8_ok = single && !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
   if (i8_ok && path != 1)
@@ -377,7 +386,10 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed;
   a.T = geo.T; a.C = geo.C; a.tpc = geo.tpc; a.batch = batch;
-  const int64_t RB = M / kRowsPerBlock;
+  a.status = status;
+  a.map = map;
+  a.map.RB = M / kRowsPerBlock;
+  const int64_t RB = nrb;
   if (var == 1) return launch_staged<1, 1>(a, xf32, RB, stream);
   if (var == 2) return launch_staged<1, 2>(a, xf32, RB, stream);
   if (var == 3) return launch_staged<1, 3>(a, xf32, RB, stream);

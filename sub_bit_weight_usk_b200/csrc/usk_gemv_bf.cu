@@ -54,6 +54,7 @@ struct GemvBfArgs {
   int T, C, tpc;
   int pdl;     // launched as a programmatic dependent: wait before reading x
   int inject;  // test hook: block 1 of row block 0 skips its partial-sum stores
+  RbMap map;   // grid row -> row block and code offset
 };
 
 constexpr int kBfThreads = 256;
@@ -105,7 +106,12 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   extern __shared__ __align__(128) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = static_cast<int>(cluster.block_rank());
-  const int rb = blockIdx.y;
+  int rb;
+  int64_t code_base;
+  if (!rb_resolve(a.map, blockIdx.y, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
+    if (threadIdx.x == 0 && crank == 0) report(a.status, USK_FLAG_RATE_MAP);
+    return;  // the whole cluster (same grid row) leaves before any cluster barrier
+  }
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = crank * a.tpc;
   const int nt = min(a.tpc, a.T - t0);
@@ -121,7 +127,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   // ---- every global load first.  The codes are never written by a neighbour
   // in a programmatic-dependent chain (the caller's contract), so they go
   // before the dependency wait and overlap the previous kernel's tail; x after.
-  const int8_t* codes_blk = a.codes + (static_cast<int64_t>(rb) * a.T + t0) * F::kTileBytes;
+  const int8_t* codes_blk = a.codes + code_base + static_cast<int64_t>(t0) * F::kTileBytes;
   uint4 cv[kCodeLoads];
 #pragma unroll
   for (int u = 0; u < kCodeLoads; ++u) {
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
 }
 
 template <int B, int D, int VAR>
-static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
+static cudaError_t launch_bf_t(GemvBfArgs a, int64_t nrb, cudaStream_t stream) {
   const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D, CodeFmt<VAR>::kTileBf).total;
   auto kern = gemv_bf_kernel<B, D, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -297,7 +303,7 @@ static cudaError_t launch_bf_t(GemvBfArgs a, int64_t RB, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.C, static_cast<unsigned>(RB), 1);
+  cfg.gridDim = dim3(a.C, static_cast<unsigned>(nrb), 1);
   cfg.blockDim = dim3(kBfThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -338,8 +344,10 @@ bool gemv_bf_supported(int64_t K, int batch, int tpc_override) {
 
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth, int var) {
+                           int tpc_override, int inject, int depth, int var, const RbMap& map, int64_t nrb) {
   GemvBfArgs a;
+  a.map = map;
+  a.map.RB = M / kRowsPerBlock;
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status;
   a.T = static_cast<int>(K / kTileCols);
@@ -349,7 +357,7 @@ cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t 
   a.C = (a.T + a.tpc - 1) / a.tpc;
   a.pdl = pdl ? 1 : 0;
   a.inject = inject;
-  const int64_t RB = M / kRowsPerBlock;
+  const int64_t RB = nrb;
   if (var == 1) return launch_bf_batch<1, 1>(a, batch, RB, stream);
   if (var == 2) return launch_bf_batch<1, 2>(a, batch, RB, stream);
   if (var == 3) return launch_bf_batch<1, 3>(a, batch, RB, stream);

@@ -131,3 +131,83 @@ def test_sizes_ex(lib):
         usk.usk_sizes_ex(4096, 4096, 2, 8)
     with pytest.raises(usk.UskError):
         usk.usk_sizes_ex(4096, 4096, 1, 3)
+
+
+def test_struct_layouts_match_the_header(lib, tmp_path):
+    """sizeof and field offsets of the C structs (gcc on include/usk.h) equal
+    the binding's ctypes mirrors."""
+    import subprocess
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stddef.h>\n#include <stdio.h>\n#include "usk.h"\n'
+        'int main(void) {\n'
+        '  printf("%zu %zu %zu\\n", sizeof(usk_params), offsetof(usk_params, slots), offsetof(usk_params, rates));\n'
+        '  printf("%zu %zu %zu\\n", sizeof(usk_sketch), offsetof(usk_sketch, pad), offsetof(usk_sketch, rates));\n'
+        '  printf("%zu %zu %zu\\n", sizeof(usk_rate_map), offsetof(usk_rate_map, count),'
+        ' offsetof(usk_rate_map, code_bytes));\n'
+        '  return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)])
+    got = [list(map(int, ln.split())) for ln in subprocess.check_output([str(exe)]).decode().split("\n") if ln]
+    P, S, R = _native.UskParams, _native.UskSketchC, _native.UskRateMapC
+    assert got[0] == [ctypes.sizeof(P), P.slots.offset, P.rates.offset]
+    assert got[1] == [ctypes.sizeof(S), S.pad.offset, S.rates.offset]
+    assert got[2] == [ctypes.sizeof(R), R.count.offset, R.code_bytes.offset]
+
+
+def test_rate_map_plan_matches_the_oracle_offsets(lib):
+    import numpy as np
+    import oracle
+    g = np.random.default_rng(5)
+    for _ in range(50):
+        n = int(g.integers(1, 40))
+        K = 256 * int(g.integers(1, 20))
+        slots = [int(v) for v in g.choice([2, 4, 8], size=n)]
+        off, order, count, total = usk.usk_rate_map_plan(64 * n, K, slots)
+        ooff, ototal = oracle.vr_offsets(64 * n, K, slots)
+        assert off == ooff.tolist() and total == ototal
+        assert count == (slots.count(2), slots.count(4), slots.count(8))
+        # grouped by slot count, increasing within a group, a permutation
+        assert sorted(order) == list(range(n))
+        keys = [(slots[rb], rb) for rb in order]
+        assert keys == sorted(keys)
+    assert usk.usk_rate_map_plan(0, 256, []) == ([], [], (0, 0, 0), 0)
+    with pytest.raises(usk.UskError):
+        usk.usk_rate_map_plan(128, 256, [2, 6])
+    with pytest.raises(usk.UskError):
+        usk.usk_rate_map_plan(100, 256, [2])
+
+
+def test_rate_map_argument_errors(lib):
+    fake = ctypes.c_void_p(16 * 1024)
+    good = _native.UskRateMapC(16 * 1024, 16 * 1024)
+    good.count[0], good.count[1], good.count[2] = 1, 0, 1
+    good.code_bytes = 256 * (2 + 8)
+
+    def params(rm, version=1, slots=0):
+        p = _native.UskParams(version, 0, 0, 1, slots)
+        p.rates = ctypes.pointer(rm)
+        return p
+
+    def sketch(rm, version=1, slots=0):
+        s = _native.UskSketchC(128, 256, 0, 16 * 1024, 16 * 1024, version, 1, slots, 0)
+        s.rates = ctypes.pointer(rm)
+        return s
+
+    bad_counts = _native.UskRateMapC(16 * 1024, 16 * 1024)
+    bad_counts.count[0], bad_counts.code_bytes = 1, 512  # 1 of 2 row blocks
+    bad_bytes = _native.UskRateMapC(16 * 1024, 16 * 1024)
+    bad_bytes.count[0], bad_bytes.count[2], bad_bytes.code_bytes = 1, 1, 4096
+    no_tables = _native.UskRateMapC(None, None)
+    no_tables.count[1], no_tables.code_bytes = 2, 2048
+    odd = _native.UskRateMapC(16 * 1024 + 4, 16 * 1024)
+    odd.count[1], odd.code_bytes = 2, 2048
+    for rm, want in ((bad_counts, 6), (bad_bytes, 6), (no_tables, 1), (odd, 10)):
+        assert lib.usk_build(fake, 1, 128, 256, 256, None, ctypes.byref(params(rm)), fake, fake, None, None) == want
+        assert lib.usk_gemv(ctypes.byref(sketch(rm)), fake, 1, 1, fake, None, None) == want
+        assert lib.usk_gemm(ctypes.byref(sketch(rm)), fake, 16, fake, None, 0, None, None) == want
+    # a rate map only with format 1 and the default slot count
+    for version, slots in ((2, 0), (3, 0), (4, 0), (1, 8)):
+        p = params(good, version, slots)
+        assert lib.usk_build(fake, 1, 128, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 6
+        assert lib.usk_gemv(ctypes.byref(sketch(good, version, slots)), fake, 1, 1, fake, None, None) == 6
