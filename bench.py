@@ -14,7 +14,10 @@ of a 28672x8192 layer in format 1 (per-weight rehash and gather) and in format 3
 (bucket sums of x, then dense codes), reported under "colshared"; a fifth runs
 the three calls on the 4-bit-code sketch (format 4) of the layer ("q4"), and a
 sixth K builds and K batch-1 GEMVs of the layer at 2 and 8 hash slots per class
-(0.25 and 1 bit/weight, the rates of the importance-aware allocation, "rates").
+(0.25 and 1 bit/weight, the rates of the importance-aware allocation, "rates"),
+and a seventh the three calls on a sketch whose 64-row blocks carry their own
+rates, allocated at 0.5 bit/weight from the E[a^2] of each block's outputs on
+the layer with one lognormal gain per row block ("row_block_rates").
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl usk|reference]
 
@@ -129,6 +132,18 @@ def colshared_rooflines(peaks, t_build_s, t_gemv_s, t_gemv_ab_s, traffic):
     return {"usk_build": line((BUILD_BYTES - 4 * K) / t_build_s / 1e9, traffic.get("cs_usk_build")),
             "usk_gemv": line(GEMV_BYTES / t_gemv_s / 1e9, traffic.get("cs_usk_gemv")),
             "usk_gemv_%dx%d" % (AB_M, AB_K): line(ab_bytes / t_gemv_ab_s / 1e9, traffic.get("cs_usk_gemv_ab"))}
+
+
+def row_block_workload(cfg, usk):
+    """The layer with one lognormal gain per 64-row block (rows of unequal
+    output energy) and its per-row-block rates: importance of a block = E[a^2]
+    of its outputs over the calibration rows, slots from usk_plan_slots at 0.5
+    bit/weight.  Returns (W bf16 bits, slot list)."""
+    RB = M // 64
+    Wv = gen.scale_row_blocks(cfg["W"], gen.row_block_gains(RB, cfg["seed"]))
+    a = gen.bf16_bits_to_f32(cfg["x"]) @ gen.bf16_bits_to_f32(Wv).T  # calibration outputs [rows, M]
+    imp = (a.astype(np.float64) ** 2).reshape(a.shape[0], RB, 64).mean(axis=(0, 2))
+    return Wv, usk.usk_plan_slots([64 * K] * RB, imp.tolist(), 0.5)
 
 
 def source_sha(name):
@@ -475,6 +490,28 @@ def run_usk(args):
     graphs4 = prepare((gemv_hash, gemv_matrix))
     graphs5 = prepare((build4, gemv4, gemm4))
     graphs6 = prepare((build_rate(2), gemv_rate(2), build_rate(8), gemv_rate(8)))
+
+    # per-row-block rates on the row-gain layer
+    Wv_h, vr_slots = row_block_workload(cfg, usk)
+    Wv = torch.from_numpy(Wv_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    Wvs = [Wv.clone() for _ in range(N_WCOPIES)]
+    rmap = usk.usk_rate_map(M, K, vr_slots, dev)
+    skv = usk.usk_build(Wv, imp, seed, rates=rmap)
+    sksv = [usk.Sketch(M, K, seed, skv.codes.clone(), skv.scales.clone(), usk.FORMAT_MAXKEY, 1, 0, rmap)
+            for _ in range(N_SKETCHES)]
+    vr_groups = sum(1 for c in rmap.count if c > 0)
+
+    def build_vr(i):
+        b = sksv[i % N_SKETCHES]
+        usk.usk_build(Wvs[i % N_WCOPIES], imp, seed, codes=b.codes, scales=b.scales, status=status, rates=rmap)
+
+    def gemv_vr(i):
+        usk.usk_gemv(sksv[(i + N_SKETCHES // 2) % N_SKETCHES], x1, y=y1, pdl=True)
+
+    def gemm_vr(i):
+        usk.usk_gemm(sksv[(i + N_SKETCHES // 4) % N_SKETCHES], x16, y=y16, status=status)
+
+    graphs7 = prepare((build_vr, gemv_vr, gemm_vr))
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
@@ -484,6 +521,7 @@ def run_usk(args):
     t_hash, t_matrix, _ = timed(graphs4)
     t_build4, t_gemv4, t_gemm4, _ = timed(graphs5)
     t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8, _ = timed(graphs6)
+    t_build_v, t_gemv_v, t_gemm_v, _ = timed(graphs7)
     sampler.stop()
     t_step = t_total / max(args.steps, 1)
 
@@ -505,9 +543,11 @@ def run_usk(args):
 
     # max over ranks
     (t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2, t_build3, t_gemv3, t_hash,
-     t_matrix, t_build4, t_gemv4, t_gemm4, t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8) = max_over_ranks(
+     t_matrix, t_build4, t_gemv4, t_gemm4, t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8, t_build_v, t_gemv_v,
+     t_gemm_v) = max_over_ranks(
         [t_gemv, t_build, t_gemm, t_step, t_total, t_e2e, t_build2, t_gemv2, t_gemm2, t_build3, t_gemv3, t_hash,
-         t_matrix, t_build4, t_gemv4, t_gemm4, t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8], device=dev)
+         t_matrix, t_build4, t_gemv4, t_gemm4, t_build_r2, t_gemv_r2, t_build_r8, t_gemv_r8, t_build_v, t_gemv_v,
+         t_gemm_v], device=dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -613,6 +653,21 @@ def run_usk(args):
                         "usk_build_gweights_per_s": round(world * N_W / t_build_r8 / 1e9, 3)},
             "gpu_launches": 4 * args.steps,
         },
+        "row_block_rates": {
+            "format": "format 1 with one slot count per 64-row block (2, 4 or 8 hash slots per class), codes of "
+                      "the blocks back to back; the layer with a lognormal(0, 0.5^2) gain per row block, rates "
+                      "from usk_plan_slots at 0.5 bit/weight with importance = E[a^2] of each block's outputs "
+                      "over the %d calibration rows; column importance as the headline" % GEMM_BATCH,
+            "timing": "seventh timed region: K builds, K GEMVs (batch 1), K GEMMs (batch 16) as CUDA graphs; "
+                      "each call launches one kernel per slot group present",
+            "row_blocks_by_slots": {"2": rmap.count[0], "4": rmap.count[1], "8": rmap.count[2]},
+            "bits_per_weight": round(8.0 * rmap.code_bytes / N_W, 4),
+            "usk_gemv_gbs": round(world * (GEMV_BYTES - N_W // 16 + rmap.code_bytes) / t_gemv_v / 1e9, 3),
+            "usk_build_gweights_per_s": round(world * N_W / t_build_v / 1e9, 3),
+            "kernel_us": {"usk_build": round(t_build_v * 1e6, 3), "usk_gemv": round(t_gemv_v * 1e6, 3),
+                          "usk_gemm": round(t_gemm_v * 1e6, 3)},
+            "gpu_launches": 3 * vr_groups * args.steps,
+        },
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -638,10 +693,14 @@ def run_profile_case(args):
         fmt = {"version": usk.FORMAT_COLSHARED}
     elif case.endswith("_q4"):
         fmt = {"version": usk.FORMAT_Q4}
+    if case.endswith("_vr"):  # per-row-block rates on the row-gain layer
+        Wv_h, vr_slots = row_block_workload(cfg, usk)
+        W = torch.from_numpy(Wv_h.view(np.int16)).to(dev).view(torch.bfloat16)
+        fmt = {"rates": usk.usk_rate_map(M, K, vr_slots, dev)}
     if case.endswith("_ab"):  # the 28672 x 8192 A/B shape, device-drawn weights
         W = gen.device_weights_normal(AB_M, AB_K, 3, 0.02, dev)
         x1 = torch.from_numpy(gen.activations(1, AB_K, 3, "bf16").view(np.int16)).to(dev).view(torch.bfloat16)
-    imp_c = imp if (not fmt or case.endswith("_q4")) and not case.endswith("_ab") else None
+    imp_c = imp if (not fmt or case.endswith("_q4") or case.endswith("_vr")) and not case.endswith("_ab") else None
     sk = usk.usk_build(W, imp_c, cfg["seed"], **fmt)
     torch.cuda.synchronize()
     for _ in range(3 + 3):  # 3 warm-up launches, then 3 to capture
@@ -665,7 +724,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-case", choices=["build", "gemv", "gemm", "build_amm", "gemv_amm", "gemm_amm",
                                                "build_cs", "gemv_cs", "gemv_ab", "gemv_cs_ab", "build_q4", "gemv_q4",
-                                               "gemm_q4"],
+                                               "gemm_q4", "build_vr", "gemv_vr", "gemm_vr"],
                     default=None,
                     help="run 6 launches of one kernel on the bench workload (for ncu) and exit")
     args = ap.parse_args(argv)

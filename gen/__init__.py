@@ -123,6 +123,21 @@ def layer(batch: int = 1, M: int = 4096, K: int = 4096):
     }
 
 
+def row_block_gains(RB: int, seed: int, sigma: float = 0.5) -> np.ndarray:
+    """One lognormal gain exp(N(0, sigma^2)) per 64-row block: rows of unequal
+    output energy (stream of its own)."""
+    return np.exp(rng(seed, 7).normal(0.0, sigma, size=RB)).astype(np.float32)
+
+
+def scale_row_blocks(W: np.ndarray, gains: np.ndarray) -> np.ndarray:
+    """W (bf16 bits or float32) with 64-row block rb multiplied by gains[rb],
+    rounded back to the input type."""
+    M, K = W.shape
+    Wf = bf16_bits_to_f32(W) if W.dtype == np.uint16 else W
+    out = (Wf.reshape(M // 64, 64, K) * gains[:, None, None].astype(np.float32)).reshape(M, K)
+    return f32_to_bf16_bits(out) if W.dtype == np.uint16 else out.astype(np.float32)
+
+
 def llama7b_layer(name: str, batch: int = 1):
     """One linear of the 7B layer set (seed 2 + its index)."""
     idx = LLAMA7B_ORDER.index(name)
