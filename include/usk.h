@@ -270,6 +270,7 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
  * Other batches, multi-row and 4-bit sketches: bf16 tensor path (each hash row
  * gathered, the code of largest magnitude kept), exact products, fp32 accumulation; fp32 x
  * is split into two bf16 terms (|error| <= 2^-16 |x| per element).
+ * A sketch with a rate map: one launch per slot group present, bf16 path.
  * batch == 0 or M == 0 is a no-op; K == 0 writes y = 0.  Deterministic for a
  * given shape (the summation order is fixed). */
 USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
@@ -290,6 +291,8 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
  * fp32 accumulation in tensor memory.
  *   x_bf16 [batch, K] bf16, 16-byte aligned.  y [batch, M] fp32.
  *   ws / ws_bytes: unused by this version (may be NULL / 0).
+ * A sketch with a rate map: one launch per slot group present; a 128-row tile
+ * takes two row blocks of one group.
  * M == 0 is a no-op; K == 0 writes y = 0. */
 USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y,
                     void* ws, size_t ws_bytes, uint32_t* d_status, void* stream);
