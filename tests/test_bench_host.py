@@ -69,3 +69,25 @@ def test_max_over_ranks_two_gloo_ranks():
 
 def test_single_process_identity():
     assert bench.max_over_ranks([3.0, 4.0]) == [3.0, 4.0]
+
+
+def test_row_block_workload_allocation():
+    """The bench's per-row-block-rate workload: the allocation keeps the 0.5
+    bit/weight budget, mixes rates, and gives no block fewer slots than a block
+    of smaller output energy (the gain per block drives E[a^2])."""
+    import numpy as np
+    import gen
+    import oracle
+    import sub_bit_weight_usk_b200 as usk
+    cfg = gen.layer(bench.GEMM_BATCH)
+    Wv, slots = bench.row_block_workload(cfg, usk)
+    RB = bench.M // 64
+    assert Wv.shape == (bench.M, bench.K) and Wv.dtype == np.uint16 and len(slots) == RB
+    assert set(slots) <= {2, 4, 8} and len(set(slots)) == 3
+    assert bench.K * sum(slots) * 8 <= 0.5 * bench.M * bench.K
+    xf = gen.bf16_bits_to_f32(cfg["x"])
+    a = xf @ gen.bf16_bits_to_f32(Wv).T
+    imp = (a.astype(np.float64) ** 2).reshape(a.shape[0], RB, 64).mean(axis=(0, 2))
+    assert slots == oracle.plan_slots([64 * bench.K] * RB, imp.tolist(), 0.5)
+    order = np.argsort(imp)
+    assert all(slots[order[i]] <= slots[order[i + 1]] for i in range(RB - 1))
