@@ -251,7 +251,8 @@ USK_API usk_status usk_rate_map_plan(int64_t M, int64_t K, const uint32_t* slots
  *   codes      int8 output, 16-byte aligned: M*K/16 bytes (usk_sizes_ex for
  *              other formats and slot counts; rate-map code_bytes with
  *              params->rates).   scales [M/64] output.
- *   params->rates  per-row-block rates: one launch per slot group present.
+ *   params->rates  per-row-block rates: still one launch; each row block uses
+ *              its own slot count.
  *   d_status   optional device word for USK_FLAG_* bits.
  * M == 0 is a no-op; K == 0 writes zero scales.  Codes and scales are
  * bit-identical for any launch geometry. */
@@ -270,7 +271,7 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
  * Other batches, multi-row and 4-bit sketches: bf16 tensor path (each hash row
  * gathered, the code of largest magnitude kept), exact products, fp32 accumulation; fp32 x
  * is split into two bf16 terms (|error| <= 2^-16 |x| per element).
- * A sketch with a rate map: one launch per slot group present, bf16 path.
+ * A sketch with a rate map: one launch, each row block at its slot count, bf16 path.
  * batch == 0 or M == 0 is a no-op; K == 0 writes y = 0.  Deterministic for a
  * given shape (the summation order is fixed). */
 USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
@@ -291,8 +292,8 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
  * fp32 accumulation in tensor memory.
  *   x_bf16 [batch, K] bf16, 16-byte aligned.  y [batch, M] fp32.
  *   ws / ws_bytes: unused by this version (may be NULL / 0).
- * A sketch with a rate map: one launch per slot group present; a 128-row tile
- * takes two row blocks of one group.
+ * A sketch with a rate map: one launch; a 128-row tile takes two row blocks of
+ * the same slot count.
  * M == 0 is a no-op; K == 0 writes y = 0. */
 USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y,
                     void* ws, size_t ws_bytes, uint32_t* d_status, void* stream);

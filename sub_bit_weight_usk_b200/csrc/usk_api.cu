@@ -1,7 +1,6 @@
 // usk_api.cu -- the C ABI of libusk (declared in include/usk.h): argument
-// validation, then one kernel launch per call (one per slot group for a sketch
-// with per-row-block rates).  No allocation, no global state beyond CUDA's
-// cached kernel attributes.
+// validation, then one kernel launch per call.  No allocation, no global state
+// beyond CUDA's cached kernel attributes.
 #include <algorithm>
 #include <cstdint>
 #include <vector>
@@ -15,7 +14,7 @@ namespace usk {
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
                          cudaStream_t stream, int cluster_override, int inject, int var, const RbMap& map,
-                         int64_t nrb);
+                         int64_t nrb, int64_t g1, int64_t g2);
 cudaError_t launch_build_amm(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, uint64_t seed, int depth,
                              int8_t* codes, uint16_t* scales, uint32_t* status, cudaStream_t stream,
                              int cluster_override, int inject);
@@ -28,10 +27,10 @@ cudaError_t launch_gemv_cs(const int8_t* codes, const uint16_t* scales, int64_t 
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
                         cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var,
-                        const RbMap& map, int64_t nrb);
+                        const RbMap& map, int64_t nrb, int64_t g1, int64_t g2);
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth, int var, const RbMap& map, int64_t nrb);
+                        int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2);
 bool gemm_supported(int64_t K, int batch, int depth, int var);
 }  // namespace usk
 
@@ -87,22 +86,19 @@ usk_status check_rate_map(const usk_rate_map* m, int64_t M, int64_t K) {
   return USK_OK;
 }
 
-// Launch groups of a sketch: one per slot count present (rate map), else one
-// over every row block.  fn(layout, RbMap, row blocks) returns a cudaError_t.
-template <class Fn>
-cudaError_t for_each_group(const usk_rate_map* rm, int64_t M, int layout, Fn&& fn) {
+// The row-block map of one launch: identity for a uniform sketch; with a rate
+// map, its order and offsets, and where the 4- and 8-slot groups start in the
+// order list (the kernels pick each block's code layout from that).
+struct Launch {
+  usk::RbMap map;
+  int64_t nrb, g1, g2;
+};
+
+Launch launch_of(const usk_rate_map* rm, int64_t M) {
   const int64_t RB = M / USK_ROWS_PER_BLOCK;
-  if (!rm) return fn(layout, usk::RbMap{nullptr, nullptr, 0, RB}, RB);
-  static const int kLayouts[3] = {2, 0, 3};  // 2, 4 and 8 slots
-  int64_t start = 0;
-  for (int g = 0; g < 3; ++g) {
-    if (rm->count[g] > 0) {
-      cudaError_t e = fn(kLayouts[g], usk::RbMap{rm->order + start, rm->offset, rm->code_bytes, RB}, rm->count[g]);
-      if (e != cudaSuccess) return e;
-    }
-    start += rm->count[g];
-  }
-  return cudaSuccess;
+  if (!rm) return Launch{usk::RbMap{nullptr, nullptr, 0, RB}, RB, 0, 0};
+  return Launch{usk::RbMap{rm->order, rm->offset, rm->code_bytes, RB}, RB, rm->count[0],
+                rm->count[0] + rm->count[1]};
 }
 
 usk_status check_sketch(const usk_sketch* s) {
@@ -299,11 +295,11 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
   else if (amm)
     e = usk::launch_build_amm(W, wdtype == USK_BF16, M, K, ldw, params->seed, depth, codes, scales, d_status, s,
                               g_build_cluster, g_inject == 1);
-  else
-    e = for_each_group(rm, M, layout, [&](int lay, const usk::RbMap& map, int64_t nrb) {
-      return usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes, scales, d_status,
-                               s, g_build_cluster, g_inject == 1, lay, map, nrb);
-    });
+  else {
+    const Launch l = launch_of(rm, M);
+    e = usk::launch_build(W, wdtype == USK_BF16, M, K, ldw, importance, params->seed, codes, scales, d_status, s,
+                          g_build_cluster, g_inject == 1, layout, l.map, l.nrb, l.g1, l.g2);
+  }
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -331,14 +327,12 @@ USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtyp
     if (e != cudaSuccess) return USK_ERR_CUDA;
     return from_cuda(cudaGetLastError());
   }
-  cudaError_t e = for_each_group(
-      sketch->rates, sketch->M, layout_of(sketch->version, sketch->slots),
-      [&](int lay, const usk::RbMap& map, int64_t nrb) {
-        return usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
-                                xdtype == USK_F32, static_cast<int>(batch), y, d_status, (flags & USK_GEMV_PDL) != 0,
-                                g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows, g_inject == 3,
-                                format_depth(sketch->version, sketch->depth), lay, map, nrb);
-      });
+  const Launch l = launch_of(sketch->rates, sketch->M);
+  cudaError_t e = usk::launch_gemv(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x,
+                                   xdtype == USK_F32, static_cast<int>(batch), y, d_status,
+                                   (flags & USK_GEMV_PDL) != 0, g_gemv_path, s, g_gemv_tiles_per_block, g_gemv_rows,
+                                   g_inject == 3, format_depth(sketch->version, sketch->depth),
+                                   layout_of(sketch->version, sketch->slots), l.map, l.nrb, l.g1, l.g2);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -368,10 +362,10 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
     return from_cuda(cudaMemsetAsync(y, 0, sizeof(float) * static_cast<size_t>(batch * sketch->M), s));
   if (!x_bf16) return USK_ERR_NULL;
   if (!aligned16(x_bf16) || !aligned16(y)) return USK_ERR_ALIGN;
-  cudaError_t e = for_each_group(sketch->rates, sketch->M, layout, [&](int lay, const usk::RbMap& map, int64_t nrb) {
-    return usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
-                            static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, lay, map, nrb);
-  });
+  const Launch l = launch_of(sketch->rates, sketch->M);
+  cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
+                                   static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, layout, l.map,
+                                   l.nrb, l.g1, l.g2);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }

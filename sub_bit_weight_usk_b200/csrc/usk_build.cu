@@ -51,6 +51,7 @@ struct BuildArgs {
   int nbuf;  // weight-tile buffers (1 or 2)
   int inject;  // test hook: block (0, 0) skips the copy of its first tile
   RbMap map;   // grid row -> row block and code offset
+  int64_t g1, g2;  // per-row-block rates: first grid rows of the 4- and 8-slot groups
 };
 
 // Shared-memory layout (byte offsets from a 128-byte aligned base).
@@ -77,7 +78,7 @@ __host__ __device__ inline BuildLayout build_layout(bool bf16, bool has_imp, int
 // 256 x slots buckets per tile) and 8-bit codes, or 8 slots with 4-bit codes
 // (scale max |v| / 7, codes clamp(rint(v / s), -7, 7) packed two per byte).
 template <bool BF16, bool HAS_IMP, int VAR>
-__global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
+__device__ __forceinline__ void build_body(const BuildArgs& a, const CUtensorMap* wmap, int64_t grid_row) {
   using F = CodeFmt<VAR>;
   constexpr bool Q4 = F::kNibble;
   constexpr bool kSingle = BF16 && !HAS_IMP;
@@ -96,7 +97,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   const int crank = static_cast<int>(cluster.block_rank());
   int rb;
   int64_t code_base;
-  if (!rb_resolve(a.map, blockIdx.y, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
+  if (!rb_resolve(a.map, grid_row, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
     if (threadIdx.x == 0 && crank == 0) report(a.status, USK_FLAG_RATE_MAP);
     return;  // the whole cluster (same grid row) leaves before any cluster barrier
   }
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   // first half of a split cluster barrier; its wait, before the first remote
   // access, guarantees that every block of the cluster has started
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-  if (tid == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&wmap)) : "memory");
+  if (tid == 0) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(wmap)) : "memory");
 
   // importance of this lane's 8 columns, one tile ahead (the loads of tile 0
   // go out before the weight copies fill the memory queues)
@@ -124,7 +125,7 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
     const int buf = i % a.nbuf;
     const uint32_t bar = s0 + L.bars + 8 * buf;
     mbar_arrive_expect_tx(bar, kTileBytes);
-    tma_load_2d(s0 + L.wbuf + buf * kTileBytes, &wmap, tc * kTileCols, rb * kRowsPerBlock, bar);
+    tma_load_2d(s0 + L.wbuf + buf * kTileBytes, wmap, tc * kTileCols, rb * kRowsPerBlock, bar);
   };
   // ---- init: the first tile copies go out first, then the winner and key
   // words of both slots are cleared while the weights stream in
@@ -383,6 +384,22 @@ __global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs
   report(a.status, flags);
 }
 
+template <bool BF16, bool HAS_IMP, int VAR>
+__global__ void __launch_bounds__(kBuildThreads, 2) build_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
+  build_body<BF16, HAS_IMP, VAR>(a, &wmap, blockIdx.y);
+}
+
+// Per-row-block rates in one launch: grid row g is entry g of the rate map's
+// order list (grouped by slot count), so its group -- and the compile-time code
+// layout -- follows from g; every block of a cluster shares g.
+template <bool BF16, bool HAS_IMP>
+__global__ void __launch_bounds__(kBuildThreads, 2) build_vr_kernel(const BuildArgs a, const __grid_constant__ CUtensorMap wmap) {
+  const int64_t g = blockIdx.y;
+  if (g < a.g1) build_body<BF16, HAS_IMP, 2>(a, &wmap, g);
+  else if (g < a.g2) build_body<BF16, HAS_IMP, 0>(a, &wmap, g);
+  else build_body<BF16, HAS_IMP, 3>(a, &wmap, g);
+}
+
 // ---------------------------------------------------------------- launch
 
 struct BuildPlan {
@@ -415,7 +432,10 @@ static BuildPlan plan_build(int T, bool bf16, bool has_imp, int cluster_override
 
 template <bool BF16, bool HAS_IMP, int VAR>
 static cudaError_t launch_build_t(BuildArgs a, int64_t nrb, cudaStream_t stream, int cluster_override) {
-  const BuildPlan p = plan_build(a.T, BF16, HAS_IMP, cluster_override, CodeFmt<VAR>::kBuckets);
+  // a rate map: one launch over every row block, shared memory planned for 8 slots
+  const bool vr = a.map.order != nullptr;
+  const BuildPlan p =
+      plan_build(a.T, BF16, HAS_IMP, cluster_override, vr ? CodeFmt<3>::kBuckets : CodeFmt<VAR>::kBuckets);
   // tensor map over W [M, K] (row stride ldw), one 64 x 256 box per tile
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -432,7 +452,7 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t nrb, cudaStream_t stream,
   a.C = p.C;
   a.tpc = p.tpc;
   a.nbuf = p.nbuf;
-  auto kern = build_kernel<BF16, HAS_IMP, VAR>;
+  auto kern = vr ? build_vr_kernel<BF16, HAS_IMP> : build_kernel<BF16, HAS_IMP, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(p.smem));
   if (e != cudaSuccess) return e;
   if (p.C > 8) {
@@ -457,11 +477,14 @@ static cudaError_t launch_build_t(BuildArgs a, int64_t nrb, cudaStream_t stream,
 cudaError_t launch_build(const void* W, bool bf16, int64_t M, int64_t K, int64_t ldw, const float* imp,
                          uint64_t seed, int8_t* codes, uint16_t* scales, uint32_t* status,
                          cudaStream_t stream, int cluster_override, int inject, int var, const RbMap& map,
-                         int64_t nrb) {
+                         int64_t nrb, int64_t g1, int64_t g2) {
   BuildArgs a;
   a.inject = inject;
   a.map = map;
   a.map.RB = M / kRowsPerBlock;
+  a.g1 = g1;
+  a.g2 = g2;
+  if (map.order != nullptr) var = 0;  // the rate-map kernel covers every layout
   a.W = W; a.ldw = ldw; a.K = K; a.imp = imp; a.seed = seed;
   a.codes = codes; a.scales = scales; a.status = status;
   a.T = static_cast<int>(K / kTileCols);

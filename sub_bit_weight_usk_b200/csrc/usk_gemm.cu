@@ -79,6 +79,7 @@ struct GemmArgs {
   int inject;  // test hook: block (0, 0) skips the x copy of its first chunk
   RbMap map;    // grid rows -> row blocks and code offsets
   int64_t nrb;  // row blocks of this launch (a tile takes grid rows 2 mt and 2 mt + 1)
+  int64_t g1, g2;  // per-row-block rates: where the 4- and 8-slot groups start in the order list
 };
 
 struct GemmLayout {
@@ -173,8 +174,11 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
 // of largest magnitude)
 // VAR: code layout (CodeFmt; D == 1 unless VAR == 0): the widen warp expands
 // each row block's stored tile (512 to 2048 bytes) into 256 x slots bf16.
+// mt: the tile within its slot group; order0 / nrb: where the group starts in
+// the order list and its row blocks (the whole matrix for a uniform sketch).
 template <int D, int VAR>
-__global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
+__device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* xmap, int mt, int64_t order0,
+                                          int64_t nrb) {
   using F = CodeFmt<VAR>;
   constexpr bool Q4 = F::kNibble;
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
@@ -184,7 +188,6 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   extern __shared__ __align__(16) uint8_t sm_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int ks = static_cast<int>(cluster.block_rank());
-  const int mt = blockIdx.y;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   const uint32_t raw_s = smem_u32(sm_raw);
@@ -204,13 +207,15 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   // the tile's two row blocks and where their codes start
-  const bool second_rb = 2 * static_cast<int64_t>(mt) + 1 < a.nrb;
+  const bool second_rb = 2 * static_cast<int64_t>(mt) + 1 < nrb;
   int rbA = 0, rbB = 0;
   int64_t cbA = 0, cbB = 0;
   {
     const int64_t rb_bytes = static_cast<int64_t>(a.T) * kRbBytes;
-    bool ok = rb_resolve(a.map, 2 * static_cast<int64_t>(mt), rb_bytes, rbA, cbA);
-    if (second_rb) ok = ok && rb_resolve(a.map, 2 * static_cast<int64_t>(mt) + 1, rb_bytes, rbB, cbB);
+    RbMap gm = a.map;
+    if (gm.order != nullptr) gm.order += order0;
+    bool ok = rb_resolve(gm, 2 * static_cast<int64_t>(mt), rb_bytes, rbA, cbA);
+    if (second_rb) ok = ok && rb_resolve(gm, 2 * static_cast<int64_t>(mt) + 1, rb_bytes, rbB, cbB);
     if (!ok) {
       if (tid == 0 && ks == 0) report(a.status, USK_FLAG_RATE_MAP);
       return;  // the whole cluster (same tile) leaves before any barrier or allocation
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
       }
       *abort_flag = 0u;
       mbar_fence_init();
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(xmap)) : "memory");
       // the block's codes: two contiguous runs (one per row block)
       const uint32_t bytes = static_cast<uint32_t>(tcta) * kRbBytes;
       mbar_arrive_expect_tx(codes_bar, bytes * (second_rb ? 2u : 1u));
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
       }
       if (lane == 0 && !(a.inject && c == 0 && ks == 0 && mt == 0)) {
         mbar_arrive_expect_tx(full_s + 8 * s, bstage);
-        tma_load_2d(s0 + L.b + s * bstage, &xmap, t_begin * kTileCols + c * kBK, 0, full_s + 8 * s);
+        tma_load_2d(s0 + L.b + s * bstage, xmap, t_begin * kTileCols + c * kBK, 0, full_s + 8 * s);
       }
       __syncwarp();
     }
@@ -482,6 +487,24 @@ __global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a,
   }
 }
 
+template <int D, int VAR>
+__global__ void __launch_bounds__(kGemmThreads, 2) gemm_kernel(const GemmArgs a, const __grid_constant__ CUtensorMap xmap) {
+  gemm_body<D, VAR>(a, &xmap, static_cast<int>(blockIdx.y), 0, a.nrb);
+}
+
+// Per-row-block rates in one launch: the tiles of the 2-, 4- and 8-slot groups
+// follow one another in grid y (a tile never mixes groups; an odd group leaves
+// a one-block tile), so grid row y gives the group, its layout and its tile.
+__global__ void __launch_bounds__(kGemmThreads, 2) gemm_vr_kernel(const GemmArgs a,
+                                                                  const __grid_constant__ CUtensorMap xmap) {
+  const int64_t c0 = a.g1, c1 = a.g2 - a.g1, c2 = a.map.RB - a.g2;
+  const int64_t t0 = (c0 + 1) / 2, t1 = (c1 + 1) / 2;
+  const int64_t y = blockIdx.y;
+  if (y < t0) gemm_body<1, 2>(a, &xmap, static_cast<int>(y), 0, c0);
+  else if (y < t0 + t1) gemm_body<1, 0>(a, &xmap, static_cast<int>(y - t0), a.g1, c1);
+  else gemm_body<1, 3>(a, &xmap, static_cast<int>(y - t0 - t1), a.g2, c2);
+}
+
 // ---------------------------------------------------------------- launch
 
 constexpr uint32_t kSmemLimit = 227u * 1024u;
@@ -569,7 +592,14 @@ bool gemm_supported(int64_t K, int batch, int depth, int var) {
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth, int var, const RbMap& map, int64_t nrb) {
+                        int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2) {
+  // a rate map: one launch over the tiles of every slot group, planned for the
+  // 8-slot layout (the largest staged and widened tiles)
+  const bool vr = map.order != nullptr;
+  if (vr) {
+    depth = 1;
+    var = 3;
+  }
   if ((depth != 1 && depth != 2 && depth != 4) || (var != 0 && depth != 1) || var < 0 || var > 3)
     return cudaErrorInvalidValue;
   GemmArgs a;
@@ -580,7 +610,9 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.map = map;
   a.map.RB = M / kRowsPerBlock;
   a.nrb = nrb;
-  const int64_t m_tiles = (nrb + 1) / 2;
+  a.g1 = g1;
+  a.g2 = g2;
+  const int64_t m_tiles = vr ? (g1 + 1) / 2 + (g2 - g1 + 1) / 2 + (a.map.RB - g2 + 1) / 2 : (nrb + 1) / 2;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth, var);
@@ -604,7 +636,8 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  auto kern = var == 1 ? gemm_kernel<1, 1>
+  auto kern = vr ? gemm_vr_kernel
+             : var == 1 ? gemm_kernel<1, 1>
              : var == 2 ? gemm_kernel<1, 2>
              : var == 3 ? gemm_kernel<1, 3>
              : (depth == 4 ? gemm_kernel<4, 0> : (depth == 2 ? gemm_kernel<2, 0> : gemm_kernel<1, 0>));

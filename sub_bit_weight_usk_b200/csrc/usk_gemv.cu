@@ -44,6 +44,7 @@ struct GemvArgs {
   int batch;  // 1..15
   uint32_t* status;
   RbMap map;  // grid row -> row block and code offset
+  int64_t g1, g2;  // per-row-block rates: first grid rows of the 4- and 8-slot groups
 };
 
 constexpr int kGemvThreads = 256;
@@ -86,7 +87,7 @@ __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *rein
 // tile and reduced to the code of largest magnitude)
 // VAR: code layout (CodeFmt; D == 1 unless VAR == 0).
 template <int NB, bool XF32, int D, int VAR>
-__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
+__device__ __forceinline__ void gemv_body(const GemvArgs& a, int64_t grid_row) {
   using F = CodeFmt<VAR>;
   constexpr bool Q4 = F::kNibble;
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
@@ -97,7 +98,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
   const int crank = static_cast<int>(cluster.block_rank());
   int rb;
   int64_t code_base;
-  if (!rb_resolve(a.map, blockIdx.y, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
+  if (!rb_resolve(a.map, grid_row, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
     if (threadIdx.x == 0 && crank == 0) report(a.status, USK_FLAG_RATE_MAP);
     return;  // the whole cluster (same grid row) leaves before any cluster barrier
   }
@@ -300,9 +301,27 @@ static GemvGeometry gemv_geometry(int64_t K, int tpc_override) {
 }
 
 template <int NB, bool XF32, int D, int VAR>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvArgs a) {
+  gemv_body<NB, XF32, D, VAR>(a, blockIdx.y);
+}
+
+// Per-row-block rates in one launch: grid row g is entry g of the rate map's
+// order list (grouped by slot count), so its code layout follows from g.
+template <int NB, bool XF32>
+__global__ void __launch_bounds__(kGemvThreads) gemv_vr_kernel(const GemvArgs a) {
+  const int64_t g = blockIdx.y;
+  if (g < a.g1) gemv_body<NB, XF32, 1, 2>(a, g);
+  else if (g < a.g2) gemv_body<NB, XF32, 1, 0>(a, g);
+  else gemv_body<NB, XF32, 1, 3>(a, g);
+}
+
+template <int NB, bool XF32, int D, int VAR>
 static cudaError_t launch_gemv_t(const GemvArgs& a, int64_t nrb, cudaStream_t stream) {
-  const size_t smem = gemv_layout(a.tpc, NB, a.batch, XF32, D, CodeFmt<VAR>::kTileBf).total;
-  auto kern = gemv_kernel<NB, XF32, D, VAR>;
+  // a rate map: one launch over every row block, shared memory for 8 slots
+  const bool vr = a.map.order != nullptr;
+  const size_t smem =
+      gemv_layout(a.tpc, NB, a.batch, XF32, D, vr ? CodeFmt<3>::kTileBf : CodeFmt<VAR>::kTileBf).total;
+  auto kern = vr ? gemv_vr_kernel<NB, XF32> : gemv_kernel<NB, XF32, D, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -332,7 +351,8 @@ cudaError_t launch_gemv_slab(const int8_t* codes, const uint16_t* scales, int64_
 bool gemv_bf_supported(int64_t K, int batch, int tpc_override);
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth, int var, const RbMap& map, int64_t nrb);
+                           int tpc_override, int inject, int depth, int var, const RbMap& map, int64_t nrb,
+                           int64_t g1, int64_t g2);
 
 template <int D, int VAR>
 static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaStream_t stream) {
@@ -357,7 +377,7 @@ static cudaError_t launch_staged(const GemvArgs& a, bool xf32, int64_t RB, cudaS
 cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const void* x, bool xf32, int batch, float* y, uint32_t* status, bool pdl, int path,
                         cudaStream_t stream, int tpc_override, int rows_override, int inject, int depth, int var,
-                        const RbMap& map, int64_t nrb) {
+                        const RbMap& map, int64_t nrb, int64_t g1, int64_t g2) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // automatic choice (measured on B200, graphs of back-to-back calls):
@@ -376,7 +396,7 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
       path == 4 || (!single && path != 1) || (path == 0 && (batch > 1 || (K <= 4096 && M <= 4096)));
   if (!xf32 && direct && gemv_bf_supported(K, batch, tpc_override))
     return launch_gemv_bf(codes, scales, M, K, seed, static_cast<const uint16_t*>(x), batch, y, status, pdl, stream,
-                          tpc_override, inject, depth, var, map, nrb);
+                          tpc_override, inject, depth, var, map, nrb, g1, g2);
   const GemvGeometry geo = gemv_geometry(K, tpc_override);
   const bool i8_ok = single && !xf32 && batch <= 4 && batch * geo.tpc * 32 <= 1024;
   if (i8_ok && path != 1)
@@ -389,7 +409,10 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.status = status;
   a.map = map;
   a.map.RB = M / kRowsPerBlock;
+  a.g1 = g1;
+  a.g2 = g2;
   const int64_t RB = nrb;
+  if (map.order != nullptr) return launch_staged<1, 0>(a, xf32, RB, stream);  // covers every layout
   if (var == 1) return launch_staged<1, 1>(a, xf32, RB, stream);
   if (var == 2) return launch_staged<1, 2>(a, xf32, RB, stream);
   if (var == 3) return launch_staged<1, 3>(a, xf32, RB, stream);

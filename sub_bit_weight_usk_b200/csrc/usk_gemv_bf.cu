@@ -55,6 +55,7 @@ struct GemvBfArgs {
   int pdl;     // launched as a programmatic dependent: wait before reading x
   int inject;  // test hook: block 1 of row block 0 skips its partial-sum stores
   RbMap map;   // grid row -> row block and code offset
+  int64_t g1, g2;  // per-row-block rates: first grid rows of the 4- and 8-slot groups
 };
 
 constexpr int kBfThreads = 256;
@@ -96,7 +97,7 @@ __device__ __forceinline__ void st_async_f32(uint32_t remote_addr, float v, uint
 // VAR: code layout (CodeFmt; D == 1 unless VAR == 0): 2, 4 or 8 slots per
 // class, 8-bit codes, or 8 slots with 4-bit codes (32 codes per 16-byte load).
 template <int B, int D, int VAR>
-__global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a) {
+__device__ __forceinline__ void gemv_bf_body(const GemvBfArgs& a, int64_t grid_row) {
   using F = CodeFmt<VAR>;
   constexpr bool Q4 = F::kNibble;
   constexpr uint32_t kNc = 32u / D;  // classes per slot in one hash row
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
   const int crank = static_cast<int>(cluster.block_rank());
   int rb;
   int64_t code_base;
-  if (!rb_resolve(a.map, blockIdx.y, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
+  if (!rb_resolve(a.map, grid_row, static_cast<int64_t>(a.T) * F::kTileBytes, rb, code_base)) {
     if (threadIdx.x == 0 && crank == 0) report(a.status, USK_FLAG_RATE_MAP);
     return;  // the whole cluster (same grid row) leaves before any cluster barrier
   }
@@ -293,9 +294,26 @@ __global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a)
 }
 
 template <int B, int D, int VAR>
+__global__ void __launch_bounds__(kBfThreads) gemv_bf_kernel(const GemvBfArgs a) {
+  gemv_bf_body<B, D, VAR>(a, blockIdx.y);
+}
+
+// Per-row-block rates in one launch: grid row g is entry g of the rate map's
+// order list (grouped by slot count), so its code layout follows from g.
+template <int B>
+__global__ void __launch_bounds__(kBfThreads) gemv_bf_vr_kernel(const GemvBfArgs a) {
+  const int64_t g = blockIdx.y;
+  if (g < a.g1) gemv_bf_body<B, 1, 2>(a, g);
+  else if (g < a.g2) gemv_bf_body<B, 1, 0>(a, g);
+  else gemv_bf_body<B, 1, 3>(a, g);
+}
+
+template <int B, int D, int VAR>
 static cudaError_t launch_bf_t(GemvBfArgs a, int64_t nrb, cudaStream_t stream) {
-  const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D, CodeFmt<VAR>::kTileBf).total;
-  auto kern = gemv_bf_kernel<B, D, VAR>;
+  // a rate map: one launch over every row block, shared memory for 8 slots
+  const bool vr = a.map.order != nullptr;
+  const size_t smem = gemv_bf_layout(a.tpc, B, a.C, D, vr ? CodeFmt<3>::kTileBf : CodeFmt<VAR>::kTileBf).total;
+  auto kern = vr ? gemv_bf_vr_kernel<B> : gemv_bf_kernel<B, D, VAR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -344,10 +362,17 @@ bool gemv_bf_supported(int64_t K, int batch, int tpc_override) {
 
 cudaError_t launch_gemv_bf(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                            const uint16_t* x, int batch, float* y, uint32_t* status, bool pdl, cudaStream_t stream,
-                           int tpc_override, int inject, int depth, int var, const RbMap& map, int64_t nrb) {
+                           int tpc_override, int inject, int depth, int var, const RbMap& map, int64_t nrb,
+                           int64_t g1, int64_t g2) {
   GemvBfArgs a;
   a.map = map;
   a.map.RB = M / kRowsPerBlock;
+  a.g1 = g1;
+  a.g2 = g2;
+  if (map.order != nullptr) {  // the rate-map kernel covers every layout (depth 1)
+    var = 0;
+    depth = 1;
+  }
   a.codes = codes; a.scales = scales; a.x = x; a.y = y;
   a.M = M; a.K = K; a.seed = seed; a.status = status;
   a.T = static_cast<int>(K / kTileCols);

@@ -108,7 +108,7 @@ def test_vr_gemv_matches_oracle(slots, xdtype):
 @pytest.mark.parametrize("path", [1, 2, 3, 4])
 def test_vr_gemv_paths_and_pdl(path):
     """Forced paths: the integer paths read uniform 4-slot sketches only, so a
-    rate map takes a bf16 path; PDL launches of the groups give the same y."""
+    rate map takes a bf16 path; a PDL launch gives the same y."""
     slots = [8, 2, 4, 2, 8]
     W = gen.weights_student_t(320, 1024, 66, 4.0, 0.02, 0.001, 20.0, "bf16")
     sk, o = _oracle_sketch(W, None, 10, slots)
