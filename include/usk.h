@@ -141,7 +141,7 @@ typedef enum {
   USK_ERR_DTYPE = 3,           /* unknown usk_dtype                              */
   USK_ERR_BATCH = 4,           /* batch outside the call's range                 */
   USK_ERR_WORKSPACE = 5,       /* workspace missing or too small                 */
-  USK_ERR_PARAMS = 6,          /* params NULL, unknown format, bad depth or flags */
+  USK_ERR_PARAMS = 6,          /* params NULL, unknown format, bad depth, slots, flags or rate map */
   USK_ERR_CUDA = 7,            /* a CUDA runtime call or a launch failed         */
   USK_ERR_NONFINITE = 8,       /* (flag decoding) non-finite weight              */
   USK_ERR_TIMEOUT = 9,         /* (flag decoding) a bounded device wait gave up  */

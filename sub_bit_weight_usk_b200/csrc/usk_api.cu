@@ -145,8 +145,8 @@ USK_API const char* usk_status_str(usk_status status) {
     case USK_ERR_BATCH: return "batch outside the range of this call";
     case USK_ERR_WORKSPACE: return "workspace missing or too small";
     case USK_ERR_PARAMS:
-      return "params NULL, unknown format, bad depth, non-zero flags, importance with format 2 or 3, or usk_gemm "
-             "on a format-3 sketch";
+      return "params NULL, unknown format, bad depth or slot count, non-zero flags, importance with format 2 or 3, "
+             "a rate map that is not for format 1 or whose counts do not match, or usk_gemm on a format-3 sketch";
     case USK_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
     case USK_ERR_NONFINITE: return "non-finite weight";
     case USK_ERR_TIMEOUT: return "a bounded device wait gave up";
