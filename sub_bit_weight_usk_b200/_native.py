@@ -206,6 +206,14 @@ class RateMap:
     code_bytes: int
 
     def as_c(self) -> UskRateMapC:
+        n = len(self.slots)
+        for t, dt, name in ((self.offset, torch.int64, "offset"), (self.order, torch.int32, "order")):
+            if t.dtype != dt or not t.is_contiguous() or t.numel() != n:
+                raise ValueError("RateMap.%s must be a contiguous %s tensor of %d entries" % (name, dt, n))
+            if n and not t.is_cuda:
+                raise ValueError("RateMap.%s must be on the GPU (the kernels read it)" % name)
+        if sum(self.count) != n:
+            raise ValueError("RateMap.count must add up to the row blocks")
         c = UskRateMapC(self.offset.data_ptr() if self.offset.numel() else None,
                         self.order.data_ptr() if self.order.numel() else None)
         for g in range(3):

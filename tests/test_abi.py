@@ -211,3 +211,24 @@ def test_rate_map_argument_errors(lib):
         p = params(good, version, slots)
         assert lib.usk_build(fake, 1, 128, 256, 256, None, ctypes.byref(p), fake, fake, None, None) == 6
         assert lib.usk_gemv(ctypes.byref(sketch(good, version, slots)), fake, 1, 1, fake, None, None) == 6
+
+
+def test_rate_map_binding_checks(lib):
+    """The binding refuses rate tables that the kernels could not read."""
+    import torch
+    off, order, count, total = usk.usk_rate_map_plan(128, 256, [2, 8])
+    cpu = usk.RateMap([2, 8], torch.tensor(off, dtype=torch.int64), torch.tensor(order, dtype=torch.int32),
+                      count, total)
+    with pytest.raises(ValueError):
+        cpu.as_c()  # host tensors
+    wrong = usk.RateMap([2, 8], torch.tensor(off, dtype=torch.int32), torch.tensor(order, dtype=torch.int32),
+                        count, total)
+    with pytest.raises(ValueError):
+        wrong.as_c()
+    short = usk.RateMap([2, 8], torch.tensor(off[:1], dtype=torch.int64), torch.tensor(order, dtype=torch.int32),
+                        count, total)
+    with pytest.raises(ValueError):
+        short.as_c()
+    empty = usk.RateMap([], torch.zeros(0, dtype=torch.int64), torch.zeros(0, dtype=torch.int32), (0, 0, 0), 0)
+    c = empty.as_c()
+    assert c.code_bytes == 0 and list(c.count) == [0, 0, 0]
