@@ -49,7 +49,7 @@ def build(force: bool = False) -> str:
     """Compile usk_oracle.c into liboracle.so next to it (gcc, IEEE-strict)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".tmp.%d" % os.getpid()
-        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math",
+        cmd = ["gcc", "-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
                "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"]
         subprocess.check_call(cmd)
         os.replace(tmp, _LIB)
@@ -132,6 +132,12 @@ def _load():
         lib.orc_f32_to_f16_array.restype = None
         lib.orc_f16_to_f32_array.argtypes = [vp, vp, i64]
         lib.orc_f16_to_f32_array.restype = None
+        lib.orc_threads.argtypes = [ctypes.c_int]
+        lib.orc_threads.restype = ctypes.c_int
+        lib.orc_build_mt.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, u64, vp, vp, ctypes.c_int]
+        lib.orc_build_mt.restype = ctypes.c_int
+        lib.orc_gemv_f64_mt.argtypes = [vp, vp, i64, i64, u64, vp, ctypes.c_int, i64, vp, ctypes.c_int]
+        lib.orc_gemv_f64_mt.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -521,6 +527,45 @@ def gemv_f64(codes, scales, M, K, x, seed=0, rows=None):
                               _ptr(r), 0 if r is None else len(r), _ptr(y))
     if st:
         raise ValueError("orc_gemv_f64 status %d" % st)
+    return y
+
+
+def threads(n: int = 0) -> int:
+    """Host threads the all-core functions use for `n` (0 = all available)."""
+    return int(_load().orc_threads(int(n)))
+
+
+def build_sketch_mt(W, importance=None, seed=0, threads=0):
+    """build_sketch (format 1) with the row blocks spread over host threads:
+    the same sequential code per row block, so the same codes and scales.
+    Returns dict(status, codes, scales)."""
+    W, dt = _weights(W)
+    M, K = W.shape
+    imp = None if importance is None else np.ascontiguousarray(importance, dtype=np.float32)
+    nb = M * K // 16 if (M % 64 == 0 and K % 256 == 0 and M >= 0 and K >= 0) else 0
+    codes = np.empty(max(nb, 1), dtype=np.int8)
+    scales = np.zeros(max(M // 64, 1), dtype=np.uint16)
+    st = _load().orc_build_mt(_ptr(W), dt, M, K, K, _ptr(imp), seed, _ptr(codes), _ptr(scales), int(threads))
+    return {"status": st, "codes": codes[:nb], "scales": scales[: M // 64]}
+
+
+def gemv_f64_mt(codes, scales, M, K, x, seed=0, threads=0):
+    """gemv_f64 over all rows with runs of 64 rows spread over host threads
+    (the same float64 sums row by row)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint16)
+    x = np.ascontiguousarray(x)
+    if x.ndim == 1:
+        x = x[None, :]
+    xdt = F32 if x.dtype == np.float32 else BF16 if x.dtype == np.uint16 else None
+    if xdt is None:
+        raise TypeError("x must be float32 or uint16 (bf16 bits)")
+    batch = x.shape[0]
+    y = np.zeros((batch, M), dtype=np.float64)
+    st = _load().orc_gemv_f64_mt(_ptr(codes), _ptr(scales), M, K, seed, _ptr(x), xdt, batch, _ptr(y),
+                                 int(threads))
+    if st:
+        raise ValueError("orc_gemv_f64_mt status %d" % st)
     return y
 
 

@@ -1059,3 +1059,89 @@ int orc_vr_gemv_f64(const int8_t* codes, const uint16_t* scales, int64_t M, int6
   free(wrow);
   return ORC_OK;
 }
+
+/* ------------------------------------------------- all-core baseline mode */
+
+/* The same format-1 build and float64 product, spread over `nthreads` host
+ * threads (OpenMP; 0 = all the runtime offers) for the CPU baseline and for
+ * whole-model checks.  Nothing is recomputed differently: row blocks are
+ * independent in the method (a bucket's members all lie in one 64-row block,
+ * Metodologia §1 of the explainer, and the scale is per block), so each run of
+ * row blocks is handed, unchanged, to the sequential orc_build_rows /
+ * orc_gemv_f64 above.  The result is therefore identical to the single-thread
+ * call; the status is the one the sequential scan would return (a non-finite
+ * weight anywhere wins over a scale overflow).  Compiled without OpenMP the
+ * loops simply run on one thread. */
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int orc_threads(int nthreads) {
+#ifdef _OPENMP
+  return nthreads > 0 ? nthreads : omp_get_max_threads();
+#else
+  (void)nthreads;
+  return 1;
+#endif
+}
+
+int orc_build_mt(const void* W, int dtype, int64_t M, int64_t K, int64_t ldw,
+                 const float* imp, uint64_t seed, int8_t* codes, uint16_t* scales,
+                 int nthreads) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (dtype != 0 && dtype != 1) return ORC_ERR_DTYPE;
+  if (M == 0 || K == 0) return orc_build_rows(W, dtype, M, K, ldw, imp, seed, 0, codes, scales, NULL, NULL);
+  if (!W || !codes || !scales || ldw < K) return ORC_ERR_NULL;
+  const int64_t RB = M / ROWS_PER_BLOCK;
+  const size_t esz = dtype == 0 ? 4 : 2;
+  int any_nonfinite = 0, any_overflow = 0, any_other = 0;
+  int64_t rb;
+  (void)nthreads;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(orc_threads(nthreads)) \
+    reduction(| : any_nonfinite, any_overflow, any_other)
+  for (rb = 0; rb < RB; ++rb) {
+    const char* wrb = (const char*)W + (size_t)(rb * ROWS_PER_BLOCK) * (size_t)ldw * esz;
+    int s = orc_build_rows(wrb, dtype, ROWS_PER_BLOCK, K, ldw, imp, seed, rb, codes + rb * 4 * K, scales + rb,
+                           NULL, NULL);
+    if (s == ORC_ERR_NONFINITE) any_nonfinite = 1;
+    else if (s == ORC_ERR_SCALE_OVERFLOW) any_overflow = 1;
+    else if (s != ORC_OK) any_other = s;
+  }
+  if (any_other) return any_other; /* argument errors: the same for every row block */
+  if (any_nonfinite) return ORC_ERR_NONFINITE;
+  if (any_overflow) return ORC_ERR_SCALE_OVERFLOW;
+  return ORC_OK;
+}
+
+/* y [batch, M] = W_hat x^T in float64 over all rows, rows spread over threads in
+ * runs of 64; each run is one orc_gemv_f64 call on its row list. */
+int orc_gemv_f64_mt(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K,
+                    uint64_t seed, const void* x, int xdtype, int64_t batch, double* y,
+                    int nthreads) {
+  int st = check_shape(M, K);
+  if (st) return st;
+  if (xdtype != 0 && xdtype != 1) return ORC_ERR_DTYPE;
+  if (batch < 0) return ORC_ERR_SHAPE;
+  if (M == 0 || batch == 0) return ORC_OK;
+  if (!y) return ORC_ERR_NULL;
+  const int64_t RB = M / ROWS_PER_BLOCK;
+  int err = 0;
+  int64_t rb;
+  (void)nthreads;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(orc_threads(nthreads)) reduction(| : err)
+  for (rb = 0; rb < RB; ++rb) {
+    int64_t rows[ROWS_PER_BLOCK];
+    double part[ROWS_PER_BLOCK * 16];
+    for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) rows[r] = rb * ROWS_PER_BLOCK + r;
+    for (int64_t t0 = 0; t0 < batch; t0 += 16) {
+      const int64_t nb = batch - t0 < 16 ? batch - t0 : 16;
+      const char* xt = (const char*)x + (size_t)(t0 * K) * (size_t)(xdtype == 0 ? 4 : 2);
+      int s = orc_gemv_f64(codes, scales, M, K, seed, xt, xdtype, nb, rows, ROWS_PER_BLOCK, part);
+      if (s) { err |= s; continue; }
+      for (int64_t t = 0; t < nb; ++t)
+        for (int64_t r = 0; r < ROWS_PER_BLOCK; ++r) y[(t0 + t) * M + rows[r]] = part[t * ROWS_PER_BLOCK + r];
+    }
+  }
+  return err ? ORC_ERR_NULL : ORC_OK;
+}
