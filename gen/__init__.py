@@ -39,8 +39,9 @@ def rng(seed: int, stream: int) -> np.random.Generator:
 def f32_to_bf16_bits(a) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); uint16 bits."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    u = a.view(np.uint32)
+    # 32-bit arithmetic cannot wrap for non-NaN patterns (at most 0xFF807FFF)
+    r = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
     nan = np.isnan(a)
     if nan.any():
         r[nan] = 0x7FC0
