@@ -550,6 +550,7 @@ def run_usk(args):
     y1 = torch.empty((1, M), device=dev)
     y4 = torch.empty((4, M), device=dev)
     y16 = torch.empty((GEMM_BATCH, M), device=dev)
+    ws_lay = torch.zeros(usk.usk_gemv_multi_ws_bytes([sks[0]], 1), dtype=torch.uint8, device=dev)
 
     def lay_build(i):
         b = sks[i % N_SKETCHES]
@@ -560,7 +561,9 @@ def run_usk(args):
     add("layer", [("usk_build", lay_build, 1),
                   ("usk_gemv", lambda i: usk.usk_gemv(sks[(i + 128) % N_SKETCHES], x1, y=y1, pdl=True), 1),
                   ("usk_gemv_b4", lambda i: usk.usk_gemv(sks[(i + 160) % N_SKETCHES], x4, y=y4, pdl=True), 1),
-                  ("usk_gemm", lambda i: usk.usk_gemm(sks[(i + 64) % N_SKETCHES], x16, y=y16, status=status), 1)],
+                  ("usk_gemm", lambda i: usk.usk_gemm(sks[(i + 64) % N_SKETCHES], x16, y=y16, status=status), 1),
+                  ("usk_gemv_multi", lambda i: usk.usk_gemv_multi([sks[(i + 192) % N_SKETCHES]], [x1], [y1],
+                                                                  ws=ws_lay, pdl=True), 1)],
         None)
 
     # ---------------------------------------------------------- small (fp32 weights)
@@ -611,8 +614,29 @@ def run_usk(args):
         for e in stack:
             torch.mm(e["x1"], e["W"].t(), out=e["ybf"])
 
+    # the same token with usk_gemv_multi: per layer one launch each for the
+    # products a transformer's data flow leaves independent -- q, k, v (one
+    # input), o, gate and up (one input), down -- 128 launches per token, all
+    # sharing one workspace in stream order
+    groups = []
+    for layer in range(STACK_LAYERS):
+        es = [e for e in stack if e["layer"] == layer]
+        by = {e["name"]: e for e in es}
+        for names in (("q", "k", "v"), ("o",), ("gate", "up"), ("down",)):
+            groups.append([by[nm] for nm in names])
+    ws_tok = torch.zeros(max(usk.usk_gemv_multi_ws_bytes([e["sk"] for e in g_], 1) for g_ in groups),
+                         dtype=torch.uint8, device=dev)
+    calls = [(usk.MultiCall([e["sk"] for e in g_], [e["x1"] for e in g_], [e["y"][:1] for e in g_]), g_)
+             for g_ in groups]
+
+    def stack_token_multi(i):
+        for c, g_ in calls:
+            usk.usk_gemv_multi([e["sk"] for e in g_], [e["x1"] for e in g_], [e["y"][:1] for e in g_], ws=ws_tok,
+                               pdl=True, call=c)
+
     n_lin = len(stack)
     add("stack7b", [("model_build", stack_build, n_lin), ("token_decode", stack_token, n_lin),
+                    ("token_decode_grouped", stack_token_multi, len(groups)),
                     ("token_dense_bf16_torch", stack_dense, n_lin, False)], None)
 
     # 7B layer set: per shape, cycling over the stack's linears of that shape
@@ -639,8 +663,19 @@ def run_usk(args):
             e = lst[(i + 3 * n // 4) % n]
             usk.usk_gemm(e["sk"], e["x16"], y=e["y"], status=status)
 
+        ws_s = torch.zeros(max(16, usk.usk_gemv_multi_ws_bytes([lst[0]["sk"]], 4)), dtype=torch.uint8, device=dev)
+
+        def gm1(i, lst=lst, n=n, ws_s=ws_s):
+            e = lst[(i + n // 2) % n]
+            usk.usk_gemv_multi([e["sk"]], [e["x1"]], [e["y"][:1]], ws=ws_s, pdl=True)
+
+        def gm4(i, lst=lst, n=n, ws_s=ws_s):
+            e = lst[(i + n // 4) % n]
+            usk.usk_gemv_multi([e["sk"]], [e["x4"]], [e["y"][:4]], ws=ws_s, pdl=True)
+
         set_phases += [(shp + "/usk_build", b_, 1), (shp + "/usk_gemv_b1", g1, 1), (shp + "/usk_gemv_b4", g4, 1),
-                       (shp + "/usk_gemm_b16", gm, 1)]
+                       (shp + "/usk_gemm_b16", gm, 1), (shp + "/usk_gemv_multi_b1", gm1, 1),
+                       (shp + "/usk_gemv_multi_b4", gm4, 1)]
     add("llama7b_set", set_phases, None)
 
     # ---------------------------------------------------------- 70B MLP shapes
@@ -667,6 +702,12 @@ def run_usk(args):
             usk.usk_gemv(e["sks"][(i + 5) % AB_COPIES], xs[1], y=e["y"][:1], pdl=True)
 
         mlp_phases.append((shp + "/usk_gemv_b1", mg1, 1))
+        ws_m = torch.zeros(max(16, usk.usk_gemv_multi_ws_bytes([e["sks"][0]], 1)), dtype=torch.uint8, device=dev)
+
+        def mgm1(i, e=e, xs=xs, ws_m=ws_m):
+            usk.usk_gemv_multi([e["sks"][(i + 7) % AB_COPIES]], [xs[1]], [e["y"][:1]], ws=ws_m, pdl=True)
+
+        mlp_phases.append((shp + "/usk_gemv_multi_b1", mgm1, 1))
         for bb in (16, 32, 64):
             def mgm(i, e=e, xs=xs, bb=bb):
                 usk.usk_gemm(e["sks"][(i + bb) % AB_COPIES], xs[bb], y=e["y"][:bb], status=status)
@@ -809,6 +850,7 @@ def run_usk(args):
     agg = aggregate(world, [t_gemv], [t_build], [t_step])
     rl = rooflines(peaks, t_build, t_gemv, t_gemm, tr)
     rl["usk_gemv_b4"] = R.gather_line(gemv_bytes(M, K, 4), N_W, t_gemv4)
+    rl["usk_gemv_multi"] = R.gather_line(GEMV_BYTES, N_W, L["usk_gemv_multi"])
     e2e_bytes_c = (c_e2e or {}).get("h2d_bytes", 2 * K) + (c_e2e or {}).get("d2h_bytes", 4 * M)
     clocks = sampler.summary()
     info = cpu_info()
@@ -839,7 +881,7 @@ def run_usk(args):
                    "parallelism": "replicas" if world > 1 else "single"},
         "usk_build_gweights_per_s": round(agg["build_gweights_s"], 3),
         "kernel_us": {"usk_build": _us(t_build), "usk_gemv": _us(t_gemv), "usk_gemv_b4": _us(t_gemv4),
-                      "usk_gemm": _us(t_gemm)},
+                      "usk_gemm": _us(t_gemm), "usk_gemv_multi": _us(L["usk_gemv_multi"])},
         "spread": _spread(times["layer"]),
         "roofline": rl["usk_gemv"],
         "rooflines": rl,
@@ -889,7 +931,8 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
     # 7B layer set
     st = med["llama7b_set"]
     shapes = {"4096x4096": (4096, 4096, 4), "11008x4096": (11008, 4096, 2), "4096x11008": (4096, 11008, 1)}
-    per_shape, totals = {}, {"usk_build": 0.0, "usk_gemv_b1": 0.0, "usk_gemv_b4": 0.0, "usk_gemm_b16": 0.0}
+    per_shape, totals = {}, {"usk_build": 0.0, "usk_gemv_b1": 0.0, "usk_gemv_b4": 0.0, "usk_gemm_b16": 0.0,
+                             "usk_gemv_multi_b1": 0.0, "usk_gemv_multi_b4": 0.0}
     n_set = 0
     for shp, (m, k, cnt) in shapes.items():
         d = {c: st[shp + "/" + c] for c in totals}
@@ -902,7 +945,9 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
                           "usk_gemv_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_b1"]),
                           "usk_gemv_b4": R.gather_line(gemv_bytes(m, k, 4), m * k, d["usk_gemv_b4"]),
                           "usk_gemm_b16": R.gather_line(gemv_bytes(m, k, 16), m * k, d["usk_gemm_b16"],
-                                                        flops=2 * m * k * 16)}}
+                                                        flops=2 * m * k * 16),
+                          "usk_gemv_multi_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_multi_b1"]),
+                          "usk_gemv_multi_b4": R.gather_line(gemv_bytes(m, k, 4), m * k, d["usk_gemv_multi_b4"])}}
     out["llama7b_set"] = {
         "workload": "Llama-7B-shaped layer set: q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008, bf16 "
                     "N(0, 0.02^2) (device-drawn), no importance; each shape's calls cycle over the 32 layers' "
@@ -922,7 +967,8 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
             "kernel_us": {c: _us(v) for c, v in d.items()},
             "usk_build_gweights_per_s": round(world * m * k / d["usk_build"] / 1e9, 3),
             "rooflines": {"usk_build": R.hbm_line(build_bytes(m, k, 2, False), d["usk_build"]),
-                          "usk_gemv_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_b1"])},
+                          "usk_gemv_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_b1"]),
+                          "usk_gemv_multi_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_multi_b1"])},
         }
         for bb in (16, 32, 64):
             t = d["usk_gemm_b%d" % bb]
@@ -941,6 +987,7 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
     tok_bytes = sum(gemv_bytes(m, k, 1) for m, k in gen.LLAMA7B_SHAPES.values()) * STACK_LAYERS
     dense_bytes = sum(2 * m * k + 2 * k + 2 * m for m, k in gen.LLAMA7B_SHAPES.values()) * STACK_LAYERS
     t_tok, t_dense, t_mb = s7["token_decode"], s7["token_dense_bf16_torch"], s7["model_build"]
+    t_tokg = s7["token_decode_grouped"]
     out["stack7b"] = {
         "workload": "32-layer 7B-shaped stack, 224 linears (q/k/v/o 4096x4096, gate/up 11008x4096, down "
                     "4096x11008 per layer), %.3f G weights, bf16 N(0, 0.02^2) device-drawn, one seed per linear; "
@@ -954,6 +1001,12 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
         "token_decode_roofline": dict(R.gather_line(tok_bytes, n_stack, t_tok),
                                       survey_issue_roof_ms=0.87),
         "tokens_per_s": round(1.0 / t_tok, 2),
+        "token_decode_grouped_ms": round(t_tokg * 1e3, 4),
+        "token_decode_grouped_us_per_linear": round(t_tokg / 224 * 1e6, 3),
+        "token_decode_grouped_roofline": R.gather_line(tok_bytes, n_stack, t_tokg),
+        "token_decode_grouped_vs_dense_speedup": round(t_dense / t_tokg, 3),
+        "grouped": "usk_gemv_multi, one launch per group of products a transformer's data flow leaves "
+                   "independent: (q, k, v), (o), (gate, up), (down) -- 128 launches per token",
         "dense_bf16_torch_token_ms": round(t_dense * 1e3, 4),
         "dense_bf16_torch_hbm_frac": round(dense_bytes / t_dense / R.hbm, 4),
         "decode_vs_dense_speedup": round(t_dense / t_tok, 3),

@@ -286,6 +286,40 @@ USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype x
 USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
                                float* y, uint32_t flags, uint32_t* d_status, void* stream);
 
+/* Several independent products in one launch (Metodologia §4, as usk_gemv):
+ * y[l] = W_hat_l x[l] for l < n, n in 0..16, batch 0..8, bf16 x only.
+ * A persistent kernel streams every 64-row x 1024-column piece of every
+ * sketch through shared memory with bulk copies a few pieces ahead of the
+ * math, so the copies of one piece (and of the next sketch) overlap the math
+ * of others; a row whose K spans several pieces is summed through the
+ * workspace in a fixed order (deterministic for a given list of shapes).
+ *   sketches  n sketches (host array), one format, depth and slot count among
+ *             them: format 1 (any slot count), 2 or 4; no rate map; format 3
+ *             is usk_gemv only (USK_ERR_PARAMS).
+ *   x, y      HOST arrays of n DEVICE pointers: x[l] [batch, K_l] bf16,
+ *             16-byte aligned; y[l] [batch, M_l] fp32.  The products must be
+ *             independent: no y[l] may overlap another y or any x.
+ *   ws        caller-owned device workspace of at least the bytes
+ *             usk_gemv_multi_ws_bytes returns for the same list and batch
+ *             (0 when every K <= 1024; ws may then be NULL), 16-byte aligned,
+ *             zero-filled before its first use.  It starts with one arrival
+ *             counter per split row block, which every call that completes
+ *             without USK_FLAG_TIMEOUT returns to zero, then the partial sums,
+ *             which need no clearing; so calls that follow one another in a
+ *             stream can share it, while calls that may run at the same time
+ *             need one each.  After a timeout, fill it with zeros again.
+ *   flags     USK_GEMV_PDL as in usk_gemv_ex: the first pieces' codes are
+ *             fetched before the previous kernel in the stream completes (x,
+ *             y and ws only after it).  Other bits: USK_ERR_PARAMS.
+ * Errors: USK_ERR_SHAPE (n), USK_ERR_BATCH, USK_ERR_DTYPE (fp32 x),
+ * USK_ERR_PARAMS, USK_ERR_NULL, USK_ERR_ALIGN, USK_ERR_WORKSPACE (ws missing or
+ * smaller than required).  Sketches with M == 0 are skipped; K == 0 writes
+ * y[l] = 0. */
+USK_API usk_status usk_gemv_multi_ws_bytes(int64_t n, const usk_sketch* sketches, int64_t batch, size_t* ws_bytes);
+USK_API usk_status usk_gemv_multi(int64_t n, const usk_sketch* sketches, const void* const* x, usk_dtype xdtype,
+                                  int64_t batch, float* const* y, void* ws, size_t ws_bytes, uint32_t flags,
+                                  uint32_t* d_status, void* stream);
+
 /* y = W_hat x for batch 16..256 (multiple of 16) on the tcgen05 tensor cores:
  * decoded bf16 tiles of W_hat are written to tensor memory and multiplied with
  * bf16 x tiles (copied into shared memory by the tensor memory accelerator),
@@ -319,9 +353,10 @@ USK_API void usk_debug_set_gemv_path(int path);
 USK_API void usk_debug_set_gemv_rows(int rows);
 
 /* Test hook for the failure path (host-made; no device fault): kernel = 1 makes
- * usk_build, 2 usk_gemm, 3 usk_gemv skip one bulk or tensor copy in thread
- * block (0, 0) (for the usk_gemv path without copies: the partial sums of
- * block 1 of row block 0), so a bounded wait gives up after about 1 s and sets
+ * usk_build, 2 usk_gemm, 3 usk_gemv, 4 usk_gemv_multi skip one bulk or tensor
+ * copy in thread block (0, 0) (for the usk_gemv path without copies: the
+ * partial sums of block 1 of row block 0), so a bounded wait gives up after
+ * about 1 s and sets
  * USK_FLAG_TIMEOUT; the kernel still completes and the context stays usable.
  * 0 switches it off.  Process-wide. */
 USK_API void usk_debug_inject_timeout(int kernel);

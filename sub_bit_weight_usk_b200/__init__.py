@@ -7,7 +7,8 @@ column-shared projection W_hat = S . P^T, multiplied as S (P^T x); format 4:
 format 1 with 4-bit codes and 8 weights per bucket; format 1 at 2, 4 or 8 hash
 slots per class, per sketch or per 64-row block); ``usk_gemv`` (batch 1-15)
 and ``usk_gemm`` (batch 16-256) multiply the sketch with activations, rebuilding
-every weight on the fly.  PyTorch supplies device memory and streams only.
+every weight on the fly; ``usk_gemv_multi`` runs several independent batch 1-8
+products in one persistent launch.  PyTorch supplies device memory and streams only.
 """
 from ._native import (  # noqa: F401
     FLAG_BAD_IMPORTANCE,
@@ -36,6 +37,9 @@ from ._native import (  # noqa: F401
     usk_format_version,
     usk_gemm,
     usk_gemv,
+    usk_gemv_multi,
+    usk_gemv_multi_ws_bytes,
+    MultiCall,
     usk_plan_slots,
     usk_rate_map,
     usk_rate_map_plan,

@@ -66,7 +66,8 @@ class UskSketchC(ctypes.Structure):
 
 _lib = None
 
-EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_rate_map_plan", "usk_build", "usk_gemv", "usk_gemv_ex", "usk_gemm", "usk_status_str",
+EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_rate_map_plan", "usk_build", "usk_gemv", "usk_gemv_ex",
+            "usk_gemv_multi", "usk_gemv_multi_ws_bytes", "usk_gemm", "usk_status_str",
             "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_set_gemv_rows",
             "usk_debug_inject_timeout"]
 GEMV_PDL = 1
@@ -99,6 +100,11 @@ def load_library(path: str = LIB_PATH):
     lib.usk_gemv.restype = ctypes.c_int
     lib.usk_gemv_ex.argtypes = [ctypes.POINTER(UskSketchC), vp, ctypes.c_int, i64, vp, ctypes.c_uint32, vp, vp]
     lib.usk_gemv_ex.restype = ctypes.c_int
+    lib.usk_gemv_multi_ws_bytes.argtypes = [i64, ctypes.POINTER(UskSketchC), i64, ctypes.POINTER(ctypes.c_size_t)]
+    lib.usk_gemv_multi_ws_bytes.restype = ctypes.c_int
+    lib.usk_gemv_multi.argtypes = [i64, ctypes.POINTER(UskSketchC), ctypes.POINTER(vp), ctypes.c_int, i64,
+                                   ctypes.POINTER(vp), vp, ctypes.c_size_t, ctypes.c_uint32, vp, vp]
+    lib.usk_gemv_multi.restype = ctypes.c_int
     lib.usk_gemm.argtypes = [ctypes.POINTER(UskSketchC), vp, i64, vp, vp, ctypes.c_size_t, vp, vp]
     lib.usk_gemm.restype = ctypes.c_int
     lib.usk_status_str.argtypes = [ctypes.c_int]
@@ -311,6 +317,56 @@ def usk_gemv(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
                                     GEMV_PDL if pdl else 0, _ptr(status), _stream(stream))
     _check(st, "usk_gemv")
     return y
+
+
+class MultiCall:
+    """Marshalled arguments of one usk_gemv_multi list (built once, reusable:
+    the ctypes arrays stay alive with this object)."""
+
+    def __init__(self, sketches, xs, ys):
+        n = len(sketches)
+        self.n = n
+        self._c = [sk.as_c() for sk in sketches]
+        self.sk = (UskSketchC * max(n, 1))(*self._c)
+        self.x = (ctypes.c_void_p * max(n, 1))(*[x.data_ptr() for x in xs])
+        self.y = (ctypes.c_void_p * max(n, 1))(*[y.data_ptr() for y in ys])
+
+
+def usk_gemv_multi_ws_bytes(sketches, batch: int) -> int:
+    """Workspace bytes usk_gemv_multi needs for this list of sketches and batch."""
+    n = len(sketches)
+    arr = (UskSketchC * max(n, 1))(*[sk.as_c() for sk in sketches])
+    out = ctypes.c_size_t()
+    _check(load_library().usk_gemv_multi_ws_bytes(n, arr, int(batch), ctypes.byref(out)), "usk_gemv_multi_ws_bytes")
+    return out.value
+
+
+def usk_gemv_multi(sketches, xs, ys=None, ws: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                   stream=None, pdl: bool = False, call: MultiCall | None = None):
+    """y[l] = W_hat_l x[l]^T for several sketches in one launch (batch 1..8, bf16
+    x).  ys are allocated when not given.  ws: a zero-filled uint8 CUDA tensor of
+    at least usk_gemv_multi_ws_bytes bytes (allocated with torch.zeros when None;
+    pass the same one to consecutive calls on a stream).  Returns ys."""
+    xs = [x if x.dim() == 2 else x[None, :] for x in xs]
+    _need_cuda(*xs, ws, status)
+    for x in xs:
+        if x.dtype != torch.bfloat16 or not x.is_contiguous():
+            raise TypeError("usk_gemv_multi takes contiguous bfloat16 x")
+    batch = xs[0].shape[0] if xs else 0
+    if any(x.shape[0] != batch for x in xs):
+        raise ValueError("every x of one call has the same batch")
+    if ys is None:
+        ys = [torch.empty((batch, sk.M), dtype=torch.float32, device=x.device) for sk, x in zip(sketches, xs)]
+    if ws is None:
+        need = usk_gemv_multi_ws_bytes(sketches, batch)
+        ws = torch.zeros(max(need, 16), dtype=torch.uint8, device=xs[0].device) if xs else None
+    if call is None:
+        call = MultiCall(sketches, xs, ys)
+    st = load_library().usk_gemv_multi(call.n, call.sk, call.x, USK_BF16, batch, call.y, _ptr(ws),
+                                       ws.numel() if ws is not None else 0, GEMV_PDL if pdl else 0, _ptr(status),
+                                       _stream(stream))
+    _check(st, "usk_gemv_multi")
+    return ys
 
 
 def usk_gemm(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,

@@ -32,6 +32,11 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
                         int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2);
 bool gemm_supported(int64_t K, int batch, int depth, int var);
+size_t gemv_multi_ws_bytes(int n, const int64_t* Ms, const int64_t* Ks, int batch, int depth, int var);
+cudaError_t launch_gemv_multi(int n, const int8_t* const* codes, const uint16_t* const* scales, const int64_t* Ms,
+                              const int64_t* Ks, const uint64_t* seeds, const uint16_t* const* x, float* const* y,
+                              int batch, void* ws, uint32_t* status, bool pdl, cudaStream_t stream, int inject,
+                              int depth, int var);
 }  // namespace usk
 
 namespace {
@@ -128,7 +133,36 @@ int g_build_cluster = 0;
 int g_gemv_tiles_per_block = 0;
 int g_gemv_path = 0;
 int g_gemv_rows = 0;
-int g_inject = 0;  // 1 build, 2 gemm, 3 gemv (integer path): skip one copy/commit in block (0, 0)
+int g_inject = 0;  // 1 build, 2 gemm, 3 gemv, 4 gemv_multi: skip one copy/commit in block (0, 0)
+
+constexpr int64_t kMultiMax = 16;  // sketches per usk_gemv_multi launch
+
+// Checks of a usk_gemv_multi list shared by the call and its workspace query:
+// every sketch valid, one format / depth / slot count, no rate map, not format
+// 3.  Fills the shapes of the sketches that have work (M > 0 and K > 0).
+usk_status check_multi(int64_t n, const usk_sketch* sk, int64_t batch, int64_t* Ms, int64_t* Ks, int* idx,
+                       int* nwork) {
+  if (n < 0 || n > kMultiMax) return USK_ERR_SHAPE;
+  if (batch < 0 || batch > 8) return USK_ERR_BATCH;
+  *nwork = 0;
+  if (n == 0) return USK_OK;
+  if (!sk) return USK_ERR_NULL;
+  for (int64_t l = 0; l < n; ++l) {
+    usk_status st = check_sketch(&sk[l]);
+    if (st != USK_OK) return st;
+    if (sk[l].rates || sk[l].version == USK_FORMAT_COLSHARED) return USK_ERR_PARAMS;
+    if (format_depth(sk[l].version, sk[l].depth) != format_depth(sk[0].version, sk[0].depth) ||
+        layout_of(sk[l].version, sk[l].slots) != layout_of(sk[0].version, sk[0].slots))
+      return USK_ERR_PARAMS;
+    if (sk[l].M > 0 && sk[l].K > 0) {
+      Ms[*nwork] = sk[l].M;
+      Ks[*nwork] = sk[l].K;
+      idx[*nwork] = static_cast<int>(l);
+      ++*nwork;
+    }
+  }
+  return USK_OK;
+}
 
 }  // namespace
 
@@ -366,6 +400,76 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
                                    static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, layout, l.map,
                                    l.nrb, l.g1, l.g2);
+  if (e != cudaSuccess) return USK_ERR_CUDA;
+  return from_cuda(cudaGetLastError());
+}
+
+USK_API usk_status usk_gemv_multi_ws_bytes(int64_t n, const usk_sketch* sketches, int64_t batch, size_t* ws_bytes) {
+  int64_t Ms[kMultiMax], Ks[kMultiMax];
+  int idx[kMultiMax], nw = 0;
+  usk_status st = check_multi(n, sketches, batch, Ms, Ks, idx, &nw);
+  if (st != USK_OK) return st;
+  if (!ws_bytes) return USK_ERR_NULL;
+  const usk_sketch* k0 = nw > 0 ? &sketches[idx[0]] : nullptr;
+  *ws_bytes = (nw > 0 && batch > 0) ? usk::gemv_multi_ws_bytes(nw, Ms, Ks, static_cast<int>(batch),
+                                                              format_depth(k0->version, k0->depth),
+                                                              layout_of(k0->version, k0->slots))
+                                    : 0;
+  return USK_OK;
+}
+
+USK_API usk_status usk_gemv_multi(int64_t n, const usk_sketch* sketches, const void* const* x, usk_dtype xdtype,
+                                  int64_t batch, float* const* y, void* ws, size_t ws_bytes, uint32_t flags,
+                                  uint32_t* d_status, void* stream) {
+  int64_t Ms[kMultiMax], Ks[kMultiMax];
+  int idx[kMultiMax], nw = 0;
+  usk_status st = check_multi(n, sketches, batch, Ms, Ks, idx, &nw);
+  if (st != USK_OK) return st;
+  if (xdtype != USK_BF16) return USK_ERR_DTYPE;  // fp32 x: usk_gemv
+  if ((flags & ~static_cast<uint32_t>(USK_GEMV_PDL)) != 0) return USK_ERR_PARAMS;
+  if (n == 0 || batch == 0) return USK_OK;
+  if (!x || !y) return USK_ERR_NULL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int64_t l = 0; l < n; ++l) {
+    if (sketches[l].M == 0) continue;
+    if (!y[l]) return USK_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(y[l]) & 3u) != 0) return USK_ERR_ALIGN;
+    if (sketches[l].K == 0) continue;
+    if (!x[l]) return USK_ERR_NULL;
+    if (!aligned16(x[l])) return USK_ERR_ALIGN;
+  }
+  const usk_sketch* kw = nw > 0 ? &sketches[idx[0]] : nullptr;
+  const size_t need = nw > 0 ? usk::gemv_multi_ws_bytes(nw, Ms, Ks, static_cast<int>(batch),
+                                                        format_depth(kw->version, kw->depth),
+                                                        layout_of(kw->version, kw->slots))
+                             : 0;
+  if (need > 0) {
+    if (!ws || ws_bytes < need) return USK_ERR_WORKSPACE;
+    if (!aligned16(ws)) return USK_ERR_ALIGN;
+  }
+  for (int64_t l = 0; l < n; ++l)  // K == 0: y = 0
+    if (sketches[l].M > 0 && sketches[l].K == 0) {
+      cudaError_t e = cudaMemsetAsync(y[l], 0, sizeof(float) * static_cast<size_t>(batch * sketches[l].M), s);
+      if (e != cudaSuccess) return USK_ERR_CUDA;
+    }
+  if (nw == 0) return USK_OK;
+  const int8_t* codes[kMultiMax];
+  const uint16_t* scales[kMultiMax];
+  const uint16_t* xs[kMultiMax];
+  float* ys[kMultiMax];
+  uint64_t seeds[kMultiMax];
+  for (int w = 0; w < nw; ++w) {
+    const usk_sketch& k = sketches[idx[w]];
+    codes[w] = k.codes;
+    scales[w] = k.scales;
+    seeds[w] = k.seed;
+    xs[w] = static_cast<const uint16_t*>(x[idx[w]]);
+    ys[w] = y[idx[w]];
+  }
+  const usk_sketch& k0 = sketches[idx[0]];
+  cudaError_t e = usk::launch_gemv_multi(nw, codes, scales, Ms, Ks, seeds, xs, ys, static_cast<int>(batch), ws,
+                                         d_status, (flags & USK_GEMV_PDL) != 0, s, g_inject == 4,
+                                         format_depth(k0.version, k0.depth), layout_of(k0.version, k0.slots));
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
