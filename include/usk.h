@@ -320,6 +320,35 @@ USK_API usk_status usk_gemv_multi(int64_t n, const usk_sketch* sketches, const v
                                   int64_t batch, float* const* y, void* ws, size_t ws_bytes, uint32_t flags,
                                   uint32_t* d_status, void* stream);
 
+/* usk_gemv_multi for callers that may not allocate device memory: the same
+ * products, with the scratch the call needs (the arrival counters and partial
+ * sums of split rows) held in a fixed array inside the library instead of a
+ * caller workspace.  Meant for code that runs where allocation is not an
+ * option -- a plug-in or an inference engine that hands this library only
+ * its input and output buffers and owns every other byte of device memory,
+ * or a real-time loop that must not call cudaMalloc after start-up (it can
+ * synchronise the device and its time is unbounded).  The paper has no
+ * counterpart; this is a calling convention of the library.
+ *   Arguments, results, formats and errors as usk_gemv_multi, without ws.
+ *   The fixed array holds USK_GEMV_MULTI_STATIC_BYTES bytes on every device
+ *   that loads the library, from load until the process exits.  A list whose
+ *   workspace (usk_gemv_multi_ws_bytes for the same list and batch) is larger
+ *   is refused with USK_ERR_WORKSPACE before anything is launched (for
+ *   instance one 4096 x 4096 sketch at batch 8 on a 148-SM B200, whose rows
+ *   split into 4 pieces: 512 KiB of partial sums plus the counters).
+ *   The call allocates nothing: it makes no cudaMalloc, cudaFree or other
+ *   allocating call.  Its first call on a device looks up the array's device
+ *   address (cudaGetSymbolAddress, with that device current); make that first
+ *   call before any stream capture.  Each call first clears the counters on
+ *   `stream` (cudaMemsetAsync), then launches.
+ *   Every call shares the one array: calls that may overlap on the GPU (other
+ *   streams, other threads, concurrent graph branches) race on it and give
+ *   wrong results; keep them in one stream order. */
+#define USK_GEMV_MULTI_STATIC_BYTES (512u * 1024u)
+USK_API usk_status usk_gemv_multi_static(int64_t n, const usk_sketch* sketches, const void* const* x,
+                                         usk_dtype xdtype, int64_t batch, float* const* y, uint32_t flags,
+                                         uint32_t* d_status, void* stream);
+
 /* y = W_hat x for batch 16..256 (multiple of 16) on the tcgen05 tensor cores:
  * decoded bf16 tiles of W_hat are written to tensor memory and multiplied with
  * bf16 x tiles (copied into shared memory by the tensor memory accelerator),

@@ -67,7 +67,7 @@ class UskSketchC(ctypes.Structure):
 _lib = None
 
 EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_rate_map_plan", "usk_build", "usk_gemv", "usk_gemv_ex",
-            "usk_gemv_multi", "usk_gemv_multi_ws_bytes", "usk_gemm", "usk_status_str",
+            "usk_gemv_multi", "usk_gemv_multi_ws_bytes", "usk_gemv_multi_static", "usk_gemm", "usk_status_str",
             "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_set_gemv_rows",
             "usk_debug_inject_timeout"]
 GEMV_PDL = 1
@@ -105,6 +105,9 @@ def load_library(path: str = LIB_PATH):
     lib.usk_gemv_multi.argtypes = [i64, ctypes.POINTER(UskSketchC), ctypes.POINTER(vp), ctypes.c_int, i64,
                                    ctypes.POINTER(vp), vp, ctypes.c_size_t, ctypes.c_uint32, vp, vp]
     lib.usk_gemv_multi.restype = ctypes.c_int
+    lib.usk_gemv_multi_static.argtypes = [i64, ctypes.POINTER(UskSketchC), ctypes.POINTER(vp), ctypes.c_int, i64,
+                                          ctypes.POINTER(vp), ctypes.c_uint32, vp, vp]
+    lib.usk_gemv_multi_static.restype = ctypes.c_int
     lib.usk_gemm.argtypes = [ctypes.POINTER(UskSketchC), vp, i64, vp, vp, ctypes.c_size_t, vp, vp]
     lib.usk_gemm.restype = ctypes.c_int
     lib.usk_status_str.argtypes = [ctypes.c_int]

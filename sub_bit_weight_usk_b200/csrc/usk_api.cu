@@ -37,6 +37,10 @@ cudaError_t launch_gemv_multi(int n, const int8_t* const* codes, const uint16_t*
                               const int64_t* Ks, const uint64_t* seeds, const uint16_t* const* x, float* const* y,
                               int batch, void* ws, uint32_t* status, bool pdl, cudaStream_t stream, int inject,
                               int depth, int var);
+cudaError_t launch_gemv_multi_static(int n, const int8_t* const* codes, const uint16_t* const* scales,
+                                     const int64_t* Ms, const int64_t* Ks, const uint64_t* seeds,
+                                     const uint16_t* const* x, float* const* y, int batch, uint32_t* status, bool pdl,
+                                     cudaStream_t stream, int depth, int var);
 }  // namespace usk
 
 namespace {
@@ -474,7 +478,61 @@ USK_API usk_status usk_gemv_multi(int64_t n, const usk_sketch* sketches, const v
   return from_cuda(cudaGetLastError());
 }
 
-// Test hooks: launch-geometry overrides (0 restores the defaults).  They change
+USK_API usk_status usk_gemv_multi_static(int64_t n, const usk_sketch* sketches, const void* const* x,
+                                         usk_dtype xdtype, int64_t batch, float* const* y, uint32_t flags,
+                                         uint32_t* d_status, void* stream) {
+  int64_t Ms[kMultiMax], Ks[kMultiMax];
+  int idx[kMultiMax], nw = 0;
+  usk_status st = check_multi(n, sketches, batch, Ms, Ks, idx, &nw);
+  if (st != USK_OK) return st;
+  if (xdtype != USK_BF16) return USK_ERR_DTYPE;
+  if ((flags & ~static_cast<uint32_t>(USK_GEMV_PDL)) != 0) return USK_ERR_PARAMS;
+  if (n == 0 || batch == 0) return USK_OK;
+  if (!x || !y) return USK_ERR_NULL;
+  for (int64_t l = 0; l < n; ++l) {
+    if (sketches[l].M == 0) continue;
+    if (!y[l]) return USK_ERR_NULL;
+    if ((reinterpret_cast<uintptr_t>(y[l]) & 3u) != 0) return USK_ERR_ALIGN;
+    if (sketches[l].K == 0) continue;
+    if (!x[l]) return USK_ERR_NULL;
+    if (!aligned16(x[l])) return USK_ERR_ALIGN;
+  }
+  int depth = 1, layout = 0;
+  if (nw > 0) {
+    const usk_sketch& k0 = sketches[idx[0]];
+    depth = format_depth(k0.version, k0.depth);
+    layout = layout_of(k0.version, k0.slots);
+    // the list's scratch must fit the library's fixed array
+    if (usk::gemv_multi_ws_bytes(nw, Ms, Ks, static_cast<int>(batch), depth, layout) > USK_GEMV_MULTI_STATIC_BYTES)
+      return USK_ERR_WORKSPACE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int64_t l = 0; l < n; ++l)  // K == 0: y = 0
+    if (sketches[l].M > 0 && sketches[l].K == 0) {
+      cudaError_t e = cudaMemsetAsync(y[l], 0, sizeof(float) * static_cast<size_t>(batch * sketches[l].M), s);
+      if (e != cudaSuccess) return USK_ERR_CUDA;
+    }
+  if (nw == 0) return USK_OK;
+  const int8_t* codes[kMultiMax];
+  const uint16_t* scales[kMultiMax];
+  const uint16_t* xs[kMultiMax];
+  float* ys[kMultiMax];
+  uint64_t seeds[kMultiMax];
+  for (int w = 0; w < nw; ++w) {
+    const usk_sketch& k = sketches[idx[w]];
+    codes[w] = k.codes;
+    scales[w] = k.scales;
+    seeds[w] = k.seed;
+    xs[w] = static_cast<const uint16_t*>(x[idx[w]]);
+    ys[w] = y[idx[w]];
+  }
+  cudaError_t e = usk::launch_gemv_multi_static(nw, codes, scales, Ms, Ks, seeds, xs, ys, static_cast<int>(batch),
+                                                d_status, (flags & USK_GEMV_PDL) != 0, s, depth, layout);
+  if (e != cudaSuccess) return USK_ERR_CUDA;
+  return from_cuda(cudaGetLastError());
+}
+
+// Test hooks: launch-geometry overrides// Test hooks: launch-geometry overrides (0 restores the defaults).  They change
 // how work is split between thread blocks, never the result.
 USK_API void usk_debug_set_geometry(int build_cluster, int gemv_tiles_per_block) {
   g_build_cluster = build_cluster;

@@ -39,6 +39,7 @@
 //    before it leaves; that call's outputs and workspace counters are then
 //    undefined.
 #include <cuda/atomic>
+#include <mutex>
 
 #include "usk_common.cuh"
 
@@ -633,6 +634,63 @@ cudaError_t launch_gemv_multi(int n, const int8_t* const* codes, const uint16_t*
   if (depth == 2) return ml_launch_b<2, 0>(a, slots, stream);
   if (depth == 4) return ml_launch_b<4, 0>(a, slots, stream);
   return ml_launch_b<1, 0>(a, slots, stream);
+}
+
+// ---------------------------------------------------------------- fixed scratch
+//
+// usk_gemv_multi_static: the same launch with the workspace in this array
+// instead of caller memory, for callers that may not allocate device memory.
+// The array lives in every device's copy of this module from the moment the
+// library is loaded until the process exits.  Host code must not hand the
+// array's name to a kernel (on the host it only stands for the symbol); the
+// device address comes from cudaGetSymbolAddress, looked up once per device
+// with that device current, the first time the entry point runs there.
+static __device__ __align__(256) uint8_t g_ml_scratch[USK_GEMV_MULTI_STATIC_BYTES];
+
+static cudaError_t ml_static_scratch(void** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_ml_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+// Bytes at the start of the workspace that must be zero when a launch starts
+// (the arrival counters; 0 when no row is split).
+static size_t ml_counter_bytes(int n, const int64_t* Ms, const int64_t* Ks, int batch, int depth, int var) {
+  int64_t slots = 0;
+  if (ml_slots_any(batch, depth, var, &slots) != cudaSuccess) slots = 296;
+  const MlPlan p = ml_plan(n, Ms, Ks, ml_bucket(batch), slots, nullptr);
+  return p.counters ? (static_cast<size_t>(p.counters) * 4u + 255u) & ~static_cast<size_t>(255u) : 0;
+}
+
+// The caller has checked that the list's workspace fits the array.  The
+// counters are cleared on the stream first (a call that gave up could have
+// left them non-zero), then the kernel runs on the array.
+cudaError_t launch_gemv_multi_static(int n, const int8_t* const* codes, const uint16_t* const* scales,
+                                     const int64_t* Ms, const int64_t* Ks, const uint64_t* seeds,
+                                     const uint16_t* const* x, float* const* y, int batch, uint32_t* status, bool pdl,
+                                     cudaStream_t stream, int depth, int var) {
+  void* base = nullptr;
+  cudaError_t e = ml_static_scratch(&base);
+  if (e != cudaSuccess) return e;
+  const size_t cnt = ml_counter_bytes(n, Ms, Ks, batch, depth, var);
+  if (cnt > 0) {
+    e = cudaMemsetAsync(base, 0, cnt, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_gemv_multi(n, codes, scales, Ms, Ks, seeds, x, y, batch, base, status, pdl, stream, 0, depth, var);
 }
 
 }  // namespace usk
