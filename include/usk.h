@@ -167,9 +167,15 @@ typedef enum { USK_F32 = 0, USK_BF16 = 1 } usk_dtype;
  *               group per launch);
  *   count[g]    host value: row blocks at 2 (g = 0), 4 (g = 1) and 8 (g = 2) slots;
  *   code_bytes  host value: K * sum of the slots (the codes array's size).
- * The library checks the counts against M on the host; on the device an order
- * entry outside [0, M/64) or an offset whose block would end past code_bytes
- * skips that row block (its outputs are not written) and sets USK_FLAG_RATE_MAP. */
+ * order must be a permutation of the row blocks grouped by slot count, as
+ * usk_rate_map_plan produces.  The library checks the counts against M on the
+ * host; on the device an order entry outside [0, M/64), an offset whose block
+ * would end past code_bytes, or a block whose extent (offset[rb + 1] -
+ * offset[rb], or code_bytes - offset[rb] for the last) is not K times its
+ * group's slot count skips that row block (its outputs are not written; the
+ * other row block of a usk_gemm tile is still computed) and sets
+ * USK_FLAG_RATE_MAP.  A duplicated entry is not detected: the block it
+ * replaces is neither built nor multiplied. */
 typedef struct {
   const int64_t* offset;
   const int32_t* order;
@@ -264,14 +270,22 @@ USK_API usk_status usk_build(const void* W, usk_dtype wdtype, int64_t M, int64_t
  * fly: every weight is rehashed and its bucket gathered; W_hat is never stored).
  *   x  [batch, K] row-major, fp32 or bf16 per xdtype, 16-byte aligned.
  *   y  [batch, M] fp32 output (y[t*M + i] = sum_j w_hat[i][j] x[t][j]).
- * Single-row 8-bit sketches (format 1, or format 2 at depth 1), bf16 x at batch <= 4:
- * integer tensor path, exact sum of code * x (x split
- * into byte digit planes per block; elements outside 2^22 of the block's
- * largest are added by an exact correction), one rounding to fp32 at the end.
- * Other batches, multi-row and 4-bit sketches: bf16 tensor path (each hash row
- * gathered, the code of largest magnitude kept), exact products, fp32 accumulation; fp32 x
- * is split into two bf16 terms (|error| <= 2^-16 |x| per element).
- * A sketch with a rate map: one launch, each row block at its slot count, bf16 path.
+ * Paths, chosen from the shape (measured on B200):
+ *   - bf16 x on uniform 4-slot single-row sketches (format 1, or format 2 at
+ *     depth 1) of more than 2 x SMs row blocks (e.g. 28672 rows) and
+ *     batch * K <= 16384: integer tensor path over row slabs (int8 codes x x
+ *     split into byte digit planes, exact integer sums, one rounding at the end);
+ *   - bf16 x at batch 2..8, or batch 1 with K <= 4096 and M <= 4096, and every
+ *     multi-row or 4-bit sketch at batch <= 8: bf16 tensor path with the x
+ *     fragments read straight from global memory (each hash row gathered, the
+ *     code of largest magnitude kept; exact products, fp32 accumulation);
+ *   - other bf16 x at batch 1 on single-row sketches: integer tensor path with
+ *     thread-block clusters along K (digit planes as above);
+ *   - fp32 x, batch 9..15, and the rest: bf16 tensor path with x staged in
+ *     shared memory; fp32 x is split into two bf16 terms (|error| <= 2^-16 |x|
+ *     per element).
+ * A sketch with a rate map: one launch, each row block at its slot count, bf16
+ * paths (direct x at batch <= 8 with bf16 x, else staged).
  * batch == 0 or M == 0 is a no-op; K == 0 writes y = 0.  Deterministic for a
  * given shape (the summation order is fixed). */
 USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
@@ -279,9 +293,11 @@ USK_API usk_status usk_gemv(const usk_sketch* sketch, const void* x, usk_dtype x
 
 /* usk_gemv with launch flags.  USK_GEMV_PDL: launch as a programmatic
  * dependent of the previous kernel in the stream; the kernel prefetches the
- * sketch codes before waiting for that kernel, so the caller guarantees that
- * no kernel still running in the stream writes this sketch (x and y may be
- * produced / consumed by neighbouring kernels).  Other bits: USK_ERR_PARAMS. */
+ * sketch codes (and reads a rate map's order and offset tables) before
+ * waiting for that kernel, so the caller guarantees that no kernel still
+ * running in the stream writes this sketch's codes, scales or rate-map tables
+ * (x and y may be produced / consumed by neighbouring kernels).  Other bits:
+ * USK_ERR_PARAMS. */
 #define USK_GEMV_PDL 1u
 USK_API usk_status usk_gemv_ex(const usk_sketch* sketch, const void* x, usk_dtype xdtype, int64_t batch,
                                float* y, uint32_t flags, uint32_t* d_status, void* stream);
@@ -356,7 +372,8 @@ USK_API usk_status usk_gemv_multi_static(int64_t n, const usk_sketch* sketches, 
  *   x_bf16 [batch, K] bf16, 16-byte aligned.  y [batch, M] fp32.
  *   ws / ws_bytes: unused by this version (may be NULL / 0).
  * A sketch with a rate map: one launch; a 128-row tile takes two row blocks of
- * the same slot count.
+ * the same slot count; the launch is planned for the 8-slot layout, so K is
+ * limited as for a uniform 8-slot sketch (USK_ERR_SHAPE beyond it).
  * M == 0 is a no-op; K == 0 writes y = 0. */
 USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y,
                     void* ws, size_t ws_bytes, uint32_t* d_status, void* stream);

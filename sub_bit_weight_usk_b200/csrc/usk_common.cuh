@@ -239,6 +239,25 @@ __device__ __forceinline__ void atoms_min_u64_off(uint32_t addr, uint64_t v) {
   asm volatile("red.shared.min.u64 [%0+%2], %1;" ::"r"(addr), "l"(v), "n"(OFF) : "memory");
 }
 
+// Address of the same shared-memory offset in cluster rank `rank`'s block.
+__device__ __forceinline__ uint32_t mapa_cluster(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// One-way 16-byte store into a peer block's shared memory; completes 16 bytes
+// of the transaction count of the peer's mbarrier `remote_bar` (both cluster
+// addresses from mapa_cluster).
+__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, float a, float b, float c, float d,
+                                            uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   remote_addr),
+               "r"(__float_as_uint(a)), "r"(__float_as_uint(b)), "r"(__float_as_uint(c)), "r"(__float_as_uint(d)),
+               "r"(remote_bar)
+               : "memory");
+}
+
 __device__ __forceinline__ void report(uint32_t* d_status, uint32_t flags) {
   if (flags && d_status) atomicOr(d_status, flags);
 }
@@ -353,9 +372,10 @@ __device__ __forceinline__ void bf16_parts(uint32_t b, int& e_eff, int& mant) {
 // Row blocks of one launch.  Uniform sketches: grid row g is row block g, its
 // codes at g * T * tile bytes.  Per-row-block rates: grid row g is row block
 // order[g] of the launch's slot group, its codes at offset[rb]; an entry out of
-// range (rb outside [0, RB), or a block ending past code_bytes, or an offset not
-// 16-byte aligned) is reported and skipped by the whole cluster (every block of
-// a cluster shares the grid row, so they all skip together).
+// range (rb outside [0, RB), a block ending past code_bytes, an offset not
+// 16-byte aligned, or a block whose extent offset[rb + 1] - offset[rb] (the
+// end of the codes for the last block) is not its group's) is reported and
+// skipped by the whole cluster (every block of a cluster shares the grid row).
 struct RbMap {
   const int32_t* order;   // nullptr: identity
   const int64_t* offset;
@@ -373,6 +393,10 @@ __device__ __forceinline__ bool rb_resolve(const RbMap& m, int64_t g, int64_t rb
   if (r < 0 || r >= m.RB) return false;
   const int64_t o = m.offset[r];
   if (o < 0 || (o & 15) != 0 || o + rb_bytes > m.code_bytes) return false;
+  // the block's extent in the table (blocks are back to back in matrix order)
+  // must be its group's: a block listed in the wrong slot group is refused
+  const int64_t end = r + 1 < m.RB ? m.offset[r + 1] : m.code_bytes;
+  if (end - o != rb_bytes) return false;
   rb = static_cast<int>(r);
   off = o;
   return true;

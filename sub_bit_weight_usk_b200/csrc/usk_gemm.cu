@@ -206,20 +206,21 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(sm + L.misc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
-  // the tile's two row blocks and where their codes start
-  const bool second_rb = 2 * static_cast<int64_t>(mt) + 1 < nrb;
+  // the tile's two row blocks and where their codes start; with a rate map a
+  // block whose entry is out of range is skipped on its own (its rows are
+  // neither decoded nor written), the other one of the tile still computed
+  bool okA = false, okB = false;
   int rbA = 0, rbB = 0;
   int64_t cbA = 0, cbB = 0;
   {
+    const bool has_b = 2 * static_cast<int64_t>(mt) + 1 < nrb;
     const int64_t rb_bytes = static_cast<int64_t>(a.T) * kRbBytes;
     RbMap gm = a.map;
     if (gm.order != nullptr) gm.order += order0;
-    bool ok = rb_resolve(gm, 2 * static_cast<int64_t>(mt), rb_bytes, rbA, cbA);
-    if (second_rb) ok = ok && rb_resolve(gm, 2 * static_cast<int64_t>(mt) + 1, rb_bytes, rbB, cbB);
-    if (!ok) {
-      if (tid == 0 && ks == 0) report(a.status, USK_FLAG_RATE_MAP);
-      return;  // the whole cluster (same tile) leaves before any barrier or allocation
-    }
+    okA = rb_resolve(gm, 2 * static_cast<int64_t>(mt), rb_bytes, rbA, cbA);
+    if (has_b) okB = rb_resolve(gm, 2 * static_cast<int64_t>(mt) + 1, rb_bytes, rbB, cbB);
+    if ((!okA || (has_b && !okB)) && tid == 0 && ks == 0) report(a.status, USK_FLAG_RATE_MAP);
+    if (!okA && !okB) return;  // the whole cluster (same tile) leaves before any barrier or allocation
   }
 
   if (warp == kMmaWarp0) {
@@ -237,11 +238,11 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
       *abort_flag = 0u;
       mbar_fence_init();
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(xmap)) : "memory");
-      // the block's codes: two contiguous runs (one per row block)
+      // the block's codes: two contiguous runs (one per valid row block)
       const uint32_t bytes = static_cast<uint32_t>(tcta) * kRbBytes;
-      mbar_arrive_expect_tx(codes_bar, bytes * (second_rb ? 2u : 1u));
-      bulk_g2s(s0 + L.codes, a.codes + cbA + static_cast<int64_t>(t_begin) * kRbBytes, bytes, codes_bar);
-      if (second_rb)
+      mbar_arrive_expect_tx(codes_bar, bytes * ((okA ? 1u : 0u) + (okB ? 1u : 0u)));
+      if (okA) bulk_g2s(s0 + L.codes, a.codes + cbA + static_cast<int64_t>(t_begin) * kRbBytes, bytes, codes_bar);
+      if (okB)
         bulk_g2s(s0 + L.codes + bytes, a.codes + cbB + static_cast<int64_t>(t_begin) * kRbBytes, bytes, codes_bar);
     }
     __syncwarp();
@@ -268,7 +269,7 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     const int g = tid >> 7;
     const int rbl = m >> 6;
     const uint32_t r = static_cast<uint32_t>(m & 63);
-    const bool row_ok = m < kRowsPerBlock || second_rb;
+    const bool row_ok = m < kRowsPerBlock ? okA : okB;
     // this thread's tensor-memory lane (= its row) in the A stages
     const uint32_t a_taddr = tmem_d + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + a.a_col;
     // loop exits are warp-uniform: tcgen05.st is a whole-warp instruction
@@ -427,7 +428,7 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     const int m = sub * 32 + lane;
     const int rbm = m < kRowsPerBlock ? rbA : rbB;
     const int64_t row = static_cast<int64_t>(rbm) * kRowsPerBlock + (m & 63);
-    const bool row_ok = m < kRowsPerBlock || second_rb;
+    const bool row_ok = m < kRowsPerBlock ? okA : okB;
     const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[rbm])) : 0.0f;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     float* part = reinterpret_cast<float*>(sm + L.b);  // [N][128]: the x stage ring is free now
@@ -468,7 +469,7 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
 #pragma unroll
       for (int s = 0; s < 16; ++s) acc += v[s];
       const int n = q / kBM, mm = q % kBM;
-      if (mm < kRowsPerBlock || second_rb) {
+      if (mm < kRowsPerBlock ? okA : okB) {
         const int rbm = mm < kRowsPerBlock ? rbA : rbB;
         const int64_t orow = static_cast<int64_t>(rbm) * kRowsPerBlock + (mm & 63);
         const float sc = __half2float(__ushort_as_half(a.scales[rbm]));

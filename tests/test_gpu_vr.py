@@ -191,11 +191,13 @@ def test_vr_bad_map_entries_are_skipped_and_flagged():
     bad_order = usk.RateMap(slots, good.offset.clone(), good.order.clone(), good.count, good.code_bytes)
     bad_order.order[0] = 99  # the 2-slot group's only entry
     bad_off = usk.RateMap(slots, good.offset.clone(), good.order.clone(), good.count, good.code_bytes)
-    bad_off.offset[1] = good.code_bytes  # row block 1 (8 slots) would end past the codes
+    # row block 1 (8 slots) would end past the codes, and row block 0's extent
+    # (up to row block 1's offset) no longer matches its 2 slots: both skipped
+    bad_off.offset[1] = good.code_bytes
     off = good.offset.cpu().tolist()
     x1 = to_dev(gen.activations(1, K, 77, "bf16"))
     x16 = to_dev(gen.activations(16, K, 77, "bf16"))
-    for rm, skipped in ((bad_order, 0), (bad_off, 1)):
+    for rm, skipped in ((bad_order, {0}), (bad_off, {0, 1})):
         st = status_tensor()
         codes = torch.zeros(good.code_bytes, dtype=torch.int8, device="cuda")
         scales = torch.zeros(M // 64, dtype=torch.int16, device="cuda")
@@ -205,7 +207,7 @@ def test_vr_bad_map_entries_are_skipped_and_flagged():
         c = codes.cpu().numpy()
         for rb, S in enumerate(slots):
             seg = slice(off[rb], off[rb] + S * K)
-            if rb == skipped:
+            if rb in skipped:
                 assert not c[seg].any()
             else:
                 assert np.array_equal(c[seg], o["codes"][seg])
@@ -220,12 +222,41 @@ def test_vr_bad_map_entries_are_skipped_and_flagged():
             torch.cuda.synchronize()
             assert int(st.item()) & usk.FLAG_RATE_MAP
             yc = y.cpu().numpy()
-            blk = slice(64 * skipped, 64 * skipped + 64)
-            assert np.all(yc[:, blk] == 7.0)  # not written
             keep = np.ones(M, bool)
-            keep[blk] = False
-            if not gemm:
-                assert rel_err(yc[:, keep], ref[:, keep]) <= TOL
+            for rb in skipped:
+                assert np.all(yc[:, 64 * rb:64 * rb + 64] == 7.0)  # not written
+                keep[64 * rb:64 * rb + 64] = False
+            r = ref if not gemm else oracle.gemv_vr_f64(o["codes"], o["scales"], M, K,
+                                                        gen.activations(16, K, 77, "bf16"), 4, slots)
+            assert rel_err(yc[:, keep], r[:, keep]) <= TOL
+
+
+def test_vr_gemm_pair_keeps_the_valid_block():
+    """A 128-row GEMM tile pairs two row blocks of one slot group; when one of
+    them has a bad entry, only its rows are skipped: the partner block's
+    outputs are still computed (GEMV and GEMM against the oracle)."""
+    slots = [4, 4, 2]
+    M, K = 192, 1024
+    W = gen.weights_student_t(M, K, 80, 4.0, 0.02, 0.001, 20.0, "bf16")
+    o = oracle.build_sketch_vr(W, None, 5, slots)
+    good = usk.usk_rate_map(M, K, slots)
+    assert good.order.cpu().tolist() == [2, 0, 1]  # the 2-slot group, then the 4-slot pair
+    bad = usk.RateMap(slots, good.offset.clone(), good.order.clone(), good.count, good.code_bytes)
+    bad.order[2] = 99  # row block 1's entry: the second block of the 4-slot tile
+    sk = usk.Sketch(M, K, 5, torch.from_numpy(o["codes"].copy()).cuda(),
+                    torch.from_numpy(o["scales"].view(np.int16).copy()).cuda(), usk.FORMAT_MAXKEY, 1, 0, bad)
+    for batch, gemm in ((1, False), (16, True)):
+        x = gen.activations(batch, K, 81, "bf16")
+        st = status_tensor()
+        y = torch.full((batch, M), 7.0, device="cuda")
+        (usk.usk_gemm if gemm else usk.usk_gemv)(sk, to_dev(x), y=y, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) & usk.FLAG_RATE_MAP
+        yc = y.cpu().numpy()
+        assert np.all(yc[:, 64:128] == 7.0)
+        keep = np.r_[0:64, 128:192]
+        ref = oracle.gemv_vr_f64(o["codes"], o["scales"], M, K, x, 5, slots)
+        assert rel_err(yc[:, keep], ref[:, keep]) <= TOL
 
 
 def test_vr_timeouts_reported_then_recover():
@@ -249,3 +280,19 @@ def test_vr_timeouts_reported_then_recover():
     _compare_build(W, None, 0, slots)
     _check_product(sk, o, x1)
     _check_product(sk, o, x16, gemm=True)
+
+
+@pytest.mark.parametrize("call", ["gemm16", "gemv9", "gemv_f32"])
+def test_vr_long_k_products(call):
+    """K = 11008 (43 tiles) with per-row-block rates: the launches are planned
+    for the 8-slot layout; each product runs and matches the oracle."""
+    slots = [8, 2, 4, 8]
+    M, K = 256, 11008
+    W = gen.weights_normal(M, K, 82, 0.02, "bf16")
+    sk, o = _oracle_sketch(W, None, 6, slots)
+    if call == "gemm16":
+        _check_product(sk, o, gen.activations(16, K, 83, "bf16"), gemm=True)
+    elif call == "gemv9":
+        _check_product(sk, o, gen.activations(9, K, 83, "bf16"))
+    else:
+        _check_product(sk, o, gen.activations(2, K, 83, "f32"))
