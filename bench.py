@@ -1196,8 +1196,13 @@ def run_profile_case(args):
         not (case.endswith("_ab") or case.endswith("_70b")) else None
     sk = usk.usk_build(W, imp_c, cfg["seed"], **fmt)
     torch.cuda.synchronize()
+    ws = None
+    if case.startswith("gemv_multi"):
+        ws = torch.zeros(max(16, usk.usk_gemv_multi_ws_bytes([sk], 1)), dtype=torch.uint8, device=dev)
     for _ in range(3 + 3):  # 3 warm-up launches, then 3 to capture
-        if case.startswith("build"):
+        if case.startswith("gemv_multi"):
+            usk.usk_gemv_multi([sk], [x1], ws=ws)
+        elif case.startswith("build"):
             usk.usk_build(W, imp_c, cfg["seed"], codes=sk.codes, scales=sk.scales, **fmt)
         elif case.startswith("gemv"):
             usk.usk_gemv(sk, x1)
@@ -1210,7 +1215,7 @@ def run_profile_case(args):
 
 PROFILE_CASES = ["build", "gemv", "gemm", "build_amm", "gemv_amm", "gemm_amm", "build_cs", "gemv_cs", "gemv_ab",
                  "gemv_cs_ab", "build_q4", "gemv_q4", "gemm_q4", "build_vr", "gemv_vr", "gemm_vr", "build_70b",
-                 "gemm_70b"]
+                 "gemm_70b", "gemv_70b", "gemv_multi", "gemv_multi_70b"]
 
 
 def main(argv=None):

@@ -398,6 +398,11 @@ USK_API void usk_debug_set_gemv_path(int path);
  * choice.  Results stay within the products' tolerance; process-wide. */
 USK_API void usk_debug_set_gemv_rows(int rows);
 
+/* Test hook: thread blocks along K per 128-row tile of usk_gemm (1..16, used
+ * where that many tiles per block fit; 0 = the library's choice).  Results
+ * stay within the products' tolerance; process-wide. */
+USK_API void usk_debug_set_gemm_splits(int splits);
+
 /* Test hook for the failure path (host-made; no device fault): kernel = 1 makes
  * usk_build, 2 usk_gemm, 3 usk_gemv, 4 usk_gemv_multi skip one bulk or tensor
  * copy in thread block (0, 0) (for the usk_gemv path without copies: the

@@ -561,10 +561,12 @@ static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, int var) {
 }
 
 // Blocks along K per 128-row tile: minimise (waves of blocks) x (tiles per
-// block + 4), the 4 standing for a block's fixed cost in tiles (prologue,
-// pipeline fill, epilogue and the cluster reduction: 4 to 5 us measured against
-// about 1.3 us per tile at batch 16), within the shared-memory bound on tiles
-// per block and clusters of at most 16.
+// block + 6 + the cluster's launch penalty), in units of about one tile's
+// time.  Fitted to split sweeps on B200 (4096 x 4096, 11008 x 4096, 4096 x
+// 11008, 28672 x 8192 at batch 16 and 64): a block's fixed cost (prologue,
+// pipeline fill, epilogue, cluster reduction) is about 6 tiles; clusters of
+// 5 to 8 blocks cost about 5 tiles more, larger ones about 14 more.  Within the
+// shared-memory bound on tiles per block and clusters of at most 16.
 static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, int var) {
   const int max_tiles = gemm_max_tiles(N, depth, var);
   const int64_t slots = static_cast<int64_t>(sms) * (512 / static_cast<int>(gemm_tmem_cols(N)));
@@ -574,9 +576,7 @@ static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, int va
     const int tpb = (T + s - 1) / s;
     if (tpb > max_tiles) continue;
     const int64_t waves = (m_tiles * s + slots - 1) / slots;
-    // clusters above 4 blocks launch with a visible spread (up to 3 us measured
-    // for 8 blocks of 704 threads): charge them 2 tiles more
-    const int64_t cost = waves * (tpb + 4 + (s > 4 ? 2 : 0));
+    const int64_t cost = waves * (tpb + 6 + (s > 4 ? 5 : 0) + (s > 8 ? 9 : 0));
     if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
       best = s;
@@ -593,7 +593,8 @@ bool gemm_supported(int64_t K, int batch, int depth, int var) {
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
-                        int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2) {
+                        int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2,
+                        int splits_override) {
   // a rate map: one launch over the tiles of every slot group, planned for the
   // 8-slot layout (the largest staged and widened tiles)
   const bool vr = map.order != nullptr;
@@ -617,6 +618,10 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth, var);
+  if (splits_override > 0) {  // test hook: a given split, where its tiles fit
+    const int s = splits_override < a.T ? splits_override : a.T;
+    if (s <= 16 && (a.T + s - 1) / s <= gemm_max_tiles(batch, depth, var)) a.splits = s;
+  }
   if (a.splits < 1) return cudaErrorInvalidValue;  // K beyond 16 blocks x the tiles one block can stage
   a.tmem_cols = gemm_tmem_cols(batch);
   a.a_col = gemm_a_col(batch);

@@ -54,8 +54,9 @@ def test_gemm_wait_timeout_reported_then_recovers():
 @pytest.mark.parametrize("path", [2, 3, 4])
 def test_gemv_wait_timeout_reported_then_recovers(path):
     """Path 3 skips a code copy; paths 2 and 4 (no copies) have block 1 of row
-    block 0 skip its partial sums, so the first block's wait gives up."""
-    K = 2048 if path in (2, 4) else 256
+    block 0 skip its partial sums, so the first block's wait gives up (K spans
+    two blocks of the path's default tiles per block: 8 for path 2, 4 for 4)."""
+    K = {2: 4096, 3: 256, 4: 2048}[path]
     W = gen.weights_normal(64, K, 4, 0.02, "bf16")
     sk = usk.usk_build(to_dev(W), None, 2)
     x = gen.activations(1, K, 5, "bf16")
