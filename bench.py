@@ -850,7 +850,7 @@ def run_usk(args):
     agg = aggregate(world, [t_gemv], [t_build], [t_step])
     rl = rooflines(peaks, t_build, t_gemv, t_gemm, tr)
     rl["usk_gemv_b4"] = R.gather_line(gemv_bytes(M, K, 4), N_W, t_gemv4)
-    rl["usk_gemv_multi"] = R.gather_line(GEMV_BYTES, N_W, L["usk_gemv_multi"])
+    rl["usk_gemv_multi"] = R.gather_line(GEMV_BYTES, N_W, L["usk_gemv_multi"], tr.get("multi_usk_gemv"))
     e2e_bytes_c = (c_e2e or {}).get("h2d_bytes", 2 * K) + (c_e2e or {}).get("d2h_bytes", 4 * M)
     clocks = sampler.summary()
     info = cpu_info()
@@ -963,16 +963,21 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
     for shp in ("28672x8192", "8192x28672"):
         m, k = (int(v) for v in shp.split("x"))
         d = {c.split("/")[1]: v for c, v in mm.items() if c.startswith(shp + "/")}
+        # ncu traffic was taken on the 28672 x 8192 shape
+        tk = (lambda key: tr.get(key)) if shp == "28672x8192" else (lambda key: None)
         per[shp] = {
             "kernel_us": {c: _us(v) for c, v in d.items()},
             "usk_build_gweights_per_s": round(world * m * k / d["usk_build"] / 1e9, 3),
-            "rooflines": {"usk_build": R.hbm_line(build_bytes(m, k, 2, False), d["usk_build"]),
-                          "usk_gemv_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_b1"]),
-                          "usk_gemv_multi_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_multi_b1"])},
+            "rooflines": {"usk_build": R.hbm_line(build_bytes(m, k, 2, False), d["usk_build"], tk("mlp70b_usk_build")),
+                          "usk_gemv_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_b1"],
+                                                       tk("mlp70b_usk_gemv_b1")),
+                          "usk_gemv_multi_b1": R.gather_line(gemv_bytes(m, k, 1), m * k, d["usk_gemv_multi_b1"],
+                                                             tk("mlp70b_usk_gemv_multi_b1"))},
         }
         for bb in (16, 32, 64):
             t = d["usk_gemm_b%d" % bb]
-            ln = R.gather_line(gemv_bytes(m, k, bb), m * k, t, flops=2 * m * k * bb)
+            ln = R.gather_line(gemv_bytes(m, k, bb), m * k, t, tk("mlp70b_usk_gemm_b64") if bb == 64 else None,
+                               flops=2 * m * k * bb)
             # the survey's decode roof at 28672x8192, batch 64 (issue, ~5 ops/weight): 31.6 us
             ln["decode_roof_us"] = round(5 * m * k / (SMS * 128 * R.clk) * 1e6, 3)
             per[shp]["rooflines"]["usk_gemm_b%d" % bb] = ln
