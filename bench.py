@@ -464,6 +464,7 @@ class Bench:
         import torch.distributed as dist
         torch = self.torch
         out = {name: [] for name, _, _ in region}
+        torch.cuda.nvtx.range_push("timed")  # lets a profiler keep to the timed launches
         for _ in range(REPEATS):
             if self.world > 1:
                 dist.barrier()
@@ -483,6 +484,7 @@ class Bench:
                 dist.barrier()
             for k, (name, _, _) in enumerate(region):
                 out[name].append(ev[k].elapsed_time(ev[k + 1]) * 1e-3 / max(self.steps, 1))
+        torch.cuda.nvtx.range_pop()
         for _, _, lps in region:
             self.launches += REPEATS * self.steps * lps
         self._check("in the timed region")
