@@ -403,6 +403,11 @@ USK_API void usk_debug_set_gemv_rows(int rows);
  * stay within the products' tolerance; process-wide. */
 USK_API void usk_debug_set_gemm_splits(int splits);
 
+/* Test hook: MMA issuer warps of usk_gemm (1, 2 or 4, at most the default for
+ * the batch: 4 up to 64, 2 up to 128, 1 above; 0 = the library's choice).
+ * Results stay within the products' tolerance; process-wide. */
+USK_API void usk_debug_set_gemm_issuers(int issuers);
+
 /* Test hook for the failure path (host-made; no device fault): kernel = 1 makes
  * usk_build, 2 usk_gemm, 3 usk_gemv, 4 usk_gemv_multi skip one bulk or tensor
  * copy in thread block (0, 0) (for the usk_gemv path without copies: the

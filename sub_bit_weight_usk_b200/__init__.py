@@ -34,6 +34,7 @@ from ._native import (  # noqa: F401
     usk_debug_set_gemv_path,
     usk_debug_set_gemv_rows,
     usk_debug_set_gemm_splits,
+    usk_debug_set_gemm_issuers,
     usk_debug_set_geometry,
     usk_format_version,
     usk_gemm,

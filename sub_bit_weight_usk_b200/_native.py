@@ -69,7 +69,7 @@ _lib = None
 EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_rate_map_plan", "usk_build", "usk_gemv", "usk_gemv_ex",
             "usk_gemv_multi", "usk_gemv_multi_ws_bytes", "usk_gemv_multi_static", "usk_gemm", "usk_status_str",
             "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_set_gemv_rows",
-            "usk_debug_set_gemm_splits", "usk_debug_inject_timeout"]
+            "usk_debug_set_gemm_splits", "usk_debug_set_gemm_issuers", "usk_debug_inject_timeout"]
 GEMV_PDL = 1
 
 
@@ -122,6 +122,8 @@ def load_library(path: str = LIB_PATH):
     lib.usk_debug_set_gemv_rows.restype = None
     lib.usk_debug_set_gemm_splits.argtypes = [ctypes.c_int]
     lib.usk_debug_set_gemm_splits.restype = None
+    lib.usk_debug_set_gemm_issuers.argtypes = [ctypes.c_int]
+    lib.usk_debug_set_gemm_issuers.restype = None
     lib.usk_debug_inject_timeout.argtypes = [ctypes.c_int]
     lib.usk_debug_inject_timeout.restype = None
     _lib = lib
@@ -408,6 +410,11 @@ def usk_debug_set_gemv_rows(rows: int = 0) -> None:
 def usk_debug_set_gemm_splits(splits: int = 0) -> None:
     """Blocks along K per 128-row tile of usk_gemm (0 = automatic)."""
     load_library().usk_debug_set_gemm_splits(int(splits))
+
+
+def usk_debug_set_gemm_issuers(issuers: int = 0) -> None:
+    """MMA issuer warps of usk_gemm (1, 2 or 4; 0 = automatic)."""
+    load_library().usk_debug_set_gemm_issuers(int(issuers))
 
 
 def usk_debug_inject_timeout(kernel: int = 0) -> None:

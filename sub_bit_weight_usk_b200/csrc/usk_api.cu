@@ -31,7 +31,7 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
                         int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2,
-                        int splits_override);
+                        int splits_override, int issuers_override);
 bool gemm_supported(int64_t K, int batch, int depth, int var);
 size_t gemv_multi_ws_bytes(int n, const int64_t* Ms, const int64_t* Ks, int batch, int depth, int var);
 cudaError_t launch_gemv_multi(int n, const int8_t* const* codes, const uint16_t* const* scales, const int64_t* Ms,
@@ -139,6 +139,7 @@ int g_gemv_tiles_per_block = 0;
 int g_gemv_path = 0;
 int g_gemv_rows = 0;
 int g_gemm_splits = 0;
+int g_gemm_issuers = 0;
 int g_inject = 0;  // 1 build, 2 gemm, 3 gemv, 4 gemv_multi: skip one copy/commit in block (0, 0)
 
 constexpr int64_t kMultiMax = 16;  // sketches per usk_gemv_multi launch
@@ -405,7 +406,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   const Launch l = launch_of(sketch->rates, sketch->M);
   cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
                                    static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, layout, l.map,
-                                   l.nrb, l.g1, l.g2, g_gemm_splits);
+                                   l.nrb, l.g1, l.g2, g_gemm_splits, g_gemm_issuers);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }
@@ -546,6 +547,8 @@ USK_API void usk_debug_set_gemv_path(int path) { g_gemv_path = path; }
 USK_API void usk_debug_set_gemv_rows(int rows) { g_gemv_rows = rows; }
 
 USK_API void usk_debug_set_gemm_splits(int splits) { g_gemm_splits = splits; }
+
+USK_API void usk_debug_set_gemm_issuers(int issuers) { g_gemm_issuers = issuers; }
 
 USK_API void usk_debug_inject_timeout(int kernel) { g_inject = kernel; }
 

@@ -104,8 +104,8 @@ __host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int de
 // Tensor memory: the issuers' fp32 accumulators [0, I N), then the A stages,
 // 32 columns (128 rows x 64 bf16) each, from column a_col(N).
 __host__ __device__ inline int gemm_issuers(int N) { return N <= 64 ? 4 : (N <= 128 ? 2 : 1); }
-__host__ __device__ inline uint32_t gemm_a_col(int N) {
-  return (static_cast<uint32_t>(gemm_issuers(N) * N) + 31u) & ~31u;
+__host__ __device__ inline uint32_t gemm_a_col(int N, int I) {
+  return (static_cast<uint32_t>(I * N) + 31u) & ~31u;
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -520,7 +520,9 @@ static uint32_t var_tile_bf(int var) {
 }
 
 // 256 columns (two blocks per SM) when four stages fit next to the accumulators, else 512
-__host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N) + 4u * 32u <= 256u ? 256u : 512u; }
+__host__ __device__ inline uint32_t gemm_tmem_cols(int N, int I) {
+  return gemm_a_col(N, I) + 4u * 32u <= 256u ? 256u : 512u;
+}
 
 // Pipeline stages for batch N and tpb tiles per block: as many as tensor
 // memory and shared memory (the B stages next to the staged codes; half of the
@@ -531,10 +533,10 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int N) { return gemm_a_col(N)
 // mbarrier has one in-order waiter per role.  Otherwise consecutive uses of a
 // stage belong to different warps, and a warp running ahead can take a
 // completed phase of use n - 2 for use n (a phase wait only tells parity).
-static int gemm_stages(int N, int tpb, int depth, int var) {
-  const uint32_t cols = gemm_tmem_cols(N);
+static int gemm_stages(int N, int tpb, int depth, int var, int I) {
+  const uint32_t cols = gemm_tmem_cols(N, I);
   const uint32_t smem_cap = cols == 256u ? 233472u / 2u - 1024u : kSmemLimit;
-  int S = static_cast<int>((cols - gemm_a_col(N)) / 32u);
+  int S = static_cast<int>((cols - gemm_a_col(N, I)) / 32u);
   if (S > kMaxStages) S = kMaxStages;
   S &= ~3;
   while (S >= 4 && gemm_layout(N, tpb, S, depth, var_tile_bytes(var), var_tile_bf(var)).total + 1024u > smem_cap)
@@ -544,18 +546,18 @@ static int gemm_stages(int N, int tpb, int depth, int var) {
 
 // Largest number of tiles per block (codes staged up front) that still leaves
 // a four-stage pipeline for batch N.
-static int gemm_max_tiles(int N, int depth, int var) {
+static int gemm_max_tiles(int N, int depth, int var, int I) {
   int t = kMaxTiles;
-  while (t > 1 && gemm_stages(N, t, depth, var) == 0) --t;
+  while (t > 1 && gemm_stages(N, t, depth, var, I) == 0) --t;
   return t;
 }
 
 // Dynamic shared memory of a launch: the layout, padded so that no more blocks
 // share an SM than its 512 tensor-memory columns hold (a block waiting in
 // tcgen05.alloc for a co-resident block of its own cluster would never proceed).
-static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, int var) {
+static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, int var, int I) {
   const uint32_t smem = gemm_layout(N, tpb, S, depth, var_tile_bytes(var), var_tile_bf(var)).total + 1024u;
-  const uint32_t max_blocks = 512u / gemm_tmem_cols(N);
+  const uint32_t max_blocks = 512u / gemm_tmem_cols(N, I);
   const uint32_t floor_bytes = 233472u / (max_blocks + 1u) + 1u - 1024u;  // 228 KiB per SM, 1 KiB reserved per block
   return smem > floor_bytes ? smem : floor_bytes;
 }
@@ -567,19 +569,39 @@ static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, int var) {
 // pipeline fill, epilogue, cluster reduction) is about 6 tiles; clusters of
 // 5 to 8 blocks cost about 5 tiles more, larger ones about 14 more.  Within the
 // shared-memory bound on tiles per block and clusters of at most 16.
-static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, int var) {
-  const int max_tiles = gemm_max_tiles(N, depth, var);
-  const int64_t slots = static_cast<int64_t>(sms) * (512 / static_cast<int>(gemm_tmem_cols(N)));
-  int best = -1;
+//
+// The MMA issuer count I is chosen with it: the default (4 up to batch 64, 2 up
+// to 128, 1 above) keeps one block per SM where the accumulators need 512
+// tensor-memory columns (batch 48 and 64); half the issuers fit two blocks per
+// SM, which pays when there are more blocks than SMs (28672 x 8192 at batch 64:
+// one wave of 224 instead of 1.5).  Two co-resident blocks share the SM, so
+// such a plan is charged 1.5x per wave.
+struct GemmPlan {
+  int splits, I;
+};
+
+static GemmPlan gemm_plan(int64_t m_tiles, int T, int N, int sms, int depth, int var, int issuers_override) {
+  const int I0 = gemm_issuers(N);
+  GemmPlan best{-1, I0};
   int64_t best_cost = -1;
-  for (int s = 1; s <= 16 && s <= T; ++s) {
-    const int tpb = (T + s - 1) / s;
-    if (tpb > max_tiles) continue;
-    const int64_t waves = (m_tiles * s + slots - 1) / slots;
-    const int64_t cost = waves * (tpb + 6 + (s > 4 ? 5 : 0) + (s > 8 ? 9 : 0));
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = s;
+  for (int I = I0; I >= 1; I /= 2) {
+    if (issuers_override > 0 && I != issuers_override) continue;
+    if (issuers_override <= 0 && I != I0 && !(gemm_tmem_cols(N, I0) == 512u && gemm_tmem_cols(N, I) == 256u))
+      continue;  // fewer issuers only where that fits a second block per SM
+    const int max_tiles = gemm_max_tiles(N, depth, var, I);
+    const int per_sm = 512 / static_cast<int>(gemm_tmem_cols(N, I));
+    const int64_t slots = static_cast<int64_t>(sms) * per_sm;
+    for (int s = 1; s <= 16 && s <= T; ++s) {
+      const int tpb = (T + s - 1) / s;
+      if (tpb > max_tiles) continue;
+      const int64_t blocks = m_tiles * s;
+      const int64_t waves = (blocks + slots - 1) / slots;
+      int64_t cost = 2 * waves * (tpb + 6 + (s > 4 ? 5 : 0) + (s > 8 ? 9 : 0));
+      if (I != I0 && blocks > sms) cost = cost * 3 / 2;  // two blocks sharing an SM
+      if (best_cost < 0 || cost < best_cost) {
+        best_cost = cost;
+        best = GemmPlan{s, I};
+      }
     }
   }
   return best;
@@ -588,13 +610,13 @@ static int gemm_splits(int64_t m_tiles, int T, int N, int sms, int depth, int va
 // Whether K fits: at most 16 blocks along K, each staging the codes of up to
 // gemm_max_tiles(batch) tiles (32 for every batch: K <= 131072).
 bool gemm_supported(int64_t K, int batch, int depth, int var) {
-  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch, depth, var));
+  return K / kTileCols <= 16 * static_cast<int64_t>(gemm_max_tiles(batch, depth, var, gemm_issuers(batch)));
 }
 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
                         int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2,
-                        int splits_override) {
+                        int splits_override, int issuers_override) {
   // a rate map: one launch over the tiles of every slot group, planned for the
   // 8-slot layout (the largest staged and widened tiles)
   const bool vr = map.order != nullptr;
@@ -617,19 +639,25 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   const int64_t m_tiles = vr ? (g1 + 1) / 2 + (g2 - g1 + 1) / 2 + (a.map.RB - g2 + 1) / 2 : (nrb + 1) / 2;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  a.splits = gemm_splits(m_tiles, a.T, batch, sms, depth, var);
+  // test hook: a given issuer count (1, 2 or 4 dividing the default's work)
+  const int io = (issuers_override == 1 || issuers_override == 2 || issuers_override == 4) &&
+                         issuers_override <= gemm_issuers(batch)
+                     ? issuers_override
+                     : 0;
+  const GemmPlan plan = gemm_plan(m_tiles, a.T, batch, sms, depth, var, io);
+  a.splits = plan.splits;
+  a.I = plan.I;
   if (splits_override > 0) {  // test hook: a given split, where its tiles fit
     const int s = splits_override < a.T ? splits_override : a.T;
-    if (s <= 16 && (a.T + s - 1) / s <= gemm_max_tiles(batch, depth, var)) a.splits = s;
+    if (s <= 16 && (a.T + s - 1) / s <= gemm_max_tiles(batch, depth, var, a.I)) a.splits = s;
   }
   if (a.splits < 1) return cudaErrorInvalidValue;  // K beyond 16 blocks x the tiles one block can stage
-  a.tmem_cols = gemm_tmem_cols(batch);
-  a.a_col = gemm_a_col(batch);
-  a.I = gemm_issuers(batch);
+  a.tmem_cols = gemm_tmem_cols(batch, a.I);
+  a.a_col = gemm_a_col(batch, a.I);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
-  a.S = gemm_stages(batch, tcta_max, depth, var);
+  a.S = gemm_stages(batch, tcta_max, depth, var, a.I);
   if (a.S < 4 || a.S % 4 != 0) return cudaErrorInvalidValue;
-  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth, var);
+  const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth, var, a.I);
   // tensor map over x [batch, K] bf16: one 64-column x batch box per chunk, 128-byte swizzle
   const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;

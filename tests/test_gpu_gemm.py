@@ -99,3 +99,22 @@ def test_gemm_zero_sketch_and_errors():
     with pytest.raises(usk.UskError) as e:
         usk.usk_gemm(sk, x[:8])  # below 16: usk_gemv's range
     assert e.value.status == 4
+
+
+@pytest.mark.parametrize("issuers", [1, 2, 4])
+@pytest.mark.parametrize("batch", [16, 48, 64, 128])
+def test_gemm_issuer_counts(issuers, batch):
+    """Every MMA issuer count the planner may pick (forced through the test
+    hook where it does not exceed the batch's default), with and without a K
+    split: same products within the tolerance."""
+    W = gen.weights_student_t(512, 2048, 13, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _sketch(W, 21)
+    x = gen.activations(batch, 2048, 22, "bf16")
+    try:
+        usk.usk_debug_set_gemm_issuers(issuers)
+        for splits in (0, 1, 2):
+            usk.usk_debug_set_gemm_splits(splits)
+            _check(sk, o, x)
+    finally:
+        usk.usk_debug_set_gemm_issuers(0)
+        usk.usk_debug_set_gemm_splits(0)
