@@ -10,12 +10,15 @@
 //    of whole hash tiles along K; blocks that split K for the same rows form a
 //    cluster and add their fp32 partials through distributed shared memory in
 //    rank order (deterministic, no workspace).
-//  * At start the block's int8 codes (2 row blocks x its tiles) arrive in
-//    shared memory with two bulk copies; a widen warp converts each tile's
-//    2 x 1024 codes to bf16 once (instead of once per use: 16 uses) with an
-//    exact integer/FMA-pipe bit trick (the conversion unit of one sub-partition
-//    was measured as the bottleneck), into a ring of tile buffers guarded by
-//    ready/free mbarriers.
+//  * The block's int8 codes (2 row blocks x its tiles) stream through a ring
+//    of 8 raw tile slots, one bulk copy per row block and tile completing on
+//    the slot's mbarrier; the widen warp refills a slot as soon as it has
+//    read it (staging all tiles would hold shared memory that pipeline
+//    stages and a second block per SM use better).  The widen warp converts
+//    each tile's 2 x 1024 codes to bf16 once (instead of once per use: 16
+//    uses) with an exact integer/FMA-pipe bit trick (the conversion unit of
+//    one sub-partition was measured as the bottleneck), into a ring of tile
+//    buffers guarded by ready/free mbarriers.
 //  * 16 decoder warps: per 64-column chunk each thread rebuilds 2 octets of one
 //    row -- one multiply-add of the hash per octet, one 16-byte conflict-free
 //    gather of the 8 bf16 codes (class = (octet + row) mod 32) -- and writes
@@ -56,11 +59,12 @@ constexpr int kMmaWarp0 = kDecWarps + 2;   // first MMA warp; it also owns the T
 constexpr int kMaxIssuers = 4;             // MMA warps: a tcgen05.mma holds its issuing warp ~180 cycles
 constexpr int kGemmThreads = (kDecWarps + 2 + kMaxIssuers) * 32;
 constexpr int kTileRing = 4;               // bf16 tile-code buffers
+constexpr int kRawRingMin = 8;             // raw tile-code slots (fewer only when a block has fewer tiles)
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kMaxStages = 16;  // pipeline stages (A in tensor memory, B in shared memory)
-constexpr int kMaxTiles = 32;  // hash tiles per block (codes staged up front)
+constexpr int kMaxTiles = 32;  // hash tiles per block (keys of each kept in shared memory)
 
 struct GemmArgs {
   const int8_t* codes;
@@ -76,6 +80,7 @@ struct GemmArgs {
   uint32_t a_col;  // first tensor-memory column of the A stages
   int S;           // pipeline stages
   int I;           // MMA issuer warps, each with its own accumulator (columns [i N, (i + 1) N))
+  int R;           // raw tile-code slots: min(tiles per block, kRawRingMin)
   int inject;  // test hook: block (0, 0) skips the x copy of its first chunk
   RbMap map;    // grid rows -> row blocks and code offsets
   int64_t nrb;  // row blocks of this launch (a tile takes grid rows 2 mt and 2 mt + 1)
@@ -88,15 +93,16 @@ struct GemmLayout {
 
 // tile_bytes / tile_bf: stored and widened bytes per row block and tile
 __host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int depth, uint32_t tile_bytes,
-                                                  uint32_t tile_bf) {
+                                                  uint32_t tile_bf, int R) {
   GemmLayout L;
   L.b = 0;  // [S][N x 64] bf16, SW128; after the main loop the K-split partials [N][128] fp32
   const uint32_t ring = static_cast<uint32_t>(S) * N * kBK * 2, parts = static_cast<uint32_t>(N) * kBM * 4;
   L.cbf = L.b + (ring > parts ? ring : parts);                         // bf16 [kTileRing][2][1024 or 2048]
-  L.codes = L.cbf + kTileRing * 2u * tile_bf;                          // codes [2][tcta][tile_bytes]
-  L.keys = L.codes + 2u * tcta * tile_bytes;                           // uint2 [2][tcta][depth]
-  L.bars = (L.keys + 2u * tcta * depth * 8u + 7u) & ~7u;  // full[S], empty[S], codes, done, ready[ring], free[ring]
-  L.misc = L.bars + (2 * S + 2 + 2 * kTileRing) * 8;                   // tmem holder, abort
+  L.codes = L.cbf + kTileRing * 2u * tile_bf;                          // raw codes [R][2][tile_bytes]
+  L.keys = L.codes + static_cast<uint32_t>(R) * 2u * tile_bytes;       // uint2 [2][tcta][depth]
+  // full[S], empty[S], done, ready[ring], free[ring], raw[R]
+  L.bars = (L.keys + 2u * tcta * depth * 8u + 7u) & ~7u;
+  L.misc = L.bars + (2 * S + 1 + 2 * kTileRing + R) * 8;               // tmem holder, abort
   L.total = L.misc + 16;
   return L;
 }
@@ -199,10 +205,11 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
   const int tcta = t_end - t_begin;
   const int nk = tcta * (kTileCols / kBK);  // 64-column chunks
   const int S = a.S;
-  const GemmLayout L = gemm_layout(a.N, tcta, S, D, kRbBytes, kRbBf);
+  const int R = a.R;
+  const GemmLayout L = gemm_layout(a.N, tcta, S, D, kRbBytes, kRbBf, R);
   const uint32_t bstage = static_cast<uint32_t>(a.N) * kBK * 2;
-  const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * S, codes_bar = empty_s + 8 * S;
-  const uint32_t done_bar = codes_bar + 8, ready_s = done_bar + 8, free_s = ready_s + 8 * kTileRing;
+  const uint32_t full_s = s0 + L.bars, empty_s = full_s + 8 * S, done_bar = empty_s + 8 * S;
+  const uint32_t ready_s = done_bar + 8, free_s = ready_s + 8 * kTileRing, rawbar_s = free_s + 8 * kTileRing;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(sm + L.misc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
@@ -222,6 +229,17 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     if ((!okA || (has_b && !okB)) && tid == 0 && ks == 0) report(a.status, USK_FLAG_RATE_MAP);
     if (!okA && !okB) return;  // the whole cluster (same tile) leaves before any barrier or allocation
   }
+  // raw ring slot r holds tile t = r (mod R) of both row blocks; one
+  // expect-tx arrive and one bulk copy per valid row block fill it
+  const uint32_t raw_tx = kRbBytes * ((okA ? 1u : 0u) + (okB ? 1u : 0u));
+  auto issue_raw = [&](int t) {
+    const uint32_t slot = s0 + L.codes + static_cast<uint32_t>(t % R) * (2u * kRbBytes);
+    const uint32_t bar = rawbar_s + 8u * static_cast<uint32_t>(t % R);
+    mbar_arrive_expect_tx(bar, raw_tx);
+    const int64_t toff = static_cast<int64_t>(t_begin + t) * kRbBytes;
+    if (okA) bulk_g2s(slot, a.codes + cbA + toff, kRbBytes, bar);
+    if (okB) bulk_g2s(slot + kRbBytes, a.codes + cbB + toff, kRbBytes, bar);
+  };
 
   if (warp == kMmaWarp0) {
     if (lane == 0) {
@@ -229,21 +247,17 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
         mbar_init(full_s + 8 * s, 128 + 1);  // one decoder group + the x copy
         mbar_init(empty_s + 8 * s, 1);
       }
-      mbar_init(codes_bar, 1);
       mbar_init(done_bar, a.I);
       for (int q = 0; q < kTileRing; ++q) {
         mbar_init(ready_s + 8 * q, 32);           // the widen warp
         mbar_init(free_s + 8 * q, kDecThreads);   // every decoder
       }
+      for (int r = 0; r < R; ++r) mbar_init(rawbar_s + 8 * r, 1);
       *abort_flag = 0u;
       mbar_fence_init();
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(xmap)) : "memory");
-      // the block's codes: two contiguous runs (one per valid row block)
-      const uint32_t bytes = static_cast<uint32_t>(tcta) * kRbBytes;
-      mbar_arrive_expect_tx(codes_bar, bytes * ((okA ? 1u : 0u) + (okB ? 1u : 0u)));
-      if (okA) bulk_g2s(s0 + L.codes, a.codes + cbA + static_cast<int64_t>(t_begin) * kRbBytes, bytes, codes_bar);
-      if (okB)
-        bulk_g2s(s0 + L.codes + bytes, a.codes + cbB + static_cast<int64_t>(t_begin) * kRbBytes, bytes, codes_bar);
+      // the first R tiles' codes (the widen warp issues the rest)
+      for (int t = 0; t < R && t < tcta; ++t) issue_raw(t);
     }
     __syncwarp();
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -328,10 +342,16 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
       mbar_arrive(full_s + 8 * s);
     }
   } else if (warp == kWidenWarp) {
-    // ---------------- tile codes int8 -> bf16 (exact), kTileRing tiles ahead
-    if (!__all_sync(0xFFFFFFFFu, mbar_wait(codes_bar, 0))) aborted = true;
+    // ---------------- tile codes int8 -> bf16 (exact), kTileRing tiles ahead;
+    // the raw codes stream in R tiles ahead (this warp refills a raw slot once
+    // it has read it)
+    int consumed = 0;  // raw tiles read by this warp
     for (int t = 0; t < tcta && !aborted; ++t) {
       const int q = t % kTileRing;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(rawbar_s + 8 * (t % R), static_cast<uint32_t>(t / R) & 1u))) {
+        aborted = true;
+        break;
+      }
       if (t >= kTileRing &&
           !__all_sync(0xFFFFFFFFu, mbar_wait(free_s + 8 * q, static_cast<uint32_t>(t / kTileRing - 1) & 1u))) {
         aborted = true;
@@ -339,11 +359,12 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
       }
       // 2 x kRbBytes stored bytes, 16 per lane per step; all loads in flight first
       constexpr int kSteps = static_cast<int>(2u * kRbBytes / 512u);
+      const uint32_t slot = s0 + L.codes + static_cast<uint32_t>(t % R) * (2u * kRbBytes);
       uint4 w[kSteps];
 #pragma unroll
       for (int i = 0; i < kSteps; ++i) {
         const uint32_t idx = static_cast<uint32_t>(lane) * 16u + static_cast<uint32_t>(i) * 512u;
-        w[i] = lds128(s0 + L.codes + ((idx / kRbBytes) * tcta + t) * kRbBytes + (idx % kRbBytes));
+        w[i] = lds128(slot + idx);  // [row block][kRbBytes] within the slot
       }
 #pragma unroll
       for (int i = 0; i < kSteps; ++i) {
@@ -366,7 +387,20 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
         }
       }
       mbar_arrive(ready_s + 8 * q);
+      // the raw slot has been read (its values used above): refill it with tile
+      // t + R (generic reads ordered before the async-proxy copy)
+      consumed = t + 1;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0 && t + R < tcta) issue_raw(t + R);
+      __syncwarp();
     }
+    // after a wait gave up: wait (bounded) for the raw copies still in flight
+    if (aborted && lane == 0) {
+      const int issued = tcta < consumed + R ? tcta : consumed + R;
+      for (int t = consumed; t < issued; ++t) mbar_wait(rawbar_s + 8 * (t % R), static_cast<uint32_t>(t / R) & 1u);
+    }
+    __syncwarp();
   } else if (warp == kCopyWarp) {
     // ---------------- x tiles, up to S chunks ahead of the MMAs.  The whole
     // warp runs the loop (a lane spinning elsewhere would steal the warp from
@@ -524,9 +558,16 @@ __host__ __device__ inline uint32_t gemm_tmem_cols(int N, int I) {
   return gemm_a_col(N, I) + 4u * 32u <= 256u ? 256u : 512u;
 }
 
+// Raw tile-code slots for tpb tiles per block: min(tpb, kRawRingMin).  A ring
+// of 8 was measured no slower than one slot per tile on every shape (and
+// 21% faster at 28672x8192 batch 64, where the smaller footprint lets two
+// blocks share an SM), even where staging every tile would cost no stages.
+static int gemm_raw_ring(int tpb) { return tpb < kRawRingMin ? tpb : kRawRingMin; }
+
 // Pipeline stages for batch N and tpb tiles per block: as many as tensor
-// memory and shared memory (the B stages next to the staged codes; half of the
-// SM's when two blocks share it) hold, at most kMaxStages; 0 if fewer than 4.
+// memory and shared memory (the B stages next to the raw code ring and the
+// keys; half of the SM's when two blocks share it) hold, at most kMaxStages;
+// 0 if fewer than 4.
 //
 // S is a multiple of 4: stage s = c mod S is then always filled by decoder
 // group s mod 4 and consumed by MMA warp s mod I (I divides 4), so every
@@ -539,13 +580,13 @@ static int gemm_stages(int N, int tpb, int depth, int var, int I) {
   int S = static_cast<int>((cols - gemm_a_col(N, I)) / 32u);
   if (S > kMaxStages) S = kMaxStages;
   S &= ~3;
-  while (S >= 4 && gemm_layout(N, tpb, S, depth, var_tile_bytes(var), var_tile_bf(var)).total + 1024u > smem_cap)
-    S -= 4;
+  const uint32_t tb = var_tile_bytes(var), tbf = var_tile_bf(var);
+  while (S >= 4 && gemm_layout(N, tpb, S, depth, tb, tbf, gemm_raw_ring(tpb)).total + 1024u > smem_cap) S -= 4;
   return S >= 4 ? S : 0;
 }
 
-// Largest number of tiles per block (codes staged up front) that still leaves
-// a four-stage pipeline for batch N.
+// Largest number of tiles per block (the keys of every tile are kept) that
+// still leaves a four-stage pipeline for batch N.
 static int gemm_max_tiles(int N, int depth, int var, int I) {
   int t = kMaxTiles;
   while (t > 1 && gemm_stages(N, t, depth, var, I) == 0) --t;
@@ -556,7 +597,8 @@ static int gemm_max_tiles(int N, int depth, int var, int I) {
 // share an SM than its 512 tensor-memory columns hold (a block waiting in
 // tcgen05.alloc for a co-resident block of its own cluster would never proceed).
 static uint32_t gemm_smem_bytes(int N, int tpb, int S, int depth, int var, int I) {
-  const uint32_t smem = gemm_layout(N, tpb, S, depth, var_tile_bytes(var), var_tile_bf(var)).total + 1024u;
+  const uint32_t tb = var_tile_bytes(var), tbf = var_tile_bf(var);
+  const uint32_t smem = gemm_layout(N, tpb, S, depth, tb, tbf, gemm_raw_ring(tpb)).total + 1024u;
   const uint32_t max_blocks = 512u / gemm_tmem_cols(N, I);
   const uint32_t floor_bytes = 233472u / (max_blocks + 1u) + 1u - 1024u;  // 228 KiB per SM, 1 KiB reserved per block
   return smem > floor_bytes ? smem : floor_bytes;
@@ -655,6 +697,7 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.tmem_cols = gemm_tmem_cols(batch, a.I);
   a.a_col = gemm_a_col(batch, a.I);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
+  a.R = gemm_raw_ring(tcta_max);
   a.S = gemm_stages(batch, tcta_max, depth, var, a.I);
   if (a.S < 4 || a.S % 4 != 0) return cudaErrorInvalidValue;
   const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth, var, a.I);
