@@ -559,11 +559,13 @@ def run_usk(args):
         usk.usk_build(Ws[i % N_WCOPIES], imp, seed, codes=b.codes, scales=b.scales, status=status)
 
     # consecutive decode calls launch as programmatic dependents of the previous
-    # one (their code prefetch overlaps the previous call's tail)
+    # one (their code prefetch -- and for usk_gemm the set-up and decoding into
+    # tensor memory -- overlaps the previous call's tail)
     add("layer", [("usk_build", lay_build, 1),
                   ("usk_gemv", lambda i: usk.usk_gemv(sks[(i + 128) % N_SKETCHES], x1, y=y1, pdl=True), 1),
                   ("usk_gemv_b4", lambda i: usk.usk_gemv(sks[(i + 160) % N_SKETCHES], x4, y=y4, pdl=True), 1),
-                  ("usk_gemm", lambda i: usk.usk_gemm(sks[(i + 64) % N_SKETCHES], x16, y=y16, status=status), 1),
+                  ("usk_gemm", lambda i: usk.usk_gemm(sks[(i + 64) % N_SKETCHES], x16, y=y16, status=status,
+                                                      pdl=True), 1),
                   ("usk_gemv_multi", lambda i: usk.usk_gemv_multi([sks[(i + 192) % N_SKETCHES]], [x1], [y1],
                                                                   ws=ws_lay, pdl=True), 1)],
         None)
@@ -687,7 +689,7 @@ def run_usk(args):
 
         def gm(i, lst=lst, n=n):
             e = lst[(i + 3 * n // 4) % n]
-            usk.usk_gemm(e["sk"], e["x16"], y=e["y"], status=status)
+            usk.usk_gemm(e["sk"], e["x16"], y=e["y"], status=status, pdl=True)
 
         ws_s = torch.zeros(max(16, usk.usk_gemv_multi_ws_bytes([lst[0]["sk"]], 4)), dtype=torch.uint8, device=dev)
 
@@ -736,7 +738,7 @@ def run_usk(args):
         mlp_phases.append((shp + "/usk_gemv_multi_b1", mgm1, 1))
         for bb in (16, 32, 64):
             def mgm(i, e=e, xs=xs, bb=bb):
-                usk.usk_gemm(e["sks"][(i + bb) % AB_COPIES], xs[bb], y=e["y"][:bb], status=status)
+                usk.usk_gemm(e["sks"][(i + bb) % AB_COPIES], xs[bb], y=e["y"][:bb], status=status, pdl=True)
             mlp_phases.append((shp + "/usk_gemm_b%d" % bb, mgm, 1))
     add("mlp70b", mlp_phases, None)
 
@@ -751,7 +753,8 @@ def run_usk(args):
 
     add("absmaxmin", [("usk_build", amm_build, 1),
                       ("usk_gemv", lambda i: usk.usk_gemv(sks2[(i + 128) % N_SKETCHES], x1, y=y1, pdl=True), 1),
-                      ("usk_gemm", lambda i: usk.usk_gemm(sks2[(i + 64) % N_SKETCHES], x16, y=y16, status=status),
+                      ("usk_gemm", lambda i: usk.usk_gemm(sks2[(i + 64) % N_SKETCHES], x16, y=y16, status=status,
+                                                                          pdl=True),
                        1)], None)
 
     # ---------------------------------------------------------- format 3 and the matrix-vs-hash A/B
@@ -782,7 +785,8 @@ def run_usk(args):
 
     add("q4", [("usk_build", q4_build, 1),
                ("usk_gemv", lambda i: usk.usk_gemv(sks4[(i + 128) % N_SKETCHES], x1, y=y1, pdl=True), 1),
-               ("usk_gemm", lambda i: usk.usk_gemm(sks4[(i + 64) % N_SKETCHES], x16, y=y16, status=status), 1)],
+               ("usk_gemm", lambda i: usk.usk_gemm(sks4[(i + 64) % N_SKETCHES], x16, y=y16, status=status,
+                                                                   pdl=True), 1)],
         None)
 
     # ---------------------------------------------------------- format 1 at 2 and 8 slots
@@ -813,7 +817,7 @@ def run_usk(args):
                             ("usk_gemv", lambda i: usk.usk_gemv(sksv[(i + 128) % N_SKETCHES], x1, y=y1, pdl=True),
                              1),
                             ("usk_gemm", lambda i: usk.usk_gemm(sksv[(i + 64) % N_SKETCHES], x16, y=y16,
-                                                                status=status), 1)], None)
+                                                                status=status, pdl=True), 1)], None)
 
     # ---------------------------------------------------------- timed regions
     sampler = ClockSampler(local)
@@ -899,7 +903,8 @@ def run_usk(args):
                              "steps + one untimed replay of every graph; the K-step region timed %d times with "
                              "CUDA events on the replay stream (a device spin covers the host's enqueue), median "
                              "per call reported, min/max under 'spread'" % REPEATS,
-                   "gemv_launch": "programmatic dependent launch (USK_GEMV_PDL) between consecutive GEMV calls",
+                   "gemv_launch": "programmatic dependent launch (USK_GEMV_PDL, USK_GEMM_PDL) between consecutive "
+                                  "GEMV and GEMM calls",
                    "l2": "L2 flushed before each timed repeat (a %d MiB read); within a repeat builds cycle over %d "
                          "weight copies (%d MiB) and the decodes touch %d distinct sketch copies (1 MiB each), so "
                          "every decode reads its codes from HBM"

@@ -378,6 +378,19 @@ USK_API usk_status usk_gemv_multi_static(int64_t n, const usk_sketch* sketches, 
 USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y,
                     void* ws, size_t ws_bytes, uint32_t* d_status, void* stream);
 
+/* usk_gemm with launch flags (Metodologia §4, as usk_gemm).  USK_GEMM_PDL:
+ * launch as a programmatic dependent of the previous kernel in the stream.
+ * Before waiting for that kernel a block sets up, copies its share of the
+ * sketch codes (and reads a rate map's order and offset tables), widens them
+ * and decodes the first tiles into tensor memory; x, the scales, y and
+ * d_status are touched only after the wait.  So the caller guarantees that no
+ * kernel still running in the stream writes this sketch's codes or rate-map
+ * tables (x and y may be produced / consumed by neighbouring kernels).  The
+ * results are those of usk_gemm.  Other bits: USK_ERR_PARAMS. */
+#define USK_GEMM_PDL 1u
+USK_API usk_status usk_gemm_ex(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y,
+                               uint32_t flags, uint32_t* d_status, void* stream);
+
 /* Test hook: override the launch geometry (0 = default).  build_cluster is the
  * number of thread blocks per row block in usk_build (1..8); gemv_tiles_per_block
  * the number of hash tiles per thread block in usk_gemv.  Results are

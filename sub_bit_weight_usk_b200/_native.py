@@ -67,10 +67,12 @@ class UskSketchC(ctypes.Structure):
 _lib = None
 
 EXPORTED = ["usk_sizes", "usk_sizes_ex", "usk_plan_slots", "usk_rate_map_plan", "usk_build", "usk_gemv", "usk_gemv_ex",
-            "usk_gemv_multi", "usk_gemv_multi_ws_bytes", "usk_gemv_multi_static", "usk_gemm", "usk_status_str",
+            "usk_gemv_multi", "usk_gemv_multi_ws_bytes", "usk_gemv_multi_static", "usk_gemm", "usk_gemm_ex",
+            "usk_status_str",
             "usk_format_version", "usk_debug_set_geometry", "usk_debug_set_gemv_path", "usk_debug_set_gemv_rows",
             "usk_debug_set_gemm_splits", "usk_debug_set_gemm_issuers", "usk_debug_inject_timeout"]
 GEMV_PDL = 1
+GEMM_PDL = 1
 
 
 def load_library(path: str = LIB_PATH):
@@ -110,6 +112,8 @@ def load_library(path: str = LIB_PATH):
     lib.usk_gemv_multi_static.restype = ctypes.c_int
     lib.usk_gemm.argtypes = [ctypes.POINTER(UskSketchC), vp, i64, vp, vp, ctypes.c_size_t, vp, vp]
     lib.usk_gemm.restype = ctypes.c_int
+    lib.usk_gemm_ex.argtypes = [ctypes.POINTER(UskSketchC), vp, i64, vp, ctypes.c_uint32, vp, vp]
+    lib.usk_gemm_ex.restype = ctypes.c_int
     lib.usk_status_str.argtypes = [ctypes.c_int]
     lib.usk_status_str.restype = ctypes.c_char_p
     lib.usk_format_version.argtypes = []
@@ -377,8 +381,13 @@ def usk_gemv_multi(sketches, xs, ys=None, ws: torch.Tensor | None = None, status
 
 
 def usk_gemm(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
-             status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """y [batch, M] fp32 = W_hat x^T for bf16 x [batch, K], batch 16..256 (multiple of 16)."""
+             status: torch.Tensor | None = None, stream=None, pdl: bool = False) -> torch.Tensor:
+    """y [batch, M] fp32 = W_hat x^T for bf16 x [batch, K], batch 16..256 (multiple of 16).
+
+    pdl=True launches as a programmatic dependent of the previous kernel in the
+    stream (usk_gemm_ex with USK_GEMM_PDL): set-up, code copies and decoding
+    overlap that kernel; x, scales, y and status wait for it.  The caller
+    guarantees that no kernel still running in the stream writes the sketch."""
     _need_cuda(x, y, status)
     if x.dtype != torch.bfloat16 or not x.is_contiguous() or x.dim() != 2:
         raise TypeError("x must be a contiguous 2-D bfloat16 tensor")
@@ -386,8 +395,8 @@ def usk_gemm(sketch: Sketch, x: torch.Tensor, y: torch.Tensor | None = None,
     if y is None:
         y = torch.empty((batch, sketch.M), dtype=torch.float32, device=x.device)
     sk = sketch.as_c()
-    st = load_library().usk_gemm(ctypes.byref(sk), _ptr(x), batch, _ptr(y), None, 0, _ptr(status),
-                                 _stream(stream))
+    st = load_library().usk_gemm_ex(ctypes.byref(sk), _ptr(x), batch, _ptr(y), GEMM_PDL if pdl else 0,
+                                    _ptr(status), _stream(stream))
     _check(st, "usk_gemm")
     return y
 

@@ -31,7 +31,7 @@ cudaError_t launch_gemv(const int8_t* codes, const uint16_t* scales, int64_t M, 
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
                         int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2,
-                        int splits_override, int issuers_override);
+                        int splits_override, int issuers_override, bool pdl);
 bool gemm_supported(int64_t K, int batch, int depth, int var);
 size_t gemv_multi_ws_bytes(int n, const int64_t* Ms, const int64_t* Ks, int batch, int depth, int var);
 cudaError_t launch_gemv_multi(int n, const int8_t* const* codes, const uint16_t* const* scales, const int64_t* Ms,
@@ -387,6 +387,12 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
                     size_t ws_bytes, uint32_t* d_status, void* stream) {
   (void)ws;
   (void)ws_bytes;
+  return usk_gemm_ex(sketch, x_bf16, batch, y, 0u, d_status, stream);
+}
+
+USK_API usk_status usk_gemm_ex(const usk_sketch* sketch, const uint16_t* x_bf16, int64_t batch, float* y,
+                               uint32_t flags, uint32_t* d_status, void* stream) {
+  if ((flags & ~static_cast<uint32_t>(USK_GEMM_PDL)) != 0) return USK_ERR_PARAMS;
   usk_status st = check_sketch(sketch);
   if (st != USK_OK) return st;
   if (sketch->version == USK_FORMAT_COLSHARED) return USK_ERR_PARAMS;  // format 3: usk_gemv only
@@ -406,7 +412,7 @@ USK_API usk_status usk_gemm(const usk_sketch* sketch, const uint16_t* x_bf16, in
   const Launch l = launch_of(sketch->rates, sketch->M);
   cudaError_t e = usk::launch_gemm(sketch->codes, sketch->scales, sketch->M, sketch->K, sketch->seed, x_bf16,
                                    static_cast<int>(batch), y, d_status, s, g_inject == 2, depth, layout, l.map,
-                                   l.nrb, l.g1, l.g2, g_gemm_splits, g_gemm_issuers);
+                                   l.nrb, l.g1, l.g2, g_gemm_splits, g_gemm_issuers, (flags & USK_GEMM_PDL) != 0);
   if (e != cudaSuccess) return USK_ERR_CUDA;
   return from_cuda(cudaGetLastError());
 }

@@ -82,6 +82,8 @@ struct GemmArgs {
   int I;           // MMA issuer warps, each with its own accumulator (columns [i N, (i + 1) N))
   int R;           // raw tile-code slots: min(tiles per block, kRawRingMin)
   int inject;  // test hook: block (0, 0) skips the x copy of its first chunk
+  int pdl;     // launched as a programmatic dependent: x, scales, y and status only after the wait
+  int early;   // let dependents launch after set-up (else after the main loop)
   RbMap map;    // grid rows -> row blocks and code offsets
   int64_t nrb;  // row blocks of this launch (a tile takes grid rows 2 mt and 2 mt + 1)
   int64_t g1, g2;  // per-row-block rates: where the 4- and 8-slot groups start in the order list
@@ -226,7 +228,10 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     if (gm.order != nullptr) gm.order += order0;
     okA = rb_resolve(gm, 2 * static_cast<int64_t>(mt), rb_bytes, rbA, cbA);
     if (has_b) okB = rb_resolve(gm, 2 * static_cast<int64_t>(mt) + 1, rb_bytes, rbB, cbB);
-    if ((!okA || (has_b && !okB)) && tid == 0 && ks == 0) report(a.status, USK_FLAG_RATE_MAP);
+    if ((!okA || (has_b && !okB)) && tid == 0 && ks == 0) {
+      if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+      report(a.status, USK_FLAG_RATE_MAP);
+    }
     if (!okA && !okB) return;  // the whole cluster (same tile) leaves before any barrier or allocation
   }
   // raw ring slot r holds tile t = r (mod R) of both row blocks; one
@@ -274,6 +279,10 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
   tc_fence_after();
   const uint32_t tmem_d = *tmem_holder;
   bool aborted = false;
+  // dependents may launch now (grids of more blocks than SMs): their set-up,
+  // code copies and decoding into tensor memory overlap this block's main
+  // loop and epilogue
+  if (a.early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp < kDecWarps) {
     // ---------------- decoders: group g = warp / 4 rebuilds chunk g (octets
@@ -296,7 +305,9 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
       }
       const int s = c % S;
       if (c >= S) {
-        // the MMAs that read this A stage have completed
+        // the MMAs that read this A stage have completed (they need x: under a
+        // programmatic launch the bounded wait starts after the previous kernel)
+        if (c - 4 < S && a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
         if (!__all_sync(0xFFFFFFFFu, mbar_wait(empty_s + 8 * s, static_cast<uint32_t>(c / S - 1) & 1u))) {
           aborted = true;
           break;
@@ -352,6 +363,9 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
         aborted = true;
         break;
       }
+      // the decoders free a tile buffer only as the MMAs advance (they need x):
+      // under a programmatic launch the bounded wait starts after the previous kernel
+      if (t == kTileRing && a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
       if (t >= kTileRing &&
           !__all_sync(0xFFFFFFFFu, mbar_wait(free_s + 8 * q, static_cast<uint32_t>(t / kTileRing - 1) & 1u))) {
         aborted = true;
@@ -405,6 +419,9 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     // ---------------- x tiles, up to S chunks ahead of the MMAs.  The whole
     // warp runs the loop (a lane spinning elsewhere would steal the warp from
     // the issuing lane); lane 0 issues.
+    // x may come from the previous kernel in the stream: it is read only after
+    // that kernel has completed (the codes and the decoding did not wait)
+    if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
     int s = 0;
     uint32_t ph = 0;
     for (int c = 0; c < nk && !aborted; ++c, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
@@ -422,6 +439,7 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     // ---------------- MMAs: warp i takes chunks i, i + I, ... into accumulator i
     // (whole warp in the loop, lane 0 issues)
     const int i = warp - kMmaWarp0;
+    if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");  // the x stages follow the previous kernel
     const uint32_t idesc = idesc_bf16_f32(a.N);
     const uint32_t d_tm = tmem_d + static_cast<uint32_t>(i * a.N);
     for (int c = i; c < nk && !aborted; c += a.I) {
@@ -452,7 +470,13 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // otherwise dependents launch now, over the epilogue: launched earlier, they
+  // would take second slots on busy SMs and leave the next call unbalanced
+  if (!a.early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const bool failed = *abort_flag != 0u;
+  // scales, y and status after the previous kernel (the copy warp has already
+  // waited, so this returns at once)
+  if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (failed && tid == 0) report(a.status, USK_FLAG_TIMEOUT);
 
   // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31; the
@@ -658,7 +682,7 @@ bool gemm_supported(int64_t K, int batch, int depth, int var) {
 cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, int64_t K, uint64_t seed,
                         const uint16_t* x, int batch, float* y, uint32_t* status, cudaStream_t stream, int inject,
                         int depth, int var, const RbMap& map, int64_t nrb, int64_t g1, int64_t g2,
-                        int splits_override, int issuers_override) {
+                        int splits_override, int issuers_override, bool pdl) {
   // a rate map: one launch over the tiles of every slot group, planned for the
   // 8-slot layout (the largest staged and widened tiles)
   const bool vr = map.order != nullptr;
@@ -670,7 +694,7 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
     return cudaErrorInvalidValue;
   GemmArgs a;
   a.codes = codes; a.scales = scales; a.y = y;
-  a.M = M; a.K = K; a.seed = seed; a.status = status; a.inject = inject;
+  a.M = M; a.K = K; a.seed = seed; a.status = status; a.inject = inject; a.pdl = pdl ? 1 : 0;
   a.T = static_cast<int>(K / kTileCols);
   a.N = batch;
   a.map = map;
@@ -698,6 +722,10 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   a.a_col = gemm_a_col(batch, a.I);
   const int tcta_max = (a.T + a.splits - 1) / a.splits;
   a.R = gemm_raw_ring(tcta_max);
+  // measured: the early trigger pays where the grid already doubles up on SMs
+  // (28672x8192 batch 64: 65.3 -> 61.3 us), the late one where it does not
+  // (4096x11008 batch 16: 22.2 -> 17.1 us; 4096x4096: 10.1 -> 9.3 us)
+  a.early = static_cast<int64_t>(a.splits) * m_tiles > sms ? 1 : 0;
   a.S = gemm_stages(batch, tcta_max, depth, var, a.I);
   if (a.S < 4 || a.S % 4 != 0) return cudaErrorInvalidValue;
   const size_t smem = gemm_smem_bytes(batch, tcta_max, a.S, depth, var, a.I);
@@ -729,13 +757,15 @@ cudaError_t launch_gemm(const int8_t* codes, const uint16_t* scales, int64_t M, 
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = a.splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.pdl ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, a, xmap);
 }
 

@@ -83,6 +83,8 @@ def test_argument_errors_return_before_any_launch(lib):
     assert lib.usk_gemm(ctypes.byref(sk), fake, 8, fake, None, 0, None, None) == 4
     assert lib.usk_gemm(ctypes.byref(sk), fake, 24, fake, None, 0, None, None) == 4
     assert lib.usk_gemm(ctypes.byref(sk), fake, 512, fake, None, 0, None, None) == 4
+    assert lib.usk_gemm_ex(ctypes.byref(sk), fake, 16, fake, 2, None, None) == 6  # unknown flag bit
+    assert lib.usk_gemm_ex(ctypes.byref(sk), fake, 24, fake, 1, None, None) == 4
     for version, depth in ((2, 3), (2, 0), (1, 2), (5, 1)):
         bad_sk = _native.UskSketchC(64, 256, 0, 16 * 1024, 16 * 1024, version, depth)
         assert lib.usk_gemv(ctypes.byref(bad_sk), fake, 1, 1, fake, None, None) == 6

@@ -118,3 +118,86 @@ def test_gemm_issuer_counts(issuers, batch):
     finally:
         usk.usk_debug_set_gemm_issuers(0)
         usk.usk_debug_set_gemm_splits(0)
+
+
+@pytest.mark.parametrize("M,K,batch", [(256, 1024, 16), (128, 4352, 64), (4096, 4096, 16)])
+def test_gemm_pdl_after_producer(M, K, batch):
+    """Launched as a programmatic dependent: x is written by the kernel just
+    before (after a long spin, so an early read would see the zeros), y is
+    filled with NaN by another kernel before that; the dependent GEMM gives the
+    bits of the plain launch."""
+    W = gen.weights_student_t(M, K, 17, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _sketch(W, 8)
+    xh = gen.activations(batch, K, 18, "bf16")
+    x_src = to_dev(xh)
+    ref = usk.usk_gemm(sk, x_src).clone()
+    st = status_tensor()
+    x = torch.zeros_like(x_src)
+    y = torch.empty((batch, M), dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        x.zero_()
+        y.fill_(float("nan"))
+        torch.cuda._sleep(2_000_000)
+        torch.mul(x_src, 1, out=x)
+        usk.usk_gemm(sk, x, y=y, status=st, pdl=True)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert torch.equal(y, ref), "dependent launch differs from the plain one"
+    e = rel_err(y.cpu().numpy(), oracle.gemv_f64(o["codes"], o["scales"], M, K, xh, sk.seed))
+    assert e <= TOL
+
+
+def test_gemm_pdl_chain_in_graph():
+    """A CUDA graph of back-to-back dependent GEMMs, each reading the x that the
+    elementwise kernel before it wrote and writing its own y: every output has
+    the bits of the plain launch."""
+    shapes = [(256, 1024), (4096, 4096), (128, 4352), (4096, 4096)]
+    sks, xs_src, refs = [], [], []
+    for i, (M, K) in enumerate(shapes):
+        W = gen.weights_normal(M, K, 30 + i, 0.02, "bf16")
+        sk, _ = _sketch(W, 40 + i)
+        sks.append(sk)
+        xs_src.append(to_dev(gen.activations(16 * (1 + i % 2), K, 50 + i, "bf16")))
+        refs.append(usk.usk_gemm(sk, xs_src[-1]).clone())
+    xs = [torch.zeros_like(x) for x in xs_src]
+    ys = [torch.full_like(r, float("nan")) for r in refs]
+    st = status_tensor()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for sk, xsrc, x, y in zip(sks, xs_src, xs, ys):
+            torch.mul(xsrc, 1, out=x)
+            usk.usk_gemm(sk, x, y=y, status=st, pdl=True)
+    for _ in range(2):
+        for x, y in zip(xs, ys):
+            x.zero_()
+            y.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        for y, r in zip(ys, refs):
+            assert torch.equal(y, r)
+    del g
+
+
+def test_gemm_pdl_back_to_back_same_output():
+    """Dependent GEMMs one after another on one y: each launch starts while the
+    one before runs (that one triggers its dependents early), and y ends with
+    the last product's bits (no write of an earlier launch lands after it)."""
+    M, K = 4096, 4096
+    a, _ = _sketch(gen.weights_normal(M, K, 61, 0.02, "bf16"), 62)
+    b, _ = _sketch(gen.weights_normal(M, K, 63, 0.02, "bf16"), 64)
+    x = to_dev(gen.activations(16, K, 65, "bf16"))
+    ref_b = usk.usk_gemm(b, x).clone()
+    ref_a = usk.usk_gemm(a, x).clone()
+    y = torch.empty_like(ref_b)
+    for n in (2, 5, 8):
+        y.fill_(float("nan"))
+        for i in range(n):
+            usk.usk_gemm(a if (n - 1 - i) % 2 else b, x, y=y, pdl=True)
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref_b)
+    usk.usk_gemm(a, x, y=y, pdl=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref_a)
