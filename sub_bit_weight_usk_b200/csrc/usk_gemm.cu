@@ -104,7 +104,7 @@ __host__ __device__ inline GemmLayout gemm_layout(int N, int tcta, int S, int de
   L.keys = L.codes + static_cast<uint32_t>(R) * 2u * tile_bytes;       // uint2 [2][tcta][depth]
   // full[S], empty[S], done, ready[ring], free[ring], raw[R]
   L.bars = (L.keys + 2u * tcta * depth * 8u + 7u) & ~7u;
-  L.misc = L.bars + (2 * S + 1 + 2 * kTileRing + R) * 8;               // tmem holder, abort
+  L.misc = L.bars + (2 * S + 1 + 2 * kTileRing + R) * 8;               // tmem holder, abort, 2 scales
   L.total = L.misc + 16;
   return L;
 }
@@ -167,14 +167,23 @@ __device__ __forceinline__ void mma_commit(uint32_t mbar) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+// 4 columns of this thread's lane into r without waiting: r must not be read
+// before tmem_ld_wait4 has been given it
+__device__ __forceinline__ void tmem_ld4_async(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Waits for this thread's tensor-memory loads; the registers are operands, so
+// no use of them is scheduled before the wait
+__device__ __forceinline__ void tmem_ld_wait4(uint32_t (&r)[4][4]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0][0]), "+r"(r[0][1]), "+r"(r[0][2]), "+r"(r[0][3]), "+r"(r[1][0]), "+r"(r[1][1]),
+                 "+r"(r[1][2]), "+r"(r[1][3]), "+r"(r[2][0]), "+r"(r[2][1]), "+r"(r[2][2]), "+r"(r[2][3]),
+                 "+r"(r[3][0]), "+r"(r[3][1]), "+r"(r[3][2]), "+r"(r[3][3])
+               :
+               : "memory");
 }
 
 // D = hash rows of the sketch (1: format 1 or format 2 at depth 1; 2, 4: the
@@ -214,6 +223,7 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
   const uint32_t ready_s = done_bar + 8, free_s = ready_s + 8 * kTileRing, rawbar_s = free_s + 8 * kTileRing;
   volatile uint32_t* tmem_holder = reinterpret_cast<volatile uint32_t*>(sm + L.misc);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(sm + L.misc + 4);
+  volatile float* scale_s = reinterpret_cast<volatile float*>(sm + L.misc + 8);  // the tile's two row-block scales
   uint2* keytab = reinterpret_cast<uint2*>(sm + L.keys);
   // the tile's two row blocks and where their codes start; with a rate map a
   // block whose entry is out of range is skipped on its own (its rows are
@@ -422,6 +432,8 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     // x may come from the previous kernel in the stream: it is read only after
     // that kernel has completed (the codes and the decoding did not wait)
     if (a.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // the scales for the epilogue, read once here, off its path
+    if (lane < 2) scale_s[lane] = __half2float(__ushort_as_half(a.scales[lane ? rbB : rbA]));
     int s = 0;
     uint32_t ph = 0;
     for (int c = 0; c < nk && !aborted; ++c, s = (s + 1 == S) ? 0 : s + 1, ph ^= (s == 0) ? 1u : 0u) {
@@ -487,17 +499,28 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
     const int rbm = m < kRowsPerBlock ? rbA : rbB;
     const int64_t row = static_cast<int64_t>(rbm) * kRowsPerBlock + (m & 63);
     const bool row_ok = m < kRowsPerBlock ? okA : okB;
-    const float scale = row_ok ? __half2float(__ushort_as_half(a.scales[rbm])) : 0.0f;
+    const float scale = row_ok ? scale_s[m < kRowsPerBlock ? 0 : 1] : 0.0f;
     const uint32_t lane_base = static_cast<uint32_t>(sub * 32) << 16;
     float* part = reinterpret_cast<float*>(sm + L.b);  // [N][128]: the x stage ring is free now
     for (int n0 = 8 * grp; n0 < a.N; n0 += 8 * kDecGroups) {
+      // the issuers' accumulators, every issuer's load in flight per wait (4
+      // columns at a time), summed in issuer order
       float v[8];
-      tmem_ld8(tmem_d + lane_base + n0, v);
-      for (int i = 1; i < a.I; ++i) {  // the issuers' accumulators, in order
-        float u[8];
-        tmem_ld8(tmem_d + lane_base + static_cast<uint32_t>(i * a.N) + n0, u);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] += u[e];
+      for (int h = 0; h < 2; ++h) {
+        uint32_t u[kMaxIssuers][4] = {};
+#pragma unroll
+        for (int i = 0; i < kMaxIssuers; ++i)
+          if (i < a.I) tmem_ld4_async(tmem_d + lane_base + static_cast<uint32_t>(i * a.N) + n0 + 4u * h, u[i]);
+        tmem_ld_wait4(u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float t = __uint_as_float(u[0][e]);
+#pragma unroll
+          for (int i = 1; i < kMaxIssuers; ++i)
+            if (i < a.I) t += __uint_as_float(u[i][e]);
+          v[4 * h + e] = t;
+        }
       }
       if (a.splits == 1) {
         if (row_ok) {
@@ -530,8 +553,7 @@ __device__ __forceinline__ void gemm_body(const GemmArgs& a, const CUtensorMap* 
       if (mm < kRowsPerBlock ? okA : okB) {
         const int rbm = mm < kRowsPerBlock ? rbA : rbB;
         const int64_t orow = static_cast<int64_t>(rbm) * kRowsPerBlock + (mm & 63);
-        const float sc = __half2float(__ushort_as_half(a.scales[rbm]));
-        a.y[static_cast<int64_t>(n) * a.M + orow] = acc * sc;
+        a.y[static_cast<int64_t>(n) * a.M + orow] = acc * scale_s[mm < kRowsPerBlock ? 0 : 1];
       }
     }
     cluster.sync();
