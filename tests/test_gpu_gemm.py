@@ -201,3 +201,31 @@ def test_gemm_pdl_back_to_back_same_output():
     usk.usk_gemm(a, x, y=y, pdl=True)
     torch.cuda.synchronize()
     assert torch.equal(y, ref_a)
+
+
+@pytest.mark.parametrize("fmt", ["amm2", "amm4", "q4"])
+def test_gemm_pdl_formats(fmt):
+    """Formats 2 (depth 2, 4) and 4 as programmatic dependents of the kernel that
+    writes x: the plain launch's bits, and within the tolerance of the oracle."""
+    M, K = 256, 2048
+    W = gen.weights_student_t(M, K, 74, 4.0, 0.02, 0.001, 20.0, "bf16")
+    if fmt == "q4":
+        o = oracle.build_sketch_q4(W, None, 15)
+        sk = sketch_from_oracle(o, M, K, 15, usk.FORMAT_Q4, 1)
+        ref_fn = lambda xh: oracle.gemv_q4_f64(o["codes"], o["scales"], M, K, xh, 15)  # noqa: E731
+    else:
+        d = 2 if fmt == "amm2" else 4
+        o = oracle.build_sketch_amm(W, 15, d)
+        sk = sketch_from_oracle(o, M, K, 15, usk.FORMAT_ABSMAXMIN, d)
+        ref_fn = lambda xh: oracle.gemv_amm_f64(o["codes"], o["scales"], M, K, xh, 15, d)  # noqa: E731
+    xh = gen.activations(32, K, 75, "bf16")
+    x_src = to_dev(xh)
+    ref = usk.usk_gemm(sk, x_src).clone()
+    x = torch.zeros_like(x_src)
+    y = torch.full_like(ref, float("nan"))
+    torch.cuda._sleep(1_000_000)
+    torch.mul(x_src, 1, out=x)
+    usk.usk_gemm(sk, x, y=y, pdl=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+    assert rel_err(y.cpu().numpy(), ref_fn(xh)) <= TOL

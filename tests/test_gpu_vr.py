@@ -296,3 +296,21 @@ def test_vr_long_k_products(call):
         _check_product(sk, o, gen.activations(9, K, 83, "bf16"))
     else:
         _check_product(sk, o, gen.activations(2, K, 83, "f32"))
+
+
+@pytest.mark.parametrize("batch", [16, 64])
+def test_vr_gemm_pdl(batch):
+    """A rate-mapped GEMM launched as a programmatic dependent of the kernel that
+    writes its x gives the plain launch's bits."""
+    slots = [8, 2, 4, 2, 8]
+    W = gen.weights_student_t(320, 2048, 72, 4.0, 0.02, 0.001, 20.0, "bf16")
+    sk, o = _oracle_sketch(W, None, 13, slots)
+    x_src = to_dev(gen.activations(batch, 2048, 73, "bf16"))
+    ref = usk.usk_gemm(sk, x_src).clone()
+    x = torch.zeros_like(x_src)
+    y = torch.full_like(ref, float("nan"))
+    torch.cuda._sleep(1_000_000)
+    torch.mul(x_src, 1, out=x)
+    usk.usk_gemm(sk, x, y=y, pdl=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
