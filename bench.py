@@ -1009,7 +1009,8 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
             t = d["usk_gemm_b%d" % bb]
             ln = R.gather_line(gemv_bytes(m, k, bb), m * k, t, tk("mlp70b_usk_gemm_b64") if bb == 64 else None,
                                flops=2 * m * k * bb)
-            # the survey's decode roof at 28672x8192, batch 64 (issue, ~5 ops/weight): 31.6 us
+            # issue-bound decode roof: about 5 lane operations per weight at 128 lanes
+            # per clock per SM (31.6 us at 28672x8192)
             ln["decode_roof_us"] = round(5 * m * k / (SMS * 128 * R.clk) * 1e6, 3)
             per[shp]["rooflines"]["usk_gemm_b%d" % bb] = ln
     out["mlp70b"] = {"workload": "70B-MLP-shaped 28672x8192 and 8192x28672 bf16 N(0, 0.02^2) (device-drawn), "
@@ -1036,7 +1037,7 @@ def region_reports(med, times, R, tr, world, peaks, rmap):
         "token_decode_ms": round(t_tok * 1e3, 4),
         "token_decode_us_per_linear": round(t_tok / 224 * 1e6, 3),
         "token_decode_roofline": dict(R.gather_line(tok_bytes, n_stack, t_tok),
-                                      survey_issue_roof_ms=0.87),
+                                      issue_roof_ms=round(5 * n_stack / (SMS * 128 * R.clk) * 1e3, 3)),
         "tokens_per_s": round(1.0 / t_tok, 2),
         "token_decode_grouped_ms": round(t_tokg * 1e3, 4),
         "token_decode_grouped_us_per_linear": round(t_tokg / 224 * 1e6, 3),

@@ -91,3 +91,39 @@ def test_row_block_workload_allocation():
     assert slots == oracle.plan_slots([64 * bench.K] * RB, imp.tolist(), 0.5)
     order = np.argsort(imp)
     assert all(slots[order[i]] <= slots[order[i + 1]] for i in range(RB - 1))
+
+
+def test_region_reports_assemble_from_synthetic_timings():
+    """Every region report of the bench line assembles from timings alone (no
+    GPU): each phase the bench times gets a synthetic per-call time, and the
+    report carries the regions, their kernel times and JSON-clean values."""
+    from types import SimpleNamespace
+    phases = {
+        "layer": ["usk_build", "usk_gemv", "usk_gemv_b4", "usk_gemm", "usk_gemv_multi"],
+        "small": ["usk_build", "usk_gemv_f32x", "usk_gemv_bf16x"],
+        "llama7b_set": ["%s/%s" % (s, c) for s in ("4096x4096", "11008x4096", "4096x11008")
+                        for c in ("usk_build", "usk_gemv_b1", "usk_gemv_b4", "usk_gemm_b16", "usk_gemv_multi_b1",
+                                  "usk_gemv_multi_b4")],
+        "mlp70b": ["%s/%s" % (s, c) for s in ("28672x8192", "8192x28672")
+                   for c in ("usk_build", "usk_gemv_b1", "usk_gemv_multi_b1", "usk_gemm_b16", "usk_gemm_b32",
+                             "usk_gemm_b64")],
+        "stack7b": ["model_build", "token_decode", "token_decode_grouped", "token_decode_concurrent",
+                    "token_dense_bf16_torch"],
+        "absmaxmin": ["usk_build", "usk_gemv", "usk_gemm"],
+        "colshared": ["usk_build", "usk_gemv", "ab_hash_gemv", "ab_matrix_gemv"],
+        "q4": ["usk_build", "usk_gemv", "usk_gemm"],
+        "rates": ["slots_2/usk_build", "slots_2/usk_gemv", "slots_8/usk_build", "slots_8/usk_gemv"],
+        "row_block_rates": ["usk_build", "usk_gemv", "usk_gemm"],
+    }
+    med = {r: {p: 1e-5 * (1 + i) for i, p in enumerate(ps)} for r, ps in phases.items()}
+    times = {r: {p: [v, 1.1 * v] for p, v in d.items()} for r, d in med.items()}
+    peaks = {"hbm_gbs": 6540.2, "bf16_tflops": 1645.9, "sm_max_mhz": 1965.0, "source": "measured"}
+    rmap = SimpleNamespace(count=[22, 31, 11], code_bytes=bench.N_W // 16)
+    out = bench.region_reports(med, times, bench.Roof(peaks), {}, 1, peaks, rmap)
+    for region in ("small", "llama7b_set", "mlp70b", "stack7b", "absmaxmin", "colshared", "q4", "rates",
+                   "row_block_rates"):
+        assert region in out, region
+    assert out["small"]["kernel_us"]["usk_build"] == pytest.approx(10.0)
+    assert out["mlp70b"]["per_shape"]["28672x8192"]["rooflines"]["usk_gemm_b64"]["decode_roof_us"] > 0
+    assert out["stack7b"]["token_decode_roofline"]["issue_roof_ms"] == pytest.approx(0.87, rel=0.01)
+    json.dumps(out)
